@@ -1,0 +1,451 @@
+/*
+ * FreeSolo sparse-attention forward pass: plain float64 CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU-baseline
+ * leg of the benchmark may load this code.  The CUDA library never links, calls or
+ * includes it, and this file includes nothing from the CUDA library.
+ *
+ * Source: "FreeSolo" technical summary (picx.dev/p/IEuVxx), section "Methodology":
+ *   §3.1 Range Separation  eq. (2)   o_i = o_i^sr + alpha_h o_i^lr
+ *   §3.2 Local Branch      eq. (3)   RoPE logits inside the look-back radius w
+ *                          eq. (4)   softmax readout over the local set L_i
+ *   §3.3 Long-Range Branch eq. (5)   cell summaries kbar_c, p_c, a_c over s-token cells
+ *                          eq. (7)   cell score r_ic with the erf position prior
+ *                          eq. (8)   FS-L pruning A_i = Recent_W(C_i) u TopP(a_c)
+ *                          eq. (9)   NoPE token readout over the selected cells, RMSNorm
+ * "Introduction and Theoretical Foundation": RoPE (Su et al.) stays inside the
+ * local window; long-range routing and readout use unrotated vectors.
+ *
+ * Readings where the page is silent or garbled (each is also listed in the design notes):
+ *   - L_i = { j : max(0, i-w) <= j <= i }            ("look-back radius w", §3.2)
+ *   - C_i = { c : (c+1)s <= i-w }, full cells only    (eq. (6) is missing from the page)
+ *   - RoPE: interleaved pairs (2m, 2m+1), theta_m = base^(-2m/d) (Su et al.)
+ *   - RMSNorm(u) = u / sqrt(mean(u^2) + eps), no learned gain
+ *   - ties in TopP and top-K: larger value first, then the lower cell index
+ *   - |A_i| < K: all of A_i is selected; S_i empty gives o^lr = 0
+ *   - W < 0 and P < 0 together mean "no pruning" (base FS: A_i = C_i)
+ *
+ * Every quantity is computed in double from the float32 inputs (bf16 inputs are
+ * passed as their exact float32 values).  No tiling, fusion or reordering beyond
+ * what the equations state; the only memo is that the rotated keys and the cell
+ * summaries of a (batch, head) are computed once and reused by its rows.
+ *
+ * Parity status: pinned (brute force, closed forms, invariants); see the tests.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    int B, H, Nq, Nk, d;     /* Q is [B,H,Nq,d]; K,V are [B,H,Nk,d]; row-major */
+    int w, s, K;             /* look-back radius, cell size, cells kept per query */
+    int W, P;                /* FS-L recent / norm budgets; both < 0 => no pruning */
+    double rope_base;        /* RoPE base (10000) */
+    double rms_eps;          /* RMSNorm epsilon */
+    long long pos0;          /* absolute position of key index 0 (shift checks) */
+    const double *alpha;     /* [H] range-combination weights, eq. (2) */
+    const double *lambda;    /* [H] prior weights, eq. (7); NULL => 0 */
+    const double *sigma;     /* [H] prior widths, eq. (7); NULL => unused */
+    int mutation;            /* 0 always, except tests that plant a known mistake */
+} orc_params;
+
+/* Planted mistakes, used only by the pin-sensitivity tests. */
+enum {
+    MUT_NONE = 0,
+    MUT_ROPE_KEY_SIGN = 1,   /* keys rotated by R(-j): breaks eq. (3) */
+    MUT_DROP_PRIOR = 2,      /* eq. (7) without the erf term */
+    MUT_WINDOW_SHORT = 3,    /* L_i starts at i-w+1 */
+    MUT_CAND_LOOSE = 4,      /* C_i takes cells with c*s <= i-w (overlapping the window) */
+    MUT_AMAX_MEAN = 5,       /* a_c = mean norm instead of max (eq. (5)) */
+    MUT_NO_EPS = 6,          /* RMSNorm without eps */
+    MUT_ALPHA_ON_SR = 7,     /* o = alpha*o^sr + o^lr (eq. (2) transposed) */
+    MUT_ROPE_IN_READOUT = 8, /* long-range readout uses rotated vectors */
+    MUT_SCALE_D = 9,         /* logits scaled by 1/d instead of 1/sqrt(d) */
+    MUT_TIE_HIGH_INDEX = 10, /* ties broken toward the higher cell index */
+};
+
+int orc_num_cells(const orc_params *p) { return p->s > 0 ? p->Nk / p->s : 0; }
+
+static int pruning_on(const orc_params *p) { return !(p->W < 0 && p->P < 0); }
+
+/* |C_i| for the key-index position i of a query: cells c with (c+1)s <= i-w. */
+int orc_candidate_count(const orc_params *p, long long i)
+{
+    long long lim = i - p->w;                 /* (c+1)s <= lim */
+    if (p->mutation == MUT_CAND_LOOSE) lim += p->s;
+    if (lim < p->s) return 0;
+    long long n = lim / p->s;
+    int C = orc_num_cells(p);
+    return (int)(n < C ? n : C);
+}
+
+/* ---- small deterministic sort: by value descending, then index ascending ---- */
+typedef struct { double v; int idx; } vi_pair;
+
+static int beats(const vi_pair *a, const vi_pair *b, int tie_high)
+{
+    if (a->v > b->v) return 1;
+    if (a->v < b->v) return 0;
+    return tie_high ? (a->idx > b->idx) : (a->idx < b->idx);
+}
+
+static void sort_desc(vi_pair *x, int n, vi_pair *tmp, int tie_high)
+{   /* bottom-up merge sort; stable and O(n log n) */
+    for (int width = 1; width < n; width *= 2) {
+        for (int lo = 0; lo < n; lo += 2 * width) {
+            int mid = lo + width < n ? lo + width : n;
+            int hi = lo + 2 * width < n ? lo + 2 * width : n;
+            int a = lo, b = mid, o = lo;
+            while (a < mid && b < hi) tmp[o++] = beats(&x[b], &x[a], tie_high) ? x[b++] : x[a++];
+            while (a < mid) tmp[o++] = x[a++];
+            while (b < hi) tmp[o++] = x[b++];
+        }
+        memcpy(x, tmp, sizeof(vi_pair) * (size_t)n);
+    }
+}
+
+static int cmp_int(const void *a, const void *b)
+{
+    int x = *(const int *)a, y = *(const int *)b;
+    return (x > y) - (x < y);
+}
+
+/* ---- eq. (5): cell summaries of one (b,h) head ---- */
+static void summaries_bh(const orc_params *p, const float *Kbh, double *kbar, double *amax)
+{
+    const int C = orc_num_cells(p), d = p->d, s = p->s;
+    for (int c = 0; c < C; c++) {
+        double *kb = kbar + (size_t)c * d;
+        for (int m = 0; m < d; m++) kb[m] = 0.0;
+        double best = 0.0, normsum = 0.0;
+        for (int t = 0; t < s; t++) {
+            const float *k = Kbh + ((size_t)c * s + t) * d;
+            double sq = 0.0;
+            for (int m = 0; m < d; m++) {
+                kb[m] += (double)k[m];
+                sq += (double)k[m] * (double)k[m];
+            }
+            double nrm = sqrt(sq);
+            normsum += nrm;
+            if (t == 0 || nrm > best) best = nrm;
+        }
+        for (int m = 0; m < d; m++) kb[m] /= (double)s;
+        amax[c] = (p->mutation == MUT_AMAX_MEAN) ? normsum / s : best;
+    }
+}
+
+/* Summaries for every (b,h): kbar [B,H,C,d], amax [B,H,C]. */
+void orc_cell_summaries(const orc_params *p, const float *K, double *kbar, double *amax)
+{
+    const int C = orc_num_cells(p);
+    #pragma omp parallel for schedule(dynamic)
+    for (int bh = 0; bh < p->B * p->H; bh++)
+        summaries_bh(p, K + (size_t)bh * p->Nk * p->d, kbar + (size_t)bh * C * p->d,
+                     amax + (size_t)bh * C);
+}
+
+/* ---- eq. (8): admitted cells A for a candidate prefix of n cells (ascending) ---- */
+int orc_admitted(const orc_params *p, const double *amax_bh, int n, int *out)
+{
+    if (n <= 0) return 0;
+    if (!pruning_on(p)) {
+        for (int c = 0; c < n; c++) out[c] = c;
+        return n;
+    }
+    char *in = (char *)calloc((size_t)n, 1);
+    int W = p->W < 0 ? 0 : p->W, P = p->P < 0 ? 0 : p->P;
+    for (int c = n - W; c < n; c++)                     /* Recent_W(C_i) */
+        if (c >= 0) in[c] = 1;
+    if (P > 0) {                                        /* TopP over C_i by a_c */
+        vi_pair *x = (vi_pair *)malloc(sizeof(vi_pair) * (size_t)n);
+        vi_pair *tmp = (vi_pair *)malloc(sizeof(vi_pair) * (size_t)n);
+        for (int c = 0; c < n; c++) { x[c].v = amax_bh[c]; x[c].idx = c; }
+        sort_desc(x, n, tmp, p->mutation == MUT_TIE_HIGH_INDEX);
+        for (int t = 0; t < P && t < n; t++) in[x[t].idx] = 1;
+        free(x); free(tmp);
+    }
+    int cnt = 0;
+    for (int c = 0; c < n; c++) if (in[c]) out[cnt++] = c;
+    free(in);
+    return cnt;
+}
+
+/* ---- RoPE (Su et al.): interleaved pairs rotated by pos * theta_m ---- */
+static void rope_rotate(const orc_params *p, const float *x, long long pos, double *out)
+{
+    const int d = p->d;
+    for (int m = 0; m < d / 2; m++) {
+        double theta = pow(p->rope_base, -2.0 * m / (double)d);
+        double ang = (double)pos * theta;
+        double cs = cos(ang), sn = sin(ang);
+        double x0 = x[2 * m], x1 = x[2 * m + 1];
+        out[2 * m] = x0 * cs - x1 * sn;
+        out[2 * m + 1] = x0 * sn + x1 * cs;
+    }
+}
+
+static double logit_scale(const orc_params *p)
+{
+    return p->mutation == MUT_SCALE_D ? 1.0 / p->d : 1.0 / sqrt((double)p->d);
+}
+
+/* ---- eq. (7) + top-K for one query row ----
+ * idx_out[K]: selected cells ascending, -1 padded.  If acells/ascores are given they
+ * receive A_i and the scores r_ic (in A_i's ascending order).  Returns |A_i|. */
+static int select_row(const orc_params *p, const float *qrow, long long i, int h,
+                      const double *kbar_bh, const double *amax_bh,
+                      int *idx_out, int *acells, double *ascores)
+{
+    const int d = p->d, Kc = p->K;
+    int n = orc_candidate_count(p, i);
+    int *A = (int *)malloc(sizeof(int) * (size_t)(n > 0 ? n : 1));
+    int nA = orc_admitted(p, amax_bh, n, A);
+    vi_pair *x = (vi_pair *)malloc(sizeof(vi_pair) * (size_t)(nA > 0 ? nA : 1));
+    vi_pair *tmp = (vi_pair *)malloc(sizeof(vi_pair) * (size_t)(nA > 0 ? nA : 1));
+    double lam = p->lambda ? p->lambda[h] : 0.0;
+    if (p->mutation == MUT_DROP_PRIOR) lam = 0.0;
+    double sig = p->sigma ? p->sigma[h] : 1.0;
+    double pos_i = (double)(p->pos0 + i);
+    for (int t = 0; t < nA; t++) {
+        int c = A[t];
+        const double *kb = kbar_bh + (size_t)c * d;
+        double dot = 0.0;
+        for (int m = 0; m < d; m++) dot += (double)qrow[m] * kb[m];
+        double r = dot * logit_scale(p);
+        if (lam != 0.0) {
+            double p_c = (double)p->pos0 + (c + 0.5) * p->s;
+            r += lam * amax_bh[c] * erf((pos_i - p_c) / (2.0 * sig));
+        }
+        x[t].v = r; x[t].idx = c;
+        if (acells) acells[t] = c;
+        if (ascores) ascores[t] = r;
+    }
+    sort_desc(x, nA, tmp, p->mutation == MUT_TIE_HIGH_INDEX);
+    int keep = nA < Kc ? nA : Kc;
+    for (int t = 0; t < keep; t++) idx_out[t] = x[t].idx;
+    qsort(idx_out, (size_t)keep, sizeof(int), cmp_int);
+    for (int t = keep; t < Kc; t++) idx_out[t] = -1;
+    free(A); free(x); free(tmp);
+    return nA;
+}
+
+/* ---- eq. (9): NoPE token readout over the selected cells, then RMSNorm ---- */
+static void readout_row(const orc_params *p, const float *qrow, long long i,
+                        const float *Kbh, const float *Vbh, const int *idx,
+                        double *u_out, double *olr_out)
+{
+    const int d = p->d, s = p->s, Kc = p->K;
+    int ncell = 0;
+    for (int t = 0; t < Kc; t++) if (idx[t] >= 0) ncell++;
+    double *u = (double *)calloc((size_t)d, sizeof(double));
+    if (ncell > 0) {
+        int ntok = ncell * s;
+        double *lg = (double *)malloc(sizeof(double) * (size_t)ntok);
+        double *qv = (double *)malloc(sizeof(double) * (size_t)d);
+        double *kv = (double *)malloc(sizeof(double) * (size_t)d);
+        if (p->mutation == MUT_ROPE_IN_READOUT) rope_rotate(p, qrow, p->pos0 + i, qv);
+        else for (int m = 0; m < d; m++) qv[m] = qrow[m];
+        int t = 0;
+        double mx = -INFINITY;
+        for (int e = 0; e < Kc; e++) {
+            if (idx[e] < 0) continue;
+            for (int j = idx[e] * s; j < (idx[e] + 1) * s; j++, t++) {
+                const float *k = Kbh + (size_t)j * d;
+                if (p->mutation == MUT_ROPE_IN_READOUT) rope_rotate(p, k, p->pos0 + j, kv);
+                else for (int m = 0; m < d; m++) kv[m] = k[m];
+                double dot = 0.0;
+                for (int m = 0; m < d; m++) dot += qv[m] * kv[m];
+                lg[t] = dot * logit_scale(p);
+                if (lg[t] > mx) mx = lg[t];
+            }
+        }
+        double den = 0.0;
+        t = 0;
+        for (int e = 0; e < Kc; e++) {
+            if (idx[e] < 0) continue;
+            for (int j = idx[e] * s; j < (idx[e] + 1) * s; j++, t++) {
+                double pj = exp(lg[t] - mx);
+                den += pj;
+                const float *v = Vbh + (size_t)j * d;
+                for (int m = 0; m < d; m++) u[m] += pj * (double)v[m];
+            }
+        }
+        for (int m = 0; m < d; m++) u[m] /= den;
+        free(lg); free(qv); free(kv);
+    }
+    double ms = 0.0;
+    for (int m = 0; m < d; m++) ms += u[m] * u[m];
+    ms /= d;
+    double eps = p->mutation == MUT_NO_EPS ? 0.0 : p->rms_eps;
+    double inv = (ncell > 0 && ms + eps > 0.0) ? 1.0 / sqrt(ms + eps) : 0.0;
+    for (int m = 0; m < d; m++) {
+        if (u_out) u_out[m] = u[m];
+        olr_out[m] = u[m] * inv;
+    }
+    free(u);
+}
+
+/* ---- eqs. (3)-(4): RoPE attention over L_i = [max(0,i-w), i] ---- */
+static void window_row(const orc_params *p, const double *qrot, long long i,
+                       const double *krot_bh, const float *Vbh, double *osr)
+{
+    const int d = p->d;
+    long long lo = i - p->w;
+    if (p->mutation == MUT_WINDOW_SHORT) lo += 1;
+    if (lo < 0) lo = 0;
+    long long n = i - lo + 1;
+    double *lg = (double *)malloc(sizeof(double) * (size_t)n);
+    double mx = -INFINITY;
+    for (long long j = lo; j <= i; j++) {
+        const double *k = krot_bh + (size_t)j * d;
+        double dot = 0.0;
+        for (int m = 0; m < d; m++) dot += qrot[m] * k[m];
+        lg[j - lo] = dot * logit_scale(p);
+        if (lg[j - lo] > mx) mx = lg[j - lo];
+    }
+    double den = 0.0;
+    for (int m = 0; m < d; m++) osr[m] = 0.0;
+    for (long long j = lo; j <= i; j++) {
+        double pj = exp(lg[j - lo] - mx);
+        den += pj;
+        const float *v = Vbh + (size_t)j * d;
+        for (int m = 0; m < d; m++) osr[m] += pj * (double)v[m];
+    }
+    for (int m = 0; m < d; m++) osr[m] /= den;
+    free(lg);
+}
+
+/* Per-(b,h) state shared by that head's rows. */
+typedef struct { double *kbar, *amax, *krot; } head_state;
+
+static void head_prepare(const orc_params *p, const float *Kbh, head_state *st)
+{
+    const int C = orc_num_cells(p), d = p->d;
+    st->kbar = (double *)malloc(sizeof(double) * (size_t)(C > 0 ? C : 1) * d);
+    st->amax = (double *)malloc(sizeof(double) * (size_t)(C > 0 ? C : 1));
+    st->krot = (double *)malloc(sizeof(double) * (size_t)p->Nk * d);
+    summaries_bh(p, Kbh, st->kbar, st->amax);
+    #pragma omp parallel for schedule(static)
+    for (int j = 0; j < p->Nk; j++) {
+        long long pos = p->pos0 + j;
+        if (p->mutation == MUT_ROPE_KEY_SIGN) pos = -pos;
+        rope_rotate(p, Kbh + (size_t)j * d, pos, st->krot + (size_t)j * d);
+    }
+}
+
+static void head_release(head_state *st) { free(st->kbar); free(st->amax); free(st->krot); }
+
+/* ---- eq. (2) for a list of rows ----
+ * rows: flat indices (b*H + h)*Nq + r, or NULL for all B*H*Nq rows in order.
+ * O [nrows, d]; idx_out [nrows, K] (may be NULL); olr_out/osr_out [nrows, d] (may be NULL).
+ * Returns 0, or -1 on invalid arguments. */
+int orc_forward(const orc_params *p, const float *Q, const float *K, const float *V,
+                long long nrows, const long long *rows,
+                double *O, int *idx_out, double *olr_out, double *osr_out)
+{
+    if (p->d <= 0 || (p->d & 1) || p->s <= 0 || p->K < 0 || p->w < 0) return -1;
+    if (p->Nq > p->Nk) return -1;
+    const int d = p->d, BH = p->B * p->H;
+    const long long total = (long long)BH * p->Nq;
+    if (!rows) nrows = total;
+    /* bucket the requested rows by head so that each head is prepared once */
+    long long *order = (long long *)malloc(sizeof(long long) * (size_t)(nrows > 0 ? nrows : 1));
+    long long *start = (long long *)calloc((size_t)BH + 1, sizeof(long long));
+    for (long long t = 0; t < nrows; t++) {
+        long long f = rows ? rows[t] : t;
+        if (f < 0 || f >= total) { free(order); free(start); return -1; }
+        start[f / p->Nq + 1]++;
+    }
+    for (int bh = 0; bh < BH; bh++) start[bh + 1] += start[bh];
+    long long *fill = (long long *)malloc(sizeof(long long) * (size_t)BH);
+    for (int bh = 0; bh < BH; bh++) fill[bh] = start[bh];
+    for (long long t = 0; t < nrows; t++) {
+        long long f = rows ? rows[t] : t;
+        order[fill[f / p->Nq]++] = t;
+    }
+    free(fill);
+
+    for (int bh = 0; bh < BH; bh++) {
+        if (start[bh] == start[bh + 1]) continue;
+        const int h = bh % p->H;
+        const float *Kbh = K + (size_t)bh * p->Nk * d;
+        const float *Vbh = V + (size_t)bh * p->Nk * d;
+        head_state st;
+        head_prepare(p, Kbh, &st);
+        #pragma omp parallel for schedule(dynamic, 4)
+        for (long long e = start[bh]; e < start[bh + 1]; e++) {
+            long long t = order[e];
+            long long f = rows ? rows[t] : t;
+            int r = (int)(f % p->Nq);
+            long long i = (long long)(p->Nk - p->Nq) + r;   /* key-index position of row r */
+            const float *qrow = Q + (size_t)f * d;
+            double *qrot = (double *)malloc(sizeof(double) * (size_t)d);
+            double *osr = (double *)malloc(sizeof(double) * (size_t)d);
+            double *olr = (double *)malloc(sizeof(double) * (size_t)d);
+            int *idx = (int *)malloc(sizeof(int) * (size_t)(p->K > 0 ? p->K : 1));
+            rope_rotate(p, qrow, p->pos0 + i, qrot);
+            window_row(p, qrot, i, st.krot, Vbh, osr);
+            select_row(p, qrow, i, h, st.kbar, st.amax, idx, NULL, NULL);
+            readout_row(p, qrow, i, Kbh, Vbh, idx, NULL, olr);
+            double a = p->alpha ? p->alpha[h] : 0.0;
+            for (int m = 0; m < d; m++) {
+                O[(size_t)t * d + m] = (p->mutation == MUT_ALPHA_ON_SR)
+                                           ? a * osr[m] + olr[m] : osr[m] + a * olr[m];
+                if (olr_out) olr_out[(size_t)t * d + m] = olr[m];
+                if (osr_out) osr_out[(size_t)t * d + m] = osr[m];
+            }
+            if (idx_out) memcpy(idx_out + (size_t)t * p->K, idx, sizeof(int) * (size_t)p->K);
+            free(qrot); free(osr); free(olr); free(idx);
+        }
+        head_release(&st);
+    }
+    free(order); free(start);
+    return 0;
+}
+
+/* ---- single-step entry points for the tests ---- */
+
+/* Selection for one row (b,h,r) given its head's summaries.  Writes idx_out[K];
+ * acells/ascores (capacity >= |C_i|) receive A_i and its scores.  Returns |A_i|. */
+int orc_select_row(const orc_params *p, const float *Q, const double *kbar, const double *amax,
+                   int b, int h, int r, int *idx_out, int *acells, double *ascores)
+{
+    const int C = orc_num_cells(p);
+    size_t bh = (size_t)b * p->H + h;
+    long long i = (long long)(p->Nk - p->Nq) + r;
+    return select_row(p, Q + (bh * p->Nq + r) * p->d, i, h, kbar + bh * C * p->d,
+                      amax + bh * C, idx_out, acells, ascores);
+}
+
+/* Readout for one row on caller-given cells idx[K] (ascending, -1 padded). */
+void orc_readout_row(const orc_params *p, const float *Q, const float *K, const float *V,
+                     int b, int h, int r, const int *idx, double *u_out, double *olr_out)
+{
+    size_t bh = (size_t)b * p->H + h;
+    long long i = (long long)(p->Nk - p->Nq) + r;
+    readout_row(p, Q + (bh * p->Nq + r) * p->d, i, K + bh * p->Nk * p->d,
+                V + bh * p->Nk * p->d, idx, u_out, olr_out);
+}
+
+/* Readout for many rows, each on its own caller-given cells (rows as in orc_forward). */
+void orc_readout_rows(const orc_params *p, const float *Q, const float *K, const float *V,
+                      long long nrows, const long long *rows, const int *idx,
+                      double *u_out, double *olr_out)
+{
+    #pragma omp parallel for schedule(dynamic, 8)
+    for (long long t = 0; t < nrows; t++) {
+        long long f = rows[t];
+        int r = (int)(f % p->Nq);
+        long long bh = f / p->Nq;
+        orc_readout_row(p, Q, K, V, (int)(bh / p->H), (int)(bh % p->H), r,
+                        idx + (size_t)t * p->K, u_out ? u_out + (size_t)t * p->d : NULL,
+                        olr_out + (size_t)t * p->d);
+    }
+}
+
+/* RoPE rotation of one vector at an absolute position (exposed for the eq. (3) check). */
+void orc_rope(const orc_params *p, const float *x, long long pos, double *out)
+{
+    rope_rotate(p, x, pos, out);
+}

@@ -1,0 +1,328 @@
+"""Pins for the float64 oracle (CPU only).
+
+The oracle is checked against things other than itself: a brute-force dense-mask
+restatement on tiny inputs, library attention (torch SDPA in float64) in the special
+cases where the method reduces to it, closed forms, invariants stated on the
+"FreeSolo" summary page, and hand-worked fixtures under tests/golden/.  A final test
+plants known mistakes in the oracle and checks that some pin catches each one.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import Workload, generate, small
+from tests._brute import brute_forward, rope_complex, sel_to_idx
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def make_problem(inp, mutation=0, **over):
+    wl = inp.wl
+    kw = dict(w=wl.w, s=wl.s, K_cells=wl.K, W=wl.W, P=wl.P, alpha=inp.alpha,
+              lam=inp.lam, sigma=inp.sigma, rope_base=wl.rope_base, rms_eps=wl.rms_eps)
+    kw.update(over)
+    return oracle.Problem(inp.Q, inp.K, inp.V, mutation=mutation, **kw)
+
+
+def tiny(**kw):
+    base = dict(B=1, H=2, Nq=192, Nk=192, d=8, w=32, s=8, K=3, W=2, P=3, seed=5)
+    base.update(kw)
+    return generate(small("tiny", **base))
+
+
+TINY_CASES = {
+    "prune": dict(),
+    "noprune": dict(W=-1, P=-1),
+    "prior": dict(lam=0.5, sigma=24.0),
+    "decode": dict(Nq=40, Nk=200),
+    "bigK": dict(K=40, W=-1, P=-1),
+    "needles": dict(needles=2, needle_queries=6, Nq=256, Nk=256),
+    "rag": dict(Nq=150, Nk=203),
+}
+
+
+# ---------------------------------------------------------------- brute force
+@pytest.mark.parametrize("case", sorted(TINY_CASES))
+def test_oracle_matches_bruteforce(case):
+    inp = tiny(**TINY_CASES[case])
+    wl = inp.wl
+    prob = make_problem(inp)
+    O, idx = prob.forward(want_idx=True)
+    Ob, sel, _, _, _ = brute_forward(inp.Q, inp.K, inp.V, w=wl.w, s=wl.s, K_cells=wl.K,
+                                     W=wl.W, P=wl.P, alpha=inp.alpha, lam=inp.lam,
+                                     sigma=inp.sigma, rope_base=wl.rope_base,
+                                     rms_eps=wl.rms_eps)
+    np.testing.assert_array_equal(idx, sel_to_idx(sel, wl.K))
+    np.testing.assert_allclose(O, Ob, rtol=0, atol=1e-12)
+
+
+def test_oracle_matches_bruteforce_with_exact_ties():
+    """Duplicated cells give exact ties in a_c and in the scores (tie rule G9)."""
+    inp = tiny(H=1, Nq=160, Nk=160, seed=9)
+    K = inp.K.copy()
+    s = inp.wl.s
+    for c in (1, 4, 7, 10):                     # four identical cells
+        K[0, 0, c * s:(c + 1) * s] = K[0, 0, 0:s]
+    inp.K = K
+    wl = inp.wl
+    for W_, P_ in ((2, 3), (0, 2), (-1, -1)):
+        prob = make_problem(inp, W=W_, P=P_)
+        O, idx = prob.forward(want_idx=True)
+        Ob, sel, _, _, _ = brute_forward(inp.Q, inp.K, inp.V, w=wl.w, s=s, K_cells=wl.K,
+                                         W=W_, P=P_, alpha=inp.alpha)
+        np.testing.assert_array_equal(idx, sel_to_idx(sel, wl.K))
+        np.testing.assert_allclose(O, Ob, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- eq. (3) identity
+def test_rope_relative_identity():
+    """(R(i)q)^T (R(j)k) = q^T R(j-i) k, and R preserves norms (eq. (3))."""
+    inp = tiny(d=64, seed=3)
+    prob = make_problem(inp)
+    rng = np.random.default_rng(0)
+    for _ in range(20):
+        q = rng.standard_normal(64).astype(np.float32)
+        k = rng.standard_normal(64).astype(np.float32)
+        i, j = (int(v) for v in rng.integers(0, 300000, 2))
+        lhs = prob.rope(q, i) @ prob.rope(k, j)
+        rhs = q.astype(np.float64) @ prob.rope(k, j - i)
+        assert abs(lhs - rhs) < 1e-9 * (1 + abs(lhs))
+        assert abs(np.linalg.norm(prob.rope(q, i)) - np.linalg.norm(q.astype(np.float64))) < 1e-12
+
+
+def test_rope_against_complex_rotation():
+    inp = tiny(d=64, seed=4)
+    prob = make_problem(inp)
+    x = np.random.default_rng(1).standard_normal(64).astype(np.float32)
+    for pos in (0, 1, 17, 4096, 262271):
+        ref = rope_complex(x[None, :].astype(np.float64), np.array([pos]), 64, 10000.0)[0]
+        # theta_m rounding (1e-16 relative) times pos ~ 2.6e5 bounds the difference
+        np.testing.assert_allclose(prob.rope(x, pos), ref, rtol=0, atol=1e-9)
+
+
+# ---------------------------------------------------------------- library reductions
+def _sdpa(q, k, v, mask):
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float64))[None, None]
+    out = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v),
+                                                           attn_mask=t(mask).bool())
+    return out[0, 0].numpy()
+
+
+def test_full_window_is_causal_rope_attention():
+    """w >= N and alpha = 0: the output is full causal RoPE attention."""
+    inp = generate(small("full", Nq=256, Nk=256, d=64, w=10_000, s=32, K=4, seed=21))
+    prob = make_problem(inp, alpha=np.zeros(2))
+    O = prob.forward()
+    N = 256
+    mask = np.tril(np.ones((N, N), bool))
+    for h in range(2):
+        pos = np.arange(N)
+        qr = rope_complex(inp.Q[0, h].astype(np.float64), pos, 64, 10000.0)
+        kr = rope_complex(inp.K[0, h].astype(np.float64), pos, 64, 10000.0)
+        ref = _sdpa(qr, kr, inp.V[0, h], mask)
+        np.testing.assert_allclose(O[0, h], ref, rtol=0, atol=1e-12)
+
+
+def test_alpha_zero_is_sliding_window_attention():
+    inp = generate(small("sw", Nq=300, Nk=300, d=64, w=64, s=16, K=4, seed=22))
+    prob = make_problem(inp, alpha=np.zeros(2))
+    O = prob.forward()
+    i = np.arange(300)
+    mask = (i[None, :] <= i[:, None]) & (i[None, :] >= i[:, None] - 64)
+    for h in range(2):
+        qr = rope_complex(inp.Q[0, h].astype(np.float64), i, 64, 10000.0)
+        kr = rope_complex(inp.K[0, h].astype(np.float64), i, 64, 10000.0)
+        np.testing.assert_allclose(O[0, h], _sdpa(qr, kr, inp.V[0, h], mask), rtol=0, atol=1e-12)
+
+
+def test_long_range_with_all_cells_is_dense_nope_attention():
+    """No pruning, K >= |C_i|, lambda = 0: u_i is dense NoPE attention over the prefix."""
+    inp = generate(small("dense", Nq=400, Nk=400, d=64, w=64, s=16, K=64, W=-1, P=-1,
+                         seed=23))
+    prob = make_problem(inp)
+    _, _, olr, _ = prob.forward(want_idx=True, want_parts=True)
+    N, s, w = 400, 16, 64
+    i = np.arange(N)
+    n = np.where(i - w >= s, (i - w) // s, 0)
+    mask = np.arange(N)[None, :] < (n * s)[:, None]
+    has = n > 0
+    for h in range(2):
+        q = inp.Q[0, h].astype(np.float64)
+        k = inp.K[0, h].astype(np.float64)
+        # SDPA rows with an empty mask are undefined; give them one dummy key
+        m2 = mask.copy()
+        m2[~has, 0] = True
+        u = _sdpa(q, k, inp.V[0, h], m2)
+        ms = (u ** 2).mean(axis=1, keepdims=True)
+        ref = np.where(has[:, None], u / np.sqrt(ms + 1e-6), 0.0)
+        np.testing.assert_allclose(olr[0, h], ref, rtol=0, atol=1e-11)
+
+
+# ---------------------------------------------------------------- closed forms
+def test_softmax_rows_sum_to_one():
+    """V = 1: o^sr = 1 and o^lr = 1/sqrt(1+eps) wherever a cell is selected (eqs. (4), (9))."""
+    inp = tiny(d=16, Nq=200, Nk=200, seed=8)
+    inp.V = np.ones_like(inp.V)
+    prob = make_problem(inp)
+    O, idx, olr, osr = prob.forward(want_idx=True, want_parts=True)
+    np.testing.assert_allclose(osr, 1.0, rtol=0, atol=1e-13)
+    has = (idx >= 0).any(axis=-1)
+    assert has.any() and (~has).any()
+    np.testing.assert_allclose(olr[has], 1.0 / math.sqrt(1.0 + 1e-6), rtol=0, atol=1e-13)
+    np.testing.assert_array_equal(olr[~has], 0.0)
+    a = inp.alpha[None, :, None, None]
+    np.testing.assert_allclose(O, osr + a * olr, rtol=0, atol=1e-13)
+
+
+def test_rmsnorm_closed_form():
+    """mean(o_lr^2) = mean(u^2) / (mean(u^2) + eps) for the oracle's own u (eq. (9))."""
+    inp = tiny(d=64, Nq=256, Nk=256, seed=12)
+    prob = make_problem(inp, rms_eps=1e-4)
+    _, idx = prob.forward(want_idx=True)
+    rows = np.arange(inp.wl.B * inp.wl.H * inp.wl.Nq)
+    u, olr = prob.readout_rows(rows, idx.reshape(-1, inp.wl.K))
+    has = (idx.reshape(-1, inp.wl.K) >= 0).any(axis=1)
+    mu = (u[has] ** 2).mean(axis=1)
+    np.testing.assert_allclose((olr[has] ** 2).mean(axis=1), mu / (mu + 1e-4), rtol=1e-12)
+
+
+def test_summaries_closed_form():
+    """eq. (5): a cell of identical keys has kbar = that key and a_c = its norm;
+    a cell with one long key has a_c = that key's norm."""
+    inp = tiny(H=1, Nq=64, Nk=64, d=8, s=8, seed=2)
+    K = inp.K.copy()
+    K[0, 0, 0:8] = K[0, 0, 3]
+    K[0, 0, 8:16] *= 0.01
+    K[0, 0, 13] = np.float32([3, 4, 0, 0, 0, 0, 0, 0])
+    inp.K = K
+    kbar, amax = make_problem(inp).summaries()
+    np.testing.assert_allclose(kbar[0, 0, 0], K[0, 0, 3], rtol=1e-7)
+    assert abs(amax[0, 0, 0] - np.linalg.norm(K[0, 0, 3].astype(np.float64))) < 1e-12
+    assert abs(amax[0, 0, 1] - 5.0) < 1e-12
+    np.testing.assert_allclose(kbar[0, 0, 2], K[0, 0, 16:24].astype(np.float64).mean(0), rtol=1e-12)
+
+
+def test_candidate_count_closed_form():
+    """C_i = {c : (c+1)s <= i - w}: empty before i = w + s, then one cell per s tokens."""
+    prob = make_problem(tiny(w=512, s=32, Nq=2048, Nk=2048, d=8))
+    assert prob.candidate_count(0) == 0
+    assert prob.candidate_count(512 + 31) == 0
+    assert prob.candidate_count(512 + 32) == 1
+    assert prob.candidate_count(512 + 63) == 1
+    assert prob.candidate_count(512 + 64) == 2
+    assert prob.candidate_count(2047) == (2047 - 512) // 32
+
+
+def test_admitted_set_invariants():
+    """|A_i| <= W + P, Recent_W is inside A_i, A_i is inside C_i (eq. (8))."""
+    inp = tiny(Nq=512, Nk=512, seed=14)
+    prob = make_problem(inp, W=3, P=5)
+    _, amax = prob.summaries()
+    for n in range(0, prob.C + 1):
+        A = prob.admitted(amax[0, 0], n)
+        assert len(A) <= 8 and len(A) == len(set(A.tolist()))
+        assert all(0 <= c < n for c in A)
+        assert set(range(max(0, n - 3), n)) <= set(A.tolist())
+        if n <= 5:                               # TopP alone already covers C_i
+            assert len(A) == n
+
+
+def test_shift_invariance():
+    """Shifting tokens, cells and queries together by a multiple of s leaves o unchanged
+    ("Position Independence": RoPE is relative, the erf prior depends on i - p_c)."""
+    inp = tiny(d=64, Nq=64, Nk=256, w=48, s=8, K=4, lam=0.7, sigma=20.0, seed=15)
+    base = make_problem(inp).forward()
+    for pos0 in (8, 800, 123456):
+        shifted = make_problem(inp, pos0=pos0).forward()
+        np.testing.assert_allclose(shifted, base, rtol=0, atol=1e-11)
+
+
+def test_needles_are_selected():
+    """Planted high-norm cells aligned with a query are selected by that query."""
+    inp = generate(small("needle", B=1, H=2, Nq=2048, Nk=2048, d=64, w=512, s=32, K=4,
+                         W=4, P=8, needles=3, needle_queries=5, seed=31))
+    _, idx = make_problem(inp).forward(want_idx=True)
+    assert len(inp.needle_cells) == 6
+    for b, h, c, rows in inp.needle_cells:
+        for r in rows:
+            assert c in idx[b, h, r], (b, h, c, r)
+
+
+# ---------------------------------------------------------------- golden fixtures
+def _read_fixture(name):
+    hdr, rows = {}, []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if not line:
+                continue
+            if ":" in line:
+                k, v = line.split(":")
+                rows.append((int(k), [int(t) for t in v.split()]))
+            else:
+                toks = line.split()
+                hdr[toks[0]] = [float(t) for t in toks[1:]]
+    return hdr, rows
+
+
+def test_golden_prune_eq8():
+    hdr, rows = _read_fixture("prune_eq8.txt")
+    a = np.array(hdr["a"], np.float64)
+    inp = tiny(H=1, Nq=8, Nk=64, d=8, s=8)
+    prob = make_problem(inp, W=int(hdr["W"][0]), P=int(hdr["P"][0]))
+    for n, cells in rows:
+        assert prob.admitted(a, n).tolist() == cells, n
+
+
+def test_golden_select_ties_eq7():
+    hdr, rows = _read_fixture("select_ties_eq7.txt")
+    x = np.array(hdr["x"], np.float32)
+    Q = np.zeros((1, 1, 1, 2), np.float32)
+    Q[..., 0] = 1.0
+    K = np.zeros((1, 1, 8, 2), np.float32)
+    K[0, 0, :, 0] = x
+    V = np.zeros_like(K)
+    for Kc, cells in rows:
+        prob = oracle.Problem(Q, K, V, w=0, s=1, K_cells=Kc, W=-1, P=-1, alpha=[1.0])
+        kbar, amax = prob.summaries()
+        idx, acells, scores = prob.select_row(kbar, amax, 0, 0, 0)
+        assert acells.tolist() == list(range(7))
+        np.testing.assert_allclose(scores, x[:7].astype(np.float64) / math.sqrt(2), rtol=1e-15)
+        assert idx.tolist() == cells, Kc
+
+
+# ---------------------------------------------------------------- sensitivity
+def _pins_fail(mutation):
+    """Run a compact set of the pins above against a mutated oracle; True if any fails."""
+    failures = []
+    inp = tiny(d=16, Nq=200, Nk=200, lam=0.8, sigma=16.0, seed=41)
+    wl = inp.wl
+    for W_, P_ in ((2, 3), (-1, -1)):
+        prob = make_problem(inp, mutation=mutation, W=W_, P=P_)
+        O, idx = prob.forward(want_idx=True)
+        Ob, sel, _, _, _ = brute_forward(inp.Q, inp.K, inp.V, w=wl.w, s=wl.s, K_cells=wl.K,
+                                         W=W_, P=P_, alpha=inp.alpha, lam=inp.lam,
+                                         sigma=inp.sigma)
+        if not np.array_equal(idx, sel_to_idx(sel, wl.K)) or np.abs(O - Ob).max() > 1e-12:
+            failures.append("brute")
+    try:
+        hdr, rows = _read_fixture("prune_eq8.txt")
+        p2 = make_problem(tiny(H=1, Nq=8, Nk=64, d=8, s=8), mutation=mutation, W=2, P=3)
+        if any(p2.admitted(np.array(hdr["a"]), n).tolist() != c for n, c in rows):
+            failures.append("golden_prune")
+    except Exception:
+        failures.append("golden_prune")
+    return failures
+
+
+@pytest.mark.parametrize("mutation", sorted(oracle.MUTATIONS))
+def test_planted_mistakes_are_caught(mutation):
+    assert _pins_fail(mutation), "mutation %s passed every pin" % mutation
+
+
+def test_unmutated_oracle_passes_the_sensitivity_pins():
+    assert _pins_fail(0) == []
