@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""FreeSolo forward-pass benchmark: query-tokens/s on one B200 and % of roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+The timed workload is the long prefill: B=1, H=16, N=65536, d=64, w=512, s=32, K=32,
+W=16, P=48, bf16, synthetic inputs (workloads.CONFIGS["prefill64k"]).  A step is one
+fs_forward call through the C ABI over the whole batch (cell summaries, pruning,
+selection, readout, window + combine).  Inputs are resident in HBM when timing starts;
+Q+K+V (384 MiB) exceed the 126 MB L2, so no flush is done between steps.
+
+With N > 1 (torchrun), each rank runs an independent replica of the workload on its own
+GPU (the heads of different sequences share nothing, so no collective is needed): weak
+scaling, value = all ranks' query tokens / the slowest rank's time.
+
+--impl reference times the float64 CPU oracle on the host cores on a bounded sample of
+the same workload (rank 0 only).
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FreeSolo fwd query-tokens/s at N=16k/64k/256k on 1 B200; % of roofline"
+UNIT = "query-tokens/s"
+WORKLOAD = "prefill64k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+# fp32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flop (FMA) x SM clock
+SMS, FP32_LANES = 148, 128
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--quick", action="store_true", help="skip e2e, CPU baseline, extras")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class Clocks:
+    """nvidia-smi samples of one GPU every 200 ms while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = str(gpu_index)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.Q, "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", self.gpu], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def reduce_max(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def gpu_index(local):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local < len(ids):
+            return ids[local]
+    return str(local)
+
+
+# ------------------------------------------------------------------ work model
+def algorithmic_work(wl, n_sel_cells):
+    """Per-launch algorithmic bytes / flops of each kernel for one forward pass."""
+    BH = wl.B * wl.H
+    C = wl.Nk // wl.s
+    e = 2 if wl.dtype == "bf16" else 4
+    q0 = wl.Nk - wl.Nq
+    i = q0 + np.arange(wl.Nq, dtype=np.int64)
+    win = np.minimum(i, wl.w) + 1                    # |L_i| = min(i, w) + 1 keys
+    win_keys = int(win.sum()) * BH
+    qkv = BH * (wl.Nq + 2 * wl.Nk) * wl.d * e
+    o = BH * wl.Nq * wl.d * e
+    return {
+        "cell_summaries": ("hbm", BH * C * wl.s * wl.d * e + BH * C * (wl.d + 1) * 4),
+        "exit_times": ("hbm", BH * C * 8),
+        "select_topk": ("hbm", BH * wl.Nq * wl.d * e + BH * C * wl.d * 4 + BH * wl.Nq * wl.K * 4),
+        "readout": ("alu", 4 * wl.d * wl.s * n_sel_cells),
+        "window_combine": ("alu", 4 * wl.d * win_keys),
+        "_path_bytes": qkv + o + BH * C * (wl.d + 1) * 4 * 2,
+        "_window_flops": 4 * wl.d * win_keys,
+        "_readout_flops": 4 * wl.d * wl.s * n_sel_cells,
+    }
+
+
+def source_hash(kernel):
+    files = {"readout": "fs_readout.cu", "window_combine": "fs_window.cu",
+             "cell_summaries": "fs_summaries.cu", "exit_times": "fs_prune.cu",
+             "select_topk": "fs_select.cu"}
+    path = os.path.join(ROOT, "long_context_sparse_head_b200", "csrc", files.get(kernel, ""))
+    if not os.path.isfile(path):
+        return None
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if its kernel source matches."""
+    path = os.path.join(ROOT, "profiles", "traffic_%s_%s.txt" % (kernel, workload))
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("source_sha256_16") != source_hash(kernel):
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def oracle_sample(inp, max_seconds, rows_per_head_stride):
+    """Time the float64 oracle on every `stride`-th query row of every head."""
+    import oracle
+    wl = inp.wl
+    prob = oracle.Problem(inp.Q, inp.K, inp.V, w=wl.w, s=wl.s, K_cells=wl.K, W=wl.W, P=wl.P,
+                          alpha=inp.alpha, lam=inp.lam, sigma=inp.sigma,
+                          rope_base=wl.rope_base, rms_eps=wl.rms_eps)
+    BH = wl.B * wl.H
+    done_rows, t_total = 0, 0.0
+    for bh in range(BH):
+        rows = bh * wl.Nq + np.arange(0, wl.Nq, rows_per_head_stride, dtype=np.int64)
+        t = time.perf_counter()
+        prob.forward(rows=rows)
+        t_total += time.perf_counter() - t
+        done_rows += len(rows)
+        if t_total > max_seconds:
+            break
+    # a query token is one position across all H heads
+    return (done_rows / wl.H) / t_total, done_rows, t_total, bh + 1
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+# ------------------------------------------------------------------ arms
+def run_reference(args):
+    """The float64 oracle on the host cores; each step is one head's every-8th query row."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from workloads import CONFIGS, generate
+    wl = CONFIGS[args.workload]
+    inp = generate(wl)
+    prob = oracle.Problem(inp.Q, inp.K, inp.V, w=wl.w, s=wl.s, K_cells=wl.K, W=wl.W, P=wl.P,
+                          alpha=inp.alpha, lam=inp.lam, sigma=inp.sigma,
+                          rope_base=wl.rope_base, rms_eps=wl.rms_eps)
+    stride, BH = 8, wl.B * wl.H
+    t_sum, rows_sum, times = 0.0, 0, []
+    for k in range(args.warmup + args.steps):
+        bh = k % BH
+        rows = bh * wl.Nq + np.arange((k // BH) % stride, wl.Nq, stride, dtype=np.int64)
+        t0 = time.perf_counter()
+        prob.forward(rows=rows)
+        dt = time.perf_counter() - t0
+        if k >= args.warmup:
+            times.append(dt)
+            t_sum += dt
+            rows_sum += len(rows)
+    value = (rows_sum / wl.H) / t_sum              # a query token spans all H heads
+    sample = ("per step: every %dth query row of one head (%d rows, all of that head's "
+              "rotated keys and cell summaries), cycling over the %d heads" %
+              (stride, wl.Nq // stride, BH))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * float(np.mean(times)), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(wl, world),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(wl, world):
+    return {"workload": "%s: B=%d H=%d Nq=%d Nk=%d d=%d w=%d s=%d K=%d W=%d P=%d lambda=0 %s"
+                        % (wl.name, wl.B, wl.H, wl.Nq, wl.Nk, wl.d, wl.w, wl.s, wl.K, wl.W,
+                           wl.P, wl.dtype),
+            "global_batch": wl.B * world, "seq_len": wl.Nk, "heads": wl.H,
+            "parallelism": "replicas" if world > 1 else "single",
+            "l2": "inputs larger than L2 (Q+K+V %d MiB vs 126 MB); no flush"
+                  % ((wl.B * wl.H * (wl.Nq + 2 * wl.Nk) * wl.d * 2) >> 20)}
+
+
+def make_params(fs, inp, **over):
+    wl = inp.wl
+    kw = dict(B=wl.B, H=wl.H, Nq=wl.Nq, Nk=wl.Nk, d=wl.d, w=wl.w, s=wl.s, K=wl.K, W=wl.W,
+              P=wl.P, alpha=inp.alpha, lam=inp.lam, sigma=inp.sigma, rope_base=wl.rope_base,
+              rms_eps=wl.rms_eps, dtype=wl.dtype)
+    kw.update(over)
+    return fs.Params(**kw)
+
+
+def time_workload(fs, torch, inp, steps, warmup, archive=False):
+    """Device time per fs_forward step (ms); archive=True passes precomputed summaries."""
+    wl = inp.wl
+    p = make_params(fs, inp)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    Q, K, V = (torch.from_numpy(x).cuda().to(dt) for x in (inp.Q, inp.K, inp.V))
+    O = torch.empty_like(Q)
+    ws = fs.alloc_workspace(p)
+    kbar = amax = None
+    if archive:
+        kbar = torch.empty((wl.B, wl.H, p.C, wl.d), dtype=torch.float32, device="cuda")
+        amax = torch.empty((wl.B, wl.H, p.C), dtype=torch.float32, device="cuda")
+        fs.cell_summaries(p, K, kbar, amax)
+    for _ in range(warmup):
+        fs.forward(p, Q, K, V, O, ws, kbar=kbar, amax=amax)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fs.forward(p, Q, K, V, O, ws, kbar=kbar, amax=amax)
+    b.record()
+    torch.cuda.synchronize()
+    fs.sync_status(ws)
+    return a.elapsed_time(b) / steps
+
+
+def run_ours(args):
+    import torch
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    import long_context_sparse_head_b200 as fs
+    from workloads import CONFIGS, generate
+    fs.load()
+    pk, pk_src = peaks()
+    wl = CONFIGS[args.workload]
+    wl = wl.with_(seed=wl.seed + 1000 * rank)          # independent replica per rank
+    inp = generate(wl)
+    p = make_params(fs, inp)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    Q, K, V = (torch.from_numpy(x).cuda().to(dt).contiguous() for x in (inp.Q, inp.K, inp.V))
+    O = torch.empty_like(Q)
+    ws = fs.alloc_workspace(p)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(max(args.warmup, 3)):
+        fs.forward(p, Q, K, V, O, ws)
+    fs.sync_status(ws)
+    barrier(world)
+    torch.cuda.synchronize()
+
+    clocks = Clocks(gpu_index(local))
+    fs.kernel_times()                                 # clear
+    fs.timing_enable(True)
+    n0 = fs.launch_count()
+    clocks.start()
+    ev_a, ev_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev_a.record(stream)
+    for _ in range(args.steps):
+        fs.forward(p, Q, K, V, O, ws)
+    ev_b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    launches = fs.launch_count() - n0
+    fs.timing_enable(False)
+    ktimes = fs.kernel_times()
+    fs.sync_status(ws)
+    ms_step = reduce_max(ev_a.elapsed_time(ev_b) / args.steps, world)
+    value = wl.queries * world / (ms_step * 1e-3)
+
+    # exact |S_i| counts for the readout's algorithmic flops (outside the timed region)
+    idx = torch.empty((wl.B, wl.H, wl.Nq, wl.K), dtype=torch.int32, device="cuda")
+    kbar = torch.empty((wl.B, wl.H, p.C, wl.d), dtype=torch.float32, device="cuda")
+    amax = torch.empty((wl.B, wl.H, p.C), dtype=torch.float32, device="cuda")
+    fs.cell_summaries(p, K, kbar, amax)
+    fs.select_topk(p, Q, kbar, amax, idx, ws)
+    n_sel = int((idx >= 0).sum().item())
+    work = algorithmic_work(wl, n_sel)
+    dom = max((k for k in ktimes if ktimes[k][0] > 0), key=lambda k: ktimes[k][1])
+    cnt, tot_ms = ktimes[dom]
+    avg_s = tot_ms / cnt * 1e-3
+    bound, amount = work[dom]
+    clock_mhz = pk.get("sm_max_mhz", 1965.0)
+    if bound == "hbm":
+        peak, unit, achieved = pk["hbm_gbs"], "GB/s", amount / avg_s / 1e9
+    elif bound == "tensor":
+        peak, unit, achieved = pk["bf16_tflops_sustained"], "TFLOP/s", amount / avg_s / 1e12
+    else:
+        peak = SMS * FP32_LANES * 2 * clock_mhz * 1e6 / 1e12
+        unit, achieved = "TFLOP/s", amount / avg_s / 1e12
+    roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": profiled_traffic(dom, args.workload),
+                "peak_source": ("derived: 148 SMs x 128 FP32 lanes x 2 x %.0f MHz" % clock_mhz
+                                if bound == "alu" else pk_src),
+                "launches": cnt, "avg_ms": tot_ms / cnt,
+                "kernels_ms_per_step": {k: v[1] / max(args.steps, 1) for k, v in ktimes.items()}}
+    # whole-path roofline: compulsory bytes at HBM vs window (and all) flops at tensor peak
+    t_bytes = work["_path_bytes"] / (pk["hbm_gbs"] * 1e9)
+    t_win = work["_window_flops"] / (pk["bf16_tflops"] * 1e12)
+    t_all = (work["_window_flops"] + work["_readout_flops"]) / (pk["bf16_tflops"] * 1e12)
+    path = {"t_literal_us": 1e6 * max(t_bytes, t_win), "t_strict_us": 1e6 * max(t_bytes, t_all),
+            "frac_literal": 1e3 * max(t_bytes, t_win) / ms_step,
+            "frac_strict": 1e3 * max(t_bytes, t_all) / ms_step,
+            "selected_cells": n_sel}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": wl.dtype, "data": "synthetic", "config": config_dict(wl, world),
+            "roofline": roofline, "path_roofline": path, "gpu_launches": launches,
+            "clocks": clk}
+
+    if not args.quick:
+        # end to end through the public host-buffer entry point: pinned H2D, compute, D2H
+        hQ, hK, hV = (torch.from_numpy(x).to(dt).pin_memory() for x in (inp.Q, inp.K, inp.V))
+        hO = torch.empty(hQ.shape, dtype=dt).pin_memory()
+        scratch = torch.zeros(fs.host_scratch_size(p), dtype=torch.uint8, device="cuda")
+        for _ in range(2):
+            fs.forward_host(p, hQ, hK, hV, hO, scratch)
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_steps = max(3, min(args.steps, 10))
+        for _ in range(e2e_steps):
+            fs.forward_host(p, hQ, hK, hV, hO, scratch)
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = reduce_max(a.elapsed_time(b) / e2e_steps, world)
+        esz = hQ.element_size()
+        line["e2e"] = {"value": wl.queries * world / (e2e_ms * 1e-3), "unit": UNIT,
+                       "ms_per_step": e2e_ms,
+                       "h2d_bytes_per_step": (hQ.numel() + hK.numel() + hV.numel()) * esz,
+                       "d2h_bytes_per_step": hO.numel() * esz}
+        del scratch, hQ, hK, hV, hO
+        if world == 1:
+            rate, rows, t, heads = oracle_sample(inp, 12.0, 8)
+            line["cpu_baseline"] = {
+                "value": rate, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                "sample": "every 8th query row of %d of %d heads (%d rows, %.1f s)"
+                          % (heads, wl.B * wl.H, rows, t)}
+            # the other two sizes the metric names, as extra context (same kernels)
+            extras = {}
+            del Q, K, V, O, ws
+            torch.cuda.empty_cache()
+            for name, arch in (("prefill16k", False), ("decode256k", True)):
+                inp2 = generate(CONFIGS[name])
+                ms2 = time_workload(fs, torch, inp2, 10, 3, archive=arch)
+                extras[name] = {"value": inp2.wl.queries / (ms2 * 1e-3), "unit": UNIT,
+                                "ms_per_step": ms2,
+                                "note": "archive summaries precomputed" if arch else ""}
+                del inp2
+                torch.cuda.empty_cache()
+            line["other_workloads"] = extras
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,137 @@
+/*
+ * freesolo.h - C ABI of the FreeSolo sparse-attention forward pass for NVIDIA B200 (sm_100a).
+ *
+ * The method ("FreeSolo" technical summary, section "Methodology") gives every attention
+ * head two branches and adds them (§3.1, eq. (2)):
+ *
+ *     o_i = o_i^sr + alpha_h * o_i^lr
+ *
+ *   o_i^sr  (§3.2, eqs. (3)-(4)): softmax attention of the RoPE-rotated query over the keys
+ *           j in L_i = [max(0, i-w), i] (look-back radius w), logits q.k/sqrt(d).
+ *   o_i^lr  (§3.3, eqs. (5), (7)-(9)): the keys are cut into cells of s consecutive tokens;
+ *           each cell c has a mean key kbar_c and a max key norm a_c (eq. (5)).  The
+ *           candidates C_i are the cells lying wholly before the window, (c+1)s <= i-w.
+ *           FS-L pruning (eq. (8)) keeps A_i = the W most recent candidates plus the P
+ *           candidates of largest a_c.  Each cell of A_i is scored (eq. (7))
+ *               r_ic = q_i.kbar_c/sqrt(d) + lambda_h a_c erf((i - p_c)/(2 sigma_h)),
+ *           p_c = (c + 1/2)s, the K best form S_i, and o_i^lr = RMSNorm(u_i) where u_i is
+ *           softmax attention of the unrotated query over every token of S_i (eq. (9)).
+ *
+ * Readings where the summary is silent: RoPE pairs are interleaved (2m, 2m+1) with
+ * theta_m = base^(-2m/d); RMSNorm has no gain, u/sqrt(mean(u^2)+eps); ties in TopP and in
+ * the top-K go to the lower cell index; |A_i| < K selects all of A_i; an empty S_i gives
+ * o^lr = 0; W < 0 and P < 0 together mean no pruning (base FS, A_i = C_i).
+ *
+ * Layout: Q is [B, H, Nq, d]; K, V are [B, H, Nk, d]; O is [B, H, Nq, d]; all contiguous,
+ * row-major, of type `dtype`.  Query row r has position Nk - Nq + r among the keys, so
+ * Nq = Nk is a prefill and Nq < Nk appends Nq new tokens to an archive of Nk - Nq.
+ * Cell summaries: kbar [B, H, C, d] and amax [B, H, C], float32, C = floor(Nk / s).
+ * Selected cells: idx [B, H, Nq, K] int32, ascending, padded with -1.
+ *
+ * Ownership and errors: the caller owns every buffer; the library allocates nothing and
+ * enqueues its kernels on `stream` (a cudaStream_t; NULL is the legacy default stream).
+ * Pointers named d* / Q, K, V, O, kbar, amax, idx, ws are device pointers; the per-head
+ * arrays alpha / lambda / sigma are HOST pointers read during the call.  Argument errors
+ * are returned before anything is enqueued.  No exception crosses the ABI.
+ *
+ * Supported: d = 64, s = 32, w a multiple of s, 0 <= K <= 64, W + P <= 2048,
+ * 1 <= H <= 256; dtype bf16 or f32.  Anything else returns FS_ERR_UNSUPPORTED.
+ */
+#ifndef FREESOLO_H
+#define FREESOLO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FS_OK = 0,
+    FS_ERR_INVALID_ARG = 1,   /* NULL pointer, negative size, Nq > Nk, ... */
+    FS_ERR_UNSUPPORTED = 2,   /* a size or option outside the supported set above */
+    FS_ERR_WORKSPACE = 3,     /* workspace missing or smaller than fs_workspace_size() */
+    FS_ERR_CUDA = 4,          /* a CUDA call or kernel launch failed */
+    FS_ERR_TIMEOUT = 5        /* a kernel gave up a bounded wait (device error flag) */
+} fs_status;
+
+typedef enum { FS_BF16 = 0, FS_F32 = 1 } fs_dtype;
+
+#define FS_MAX_HEADS 256
+
+typedef struct {
+    int B, H, Nq, Nk, d;   /* batch, heads, query rows, key rows, head dim */
+    int w;                 /* look-back radius of the local branch (eq. (3)); L_i = [i-w, i] */
+    int s;                 /* cell size in tokens (eq. (5)) */
+    int K;                 /* cells kept per query (top-K of eq. (7)) */
+    int W, P;              /* FS-L recent and norm budgets (eq. (8)); W < 0 && P < 0: off */
+    float rope_base;       /* RoPE base, e.g. 10000 */
+    const float *alpha;    /* host [H]: per-head weight of the long-range branch (eq. (2)) */
+    const float *lambda;   /* host [H] or NULL (prior off): lambda_h >= 0 (eq. (7)) */
+    const float *sigma;    /* host [H] or NULL: sigma_h > 0 (eq. (7)) */
+    float rms_eps;         /* RMSNorm epsilon (eq. (9)), e.g. 1e-6 */
+    fs_dtype dtype;        /* type of Q, K, V and O; summaries are always float32 */
+} fs_params;
+
+/* Bytes of device workspace the calls below need for these parameters (> 0).
+ * The workspace's first bytes hold the device error flag read by fs_sync_status. */
+fs_status fs_workspace_size(const fs_params *p, size_t *bytes);
+
+/* Cell summaries, eq. (5): kbar [B,H,C,d] = mean key of each s-token cell, amax [B,H,C] =
+ * the largest key norm in the cell.  Only whole cells (C = floor(Nk/s)) are summarised.
+ * K is a device pointer of type p->dtype; kbar and amax are device float32 outputs. */
+fs_status fs_cell_summaries(const fs_params *p, const void *K, float *kbar, float *amax,
+                            void *stream);
+
+/* Long-range selection, eqs. (7)-(8): for every query row, the K best cells of A_i by
+ * r_ic, written to idx [B,H,Nq,K] (ascending, -1 padded).  kbar/amax are the summaries
+ * of fs_cell_summaries (or the caller's own, same layout).  ws/ws_bytes: workspace. */
+fs_status fs_select_topk(const fs_params *p, const void *Q, const float *kbar,
+                         const float *amax, int32_t *idx, void *ws, size_t ws_bytes,
+                         void *stream);
+
+/* The whole forward pass, eq. (2): O = o^sr + alpha_h o^lr.
+ * kbar/amax may be NULL (then computed here into the workspace) or caller-given summaries
+ * (e.g. an archive summarised once for decoding).  idx may be NULL (then selected here)
+ * or caller-given cells, which skips eqs. (7)-(8) and runs the readout on them. */
+fs_status fs_forward(const fs_params *p, const void *Q, const void *K, const void *V,
+                     const float *kbar, const float *amax, const int32_t *idx, void *O,
+                     void *ws, size_t ws_bytes, void *stream);
+
+/* Bytes of device scratch fs_forward_host needs: device copies of Q, K, V, O plus the
+ * workspace. */
+fs_status fs_host_scratch_size(const fs_params *p, size_t *bytes);
+
+/* fs_forward on HOST buffers hQ, hK, hV -> hO (pinned memory makes the copies async).
+ * Copies in, computes and copies out on `stream` using the caller's device scratch
+ * (fs_host_scratch_size bytes).  Returns after enqueueing; synchronize `stream` (or call
+ * fs_sync_status) before reading hO. */
+fs_status fs_forward_host(const fs_params *p, const void *hQ, const void *hK, const void *hV,
+                          void *hO, void *dscratch, size_t scratch_bytes, void *stream);
+
+/* Synchronizes `stream`, then reads and clears the device error flag in `ws`.
+ * Returns FS_ERR_TIMEOUT if a kernel gave up a bounded wait since the last check,
+ * FS_ERR_CUDA if the stream reports an error, else FS_OK. */
+fs_status fs_sync_status(void *ws, void *stream);
+
+/* Static description of a status code. */
+const char *fs_status_string(fs_status s);
+
+/* ---- diagnostics (no counterpart in the method: measurement support) ----
+ * fs_launch_count: kernels this library has launched since load (all calls, streams).
+ * fs_timing_enable(1): from now on every kernel launch is bracketed by two CUDA events
+ *   recorded on its own stream.  fs_kernel_times waits for the recorded events, writes per
+ *   kernel id (0 <= id < max_ids) the launches and summed device milliseconds since the
+ *   previous read, clears them, and returns the number of kernel ids.
+ * fs_kernel_name: the name of a kernel id, or NULL past the last one. */
+long long fs_launch_count(void);
+fs_status fs_timing_enable(int on);
+int fs_kernel_times(int max_ids, long long *launches, double *ms);
+const char *fs_kernel_name(int id);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FREESOLO_H */

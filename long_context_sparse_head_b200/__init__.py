@@ -1,0 +1,204 @@
+"""FreeSolo sparse-attention forward pass on NVIDIA B200 (sm_100a).
+
+Thin Python binding of the C-ABI library libfreesolo.so (include/freesolo.h): it only
+marshals arguments (tensor pointers, sizes, the current CUDA stream).  Every step of the
+computation runs in the library's CUDA kernels; there is no Python or CPU fallback, and
+loading fails loudly if the library has not been built (python -m
+long_context_sparse_head_b200.build).
+
+The entry points mirror the C names: `workspace_size`, `cell_summaries`, `select_topk`,
+`forward`, `host_scratch_size`, `forward_host`, `sync_status`, `status_string`.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfreesolo.so")
+
+FS_BF16, FS_F32 = 0, 1
+STATUS = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_UNSUPPORTED", 3: "FS_ERR_WORKSPACE",
+          4: "FS_ERR_CUDA", 5: "FS_ERR_TIMEOUT"}
+EXPORTS = ("fs_workspace_size", "fs_cell_summaries", "fs_select_topk", "fs_forward",
+           "fs_host_scratch_size", "fs_forward_host", "fs_sync_status", "fs_status_string",
+           "fs_launch_count", "fs_timing_enable", "fs_kernel_times", "fs_kernel_name")
+
+
+class FsError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__("%s: %s (%s)" % (where, STATUS.get(code, code), status_string(code)))
+
+
+class FsParams(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("Nq", ctypes.c_int), ("Nk", ctypes.c_int),
+        ("d", ctypes.c_int), ("w", ctypes.c_int), ("s", ctypes.c_int), ("K", ctypes.c_int),
+        ("W", ctypes.c_int), ("P", ctypes.c_int),
+        ("rope_base", ctypes.c_float),
+        ("alpha", ctypes.POINTER(ctypes.c_float)),
+        ("lambda_", ctypes.POINTER(ctypes.c_float)),
+        ("sigma", ctypes.POINTER(ctypes.c_float)),
+        ("rms_eps", ctypes.c_float),
+        ("dtype", ctypes.c_int),
+    ]
+
+
+_lib = None
+
+
+def load():
+    """Load libfreesolo.so (raises if it is missing: there is no fallback path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libfreesolo.so is not built; run "
+                               "`python -m long_context_sparse_head_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(FsParams)
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        L.fs_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
+        L.fs_cell_summaries.argtypes = [P, vp, vp, vp, vp]
+        L.fs_select_topk.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
+        L.fs_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.fs_host_scratch_size.argtypes = [P, ctypes.POINTER(sz)]
+        L.fs_forward_host.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
+        L.fs_sync_status.argtypes = [vp, vp]
+        L.fs_status_string.argtypes = [ctypes.c_int]
+        L.fs_status_string.restype = ctypes.c_char_p
+        L.fs_launch_count.argtypes = []
+        L.fs_launch_count.restype = ctypes.c_longlong
+        L.fs_timing_enable.argtypes = [ctypes.c_int]
+        L.fs_kernel_times.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_longlong),
+                                      ctypes.POINTER(ctypes.c_double)]
+        L.fs_kernel_name.argtypes = [ctypes.c_int]
+        L.fs_kernel_name.restype = ctypes.c_char_p
+        for name in EXPORTS:
+            if name not in ("fs_status_string", "fs_launch_count", "fs_kernel_name"):
+                getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(code):
+    return load().fs_status_string(int(code)).decode()
+
+
+class Params:
+    """fs_params plus the host arrays it points to (kept alive with it).
+
+    Q [B,H,Nq,d], K/V [B,H,Nk,d]; W = P = -1 turns pruning off; lam/sigma None turns the
+    erf prior off.  dtype: "bf16" or "f32".
+    """
+
+    def __init__(self, *, B, H, Nq, Nk, d=64, w=512, s=32, K=16, W=16, P=48, alpha,
+                 lam=None, sigma=None, rope_base=10000.0, rms_eps=1e-6, dtype="bf16"):
+        self.alpha = np.ascontiguousarray(alpha, np.float32)
+        self.lam = None if lam is None else np.ascontiguousarray(lam, np.float32)
+        self.sigma = None if sigma is None else np.ascontiguousarray(sigma, np.float32)
+        fp = ctypes.POINTER(ctypes.c_float)
+        c = FsParams()
+        c.B, c.H, c.Nq, c.Nk, c.d, c.w, c.s, c.K, c.W, c.P = B, H, Nq, Nk, d, w, s, K, W, P
+        c.rope_base, c.rms_eps = rope_base, rms_eps
+        c.alpha = self.alpha.ctypes.data_as(fp)
+        c.lambda_ = self.lam.ctypes.data_as(fp) if self.lam is not None else fp()
+        c.sigma = self.sigma.ctypes.data_as(fp) if self.sigma is not None else fp()
+        c.dtype = FS_BF16 if dtype == "bf16" else FS_F32
+        self.c = c
+        self.B, self.H, self.Nq, self.Nk, self.d, self.s, self.K = B, H, Nq, Nk, d, s, K
+        self.dtype = dtype
+
+    @property
+    def C(self):
+        return self.Nk // self.s
+
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(getattr(stream, "cuda_stream", stream))
+
+
+def _check(code, where):
+    if code != 0:
+        raise FsError(code, where)
+
+
+def workspace_size(params):
+    n = ctypes.c_size_t()
+    _check(load().fs_workspace_size(params.ref(), ctypes.byref(n)), "fs_workspace_size")
+    return n.value
+
+
+def host_scratch_size(params):
+    n = ctypes.c_size_t()
+    _check(load().fs_host_scratch_size(params.ref(), ctypes.byref(n)), "fs_host_scratch_size")
+    return n.value
+
+
+def alloc_workspace(params, device="cuda"):
+    """A zero-filled workspace (the device error flag must start at zero)."""
+    import torch
+    return torch.zeros(workspace_size(params), dtype=torch.uint8, device=device)
+
+
+def cell_summaries(params, K, kbar, amax, stream=None):
+    _check(load().fs_cell_summaries(params.ref(), _ptr(K), _ptr(kbar), _ptr(amax),
+                                    _stream(stream)), "fs_cell_summaries")
+
+
+def select_topk(params, Q, kbar, amax, idx, ws, stream=None):
+    _check(load().fs_select_topk(params.ref(), _ptr(Q), _ptr(kbar), _ptr(amax), _ptr(idx),
+                                 _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "fs_select_topk")
+
+
+def forward(params, Q, K, V, O, ws, kbar=None, amax=None, idx=None, stream=None):
+    _check(load().fs_forward(params.ref(), _ptr(Q), _ptr(K), _ptr(V), _ptr(kbar), _ptr(amax),
+                             _ptr(idx), _ptr(O), _ptr(ws), ws.numel() * ws.element_size(),
+                             _stream(stream)), "fs_forward")
+
+
+def forward_host(params, hQ, hK, hV, hO, dscratch, stream=None):
+    _check(load().fs_forward_host(params.ref(), _ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hO),
+                                  _ptr(dscratch), dscratch.numel() * dscratch.element_size(),
+                                  _stream(stream)), "fs_forward_host")
+
+
+def sync_status(ws, stream=None):
+    code = load().fs_sync_status(_ptr(ws), _stream(stream))
+    _check(code, "fs_sync_status")
+
+
+# ---- diagnostics -------------------------------------------------------------------
+def launch_count():
+    """Kernels the library has launched since it was loaded."""
+    return load().fs_launch_count()
+
+
+def timing_enable(on=True):
+    load().fs_timing_enable(1 if on else 0)
+
+
+def kernel_times():
+    """{kernel name: (launches, summed device ms)} since the previous read (then cleared)."""
+    n = 32
+    cnt = (ctypes.c_longlong * n)()
+    ms = (ctypes.c_double * n)()
+    k = load().fs_kernel_times(n, cnt, ms)
+    out = {}
+    for i in range(min(k, n)):
+        name = load().fs_kernel_name(i).decode()
+        out[name] = (cnt[i], ms[i])
+    return out

@@ -1,0 +1,239 @@
+// C ABI of the FreeSolo forward pass (declared in include/freesolo.h): argument checks,
+// workspace layout and the launch sequence
+//   summaries (eq. (5)) -> TopP exit table (eq. (8)) -> selection (eq. (7))
+//   -> readout (eq. (9)) -> window + combine (eqs. (2)-(4)).
+#include <cmath>
+#include <cstring>
+
+#include "fs_common.cuh"
+
+namespace fs {
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t esize(fs_dtype t) { return t == FS_BF16 ? 2 : 4; }
+
+fs_status validate(const fs_params *p) {
+    if (!p) return FS_ERR_INVALID_ARG;
+    if (p->B < 1 || p->H < 1 || p->Nq < 0 || p->Nk < 0 || p->Nq > p->Nk) return FS_ERR_INVALID_ARG;
+    if (p->d <= 0 || p->s <= 0 || p->w < 0 || p->K < 0) return FS_ERR_INVALID_ARG;
+    if ((p->W < 0) != (p->P < 0)) return FS_ERR_INVALID_ARG;     // both off or both on
+    if (p->dtype != FS_BF16 && p->dtype != FS_F32) return FS_ERR_INVALID_ARG;
+    if (!p->alpha) return FS_ERR_INVALID_ARG;
+    if (!(p->rope_base > 0.f) || !(p->rms_eps >= 0.f)) return FS_ERR_INVALID_ARG;
+    if (p->lambda) {
+        if (!p->sigma) return FS_ERR_INVALID_ARG;
+        for (int h = 0; h < p->H && h < FS_MAX_HEADS; h++)
+            if (!(p->lambda[h] >= 0.f) || !(p->sigma[h] > 0.f)) return FS_ERR_INVALID_ARG;
+    }
+    if (p->d != kD || p->s != kS || p->w % kS != 0) return FS_ERR_UNSUPPORTED;
+    if (p->K > kMaxK || p->H > FS_MAX_HEADS) return FS_ERR_UNSUPPORTED;
+    if (p->W >= 0 && (long long)p->W + p->P > kMaxAdmit) return FS_ERR_UNSUPPORTED;
+    if ((long long)p->B * p->H > 65535 || p->Nk > (1 << 30)) return FS_ERR_UNSUPPORTED;
+    return FS_OK;
+}
+
+Dev make_dev(const fs_params *p) {
+    Dev D;
+    std::memset(&D, 0, sizeof(D));
+    D.B = p->B; D.H = p->H; D.Nq = p->Nq; D.Nk = p->Nk; D.C = p->Nk / p->s;
+    D.w = p->w; D.K = p->K; D.W = p->W; D.P = p->P;
+    D.prune = (p->W >= 0);
+    D.q0 = p->Nk - p->Nq;
+    D.scale = (float)(1.0 / std::sqrt((double)p->d));
+    D.rms_eps = p->rms_eps;
+    for (int m = 0; m < kD / 2; m++)
+        D.theta[m] = (float)std::pow((double)p->rope_base, -2.0 * m / (double)p->d);
+    D.has_prior = 0;
+    for (int h = 0; h < p->H; h++) {
+        D.alpha[h] = p->alpha[h];
+        D.lambda[h] = p->lambda ? p->lambda[h] : 0.f;
+        D.inv2sigma[h] = p->lambda ? (float)(1.0 / (2.0 * (double)p->sigma[h])) : 0.f;
+        if (D.lambda[h] != 0.f) D.has_prior = 1;
+    }
+    return D;
+}
+
+WsLayout layout(const fs_params *p) {
+    const size_t BH = (size_t)p->B * p->H, C = (size_t)(p->Nk / p->s);
+    WsLayout L;
+    size_t off = 0;
+    L.flag = off;  off += 256;
+    L.exitn = off; off += align256(BH * C * 4);
+    L.kbar = off;  off += align256(BH * C * kD * 4);
+    L.amax = off;  off += align256(BH * C * 4);
+    L.idx = off;   off += align256(BH * (size_t)p->Nq * p->K * 4);
+    L.olr = off;   off += align256(BH * (size_t)p->Nq * kD * 4);
+    L.total = off;
+    return L;
+}
+
+template <typename X> X *at(void *ws, size_t off) {
+    return reinterpret_cast<X *>(static_cast<uint8_t *>(ws) + off);
+}
+
+fs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FS_OK : FS_ERR_CUDA; }
+
+// Does any query row have a long-range candidate?
+bool has_long_range(const fs_params *p) {
+    if (p->K == 0 || p->Nq == 0) return false;
+    return cand_count(p->Nk - 1, p->w, p->Nk / p->s) > 0;
+}
+
+fs_status run_forward(const fs_params *p, const void *Q, const void *K, const void *V,
+                      const float *kbar, const float *amax, const int32_t *idx, void *O,
+                      void *ws, cudaStream_t st) {
+    const Dev D = make_dev(p);
+    const WsLayout L = layout(p);
+    const float *olr = nullptr;
+    if (has_long_range(p)) {
+        const int32_t *sel = idx;
+        if (!sel) {
+            if (!kbar) {
+                float *kb = at<float>(ws, L.kbar), *am = at<float>(ws, L.amax);
+                if (launch_summaries(D, p->dtype, K, kb, am, st) != cudaSuccess) return FS_ERR_CUDA;
+                kbar = kb;
+                amax = am;
+            }
+            int *exitn = at<int>(ws, L.exitn);
+            if (D.prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
+            int32_t *wsidx = at<int32_t>(ws, L.idx);
+            if (launch_select(D, p->dtype, Q, kbar, amax, exitn, wsidx, st) != cudaSuccess)
+                return FS_ERR_CUDA;
+            sel = wsidx;
+        }
+        float *o = at<float>(ws, L.olr);
+        if (launch_readout(D, p->dtype, Q, K, V, sel, o, st) != cudaSuccess) return FS_ERR_CUDA;
+        olr = o;
+    }
+    return cuda_status(launch_window(D, p->dtype, Q, K, V, olr, O, st));
+}
+
+}  // namespace
+}  // namespace fs
+
+using namespace fs;
+
+extern "C" fs_status fs_workspace_size(const fs_params *p, size_t *bytes) {
+    fs_status s = validate(p);
+    if (s != FS_OK) return s;
+    if (!bytes) return FS_ERR_INVALID_ARG;
+    *bytes = layout(p).total;
+    return FS_OK;
+}
+
+extern "C" fs_status fs_cell_summaries(const fs_params *p, const void *K, float *kbar,
+                                       float *amax, void *stream) {
+    fs_status s = validate(p);
+    if (s != FS_OK) return s;
+    if (p->Nk / p->s == 0) return FS_OK;
+    if (!K || !kbar || !amax) return FS_ERR_INVALID_ARG;
+    return cuda_status(launch_summaries(make_dev(p), p->dtype, K, kbar, amax, (cudaStream_t)stream));
+}
+
+extern "C" fs_status fs_select_topk(const fs_params *p, const void *Q, const float *kbar,
+                                    const float *amax, int32_t *idx, void *ws, size_t ws_bytes,
+                                    void *stream) {
+    fs_status s = validate(p);
+    if (s != FS_OK) return s;
+    if (p->Nq == 0 || p->K == 0) return FS_OK;
+    if (!Q || !idx) return FS_ERR_INVALID_ARG;
+    const WsLayout L = layout(p);
+    if (!ws || ws_bytes < L.total) return FS_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    const Dev D = make_dev(p);
+    if (D.C == 0 || !has_long_range(p)) {
+        return cuda_status(cudaMemsetAsync(idx, 0xff, (size_t)p->B * p->H * p->Nq * p->K * 4, st));
+    }
+    if (!kbar || !amax) return FS_ERR_INVALID_ARG;
+    int *exitn = at<int>(ws, L.exitn);
+    if (D.prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
+    return cuda_status(launch_select(D, p->dtype, Q, kbar, amax, exitn, idx, st));
+}
+
+extern "C" fs_status fs_forward(const fs_params *p, const void *Q, const void *K, const void *V,
+                                const float *kbar, const float *amax, const int32_t *idx, void *O,
+                                void *ws, size_t ws_bytes, void *stream) {
+    fs_status s = validate(p);
+    if (s != FS_OK) return s;
+    if (p->Nq == 0) return FS_OK;
+    if (!Q || !K || !V || !O) return FS_ERR_INVALID_ARG;
+    if ((kbar == nullptr) != (amax == nullptr)) return FS_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < layout(p).total) return FS_ERR_WORKSPACE;
+    return run_forward(p, Q, K, V, kbar, amax, idx, O, ws, (cudaStream_t)stream);
+}
+
+namespace {
+struct HostScratch { size_t q, k, v, o, ws, total; };
+HostScratch host_scratch(const fs_params *p) {
+    const size_t e = esize(p->dtype), BH = (size_t)p->B * p->H;
+    HostScratch h;
+    size_t off = 0;
+    h.q = off;  off += align256(BH * p->Nq * kD * e);
+    h.k = off;  off += align256(BH * p->Nk * kD * e);
+    h.v = off;  off += align256(BH * p->Nk * kD * e);
+    h.o = off;  off += align256(BH * p->Nq * kD * e);
+    h.ws = off; off += layout(p).total;
+    h.total = off;
+    return h;
+}
+}  // namespace
+
+extern "C" fs_status fs_host_scratch_size(const fs_params *p, size_t *bytes) {
+    fs_status s = validate(p);
+    if (s != FS_OK) return s;
+    if (!bytes) return FS_ERR_INVALID_ARG;
+    *bytes = host_scratch(p).total;
+    return FS_OK;
+}
+
+extern "C" fs_status fs_forward_host(const fs_params *p, const void *hQ, const void *hK,
+                                     const void *hV, void *hO, void *dscratch,
+                                     size_t scratch_bytes, void *stream) {
+    fs_status s = validate(p);
+    if (s != FS_OK) return s;
+    if (p->Nq == 0) return FS_OK;
+    if (!hQ || !hK || !hV || !hO) return FS_ERR_INVALID_ARG;
+    const HostScratch h = host_scratch(p);
+    if (!dscratch || scratch_bytes < h.total) return FS_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t e = esize(p->dtype), BH = (size_t)p->B * p->H;
+    void *dQ = at<void>(dscratch, h.q), *dK = at<void>(dscratch, h.k);
+    void *dV = at<void>(dscratch, h.v), *dO = at<void>(dscratch, h.o);
+    void *ws = at<void>(dscratch, h.ws);
+    // one plain async copy per buffer
+    if (cudaMemcpyAsync(dQ, hQ, BH * p->Nq * kD * e, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dK, hK, BH * p->Nk * kD * e, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dV, hV, BH * p->Nk * kD * e, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return FS_ERR_CUDA;
+    s = run_forward(p, dQ, dK, dV, nullptr, nullptr, nullptr, dO, ws, st);
+    if (s != FS_OK) return s;
+    return cuda_status(cudaMemcpyAsync(hO, dO, BH * p->Nq * kD * e, cudaMemcpyDeviceToHost, st));
+}
+
+extern "C" fs_status fs_sync_status(void *ws, void *stream) {
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return FS_ERR_CUDA;
+    if (!ws) return FS_OK;
+    int flag = 0;
+    if (cudaMemcpy(&flag, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FS_ERR_CUDA;
+    if (flag != kFlagOk) {
+        const int zero = 0;
+        if (cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return FS_ERR_CUDA;
+        return FS_ERR_TIMEOUT;
+    }
+    return FS_OK;
+}
+
+extern "C" const char *fs_status_string(fs_status s) {
+    switch (s) {
+    case FS_OK: return "ok";
+    case FS_ERR_INVALID_ARG: return "invalid argument";
+    case FS_ERR_UNSUPPORTED: return "unsupported size or option";
+    case FS_ERR_WORKSPACE: return "workspace missing or too small";
+    case FS_ERR_CUDA: return "CUDA error";
+    case FS_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    }
+    return "unknown status";
+}

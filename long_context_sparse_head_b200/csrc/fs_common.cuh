@@ -1,0 +1,119 @@
+// Shared definitions of the FreeSolo CUDA library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/freesolo.h"
+
+namespace fs {
+
+constexpr int kD = 64;          // head dim supported by the kernels
+constexpr int kS = 32;          // cell size supported by the kernels
+constexpr int kMaxK = 64;       // largest top-K
+constexpr int kMaxAdmit = 2048; // largest W + P
+constexpr unsigned kFull = 0xffffffffu;
+
+// Never-leaves sentinel of the TopP exit table.
+constexpr int kNever = 0x7fffffff;
+
+// Kernel-side copy of the parameters (passed by value).
+struct Dev {
+    int B, H, Nq, Nk, C;       // C = floor(Nk / s)
+    int w, K, W, P;
+    int prune;                 // 0: base FS (A_i = C_i)
+    int has_prior;             // lambda given and not all zero
+    int q0;                    // position of query row 0 = Nk - Nq
+    float scale;               // 1 / sqrt(d)
+    float rms_eps;
+    float theta[kD / 2];       // RoPE frequencies base^(-2m/d)
+    float alpha[FS_MAX_HEADS];
+    float lambda[FS_MAX_HEADS];
+    float inv2sigma[FS_MAX_HEADS];  // 1 / (2 sigma_h)
+};
+
+// Workspace layout (byte offsets from ws; each segment 256-byte aligned).
+struct WsLayout {
+    size_t flag, exitn, kbar, amax, idx, olr, total;
+};
+
+// Device error flag codes (first int of the workspace).
+enum : int { kFlagOk = 0, kFlagTimeout = 1 };
+
+// Candidate count |C_i| for key-index position i: cells with (c+1)s <= i - w.
+__host__ __device__ inline int cand_count(int i, int w, int C) {
+    int lim = i - w;
+    if (lim < kS) return 0;
+    int n = lim / kS;
+    return n < C ? n : C;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+    return v;
+}
+
+// Load VEC consecutive elements (16 bytes) and widen to float.
+template <typename T> struct Vec;
+template <> struct Vec<float> {
+    static constexpr int N = 4;
+    __device__ __forceinline__ static void load(const float *p, float *o) {
+        float4 v = __ldg(reinterpret_cast<const float4 *>(p));
+        o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+    }
+};
+template <> struct Vec<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float *o) {
+        uint4 v = __ldg(reinterpret_cast<const uint4 *>(p));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            o[2 * e] = __uint_as_float(w[e] << 16);
+            o[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+        }
+    }
+};
+
+template <typename T> __device__ __forceinline__ float to_f(T x);
+template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// ---- kernel ids for the diagnostics (fs_kernel_times) ----
+enum KernelId : int { kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kNumKernels };
+
+// Brackets one kernel launch: counts it and, when timing is on, records events around it.
+struct LaunchScope {
+    LaunchScope(int id, cudaStream_t st);
+    ~LaunchScope();
+    int id;
+    cudaStream_t st;
+    int slot;
+};
+
+// ---- launchers (one per kernel file) ----
+cudaError_t launch_summaries(const Dev &P, fs_dtype dt, const void *K, float *kbar,
+                             float *amax, cudaStream_t st);
+cudaError_t launch_exit_times(const Dev &P, const float *amax, int *exitn, cudaStream_t st);
+cudaError_t launch_select(const Dev &P, fs_dtype dt, const void *Q, const float *kbar,
+                          const float *amax, const int *exitn, int32_t *idx, cudaStream_t st);
+cudaError_t launch_readout(const Dev &P, fs_dtype dt, const void *Q, const void *K,
+                           const void *V, const int32_t *idx, float *olr, cudaStream_t st);
+cudaError_t launch_window(const Dev &P, fs_dtype dt, const void *Q, const void *K,
+                          const void *V, const float *olr, void *O, cudaStream_t st);
+
+}  // namespace fs

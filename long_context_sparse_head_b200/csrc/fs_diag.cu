@@ -1,0 +1,87 @@
+// Launch counting and optional per-kernel device timing (measurement support only).
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "fs_common.cuh"
+
+namespace fs {
+namespace {
+
+std::atomic<long long> g_launches{0};
+std::atomic<int> g_timing{0};
+std::mutex g_mu;
+
+struct Pending { int id; cudaEvent_t a, b; };
+std::vector<Pending> g_pending;      // recorded, not yet read
+std::vector<cudaEvent_t> g_free;     // reusable events
+long long g_count[kNumKernels];
+double g_ms[kNumKernels];
+
+cudaEvent_t take_event() {
+    if (!g_free.empty()) {
+        cudaEvent_t e = g_free.back();
+        g_free.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+const char *const kNames[kNumKernels] = {"cell_summaries", "exit_times", "select_topk",
+                                         "readout", "window_combine"};
+}  // namespace
+
+LaunchScope::LaunchScope(int id_, cudaStream_t st_) : id(id_), st(st_), slot(-1) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (!g_timing.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lk(g_mu);
+    Pending p{id, take_event(), take_event()};
+    if (!p.a || !p.b) return;
+    cudaEventRecord(p.a, st);
+    slot = (int)g_pending.size();
+    g_pending.push_back(p);
+}
+
+LaunchScope::~LaunchScope() {
+    if (slot < 0) return;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (slot < (int)g_pending.size()) cudaEventRecord(g_pending[slot].b, st);
+}
+
+}  // namespace fs
+
+using namespace fs;
+
+extern "C" long long fs_launch_count(void) { return g_launches.load(); }
+
+extern "C" fs_status fs_timing_enable(int on) {
+    g_timing.store(on ? 1 : 0);
+    return FS_OK;
+}
+
+extern "C" int fs_kernel_times(int max_ids, long long *launches, double *ms) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (const Pending &p : g_pending) {
+        float t = 0.f;
+        if (cudaEventSynchronize(p.b) == cudaSuccess && cudaEventElapsedTime(&t, p.a, p.b) == cudaSuccess) {
+            g_count[p.id] += 1;
+            g_ms[p.id] += t;
+        }
+        g_free.push_back(p.a);
+        g_free.push_back(p.b);
+    }
+    g_pending.clear();
+    for (int i = 0; i < kNumKernels && i < max_ids; i++) {
+        if (launches) launches[i] = g_count[i];
+        if (ms) ms[i] = g_ms[i];
+        g_count[i] = 0;
+        g_ms[i] = 0.0;
+    }
+    return kNumKernels;
+}
+
+extern "C" const char *fs_kernel_name(int id) {
+    return (id >= 0 && id < kNumKernels) ? kNames[id] : nullptr;
+}

@@ -1,0 +1,146 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Small cases are compared on every row; the full-size workloads run exactly as the
+benchmark launches them and are compared on sampled rows (plus every needle row).
+"""
+import numpy as np
+import pytest
+import torch
+
+from workloads import CONFIGS, generate, small
+from tests._parity import (TOL, GpuRun, check_selection, expected_output, oracle_for,
+                           sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def all_rows(wl):
+    return [(b, h, r) for b in range(wl.B) for h in range(wl.H) for r in range(wl.Nq)]
+
+
+def run_case(inp, rows=None, check_needles=True, **over):
+    """Summaries, selection and output parity for one problem."""
+    wl = inp.wl
+    g = GpuRun(inp, **over)
+    prob = oracle_for(inp, **over)
+    kbar_o, amax_o = prob.summaries()
+    kbar_g, amax_g = (g.numpy(t) for t in g.summaries())
+    np.testing.assert_allclose(kbar_g, kbar_o, rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(amax_g, amax_o, rtol=1e-5, atol=1e-6)
+    idx = g.numpy(g.select())
+    rows = all_rows(wl) if rows is None else rows
+    exact, tie = check_selection(inp, (kbar_o, amax_o), idx, rows, **over)
+    assert tie <= max(2, len(rows) // 100), (exact, tie)
+    O = g.numpy(g.forward()).reshape(wl.B, wl.H, wl.Nq, wl.d)
+    assert np.isfinite(O).all()
+    got = np.stack([O[b, h, r] for b, h, r in rows])
+    want = expected_output(inp, prob, rows, idx)
+    err = np.abs(got - want).max()
+    assert err <= TOL[wl.dtype], err
+    if check_needles and over.get("K", wl.K) > 0:
+        rowset = set(rows)
+        for b, h, c, nrows in inp.needle_cells:
+            for r in nrows:
+                if (b, h, r) in rowset:
+                    assert c in idx[b, h, r], ("needle missed", b, h, c, r)
+    return g, idx, O, err
+
+
+# ---------------------------------------------------------------- small, every row
+def test_tiny2k_fp32():
+    inp = generate(CONFIGS["tiny2k"])
+    run_case(inp)
+
+
+def test_tiny2k_all_cells_no_pruning_fp32():
+    """K covers every prefix cell and pruning is off: the long-range branch is dense
+    causal NoPE attention over the prefix."""
+    inp = generate(CONFIGS["tiny2k"])
+    run_case(inp, K=64, W=-1, P=-1)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", [
+    dict(),                                           # pruning active (W+P < |C_i|)
+    dict(W=-1, P=-1),                                 # base FS
+    dict(W=0, P=5), dict(W=6, P=0),                   # one-sided budgets
+    dict(lam=0.6, sigma=300.0),                       # erf prior on
+    dict(Nq=200, Nk=1960),                            # appended queries, ragged tiles
+    dict(Nq=1000, Nk=1000),                           # Nk not a multiple of s
+    dict(w=0), dict(w=64, K=1),                       # degenerate windows / K
+    dict(K=0),                                        # no long-range branch
+    dict(Nq=300, Nk=300, w=512),                      # shorter than the window: no cells
+    dict(B=2, H=3, needles=2, needle_queries=4),      # batch, heads, needles
+])
+def test_small_cases(dtype, case):
+    kw = dict(B=1, H=2, Nq=1536, Nk=1536, K=6, W=4, P=9, dtype=dtype, seed=101)
+    kw.update(case)
+    lam = kw.pop("lam", None)
+    sigma = kw.pop("sigma", 1024.0)
+    wl = small("case", lam=lam, sigma=sigma, **kw)
+    run_case(generate(wl))
+
+
+def test_caller_idx_runs_readout_on_given_cells():
+    """fs_forward with caller cells skips selection: compare with the oracle readout on
+    those cells, and with the internally selected path when given the GPU's own cells."""
+    inp = generate(small("given", Nq=1024, Nk=1024, K=5, W=3, P=6, dtype="bf16", seed=7))
+    wl = inp.wl
+    g = GpuRun(inp)
+    idx_sel = g.select().clone()
+    O_sel = g.forward().clone()
+    O_given = g.forward(idx=idx_sel)
+    assert torch.equal(O_sel, O_given)
+    # random ascending cell lists inside each row's candidate prefix
+    rng = np.random.default_rng(3)
+    idx = -np.ones((wl.B, wl.H, wl.Nq, wl.K), np.int32)
+    prob = oracle_for(inp)
+    for b in range(wl.B):
+        for h in range(wl.H):
+            for r in range(wl.Nq):
+                n = prob.candidate_count(wl.Nk - wl.Nq + r)
+                k = min(n, int(rng.integers(0, wl.K + 1)))
+                if k:
+                    idx[b, h, r, :k] = np.sort(rng.choice(n, size=k, replace=False))
+    O = g.numpy(g.forward(idx=torch.from_numpy(idx).cuda()))
+    rows = all_rows(wl)
+    want = expected_output(inp, prob, rows, idx)
+    err = np.abs(O.reshape(-1, wl.d) - want).max()
+    assert err <= 2e-2, err
+
+
+def test_caller_summaries_match_internal():
+    inp = generate(small("sums", Nq=512, Nk=2048, K=4, W=3, P=5, dtype="bf16", seed=8))
+    g = GpuRun(inp)
+    kbar, amax = g.summaries()
+    O1 = g.forward().clone()
+    O2 = g.forward(kbar=kbar, amax=amax)
+    assert torch.equal(O1, O2)
+
+
+def test_repeated_calls_are_deterministic():
+    inp = generate(small("det", Nq=2048, Nk=2048, K=8, dtype="bf16", seed=9))
+    g = GpuRun(inp)
+    a = g.forward().clone()
+    b = g.forward().clone()
+    assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------- full-size workloads
+@pytest.mark.parametrize("name", ["prefill4k", "prefill16k", "prefill64k", "decode256k"])
+def test_full_size_sampled(name):
+    wl = CONFIGS[name]
+    inp = generate(wl)
+    needle_rows = [(b, h, r) for b, h, c, rs in inp.needle_cells for r in rs[:4]]
+    rows = sample_rows(wl, 400, seed=1, extra=needle_rows)
+    g, idx, O, err = run_case(inp, rows=rows, check_needles=False)
+    for b, h, c, rs in inp.needle_cells:           # every needle row, cheap to check
+        for r in rs:
+            assert c in idx[b, h, r], ("needle missed", b, h, c, r)
+    # properties at every row: finite, ascending selections inside the candidate prefix
+    assert np.isfinite(O).all()
+    sel = idx.reshape(-1, wl.K).astype(np.int64)
+    valid = sel >= 0
+    both = valid[:, 1:] & valid[:, :-1]
+    assert (np.diff(sel, axis=1)[both] > 0).all()
+    assert not (valid[:, 1:] & ~valid[:, :-1]).any()        # -1 only as trailing padding

@@ -8,13 +8,16 @@ The workloads stand in for the long-context retrieval evaluations the FreeSolo
 summary reports (RULER / single-needle retrieval at 4k-256k, "Empirical Validation"),
 which are not available here.  Each recipe is stated in `CONFIGS` and `generate`.
 """
+import concurrent.futures as cf
+import os
 from dataclasses import dataclass, field, replace
 from typing import Optional
 
 import numpy as np
 
 RECIPE_NOTE = (
-    "Q,K,V ~ N(0,1)/sqrt(d) (PCG64, seed per workload); bf16 workloads round to bf16 "
+    "Q,K,V ~ N(0,1)/sqrt(d) (PCG64 streams spawned from the workload seed, one per "
+    "(array, b, h)); bf16 workloads round to bf16 "
     "(nearest-even). Planted needles: a cell's keys become 3*|k_j|*u for a random unit u, "
     "and query rows placed after that cell's window edge become |q|*u. The 64k workload "
     "scales each cell's keys by LogNormal(0, 0.5)."
@@ -74,9 +77,25 @@ CONFIGS = {
 
 def round_bf16(x: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bf16 value (ties to even), kept as float32."""
-    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
-    r = (b + np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
-    return r.view(np.float32)
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.bfloat16).to(torch.float32).numpy()
+
+
+def _normal_fill(ss_children, shape, scale):
+    """N(0,1)*scale float32 array; one independent stream per leading (b, h) slice,
+    filled by a thread pool (deterministic whatever the scheduling)."""
+    out = np.empty(shape, np.float32)
+    flat = out.reshape(-1, *shape[2:])
+
+    def fill(t):
+        g = np.random.Generator(np.random.PCG64(ss_children[t]))
+        g.standard_normal(out=flat[t], dtype=np.float32)
+        flat[t] *= scale
+
+    with cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        list(ex.map(fill, range(flat.shape[0])))
+    return out
 
 
 @dataclass
@@ -98,12 +117,13 @@ def _unit(rng, d):
 
 def generate(wl: Workload) -> Inputs:
     """Draw the inputs of a workload.  Deterministic in (wl, wl.seed)."""
-    rng = np.random.Generator(np.random.PCG64(wl.seed))
     B, H, Nq, Nk, d, s, w = wl.B, wl.H, wl.Nq, wl.Nk, wl.d, wl.s, wl.w
+    kids = np.random.SeedSequence(wl.seed).spawn(3 * B * H + 1)
+    rng = np.random.Generator(np.random.PCG64(kids[-1]))
     scale = np.float32(1.0 / np.sqrt(d))
-    Q = rng.standard_normal((B, H, Nq, d), dtype=np.float32) * scale
-    K = rng.standard_normal((B, H, Nk, d), dtype=np.float32) * scale
-    V = rng.standard_normal((B, H, Nk, d), dtype=np.float32) * scale
+    Q = _normal_fill(kids[0:B * H], (B, H, Nq, d), scale)
+    K = _normal_fill(kids[B * H:2 * B * H], (B, H, Nk, d), scale)
+    V = _normal_fill(kids[2 * B * H:3 * B * H], (B, H, Nk, d), scale)
     if wl.alpha is not None:
         alpha = np.asarray(wl.alpha, np.float64)
     else:
