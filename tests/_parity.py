@@ -57,7 +57,7 @@ class GpuRun:
         p = self.p
         self.kbar = torch.empty((p.B, p.H, p.C, p.d), dtype=torch.float32, device=dev)
         self.amax = torch.empty((p.B, p.H, p.C), dtype=torch.float32, device=dev)
-        self.idx = torch.empty((p.B, p.H, p.Nq, max(p.K, 1)), dtype=torch.int32, device=dev)
+        self.idx = torch.empty((p.B, p.H, p.Nq, p.K), dtype=torch.int32, device=dev)
         self.O = torch.empty_like(self.Q)
 
     def summaries(self):

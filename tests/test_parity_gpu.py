@@ -134,9 +134,19 @@ def test_full_size_sampled(name):
     needle_rows = [(b, h, r) for b, h, c, rs in inp.needle_cells for r in rs[:4]]
     rows = sample_rows(wl, 400, seed=1, extra=needle_rows)
     g, idx, O, err = run_case(inp, rows=rows, check_needles=False)
-    for b, h, c, rs in inp.needle_cells:           # every needle row, cheap to check
+    # every needle row whose needle cell survives FS-L pruning selects it (eq. (8) can
+    # drop a low-norm needle before the query arrives; the oracle agrees on sampled rows)
+    prob = oracle_for(inp)
+    _, amax = prob.summaries()
+    kept = seen = 0
+    for b, h, c, rs in inp.needle_cells:
         for r in rs:
-            assert c in idx[b, h, r], ("needle missed", b, h, c, r)
+            n = prob.candidate_count(wl.Nk - wl.Nq + r)
+            seen += 1
+            if c in prob.admitted(amax[b, h], n):
+                kept += 1
+                assert c in idx[b, h, r], ("needle missed", b, h, c, r)
+    assert kept >= seen // 2, (kept, seen)
     # properties at every row: finite, ascending selections inside the candidate prefix
     assert np.isfinite(O).all()
     sel = idx.reshape(-1, wl.K).astype(np.int64)

@@ -146,6 +146,7 @@ def generate(wl: Workload) -> Inputs:
                 if c_hi <= 0:
                     continue
                 cells = rng.choice(c_hi, size=min(wl.needles, c_hi), replace=False)
+                used = set()                      # a query row serves one needle only
                 for c in cells:
                     c = int(c)
                     u = _unit(rng, d)
@@ -156,9 +157,14 @@ def generate(wl: Workload) -> Inputs:
                     if wl.needle_queries < 0:
                         rows = np.arange(first, Nq)
                     else:
-                        avail = Nq - first
-                        rows = np.sort(rng.choice(avail, size=min(wl.needle_queries, avail),
-                                                  replace=False)) + first
+                        want = min(wl.needle_queries, Nq - first - len(used))
+                        picked = []
+                        while len(picked) < want:
+                            r = int(rng.integers(first, Nq))
+                            if r not in used:
+                                used.add(r)
+                                picked.append(r)
+                        rows = np.array(sorted(picked), np.int64)
                     for r in rows:
                         qn = np.linalg.norm(Q[b, h, r].astype(np.float64))
                         Q[b, h, r] = (qn * u).astype(np.float32)
