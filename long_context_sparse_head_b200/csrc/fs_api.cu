@@ -65,6 +65,7 @@ WsLayout layout(const fs_params *p) {
     L.amax = off;  off += align256(BH * C * 4);
     L.idx = off;   off += align256(BH * (size_t)p->Nq * p->K * 4);
     L.olr = off;   off += align256(BH * (size_t)p->Nq * kD * 4);
+    L.rope = off;  off += align256((size_t)(128 + rope_table_rows(p->w)) * 32 * 8);
     L.total = off;
     return L;
 }
@@ -106,6 +107,11 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
         float *o = at<float>(ws, L.olr);
         if (launch_readout(D, p->dtype, Q, K, V, sel, o, st) != cudaSuccess) return FS_ERR_CUDA;
         olr = o;
+    }
+    if (p->dtype == FS_BF16) {
+        float2 *rt = at<float2>(ws, L.rope), *rb = rt + 128 * 32;
+        if (launch_rope_table(p->w, p->rope_base, rt, rb, st) != cudaSuccess) return FS_ERR_CUDA;
+        return cuda_status(launch_window_tc(D, Q, K, V, olr, O, rt, rb, at<int>(ws, L.flag), st));
     }
     return cuda_status(launch_window(D, p->dtype, Q, K, V, olr, O, st));
 }

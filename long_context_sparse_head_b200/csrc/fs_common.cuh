@@ -35,7 +35,7 @@ struct Dev {
 
 // Workspace layout (byte offsets from ws; each segment 256-byte aligned).
 struct WsLayout {
-    size_t flag, exitn, kbar, amax, idx, olr, total;
+    size_t flag, exitn, kbar, amax, idx, olr, rope, total;
 };
 
 // Device error flag codes (first int of the workspace).
@@ -94,7 +94,9 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 }
 
 // ---- kernel ids for the diagnostics (fs_kernel_times) ----
-enum KernelId : int { kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kNumKernels };
+enum KernelId : int {
+    kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kNumKernels
+};
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
 struct LaunchScope {
@@ -115,5 +117,11 @@ cudaError_t launch_readout(const Dev &P, fs_dtype dt, const void *Q, const void 
                            const void *V, const int32_t *idx, float *olr, cudaStream_t st);
 cudaError_t launch_window(const Dev &P, fs_dtype dt, const void *Q, const void *K,
                           const void *V, const float *olr, void *O, cudaStream_t st);
+// tensor-core window (bf16): angle tables, then the kernel
+int rope_table_rows(int w);
+cudaError_t launch_rope_table(int w, float rope_base, float2 *rope_t, float2 *rope_b, cudaStream_t st);
+cudaError_t launch_window_tc(const Dev &P, const void *Q, const void *K, const void *V,
+                             const float *olr, void *O, const float2 *rope_t, const float2 *rope_b,
+                             int *dev_flag, cudaStream_t st);
 
 }  // namespace fs
