@@ -118,6 +118,29 @@ fs_status fs_sync_status(void *ws, void *stream);
 /* Static description of a status code. */
 const char *fs_status_string(fs_status s);
 
+/* ---- selection without any device allocation (no counterpart in the method) ----
+ * fs_select_topk_noalloc computes exactly what fs_select_topk computes, for callers that
+ * cannot allocate device memory or hand the library a workspace: programs running inside
+ * a fixed device-memory budget planned in advance, plugins whose host framework owns all
+ * device allocations, and latency-critical loops where cudaMalloc/cudaFree would stall on
+ * a device-wide synchronization.  Its one scratch buffer, the TopP exit table, is a
+ * fixed array of FS_NOALLOC_MAX_CELLS ints (4 MiB) compiled into the library; every GPU
+ * that loads the library holds it until the process exits.  The call allocates nothing:
+ * no cudaMalloc, no cudaFree, no allocating library routine.
+ *   - With pruning on (W, P >= 0), B * H * floor(Nk / s) must not exceed
+ *     FS_NOALLOC_MAX_CELLS, else FS_ERR_UNSUPPORTED is returned before anything runs.
+ *   - The first call on a device does a one-time set-up with that device current (it
+ *     looks up the array's device address); make that first call before any stream
+ *     capture begins.
+ *   - All calls on a device share the one array, which keeps the last call's contents
+ *     (nothing in it has to start at zero: each call writes every entry it reads).  Calls
+ *     that overlap on the GPU (different streams, or threads, without ordering between
+ *     them) race on it; order them, e.g. by issuing them on one stream.
+ * Arguments, layouts and the other errors are those of fs_select_topk. */
+#define FS_NOALLOC_MAX_CELLS (1 << 20)
+fs_status fs_select_topk_noalloc(const fs_params *p, const void *Q, const float *kbar,
+                                 const float *amax, int32_t *idx, void *stream);
+
 /* ---- diagnostics (no counterpart in the method: measurement support) ----
  * fs_launch_count: kernels this library has launched since load (all calls, streams).
  * fs_timing_enable(1): from now on every kernel launch is bracketed by two CUDA events

@@ -22,7 +22,8 @@ STATUS = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_UNSUPPORTED", 3: "FS_E
           4: "FS_ERR_CUDA", 5: "FS_ERR_TIMEOUT"}
 EXPORTS = ("fs_workspace_size", "fs_cell_summaries", "fs_select_topk", "fs_forward",
            "fs_host_scratch_size", "fs_forward_host", "fs_sync_status", "fs_status_string",
-           "fs_launch_count", "fs_timing_enable", "fs_kernel_times", "fs_kernel_name")
+           "fs_launch_count", "fs_timing_enable", "fs_kernel_times", "fs_kernel_name",
+           "fs_select_topk_noalloc")
 
 
 class FsError(RuntimeError):
@@ -61,6 +62,7 @@ def load():
         L.fs_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
         L.fs_cell_summaries.argtypes = [P, vp, vp, vp, vp]
         L.fs_select_topk.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
+        L.fs_select_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp]
         L.fs_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.fs_host_scratch_size.argtypes = [P, ctypes.POINTER(sz)]
         L.fs_forward_host.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
@@ -162,6 +164,13 @@ def select_topk(params, Q, kbar, amax, idx, ws, stream=None):
     _check(load().fs_select_topk(params.ref(), _ptr(Q), _ptr(kbar), _ptr(amax), _ptr(idx),
                                  _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "fs_select_topk")
+
+
+def select_topk_noalloc(params, Q, kbar, amax, idx, stream=None):
+    """fs_select_topk without a workspace, for callers that cannot allocate device memory:
+    its scratch is a fixed array inside the library (see include/freesolo.h)."""
+    _check(load().fs_select_topk_noalloc(params.ref(), _ptr(Q), _ptr(kbar), _ptr(amax),
+                                         _ptr(idx), _stream(stream)), "fs_select_topk_noalloc")
 
 
 def forward(params, Q, K, V, O, ws, kbar=None, amax=None, idx=None, stream=None):

@@ -117,6 +117,11 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
 }
 
 }  // namespace
+
+fs_status validate_params(const fs_params *p) { return validate(p); }
+Dev make_dev_params(const fs_params *p) { return make_dev(p); }
+bool params_have_long_range(const fs_params *p) { return has_long_range(p); }
+
 }  // namespace fs
 
 using namespace fs;

@@ -107,6 +107,11 @@ struct LaunchScope {
     int slot;
 };
 
+// ---- argument checks shared by the entry points (defined in fs_api.cu) ----
+fs_status validate_params(const fs_params *p);
+Dev make_dev_params(const fs_params *p);
+bool params_have_long_range(const fs_params *p);
+
 // ---- launchers (one per kernel file) ----
 cudaError_t launch_summaries(const Dev &P, fs_dtype dt, const void *K, float *kbar,
                              float *amax, cudaStream_t st);
