@@ -53,7 +53,8 @@ typedef enum {
     FS_ERR_UNSUPPORTED = 2,   /* a size or option outside the supported set above */
     FS_ERR_WORKSPACE = 3,     /* workspace missing or smaller than fs_workspace_size() */
     FS_ERR_CUDA = 4,          /* a CUDA call or kernel launch failed */
-    FS_ERR_TIMEOUT = 5        /* a kernel gave up a bounded wait (device error flag) */
+    FS_ERR_TIMEOUT = 5,       /* a kernel gave up a bounded wait (device error flag) */
+    FS_ERR_KERNEL_CHECK = 6   /* a kernel's internal consistency check failed (device flag) */
 } fs_status;
 
 typedef enum { FS_BF16 = 0, FS_F32 = 1 } fs_dtype;
@@ -112,6 +113,8 @@ fs_status fs_forward_host(const fs_params *p, const void *hQ, const void *hK, co
 
 /* Synchronizes `stream`, then reads and clears the device error flag in `ws`.
  * Returns FS_ERR_TIMEOUT if a kernel gave up a bounded wait since the last check,
+ * FS_ERR_KERNEL_CHECK if a kernel found its inputs inconsistent (e.g. more distinct
+ * selected cells in a 128-row tile than the bound derived from W and P),
  * FS_ERR_CUDA if the stream reports an error, else FS_OK. */
 fs_status fs_sync_status(void *ws, void *stream);
 

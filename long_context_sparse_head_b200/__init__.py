@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libfreesolo.so")
 
 FS_BF16, FS_F32 = 0, 1
 STATUS = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_UNSUPPORTED", 3: "FS_ERR_WORKSPACE",
-          4: "FS_ERR_CUDA", 5: "FS_ERR_TIMEOUT"}
+          4: "FS_ERR_CUDA", 5: "FS_ERR_TIMEOUT", 6: "FS_ERR_KERNEL_CHECK"}
 EXPORTS = ("fs_workspace_size", "fs_cell_summaries", "fs_select_topk", "fs_forward",
            "fs_host_scratch_size", "fs_forward_host", "fs_sync_status", "fs_status_string",
            "fs_launch_count", "fs_timing_enable", "fs_kernel_times", "fs_kernel_name",

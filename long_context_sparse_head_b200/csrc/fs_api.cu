@@ -88,6 +88,22 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
     const Dev D = make_dev(p);
     const WsLayout L = layout(p);
     const float *olr = nullptr;
+    const bool fused = has_long_range(p) && !idx && attn_tc_supported(p);
+    if (fused) {   // bf16: selection, then one tensor-core kernel for readout + window + combine
+        if (!kbar) {
+            float *kb = at<float>(ws, L.kbar), *am = at<float>(ws, L.amax);
+            if (launch_summaries(D, p->dtype, K, kb, am, st) != cudaSuccess) return FS_ERR_CUDA;
+            kbar = kb;
+            amax = am;
+        }
+        int *exitn = at<int>(ws, L.exitn);
+        if (D.prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
+        int32_t *wsidx = at<int32_t>(ws, L.idx);
+        if (launch_select(D, p->dtype, Q, kbar, amax, exitn, wsidx, st) != cudaSuccess) return FS_ERR_CUDA;
+        float2 *rt = at<float2>(ws, L.rope), *rb = rt + 128 * 32;
+        if (launch_rope_table(p->w, p->rope_base, rt, rb, st) != cudaSuccess) return FS_ERR_CUDA;
+        return cuda_status(launch_attn_tc(D, Q, K, V, wsidx, O, rt, rb, at<int>(ws, L.flag), st));
+    }
     if (has_long_range(p)) {
         const int32_t *sel = idx;
         if (!sel) {
@@ -232,7 +248,7 @@ extern "C" fs_status fs_sync_status(void *ws, void *stream) {
     if (flag != kFlagOk) {
         const int zero = 0;
         if (cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return FS_ERR_CUDA;
-        return FS_ERR_TIMEOUT;
+        return flag == kFlagTimeout ? FS_ERR_TIMEOUT : FS_ERR_KERNEL_CHECK;
     }
     return FS_OK;
 }
@@ -245,6 +261,7 @@ extern "C" const char *fs_status_string(fs_status s) {
     case FS_ERR_WORKSPACE: return "workspace missing or too small";
     case FS_ERR_CUDA: return "CUDA error";
     case FS_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    case FS_ERR_KERNEL_CHECK: return "a kernel's consistency check failed";
     }
     return "unknown status";
 }

@@ -1,0 +1,470 @@
+// Fused long-range readout + local window + combination on the 5th-generation tensor
+// cores (bf16), "FreeSolo" summary §3.3 eq. (9), §3.2 eqs. (3)-(4), §3.1 eq. (2):
+//   u_i    = softmax_{tokens of the cells in S_i}(q_i.k_j / sqrt(d)) V        (NoPE)
+//   o_i^lr = RMSNorm(u_i)
+//   o_i^sr = softmax_{j in [i-w, i]}((R(i)q_i).(R(j)k_j) / sqrt(d)) V       (RoPE)
+//   O_i    = o_i^sr + alpha_h o_i^lr
+// with S_i given by the selection kernel (idx).
+//
+// One CTA per 128 query rows of a (batch, head); two CTAs per SM.  The readout runs over
+// U, the union of the cells the tile's rows selected (|U| <= 128, ascending), four cells
+// (128 keys) per chunk, each cell fetched by its own 32-row TMA box; a row masks the
+// cells it did not select (masked-dense on the tensor cores).  Then the window runs
+// over 128-key chunks as in the window-only kernel.  Both softmaxes accumulate in tensor
+// memory: S/P in columns [0,128), the readout's O in [128,192), the window's O in
+// [192,256).  When the first window chunk arrives, the readout is finished: the softmax
+// threads turn its O into alpha_h * RMSNorm(u) in place; the epilogue adds it to the
+// window's output.  No intermediate leaves the SM.
+//
+// Warps: 0-3 softmax (thread = query row = TMEM lane), 4 TMA, 5 MMA, 6-9 auxiliary
+// (build U and the per-row selection masks from idx, rotate Q and the window's K chunks).
+#include "tc_rope.cuh"
+
+namespace fs {
+
+namespace {
+constexpr int BM = 128, BN = 128, NSTAGE = 2;
+constexpr int UMAX = 128;                        // largest union of selected cells per tile
+constexpr int CPC = BN / kS;                     // cells per readout chunk (4)
+constexpr int W_TMA = 4, W_MMA = 5, W_AUX0 = 6, NWARPS = 10;
+constexpr int NTHREADS = NWARPS * 32;
+constexpr uint32_t TMEM_COLS = 256, S_COL = 0, OLR_COL = 128, OSR_COL = 192;
+constexpr int TILE_BYTES = BM * kD * 2;         // 128 x 64 bf16: 16 KiB
+constexpr int CELL_BYTES = kS * kD * 2;         // 32 x 64 bf16: 4 KiB
+constexpr int kAuxBarrier = 1;                  // named barrier of the 128 auxiliary threads
+
+struct AttnSmem {
+    __nv_bfloat16 qn[BM * kD];                  // Q as loaded (NoPE)
+    __nv_bfloat16 qr[BM * kD];                  // Q rotated (RoPE)
+    __nv_bfloat16 k[NSTAGE][BN * kD];
+    __nv_bfloat16 v[NSTAGE][BN * kD];
+    uint32_t mask[BM][UMAX / 32];               // row -> selected union positions
+    int ulist[UMAX];                            // union cells, ascending
+    int nU;
+    int warp_tot[4];
+    uint64_t q_full, q_ready, u_ready, s_full, p_full, o_done, drain;
+    uint64_t kv_full[NSTAGE], k_ready[NSTAGE], kv_empty[NSTAGE];
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct AttnArgs {
+    int Nq, Nk, q0, w, C, K, H;
+    float scale_log2e;      // log2(e) / sqrt(d)
+    float rms_eps;
+    float alpha[FS_MAX_HEADS];
+};
+
+__device__ __forceinline__ void aux_sync() {
+    asm volatile("bar.sync %0, %1;" ::"n"(kAuxBarrier), "n"(128) : "memory");
+}
+
+// One chunk of online softmax for this thread's row.  S is read from TMEM columns
+// [S_COL, S_COL+128); P = exp2(S*c - m) is written as bf16 pairs over [S_COL, S_COL+64).
+// Readout chunks (MASKED_CELLS): 32-column block b is valid iff bit b of sel4 is set.
+// Window chunks: column c is valid iff clo <= c <= chi.
+template <bool MASKED_CELLS>
+__device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, bool first, uint32_t sel4,
+                                              int clo, int chi, float c_log2, float &m_used, float &l) {
+    auto col_ok = [&](int c) -> bool {
+        if (MASKED_CELLS) return ((sel4 >> (c >> 5)) & 1u) != 0;
+        return c >= clo && c <= chi;
+    };
+    auto blk_any = [&](int b) -> bool {
+        if (MASKED_CELLS) return ((sel4 >> b) & 1u) != 0;
+        return clo <= chi && clo <= 32 * b + 31 && chi >= 32 * b;
+    };
+    float mx = -INFINITY;
+#pragma unroll
+    for (int b = 0; b < BN / 32; b++) {
+        if (!__any_sync(kFull, blk_any(b))) continue;
+        uint32_t r[32];
+        tc::tmem_ld32(trow + S_COL + 32 * b, r);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e++)
+            if (col_ok(32 * b + e)) mx = fmaxf(mx, __uint_as_float(r[e]));
+    }
+    mx *= c_log2;
+    const bool grow = mx > m_used + 8.f;               // lazy rescale: only past 2^8
+    const float m_new = grow ? mx : m_used;
+    const float corr = (grow && m_used != -INFINITY) ? tc::ex2(m_used - m_new) : 1.f;
+    if (!first && __any_sync(kFull, corr != 1.f)) {
+#pragma unroll
+        for (int b = 0; b < kD / 32; b++) {
+            uint32_t r[32];
+            tc::tmem_ld32(trow + o_col + 32 * b, r);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; e++) r[e] = __float_as_uint(__uint_as_float(r[e]) * corr);
+            tc::tmem_st32(trow + o_col + 32 * b, r);
+        }
+        tc::tmem_wait_st();
+    }
+    l *= corr;
+    m_used = m_new;
+    const float msub = m_used == -INFINITY ? 0.f : m_used;
+#pragma unroll
+    for (int h2 = 0; h2 < 2; h2++) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int hb = 0; hb < 2; hb++) {
+            const int b = 2 * h2 + hb;
+            if (!__any_sync(kFull, blk_any(b))) {
+#pragma unroll
+                for (int e = 0; e < 16; e++) pk[16 * hb + e] = 0u;
+                continue;
+            }
+            uint32_t r[32];
+            tc::tmem_ld32(trow + S_COL + 32 * b, r);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; e++) {
+                const int c0 = 32 * b + 2 * e;
+                const float p0 = col_ok(c0) ? tc::ex2(__uint_as_float(r[2 * e]) * c_log2 - msub) : 0.f;
+                const float p1 = col_ok(c0 + 1) ? tc::ex2(__uint_as_float(r[2 * e + 1]) * c_log2 - msub) : 0.f;
+                l += p0 + p1;
+                pk[16 * hb + e] = tc::pack_bf16x2(p0, p1);
+            }
+        }
+        tc::tmem_st32(trow + S_COL + 32 * h2, pk);
+    }
+    tc::tmem_wait_st();
+}
+}  // namespace
+
+__global__ void __launch_bounds__(NTHREADS, 2)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk32,
+               const __grid_constant__ CUtensorMap tv32, const __grid_constant__ CUtensorMap tk128,
+               const __grid_constant__ CUtensorMap tv128, const AttnArgs A,
+               const int32_t *__restrict__ idx, const float2 *__restrict__ rope_t,
+               const float2 *__restrict__ rope_b, __nv_bfloat16 *__restrict__ O, int *dev_flag) {
+    extern __shared__ uint8_t smraw[];
+    const uint32_t sbase = tc::smem_u32(smraw);
+    AttnSmem &sm = *reinterpret_cast<AttnSmem *>(smraw + (((sbase + 1023u) & ~1023u) - sbase));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y, h = bh % A.H;
+    const int r0 = blockIdx.x * BM;
+    const int pb = A.q0 + r0;
+    const int nrows = min(BM, A.Nq - r0);
+    const int jbase = pb - A.w;
+    const int last = pb + nrows - 1;
+    const int k_first = jbase < 0 ? (-jbase) / BN : 0;
+    const int nW = (last - jbase) / BN - k_first + 1;    // window chunks
+    const tc::Abort ab{dev_flag, &sm.abort};
+
+    if (threadIdx.x == 0) {
+        sm.abort = 0;
+        tc::mbar_init(&sm.q_full, 1);
+        tc::mbar_init(&sm.q_ready, 128);
+        tc::mbar_init(&sm.u_ready, 128);
+        tc::mbar_init(&sm.s_full, 1);
+        tc::mbar_init(&sm.p_full, 128);
+        tc::mbar_init(&sm.o_done, 1);
+        tc::mbar_init(&sm.drain, 1);
+        for (int s = 0; s < NSTAGE; s++) {
+            tc::mbar_init(&sm.kv_full[s], 1);
+            tc::mbar_init(&sm.k_ready[s], 128);
+            tc::mbar_init(&sm.kv_empty[s], 1);
+        }
+        tc::fence_barrier_init();
+    }
+    if (warp == W_MMA) {
+        tc::tmem_alloc(&sm.tmem_base, TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == W_TMA) {
+        if (lane == 0) {
+            tc::prefetch_tmap(&tq);
+            tc::prefetch_tmap(&tk32);
+            tc::prefetch_tmap(&tv32);
+            tc::prefetch_tmap(&tk128);
+            tc::prefetch_tmap(&tv128);
+            tc::mbar_expect_tx(&sm.q_full, TILE_BYTES);
+            tc::tma_load_3d(sm.qn, &tq, &sm.q_full, 0, r0, bh);
+            int it = 0;
+            if (tc::mbar_wait(&sm.u_ready, 0, ab)) {
+                const int nU = sm.nU, nR = (nU + CPC - 1) / CPC, total = nR + nW;
+                for (; it < total; it++) {
+                    const int s = it % NSTAGE;
+                    if (!tc::mbar_wait(&sm.kv_empty[s], ((it / NSTAGE) & 1) ^ 1, ab)) break;
+                    if (it < nR) {          // four gathered cells; unused slots read zeros
+                        tc::mbar_expect_tx(&sm.kv_full[s], 2 * CPC * CELL_BYTES);
+                        for (int j = 0; j < CPC; j++) {
+                            const int u = CPC * it + j;
+                            const int y = u < nU ? sm.ulist[u] * kS : A.Nk;   // past the end: zero fill
+                            tc::tma_load_3d(sm.k[s] + j * kS * kD, &tk32, &sm.kv_full[s], 0, y, bh);
+                            tc::tma_load_3d(sm.v[s] + j * kS * kD, &tv32, &sm.kv_full[s], 0, y, bh);
+                        }
+                    } else {                // 128 consecutive keys of the band
+                        const int jc = jbase + BN * (k_first + it - nR);
+                        tc::mbar_expect_tx(&sm.kv_full[s], 2 * TILE_BYTES);
+                        tc::tma_load_3d(sm.k[s], &tk128, &sm.kv_full[s], 0, jc, bh);
+                        tc::tma_load_3d(sm.v[s], &tv128, &sm.kv_full[s], 0, jc, bh);
+                    }
+                }
+            }
+            if (sm.abort) {   // let issued copies land before the CTA's memory is released
+                for (int j = max(0, it - NSTAGE); j < it; j++) {
+                    const uint64_t t0 = tc::globaltimer();
+                    while (!tc::mbar_try_wait(&sm.kv_full[j % NSTAGE], (j / NSTAGE) & 1) &&
+                           tc::globaltimer() - t0 < tc::kWaitLimitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp >= W_AUX0) {
+        const int t = threadIdx.x - W_AUX0 * 32, aw = t >> 5;
+        // ---- U: union of the rows' selected cells, via a bitmap over [0, C) that lives
+        //      in the (not yet loaded) K/V stages, plus a cell -> position byte table
+        uint32_t *bitmap = reinterpret_cast<uint32_t *>(&sm.k[0][0]);
+        uint8_t *cpos = reinterpret_cast<uint8_t *>(&sm.v[0][0]);
+        const int nwords = (A.C + 31) / 32;
+        for (int wd = t; wd < nwords; wd += 128) bitmap[wd] = 0u;
+        aux_sync();
+        const int32_t *myidx = idx + ((size_t)bh * A.Nq + r0 + t) * A.K;
+        if (t < nrows)
+            for (int e = 0; e < A.K; e++) {
+                const int c = myidx[e];
+                if (c >= 0 && c < A.C) atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+            }
+        aux_sync();
+        const int R = (nwords + 127) / 128, w0 = min(t * R, nwords), w1 = min(w0 + R, nwords);
+        int cnt = 0;
+        for (int wd = w0; wd < w1; wd++) cnt += __popc(bitmap[wd]);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) sm.warp_tot[aw] = incl;
+        aux_sync();
+        int pos = incl - cnt, total = 0;
+        for (int k = 0; k < 4; k++) {
+            if (k < aw) pos += sm.warp_tot[k];
+            total += sm.warp_tot[k];
+        }
+        for (int wd = w0; wd < w1; wd++) {
+            uint32_t bits = bitmap[wd];
+            while (bits) {
+                const int c = wd * 32 + __ffs(bits) - 1;
+                bits &= bits - 1;
+                if (pos < UMAX) {
+                    sm.ulist[pos] = c;
+                    cpos[c] = (uint8_t)pos;
+                }
+                pos++;
+            }
+        }
+        if (t == 0) {
+            sm.nU = min(total, UMAX);
+            if (total > UMAX) atomicExch(dev_flag, kFlagCheck);
+        }
+        aux_sync();
+        uint32_t mw[UMAX / 32] = {0u, 0u, 0u, 0u};
+        if (t < nrows)
+            for (int e = 0; e < A.K; e++) {
+                const int c = myidx[e];
+                if (c >= 0 && c < A.C) {
+                    const int p = cpos[c];
+                    if (p < UMAX) mw[p >> 5] |= 1u << (p & 31);
+                }
+            }
+#pragma unroll
+        for (int k = 0; k < UMAX / 32; k++) sm.mask[t][k] = mw[k];
+        aux_sync();                       // scratch reads done before the stages are loaded
+        tc::fence_async_shared();
+        tc::mbar_arrive(&sm.u_ready);
+        const int nR = (sm.nU + CPC - 1) / CPC, total_ck = nR + nW;
+        // ---- rotate Q for the window, then pass through (readout) or rotate (window) K
+        if (tc::mbar_wait(&sm.q_full, 0, ab)) {
+            tc::rotate_tile(sm.qn, sm.qr, t, rope_t, nullptr);
+            tc::fence_async_shared();
+            tc::mbar_arrive(&sm.q_ready);
+            for (int it = 0; it < total_ck; it++) {
+                const int s = it % NSTAGE;
+                if (!tc::mbar_wait(&sm.kv_full[s], (it / NSTAGE) & 1, ab)) break;
+                if (it >= nR) {
+                    tc::rotate_tile(sm.k[s], sm.k[s], t, rope_t,
+                                    rope_b + (size_t)(k_first + it - nR) * 32);
+                    tc::fence_async_shared();
+                }
+                tc::mbar_arrive(&sm.k_ready[s]);
+            }
+        }
+    } else if (warp == W_MMA) {
+        if (lane == 0) {
+            const uint32_t id_qk = tc::idesc_bf16(BM, BN, false, false);
+            const uint32_t id_pv = tc::idesc_bf16(BM, kD, false, true);
+            const uint32_t qn = tc::smem_u32(sm.qn), qr = tc::smem_u32(sm.qr);
+            bool ok = tc::mbar_wait(&sm.u_ready, 0, ab) && tc::mbar_wait(&sm.q_full, 0, ab);
+            const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0, total = nR + nW;
+            int issued = 0;
+            for (int it = 0; ok && it <= total; it++) {
+                if (it < total && !tc::mbar_wait(&sm.k_ready[it % NSTAGE], (it / NSTAGE) & 1, ab)) {
+                    ok = false;
+                    break;
+                }
+                if (it > 0) {   // O += P(it-1) V(it-1), into the readout's or the window's O
+                    if (!tc::mbar_wait(&sm.p_full, (it - 1) & 1, ab)) { ok = false; break; }
+                    tc::tc_fence_after();
+                    const int pj = it - 1;
+                    const uint32_t ocol = pj < nR ? OLR_COL : OSR_COL;
+                    const bool first = pj == 0 || pj == nR;
+                    const uint32_t vb = tc::smem_u32(sm.v[pj % NSTAGE]);
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; kk++)
+                        tc::mma_ts(tmem + ocol, tmem + S_COL + kk * 8, tc::sdesc_sw128(vb + kk * 2048, 16, 1024),
+                                   id_pv, (!first || kk > 0) ? 1u : 0u);
+                    tc::mma_commit(&sm.kv_empty[pj % NSTAGE]);
+                    issued++;
+                }
+                if (it < total) {   // S = Q K(it)^T with the NoPE or the rotated Q
+                    if (it == nR && !tc::mbar_wait(&sm.q_ready, 0, ab)) { ok = false; break; }
+                    tc::tc_fence_after();
+                    const uint32_t qa = it < nR ? qn : qr;
+                    const uint32_t kb = tc::smem_u32(sm.k[it % NSTAGE]);
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; kk++)
+                        tc::mma_ss(tmem + S_COL, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
+                                   tc::sdesc_sw128(kb + kk * 32, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
+                    tc::mma_commit(&sm.s_full);
+                    issued++;
+                }
+            }
+            if (ok) tc::mma_commit(&sm.o_done);
+            if (issued) {
+                tc::mma_commit(&sm.drain);
+                const uint64_t t0 = tc::globaltimer();
+                while (!tc::mbar_try_wait(&sm.drain, 0) && tc::globaltimer() - t0 < tc::kWaitLimitNs) {
+                }
+            }
+        }
+    } else {
+        // ---- softmax: thread = query row
+        const int row = warp * 32 + lane;
+        const int i = pb + row;
+        const bool rvalid = row < nrows;
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+        bool ok = tc::mbar_wait(&sm.u_ready, 0, ab);
+        const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0, total = nR + nW;
+        uint32_t mw[UMAX / 32];
+#pragma unroll
+        for (int k = 0; k < UMAX / 32; k++) mw[k] = ok ? sm.mask[row][k] : 0u;
+        float m_lr = -INFINITY, l_lr = 0.f, m_sr = -INFINITY, l_sr = 0.f;
+        for (int it = 0; ok && it < total; it++) {
+            if (!tc::mbar_wait(&sm.s_full, it & 1, ab)) { ok = false; break; }
+            tc::tc_fence_after();
+            if (it < nR) {
+                const int p0 = CPC * it;
+                const uint32_t sel4 = (mw[p0 >> 5] >> (p0 & 31)) & 0xfu;
+                softmax_chunk<true>(trow, OLR_COL, it == 0, sel4, 0, -1, A.scale_log2e, m_lr, l_lr);
+            } else {
+                if (it == nR && nR > 0) {   // readout done: O_lr <- alpha_h RMSNorm(O_lr / l)
+                    uint32_t a[32], b[32];
+                    tc::tmem_ld32(trow + OLR_COL, a);
+                    tc::tmem_ld32(trow + OLR_COL + 32, b);
+                    tc::tmem_wait_ld();
+                    const float inv_l = l_lr > 0.f ? 1.f / l_lr : 0.f;
+                    float ss = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 32; e++) {
+                        const float x = __uint_as_float(a[e]) * inv_l, y = __uint_as_float(b[e]) * inv_l;
+                        ss = fmaf(x, x, fmaf(y, y, ss));
+                    }
+                    const float f = l_lr > 0.f ? A.alpha[h] * inv_l / sqrtf(ss * (1.f / kD) + A.rms_eps) : 0.f;
+#pragma unroll
+                    for (int e = 0; e < 32; e++) {
+                        a[e] = __float_as_uint(__uint_as_float(a[e]) * f);
+                        b[e] = __float_as_uint(__uint_as_float(b[e]) * f);
+                    }
+                    tc::tmem_st32(trow + OLR_COL, a);
+                    tc::tmem_st32(trow + OLR_COL + 32, b);
+                    tc::tmem_wait_st();
+                }
+                const int jc = jbase + BN * (k_first + it - nR);
+                int clo = max(-jc, i - A.w - jc), chi = min(i - jc, BN - 1);
+                if (!rvalid) { clo = 1; chi = 0; }
+                softmax_chunk<false>(trow, OSR_COL, it == nR, 0u, clo, chi, A.scale_log2e, m_sr, l_sr);
+            }
+            tc::tc_fence_before();
+            tc::mbar_arrive(&sm.p_full);
+        }
+        if (ok && tc::mbar_wait(&sm.o_done, 0, ab)) {
+            tc::tc_fence_after();
+            const size_t orow = ((size_t)bh * A.Nq + r0 + row) * kD;
+            const float inv = l_sr > 0.f ? 1.f / l_sr : 0.f;
+#pragma unroll
+            for (int hf = 0; hf < 2; hf++) {
+                uint32_t a[32], b[32];
+                tc::tmem_ld32(trow + OSR_COL + 32 * hf, a);
+                if (nR > 0) tc::tmem_ld32(trow + OLR_COL + 32 * hf, b);
+                tc::tmem_wait_ld();
+                uint32_t outw[16];
+#pragma unroll
+                for (int e = 0; e < 16; e++) {
+                    float o0 = __uint_as_float(a[2 * e]) * inv, o1 = __uint_as_float(a[2 * e + 1]) * inv;
+                    if (nR > 0) {
+                        o0 += __uint_as_float(b[2 * e]);
+                        o1 += __uint_as_float(b[2 * e + 1]);
+                    }
+                    outw[e] = tc::pack_bf16x2(o0, o1);
+                }
+                if (rvalid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(O + orow + 32 * hf);
+#pragma unroll
+                    for (int e = 0; e < 4; e++)
+                        dst[e] = make_uint4(outw[4 * e], outw[4 * e + 1], outw[4 * e + 2], outw[4 * e + 3]);
+                }
+            }
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == W_MMA) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+bool attn_tc_supported(const fs_params *p) {
+    const int C = p->Nk / p->s;
+    if (p->dtype != FS_BF16 || C > 32768) return false;
+    const int bound = p->W >= 0 ? p->W + p->P + 10 : C;     // largest possible |U| per tile
+    return bound <= UMAX;
+}
+
+cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V,
+                           const int32_t *idx, void *O, const float2 *rope_t, const float2 *rope_b,
+                           int *dev_flag, cudaStream_t st) {
+    if (P.Nq == 0) return cudaSuccess;
+    const int BH = P.B * P.H;
+    CUtensorMap tq, tk32, tv32, tk128, tv128;
+    if (!encode_tmap_3d_bf16(&tq, Q, kD, P.Nq, BH, kD, BM) ||
+        !encode_tmap_3d_bf16(&tk32, K, kD, P.Nk, BH, kD, kS) ||
+        !encode_tmap_3d_bf16(&tv32, V, kD, P.Nk, BH, kD, kS) ||
+        !encode_tmap_3d_bf16(&tk128, K, kD, P.Nk, BH, kD, BN) ||
+        !encode_tmap_3d_bf16(&tv128, V, kD, P.Nk, BH, kD, BN))
+        return cudaErrorInvalidValue;
+    AttnArgs A;
+    A.Nq = P.Nq; A.Nk = P.Nk; A.q0 = P.q0; A.w = P.w; A.C = P.C; A.K = P.K; A.H = P.H;
+    A.scale_log2e = P.scale * 1.4426950408889634f;
+    A.rms_eps = P.rms_eps;
+    for (int hh = 0; hh < FS_MAX_HEADS; hh++) A.alpha[hh] = P.alpha[hh];
+    const size_t smem = sizeof(AttnSmem) + 1024;
+    const dim3 grid((P.Nq + BM - 1) / BM, BH);
+    LaunchScope scope(kAttnTc, st);
+    cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attn_tc_kernel<<<grid, NTHREADS, smem, st>>>(tq, tk32, tv32, tk128, tv128, A, idx, rope_t, rope_b,
+                                                 (__nv_bfloat16 *)O, dev_flag);
+    return cudaGetLastError();
+}
+
+}  // namespace fs

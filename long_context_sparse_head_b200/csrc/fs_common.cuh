@@ -39,7 +39,7 @@ struct WsLayout {
 };
 
 // Device error flag codes (first int of the workspace).
-enum : int { kFlagOk = 0, kFlagTimeout = 1 };
+enum : int { kFlagOk = 0, kFlagTimeout = 1, kFlagCheck = 2 };
 
 // Candidate count |C_i| for key-index position i: cells with (c+1)s <= i - w.
 __host__ __device__ inline int cand_count(int i, int w, int C) {
@@ -95,7 +95,8 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 
 // ---- kernel ids for the diagnostics (fs_kernel_times) ----
 enum KernelId : int {
-    kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kNumKernels
+    kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
+    kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
@@ -128,5 +129,10 @@ cudaError_t launch_rope_table(int w, float rope_base, float2 *rope_t, float2 *ro
 cudaError_t launch_window_tc(const Dev &P, const void *Q, const void *K, const void *V,
                              const float *olr, void *O, const float2 *rope_t, const float2 *rope_b,
                              int *dev_flag, cudaStream_t st);
+// fused tensor-core readout + window + combine (bf16, internally selected cells)
+bool attn_tc_supported(const fs_params *p);
+cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V,
+                           const int32_t *idx, void *O, const float2 *rope_t, const float2 *rope_b,
+                           int *dev_flag, cudaStream_t st);
 
 }  // namespace fs

@@ -17,7 +17,7 @@
 // rescale), write P = exp2(S*scale*log2e - m) as bf16 pairs over S's first 64 columns,
 // and the next MMA accumulates P V into O (columns [128,192)).  MMAs issued by one
 // thread run in order, so the next S never overwrites P before P V has read it.
-#include "tc_common.cuh"
+#include "tc_rope.cuh"
 
 namespace fs {
 
@@ -44,42 +44,6 @@ struct WinArgs {
     float scale_log2e;       // log2(e) / sqrt(d)
     int rope_nb;             // rows of the chunk-base angle table
 };
-
-// Rotate the 128 x 64 bf16 tile (128-byte swizzle: logical 16-byte chunk c of row r sits
-// at chunk c ^ (r & 7)) by angle (row + base_k) * theta_m for pair m.  Thread t of 128.
-__device__ __forceinline__ void rotate_tile(__nv_bfloat16 *tile, int t, const float2 *__restrict__ rt,
-                                            const float2 *__restrict__ rb) {
-    uint8_t *base = reinterpret_cast<uint8_t *>(tile);
-#pragma unroll 2
-    for (int j = 0; j < 8; j++) {
-        const int item = t + 128 * j;
-        const int row = item >> 3, c = item & 7;
-        uint4 *p = reinterpret_cast<uint4 *>(base + row * 128 + ((c ^ (row & 7)) << 4));
-        uint4 x = *p;
-        const float4 *tr = reinterpret_cast<const float4 *>(rt + row * 32 + 4 * c);
-        float4 a01 = __ldg(tr), a23 = __ldg(tr + 1);
-        float cs[4] = {a01.x, a01.z, a23.x, a23.z}, sn[4] = {a01.y, a01.w, a23.y, a23.w};
-        if (rb) {
-            const float4 *tb = reinterpret_cast<const float4 *>(rb + 4 * c);
-            float4 b01 = __ldg(tb), b23 = __ldg(tb + 1);
-            const float cb[4] = {b01.x, b01.z, b23.x, b23.z}, sb[4] = {b01.y, b01.w, b23.y, b23.w};
-#pragma unroll
-            for (int e = 0; e < 4; e++) {
-                const float c2 = cs[e] * cb[e] - sn[e] * sb[e];
-                const float s2 = sn[e] * cb[e] + cs[e] * sb[e];
-                cs[e] = c2;
-                sn[e] = s2;
-            }
-        }
-        uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int e = 0; e < 4; e++) {
-            const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xffff0000u);
-            w[e] = tc::pack_bf16x2(x0 * cs[e] - x1 * sn[e], x0 * sn[e] + x1 * cs[e]);
-        }
-        *p = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
 
 __device__ __forceinline__ bool in_band(int c, int clo, int chi) { return c >= clo && c <= chi; }
 }  // namespace
@@ -156,13 +120,13 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     } else if (warp >= W_ROT0) {
         const int t = threadIdx.x - W_ROT0 * 32;
         if (tc::mbar_wait(&sm.q_full, 0, ab)) {
-            rotate_tile(sm.q, t, rope_t, nullptr);
+            tc::rotate_tile(sm.q, sm.q, t, rope_t, nullptr);
             tc::fence_async_shared();
             tc::mbar_arrive(&sm.q_ready);
             for (int it = 0; it < nck; it++) {
                 const int s = it % NSTAGE;
                 if (!tc::mbar_wait(&sm.kv_full[s], (it / NSTAGE) & 1, ab)) break;
-                rotate_tile(sm.k[s], t, rope_t, rope_b + (size_t)(k_first + it) * 32);
+                tc::rotate_tile(sm.k[s], sm.k[s], t, rope_t, rope_b + (size_t)(k_first + it) * 32);
                 tc::fence_async_shared();
                 tc::mbar_arrive(&sm.k_ready[s]);
             }

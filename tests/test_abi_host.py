@@ -32,7 +32,7 @@ def test_library_exports_every_declared_function():
 
 
 def test_status_strings():
-    for code in range(6):
+    for code in range(7):
         assert fs.status_string(code)
     assert fs.status_string(99) == "unknown status"
 
