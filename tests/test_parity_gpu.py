@@ -90,7 +90,10 @@ def test_caller_idx_runs_readout_on_given_cells():
     idx_sel = g.select().clone()
     O_sel = g.forward().clone()
     O_given = g.forward(idx=idx_sel)
-    assert torch.equal(O_sel, O_given)
+    # caller-given cells take the separate readout kernel; the fused kernel selected the
+    # same cells, so the two agree within the bf16 tolerance (each is checked against the
+    # oracle on its own elsewhere)
+    assert (O_sel.float() - O_given.float()).abs().max().item() <= 2e-2
     # random ascending cell lists inside each row's candidate prefix
     rng = np.random.default_rng(3)
     idx = -np.ones((wl.B, wl.H, wl.Nq, wl.K), np.int32)
