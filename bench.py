@@ -182,6 +182,10 @@ def algorithmic_work(wl, n_sel_cells):
         "select_topk": ("hbm", BH * wl.Nq * wl.d * e + BH * C * wl.d * 4 + BH * wl.Nq * wl.K * 4),
         "readout": ("alu", 4 * wl.d * wl.s * n_sel_cells),
         "window_combine": ("alu", 4 * wl.d * win_keys),
+        "rope_table": ("hbm", (128 + wl.w // 128 + 2) * 32 * 8),
+        "window_tc": ("tensor", 4 * wl.d * win_keys),
+        "attn_tc": ("tensor", 4 * wl.d * win_keys + 4 * wl.d * wl.s * n_sel_cells),
+        "select_tc": ("hbm", BH * wl.Nq * wl.d * e + BH * C * wl.d * 4 + BH * wl.Nq * wl.K * 4),
         "_path_bytes": qkv + o + BH * C * (wl.d + 1) * 4 * 2,
         "_window_flops": 4 * wl.d * win_keys,
         "_readout_flops": 4 * wl.d * wl.s * n_sel_cells,
@@ -191,7 +195,8 @@ def algorithmic_work(wl, n_sel_cells):
 def source_hash(kernel):
     files = {"readout": "fs_readout.cu", "window_combine": "fs_window.cu",
              "cell_summaries": "fs_summaries.cu", "exit_times": "fs_prune.cu",
-             "select_topk": "fs_select.cu"}
+             "select_topk": "fs_select.cu", "window_tc": "fs_window_tc.cu",
+             "attn_tc": "fs_attn_tc.cu", "select_tc": "fs_select_tc.cu"}
     path = os.path.join(ROOT, "long_context_sparse_head_b200", "csrc", files.get(kernel, ""))
     if not os.path.isfile(path):
         return None
@@ -386,7 +391,7 @@ def run_ours(args):
     dom = max((k for k in ktimes if ktimes[k][0] > 0), key=lambda k: ktimes[k][1])
     cnt, tot_ms = ktimes[dom]
     avg_s = tot_ms / cnt * 1e-3
-    bound, amount = work[dom]
+    bound, amount = work.get(dom, ("hbm", 0))
     clock_mhz = pk.get("sm_max_mhz", 1965.0)
     if bound == "hbm":
         peak, unit, achieved = pk["hbm_gbs"], "GB/s", amount / avg_s / 1e9

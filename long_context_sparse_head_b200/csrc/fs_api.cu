@@ -99,7 +99,7 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
         int *exitn = at<int>(ws, L.exitn);
         if (D.prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
         int32_t *wsidx = at<int32_t>(ws, L.idx);
-        if (launch_select(D, p->dtype, Q, kbar, amax, exitn, wsidx, st) != cudaSuccess) return FS_ERR_CUDA;
+        if (launch_selection(p, D, Q, kbar, amax, exitn, wsidx, at<int>(ws, L.flag), st) != cudaSuccess) return FS_ERR_CUDA;
         float2 *rt = at<float2>(ws, L.rope), *rb = rt + 128 * 32;
         if (launch_rope_table(p->w, p->rope_base, rt, rb, st) != cudaSuccess) return FS_ERR_CUDA;
         return cuda_status(launch_attn_tc(D, Q, K, V, wsidx, O, rt, rb, at<int>(ws, L.flag), st));
@@ -116,7 +116,7 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
             int *exitn = at<int>(ws, L.exitn);
             if (D.prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
             int32_t *wsidx = at<int32_t>(ws, L.idx);
-            if (launch_select(D, p->dtype, Q, kbar, amax, exitn, wsidx, st) != cudaSuccess)
+            if (launch_selection(p, D, Q, kbar, amax, exitn, wsidx, at<int>(ws, L.flag), st) != cudaSuccess)
                 return FS_ERR_CUDA;
             sel = wsidx;
         }
@@ -135,6 +135,13 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
 }  // namespace
 
 fs_status validate_params(const fs_params *p) { return validate(p); }
+
+cudaError_t launch_selection(const fs_params *p, const Dev &D, const void *Q, const float *kbar,
+                             const float *amax, const int *exitn, int32_t *idx, int *dev_flag,
+                             cudaStream_t st) {
+    if (select_tc_supported(p)) return launch_select_tc(D, Q, kbar, amax, exitn, idx, dev_flag, st);
+    return launch_select(D, p->dtype, Q, kbar, amax, exitn, idx, st);
+}
 Dev make_dev_params(const fs_params *p) { return make_dev(p); }
 bool params_have_long_range(const fs_params *p) { return has_long_range(p); }
 
@@ -176,7 +183,7 @@ extern "C" fs_status fs_select_topk(const fs_params *p, const void *Q, const flo
     if (!kbar || !amax) return FS_ERR_INVALID_ARG;
     int *exitn = at<int>(ws, L.exitn);
     if (D.prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
-    return cuda_status(launch_select(D, p->dtype, Q, kbar, amax, exitn, idx, st));
+    return cuda_status(launch_selection(p, D, Q, kbar, amax, exitn, idx, at<int>(ws, L.flag), st));
 }
 
 extern "C" fs_status fs_forward(const fs_params *p, const void *Q, const void *K, const void *V,

@@ -264,7 +264,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         }
         if (t == 0) {
             sm.nU = min(total, UMAX);
-            if (total > UMAX) atomicExch(dev_flag, kFlagCheck);
+            if (total > UMAX && dev_flag) atomicExch(dev_flag, kFlagCheck);
         }
         aux_sync();
         uint32_t mw[UMAX / 32] = {0u, 0u, 0u, 0u};

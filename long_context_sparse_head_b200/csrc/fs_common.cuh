@@ -96,7 +96,7 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 // ---- kernel ids for the diagnostics (fs_kernel_times) ----
 enum KernelId : int {
     kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
-    kNumKernels
+    kSelectTc, kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
@@ -129,6 +129,14 @@ cudaError_t launch_rope_table(int w, float rope_base, float2 *rope_t, float2 *ro
 cudaError_t launch_window_tc(const Dev &P, const void *Q, const void *K, const void *V,
                              const float *olr, void *O, const float2 *rope_t, const float2 *rope_b,
                              int *dev_flag, cudaStream_t st);
+// tensor-core selection (bf16): scores against the bf16x3 split of the mean keys
+bool select_tc_supported(const fs_params *p);
+cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, const float *amax,
+                             const int *exitn, int32_t *idx, int *dev_flag, cudaStream_t st);
+// selection with whichever kernel applies (tensor cores for bf16 when supported)
+cudaError_t launch_selection(const fs_params *p, const Dev &D, const void *Q, const float *kbar,
+                             const float *amax, const int *exitn, int32_t *idx, int *dev_flag,
+                             cudaStream_t st);
 // fused tensor-core readout + window + combine (bf16, internally selected cells)
 bool attn_tc_supported(const fs_params *p);
 cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V,

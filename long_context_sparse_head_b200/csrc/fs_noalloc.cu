@@ -62,6 +62,7 @@ extern "C" fs_status fs_select_topk_noalloc(const fs_params *p, const void *Q, c
     // every entry the selection reads is written by this call's exit-time pass first, so
     // nothing in the shared array needs clearing between calls
     if (prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
-    return launch_select(D, p->dtype, Q, kbar, amax, exitn, idx, st) == cudaSuccess ? FS_OK
-                                                                                    : FS_ERR_CUDA;
+    // same kernels as fs_select_topk; with no workspace there is no device error flag
+    return launch_selection(p, D, Q, kbar, amax, exitn, idx, nullptr, st) == cudaSuccess ? FS_OK
+                                                                                          : FS_ERR_CUDA;
 }

@@ -1,0 +1,315 @@
+// Long-range cell selection on the 5th-generation tensor cores (bf16 queries),
+// "FreeSolo" summary §3.3 eqs. (7)-(8):
+//   A_i  = Recent_W(C_i) u TopP_{c in C_i}(a_c)                       (FS-L pruning)
+//   r_ic = q_i.kbar_c / sqrt(d) + lambda_h a_c erf((i - p_c) / (2 sigma_h)),  c in A_i
+//   S_i  = the K cells of A_i with the largest r_ic (ties: lower cell index)
+//
+// One CTA per 128 query rows of a (batch, head).  The rows of a tile have at most five
+// distinct candidate prefixes n (a prefix grows by one cell every s = 32 positions), so
+// U = union of their admitted sets is at most W + P + 10 cells (<= 128 here).  Warps 0-3
+// build U from the TopP exit table (ordered compaction), then stage the fp32 mean keys of
+// U as three bf16 parts hi + mid + lo (the split carries the fp32 mantissa, so the bf16
+// tensor-core products sum to the fp32 dot product up to accumulation rounding), in the
+// 128-byte-swizzled layout of a K-major MMA operand.  One thread issues
+// S = Q (hi + mid + lo)^T (M = 128, N = |U| rounded up to 16) into tensor memory.  Each
+// thread then takes its row's scores, keeps the admitted ones and finds the K-th largest
+// by bisection on order-preserving integer keys whose low 7 bits carry (127 - position):
+// keys are unique, and among scores that agree to 2^-17 relative the lower cell index
+// wins, inside the 1e-4 near-tie tolerance of the selection check.
+#include "tc_common.cuh"
+
+namespace fs {
+
+namespace {
+constexpr int BM = 128, UMAX = 128;
+constexpr int W_TMA = 4, W_MMA = 5, NWARPS = 6, NTHREADS = NWARPS * 32;
+constexpr uint32_t TMEM_COLS = 128;
+constexpr int TILE_BYTES = BM * kD * 2;
+constexpr int kSelBarrier = 1;   // named barrier of the 128 selection threads
+
+struct SelSmem {
+    __nv_bfloat16 q[BM * kD];              // Q tile (NoPE)
+    __nv_bfloat16 kb[3][UMAX * kD];        // kbar of U as hi, mid, lo bf16 parts
+    int ulist[UMAX];
+    float acell[UMAX];                     // a_c of the union cells (prior)
+    uint8_t amask[UMAX];                   // bit g: admitted for prefix n_min + g
+    int warp_cnt[4];
+    int nU;
+    uint64_t q_full, kb_ready, s_full, drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct SelArgs {
+    int Nq, Nk, q0, w, C, K, W, P, H;
+    int prune, has_prior;
+    float scale;
+    float lambda[FS_MAX_HEADS];
+    float inv2sigma[FS_MAX_HEADS];
+};
+
+__device__ __forceinline__ void sel_sync() {
+    asm volatile("bar.sync %0, %1;" ::"n"(kSelBarrier), "n"(128) : "memory");
+}
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+    const uint32_t b = __float_as_uint(f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ void split3(float x, __nv_bfloat16 &hi, __nv_bfloat16 &mid, __nv_bfloat16 &lo) {
+    hi = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(hi);
+    mid = __float2bfloat16_rn(r1);
+    lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+}
+}  // namespace
+
+__global__ void __launch_bounds__(NTHREADS, 2)
+select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const float *__restrict__ kbar,
+                 const float *__restrict__ amax, const int *__restrict__ exitn,
+                 int32_t *__restrict__ idx, int *dev_flag) {
+    extern __shared__ uint8_t smraw[];
+    const uint32_t sbase = tc::smem_u32(smraw);
+    SelSmem &sm = *reinterpret_cast<SelSmem *>(smraw + (((sbase + 1023u) & ~1023u) - sbase));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y, h = bh % A.H;
+    const int r0 = blockIdx.x * BM;
+    const int pb = A.q0 + r0;
+    const int nrows = min(BM, A.Nq - r0);
+    const int n_min = cand_count(pb, A.w, A.C);
+    const int n_max = cand_count(pb + nrows - 1, A.w, A.C);
+    const tc::Abort ab{dev_flag, &sm.abort};
+
+    if (threadIdx.x == 0) {
+        sm.abort = 0;
+        tc::mbar_init(&sm.q_full, 1);
+        tc::mbar_init(&sm.kb_ready, 128);
+        tc::mbar_init(&sm.s_full, 1);
+        tc::mbar_init(&sm.drain, 1);
+        tc::fence_barrier_init();
+    }
+    if (warp == W_MMA) {
+        tc::tmem_alloc(&sm.tmem_base, TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == W_TMA) {
+        if (lane == 0) {
+            tc::prefetch_tmap(&tq);
+            tc::mbar_expect_tx(&sm.q_full, TILE_BYTES);
+            tc::tma_load_3d(sm.q, &tq, &sm.q_full, 0, r0, bh);
+        }
+    } else if (warp == W_MMA) {
+        if (lane == 0) {
+            bool ok = tc::mbar_wait(&sm.kb_ready, 0, ab) && tc::mbar_wait(&sm.q_full, 0, ab);
+            if (ok) {
+                tc::tc_fence_after();
+                const int N = max(16, (sm.nU + 15) & ~15);
+                const uint32_t id = tc::idesc_bf16(BM, N, false, false);
+                const uint32_t qa = tc::smem_u32(sm.q);
+#pragma unroll
+                for (int part = 0; part < 3; part++) {
+                    const uint32_t kb = tc::smem_u32(sm.kb[part]);
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; kk++)
+                        tc::mma_ss(tmem, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
+                                   tc::sdesc_sw128(kb + kk * 32, 16, 1024), id, (part | kk) ? 1u : 0u);
+                }
+                tc::mma_commit(&sm.s_full);
+                tc::mma_commit(&sm.drain);
+                const uint64_t t0 = tc::globaltimer();
+                while (!tc::mbar_try_wait(&sm.drain, 0) && tc::globaltimer() - t0 < tc::kWaitLimitNs) {
+                }
+            }
+        }
+    } else {
+        const int t = threadIdx.x;     // 0..127: union builder, then the row this thread owns
+        // ---- U: ordered union of the admitted sets of the tile's prefixes n_min..n_max
+        const int *ex = exitn + (size_t)bh * A.C;
+        const float *am = amax + (size_t)bh * A.C;
+        const int ng = n_max - n_min;   // <= 4
+        int total = 0;
+        for (int c0 = 0; c0 < n_max; c0 += 128) {
+            const int c = c0 + t;
+            uint32_t amk = 0;
+            if (c < n_max) {
+                const int e = A.prune ? ex[c] : 0;
+#pragma unroll
+                for (int g = 0; g <= 4; g++) {
+                    const int n = n_min + g;
+                    if (g <= ng && c < n && (!A.prune || c >= n - A.W || n < e)) amk |= 1u << g;
+                }
+            }
+            const unsigned m = __ballot_sync(kFull, amk != 0);
+            if (lane == 0) sm.warp_cnt[warp] = __popc(m);
+            sel_sync();
+            int pos = total + __popc(m & ((1u << lane) - 1u)), tot = 0;
+            for (int k = 0; k < 4; k++) {
+                if (k < warp) pos += sm.warp_cnt[k];
+                tot += sm.warp_cnt[k];
+            }
+            if (amk && pos < UMAX) {
+                sm.ulist[pos] = c;
+                sm.amask[pos] = (uint8_t)amk;
+                sm.acell[pos] = am[c];
+            }
+            total += tot;
+            sel_sync();
+        }
+        if (t == 0) {
+            sm.nU = min(total, UMAX);
+            if (total > UMAX && dev_flag) atomicExch(dev_flag, kFlagCheck);
+        }
+        sel_sync();
+        const int nU = min(total, UMAX);
+        // ---- kbar of U as three bf16 parts, row u = union position (zero rows pad to 16)
+        const int N = max(16, (nU + 15) & ~15);
+        if (t < N) {
+            const float4 *src = reinterpret_cast<const float4 *>(kbar + ((size_t)bh * A.C + (t < nU ? sm.ulist[t] : 0)) * kD);
+#pragma unroll
+            for (int j = 0; j < 8; j++) {            // 16-byte chunk j = elements 8j..8j+7
+                float x[8];
+                if (t < nU) {
+                    const float4 a = __ldg(src + 2 * j), b = __ldg(src + 2 * j + 1);
+                    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; e++) x[e] = 0.f;
+                }
+                __align__(16) __nv_bfloat16 hi[8], mi[8], lo[8];
+#pragma unroll
+                for (int e = 0; e < 8; e++) split3(x[e], hi[e], mi[e], lo[e]);
+                const int off = t * kD + ((j ^ (t & 7)) << 3);
+                *reinterpret_cast<uint4 *>(&sm.kb[0][off]) = *reinterpret_cast<const uint4 *>(hi);
+                *reinterpret_cast<uint4 *>(&sm.kb[1][off]) = *reinterpret_cast<const uint4 *>(mi);
+                *reinterpret_cast<uint4 *>(&sm.kb[2][off]) = *reinterpret_cast<const uint4 *>(lo);
+            }
+        }
+        tc::fence_async_shared();
+        tc::mbar_arrive(&sm.kb_ready);
+
+        // ---- this thread's row: scores -> admitted keys -> K best
+        const int row = t;
+        const int i = pb + row;
+        const int n_r = cand_count(i, A.w, A.C);
+        const int g = n_r - n_min;
+        if (!tc::mbar_wait(&sm.s_full, 0, ab)) goto done;
+        {
+            tc::tc_fence_after();
+            const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+            const float lam = A.has_prior ? A.lambda[h] : 0.f;
+            const float i2s = A.inv2sigma[h];
+            uint32_t key[UMAX];
+            uint32_t kmin = 0xffffffffu, kmax = 0u;
+            int na = 0;
+#pragma unroll
+            for (int b = 0; b < UMAX / 32; b++) {
+                if (32 * b < N) {
+                    uint32_t r[32];
+                    tc::tmem_ld32(trow + 32 * b, r);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; e++) {
+                        const int u = 32 * b + e;
+                        uint32_t k = 0u;
+                        if (u < nU && ((sm.amask[u] >> g) & 1u) && row < nrows) {
+                            float sc = __uint_as_float(r[e]) * A.scale;
+                            if (lam != 0.f) {
+                                const float pc = (float)(sm.ulist[u] * kS) + 0.5f * kS;
+                                sc += lam * sm.acell[u] * erff(((float)i - pc) * i2s);
+                            }
+                            k = (order_key(sc) & ~0x7fu) | (uint32_t)(127 - u);
+                            kmin = min(kmin, k);
+                            kmax = max(kmax, k);
+                            na++;
+                        }
+                        key[u] = k;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; e++) key[32 * b + e] = 0u;
+                }
+            }
+            // K-th largest key: count(key >= lo) >= K > count(key >= hi)
+            uint32_t tau = 1u;
+            if (na > A.K) {
+                uint32_t lo = kmin, hi = kmax + 1u;       // count(>= kmin) = na > K, count(>= kmax+1) = 0
+                while (hi - lo > 1u) {
+                    const uint32_t mid = lo + ((hi - lo) >> 1);
+                    int cnt = 0;
+#pragma unroll
+                    for (int b = 0; b < UMAX / 32; b++)
+                        if (32 * b < N) {
+#pragma unroll
+                            for (int e = 0; e < 32; e++) cnt += key[32 * b + e] >= mid;
+                        }
+                    if (cnt >= A.K) {
+                        lo = mid;
+                        if (cnt == A.K) break;
+                    } else {
+                        hi = mid;
+                    }
+                }
+                tau = lo;
+            }
+            if (row < nrows) {
+                int32_t *out = idx + ((size_t)bh * A.Nq + r0 + row) * A.K;
+                int o = 0;
+#pragma unroll
+                for (int b = 0; b < UMAX / 32; b++)
+                    if (32 * b < N) {
+#pragma unroll
+                        for (int e = 0; e < 32; e++) {
+                            const int u = 32 * b + e;
+                            if (key[u] >= tau && key[u] != 0u && o < A.K) out[o++] = sm.ulist[u];
+                        }
+                    }
+                for (; o < A.K; o++) out[o] = -1;
+            }
+        }
+    done:;
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == W_MMA) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+bool select_tc_supported(const fs_params *p) {
+    if (p->dtype != FS_BF16) return false;
+    const int C = p->Nk / p->s;
+    const int bound = p->W >= 0 ? p->W + p->P + 10 : C;
+    return bound <= UMAX;
+}
+
+cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, const float *amax,
+                             const int *exitn, int32_t *idx, int *dev_flag, cudaStream_t st) {
+    if (P.Nq == 0) return cudaSuccess;
+    const int BH = P.B * P.H;
+    CUtensorMap tq;
+    if (!encode_tmap_3d_bf16(&tq, Q, kD, P.Nq, BH, kD, BM)) return cudaErrorInvalidValue;
+    SelArgs A;
+    A.Nq = P.Nq; A.Nk = P.Nk; A.q0 = P.q0; A.w = P.w; A.C = P.C; A.K = P.K;
+    A.W = P.W; A.P = P.P; A.H = P.H; A.prune = P.prune; A.has_prior = P.has_prior;
+    A.scale = P.scale;
+    for (int h = 0; h < FS_MAX_HEADS; h++) {
+        A.lambda[h] = P.lambda[h];
+        A.inv2sigma[h] = P.inv2sigma[h];
+    }
+    const size_t smem = sizeof(SelSmem) + 1024;
+    const dim3 grid((P.Nq + BM - 1) / BM, BH);
+    LaunchScope scope(kSelectTc, st);
+    cudaFuncSetAttribute(select_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    select_tc_kernel<<<grid, NTHREADS, smem, st>>>(tq, A, kbar, amax, exitn, idx, dev_flag);
+    return cudaGetLastError();
+}
+
+}  // namespace fs

@@ -55,7 +55,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
 struct Abort {
-    int *dev_flag;        // device error flag (first int of the workspace)
+    int *dev_flag;        // device error flag (first int of the workspace), or null
     volatile int *cta;    // shared abort word
 };
 
@@ -67,7 +67,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
         if (*ab.cta) return false;
         if (globaltimer() - t0 > kWaitLimitNs) {
             *ab.cta = 1;
-            atomicExch(ab.dev_flag, kFlagTimeout);
+            if (ab.dev_flag) atomicExch(ab.dev_flag, kFlagTimeout);
             return false;
         }
     }
