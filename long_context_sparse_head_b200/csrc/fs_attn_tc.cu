@@ -10,14 +10,17 @@
 // U, the union of the cells the tile's rows selected (|U| <= 128, ascending), four cells
 // (128 keys) per chunk, each cell fetched by its own 32-row TMA box; a row masks the
 // cells it did not select (masked-dense on the tensor cores).  Then the window runs
-// over 128-key chunks as in the window-only kernel.  Both softmaxes accumulate in tensor
-// memory: S/P in columns [0,128), the readout's O in [128,192), the window's O in
-// [192,256).  When the first window chunk arrives, the readout is finished: the softmax
-// threads turn its O into alpha_h * RMSNorm(u) in place; the epilogue adds it to the
-// window's output.  No intermediate leaves the SM.
+// over 128-key chunks.  Both softmaxes accumulate in tensor memory: S/P in columns
+// [0,128), the readout's O in [128,192), the window's O in [192,256).  When the first
+// window chunk arrives the readout is finished: the softmax threads turn its O into
+// alpha_h * RMSNorm(u) in place, and the epilogue adds it to the window's output.  No
+// intermediate leaves the SM.
 //
-// Warps: 0-3 softmax (thread = query row = TMEM lane), 4 TMA, 5 MMA, 6-9 auxiliary
-// (build U and the per-row selection masks from idx, rotate Q and the window's K chunks).
+// Warpgroup 0 (warps 0-3): softmax, thread = query row = TMEM lane; it holds a chunk's
+// whole 128-column S row in registers (one TMEM wait per chunk), raised to 200 registers
+// by setmaxnreg.  Warpgroup 1 (lowered to 56): warp 4 TMA, warp 5 MMA, warps 6-7
+// auxiliary (build U and the per-row selection masks from idx, rotate Q and the window's
+// K chunks).
 #include "tc_rope.cuh"
 
 namespace fs {
@@ -26,12 +29,13 @@ namespace {
 constexpr int BM = 128, BN = 128, NSTAGE = 2;
 constexpr int UMAX = 128;                        // largest union of selected cells per tile
 constexpr int CPC = BN / kS;                     // cells per readout chunk (4)
-constexpr int W_TMA = 4, W_MMA = 5, W_AUX0 = 6, NWARPS = 10;
+constexpr int W_TMA = 4, W_MMA = 5, W_AUX0 = 6, NWARPS = 8, NAUX = 64;
 constexpr int NTHREADS = NWARPS * 32;
+constexpr int REGS_SOFTMAX = 200, REGS_PRODUCER = 56;   // 128 * (200 + 56) = 256 * 128
 constexpr uint32_t TMEM_COLS = 256, S_COL = 0, OLR_COL = 128, OSR_COL = 192;
 constexpr int TILE_BYTES = BM * kD * 2;         // 128 x 64 bf16: 16 KiB
 constexpr int CELL_BYTES = kS * kD * 2;         // 32 x 64 bf16: 4 KiB
-constexpr int kAuxBarrier = 1;                  // named barrier of the 128 auxiliary threads
+constexpr int kAuxBarrier = 1;                  // named barrier of the auxiliary threads
 
 struct AttnSmem {
     __nv_bfloat16 qn[BM * kD];                  // Q as loaded (NoPE)
@@ -41,7 +45,7 @@ struct AttnSmem {
     uint32_t mask[BM][UMAX / 32];               // row -> selected union positions
     int ulist[UMAX];                            // union cells, ascending
     int nU;
-    int warp_tot[4];
+    int warp_tot[NAUX / 32];
     uint64_t q_full, q_ready, u_ready, s_full, p_full, o_done, drain;
     uint64_t kv_full[NSTAGE], k_ready[NSTAGE], kv_empty[NSTAGE];
     uint32_t tmem_base;
@@ -56,39 +60,60 @@ struct AttnArgs {
 };
 
 __device__ __forceinline__ void aux_sync() {
-    asm volatile("bar.sync %0, %1;" ::"n"(kAuxBarrier), "n"(128) : "memory");
+    asm volatile("bar.sync %0, %1;" ::"n"(kAuxBarrier), "n"(NAUX) : "memory");
+}
+
+__device__ __forceinline__ void ld_row128(uint32_t taddr, uint32_t (&s)[128]) {
+    tc::tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+    tc::tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+    tc::tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+    tc::tmem_ld32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+    tc::tmem_wait_ld();
 }
 
 // One chunk of online softmax for this thread's row.  S is read from TMEM columns
-// [S_COL, S_COL+128); P = exp2(S*c - m) is written as bf16 pairs over [S_COL, S_COL+64).
-// Readout chunks (MASKED_CELLS): 32-column block b is valid iff bit b of sel4 is set.
-// Window chunks: column c is valid iff clo <= c <= chi.
+// [S_COL, S_COL+128) in one batch; P = exp2(S*c - m) is written back as bf16 pairs over
+// [S_COL, S_COL+64).  Readout chunks (MASKED_CELLS): 32-column block b is valid iff bit b
+// of sel4 is set.  Window chunks: column j is valid iff clo <= j <= chi.  The running max
+// m (log2 units) is raised only when a chunk exceeds it by more than 8 (lazy rescale of O).
 template <bool MASKED_CELLS>
 __device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, bool first, uint32_t sel4,
                                               int clo, int chi, float c_log2, float &m_used, float &l) {
-    auto col_ok = [&](int c) -> bool {
-        if (MASKED_CELLS) return ((sel4 >> (c >> 5)) & 1u) != 0;
-        return c >= clo && c <= chi;
-    };
-    auto blk_any = [&](int b) -> bool {
-        if (MASKED_CELLS) return ((sel4 >> b) & 1u) != 0;
-        return clo <= chi && clo <= 32 * b + 31 && chi >= 32 * b;
+    uint32_t s[128];
+    ld_row128(trow + S_COL, s);
+    const bool full = MASKED_CELLS ? false : __all_sync(kFull, clo <= 0 && chi >= BN - 1);
+    auto ok = [&](int j) -> bool {
+        if (MASKED_CELLS) return ((sel4 >> (j >> 5)) & 1u) != 0;
+        return full || (j >= clo && j <= chi);
     };
     float mx = -INFINITY;
 #pragma unroll
-    for (int b = 0; b < BN / 32; b++) {
-        if (!__any_sync(kFull, blk_any(b))) continue;
-        uint32_t r[32];
-        tc::tmem_ld32(trow + S_COL + 32 * b, r);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e++)
-            if (col_ok(32 * b + e)) mx = fmaxf(mx, __uint_as_float(r[e]));
-    }
+    for (int j = 0; j < BN; j++)
+        if (ok(j)) mx = fmaxf(mx, __uint_as_float(s[j]));
     mx *= c_log2;
-    const bool grow = mx > m_used + 8.f;               // lazy rescale: only past 2^8
+    const bool grow = mx > m_used + 8.f;
     const float m_new = grow ? mx : m_used;
     const float corr = (grow && m_used != -INFINITY) ? tc::ex2(m_used - m_new) : 1.f;
+    l *= corr;
+    m_used = m_new;
+    const float msub = m_used == -INFINITY ? 0.f : m_used;
+#pragma unroll
+    for (int q = 0; q < 4; q++) {                    // P keys [32 q, 32 q + 32) -> 16 columns
+        uint32_t pk[16];
+        float lsum = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; e++) {
+            const int j = 32 * q + 2 * e;
+            const float p0 = ok(j) ? tc::ex2(fmaf(__uint_as_float(s[j]), c_log2, -msub)) : 0.f;
+            const float p1 = ok(j + 1) ? tc::ex2(fmaf(__uint_as_float(s[j + 1]), c_log2, -msub)) : 0.f;
+            lsum += p0 + p1;
+            pk[e] = tc::pack_bf16x2(p0, p1);
+        }
+        l += lsum;
+        tc::tmem_st16(trow + S_COL + 16 * q, pk);
+    }
+    // O rescale after the exponentials, when S no longer occupies registers (no MMA
+    // touches O until this thread arrives on p_full)
     if (!first && __any_sync(kFull, corr != 1.f)) {
 #pragma unroll
         for (int b = 0; b < kD / 32; b++) {
@@ -99,35 +124,6 @@ __device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, boo
             for (int e = 0; e < 32; e++) r[e] = __float_as_uint(__uint_as_float(r[e]) * corr);
             tc::tmem_st32(trow + o_col + 32 * b, r);
         }
-        tc::tmem_wait_st();
-    }
-    l *= corr;
-    m_used = m_new;
-    const float msub = m_used == -INFINITY ? 0.f : m_used;
-#pragma unroll
-    for (int h2 = 0; h2 < 2; h2++) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int hb = 0; hb < 2; hb++) {
-            const int b = 2 * h2 + hb;
-            if (!__any_sync(kFull, blk_any(b))) {
-#pragma unroll
-                for (int e = 0; e < 16; e++) pk[16 * hb + e] = 0u;
-                continue;
-            }
-            uint32_t r[32];
-            tc::tmem_ld32(trow + S_COL + 32 * b, r);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; e++) {
-                const int c0 = 32 * b + 2 * e;
-                const float p0 = col_ok(c0) ? tc::ex2(__uint_as_float(r[2 * e]) * c_log2 - msub) : 0.f;
-                const float p1 = col_ok(c0 + 1) ? tc::ex2(__uint_as_float(r[2 * e + 1]) * c_log2 - msub) : 0.f;
-                l += p0 + p1;
-                pk[16 * hb + e] = tc::pack_bf16x2(p0, p1);
-            }
-        }
-        tc::tmem_st32(trow + S_COL + 32 * h2, pk);
     }
     tc::tmem_wait_st();
 }
@@ -156,15 +152,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     if (threadIdx.x == 0) {
         sm.abort = 0;
         tc::mbar_init(&sm.q_full, 1);
-        tc::mbar_init(&sm.q_ready, 128);
-        tc::mbar_init(&sm.u_ready, 128);
+        tc::mbar_init(&sm.q_ready, NAUX);
+        tc::mbar_init(&sm.u_ready, NAUX);
         tc::mbar_init(&sm.s_full, 1);
         tc::mbar_init(&sm.p_full, 128);
         tc::mbar_init(&sm.o_done, 1);
         tc::mbar_init(&sm.drain, 1);
         for (int s = 0; s < NSTAGE; s++) {
             tc::mbar_init(&sm.kv_full[s], 1);
-            tc::mbar_init(&sm.k_ready[s], 128);
+            tc::mbar_init(&sm.k_ready[s], NAUX);
             tc::mbar_init(&sm.kv_empty[s], 1);
         }
         tc::fence_barrier_init();
@@ -178,175 +174,184 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == W_TMA) {
-        if (lane == 0) {
-            tc::prefetch_tmap(&tq);
-            tc::prefetch_tmap(&tk32);
-            tc::prefetch_tmap(&tv32);
-            tc::prefetch_tmap(&tk128);
-            tc::prefetch_tmap(&tv128);
-            tc::mbar_expect_tx(&sm.q_full, TILE_BYTES);
-            tc::tma_load_3d(sm.qn, &tq, &sm.q_full, 0, r0, bh);
-            int it = 0;
-            if (tc::mbar_wait(&sm.u_ready, 0, ab)) {
-                const int nU = sm.nU, nR = (nU + CPC - 1) / CPC, total = nR + nW;
-                for (; it < total; it++) {
-                    const int s = it % NSTAGE;
-                    if (!tc::mbar_wait(&sm.kv_empty[s], ((it / NSTAGE) & 1) ^ 1, ab)) break;
-                    if (it < nR) {          // four gathered cells; unused slots read zeros
-                        tc::mbar_expect_tx(&sm.kv_full[s], 2 * CPC * CELL_BYTES);
-                        for (int j = 0; j < CPC; j++) {
-                            const int u = CPC * it + j;
-                            const int y = u < nU ? sm.ulist[u] * kS : A.Nk;   // past the end: zero fill
-                            tc::tma_load_3d(sm.k[s] + j * kS * kD, &tk32, &sm.kv_full[s], 0, y, bh);
-                            tc::tma_load_3d(sm.v[s] + j * kS * kD, &tv32, &sm.kv_full[s], 0, y, bh);
+    if (warp >= 4) {
+        tc::regs_dec<REGS_PRODUCER>();
+        if (warp == W_TMA) {
+            if (lane == 0) {
+                tc::prefetch_tmap(&tq);
+                tc::prefetch_tmap(&tk32);
+                tc::prefetch_tmap(&tv32);
+                tc::prefetch_tmap(&tk128);
+                tc::prefetch_tmap(&tv128);
+                tc::mbar_expect_tx(&sm.q_full, TILE_BYTES);
+                tc::tma_load_3d(sm.qn, &tq, &sm.q_full, 0, r0, bh);
+                int it = 0;
+                if (tc::mbar_wait(&sm.u_ready, 0, ab)) {
+                    const int nU = sm.nU, nR = (nU + CPC - 1) / CPC, total = nR + nW;
+                    for (; it < total; it++) {
+                        const int s = it % NSTAGE;
+                        if (!tc::mbar_wait(&sm.kv_empty[s], ((it / NSTAGE) & 1) ^ 1, ab)) break;
+                        if (it < nR) {          // four gathered cells; unused slots read zeros
+                            tc::mbar_expect_tx(&sm.kv_full[s], 2 * CPC * CELL_BYTES);
+                            for (int j = 0; j < CPC; j++) {
+                                const int u = CPC * it + j;
+                                const int y = u < nU ? sm.ulist[u] * kS : A.Nk;   // past the end: zeros
+                                tc::tma_load_3d(sm.k[s] + j * kS * kD, &tk32, &sm.kv_full[s], 0, y, bh);
+                                tc::tma_load_3d(sm.v[s] + j * kS * kD, &tv32, &sm.kv_full[s], 0, y, bh);
+                            }
+                        } else {                // 128 consecutive keys of the band
+                            const int jc = jbase + BN * (k_first + it - nR);
+                            tc::mbar_expect_tx(&sm.kv_full[s], 2 * TILE_BYTES);
+                            tc::tma_load_3d(sm.k[s], &tk128, &sm.kv_full[s], 0, jc, bh);
+                            tc::tma_load_3d(sm.v[s], &tv128, &sm.kv_full[s], 0, jc, bh);
                         }
-                    } else {                // 128 consecutive keys of the band
-                        const int jc = jbase + BN * (k_first + it - nR);
-                        tc::mbar_expect_tx(&sm.kv_full[s], 2 * TILE_BYTES);
-                        tc::tma_load_3d(sm.k[s], &tk128, &sm.kv_full[s], 0, jc, bh);
-                        tc::tma_load_3d(sm.v[s], &tv128, &sm.kv_full[s], 0, jc, bh);
+                    }
+                }
+                if (sm.abort) {   // let issued copies land before the CTA's memory is released
+                    for (int j = max(0, it - NSTAGE); j < it; j++) {
+                        const uint64_t t0 = tc::globaltimer();
+                        while (!tc::mbar_try_wait(&sm.kv_full[j % NSTAGE], (j / NSTAGE) & 1) &&
+                               tc::globaltimer() - t0 < tc::kWaitLimitNs) {
+                        }
                     }
                 }
             }
-            if (sm.abort) {   // let issued copies land before the CTA's memory is released
-                for (int j = max(0, it - NSTAGE); j < it; j++) {
-                    const uint64_t t0 = tc::globaltimer();
-                    while (!tc::mbar_try_wait(&sm.kv_full[j % NSTAGE], (j / NSTAGE) & 1) &&
-                           tc::globaltimer() - t0 < tc::kWaitLimitNs) {
+        } else if (warp >= W_AUX0) {
+            const int t = threadIdx.x - W_AUX0 * 32, aw = t >> 5;
+            // ---- U: union of the rows' selected cells, via a bitmap over [0, C) that lives
+            //      in the (not yet loaded) K/V stages, plus a cell -> position byte table
+            uint32_t *bitmap = reinterpret_cast<uint32_t *>(&sm.k[0][0]);
+            uint8_t *cpos = reinterpret_cast<uint8_t *>(&sm.v[0][0]);
+            const int nwords = (A.C + 31) / 32;
+            for (int wd = t; wd < nwords; wd += NAUX) bitmap[wd] = 0u;
+            aux_sync();
+            for (int rr = t; rr < nrows; rr += NAUX) {
+                const int32_t *ri = idx + ((size_t)bh * A.Nq + r0 + rr) * A.K;
+                for (int e = 0; e < A.K; e++) {
+                    const int c = ri[e];
+                    if (c >= 0 && c < A.C) atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+                }
+            }
+            aux_sync();
+            const int R = (nwords + NAUX - 1) / NAUX, w0 = min(t * R, nwords), w1 = min(w0 + R, nwords);
+            int cnt = 0;
+            for (int wd = w0; wd < w1; wd++) cnt += __popc(bitmap[wd]);
+            int incl = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (lane == 31) sm.warp_tot[aw] = incl;
+            aux_sync();
+            int pos = incl - cnt, total = 0;
+            for (int k = 0; k < NAUX / 32; k++) {
+                if (k < aw) pos += sm.warp_tot[k];
+                total += sm.warp_tot[k];
+            }
+            for (int wd = w0; wd < w1; wd++) {
+                uint32_t bits = bitmap[wd];
+                while (bits) {
+                    const int c = wd * 32 + __ffs(bits) - 1;
+                    bits &= bits - 1;
+                    if (pos < UMAX) {
+                        sm.ulist[pos] = c;
+                        cpos[c] = (uint8_t)pos;
+                    }
+                    pos++;
+                }
+            }
+            if (t == 0) {
+                sm.nU = min(total, UMAX);
+                if (total > UMAX && dev_flag) atomicExch(dev_flag, kFlagCheck);
+            }
+            aux_sync();
+            for (int rr = t; rr < BM; rr += NAUX) {
+                uint32_t mw[UMAX / 32] = {0u, 0u, 0u, 0u};
+                if (rr < nrows) {
+                    const int32_t *ri = idx + ((size_t)bh * A.Nq + r0 + rr) * A.K;
+                    for (int e = 0; e < A.K; e++) {
+                        const int c = ri[e];
+                        if (c >= 0 && c < A.C) {
+                            const int p = cpos[c];
+                            if (p < UMAX) mw[p >> 5] |= 1u << (p & 31);
+                        }
                     }
                 }
-            }
-        }
-    } else if (warp >= W_AUX0) {
-        const int t = threadIdx.x - W_AUX0 * 32, aw = t >> 5;
-        // ---- U: union of the rows' selected cells, via a bitmap over [0, C) that lives
-        //      in the (not yet loaded) K/V stages, plus a cell -> position byte table
-        uint32_t *bitmap = reinterpret_cast<uint32_t *>(&sm.k[0][0]);
-        uint8_t *cpos = reinterpret_cast<uint8_t *>(&sm.v[0][0]);
-        const int nwords = (A.C + 31) / 32;
-        for (int wd = t; wd < nwords; wd += 128) bitmap[wd] = 0u;
-        aux_sync();
-        const int32_t *myidx = idx + ((size_t)bh * A.Nq + r0 + t) * A.K;
-        if (t < nrows)
-            for (int e = 0; e < A.K; e++) {
-                const int c = myidx[e];
-                if (c >= 0 && c < A.C) atomicOr(&bitmap[c >> 5], 1u << (c & 31));
-            }
-        aux_sync();
-        const int R = (nwords + 127) / 128, w0 = min(t * R, nwords), w1 = min(w0 + R, nwords);
-        int cnt = 0;
-        for (int wd = w0; wd < w1; wd++) cnt += __popc(bitmap[wd]);
-        int incl = cnt;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl += y;
-        }
-        if (lane == 31) sm.warp_tot[aw] = incl;
-        aux_sync();
-        int pos = incl - cnt, total = 0;
-        for (int k = 0; k < 4; k++) {
-            if (k < aw) pos += sm.warp_tot[k];
-            total += sm.warp_tot[k];
-        }
-        for (int wd = w0; wd < w1; wd++) {
-            uint32_t bits = bitmap[wd];
-            while (bits) {
-                const int c = wd * 32 + __ffs(bits) - 1;
-                bits &= bits - 1;
-                if (pos < UMAX) {
-                    sm.ulist[pos] = c;
-                    cpos[c] = (uint8_t)pos;
-                }
-                pos++;
+                for (int k = 0; k < UMAX / 32; k++) sm.mask[rr][k] = mw[k];
             }
-        }
-        if (t == 0) {
-            sm.nU = min(total, UMAX);
-            if (total > UMAX && dev_flag) atomicExch(dev_flag, kFlagCheck);
-        }
-        aux_sync();
-        uint32_t mw[UMAX / 32] = {0u, 0u, 0u, 0u};
-        if (t < nrows)
-            for (int e = 0; e < A.K; e++) {
-                const int c = myidx[e];
-                if (c >= 0 && c < A.C) {
-                    const int p = cpos[c];
-                    if (p < UMAX) mw[p >> 5] |= 1u << (p & 31);
-                }
-            }
-#pragma unroll
-        for (int k = 0; k < UMAX / 32; k++) sm.mask[t][k] = mw[k];
-        aux_sync();                       // scratch reads done before the stages are loaded
-        tc::fence_async_shared();
-        tc::mbar_arrive(&sm.u_ready);
-        const int nR = (sm.nU + CPC - 1) / CPC, total_ck = nR + nW;
-        // ---- rotate Q for the window, then pass through (readout) or rotate (window) K
-        if (tc::mbar_wait(&sm.q_full, 0, ab)) {
-            tc::rotate_tile(sm.qn, sm.qr, t, rope_t, nullptr);
+            aux_sync();                       // scratch reads done before the stages are loaded
             tc::fence_async_shared();
-            tc::mbar_arrive(&sm.q_ready);
-            for (int it = 0; it < total_ck; it++) {
-                const int s = it % NSTAGE;
-                if (!tc::mbar_wait(&sm.kv_full[s], (it / NSTAGE) & 1, ab)) break;
-                if (it >= nR) {
-                    tc::rotate_tile(sm.k[s], sm.k[s], t, rope_t,
-                                    rope_b + (size_t)(k_first + it - nR) * 32);
-                    tc::fence_async_shared();
-                }
-                tc::mbar_arrive(&sm.k_ready[s]);
-            }
-        }
-    } else if (warp == W_MMA) {
-        if (lane == 0) {
-            const uint32_t id_qk = tc::idesc_bf16(BM, BN, false, false);
-            const uint32_t id_pv = tc::idesc_bf16(BM, kD, false, true);
-            const uint32_t qn = tc::smem_u32(sm.qn), qr = tc::smem_u32(sm.qr);
-            bool ok = tc::mbar_wait(&sm.u_ready, 0, ab) && tc::mbar_wait(&sm.q_full, 0, ab);
-            const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0, total = nR + nW;
-            int issued = 0;
-            for (int it = 0; ok && it <= total; it++) {
-                if (it < total && !tc::mbar_wait(&sm.k_ready[it % NSTAGE], (it / NSTAGE) & 1, ab)) {
-                    ok = false;
-                    break;
-                }
-                if (it > 0) {   // O += P(it-1) V(it-1), into the readout's or the window's O
-                    if (!tc::mbar_wait(&sm.p_full, (it - 1) & 1, ab)) { ok = false; break; }
-                    tc::tc_fence_after();
-                    const int pj = it - 1;
-                    const uint32_t ocol = pj < nR ? OLR_COL : OSR_COL;
-                    const bool first = pj == 0 || pj == nR;
-                    const uint32_t vb = tc::smem_u32(sm.v[pj % NSTAGE]);
-#pragma unroll
-                    for (int kk = 0; kk < BN / 16; kk++)
-                        tc::mma_ts(tmem + ocol, tmem + S_COL + kk * 8, tc::sdesc_sw128(vb + kk * 2048, 16, 1024),
-                                   id_pv, (!first || kk > 0) ? 1u : 0u);
-                    tc::mma_commit(&sm.kv_empty[pj % NSTAGE]);
-                    issued++;
-                }
-                if (it < total) {   // S = Q K(it)^T with the NoPE or the rotated Q
-                    if (it == nR && !tc::mbar_wait(&sm.q_ready, 0, ab)) { ok = false; break; }
-                    tc::tc_fence_after();
-                    const uint32_t qa = it < nR ? qn : qr;
-                    const uint32_t kb = tc::smem_u32(sm.k[it % NSTAGE]);
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; kk++)
-                        tc::mma_ss(tmem + S_COL, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
-                                   tc::sdesc_sw128(kb + kk * 32, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
-                    tc::mma_commit(&sm.s_full);
-                    issued++;
+            tc::mbar_arrive(&sm.u_ready);
+            const int nR = (sm.nU + CPC - 1) / CPC, total_ck = nR + nW;
+            // ---- rotate Q for the window, then pass through (readout) or rotate (window) K
+            if (tc::mbar_wait(&sm.q_full, 0, ab)) {
+                tc::rotate_tile<NAUX>(sm.qn, sm.qr, t, rope_t, nullptr);
+                tc::fence_async_shared();
+                tc::mbar_arrive(&sm.q_ready);
+                for (int it = 0; it < total_ck; it++) {
+                    const int s = it % NSTAGE;
+                    if (!tc::mbar_wait(&sm.kv_full[s], (it / NSTAGE) & 1, ab)) break;
+                    if (it >= nR) {
+                        tc::rotate_tile<NAUX>(sm.k[s], sm.k[s], t, rope_t,
+                                              rope_b + (size_t)(k_first + it - nR) * 32);
+                        tc::fence_async_shared();
+                    }
+                    tc::mbar_arrive(&sm.k_ready[s]);
                 }
             }
-            if (ok) tc::mma_commit(&sm.o_done);
-            if (issued) {
-                tc::mma_commit(&sm.drain);
-                const uint64_t t0 = tc::globaltimer();
-                while (!tc::mbar_try_wait(&sm.drain, 0) && tc::globaltimer() - t0 < tc::kWaitLimitNs) {
+        } else if (warp == W_MMA) {
+            if (lane == 0) {
+                const uint32_t id_qk = tc::idesc_bf16(BM, BN, false, false);
+                const uint32_t id_pv = tc::idesc_bf16(BM, kD, false, true);
+                const uint32_t qn = tc::smem_u32(sm.qn), qr = tc::smem_u32(sm.qr);
+                bool ok = tc::mbar_wait(&sm.u_ready, 0, ab) && tc::mbar_wait(&sm.q_full, 0, ab);
+                const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0, total = nR + nW;
+                int issued = 0;
+                for (int it = 0; ok && it <= total; it++) {
+                    if (it < total && !tc::mbar_wait(&sm.k_ready[it % NSTAGE], (it / NSTAGE) & 1, ab)) {
+                        ok = false;
+                        break;
+                    }
+                    if (it > 0) {   // O += P(it-1) V(it-1), into the readout's or the window's O
+                        if (!tc::mbar_wait(&sm.p_full, (it - 1) & 1, ab)) { ok = false; break; }
+                        tc::tc_fence_after();
+                        const int pj = it - 1;
+                        const uint32_t ocol = pj < nR ? OLR_COL : OSR_COL;
+                        const bool first = pj == 0 || pj == nR;
+                        const uint32_t vb = tc::smem_u32(sm.v[pj % NSTAGE]);
+#pragma unroll
+                        for (int kk = 0; kk < BN / 16; kk++)
+                            tc::mma_ts(tmem + ocol, tmem + S_COL + kk * 8, tc::sdesc_sw128(vb + kk * 2048, 16, 1024),
+                                       id_pv, (!first || kk > 0) ? 1u : 0u);
+                        tc::mma_commit(&sm.kv_empty[pj % NSTAGE]);
+                        issued++;
+                    }
+                    if (it < total) {   // S = Q K(it)^T with the NoPE or the rotated Q
+                        if (it == nR && !tc::mbar_wait(&sm.q_ready, 0, ab)) { ok = false; break; }
+                        tc::tc_fence_after();
+                        const uint32_t qa = it < nR ? qn : qr;
+                        const uint32_t kb = tc::smem_u32(sm.k[it % NSTAGE]);
+#pragma unroll
+                        for (int kk = 0; kk < kD / 16; kk++)
+                            tc::mma_ss(tmem + S_COL, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
+                                       tc::sdesc_sw128(kb + kk * 32, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
+                        tc::mma_commit(&sm.s_full);
+                        issued++;
+                    }
+                }
+                if (ok) tc::mma_commit(&sm.o_done);
+                if (issued) {
+                    tc::mma_commit(&sm.drain);
+                    const uint64_t t0 = tc::globaltimer();
+                    while (!tc::mbar_try_wait(&sm.drain, 0) && tc::globaltimer() - t0 < tc::kWaitLimitNs) {
+                    }
                 }
             }
         }
     } else {
+        tc::regs_inc<REGS_SOFTMAX>();
         // ---- softmax: thread = query row
         const int row = warp * 32 + lane;
         const int i = pb + row;
@@ -386,7 +391,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     }
                     tc::tmem_st32(trow + OLR_COL, a);
                     tc::tmem_st32(trow + OLR_COL + 32, b);
-                    tc::tmem_wait_st();
                 }
                 const int jc = jbase + BN * (k_first + it - nR);
                 int clo = max(-jc, i - A.w - jc), chi = min(i - jc, BN - 1);
@@ -400,27 +404,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             tc::tc_fence_after();
             const size_t orow = ((size_t)bh * A.Nq + r0 + row) * kD;
             const float inv = l_sr > 0.f ? 1.f / l_sr : 0.f;
+            uint32_t a[64], b[64];
+            tc::tmem_ld32(trow + OSR_COL, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+            tc::tmem_ld32(trow + OSR_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+            if (nR > 0) {
+                tc::tmem_ld32(trow + OLR_COL, *reinterpret_cast<uint32_t(*)[32]>(&b[0]));
+                tc::tmem_ld32(trow + OLR_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&b[32]));
+            }
+            tc::tmem_wait_ld();
+            if (rvalid) {
+                uint4 *dst = reinterpret_cast<uint4 *>(O + orow);
 #pragma unroll
-            for (int hf = 0; hf < 2; hf++) {
-                uint32_t a[32], b[32];
-                tc::tmem_ld32(trow + OSR_COL + 32 * hf, a);
-                if (nR > 0) tc::tmem_ld32(trow + OLR_COL + 32 * hf, b);
-                tc::tmem_wait_ld();
-                uint32_t outw[16];
+                for (int q = 0; q < 8; q++) {
+                    uint32_t w4[4];
 #pragma unroll
-                for (int e = 0; e < 16; e++) {
-                    float o0 = __uint_as_float(a[2 * e]) * inv, o1 = __uint_as_float(a[2 * e + 1]) * inv;
-                    if (nR > 0) {
-                        o0 += __uint_as_float(b[2 * e]);
-                        o1 += __uint_as_float(b[2 * e + 1]);
+                    for (int e = 0; e < 4; e++) {
+                        const int j = 8 * q + 2 * e;
+                        float o0 = __uint_as_float(a[j]) * inv, o1 = __uint_as_float(a[j + 1]) * inv;
+                        if (nR > 0) {
+                            o0 += __uint_as_float(b[j]);
+                            o1 += __uint_as_float(b[j + 1]);
+                        }
+                        w4[e] = tc::pack_bf16x2(o0, o1);
                     }
-                    outw[e] = tc::pack_bf16x2(o0, o1);
-                }
-                if (rvalid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(O + orow + 32 * hf);
-#pragma unroll
-                    for (int e = 0; e < 4; e++)
-                        dst[e] = make_uint4(outw[4 * e], outw[4 * e + 1], outw[4 * e + 2], outw[4 * e + 3]);
+                    dst[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
             }
         }

@@ -120,13 +120,13 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     } else if (warp >= W_ROT0) {
         const int t = threadIdx.x - W_ROT0 * 32;
         if (tc::mbar_wait(&sm.q_full, 0, ab)) {
-            tc::rotate_tile(sm.q, sm.q, t, rope_t, nullptr);
+            tc::rotate_tile<128>(sm.q, sm.q, t, rope_t, nullptr);
             tc::fence_async_shared();
             tc::mbar_arrive(&sm.q_ready);
             for (int it = 0; it < nck; it++) {
                 const int s = it % NSTAGE;
                 if (!tc::mbar_wait(&sm.kv_full[s], (it / NSTAGE) & 1, ab)) break;
-                tc::rotate_tile(sm.k[s], sm.k[s], t, rope_t, rope_b + (size_t)(k_first + it) * 32);
+                tc::rotate_tile<128>(sm.k[s], sm.k[s], t, rope_t, rope_b + (size_t)(k_first + it) * 32);
                 tc::fence_async_shared();
                 tc::mbar_arrive(&sm.k_ready[s]);
             }

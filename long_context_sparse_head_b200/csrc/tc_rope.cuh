@@ -8,15 +8,18 @@
 namespace fs {
 namespace tc {
 
-// Rotate the 128 x 64 bf16 tile `src` into `tile` (may be the same; 128-byte swizzle: logical 16-byte chunk c of row r sits
-// at chunk c ^ (r & 7)) by angle (row + base_k) * theta_m for pair m.  Thread t of 128.
-__device__ __forceinline__ void rotate_tile(const __nv_bfloat16 *src, __nv_bfloat16 *tile, int t, const float2 *__restrict__ rt,
-                                            const float2 *__restrict__ rb) {
+// Rotate the 128 x 64 bf16 tile `src` into `tile` (may be the same buffer).  128-byte
+// swizzle: logical 16-byte chunk c of row r sits at chunk c ^ (r & 7).  Row r, pair m is
+// rotated by angle (r + base_k) * theta_m: rt[r][m] holds (cos, sin)(r theta_m) and rb[m]
+// (or null for base 0) (cos, sin)(base_k theta_m).  Thread t of NT threads.
+template <int NT>
+__device__ __forceinline__ void rotate_tile(const __nv_bfloat16 *src, __nv_bfloat16 *tile, int t,
+                                            const float2 *__restrict__ rt, const float2 *__restrict__ rb) {
     uint8_t *base = reinterpret_cast<uint8_t *>(tile);
     const uint8_t *sbase = reinterpret_cast<const uint8_t *>(src);
 #pragma unroll 2
-    for (int j = 0; j < 8; j++) {
-        const int item = t + 128 * j;
+    for (int j = 0; j < 1024 / NT; j++) {
+        const int item = t + NT * j;
         const int row = item >> 3, c = item & 7;
         const int off = row * 128 + ((c ^ (row & 7)) << 4);
         uint4 *p = reinterpret_cast<uint4 *>(base + off);
