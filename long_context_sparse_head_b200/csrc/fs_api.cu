@@ -66,6 +66,7 @@ WsLayout layout(const fs_params *p) {
     L.idx = off;   off += align256(BH * (size_t)p->Nq * p->K * 4);
     L.olr = off;   off += align256(BH * (size_t)p->Nq * kD * 4);
     L.rope = off;  off += align256((size_t)(128 + rope_table_rows(p->w)) * 32 * 8);
+    L.tiles = off; off += align256(BH * (size_t)((p->Nq + 127) / 128) * kTileRecWords * 4);
     L.total = off;
     return L;
 }
@@ -88,7 +89,7 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
     const Dev D = make_dev(p);
     const WsLayout L = layout(p);
     const float *olr = nullptr;
-    const bool fused = has_long_range(p) && !idx && attn_tc_supported(p);
+    const bool fused = has_long_range(p) && !idx && attn_tc_supported(p) && select_tc_supported(p);
     if (fused) {   // bf16: selection, then one tensor-core kernel for readout + window + combine
         if (!kbar) {
             float *kb = at<float>(ws, L.kbar), *am = at<float>(ws, L.amax);
@@ -98,11 +99,12 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
         }
         int *exitn = at<int>(ws, L.exitn);
         if (D.prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
-        int32_t *wsidx = at<int32_t>(ws, L.idx);
-        if (launch_selection(p, D, Q, kbar, amax, exitn, wsidx, at<int>(ws, L.flag), st) != cudaSuccess) return FS_ERR_CUDA;
+        uint32_t *tiles = at<uint32_t>(ws, L.tiles);
+        if (launch_select_tc(D, Q, kbar, amax, exitn, nullptr, tiles, at<int>(ws, L.flag), st) != cudaSuccess)
+            return FS_ERR_CUDA;
         float2 *rt = at<float2>(ws, L.rope), *rb = rt + 128 * 32;
         if (launch_rope_table(p->w, p->rope_base, rt, rb, st) != cudaSuccess) return FS_ERR_CUDA;
-        return cuda_status(launch_attn_tc(D, Q, K, V, wsidx, O, rt, rb, at<int>(ws, L.flag), st));
+        return cuda_status(launch_attn_tc(D, Q, K, V, tiles, O, rt, rb, at<int>(ws, L.flag), st));
     }
     if (has_long_range(p)) {
         const int32_t *sel = idx;
@@ -139,7 +141,7 @@ fs_status validate_params(const fs_params *p) { return validate(p); }
 cudaError_t launch_selection(const fs_params *p, const Dev &D, const void *Q, const float *kbar,
                              const float *amax, const int *exitn, int32_t *idx, int *dev_flag,
                              cudaStream_t st) {
-    if (select_tc_supported(p)) return launch_select_tc(D, Q, kbar, amax, exitn, idx, dev_flag, st);
+    if (select_tc_supported(p)) return launch_select_tc(D, Q, kbar, amax, exitn, idx, nullptr, dev_flag, st);
     return launch_select(D, p->dtype, Q, kbar, amax, exitn, idx, st);
 }
 Dev make_dev_params(const fs_params *p) { return make_dev(p); }

@@ -4,10 +4,11 @@
 //   o_i^lr = RMSNorm(u_i)
 //   o_i^sr = softmax_{j in [i-w, i]}((R(i)q_i).(R(j)k_j) / sqrt(d)) V       (RoPE)
 //   O_i    = o_i^sr + alpha_h o_i^lr
-// with S_i given by the selection kernel (idx).
+// with S_i given by the selection kernel's per-tile record (union U of the tile's
+// admitted cells and, per row, the positions in U it selected).
 //
 // One CTA per 128 query rows of a (batch, head); two CTAs per SM.  The readout runs over
-// U, the union of the cells the tile's rows selected (|U| <= 128, ascending), four cells
+// U (|U| <= 128, ascending), four cells
 // (128 keys) per chunk, each cell fetched by its own 32-row TMA box; a row masks the
 // cells it did not select (masked-dense on the tensor cores).  Then the window runs
 // over 128-key chunks.  Both softmaxes accumulate in tensor memory: S/P in columns
@@ -19,8 +20,7 @@
 // Warpgroup 0 (warps 0-3): softmax, thread = query row = TMEM lane; it holds a chunk's
 // whole 128-column S row in registers (one TMEM wait per chunk), raised to 200 registers
 // by setmaxnreg.  Warpgroup 1 (lowered to 56): warp 4 TMA, warp 5 MMA, warps 6-7
-// auxiliary (build U and the per-row selection masks from idx, rotate Q and the window's
-// K chunks).
+// auxiliary (stage U, rotate Q and the window's K chunks).
 #include "tc_rope.cuh"
 
 namespace fs {
@@ -42,10 +42,8 @@ struct AttnSmem {
     __nv_bfloat16 qr[BM * kD];                  // Q rotated (RoPE)
     __nv_bfloat16 k[NSTAGE][BN * kD];
     __nv_bfloat16 v[NSTAGE][BN * kD];
-    uint32_t mask[BM][UMAX / 32];               // row -> selected union positions
     int ulist[UMAX];                            // union cells, ascending
     int nU;
-    int warp_tot[NAUX / 32];
     uint64_t q_full, q_ready, u_ready, s_full, p_full, o_done, drain;
     uint64_t kv_full[NSTAGE], k_ready[NSTAGE], kv_empty[NSTAGE];
     uint32_t tmem_base;
@@ -133,7 +131,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk32,
                const __grid_constant__ CUtensorMap tv32, const __grid_constant__ CUtensorMap tk128,
                const __grid_constant__ CUtensorMap tv128, const AttnArgs A,
-               const int32_t *__restrict__ idx, const float2 *__restrict__ rope_t,
+               const uint32_t *__restrict__ tiles, const float2 *__restrict__ rope_t,
                const float2 *__restrict__ rope_b, __nv_bfloat16 *__restrict__ O, int *dev_flag) {
     extern __shared__ uint8_t smraw[];
     const uint32_t sbase = tc::smem_u32(smraw);
@@ -217,72 +215,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 }
             }
         } else if (warp >= W_AUX0) {
-            const int t = threadIdx.x - W_AUX0 * 32, aw = t >> 5;
-            // ---- U: union of the rows' selected cells, via a bitmap over [0, C) that lives
-            //      in the (not yet loaded) K/V stages, plus a cell -> position byte table
-            uint32_t *bitmap = reinterpret_cast<uint32_t *>(&sm.k[0][0]);
-            uint8_t *cpos = reinterpret_cast<uint8_t *>(&sm.v[0][0]);
-            const int nwords = (A.C + 31) / 32;
-            for (int wd = t; wd < nwords; wd += NAUX) bitmap[wd] = 0u;
+            const int t = threadIdx.x - W_AUX0 * 32;
+            // ---- U and |U| from the selection kernel's record for this tile
+            const uint32_t *rec = tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords;
+            for (int u = t; u < UMAX; u += NAUX) sm.ulist[u] = (int)__ldg(rec + kTileUlistOff + u);
+            if (t == 0) sm.nU = min((int)__ldg(rec + kTileCountOff), UMAX);
             aux_sync();
-            for (int rr = t; rr < nrows; rr += NAUX) {
-                const int32_t *ri = idx + ((size_t)bh * A.Nq + r0 + rr) * A.K;
-                for (int e = 0; e < A.K; e++) {
-                    const int c = ri[e];
-                    if (c >= 0 && c < A.C) atomicOr(&bitmap[c >> 5], 1u << (c & 31));
-                }
-            }
-            aux_sync();
-            const int R = (nwords + NAUX - 1) / NAUX, w0 = min(t * R, nwords), w1 = min(w0 + R, nwords);
-            int cnt = 0;
-            for (int wd = w0; wd < w1; wd++) cnt += __popc(bitmap[wd]);
-            int incl = cnt;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(kFull, incl, o);
-                if (lane >= o) incl += y;
-            }
-            if (lane == 31) sm.warp_tot[aw] = incl;
-            aux_sync();
-            int pos = incl - cnt, total = 0;
-            for (int k = 0; k < NAUX / 32; k++) {
-                if (k < aw) pos += sm.warp_tot[k];
-                total += sm.warp_tot[k];
-            }
-            for (int wd = w0; wd < w1; wd++) {
-                uint32_t bits = bitmap[wd];
-                while (bits) {
-                    const int c = wd * 32 + __ffs(bits) - 1;
-                    bits &= bits - 1;
-                    if (pos < UMAX) {
-                        sm.ulist[pos] = c;
-                        cpos[c] = (uint8_t)pos;
-                    }
-                    pos++;
-                }
-            }
-            if (t == 0) {
-                sm.nU = min(total, UMAX);
-                if (total > UMAX && dev_flag) atomicExch(dev_flag, kFlagCheck);
-            }
-            aux_sync();
-            for (int rr = t; rr < BM; rr += NAUX) {
-                uint32_t mw[UMAX / 32] = {0u, 0u, 0u, 0u};
-                if (rr < nrows) {
-                    const int32_t *ri = idx + ((size_t)bh * A.Nq + r0 + rr) * A.K;
-                    for (int e = 0; e < A.K; e++) {
-                        const int c = ri[e];
-                        if (c >= 0 && c < A.C) {
-                            const int p = cpos[c];
-                            if (p < UMAX) mw[p >> 5] |= 1u << (p & 31);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < UMAX / 32; k++) sm.mask[rr][k] = mw[k];
-            }
-            aux_sync();                       // scratch reads done before the stages are loaded
-            tc::fence_async_shared();
             tc::mbar_arrive(&sm.u_ready);
             const int nR = (sm.nU + CPC - 1) / CPC, total_ck = nR + nW;
             // ---- rotate Q for the window, then pass through (readout) or rotate (window) K
@@ -357,11 +295,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         const int i = pb + row;
         const bool rvalid = row < nrows;
         const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint4 m4 = __ldg(reinterpret_cast<const uint4 *>(
+            tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords + kTileMaskOff + 4 * row));
+        const uint32_t mw[UMAX / 32] = {m4.x, m4.y, m4.z, m4.w};   // selected union positions
         bool ok = tc::mbar_wait(&sm.u_ready, 0, ab);
         const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0, total = nR + nW;
-        uint32_t mw[UMAX / 32];
-#pragma unroll
-        for (int k = 0; k < UMAX / 32; k++) mw[k] = ok ? sm.mask[row][k] : 0u;
         float m_lr = -INFINITY, l_lr = 0.f, m_sr = -INFINITY, l_sr = 0.f;
         for (int it = 0; ok && it < total; it++) {
             if (!tc::mbar_wait(&sm.s_full, it & 1, ab)) { ok = false; break; }
@@ -449,7 +387,7 @@ bool attn_tc_supported(const fs_params *p) {
 }
 
 cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V,
-                           const int32_t *idx, void *O, const float2 *rope_t, const float2 *rope_b,
+                           const uint32_t *tiles, void *O, const float2 *rope_t, const float2 *rope_b,
                            int *dev_flag, cudaStream_t st) {
     if (P.Nq == 0) return cudaSuccess;
     const int BH = P.B * P.H;
@@ -469,7 +407,7 @@ cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const voi
     const dim3 grid((P.Nq + BM - 1) / BM, BH);
     LaunchScope scope(kAttnTc, st);
     cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_tc_kernel<<<grid, NTHREADS, smem, st>>>(tq, tk32, tv32, tk128, tv128, A, idx, rope_t, rope_b,
+    attn_tc_kernel<<<grid, NTHREADS, smem, st>>>(tq, tk32, tv32, tk128, tv128, A, tiles, rope_t, rope_b,
                                                  (__nv_bfloat16 *)O, dev_flag);
     return cudaGetLastError();
 }

@@ -35,8 +35,14 @@ struct Dev {
 
 // Workspace layout (byte offsets from ws; each segment 256-byte aligned).
 struct WsLayout {
-    size_t flag, exitn, kbar, amax, idx, olr, rope, total;
+    size_t flag, exitn, kbar, amax, idx, olr, rope, tiles, total;
 };
+
+// Per-tile selection record passed from the tensor-core selection kernel to the fused
+// attention kernel (128 query rows, union of at most 128 cells), in 32-bit words:
+// [0, 512) row masks [128][4] (bit u of a row: union position u selected), [512, 640)
+// union cells ascending (0xffffffff past |U|), [640] |U|.  2576 bytes, 16-byte multiple.
+constexpr int kTileMaskOff = 0, kTileUlistOff = 512, kTileCountOff = 640, kTileRecWords = 644;
 
 // Device error flag codes (first int of the workspace).
 enum : int { kFlagOk = 0, kFlagTimeout = 1, kFlagCheck = 2 };
@@ -132,7 +138,8 @@ cudaError_t launch_window_tc(const Dev &P, const void *Q, const void *K, const v
 // tensor-core selection (bf16): scores against the bf16x3 split of the mean keys
 bool select_tc_supported(const fs_params *p);
 cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, const float *amax,
-                             const int *exitn, int32_t *idx, int *dev_flag, cudaStream_t st);
+                             const int *exitn, int32_t *idx, uint32_t *tiles, int *dev_flag,
+                             cudaStream_t st);
 // selection with whichever kernel applies (tensor cores for bf16 when supported)
 cudaError_t launch_selection(const fs_params *p, const Dev &D, const void *Q, const float *kbar,
                              const float *amax, const int *exitn, int32_t *idx, int *dev_flag,
@@ -140,7 +147,7 @@ cudaError_t launch_selection(const fs_params *p, const Dev &D, const void *Q, co
 // fused tensor-core readout + window + combine (bf16, internally selected cells)
 bool attn_tc_supported(const fs_params *p);
 cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V,
-                           const int32_t *idx, void *O, const float2 *rope_t, const float2 *rope_b,
+                           const uint32_t *tiles, void *O, const float2 *rope_t, const float2 *rope_b,
                            int *dev_flag, cudaStream_t st);
 
 }  // namespace fs

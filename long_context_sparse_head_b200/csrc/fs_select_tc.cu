@@ -16,6 +16,9 @@
 // by bisection on order-preserving integer keys whose low 7 bits carry (127 - position):
 // keys are unique, and among scores that agree to 2^-17 relative the lower cell index
 // wins, inside the 1e-4 near-tie tolerance of the selection check.
+// Outputs: idx (selected cells per row, ascending, -1 padded) and/or, for the fused
+// kernel, one compact record per tile: each row's selected union positions as a 128-bit
+// mask, the union's cells and its size.
 #include "tc_common.cuh"
 
 namespace fs {
@@ -68,7 +71,7 @@ __device__ __forceinline__ void split3(float x, __nv_bfloat16 &hi, __nv_bfloat16
 __global__ void __launch_bounds__(NTHREADS, 2)
 select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const float *__restrict__ kbar,
                  const float *__restrict__ amax, const int *__restrict__ exitn,
-                 int32_t *__restrict__ idx, int *dev_flag) {
+                 int32_t *__restrict__ idx, uint32_t *__restrict__ tiles, int *dev_flag) {
     extern __shared__ uint8_t smraw[];
     const uint32_t sbase = tc::smem_u32(smraw);
     SelSmem &sm = *reinterpret_cast<SelSmem *>(smraw + (((sbase + 1023u) & ~1023u) - sbase));
@@ -134,29 +137,57 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
         const float *am = amax + (size_t)bh * A.C;
         const int ng = n_max - n_min;   // <= 4
         int total = 0;
-        for (int c0 = 0; c0 < n_max; c0 += 128) {
-            const int c = c0 + t;
-            uint32_t amk = 0;
-            if (c < n_max) {
-                const int e = A.prune ? ex[c] : 0;
+        // 1024 cells per round, eight consecutive ones per thread: the exit times are
+        // fetched with two 16-byte loads before any of them is used, then one block-wide
+        // exclusive scan orders the members
+        for (int c0 = 0; c0 < n_max; c0 += 1024) {
+            const int cb = c0 + 8 * t;
+            int e8[8];
+            if (A.prune && cb + 8 <= n_max && (reinterpret_cast<uintptr_t>(ex + cb) & 15) == 0) {
+                const int4 x0 = __ldg(reinterpret_cast<const int4 *>(ex + cb));
+                const int4 x1 = __ldg(reinterpret_cast<const int4 *>(ex + cb) + 1);
+                e8[0] = x0.x; e8[1] = x0.y; e8[2] = x0.z; e8[3] = x0.w;
+                e8[4] = x1.x; e8[5] = x1.y; e8[6] = x1.z; e8[7] = x1.w;
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; j++) e8[j] = (A.prune && cb + j < n_max) ? ex[cb + j] : 0;
+            }
+            uint32_t amk[8];
+            int cnt = 0;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const int c = cb + j;
+                amk[j] = 0;
 #pragma unroll
                 for (int g = 0; g <= 4; g++) {
                     const int n = n_min + g;
-                    if (g <= ng && c < n && (!A.prune || c >= n - A.W || n < e)) amk |= 1u << g;
+                    if (g <= ng && c < n && (!A.prune || c >= n - A.W || n < e8[j])) amk[j] |= 1u << g;
                 }
+                cnt += amk[j] != 0;
             }
-            const unsigned m = __ballot_sync(kFull, amk != 0);
-            if (lane == 0) sm.warp_cnt[warp] = __popc(m);
+            int incl = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (lane == 31) sm.warp_cnt[warp] = incl;
             sel_sync();
-            int pos = total + __popc(m & ((1u << lane) - 1u)), tot = 0;
+            int pos = total + incl - cnt, tot = 0;
             for (int k = 0; k < 4; k++) {
                 if (k < warp) pos += sm.warp_cnt[k];
                 tot += sm.warp_cnt[k];
             }
-            if (amk && pos < UMAX) {
-                sm.ulist[pos] = c;
-                sm.amask[pos] = (uint8_t)amk;
-                sm.acell[pos] = am[c];
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                if (amk[j]) {
+                    if (pos < UMAX) {
+                        sm.ulist[pos] = cb + j;
+                        sm.amask[pos] = (uint8_t)amk[j];
+                        sm.acell[pos] = A.has_prior ? am[cb + j] : 0.f;
+                    }
+                    pos++;
+                }
             }
             total += tot;
             sel_sync();
@@ -257,7 +288,21 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                 }
                 tau = lo;
             }
-            if (row < nrows) {
+            if (tiles) {   // compact record for the fused kernel: row masks | union | |U|
+                uint32_t *rec = tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords;
+                uint32_t mw[4];
+#pragma unroll
+                for (int b = 0; b < UMAX / 32; b++) {
+                    mw[b] = 0u;
+#pragma unroll
+                    for (int e = 0; e < 32; e++)
+                        if (key[32 * b + e] >= tau && key[32 * b + e] != 0u) mw[b] |= 1u << e;
+                }
+                *reinterpret_cast<uint4 *>(rec + kTileMaskOff + 4 * row) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+                rec[kTileUlistOff + t] = t < nU ? (uint32_t)sm.ulist[t] : 0xffffffffu;
+                if (t == 0) rec[kTileCountOff] = (uint32_t)nU;
+            }
+            if (idx && row < nrows) {
                 int32_t *out = idx + ((size_t)bh * A.Nq + r0 + row) * A.K;
                 int o = 0;
 #pragma unroll
@@ -291,7 +336,8 @@ bool select_tc_supported(const fs_params *p) {
 }
 
 cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, const float *amax,
-                             const int *exitn, int32_t *idx, int *dev_flag, cudaStream_t st) {
+                             const int *exitn, int32_t *idx, uint32_t *tiles, int *dev_flag,
+                             cudaStream_t st) {
     if (P.Nq == 0) return cudaSuccess;
     const int BH = P.B * P.H;
     CUtensorMap tq;
@@ -308,7 +354,7 @@ cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, con
     const dim3 grid((P.Nq + BM - 1) / BM, BH);
     LaunchScope scope(kSelectTc, st);
     cudaFuncSetAttribute(select_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    select_tc_kernel<<<grid, NTHREADS, smem, st>>>(tq, A, kbar, amax, exitn, idx, dev_flag);
+    select_tc_kernel<<<grid, NTHREADS, smem, st>>>(tq, A, kbar, amax, exitn, idx, tiles, dev_flag);
     return cudaGetLastError();
 }
 
