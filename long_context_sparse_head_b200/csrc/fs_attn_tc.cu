@@ -69,25 +69,40 @@ __device__ __forceinline__ void ld_row128(uint32_t taddr, uint32_t (&s)[128]) {
     tc::tmem_wait_ld();
 }
 
+// Column validity of a chunk: every column (FULL), the columns of the selected cells
+// (CELLS: 32-column block b valid iff bit b of sel4), or a band of the window (BAND:
+// lo <= j < lo + width).
+enum ChunkKind { FULL = 0, CELLS = 1, BAND = 2 };
+
 // One chunk of online softmax for this thread's row.  S is read from TMEM columns
 // [S_COL, S_COL+128) in one batch; P = exp2(S*c - m) is written back as bf16 pairs over
-// [S_COL, S_COL+64).  Readout chunks (MASKED_CELLS): 32-column block b is valid iff bit b
-// of sel4 is set.  Window chunks: column j is valid iff clo <= j <= chi.  The running max
-// m (log2 units) is raised only when a chunk exceeds it by more than 8 (lazy rescale of O).
-template <bool MASKED_CELLS>
+// [S_COL, S_COL+64).  The running max m (log2 units) is raised only when a chunk exceeds
+// it by more than 8 (lazy rescale of O).  Maxima and sums use eight independent partial
+// accumulators so no long dependency chain forms.
+template <int KIND>
 __device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, bool first, uint32_t sel4,
-                                              int clo, int chi, float c_log2, float &m_used, float &l) {
+                                              int lo, int width, float c_log2, float &m_used, float &l) {
     uint32_t s[128];
     ld_row128(trow + S_COL, s);
-    const bool full = MASKED_CELLS ? false : __all_sync(kFull, clo <= 0 && chi >= BN - 1);
-    auto ok = [&](int j) -> bool {
-        if (MASKED_CELLS) return ((sel4 >> (j >> 5)) & 1u) != 0;
-        return full || (j >= clo && j <= chi);
-    };
-    float mx = -INFINITY;
+    // invalid columns become -inf once: the max ignores them and exp2 turns them into 0
+    if (KIND == CELLS) {
 #pragma unroll
-    for (int j = 0; j < BN; j++)
-        if (ok(j)) mx = fmaxf(mx, __uint_as_float(s[j]));
+        for (int b = 0; b < BN / 32; b++)
+            if (!((sel4 >> b) & 1u)) {
+#pragma unroll
+                for (int e = 0; e < 32; e++) s[32 * b + e] = 0xff800000u;
+            }
+    } else if (KIND == BAND) {
+#pragma unroll
+        for (int j = 0; j < BN; j++)
+            if ((unsigned)(j - lo) >= (unsigned)width) s[j] = 0xff800000u;
+    }
+    float mp[8];
+#pragma unroll
+    for (int k = 0; k < 8; k++) mp[k] = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < BN; j++) mp[j & 7] = fmaxf(mp[j & 7], __uint_as_float(s[j]));
+    float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
     mx *= c_log2;
     const bool grow = mx > m_used + 8.f;
     const float m_new = grow ? mx : m_used;
@@ -95,21 +110,23 @@ __device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, boo
     l *= corr;
     m_used = m_new;
     const float msub = m_used == -INFINITY ? 0.f : m_used;
+    float ls[8];
+#pragma unroll
+    for (int k = 0; k < 8; k++) ls[k] = 0.f;
 #pragma unroll
     for (int q = 0; q < 4; q++) {                    // P keys [32 q, 32 q + 32) -> 16 columns
         uint32_t pk[16];
-        float lsum = 0.f;
 #pragma unroll
         for (int e = 0; e < 16; e++) {
             const int j = 32 * q + 2 * e;
-            const float p0 = ok(j) ? tc::ex2(fmaf(__uint_as_float(s[j]), c_log2, -msub)) : 0.f;
-            const float p1 = ok(j + 1) ? tc::ex2(fmaf(__uint_as_float(s[j + 1]), c_log2, -msub)) : 0.f;
-            lsum += p0 + p1;
+            const float p0 = tc::ex2(fmaf(__uint_as_float(s[j]), c_log2, -msub));
+            const float p1 = tc::ex2(fmaf(__uint_as_float(s[j + 1]), c_log2, -msub));
+            ls[e & 7] += p0 + p1;
             pk[e] = tc::pack_bf16x2(p0, p1);
         }
-        l += lsum;
         tc::tmem_st16(trow + S_COL + 16 * q, pk);
     }
+    l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
     // O rescale after the exponentials, when S no longer occupies registers (no MMA
     // touches O until this thread arrives on p_full)
     if (!first && __any_sync(kFull, corr != 1.f)) {
@@ -307,7 +324,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             if (it < nR) {
                 const int p0 = CPC * it;
                 const uint32_t sel4 = (mw[p0 >> 5] >> (p0 & 31)) & 0xfu;
-                softmax_chunk<true>(trow, OLR_COL, it == 0, sel4, 0, -1, A.scale_log2e, m_lr, l_lr);
+                softmax_chunk<CELLS>(trow, OLR_COL, it == 0, sel4, 0, 0, A.scale_log2e, m_lr, l_lr);
             } else {
                 if (it == nR && nR > 0) {   // readout done: O_lr <- alpha_h RMSNorm(O_lr / l)
                     uint32_t a[32], b[32];
@@ -331,9 +348,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     tc::tmem_st32(trow + OLR_COL + 32, b);
                 }
                 const int jc = jbase + BN * (k_first + it - nR);
-                int clo = max(-jc, i - A.w - jc), chi = min(i - jc, BN - 1);
-                if (!rvalid) { clo = 1; chi = 0; }
-                softmax_chunk<false>(trow, OSR_COL, it == nR, 0u, clo, chi, A.scale_log2e, m_sr, l_sr);
+                const int clo = max(-jc, i - A.w - jc), chi = min(i - jc, BN - 1);
+                const int width = rvalid ? max(0, chi - clo + 1) : 0;
+                if (__all_sync(kFull, clo <= 0 && chi >= BN - 1 && rvalid))
+                    softmax_chunk<FULL>(trow, OSR_COL, it == nR, 0u, 0, BN, A.scale_log2e, m_sr, l_sr);
+                else
+                    softmax_chunk<BAND>(trow, OSR_COL, it == nR, 0u, clo, width, A.scale_log2e, m_sr, l_sr);
             }
             tc::tc_fence_before();
             tc::mbar_arrive(&sm.p_full);

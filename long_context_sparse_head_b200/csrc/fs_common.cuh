@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/freesolo.h"
+#include "freesolo.h"
 
 namespace fs {
 

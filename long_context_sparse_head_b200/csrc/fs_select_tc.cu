@@ -272,13 +272,14 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                 uint32_t lo = kmin, hi = kmax + 1u;       // count(>= kmin) = na > K, count(>= kmax+1) = 0
                 while (hi - lo > 1u) {
                     const uint32_t mid = lo + ((hi - lo) >> 1);
-                    int cnt = 0;
+                    int cp[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent partial counts
 #pragma unroll
                     for (int b = 0; b < UMAX / 32; b++)
                         if (32 * b < N) {
 #pragma unroll
-                            for (int e = 0; e < 32; e++) cnt += key[32 * b + e] >= mid;
+                            for (int e = 0; e < 32; e++) cp[e & 7] += key[32 * b + e] >= mid;
                         }
+                    const int cnt = ((cp[0] + cp[1]) + (cp[2] + cp[3])) + ((cp[4] + cp[5]) + (cp[6] + cp[7]));
                     if (cnt >= A.K) {
                         lo = mid;
                         if (cnt == A.K) break;

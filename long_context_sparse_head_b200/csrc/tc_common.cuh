@@ -51,8 +51,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 
 // Every wait is bounded.  A wait that runs out of time (or sees another thread's abort)
 // records kFlagTimeout in the device error flag, raises the CTA's abort word and returns
-// false; the caller then skips to the kernel's clean-up.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+// false; the caller then skips to the kernel's clean-up.  The budget is counted in SM
+// clock cycles (cheap to read) and checked every 64 polls, so a barrier that completes
+// is seen within one poll.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;       // 2 s (clean-up drains)
+constexpr long long kWaitLimitCycles = 4000000000ll;   // >= 2 s at any SM clock <= 2 GHz
 
 struct Abort {
     int *dev_flag;        // device error flag (first int of the workspace), or null
@@ -61,14 +64,16 @@ struct Abort {
 
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const Abort &ab) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    while (true) {
+    const long long t0 = clock64();
+    for (uint32_t n = 1;; n++) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*ab.cta) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
-            *ab.cta = 1;
-            if (ab.dev_flag) atomicExch(ab.dev_flag, kFlagTimeout);
-            return false;
+        if ((n & 63) == 0) {
+            if (*ab.cta) return false;
+            if (clock64() - t0 > kWaitLimitCycles) {
+                *ab.cta = 1;
+                if (ab.dev_flag) atomicExch(ab.dev_flag, kFlagTimeout);
+                return false;
+            }
         }
     }
 }
