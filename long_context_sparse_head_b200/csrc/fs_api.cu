@@ -5,7 +5,7 @@
 #include <cmath>
 #include <cstring>
 
-#include "fs_common.cuh"
+#include "tc_rope.cuh"
 
 namespace fs {
 namespace {
@@ -67,6 +67,9 @@ WsLayout layout(const fs_params *p) {
     L.olr = off;   off += align256(BH * (size_t)p->Nq * kD * 4);
     L.rope = off;  off += align256((size_t)(128 + rope_table_rows(p->w)) * 32 * 8);
     L.tiles = off; off += align256(BH * (size_t)((p->Nq + 127) / 128) * kTileRecWords * 4);
+    L.rope_abs = off; off += align256((size_t)(kRopeLo + rope_hi_rows(p->Nk)) * 32 * 8);
+    const int kr0 = p->Nk - p->Nq - p->w > 0 ? p->Nk - p->Nq - p->w : 0;   // first rotated key
+    L.krot = off;  off += align256(BH * (size_t)(p->Nk - kr0) * kD * 2);
     L.total = off;
     return L;
 }
@@ -102,9 +105,12 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
         uint32_t *tiles = at<uint32_t>(ws, L.tiles);
         if (launch_select_tc(D, Q, kbar, amax, exitn, nullptr, tiles, at<int>(ws, L.flag), st) != cudaSuccess)
             return FS_ERR_CUDA;
-        float2 *rt = at<float2>(ws, L.rope), *rb = rt + 128 * 32;
-        if (launch_rope_table(p->w, p->rope_base, rt, rb, st) != cudaSuccess) return FS_ERR_CUDA;
-        return cuda_status(launch_attn_tc(D, Q, K, V, tiles, O, rt, rb, at<int>(ws, L.flag), st));
+        float2 *lo = at<float2>(ws, L.rope_abs), *hi = lo + kRopeLo * 32;
+        void *krot = at<void>(ws, L.krot);
+        if (launch_rope_abs_table(p->Nk, p->rope_base, lo, hi, st) != cudaSuccess ||
+            launch_rope_keys(D, K, krot, lo, hi, st) != cudaSuccess)
+            return FS_ERR_CUDA;
+        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), st));
     }
     if (has_long_range(p)) {
         const int32_t *sel = idx;

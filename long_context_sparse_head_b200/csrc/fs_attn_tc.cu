@@ -20,7 +20,8 @@
 // Warpgroup 0 (warps 0-3): softmax, thread = query row = TMEM lane; it holds a chunk's
 // whole 128-column S row in registers (one TMEM wait per chunk), raised to 200 registers
 // by setmaxnreg.  Warpgroup 1 (lowered to 56): warp 4 TMA, warp 5 MMA, warps 6-7
-// auxiliary (stage U, rotate Q and the window's K chunks).
+// auxiliary (stage U, rotate Q by its absolute positions).  The window's keys come
+// pre-rotated (absolute positions, double-precision angles) from a workspace copy.
 #include "tc_rope.cuh"
 
 namespace fs {
@@ -45,13 +46,14 @@ struct AttnSmem {
     int ulist[UMAX];                            // union cells, ascending
     int nU;
     uint64_t q_full, q_ready, u_ready, s_full, p_full, o_done, drain;
-    uint64_t kv_full[NSTAGE], k_ready[NSTAGE], kv_empty[NSTAGE];
+    uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
     uint32_t tmem_base;
     int abort;
 };
 
 struct AttnArgs {
     int Nq, Nk, q0, w, C, K, H;
+    int kr0;                // first key of the rotated copy
     float scale_log2e;      // log2(e) / sqrt(d)
     float rms_eps;
     float alpha[FS_MAX_HEADS];
@@ -146,10 +148,10 @@ __device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, boo
 
 __global__ void __launch_bounds__(NTHREADS, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk32,
-               const __grid_constant__ CUtensorMap tv32, const __grid_constant__ CUtensorMap tk128,
+               const __grid_constant__ CUtensorMap tv32, const __grid_constant__ CUtensorMap tkr128,
                const __grid_constant__ CUtensorMap tv128, const AttnArgs A,
-               const uint32_t *__restrict__ tiles, const float2 *__restrict__ rope_t,
-               const float2 *__restrict__ rope_b, __nv_bfloat16 *__restrict__ O, int *dev_flag) {
+               const uint32_t *__restrict__ tiles, const float2 *__restrict__ rope_lo,
+               const float2 *__restrict__ rope_hi, __nv_bfloat16 *__restrict__ O, int *dev_flag) {
     extern __shared__ uint8_t smraw[];
     const uint32_t sbase = tc::smem_u32(smraw);
     AttnSmem &sm = *reinterpret_cast<AttnSmem *>(smraw + (((sbase + 1023u) & ~1023u) - sbase));
@@ -175,7 +177,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         tc::mbar_init(&sm.drain, 1);
         for (int s = 0; s < NSTAGE; s++) {
             tc::mbar_init(&sm.kv_full[s], 1);
-            tc::mbar_init(&sm.k_ready[s], NAUX);
             tc::mbar_init(&sm.kv_empty[s], 1);
         }
         tc::fence_barrier_init();
@@ -196,7 +197,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 tc::prefetch_tmap(&tq);
                 tc::prefetch_tmap(&tk32);
                 tc::prefetch_tmap(&tv32);
-                tc::prefetch_tmap(&tk128);
+                tc::prefetch_tmap(&tkr128);
                 tc::prefetch_tmap(&tv128);
                 tc::mbar_expect_tx(&sm.q_full, TILE_BYTES);
                 tc::tma_load_3d(sm.qn, &tq, &sm.q_full, 0, r0, bh);
@@ -214,10 +215,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                                 tc::tma_load_3d(sm.k[s] + j * kS * kD, &tk32, &sm.kv_full[s], 0, y, bh);
                                 tc::tma_load_3d(sm.v[s] + j * kS * kD, &tv32, &sm.kv_full[s], 0, y, bh);
                             }
-                        } else {                // 128 consecutive keys of the band
+                        } else {                // 128 consecutive keys of the band (K pre-rotated)
                             const int jc = jbase + BN * (k_first + it - nR);
                             tc::mbar_expect_tx(&sm.kv_full[s], 2 * TILE_BYTES);
-                            tc::tma_load_3d(sm.k[s], &tk128, &sm.kv_full[s], 0, jc, bh);
+                            tc::tma_load_3d(sm.k[s], &tkr128, &sm.kv_full[s], 0, jc - A.kr0, bh);
                             tc::tma_load_3d(sm.v[s], &tv128, &sm.kv_full[s], 0, jc, bh);
                         }
                     }
@@ -239,22 +240,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             if (t == 0) sm.nU = min((int)__ldg(rec + kTileCountOff), UMAX);
             aux_sync();
             tc::mbar_arrive(&sm.u_ready);
-            const int nR = (sm.nU + CPC - 1) / CPC, total_ck = nR + nW;
-            // ---- rotate Q for the window, then pass through (readout) or rotate (window) K
+            // ---- rotate Q by its absolute positions for the window
             if (tc::mbar_wait(&sm.q_full, 0, ab)) {
-                tc::rotate_tile<NAUX>(sm.qn, sm.qr, t, rope_t, nullptr);
+                const uint8_t *src = reinterpret_cast<const uint8_t *>(sm.qn);
+                uint8_t *dst = reinterpret_cast<uint8_t *>(sm.qr);
+#pragma unroll 2
+                for (int j = 0; j < 1024 / NAUX; j++) {
+                    const int item = t + NAUX * j, row = item >> 3, c = item & 7;
+                    const int off = row * 128 + ((c ^ (row & 7)) << 4);   // 128-byte swizzle
+                    float cs[4], sn[4];
+                    rope_angles(pb + row, c, rope_lo, rope_hi, cs, sn);
+                    *reinterpret_cast<uint4 *>(dst + off) =
+                        rope_rotate8(*reinterpret_cast<const uint4 *>(src + off), cs, sn);
+                }
                 tc::fence_async_shared();
                 tc::mbar_arrive(&sm.q_ready);
-                for (int it = 0; it < total_ck; it++) {
-                    const int s = it % NSTAGE;
-                    if (!tc::mbar_wait(&sm.kv_full[s], (it / NSTAGE) & 1, ab)) break;
-                    if (it >= nR) {
-                        tc::rotate_tile<NAUX>(sm.k[s], sm.k[s], t, rope_t,
-                                              rope_b + (size_t)(k_first + it - nR) * 32);
-                        tc::fence_async_shared();
-                    }
-                    tc::mbar_arrive(&sm.k_ready[s]);
-                }
             }
         } else if (warp == W_MMA) {
             if (lane == 0) {
@@ -265,10 +265,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0, total = nR + nW;
                 int issued = 0;
                 for (int it = 0; ok && it <= total; it++) {
-                    if (it < total && !tc::mbar_wait(&sm.k_ready[it % NSTAGE], (it / NSTAGE) & 1, ab)) {
-                        ok = false;
-                        break;
-                    }
                     if (it > 0) {   // O += P(it-1) V(it-1), into the readout's or the window's O
                         if (!tc::mbar_wait(&sm.p_full, (it - 1) & 1, ab)) { ok = false; break; }
                         tc::tc_fence_after();
@@ -284,6 +280,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                         issued++;
                     }
                     if (it < total) {   // S = Q K(it)^T with the NoPE or the rotated Q
+                        if (!tc::mbar_wait(&sm.kv_full[it % NSTAGE], (it / NSTAGE) & 1, ab)) {
+                            ok = false;
+                            break;
+                        }
                         if (it == nR && !tc::mbar_wait(&sm.q_ready, 0, ab)) { ok = false; break; }
                         tc::tc_fence_after();
                         const uint32_t qa = it < nR ? qn : qr;
@@ -406,20 +406,22 @@ bool attn_tc_supported(const fs_params *p) {
     return bound <= UMAX;
 }
 
-cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V,
-                           const uint32_t *tiles, void *O, const float2 *rope_t, const float2 *rope_b,
+cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V, const void *Krot,
+                           const uint32_t *tiles, void *O, const float2 *rope_lo, const float2 *rope_hi,
                            int *dev_flag, cudaStream_t st) {
     if (P.Nq == 0) return cudaSuccess;
     const int BH = P.B * P.H;
-    CUtensorMap tq, tk32, tv32, tk128, tv128;
+    const int kr0 = rope_first_key(P);
+    CUtensorMap tq, tk32, tv32, tkr128, tv128;
     if (!encode_tmap_3d_bf16(&tq, Q, kD, P.Nq, BH, kD, BM) ||
         !encode_tmap_3d_bf16(&tk32, K, kD, P.Nk, BH, kD, kS) ||
         !encode_tmap_3d_bf16(&tv32, V, kD, P.Nk, BH, kD, kS) ||
-        !encode_tmap_3d_bf16(&tk128, K, kD, P.Nk, BH, kD, BN) ||
+        !encode_tmap_3d_bf16(&tkr128, Krot, kD, P.Nk - kr0, BH, kD, BN) ||
         !encode_tmap_3d_bf16(&tv128, V, kD, P.Nk, BH, kD, BN))
         return cudaErrorInvalidValue;
     AttnArgs A;
     A.Nq = P.Nq; A.Nk = P.Nk; A.q0 = P.q0; A.w = P.w; A.C = P.C; A.K = P.K; A.H = P.H;
+    A.kr0 = kr0;
     A.scale_log2e = P.scale * 1.4426950408889634f;
     A.rms_eps = P.rms_eps;
     for (int hh = 0; hh < FS_MAX_HEADS; hh++) A.alpha[hh] = P.alpha[hh];
@@ -427,7 +429,7 @@ cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const voi
     const dim3 grid((P.Nq + BM - 1) / BM, BH);
     LaunchScope scope(kAttnTc, st);
     cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_tc_kernel<<<grid, NTHREADS, smem, st>>>(tq, tk32, tv32, tk128, tv128, A, tiles, rope_t, rope_b,
+    attn_tc_kernel<<<grid, NTHREADS, smem, st>>>(tq, tk32, tv32, tkr128, tv128, A, tiles, rope_lo, rope_hi,
                                                  (__nv_bfloat16 *)O, dev_flag);
     return cudaGetLastError();
 }

@@ -35,7 +35,7 @@ struct Dev {
 
 // Workspace layout (byte offsets from ws; each segment 256-byte aligned).
 struct WsLayout {
-    size_t flag, exitn, kbar, amax, idx, olr, rope, tiles, total;
+    size_t flag, exitn, kbar, amax, idx, olr, rope, tiles, rope_abs, krot, total;
 };
 
 // Per-tile selection record passed from the tensor-core selection kernel to the fused
@@ -102,7 +102,7 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 // ---- kernel ids for the diagnostics (fs_kernel_times) ----
 enum KernelId : int {
     kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
-    kSelectTc, kNumKernels
+    kSelectTc, kRopeKeys, kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
@@ -135,6 +135,11 @@ cudaError_t launch_rope_table(int w, float rope_base, float2 *rope_t, float2 *ro
 cudaError_t launch_window_tc(const Dev &P, const void *Q, const void *K, const void *V,
                              const float *olr, void *O, const float2 *rope_t, const float2 *rope_b,
                              int *dev_flag, cudaStream_t st);
+// absolute-position RoPE tables and the rotated copy of the keys the windows read
+int rope_hi_rows(int Nk);
+cudaError_t launch_rope_abs_table(int Nk, float rope_base, float2 *lo, float2 *hi, cudaStream_t st);
+cudaError_t launch_rope_keys(const Dev &P, const void *K, void *Krot, const float2 *lo, const float2 *hi,
+                             cudaStream_t st);
 // tensor-core selection (bf16): scores against the bf16x3 split of the mean keys
 bool select_tc_supported(const fs_params *p);
 cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, const float *amax,
@@ -146,8 +151,8 @@ cudaError_t launch_selection(const fs_params *p, const Dev &D, const void *Q, co
                              cudaStream_t st);
 // fused tensor-core readout + window + combine (bf16, internally selected cells)
 bool attn_tc_supported(const fs_params *p);
-cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V,
-                           const uint32_t *tiles, void *O, const float2 *rope_t, const float2 *rope_b,
+cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V, const void *Krot,
+                           const uint32_t *tiles, void *O, const float2 *rope_lo, const float2 *rope_hi,
                            int *dev_flag, cudaStream_t st);
 
 }  // namespace fs

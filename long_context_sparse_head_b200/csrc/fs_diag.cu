@@ -31,7 +31,7 @@ cudaEvent_t take_event() {
 
 const char *const kNames[kNumKernels] = {"cell_summaries", "exit_times", "select_topk",
                                          "readout", "window_combine", "rope_table",
-                                         "window_tc", "attn_tc", "select_tc"};
+                                         "window_tc", "attn_tc", "select_tc", "rope_keys"};
 }  // namespace
 
 LaunchScope::LaunchScope(int id_, cudaStream_t st_) : id(id_), st(st_), slot(-1) {
