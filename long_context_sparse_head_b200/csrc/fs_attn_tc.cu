@@ -77,24 +77,23 @@ __device__ __forceinline__ void ld_row128(uint32_t taddr, uint32_t (&s)[128]) {
 enum ChunkKind { FULL = 0, CELLS = 1, BAND = 2 };
 
 // One chunk of online softmax for this thread's row.  S is read from TMEM columns
-// [S_COL, S_COL+128) in one batch; P = exp2(S*c - m) is written back as bf16 pairs over
-// [S_COL, S_COL+64).  The running max m (log2 units) is raised only when a chunk exceeds
-// it by more than 8 (lazy rescale of O).  Maxima and sums use eight independent partial
-// accumulators so no long dependency chain forms.
-template <int KIND>
-__device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, bool first, uint32_t sel4,
-                                              int lo, int width, float c_log2, float &m_used, float &l) {
+// [S_COL, S_COL+128) in one batch; invalid columns become -inf (the max ignores them and
+// exp2 turns them into 0), so the rest is one body for every kind of chunk.  P =
+// exp2(S*c - m) is written back as bf16 pairs over [S_COL, S_COL+64).  The running max m
+// (log2 units) is raised only when a chunk exceeds it by more than 8 (lazy rescale of O).
+// Maxima and sums use eight independent partial accumulators (no long dependency chain).
+__device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, bool first, int kind, uint32_t sel4,
+                                           int lo, int width, float c_log2, float &m_used, float &l) {
     uint32_t s[128];
     ld_row128(trow + S_COL, s);
-    // invalid columns become -inf once: the max ignores them and exp2 turns them into 0
-    if (KIND == CELLS) {
+    if (kind == CELLS) {
 #pragma unroll
         for (int b = 0; b < BN / 32; b++)
             if (!((sel4 >> b) & 1u)) {
 #pragma unroll
                 for (int e = 0; e < 32; e++) s[32 * b + e] = 0xff800000u;
             }
-    } else if (KIND == BAND) {
+    } else if (kind == BAND) {
 #pragma unroll
         for (int j = 0; j < BN; j++)
             if ((unsigned)(j - lo) >= (unsigned)width) s[j] = 0xff800000u;
@@ -321,40 +320,46 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         for (int it = 0; ok && it < total; it++) {
             if (!tc::mbar_wait(&sm.s_full, it & 1, ab)) { ok = false; break; }
             tc::tc_fence_after();
+            if (it == nR && nR > 0) {   // readout done: O_lr <- alpha_h RMSNorm(O_lr / l)
+                uint32_t a[32], b[32];
+                tc::tmem_ld32(trow + OLR_COL, a);
+                tc::tmem_ld32(trow + OLR_COL + 32, b);
+                tc::tmem_wait_ld();
+                const float inv_l = l_lr > 0.f ? 1.f / l_lr : 0.f;
+                float ss = 0.f;
+#pragma unroll
+                for (int e = 0; e < 32; e++) {
+                    const float x = __uint_as_float(a[e]) * inv_l, y = __uint_as_float(b[e]) * inv_l;
+                    ss = fmaf(x, x, fmaf(y, y, ss));
+                }
+                const float f = l_lr > 0.f ? A.alpha[h] * inv_l / sqrtf(ss * (1.f / kD) + A.rms_eps) : 0.f;
+#pragma unroll
+                for (int e = 0; e < 32; e++) {
+                    a[e] = __float_as_uint(__uint_as_float(a[e]) * f);
+                    b[e] = __float_as_uint(__uint_as_float(b[e]) * f);
+                }
+                tc::tmem_st32(trow + OLR_COL, a);
+                tc::tmem_st32(trow + OLR_COL + 32, b);
+            }
+            // one call site for every kind of chunk keeps the unrolled body in the code once
+            int kind, lo = 0, width = BN;
+            uint32_t sel4 = 0u, ocol;
+            bool first;
+            float m, l;
             if (it < nR) {
                 const int p0 = CPC * it;
-                const uint32_t sel4 = (mw[p0 >> 5] >> (p0 & 31)) & 0xfu;
-                softmax_chunk<CELLS>(trow, OLR_COL, it == 0, sel4, 0, 0, A.scale_log2e, m_lr, l_lr);
+                sel4 = (mw[p0 >> 5] >> (p0 & 31)) & 0xfu;
+                kind = CELLS; ocol = OLR_COL; first = it == 0; m = m_lr; l = l_lr;
             } else {
-                if (it == nR && nR > 0) {   // readout done: O_lr <- alpha_h RMSNorm(O_lr / l)
-                    uint32_t a[32], b[32];
-                    tc::tmem_ld32(trow + OLR_COL, a);
-                    tc::tmem_ld32(trow + OLR_COL + 32, b);
-                    tc::tmem_wait_ld();
-                    const float inv_l = l_lr > 0.f ? 1.f / l_lr : 0.f;
-                    float ss = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 32; e++) {
-                        const float x = __uint_as_float(a[e]) * inv_l, y = __uint_as_float(b[e]) * inv_l;
-                        ss = fmaf(x, x, fmaf(y, y, ss));
-                    }
-                    const float f = l_lr > 0.f ? A.alpha[h] * inv_l / sqrtf(ss * (1.f / kD) + A.rms_eps) : 0.f;
-#pragma unroll
-                    for (int e = 0; e < 32; e++) {
-                        a[e] = __float_as_uint(__uint_as_float(a[e]) * f);
-                        b[e] = __float_as_uint(__uint_as_float(b[e]) * f);
-                    }
-                    tc::tmem_st32(trow + OLR_COL, a);
-                    tc::tmem_st32(trow + OLR_COL + 32, b);
-                }
                 const int jc = jbase + BN * (k_first + it - nR);
                 const int clo = max(-jc, i - A.w - jc), chi = min(i - jc, BN - 1);
-                const int width = rvalid ? max(0, chi - clo + 1) : 0;
-                if (__all_sync(kFull, clo <= 0 && chi >= BN - 1 && rvalid))
-                    softmax_chunk<FULL>(trow, OSR_COL, it == nR, 0u, 0, BN, A.scale_log2e, m_sr, l_sr);
-                else
-                    softmax_chunk<BAND>(trow, OSR_COL, it == nR, 0u, clo, width, A.scale_log2e, m_sr, l_sr);
+                lo = clo;
+                width = rvalid ? max(0, chi - clo + 1) : 0;
+                kind = __all_sync(kFull, clo <= 0 && chi >= BN - 1 && rvalid) ? FULL : BAND;
+                ocol = OSR_COL; first = it == nR; m = m_sr; l = l_sr;
             }
+            softmax_chunk(trow, ocol, first, kind, sel4, lo, width, A.scale_log2e, m, l);
+            if (it < nR) { m_lr = m; l_lr = l; } else { m_sr = m; l_sr = l; }
             tc::tc_fence_before();
             tc::mbar_arrive(&sm.p_full);
         }

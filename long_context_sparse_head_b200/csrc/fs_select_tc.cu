@@ -68,6 +68,7 @@ __device__ __forceinline__ void split3(float x, __nv_bfloat16 &hi, __nv_bfloat16
 }
 }  // namespace
 
+template <bool PRIOR>
 __global__ void __launch_bounds__(NTHREADS, 2)
 select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const float *__restrict__ kbar,
                  const float *__restrict__ amax, const int *__restrict__ exitn,
@@ -233,8 +234,8 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
         {
             tc::tc_fence_after();
             const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-            const float lam = A.has_prior ? A.lambda[h] : 0.f;
-            const float i2s = A.inv2sigma[h];
+            const float lam = PRIOR ? A.lambda[h] : 0.f;
+            const float i2s = PRIOR ? A.inv2sigma[h] : 0.f;
             uint32_t key[UMAX];
             uint32_t kmin = 0xffffffffu, kmax = 0u;
             int na = 0;
@@ -250,7 +251,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                         uint32_t k = 0u;
                         if (u < nU && ((sm.amask[u] >> g) & 1u) && row < nrows) {
                             float sc = __uint_as_float(r[e]) * A.scale;
-                            if (lam != 0.f) {
+                            if (PRIOR) {
                                 const float pc = (float)(sm.ulist[u] * kS) + 0.5f * kS;
                                 sc += lam * sm.acell[u] * erff(((float)i - pc) * i2s);
                             }
@@ -354,8 +355,10 @@ cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, con
     const size_t smem = sizeof(SelSmem) + 1024;
     const dim3 grid((P.Nq + BM - 1) / BM, BH);
     LaunchScope scope(kSelectTc, st);
-    cudaFuncSetAttribute(select_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    select_tc_kernel<<<grid, NTHREADS, smem, st>>>(tq, A, kbar, amax, exitn, idx, tiles, dev_flag);
+    // the erf prior is a separate instantiation: without it the unrolled score loop stays small
+    auto kern = P.has_prior ? select_tc_kernel<true> : select_tc_kernel<false>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    kern<<<grid, NTHREADS, smem, st>>>(tq, A, kbar, amax, exitn, idx, tiles, dev_flag);
     return cudaGetLastError();
 }
 
