@@ -36,6 +36,7 @@ struct SelSmem {
     int ulist[UMAX];
     float acell[UMAX];                     // a_c of the union cells (prior)
     uint8_t amask[UMAX];                   // bit g: admitted for prefix n_min + g
+    uint32_t admit[5][UMAX / 32];          // per prefix n_min + g: admitted union positions
     int warp_cnt[4];
     int nU;
     uint64_t q_full, kb_ready, s_full, drain;
@@ -199,6 +200,14 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
         }
         sel_sync();
         const int nU = min(total, UMAX);
+        {   // admission masks per prefix, one 32-position word per warp
+            const uint32_t am = t < nU ? sm.amask[t] : 0u;
+#pragma unroll
+            for (int gg = 0; gg < 5; gg++) {
+                const uint32_t word = __ballot_sync(kFull, (am >> gg) & 1u);
+                if (lane == 0) sm.admit[gg][warp] = word;
+            }
+        }
         // ---- kbar of U as three bf16 parts, row u = union position (zero rows pad to 16)
         const int N = max(16, (nU + 15) & ~15);
         if (t < N) {
@@ -236,9 +245,14 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
             const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
             const float lam = PRIOR ? A.lambda[h] : 0.f;
             const float i2s = PRIOR ? A.inv2sigma[h] : 0.f;
+            uint32_t aw[UMAX / 32];                 // admitted union positions of this row
+#pragma unroll
+            for (int b = 0; b < UMAX / 32; b++) aw[b] = row < nrows ? sm.admit[g][b] : 0u;
+            const int na = __popc(aw[0]) + __popc(aw[1]) + __popc(aw[2]) + __popc(aw[3]);
             uint32_t key[UMAX];
-            uint32_t kmin = 0xffffffffu, kmax = 0u;
-            int na = 0;
+            uint32_t kmn[8], kmx[8];
+#pragma unroll
+            for (int k = 0; k < 8; k++) { kmn[k] = 0xffffffffu; kmx[k] = 0u; }
 #pragma unroll
             for (int b = 0; b < UMAX / 32; b++) {
                 if (32 * b < N) {
@@ -248,31 +262,40 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
 #pragma unroll
                     for (int e = 0; e < 32; e++) {
                         const int u = 32 * b + e;
-                        uint32_t k = 0u;
-                        if (u < nU && ((sm.amask[u] >> g) & 1u) && row < nrows) {
-                            float sc = __uint_as_float(r[e]) * A.scale;
-                            if (PRIOR) {
-                                const float pc = (float)(sm.ulist[u] * kS) + 0.5f * kS;
-                                sc += lam * sm.acell[u] * erff(((float)i - pc) * i2s);
-                            }
-                            k = (order_key(sc) & ~0x7fu) | (uint32_t)(127 - u);
-                            kmin = min(kmin, k);
-                            kmax = max(kmax, k);
-                            na++;
+                        float sc = __uint_as_float(r[e]) * A.scale;
+                        if (PRIOR) {
+                            const float pc = (float)(sm.ulist[u] * kS) + 0.5f * kS;
+                            sc += lam * sm.acell[u] * erff(((float)i - pc) * i2s);
                         }
+                        const uint32_t k = ((aw[b] >> e) & 1u) ? (order_key(sc) & ~0x7fu) | (uint32_t)(127 - u) : 0u;
                         key[u] = k;
+                        kmn[e & 7] = min(kmn[e & 7], k ? k : 0xffffffffu);
+                        kmx[e & 7] = max(kmx[e & 7], k);
                     }
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; e++) key[32 * b + e] = 0u;
                 }
             }
-            // K-th largest key: count(key >= lo) >= K > count(key >= hi)
+            const uint32_t kmin = min(min(min(kmn[0], kmn[1]), min(kmn[2], kmn[3])), min(min(kmn[4], kmn[5]), min(kmn[6], kmn[7])));
+            const uint32_t kmax = max(max(max(kmx[0], kmx[1]), max(kmx[2], kmx[3])), max(max(kmx[4], kmx[5]), max(kmx[6], kmx[7])));
+            // K-th largest key: keep count(key >= lo) = clo >= K > chi = count(key >= hi).
+            // Interpolate the next probe on the counts; a probe that fails to halve the
+            // bracket is followed by a plain bisection step (logarithmic worst case).
             uint32_t tau = 1u;
             if (na > A.K) {
-                uint32_t lo = kmin, hi = kmax + 1u;       // count(>= kmin) = na > K, count(>= kmax+1) = 0
+                uint32_t lo = kmin, hi = kmax + 1u;
+                int clo = na, chi = 0;
+                bool bisect = false;
                 while (hi - lo > 1u) {
-                    const uint32_t mid = lo + ((hi - lo) >> 1);
+                    uint32_t mid;
+                    if (bisect) {
+                        mid = lo + ((hi - lo) >> 1);
+                    } else {
+                        const uint64_t span = hi - lo;
+                        mid = lo + (uint32_t)(span * (uint64_t)(clo - A.K) / (uint64_t)(clo - chi));
+                        mid = min(max(mid, lo + 1u), hi - 1u);
+                    }
                     int cp[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent partial counts
 #pragma unroll
                     for (int b = 0; b < UMAX / 32; b++)
@@ -281,12 +304,16 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                             for (int e = 0; e < 32; e++) cp[e & 7] += key[32 * b + e] >= mid;
                         }
                     const int cnt = ((cp[0] + cp[1]) + (cp[2] + cp[3])) + ((cp[4] + cp[5]) + (cp[6] + cp[7]));
+                    const uint32_t before = hi - lo;
                     if (cnt >= A.K) {
                         lo = mid;
+                        clo = cnt;
                         if (cnt == A.K) break;
                     } else {
                         hi = mid;
+                        chi = cnt;
                     }
+                    bisect = !bisect && (hi - lo) > (before >> 1);
                 }
                 tau = lo;
             }
