@@ -121,9 +121,7 @@ __device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, boo
         for (int e = 0; e < 16; e++) {
             const int j = 32 * q + 2 * e;
             const float p0 = tc::ex2(fmaf(__uint_as_float(s[j]), c_log2, -msub));
-            // one exponential in four on the FMA pipe: the MUFU unit is the softmax's limit
-            const float x1 = fmaf(__uint_as_float(s[j + 1]), c_log2, -msub);
-            const float p1 = (e & 1) ? tc::ex2_poly(x1) : tc::ex2(x1);
+            const float p1 = tc::ex2(fmaf(__uint_as_float(s[j + 1]), c_log2, -msub));
             ls[e & 7] += p0 + p1;
             pk[e] = tc::pack_bf16x2(p0, p1);
         }

@@ -279,23 +279,12 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
             }
             const uint32_t kmin = min(min(min(kmn[0], kmn[1]), min(kmn[2], kmn[3])), min(min(kmn[4], kmn[5]), min(kmn[6], kmn[7])));
             const uint32_t kmax = max(max(max(kmx[0], kmx[1]), max(kmx[2], kmx[3])), max(max(kmx[4], kmx[5]), max(kmx[6], kmx[7])));
-            // K-th largest key: keep count(key >= lo) = clo >= K > chi = count(key >= hi).
-            // Interpolate the next probe on the counts; a probe that fails to halve the
-            // bracket is followed by a plain bisection step (logarithmic worst case).
+            // K-th largest key by bisection: count(key >= lo) >= K > count(key >= hi)
             uint32_t tau = 1u;
             if (na > A.K) {
                 uint32_t lo = kmin, hi = kmax + 1u;
-                int clo = na, chi = 0;
-                bool bisect = false;
                 while (hi - lo > 1u) {
-                    uint32_t mid;
-                    if (bisect) {
-                        mid = lo + ((hi - lo) >> 1);
-                    } else {
-                        const uint64_t span = hi - lo;
-                        mid = lo + (uint32_t)(span * (uint64_t)(clo - A.K) / (uint64_t)(clo - chi));
-                        mid = min(max(mid, lo + 1u), hi - 1u);
-                    }
+                    const uint32_t mid = lo + ((hi - lo) >> 1);
                     int cp[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent partial counts
 #pragma unroll
                     for (int b = 0; b < UMAX / 32; b++)
@@ -304,16 +293,12 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                             for (int e = 0; e < 32; e++) cp[e & 7] += key[32 * b + e] >= mid;
                         }
                     const int cnt = ((cp[0] + cp[1]) + (cp[2] + cp[3])) + ((cp[4] + cp[5]) + (cp[6] + cp[7]));
-                    const uint32_t before = hi - lo;
                     if (cnt >= A.K) {
                         lo = mid;
-                        clo = cnt;
                         if (cnt == A.K) break;
                     } else {
                         hi = mid;
-                        chi = cnt;
                     }
-                    bisect = !bisect && (hi - lo) > (before >> 1);
                 }
                 tau = lo;
             }

@@ -214,22 +214,6 @@ __device__ __forceinline__ float ex2(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-// 2^x on the FMA pipe, for x <= 8, to take load off the MUFU unit: x = n + f with
-// n = round(x) (added to the exponent field) and f in [-1/2, 1/2], where 2^f is the cubic
-// interpolating it at the four Chebyshev nodes of [-1/2, 1/2] (coefficients fitted for this
-// library; max relative error 1.0e-4, below the 2^-9 rounding of the bf16 P it feeds).
-// Arguments below -125 (including -inf for masked columns) give 0.
-__device__ __forceinline__ float ex2_poly(float x) {
-    const float xc = fmaxf(x, -125.f);
-    const float t = xc + 12582912.f;                // 1.5 * 2^23: low bits hold round(xc)
-    const float f = xc - (t - 12582912.f);
-    const float p = fmaf(fmaf(fmaf(0.05583828294622033f, f, 0.24263947854625836f), f, 0.6931367338836214f), f,
-                         0.9999245569508708f);
-    const int n = __float_as_int(t) - 0x4B400000;
-    const float r = __int_as_float(__float_as_int(p) + n * (1 << 23));
-    return x < -125.f ? 0.f : r;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
