@@ -77,33 +77,36 @@ __device__ __forceinline__ void ld_row128(uint32_t taddr, uint32_t (&s)[128]) {
 enum ChunkKind { FULL = 0, CELLS = 1, BAND = 2 };
 
 // One chunk of online softmax for this thread's row.  S is read from TMEM columns
-// [S_COL, S_COL+128) in one batch; invalid columns become -inf (the max ignores them and
-// exp2 turns them into 0), so the rest is one body for every kind of chunk.  P =
-// exp2(S*c - m) is written back as bf16 pairs over [S_COL, S_COL+64).  The running max m
-// (log2 units) is raised only when a chunk exceeds it by more than 8 (lazy rescale of O).
-// Maxima and sums use eight independent partial accumulators (no long dependency chain).
+// [S_COL, S_COL+128) in one batch.  Invalid columns must contribute exp2(-inf) = 0: a BAND
+// chunk sets them to -inf one by one; a CELLS chunk drops the 32-column block of an
+// unselected cell from the max and adds an exponent bias of -inf to the whole block, so
+// the exponentials of every kind of chunk share one body.  P = exp2(S*c - m) is written
+// back as bf16 pairs over [S_COL, S_COL+64).  The running max m (log2 units) is raised
+// only when a chunk exceeds it by more than 8 (lazy rescale of O).  The arithmetic is
+// paired (f32x2 FMA and add, three-input max) with independent partial accumulators:
+// the softmax warps are issue-bound, so instructions per element set the chunk time.
 __device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, bool first, int kind, uint32_t sel4,
                                            int lo, int width, float c_log2, float &m_used, float &l) {
     uint32_t s[128];
     ld_row128(trow + S_COL, s);
-    if (kind == CELLS) {
-#pragma unroll
-        for (int b = 0; b < BN / 32; b++)
-            if (!((sel4 >> b) & 1u)) {
-#pragma unroll
-                for (int e = 0; e < 32; e++) s[32 * b + e] = 0xff800000u;
-            }
-    } else if (kind == BAND) {
+    if (kind == BAND) {
 #pragma unroll
         for (int j = 0; j < BN; j++)
             if ((unsigned)(j - lo) >= (unsigned)width) s[j] = 0xff800000u;
     }
-    float mp[8];
+    float mx = -INFINITY;
+    bool valid[BN / 32];
 #pragma unroll
-    for (int k = 0; k < 8; k++) mp[k] = -INFINITY;
+    for (int b = 0; b < BN / 32; b++) {           // block maximum: four three-input chains
+        float a[4];
 #pragma unroll
-    for (int j = 0; j < BN; j++) mp[j & 7] = fmaxf(mp[j & 7], __uint_as_float(s[j]));
-    float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+        for (int k = 0; k < 4; k++) a[k] = __uint_as_float(s[32 * b + k]);
+#pragma unroll
+        for (int j = 4; j < 32; j += 2)
+            a[(j >> 1) & 3] = tc::max3(a[(j >> 1) & 3], __uint_as_float(s[32 * b + j]), __uint_as_float(s[32 * b + j + 1]));
+        valid[b] = kind != CELLS || ((sel4 >> b) & 1u);
+        mx = valid[b] ? tc::max3(mx, fmaxf(a[0], a[1]), fmaxf(a[2], a[3])) : mx;
+    }
     mx *= c_log2;
     const bool grow = mx > m_used + 8.f;
     const float m_new = grow ? mx : m_used;
@@ -111,23 +114,31 @@ __device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, boo
     l *= corr;
     m_used = m_new;
     const float msub = m_used == -INFINITY ? 0.f : m_used;
-    float ls[8];
+    const uint64_t c2 = tc::f2_pack(c_log2, c_log2);
+    uint64_t ls[4];
 #pragma unroll
-    for (int k = 0; k < 8; k++) ls[k] = 0.f;
+    for (int k = 0; k < 4; k++) ls[k] = tc::f2_pack(0.f, 0.f);
 #pragma unroll
     for (int q = 0; q < 4; q++) {                    // P keys [32 q, 32 q + 32) -> 16 columns
+        const float nb = valid[q] ? -msub : -INFINITY;
+        const uint64_t nb2 = tc::f2_pack(nb, nb);
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; e++) {
             const int j = 32 * q + 2 * e;
-            const float p0 = tc::ex2(fmaf(__uint_as_float(s[j]), c_log2, -msub));
-            const float p1 = tc::ex2(fmaf(__uint_as_float(s[j + 1]), c_log2, -msub));
-            ls[e & 7] += p0 + p1;
+            float x0, x1;
+            tc::f2_unpack(tc::f2_fma(tc::f2_pack(__uint_as_float(s[j]), __uint_as_float(s[j + 1])), c2, nb2), x0, x1);
+            const float p0 = tc::ex2(x0), p1 = tc::ex2(x1);
+            ls[e & 3] = tc::f2_add(ls[e & 3], tc::f2_pack(p0, p1));
             pk[e] = tc::pack_bf16x2(p0, p1);
         }
         tc::tmem_st16(trow + S_COL + 16 * q, pk);
     }
-    l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+    {
+        float a, b;
+        tc::f2_unpack(tc::f2_add(tc::f2_add(ls[0], ls[1]), tc::f2_add(ls[2], ls[3])), a, b);
+        l += a + b;
+    }
     // O rescale after the exponentials, when S no longer occupies registers (no MMA
     // touches O until this thread arrives on p_full)
     if (!first && __any_sync(kFull, corr != 1.f)) {
@@ -313,7 +324,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
         const uint4 m4 = __ldg(reinterpret_cast<const uint4 *>(
             tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords + kTileMaskOff + 4 * row));
-        const uint32_t mw[UMAX / 32] = {m4.x, m4.y, m4.z, m4.w};   // selected union positions
         bool ok = tc::mbar_wait(&sm.u_ready, 0, ab);
         const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0, total = nR + nW;
         float m_lr = -INFINITY, l_lr = 0.f, m_sr = -INFINITY, l_sr = 0.f;
@@ -348,7 +358,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             float m, l;
             if (it < nR) {
                 const int p0 = CPC * it;
-                sel4 = (mw[p0 >> 5] >> (p0 & 31)) & 0xfu;
+                const int wsel = p0 >> 5;           // word of the row's union mask, in registers
+                const uint32_t mw = wsel == 0 ? m4.x : wsel == 1 ? m4.y : wsel == 2 ? m4.z : m4.w;
+                sel4 = (mw >> (p0 & 31)) & 0xfu;
                 kind = CELLS; ocol = OLR_COL; first = it == 0; m = m_lr; l = l_lr;
             } else {
                 const int jc = jbase + BN * (k_first + it - nR);
