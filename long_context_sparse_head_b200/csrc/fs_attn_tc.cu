@@ -8,33 +8,36 @@
 // admitted cells and, per row, the positions in U it selected).
 //
 // One CTA per 128 query rows of a (batch, head); two CTAs per SM.  The readout runs over
-// U (|U| <= 128, ascending), four cells
-// (128 keys) per chunk, each cell fetched by its own 32-row TMA box; a row masks the
-// cells it did not select (masked-dense on the tensor cores).  Then the window runs
-// over 128-key chunks.  Both softmaxes accumulate in tensor memory: S/P in columns
-// [0,128), the readout's O in [128,192), the window's O in [192,256).  When the first
-// window chunk arrives the readout is finished: the softmax threads turn its O into
-// alpha_h * RMSNorm(u) in place, and the epilogue adds it to the window's output.  No
-// intermediate leaves the SM.
+// U (|U| <= 128, ascending), two cells (64 keys) per chunk, each cell fetched by its own
+// 32-row TMA box; a row masks the cells it did not select (masked-dense on the tensor
+// cores).  Then the window runs over 64-key chunks.  Both softmaxes accumulate in tensor
+// memory: two S buffers in columns [0,64) and [64,128) (chunk c uses buffer c mod 2, and
+// its P overwrites the first 32 columns of that buffer), the readout's O in [128,192), the
+// window's O in [192,256).  With two S buffers the MMA warp computes S of chunk c+1 while
+// the softmax threads work on chunk c, and a softmax warp that finishes early can start
+// the next chunk while slower warps finish this one.  When the first window chunk arrives
+// the readout is finished: the softmax threads turn its O into alpha_h * RMSNorm(u) in
+// place, and the epilogue adds it to the window's output.  No intermediate leaves the SM.
 //
 // Warpgroup 0 (warps 0-3): softmax, thread = query row = TMEM lane; it holds a chunk's
-// whole 128-column S row in registers (one TMEM wait per chunk), raised to 200 registers
-// by setmaxnreg.  Warpgroup 1 (lowered to 56): warp 4 TMA, warp 5 MMA, warps 6-7
-// auxiliary (stage U, rotate Q by its absolute positions).  The window's keys come
-// pre-rotated (absolute positions, double-precision angles) from a workspace copy.
+// S row in registers (one TMEM wait per chunk), raised to 200 registers by setmaxnreg.
+// Warpgroup 1 (lowered to 56): warp 4 TMA, warp 5 MMA, warps 6-7 auxiliary (stage U,
+// rotate Q by its absolute positions).  The window's keys come pre-rotated (absolute
+// positions, double-precision angles) from a workspace copy.
 #include "tc_rope.cuh"
 
 namespace fs {
 
 namespace {
-constexpr int BM = 128, BN = 128, NSTAGE = 2;
+constexpr int BM = 128, BN = 64, NSTAGE = 4;
 constexpr int UMAX = 128;                        // largest union of selected cells per tile
-constexpr int CPC = BN / kS;                     // cells per readout chunk (4)
-constexpr int W_TMA = 4, W_MMA = 5, W_AUX0 = 6, NWARPS = 8, NAUX = 64;
+constexpr int CPC = BN / kS;                     // cells per readout chunk (2)
+constexpr int NSOFT = 4, W_TMA = 4, W_MMA = 5, W_AUX0 = 6, NWARPS = 8, NAUX = 64;
 constexpr int NTHREADS = NWARPS * 32;
 constexpr int REGS_SOFTMAX = 200, REGS_PRODUCER = 56;   // 128 * (200 + 56) = 256 * 128
-constexpr uint32_t TMEM_COLS = 256, S_COL = 0, OLR_COL = 128, OSR_COL = 192;
+constexpr uint32_t TMEM_COLS = 256, OLR_COL = 128, OSR_COL = 192;   // S buffers at 0 and BN
 constexpr int TILE_BYTES = BM * kD * 2;         // 128 x 64 bf16: 16 KiB
+constexpr int CHUNK_BYTES = BN * kD * 2;        // 64 x 64 bf16: 8 KiB
 constexpr int CELL_BYTES = kS * kD * 2;         // 32 x 64 bf16: 4 KiB
 constexpr int kAuxBarrier = 1;                  // named barrier of the auxiliary threads
 
@@ -45,7 +48,8 @@ struct AttnSmem {
     __nv_bfloat16 v[NSTAGE][BN * kD];
     int ulist[UMAX];                            // union cells, ascending
     int nU;
-    uint64_t q_full, q_ready, u_ready, s_full, p_full, o_done, drain;
+    uint64_t q_full, q_ready, u_ready, o_ready, o_done, drain;
+    uint64_t s_full[2], p_full[2];              // per S buffer
     uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
     uint32_t tmem_base;
     int abort;
@@ -62,33 +66,26 @@ struct AttnArgs {
 __device__ __forceinline__ void aux_sync() {
     asm volatile("bar.sync %0, %1;" ::"n"(kAuxBarrier), "n"(NAUX) : "memory");
 }
-
-__device__ __forceinline__ void ld_row128(uint32_t taddr, uint32_t (&s)[128]) {
-    tc::tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-    tc::tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-    tc::tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-    tc::tmem_ld32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-    tc::tmem_wait_ld();
-}
-
 // Column validity of a chunk: every column (FULL), the columns of the selected cells
-// (CELLS: 32-column block b valid iff bit b of sel4), or a band of the window (BAND:
+// (CELLS: 32-column block b valid iff bit b of sel), or a band of the window (BAND:
 // lo <= j < lo + width).
 enum ChunkKind { FULL = 0, CELLS = 1, BAND = 2 };
 
-// One chunk of online softmax for this thread's row.  S is read from TMEM columns
-// [S_COL, S_COL+128) in one batch.  Invalid columns must contribute exp2(-inf) = 0: a BAND
-// chunk sets them to -inf one by one; a CELLS chunk drops the 32-column block of an
+// One chunk of online softmax for this thread's row, on the S buffer at TMEM address tS
+// (BN columns, read in one batch).  Invalid columns must contribute exp2(-inf) = 0: a
+// BAND chunk sets them to -inf one by one; a CELLS chunk drops the 32-column block of an
 // unselected cell from the max and adds an exponent bias of -inf to the whole block, so
 // the exponentials of every kind of chunk share one body.  P = exp2(S*c - m) is written
-// back as bf16 pairs over [S_COL, S_COL+64).  The running max m (log2 units) is raised
-// only when a chunk exceeds it by more than 8 (lazy rescale of O).  The arithmetic is
-// paired (f32x2 FMA and add, three-input max) with independent partial accumulators:
-// the softmax warps are issue-bound, so instructions per element set the chunk time.
-__device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, bool first, int kind, uint32_t sel4,
-                                           int lo, int width, float c_log2, float &m_used, float &l) {
-    uint32_t s[128];
-    ld_row128(trow + S_COL, s);
+// back as bf16 pairs over the buffer's first BN/2 columns.  The running max m (log2
+// units) is raised only when a chunk exceeds it by more than 8 (lazy rescale of O); the
+// factor O must be multiplied by is returned (1 when m stayed).  The arithmetic is paired
+// (f32x2 FMA and add, three-input max) with independent partial accumulators.
+__device__ __forceinline__ float softmax_chunk(uint32_t tS, int kind, uint32_t sel, int lo, int width,
+                                               float c_log2, float &m_used, float &l) {
+    uint32_t s[BN];
+    tc::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+    tc::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+    tc::tmem_wait_ld();
     if (kind == BAND) {
 #pragma unroll
         for (int j = 0; j < BN; j++)
@@ -104,7 +101,7 @@ __device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, boo
 #pragma unroll
         for (int j = 4; j < 32; j += 2)
             a[(j >> 1) & 3] = tc::max3(a[(j >> 1) & 3], __uint_as_float(s[32 * b + j]), __uint_as_float(s[32 * b + j + 1]));
-        valid[b] = kind != CELLS || ((sel4 >> b) & 1u);
+        valid[b] = kind != CELLS || ((sel >> b) & 1u);
         mx = valid[b] ? tc::max3(mx, fmaxf(a[0], a[1]), fmaxf(a[2], a[3])) : mx;
     }
     mx *= c_log2;
@@ -119,7 +116,7 @@ __device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, boo
 #pragma unroll
     for (int k = 0; k < 4; k++) ls[k] = tc::f2_pack(0.f, 0.f);
 #pragma unroll
-    for (int q = 0; q < 4; q++) {                    // P keys [32 q, 32 q + 32) -> 16 columns
+    for (int q = 0; q < BN / 32; q++) {              // P keys [32 q, 32 q + 32) -> 16 columns
         const float nb = valid[q] ? -msub : -INFINITY;
         const uint64_t nb2 = tc::f2_pack(nb, nb);
         uint32_t pk[16];
@@ -132,34 +129,19 @@ __device__ __forceinline__ void softmax_chunk(uint32_t trow, uint32_t o_col, boo
             ls[e & 3] = tc::f2_add(ls[e & 3], tc::f2_pack(p0, p1));
             pk[e] = tc::pack_bf16x2(p0, p1);
         }
-        tc::tmem_st16(trow + S_COL + 16 * q, pk);
+        tc::tmem_st16(tS + 16 * q, pk);
     }
-    {
-        float a, b;
-        tc::f2_unpack(tc::f2_add(tc::f2_add(ls[0], ls[1]), tc::f2_add(ls[2], ls[3])), a, b);
-        l += a + b;
-    }
-    // O rescale after the exponentials, when S no longer occupies registers (no MMA
-    // touches O until this thread arrives on p_full)
-    if (!first && __any_sync(kFull, corr != 1.f)) {
-#pragma unroll
-        for (int b = 0; b < kD / 32; b++) {
-            uint32_t r[32];
-            tc::tmem_ld32(trow + o_col + 32 * b, r);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; e++) r[e] = __float_as_uint(__uint_as_float(r[e]) * corr);
-            tc::tmem_st32(trow + o_col + 32 * b, r);
-        }
-    }
-    tc::tmem_wait_st();
+    float u, v;
+    tc::f2_unpack(tc::f2_add(tc::f2_add(ls[0], ls[1]), tc::f2_add(ls[2], ls[3])), u, v);
+    l += u + v;
+    return corr;
 }
 }  // namespace
 
 __global__ void __launch_bounds__(NTHREADS, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk32,
-               const __grid_constant__ CUtensorMap tv32, const __grid_constant__ CUtensorMap tkr128,
-               const __grid_constant__ CUtensorMap tv128, const AttnArgs A,
+               const __grid_constant__ CUtensorMap tv32, const __grid_constant__ CUtensorMap tkr64,
+               const __grid_constant__ CUtensorMap tv64, const AttnArgs A,
                const uint32_t *__restrict__ tiles, const float2 *__restrict__ rope_lo,
                const float2 *__restrict__ rope_hi, __nv_bfloat16 *__restrict__ O, int *dev_flag) {
     extern __shared__ uint8_t smraw[];
@@ -181,9 +163,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         tc::mbar_init(&sm.q_full, 1);
         tc::mbar_init(&sm.q_ready, NAUX);
         tc::mbar_init(&sm.u_ready, NAUX);
-        tc::mbar_init(&sm.s_full, 1);
-        tc::mbar_init(&sm.p_full, 128);
+        tc::mbar_init(&sm.o_ready, 1);
         tc::mbar_init(&sm.o_done, 1);
+        for (int b = 0; b < 2; b++) {
+            tc::mbar_init(&sm.s_full[b], 1);
+            tc::mbar_init(&sm.p_full[b], NSOFT);       // one arrival per softmax warp
+        }
         tc::mbar_init(&sm.drain, 1);
         for (int s = 0; s < NSTAGE; s++) {
             tc::mbar_init(&sm.kv_full[s], 1);
@@ -200,15 +185,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp >= 4) {
+    if (warp >= NSOFT) {
         tc::regs_dec<REGS_PRODUCER>();
         if (warp == W_TMA) {
             if (lane == 0) {
                 tc::prefetch_tmap(&tq);
                 tc::prefetch_tmap(&tk32);
                 tc::prefetch_tmap(&tv32);
-                tc::prefetch_tmap(&tkr128);
-                tc::prefetch_tmap(&tv128);
+                tc::prefetch_tmap(&tkr64);
+                tc::prefetch_tmap(&tv64);
                 tc::mbar_expect_tx(&sm.q_full, TILE_BYTES);
                 tc::tma_load_3d(sm.qn, &tq, &sm.q_full, 0, r0, bh);
                 int it = 0;
@@ -217,7 +202,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     for (; it < total; it++) {
                         const int s = it % NSTAGE;
                         if (!tc::mbar_wait(&sm.kv_empty[s], ((it / NSTAGE) & 1) ^ 1, ab)) break;
-                        if (it < nR) {          // four gathered cells; unused slots read zeros
+                        if (it < nR) {          // two gathered cells; unused slots read zeros
                             tc::mbar_expect_tx(&sm.kv_full[s], 2 * CPC * CELL_BYTES);
                             for (int j = 0; j < CPC; j++) {
                                 const int u = CPC * it + j;
@@ -225,11 +210,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                                 tc::tma_load_3d(sm.k[s] + j * kS * kD, &tk32, &sm.kv_full[s], 0, y, bh);
                                 tc::tma_load_3d(sm.v[s] + j * kS * kD, &tv32, &sm.kv_full[s], 0, y, bh);
                             }
-                        } else {                // 128 consecutive keys of the band (K pre-rotated)
+                        } else {                // BN consecutive keys of the band (K pre-rotated)
                             const int jc = jbase + BN * (k_first + it - nR);
-                            tc::mbar_expect_tx(&sm.kv_full[s], 2 * TILE_BYTES);
-                            tc::tma_load_3d(sm.k[s], &tkr128, &sm.kv_full[s], 0, jc - A.kr0, bh);
-                            tc::tma_load_3d(sm.v[s], &tv128, &sm.kv_full[s], 0, jc, bh);
+                            tc::mbar_expect_tx(&sm.kv_full[s], 2 * CHUNK_BYTES);
+                            tc::tma_load_3d(sm.k[s], &tkr64, &sm.kv_full[s], 0, jc - A.kr0, bh);
+                            tc::tma_load_3d(sm.v[s], &tv64, &sm.kv_full[s], 0, jc, bh);
                         }
                     }
                 }
@@ -270,41 +255,47 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             if (lane == 0) {
                 const uint32_t id_qk = tc::idesc_bf16(BM, BN, false, false);
                 const uint32_t id_pv = tc::idesc_bf16(BM, kD, false, true);
-                const uint32_t qn = tc::smem_u32(sm.qn), qr = tc::smem_u32(sm.qr);
+                // descriptors computed once; a byte offset o moves the address field by o >> 4
+                const uint64_t dqn = tc::sdesc_sw128(tc::smem_u32(sm.qn), 16, 1024);
+                const uint64_t dqr = tc::sdesc_sw128(tc::smem_u32(sm.qr), 16, 1024);
+                const uint64_t dk0 = tc::sdesc_sw128(tc::smem_u32(sm.k[0]), 16, 1024);
+                const uint64_t dv0 = tc::sdesc_sw128(tc::smem_u32(sm.v[0]), 16, 1024);
+                constexpr uint32_t kStageStep = (BN * kD * 2) >> 4;
                 bool ok = tc::mbar_wait(&sm.u_ready, 0, ab) && tc::mbar_wait(&sm.q_full, 0, ab);
                 const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0, total = nR + nW;
                 int issued = 0;
-                for (int it = 0; ok && it <= total; it++) {
-                    if (it > 0) {   // O += P(it-1) V(it-1), into the readout's or the window's O
-                        if (!tc::mbar_wait(&sm.p_full, (it - 1) & 1, ab)) { ok = false; break; }
-                        tc::tc_fence_after();
-                        const int pj = it - 1;
-                        const uint32_t ocol = pj < nR ? OLR_COL : OSR_COL;
-                        const bool first = pj == 0 || pj == nR;
-                        const uint32_t vb = tc::smem_u32(sm.v[pj % NSTAGE]);
+                // S(c) = Q K(c)^T into buffer c mod 2, with the NoPE or the rotated Q
+                auto issue_qk = [&](int c) -> bool {
+                    if (!tc::mbar_wait(&sm.kv_full[c % NSTAGE], (c / NSTAGE) & 1, ab)) return false;
+                    if (c == nR && !tc::mbar_wait(&sm.q_ready, 0, ab)) return false;
+                    tc::tc_fence_after();
+                    const uint64_t da = c < nR ? dqn : dqr;
+                    const uint64_t db = dk0 + (uint64_t)((c % NSTAGE) * kStageStep);
 #pragma unroll
-                        for (int kk = 0; kk < BN / 16; kk++)
-                            tc::mma_ts(tmem + ocol, tmem + S_COL + kk * 8, tc::sdesc_sw128(vb + kk * 2048, 16, 1024),
-                                       id_pv, (!first || kk > 0) ? 1u : 0u);
-                        tc::mma_commit(&sm.kv_empty[pj % NSTAGE]);
-                        issued++;
-                    }
-                    if (it < total) {   // S = Q K(it)^T with the NoPE or the rotated Q
-                        if (!tc::mbar_wait(&sm.kv_full[it % NSTAGE], (it / NSTAGE) & 1, ab)) {
-                            ok = false;
-                            break;
-                        }
-                        if (it == nR && !tc::mbar_wait(&sm.q_ready, 0, ab)) { ok = false; break; }
-                        tc::tc_fence_after();
-                        const uint32_t qa = it < nR ? qn : qr;
-                        const uint32_t kb = tc::smem_u32(sm.k[it % NSTAGE]);
+                    for (int kk = 0; kk < kD / 16; kk++)      // K steps of 16 columns = 32 bytes
+                        tc::mma_ss(tmem + BN * (c & 1), da + 2 * kk, db + 2 * kk, id_qk, kk > 0 ? 1u : 0u);
+                    tc::mma_commit(&sm.s_full[c & 1]);
+                    issued++;
+                    return true;
+                };
+                if (ok && total > 0) ok = issue_qk(0);
+                for (int c = 0; ok && c < total; c++) {
+                    // S(c+1) goes into the other buffer while the softmax works on chunk c; the
+                    // buffer's previous P (chunk c-1) was consumed by a P V issued before this
+                    if (c + 1 < total && !issue_qk(c + 1)) { ok = false; break; }
+                    // O += P(c) V(c), into the readout's or the window's O
+                    if (!tc::mbar_wait(&sm.p_full[c & 1], (c >> 1) & 1, ab)) { ok = false; break; }
+                    tc::tc_fence_after();
+                    const uint32_t ocol = c < nR ? OLR_COL : OSR_COL;
+                    const bool first = c == 0 || c == nR;
+                    const uint64_t db = dv0 + (uint64_t)((c % NSTAGE) * kStageStep);
 #pragma unroll
-                        for (int kk = 0; kk < kD / 16; kk++)
-                            tc::mma_ss(tmem + S_COL, tc::sdesc_sw128(qa + kk * 32, 16, 1024),
-                                       tc::sdesc_sw128(kb + kk * 32, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
-                        tc::mma_commit(&sm.s_full);
-                        issued++;
-                    }
+                    for (int kk = 0; kk < BN / 16; kk++)      // K steps of 16 keys = 2048 bytes
+                        tc::mma_ts(tmem + ocol, tmem + BN * (c & 1) + 8 * kk, db + 128 * kk, id_pv,
+                                   (!first || kk > 0) ? 1u : 0u);
+                    tc::mma_commit(&sm.kv_empty[c % NSTAGE]);
+                    tc::mma_commit(&sm.o_ready);
+                    issued++;
                 }
                 if (ok) tc::mma_commit(&sm.o_done);
                 if (issued) {
@@ -328,9 +319,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0, total = nR + nW;
         float m_lr = -INFINITY, l_lr = 0.f, m_sr = -INFINITY, l_sr = 0.f;
         for (int it = 0; ok && it < total; it++) {
-            if (!tc::mbar_wait(&sm.s_full, it & 1, ab)) { ok = false; break; }
+            if (!tc::mbar_wait(&sm.s_full[it & 1], (it >> 1) & 1, ab)) { ok = false; break; }
             tc::tc_fence_after();
             if (it == nR && nR > 0) {   // readout done: O_lr <- alpha_h RMSNorm(O_lr / l)
+                // the last readout P V may still run (S of this chunk was issued before it)
+                if (!tc::mbar_wait(&sm.o_ready, (it - 1) & 1, ab)) { ok = false; break; }
+                tc::tc_fence_after();
                 uint32_t a[32], b[32];
                 tc::tmem_ld32(trow + OLR_COL, a);
                 tc::tmem_ld32(trow + OLR_COL + 32, b);
@@ -353,14 +347,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             }
             // one call site for every kind of chunk keeps the unrolled body in the code once
             int kind, lo = 0, width = BN;
-            uint32_t sel4 = 0u, ocol;
+            uint32_t sel = 0u, ocol;
             bool first;
             float m, l;
             if (it < nR) {
                 const int p0 = CPC * it;
                 const int wsel = p0 >> 5;           // word of the row's union mask, in registers
                 const uint32_t mw = wsel == 0 ? m4.x : wsel == 1 ? m4.y : wsel == 2 ? m4.z : m4.w;
-                sel4 = (mw >> (p0 & 31)) & 0xfu;
+                sel = (mw >> (p0 & 31)) & ((1u << CPC) - 1u);
                 kind = CELLS; ocol = OLR_COL; first = it == 0; m = m_lr; l = l_lr;
             } else {
                 const int jc = jbase + BN * (k_first + it - nR);
@@ -370,14 +364,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 kind = __all_sync(kFull, clo <= 0 && chi >= BN - 1 && rvalid) ? FULL : BAND;
                 ocol = OSR_COL; first = it == nR; m = m_sr; l = l_sr;
             }
-            softmax_chunk(trow, ocol, first, kind, sel4, lo, width, A.scale_log2e, m, l);
+            const float corr = softmax_chunk(trow + BN * (it & 1), kind, sel, lo, width, A.scale_log2e, m, l);
             if (it < nR) { m_lr = m; l_lr = l; } else { m_sr = m; l_sr = l; }
+            // O rescale, after the exponentials (S no longer occupies registers); the P V of
+            // the previous chunk, which accumulates into the same O, must have finished
+            if (!first && __any_sync(kFull, corr != 1.f)) {
+                if (!tc::mbar_wait(&sm.o_ready, (it - 1) & 1, ab)) { ok = false; break; }
+                tc::tc_fence_after();
+#pragma unroll
+                for (int b = 0; b < kD / 32; b++) {
+                    uint32_t r[32];
+                    tc::tmem_ld32(trow + ocol + 32 * b, r);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; e++) r[e] = __float_as_uint(__uint_as_float(r[e]) * corr);
+                    tc::tmem_st32(trow + ocol + 32 * b, r);
+                }
+            }
+            tc::tmem_wait_st();
             tc::tc_fence_before();
-            tc::mbar_arrive(&sm.p_full);
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sm.p_full[it & 1]);
         }
         if (ok && tc::mbar_wait(&sm.o_done, 0, ab)) {
             tc::tc_fence_after();
-            const size_t orow = ((size_t)bh * A.Nq + r0 + row) * kD;
             const float inv = l_sr > 0.f ? 1.f / l_sr : 0.f;
             uint32_t a[64], b[64];
             tc::tmem_ld32(trow + OSR_COL, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
@@ -388,7 +398,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             }
             tc::tmem_wait_ld();
             if (rvalid) {
-                uint4 *dst = reinterpret_cast<uint4 *>(O + orow);
+                uint4 *dst = reinterpret_cast<uint4 *>(O + ((size_t)bh * A.Nq + r0 + row) * kD);
 #pragma unroll
                 for (int q = 0; q < 8; q++) {
                     uint32_t w4[4];
@@ -429,12 +439,12 @@ cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const voi
     if (P.Nq == 0) return cudaSuccess;
     const int BH = P.B * P.H;
     const int kr0 = rope_first_key(P);
-    CUtensorMap tq, tk32, tv32, tkr128, tv128;
+    CUtensorMap tq, tk32, tv32, tkr64, tv64;
     if (!encode_tmap_3d_bf16(&tq, Q, kD, P.Nq, BH, kD, BM) ||
         !encode_tmap_3d_bf16(&tk32, K, kD, P.Nk, BH, kD, kS) ||
         !encode_tmap_3d_bf16(&tv32, V, kD, P.Nk, BH, kD, kS) ||
-        !encode_tmap_3d_bf16(&tkr128, Krot, kD, P.Nk - kr0, BH, kD, BN) ||
-        !encode_tmap_3d_bf16(&tv128, V, kD, P.Nk, BH, kD, BN))
+        !encode_tmap_3d_bf16(&tkr64, Krot, kD, P.Nk - kr0, BH, kD, BN) ||
+        !encode_tmap_3d_bf16(&tv64, V, kD, P.Nk, BH, kD, BN))
         return cudaErrorInvalidValue;
     AttnArgs A;
     A.Nq = P.Nq; A.Nk = P.Nk; A.q0 = P.q0; A.w = P.w; A.C = P.C; A.K = P.K; A.H = P.H;
@@ -446,7 +456,7 @@ cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const voi
     const dim3 grid((P.Nq + BM - 1) / BM, BH);
     LaunchScope scope(kAttnTc, st);
     cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_tc_kernel<<<grid, NTHREADS, smem, st>>>(tq, tk32, tv32, tkr128, tv128, A, tiles, rope_lo, rope_hi,
+    attn_tc_kernel<<<grid, NTHREADS, smem, st>>>(tq, tk32, tv32, tkr64, tv64, A, tiles, rope_lo, rope_hi,
                                                  (__nv_bfloat16 *)O, dev_flag);
     return cudaGetLastError();
 }
