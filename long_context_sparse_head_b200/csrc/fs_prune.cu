@@ -7,11 +7,17 @@
 // or "never" if fewer than P cells beat it.  This kernel tabulates exit(c) once per
 // head; the selection kernels then test membership of any prefix in O(1).
 //
-// One warp per cell scans the head's a values 32 at a time (coalesced, L2-resident),
-// counting beating cells with a ballot, and stops at the P-th.
+// One warp per cell scans the head's a values 256 at a time (eight independent coalesced
+// loads per lane in flight, L2-resident), counting beating cells with a ballot per
+// 32-cell block in index order, and stops at the P-th.  The cells with the largest a scan
+// the whole head, so the kernel's time is set by those scans' round trips to L2.
 #include "fs_common.cuh"
 
 namespace fs {
+
+namespace {
+constexpr int kScanBlocks = 8;                   // 32-cell blocks loaded per round trip
+}
 
 __global__ void __launch_bounds__(256) exit_times_kernel(const float *__restrict__ amax,
                                                          int *__restrict__ exitn,
@@ -28,30 +34,202 @@ __global__ void __launch_bounds__(256) exit_times_kernel(const float *__restrict
         ex = c + 1;
     } else {
         int count = 0;
-        for (int base = 0; base < C; base += 32) {
-            const int cp = base + lane;
-            bool beats = false;
-            if (cp < C && cp != c) {
-                const float b = a[cp];
-                beats = (b > ac) || (b == ac && cp < c);
+        bool found = false;
+        for (int base = 0; base < C && !found; base += 32 * kScanBlocks) {
+            float b[kScanBlocks];
+#pragma unroll
+            for (int k = 0; k < kScanBlocks; k++) {
+                const int cp = base + 32 * k + lane;
+                b[k] = cp < C ? __ldg(a + cp) : 0.f;
             }
-            unsigned m = __ballot_sync(kFull, beats);
-            const int pc = __popc(m);
-            if (count + pc >= P) {
-                for (int k = P - count; k > 1; k--) m &= m - 1;   // drop lower set bits
-                const int cP = base + __ffs(m) - 1;                 // the P-th beating cell
-                ex = max(c + 1, cP + 1);
-                break;
+#pragma unroll
+            for (int k = 0; k < kScanBlocks; k++) {
+                const int cp = base + 32 * k + lane;
+                const bool beats = cp < C && cp != c && ((b[k] > ac) || (b[k] == ac && cp < c));
+                unsigned m = __ballot_sync(kFull, beats);
+                const int pc = __popc(m);
+                if (!found && count + pc >= P) {
+                    for (int r = P - count; r > 1; r--) m &= m - 1;   // drop lower set bits
+                    const int cP = base + 32 * k + __ffs(m) - 1;      // the P-th beating cell
+                    ex = max(c + 1, cP + 1);
+                    found = true;
+                }
+                count += pc;
             }
-            count += pc;
         }
     }
     if (lane == 0) exitn[cell] = ex;
 }
 
+// Exit times for a call whose queries span few prefixes (decode: Nq queries cover about
+// Nq / s + 1 prefixes of an archive of C cells).  Only prefixes n in [n_lo, n_hi] are
+// ever asked, so the table only has to be right there: TopP(n_lo) comes from a radix
+// select over [0, n_lo), and each later prefix n adds the one cell c = n - 1, which
+// enters TopP(n) iff it beats the weakest member (larger a; a tie goes to the lower
+// index, i.e. to the member), evicting that member at n.  Members get exit = the prefix
+// that evicts them (never, if none in range); every other cell gets c + 1, which makes
+// c < n < exit(c) false for every n >= n_lo.  One CTA per (b, h).
+namespace {
+constexpr int kRangeThreads = 512;
+constexpr int kRangeMaxSteps = 128;              // largest n_hi - n_lo this kernel takes
+
+// order-preserving integer key of a float (larger float, larger key)
+__device__ __forceinline__ uint32_t order_key(float a) {
+    const uint32_t b = __float_as_uint(a);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+}  // namespace
+
+__global__ void __launch_bounds__(kRangeThreads) topp_range_kernel(const float *__restrict__ amax,
+                                                                   int *__restrict__ exitn, int C, int P,
+                                                                   int n_lo, int n_hi) {
+    extern __shared__ uint32_t list[];           // TopP members: keys [P], then cells [P]
+    __shared__ int hist[256];
+    __shared__ int wsum[kRangeThreads / 32];
+    __shared__ uint32_t s_prefix;
+    __shared__ int s_remaining, s_count;
+    uint32_t *lkey = list;
+    int *lidx = reinterpret_cast<int *>(list + P);
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const float *a = amax + (size_t)blockIdx.x * C;
+    int *ex = exitn + (size_t)blockIdx.x * C;
+    for (int c = t; c < C; c += kRangeThreads) ex[c] = c + 1;
+    const int n0 = min(n_lo, C), m0 = min(P, n0);  // |TopP(n0)| = m0
+    if (t == 0) s_count = 0;
+    __syncthreads();
+    if (m0 > 0) {
+        // key tau of the m0-th largest a in [0, n0), and how many cells with key tau
+        // belong to TopP (the lowest-indexed ones)
+        const bool all = m0 == n0;
+        uint32_t tau = 0;
+        int remaining = m0;
+        if (!all) {
+            uint32_t mask = 0;
+            for (int shift = 24; shift >= 0; shift -= 8) {
+                for (int i = t; i < 256; i += kRangeThreads) hist[i] = 0;
+                __syncthreads();
+                for (int c = t; c < n0; c += kRangeThreads) {
+                    const uint32_t k = order_key(__ldg(a + c));
+                    if ((k & mask) == tau) atomicAdd(&hist[(k >> shift) & 255], 1);
+                }
+                __syncthreads();
+                if (warp == 0) {   // lane l holds digits 255 - 8l down to 248 - 8l
+                    int h[8], sum = 0;
+#pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        h[j] = hist[255 - 8 * lane - j];
+                        sum += h[j];
+                    }
+                    int incl = sum;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int v = __shfl_up_sync(kFull, incl, o);
+                        if (lane >= o) incl += v;
+                    }
+                    const int excl = incl - sum;
+                    if (excl < remaining && remaining <= incl) {
+                        int cum = excl, d = 255 - 8 * lane;
+#pragma unroll
+                        for (int j = 0; j < 8; j++) {
+                            if (cum + h[j] >= remaining) {
+                                d = 255 - 8 * lane - j;
+                                break;
+                            }
+                            cum += h[j];
+                        }
+                        s_prefix = tau | ((uint32_t)d << shift);
+                        s_remaining = remaining - cum;
+                    }
+                }
+                __syncthreads();
+                tau = s_prefix;
+                remaining = s_remaining;
+                mask |= 255u << shift;
+                __syncthreads();
+            }
+        }
+        // members of TopP(n0), in rounds of kRangeThreads cells in index order (the rank of
+        // a tau-valued cell among its equals decides ties)
+        int eq_before = 0;
+        for (int base = 0; base < n0; base += kRangeThreads) {
+            const int c = base + t;
+            uint32_t k = 0;
+            bool gt = false, eq = false;
+            if (c < n0) {
+                k = order_key(__ldg(a + c));
+                gt = all || k > tau;
+                eq = !all && k == tau;
+            }
+            const unsigned bal = __ballot_sync(kFull, eq);
+            if (lane == 0) wsum[warp] = __popc(bal);
+            __syncthreads();
+            int before = eq_before + __popc(bal & ((1u << lane) - 1u)), tot = 0;
+            for (int w2 = 0; w2 < kRangeThreads / 32; w2++) {
+                if (w2 < warp) before += wsum[w2];
+                tot += wsum[w2];
+            }
+            if (gt || (eq && before < remaining)) {
+                const int slot = atomicAdd(&s_count, 1);
+                lkey[slot] = k;
+                lidx[slot] = c;
+                ex[c] = kNever;
+            }
+            eq_before += tot;
+            __syncthreads();
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {   // prefixes n0 + 1 .. n_hi, one joining cell each
+        int cnt = s_count;
+        for (int n = n0 + 1; n <= n_hi && n <= C; n++) {
+            const int c = n - 1;
+            const uint32_t kc = order_key(__ldg(a + c));
+            if (cnt < P) {                       // fewer than P cells yet: all are members
+                if (lane == 0) {
+                    lkey[cnt] = kc;
+                    lidx[cnt] = c;
+                    ex[c] = kNever;
+                }
+                cnt++;
+                __syncwarp();
+                continue;
+            }
+            uint32_t wk = 0xffffffffu;           // weakest: smallest key, then highest cell
+            int wi = -1, ws = -1;
+            for (int j = lane; j < cnt; j += 32) {
+                const uint32_t kj = lkey[j];
+                const int ij = lidx[j];
+                if (kj < wk || (kj == wk && ij > wi)) { wk = kj; wi = ij; ws = j; }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const uint32_t k2 = __shfl_xor_sync(kFull, wk, o);
+                const int i2 = __shfl_xor_sync(kFull, wi, o), s2 = __shfl_xor_sync(kFull, ws, o);
+                if (k2 < wk || (k2 == wk && i2 > wi)) { wk = k2; wi = i2; ws = s2; }
+            }
+            if (kc > wk && lane == 0) {          // c enters TopP(n), the weakest leaves at n
+                ex[wi] = n;
+                lkey[ws] = kc;
+                lidx[ws] = c;
+                ex[c] = kNever;
+            }
+            __syncwarp();
+        }
+    }
+}
+
 cudaError_t launch_exit_times(const Dev &P, const float *amax, int *exitn, cudaStream_t st) {
     const long long ncell = (long long)P.B * P.H * P.C;
     if (ncell == 0) return cudaSuccess;
+    if (P.P > 0 && P.Nq > 0) {
+        const int n_lo = cand_count(P.q0, P.w, P.C), n_hi = cand_count(P.q0 + P.Nq - 1, P.w, P.C);
+        if (n_hi - n_lo <= kRangeMaxSteps) {
+            LaunchScope scope(kExitTimes, st);
+            topp_range_kernel<<<(unsigned)(P.B * P.H), kRangeThreads, (size_t)P.P * 8, st>>>(amax, exitn, P.C, P.P,
+                                                                                               n_lo, n_hi);
+            return cudaGetLastError();
+        }
+    }
     const int warps = 8;
     const long long blocks = (ncell + warps - 1) / warps;
     LaunchScope scope(kExitTimes, st);
