@@ -24,19 +24,19 @@
 namespace fs {
 
 namespace {
-constexpr int BM = 128, UMAX = 128;
-constexpr int W_TMA = 4, W_MMA = 5, NWARPS = 6, NTHREADS = NWARPS * 32;
+constexpr int BM = 128, UMAX = 128;              // largest union; UM = 80 or UMAX per launch
+constexpr int W_MMA = 4, NWARPS = 5, NTHREADS = NWARPS * 32;   // warp 4: Q load, then the MMA
 constexpr uint32_t TMEM_COLS = 128;
 constexpr int TILE_BYTES = BM * kD * 2;
 constexpr int kSelBarrier = 1;   // named barrier of the 128 selection threads
 
-struct SelSmem {
+template <int UM> struct SelSmem {       // UM: capacity of the union (a multiple of 16)
     __nv_bfloat16 q[BM * kD];              // Q tile (NoPE)
-    __nv_bfloat16 kb[3][UMAX * kD];        // kbar of U as hi, mid, lo bf16 parts
-    int ulist[UMAX];
-    float acell[UMAX];                     // a_c of the union cells (prior)
-    uint8_t amask[UMAX];                   // bit g: admitted for prefix n_min + g
-    uint32_t admit[5][UMAX / 32];          // per prefix n_min + g: admitted union positions
+    __nv_bfloat16 kb[3][UM * kD];          // kbar of U as hi, mid, lo bf16 parts
+    int ulist[UM];
+    float acell[UM];                       // a_c of the union cells (prior)
+    uint8_t amask[UM];                     // bit g: admitted for prefix n_min + g
+    uint32_t admit[5][(UM + 31) / 32];     // per prefix n_min + g: admitted union positions
     int warp_cnt[4];
     int nU;
     uint64_t q_full, kb_ready, s_full, drain;
@@ -69,14 +69,16 @@ __device__ __forceinline__ void split3(float x, __nv_bfloat16 &hi, __nv_bfloat16
 }
 }  // namespace
 
-template <bool PRIOR>
-__global__ void __launch_bounds__(NTHREADS, 2)
+// UM = 80 (|U| <= 80: three CTAs of five warps per SM, at most four warps per SM
+// sub-partition, so up to 128 registers) or 128 (two CTAs per SM)
+template <bool PRIOR, int UM>
+__global__ void __launch_bounds__(NTHREADS, UM <= 80 ? 3 : 2)
 select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const float *__restrict__ kbar,
                  const float *__restrict__ amax, const int *__restrict__ exitn,
                  int32_t *__restrict__ idx, uint32_t *__restrict__ tiles, int *dev_flag) {
     extern __shared__ uint8_t smraw[];
     const uint32_t sbase = tc::smem_u32(smraw);
-    SelSmem &sm = *reinterpret_cast<SelSmem *>(smraw + (((sbase + 1023u) & ~1023u) - sbase));
+    SelSmem<UM> &sm = *reinterpret_cast<SelSmem<UM> *>(smraw + (((sbase + 1023u) & ~1023u) - sbase));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.y, h = bh % A.H;
     const int r0 = blockIdx.x * BM;
@@ -103,14 +105,11 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == W_TMA) {
+    if (warp == W_MMA) {
         if (lane == 0) {
             tc::prefetch_tmap(&tq);
             tc::mbar_expect_tx(&sm.q_full, TILE_BYTES);
             tc::tma_load_3d(sm.q, &tq, &sm.q_full, 0, r0, bh);
-        }
-    } else if (warp == W_MMA) {
-        if (lane == 0) {
             bool ok = tc::mbar_wait(&sm.kb_ready, 0, ab) && tc::mbar_wait(&sm.q_full, 0, ab);
             if (ok) {
                 tc::tc_fence_after();
@@ -183,7 +182,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
 #pragma unroll
             for (int j = 0; j < 8; j++) {
                 if (amk[j]) {
-                    if (pos < UMAX) {
+                    if (pos < UM) {
                         sm.ulist[pos] = cb + j;
                         sm.amask[pos] = (uint8_t)amk[j];
                         sm.acell[pos] = A.has_prior ? am[cb + j] : 0.f;
@@ -195,17 +194,18 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
             sel_sync();
         }
         if (t == 0) {
-            sm.nU = min(total, UMAX);
-            if (total > UMAX && dev_flag) atomicExch(dev_flag, kFlagCheck);
+            sm.nU = min(total, UM);
+            if (total > UM && dev_flag) atomicExch(dev_flag, kFlagCheck);
         }
         sel_sync();
-        const int nU = min(total, UMAX);
+        const int nU = min(total, UM);
+        constexpr int NW = (UM + 31) / 32;      // admission words
         {   // admission masks per prefix, one 32-position word per warp
             const uint32_t am = t < nU ? sm.amask[t] : 0u;
 #pragma unroll
             for (int gg = 0; gg < 5; gg++) {
                 const uint32_t word = __ballot_sync(kFull, (am >> gg) & 1u);
-                if (lane == 0) sm.admit[gg][warp] = word;
+                if (lane == 0 && warp < NW) sm.admit[gg][warp] = word;
             }
         }
         // ---- kbar of U as three bf16 parts, row u = union position (zero rows pad to 16)
@@ -245,36 +245,35 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
             const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
             const float lam = PRIOR ? A.lambda[h] : 0.f;
             const float i2s = PRIOR ? A.inv2sigma[h] : 0.f;
-            uint32_t aw[UMAX / 32];                 // admitted union positions of this row
+            uint32_t aw[NW];                        // admitted union positions of this row
 #pragma unroll
-            for (int b = 0; b < UMAX / 32; b++) aw[b] = row < nrows ? sm.admit[g][b] : 0u;
-            const int na = __popc(aw[0]) + __popc(aw[1]) + __popc(aw[2]) + __popc(aw[3]);
-            uint32_t key[UMAX];
+            for (int b = 0; b < NW; b++) aw[b] = row < nrows ? sm.admit[g][b] : 0u;
+            int na = 0;
+#pragma unroll
+            for (int b = 0; b < NW; b++) na += __popc(aw[b]);
+            // raw scores of the N used columns, loaded in 16-column blocks before one wait
+            uint32_t key[UM];
+#pragma unroll
+            for (int b = 0; b < UM / 16; b++)
+                if (16 * b < N) tc::tmem_ld16(trow + 16 * b, &key[16 * b]);
+            tc::tmem_wait_ld();
             uint32_t kmn[8], kmx[8];
 #pragma unroll
             for (int k = 0; k < 8; k++) { kmn[k] = 0xffffffffu; kmx[k] = 0u; }
 #pragma unroll
-            for (int b = 0; b < UMAX / 32; b++) {
-                if (32 * b < N) {
-                    uint32_t r[32];
-                    tc::tmem_ld32(trow + 32 * b, r);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; e++) {
-                        const int u = 32 * b + e;
-                        float sc = __uint_as_float(r[e]) * A.scale;
-                        if (PRIOR) {
-                            const float pc = (float)(sm.ulist[u] * kS) + 0.5f * kS;
-                            sc += lam * sm.acell[u] * erff(((float)i - pc) * i2s);
-                        }
-                        const uint32_t k = ((aw[b] >> e) & 1u) ? (order_key(sc) & ~0x7fu) | (uint32_t)(127 - u) : 0u;
-                        key[u] = k;
-                        kmn[e & 7] = min(kmn[e & 7], k ? k : 0xffffffffu);
-                        kmx[e & 7] = max(kmx[e & 7], k);
+            for (int u = 0; u < UM; u++) {
+                if (16 * (u / 16) < N) {
+                    float sc = __uint_as_float(key[u]) * A.scale;
+                    if (PRIOR) {
+                        const float pc = (float)(sm.ulist[u] * kS) + 0.5f * kS;
+                        sc += lam * sm.acell[u] * erff(((float)i - pc) * i2s);
                     }
+                    const uint32_t k = ((aw[u >> 5] >> (u & 31)) & 1u) ? (order_key(sc) & ~0x7fu) | (uint32_t)(127 - u) : 0u;
+                    key[u] = k;
+                    kmn[u & 7] = min(kmn[u & 7], k ? k : 0xffffffffu);
+                    kmx[u & 7] = max(kmx[u & 7], k);
                 } else {
-#pragma unroll
-                    for (int e = 0; e < 32; e++) key[32 * b + e] = 0u;
+                    key[u] = 0u;
                 }
             }
             const uint32_t kmin = min(min(min(kmn[0], kmn[1]), min(kmn[2], kmn[3])), min(min(kmn[4], kmn[5]), min(kmn[6], kmn[7])));
@@ -287,10 +286,10 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                     const uint32_t mid = lo + ((hi - lo) >> 1);
                     int cp[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent partial counts
 #pragma unroll
-                    for (int b = 0; b < UMAX / 32; b++)
-                        if (32 * b < N) {
+                    for (int b = 0; b < UM / 16; b++)
+                        if (16 * b < N) {
 #pragma unroll
-                            for (int e = 0; e < 32; e++) cp[e & 7] += key[32 * b + e] >= mid;
+                            for (int e = 0; e < 16; e++) cp[e & 7] += key[16 * b + e] >= mid;
                         }
                     const int cnt = ((cp[0] + cp[1]) + (cp[2] + cp[3])) + ((cp[4] + cp[5]) + (cp[6] + cp[7]));
                     if (cnt >= A.K) {
@@ -304,14 +303,10 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
             }
             if (tiles) {   // compact record for the fused kernel: row masks | union | |U|
                 uint32_t *rec = tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords;
-                uint32_t mw[4];
+                uint32_t mw[UMAX / 32] = {0u, 0u, 0u, 0u};
 #pragma unroll
-                for (int b = 0; b < UMAX / 32; b++) {
-                    mw[b] = 0u;
-#pragma unroll
-                    for (int e = 0; e < 32; e++)
-                        if (key[32 * b + e] >= tau && key[32 * b + e] != 0u) mw[b] |= 1u << e;
-                }
+                for (int u = 0; u < UM; u++)
+                    if (key[u] >= tau && key[u] != 0u) mw[u >> 5] |= 1u << (u & 31);
                 *reinterpret_cast<uint4 *>(rec + kTileMaskOff + 4 * row) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
                 rec[kTileUlistOff + t] = t < nU ? (uint32_t)sm.ulist[t] : 0xffffffffu;
                 if (t == 0) rec[kTileCountOff] = (uint32_t)nU;
@@ -320,14 +315,8 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                 int32_t *out = idx + ((size_t)bh * A.Nq + r0 + row) * A.K;
                 int o = 0;
 #pragma unroll
-                for (int b = 0; b < UMAX / 32; b++)
-                    if (32 * b < N) {
-#pragma unroll
-                        for (int e = 0; e < 32; e++) {
-                            const int u = 32 * b + e;
-                            if (key[u] >= tau && key[u] != 0u && o < A.K) out[o++] = sm.ulist[u];
-                        }
-                    }
+                for (int u = 0; u < UM; u++)
+                    if (16 * (u / 16) < N && key[u] >= tau && key[u] != 0u && o < A.K) out[o++] = sm.ulist[u];
                 for (; o < A.K; o++) out[o] = -1;
             }
         }
@@ -349,6 +338,21 @@ bool select_tc_supported(const fs_params *p) {
     return bound <= UMAX;
 }
 
+namespace {
+// the largest union a tile of this call can have (W + P + 10 with pruning, else C)
+int union_bound(const Dev &P) { return P.prune ? P.W + P.P + 10 : P.C; }
+template <int UM> cudaError_t launch_um(const CUtensorMap &tq, const SelArgs &A, bool prior, dim3 grid,
+                                         const float *kbar, const float *amax, const int *exitn, int32_t *idx,
+                                         uint32_t *tiles, int *dev_flag, cudaStream_t st) {
+    const size_t smem = sizeof(SelSmem<UM>) + 1024;
+    // the erf prior is a separate instantiation: without it the unrolled score loop stays small
+    auto kern = prior ? select_tc_kernel<true, UM> : select_tc_kernel<false, UM>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    kern<<<grid, NTHREADS, smem, st>>>(tq, A, kbar, amax, exitn, idx, tiles, dev_flag);
+    return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, const float *amax,
                              const int *exitn, int32_t *idx, uint32_t *tiles, int *dev_flag,
                              cudaStream_t st) {
@@ -364,14 +368,11 @@ cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, con
         A.lambda[h] = P.lambda[h];
         A.inv2sigma[h] = P.inv2sigma[h];
     }
-    const size_t smem = sizeof(SelSmem) + 1024;
     const dim3 grid((P.Nq + BM - 1) / BM, BH);
     LaunchScope scope(kSelectTc, st);
-    // the erf prior is a separate instantiation: without it the unrolled score loop stays small
-    auto kern = P.has_prior ? select_tc_kernel<true> : select_tc_kernel<false>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<grid, NTHREADS, smem, st>>>(tq, A, kbar, amax, exitn, idx, tiles, dev_flag);
-    return cudaGetLastError();
+    if (union_bound(P) <= 80)
+        return launch_um<80>(tq, A, P.has_prior, grid, kbar, amax, exitn, idx, tiles, dev_flag, st);
+    return launch_um<UMAX>(tq, A, P.has_prior, grid, kbar, amax, exitn, idx, tiles, dev_flag, st);
 }
 
 }  // namespace fs
