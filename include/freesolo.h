@@ -144,6 +144,49 @@ const char *fs_status_string(fs_status s);
 fs_status fs_select_topk_noalloc(const fs_params *p, const void *Q, const float *kbar,
                                  const float *amax, int32_t *idx, void *stream);
 
+/* ---- FS-L streaming cache ("FreeSolo" summary, "Practical Implications" 3: bounded
+ * memory, O((P+W)s + w + B + s)d token state per head, independent of sequence length) ----
+ * Tokens arrive in blocks of at most max_block (the B of that bound); after each block,
+ * attention can be computed for any of its most recent positions from the cache alone.
+ * The cache keeps, per (batch, head):
+ *   - a ring of the last max_block + w + 2s tokens (raw keys, RoPE-rotated keys, values):
+ *     the window of every query still to come plus the cells not yet candidates;
+ *   - the candidate cells some upcoming query may still admit under eq. (8): the W most
+ *     recent candidates and the TopP by max key norm, at most W + P + 2*ceil(max_block/s)
+ *     + 4 cells, each with its keys, values, mean key and max norm (eq. (5)).
+ * A cell leaves when no prefix still in reach admits it.  This is exact, not an
+ * approximation: as the prefix grows a cell's rank by norm never improves, so a cell out
+ * of TopP never re-enters it, and one older than the W most recent never becomes recent
+ * again.  Base FS (no pruning) has no bounded state: W < 0 or P < 0 is FS_ERR_UNSUPPORTED.
+ *
+ * `cache` is a caller-owned device buffer of fs_cache_bytes bytes; every call on one cache
+ * must pass the same p (B, H, d, w, s, K, W, P, dtype, rope_base, alpha, lambda, sigma,
+ * rms_eps; Nq and Nk are ignored) and the same max_block (1 <= max_block <= 65536).
+ * Calls enqueue on `stream` and must be ordered (one stream).  Errors found on the device
+ * (e.g. attending more positions than have been appended) set the cache's error flag,
+ * read by fs_cache_status. */
+fs_status fs_cache_bytes(const fs_params *p, int max_block, size_t *bytes);
+
+/* Empties the cache (no tokens). */
+fs_status fs_cache_reset(const fs_params *p, int max_block, void *cache, size_t cache_bytes,
+                         void *stream);
+
+/* Appends n_new tokens (0 <= n_new <= max_block): K_new, V_new are device [B,H,n_new,d]
+ * of type p->dtype, at positions t .. t+n_new-1 where t counts the tokens appended so far. */
+fs_status fs_cache_append(const fs_params *p, int max_block, void *cache, size_t cache_bytes,
+                          const void *K_new, const void *V_new, int n_new, void *stream);
+
+/* O = o^sr + alpha_h o^lr (eq. (2)) for the n_q most recent positions t-n_q .. t-1
+ * (1 <= n_q <= max_block, n_q <= t): Q_new and O are device [B,H,n_q,d] of type p->dtype.
+ * idx, if not NULL, receives the selected cells [B,H,n_q,K] (ascending, -1 padded). */
+fs_status fs_cache_attend(const fs_params *p, int max_block, void *cache, size_t cache_bytes,
+                          const void *Q_new, int n_q, int32_t *idx, void *O, void *stream);
+
+/* Synchronizes `stream`, then reads and clears the cache's error flag: FS_ERR_KERNEL_CHECK
+ * if a call found its inputs inconsistent (n_q > t, or a state invariant broken),
+ * FS_ERR_CUDA if the stream reports an error, else FS_OK. */
+fs_status fs_cache_status(void *cache, void *stream);
+
 /* ---- diagnostics (no counterpart in the method: measurement support) ----
  * fs_launch_count: kernels this library has launched since load (all calls, streams).
  * fs_timing_enable(1): from now on every kernel launch is bracketed by two CUDA events

@@ -7,7 +7,9 @@ loading fails loudly if the library has not been built (python -m
 long_context_sparse_head_b200.build).
 
 The entry points mirror the C names: `workspace_size`, `cell_summaries`, `select_topk`,
-`forward`, `host_scratch_size`, `forward_host`, `sync_status`, `status_string`.
+`forward`, `host_scratch_size`, `forward_host`, `sync_status`, `status_string`, and the
+FS-L streaming cache `cache_bytes`, `cache_reset`, `cache_append`, `cache_attend`,
+`cache_status`.
 """
 import ctypes
 import os
@@ -23,7 +25,8 @@ STATUS = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_UNSUPPORTED", 3: "FS_E
 EXPORTS = ("fs_workspace_size", "fs_cell_summaries", "fs_select_topk", "fs_forward",
            "fs_host_scratch_size", "fs_forward_host", "fs_sync_status", "fs_status_string",
            "fs_launch_count", "fs_timing_enable", "fs_kernel_times", "fs_kernel_name",
-           "fs_select_topk_noalloc")
+           "fs_select_topk_noalloc", "fs_cache_bytes", "fs_cache_reset", "fs_cache_append",
+           "fs_cache_attend", "fs_cache_status")
 
 
 class FsError(RuntimeError):
@@ -74,6 +77,11 @@ def load():
         L.fs_timing_enable.argtypes = [ctypes.c_int]
         L.fs_kernel_times.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_longlong),
                                       ctypes.POINTER(ctypes.c_double)]
+        L.fs_cache_bytes.argtypes = [P, ctypes.c_int, ctypes.POINTER(sz)]
+        L.fs_cache_reset.argtypes = [P, ctypes.c_int, vp, sz, vp]
+        L.fs_cache_append.argtypes = [P, ctypes.c_int, vp, sz, vp, vp, ctypes.c_int, vp]
+        L.fs_cache_attend.argtypes = [P, ctypes.c_int, vp, sz, vp, ctypes.c_int, vp, vp, vp]
+        L.fs_cache_status.argtypes = [vp, vp]
         L.fs_kernel_name.argtypes = [ctypes.c_int]
         L.fs_kernel_name.restype = ctypes.c_char_p
         for name in EXPORTS:
@@ -188,6 +196,44 @@ def forward_host(params, hQ, hK, hV, hO, dscratch, stream=None):
 def sync_status(ws, stream=None):
     code = load().fs_sync_status(_ptr(ws), _stream(stream))
     _check(code, "fs_sync_status")
+
+
+# ---- FS-L streaming cache ----------------------------------------------------------
+def cache_bytes(params, max_block):
+    n = ctypes.c_size_t()
+    _check(load().fs_cache_bytes(params.ref(), int(max_block), ctypes.byref(n)), "fs_cache_bytes")
+    return n.value
+
+
+def alloc_cache(params, max_block, device="cuda", stream=None):
+    """A cache buffer of cache_bytes(params, max_block) bytes, emptied by fs_cache_reset."""
+    import torch
+    cache = torch.empty(cache_bytes(params, max_block), dtype=torch.uint8, device=device)
+    cache_reset(params, max_block, cache, stream)
+    return cache
+
+
+def cache_reset(params, max_block, cache, stream=None):
+    _check(load().fs_cache_reset(params.ref(), int(max_block), _ptr(cache), cache.numel(),
+                                 _stream(stream)), "fs_cache_reset")
+
+
+def cache_append(params, max_block, cache, K_new, V_new, stream=None):
+    """Appends K_new, V_new [B,H,n_new,d] (n_new <= max_block) to the stream."""
+    _check(load().fs_cache_append(params.ref(), int(max_block), _ptr(cache), cache.numel(),
+                                  _ptr(K_new), _ptr(V_new), int(K_new.shape[2]), _stream(stream)),
+           "fs_cache_append")
+
+
+def cache_attend(params, max_block, cache, Q_new, O, idx=None, stream=None):
+    """O [B,H,n_q,d] for the n_q = Q_new.shape[2] most recent positions."""
+    _check(load().fs_cache_attend(params.ref(), int(max_block), _ptr(cache), cache.numel(),
+                                  _ptr(Q_new), int(Q_new.shape[2]), _ptr(idx), _ptr(O),
+                                  _stream(stream)), "fs_cache_attend")
+
+
+def cache_status(cache, stream=None):
+    _check(load().fs_cache_status(_ptr(cache), _stream(stream)), "fs_cache_status")
 
 
 # ---- diagnostics -------------------------------------------------------------------

@@ -99,3 +99,18 @@ def test_workspace_size_grows_with_problem():
     b = fs.workspace_size(params(Nq=4096, Nk=4096))
     assert 0 < a < b
     assert fs.host_scratch_size(params()) > a
+
+
+def test_cache_memory_is_bounded():
+    """The FS-L streaming cache's size depends on the budgets and the block size, never on
+    how many tokens pass through it; base FS (no pruning) has no bounded state."""
+    import numpy as np
+    p = fs.Params(B=1, H=16, Nq=1, Nk=1, K=32, W=16, P=48, alpha=np.ones(16), dtype="bf16")
+    assert fs.cache_bytes(p, 1) < fs.cache_bytes(p, 64) < fs.cache_bytes(p, 4096)
+    q = fs.Params(B=1, H=16, Nq=1, Nk=1, K=32, W=-1, P=-1, alpha=np.ones(16), dtype="bf16")
+    with pytest.raises(fs.FsError) as e:
+        fs.cache_bytes(q, 1)
+    assert e.value.code == 2
+    with pytest.raises(fs.FsError) as e:
+        fs.cache_bytes(p, 0)
+    assert e.value.code == 1
