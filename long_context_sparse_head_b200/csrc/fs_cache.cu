@@ -33,7 +33,17 @@ namespace fs {
 namespace {
 
 constexpr int kMaxBlock = 65536;
-constexpr int kAppendThreads = 256, kAttendThreads = 128;
+constexpr int kAppendThreads = 256;
+// Attend: each warp stages 32-token blocks of key and value rows in shared memory (input
+// type, rows padded by 16 bytes against bank conflicts), double-buffered.
+template <typename T> struct AttendCfg {
+    static constexpr int kWarps = sizeof(T) == 2 ? 8 : 4;
+    static constexpr int kThreads = kWarps * 32;
+    static constexpr int kRowBytes = kD * (int)sizeof(T);
+    static constexpr int kRowStride = kRowBytes + 16;
+    static constexpr int kBlockBytes = kS * kRowStride;         // one 32-row block
+    static constexpr int kWarpBytes = 4 * kBlockBytes;          // (K, V) x 2 buffers
+};
 constexpr int kFlagOff = 0;                     // int error flag at the start of the cache
 constexpr size_t kHeadBytes = 256;
 
@@ -76,7 +86,7 @@ struct CacheArgs {
     int R, M, maxnew, max_block;
     int w, K, W, P, H;
     int has_prior;
-    double rope_base;
+    double theta[kD / 2];   // RoPE frequencies base^(-2m/d), double precision
     float scale;       // 1 / sqrt(d)
     float rms_eps;
     size_t o_t, o_rk, o_rr, o_rv, o_cell, o_exit, o_a, o_kbar, o_ck, o_cv, bh_bytes;
@@ -91,11 +101,21 @@ __device__ __forceinline__ int cand_count_ll(long long i, int w) {
     return lim < kS ? 0 : (int)(lim / kS);
 }
 
-// (cos, sin)(pos * theta_m), theta_m = base^(-2m/d), in double precision
-__device__ __forceinline__ void rope_cs(long long pos, int m, double base, float &c, float &s) {
-    const double theta = pow(base, -2.0 * m / (double)kD);
+__device__ __forceinline__ uint32_t tc_smem(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// (cos, sin)(pos * theta_m) in double precision, rounded to float.  The angle (up to
+// ~1e9 rad) is first reduced to [-pi, pi] by Cody-Waite: 2 pi = kTwoPiHi + kTwoPiLo with
+// kTwoPiHi holding 24 significant bits, so k * kTwoPiHi is exact for |k| < 2^29 and the
+// reduced angle is good to ~1e-10 rad; sincos then works on a small argument.
+__device__ __forceinline__ void rope_cs(long long pos, double theta, float &c, float &s) {
+    constexpr double kTwoPiHi = 6.2831854820251465, kTwoPiLo = -1.748455600074497e-07;
+    const double x = (double)pos * theta;
+    const double k = rint(x * 0.15915494309189535);           // x / (2 pi), rounded
+    const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, x));
     double sn, cs;
-    sincos((double)pos * theta, &sn, &cs);
+    sincos(r, &sn, &cs);
     c = (float)cs;
     s = (float)sn;
 }
@@ -144,7 +164,7 @@ __global__ void __launch_bounds__(kAppendThreads) cache_append_kernel(uint8_t *c
         const size_t dst = (size_t)(pos % A.R) * kD + 2 * m;
         const float k0 = to_f<T>(Kn[src]), k1 = to_f<T>(Kn[src + 1]);
         float c, sn;
-        rope_cs(pos, m, A.rope_base, c, sn);
+        rope_cs(pos, A.theta[m], c, sn);
         rk[dst] = Kn[src];
         rk[dst + 1] = Kn[src + 1];
         rr[dst] = from_f<T>(k0 * c - k1 * sn);
@@ -267,45 +287,86 @@ __global__ void __launch_bounds__(kAppendThreads) cache_append_kernel(uint8_t *c
     if (t == 0) *S.t = t1;
 }
 
+// Copies a 32-row block (row r at rows(r)) into dst with cp.async: eight lanes per 128
+// bytes of a row, so each instruction moves whole cache lines.
+template <typename T, typename RowFn>
+__device__ __forceinline__ void stage_block(uint8_t *dst, RowFn rows, int lane) {
+    using C = AttendCfg<T>;
+    constexpr int CPR = C::kRowBytes / 16;                       // 16-byte chunks per row
+    const uint32_t base = tc_smem(dst);
+#pragma unroll
+    for (int k = 0; k < kS * CPR / 32; k++) {
+        const int q = lane + 32 * k, row = q / CPR, c = q % CPR;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(base + row * C::kRowStride + 16 * c),
+                     "l"(reinterpret_cast<const uint8_t *>(rows(row)) + 16 * c)
+                     : "memory");
+    }
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// q (shared, float) . row (shared, T), 64 dims
+template <typename T> __device__ __forceinline__ float dot64_smem(const float *q, const uint8_t *row) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < AttendCfg<T>::kRowBytes / 16; c++) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(row + 16 * c);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        if (sizeof(T) == 2) {
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                acc[e] = fmaf(q[8 * c + 2 * e], __uint_as_float(w[e] << 16), acc[e]);
+                acc[e] = fmaf(q[8 * c + 2 * e + 1], __uint_as_float(w[e] & 0xffff0000u), acc[e]);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; e++) acc[e] = fmaf(q[4 * c + e], __uint_as_float(w[e]), acc[e]);
+        }
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
 // Online softmax state of one warp: running max m, sum l, and two output dims per lane.
+// add(): one 32-token block, lane j holding token j's score (-inf if invalid), the value
+// rows staged at vb; lane = dim pair for P V.
 struct Online {
     float m = -INFINITY, l = 0.f, a0 = 0.f, a1 = 0.f;
-    // one 32-token block: sc = this lane's score (-inf if invalid), vrow(j) = value row of token j
-    template <typename T> __device__ __forceinline__ void block(float sc, const T *v, size_t vstride, int lane) {
+    template <typename T> __device__ __forceinline__ void add(float sc, const uint8_t *vb, int lane) {
         const float mc = warp_max(sc);
         if (mc == -INFINITY) return;
         const float mn = fmaxf(m, mc);
         const float corr = m == -INFINITY ? 0.f : expf(m - mn);
         const float p = sc == -INFINITY ? 0.f : expf(sc - mn);
         l = l * corr + warp_sum(p);
-        a0 *= corr;
-        a1 *= corr;
+        float b0[2] = {a0 * corr, 0.f}, b1[2] = {a1 * corr, 0.f};   // two chains per dim
 #pragma unroll 8
         for (int j = 0; j < kS; j++) {
             const float pj = __shfl_sync(kFull, p, j);
-            const T *vr = v + (size_t)j * vstride + 2 * lane;
-            a0 = fmaf(pj, to_f<T>(vr[0]), a0);
-            a1 = fmaf(pj, to_f<T>(vr[1]), a1);
+            const uint8_t *row = vb + j * AttendCfg<T>::kRowStride;
+            float v0, v1;
+            if (sizeof(T) == 2) {
+                const uint32_t w = *reinterpret_cast<const uint32_t *>(row + 4 * lane);
+                v0 = __uint_as_float(w << 16);
+                v1 = __uint_as_float(w & 0xffff0000u);
+            } else {
+                const float2 f2 = *reinterpret_cast<const float2 *>(row + 8 * lane);
+                v0 = f2.x;
+                v1 = f2.y;
+            }
+            b0[j & 1] = fmaf(pj, v0, b0[j & 1]);
+            b1[j & 1] = fmaf(pj, v1, b1[j & 1]);
         }
+        a0 = b0[0] + b0[1];
+        a1 = b1[0] + b1[1];
         m = mn;
     }
 };
 
-// q (shared, float) . key row (global, T), 64 dims
-template <typename T> __device__ __forceinline__ float dot64(const float *q, const T *k) {
-    float acc = 0.f;
-#pragma unroll
-    for (int c = 0; c < kD / Vec<T>::N; c++) {
-        float x[Vec<T>::N];
-        Vec<T>::load(k + c * Vec<T>::N, x);
-#pragma unroll
-        for (int e = 0; e < Vec<T>::N; e++) acc = fmaf(q[c * Vec<T>::N + e], x[e], acc);
-    }
-    return acc;
-}
-
-// Folds the four warps' online states into out[64] = acc / l (0 where nothing was attended).
-__device__ __forceinline__ void fold_warps(const Online &o, float (*s_m)[4], float (*s_l)[4], float (*s_acc)[kD],
+// Folds the NW warps' online states into out[64] = acc / l (0 where nothing was attended).
+template <int NW>
+__device__ __forceinline__ void fold_warps(const Online &o, float (*s_m)[NW], float (*s_l)[NW], float (*s_acc)[kD],
                                            float *out, int t, int warp, int lane) {
     if (lane == 0) {
         (*s_m)[warp] = o.m;
@@ -316,10 +377,10 @@ __device__ __forceinline__ void fold_warps(const Online &o, float (*s_m)[4], flo
     __syncthreads();
     if (t < kD) {
         float mx = -INFINITY;
-        for (int w2 = 0; w2 < 4; w2++) mx = fmaxf(mx, (*s_m)[w2]);
+        for (int w2 = 0; w2 < NW; w2++) mx = fmaxf(mx, (*s_m)[w2]);
         float num = 0.f, den = 0.f;
         if (mx != -INFINITY)
-            for (int w2 = 0; w2 < 4; w2++) {
+            for (int w2 = 0; w2 < NW; w2++) {
                 if ((*s_m)[w2] == -INFINITY) continue;
                 const float f = expf((*s_m)[w2] - mx);
                 num = fmaf(s_acc[w2][t], f, num);
@@ -331,15 +392,19 @@ __device__ __forceinline__ void fold_warps(const Online &o, float (*s_m)[4], flo
 }
 
 template <typename T, bool PRIOR>
-__global__ void __launch_bounds__(kAttendThreads) cache_attend_kernel(uint8_t *cache, const T *__restrict__ Qn,
+__global__ void __launch_bounds__(AttendCfg<T>::kThreads) cache_attend_kernel(uint8_t *cache, const T *__restrict__ Qn,
                                                                       int n_q, int32_t *__restrict__ idx,
                                                                       T *__restrict__ O, const CacheArgs A) {
-    extern __shared__ int shi[];                 // per slot: score, flags (1 admitted, 2 selected), cell
-    float *s_score = reinterpret_cast<float *>(shi);
-    int *s_flag = shi + A.M, *s_cell = shi + 2 * A.M, *s_list = shi + 3 * A.M;   // s_list: K slots
+    using Cfg = AttendCfg<T>;
+    constexpr int NW = Cfg::kWarps, NT = Cfg::kThreads;
+    // dynamic: per warp the staged (K, V) blocks x 2; per slot a sort key (0: not admitted;
+    // else score order in the high word, lower cell first in the low word), its cell and a
+    // selected flag; the selected slots [K]
+    extern __shared__ __align__(16) uint8_t shb[];
+    unsigned long long *s_key = reinterpret_cast<unsigned long long *>(shb + NW * Cfg::kWarpBytes);
+    int *s_cell = reinterpret_cast<int *>(s_key + A.M), *s_sel = s_cell + A.M, *s_list = s_sel + A.M;
     __shared__ float s_qn[kD], s_qr[kD], s_u[kD], s_o[kD];
-    __shared__ float s_m[4], s_l[4], s_acc[4][kD], s_ss[2];
-    __shared__ int s_nsel;
+    __shared__ float s_m[NW], s_l[NW], s_acc[NW][kD], s_ss[2];
     const int r = blockIdx.x, bh = blockIdx.y, h = bh % A.H;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const Slots S = slots_of(cache, A, bh);
@@ -354,71 +419,94 @@ __global__ void __launch_bounds__(kAttendThreads) cache_attend_kernel(uint8_t *c
     if (t < kD / 2) {
         const float q0 = to_f<T>(q[2 * t]), q1 = to_f<T>(q[2 * t + 1]);
         float c, sn;
-        rope_cs(i, t, A.rope_base, c, sn);
+        rope_cs(i, A.theta[t], c, sn);
         s_qn[2 * t] = q0;
         s_qn[2 * t + 1] = q1;
         s_qr[2 * t] = q0 * c - q1 * sn;
         s_qr[2 * t + 1] = q0 * sn + q1 * c;
     }
-    if (t == 0) s_nsel = 0;
     __syncthreads();
 
-    // 1. admission (eq. (8)) and scores (eq. (7)) over the slots, one warp per slot
-    for (int x = warp; x < A.M; x += kAttendThreads / 32) {
+    // 1. admission (eq. (8)) and scores (eq. (7)) over the slots, one thread per slot (the
+    //    mean-key loads of all slots are in flight together)
+    for (int x = t; x < A.M; x += NT) {
         const int c = S.cell[x];
         const bool adm = c >= 0 && c < n && (c >= n - A.W || n < S.exit[x]);
         float sc = 0.f;
         if (adm) {
-            const float *kb = S.kbar + (size_t)x * kD;
-            sc = warp_sum(fmaf(s_qn[2 * lane], kb[2 * lane], s_qn[2 * lane + 1] * kb[2 * lane + 1])) * A.scale;
+            const float4 *kb = reinterpret_cast<const float4 *>(S.kbar + (size_t)x * kD);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int e = 0; e < kD / 4; e++) {
+                const float4 v = __ldg(kb + e);
+                acc[e & 3] = fmaf(s_qn[4 * e], v.x, fmaf(s_qn[4 * e + 1], v.y,
+                             fmaf(s_qn[4 * e + 2], v.z, fmaf(s_qn[4 * e + 3], v.w, acc[e & 3]))));
+            }
+            sc = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * A.scale;
             if (PRIOR) {
                 const float dpos = (float)(i - (long long)c * kS) - 0.5f * kS;   // i - p_c
                 sc += A.lambda[h] * S.a[x] * erff(dpos * A.inv2sigma[h]);
             }
         }
-        if (lane == 0) {
-            s_score[x] = sc;
-            s_flag[x] = adm ? 1 : 0;
-            s_cell[x] = c;
-        }
+        const uint32_t ob = __float_as_uint(sc);
+        const uint32_t ok = (ob & 0x80000000u) ? ~ob : (ob | 0x80000000u);
+        s_key[x] = adm ? ((unsigned long long)ok << 32) | (0xffffffffu - (uint32_t)c) : 0ull;
+        s_cell[x] = c;
     }
     __syncthreads();
-    // 2. top-K: a slot is selected if fewer than K admitted slots rank above it (higher
-    //    score, or equal score and lower cell)
-    for (int x = t; x < A.M; x += kAttendThreads) {
-        if (!(s_flag[x] & 1)) continue;
-        const float sx = s_score[x];
-        const int cx = s_cell[x];
+    // 2. top-K: a slot is selected if fewer than K admitted slots have a larger key (higher
+    //    score, or equal score and lower cell): a branch-free count over the keys
+    for (int x = t; x < A.M; x += NT) {
+        const unsigned long long kx = s_key[x];
         int rank = 0;
-        for (int y = 0; y < A.M; y++)
-            if (s_flag[y] & 1) {
-                const float sy = s_score[y];
-                rank += (sy > sx) || (sy == sx && s_cell[y] < cx);
-            }
-        if (rank < A.K) atomicOr(&s_flag[x], 2);
+#pragma unroll 4
+        for (int y = 0; y < A.M; y++) rank += s_key[y] > kx;
+        s_sel[x] = kx != 0ull && rank < A.K;
     }
     __syncthreads();
-    for (int x = t; x < A.M; x += kAttendThreads) {   // selected slots in ascending cell order
-        if (!(s_flag[x] & 2)) continue;
+    for (int x = t; x < A.M; x += NT) {   // selected slots in ascending cell order
+        if (!s_sel[x]) continue;
+        const int cx = s_cell[x];
         int pos = 0;
-        for (int y = 0; y < A.M; y++) pos += (s_flag[y] & 2) && s_cell[y] < s_cell[x];
+#pragma unroll 4
+        for (int y = 0; y < A.M; y++) pos += s_sel[y] & (s_cell[y] < cx);
         s_list[pos] = x;
-        atomicAdd(&s_nsel, 1);
     }
     __syncthreads();
-    const int nsel = s_nsel;
+    int nsel = 0;
+    for (int y = 0; y < A.M; y++) nsel += s_sel[y];
     if (idx && t < A.K) idx[((size_t)bh * n_q + r) * A.K + t] = t < nsel ? s_cell[s_list[t]] : -1;
 
     // 3. readout (eq. (9)): NoPE softmax over every token of the selected cells; warp w
     //    takes cells w, w+4, ...; lane = token for the scores, lane = dim pair for P V
     const T *ck = reinterpret_cast<const T *>(S.ck), *cv = reinterpret_cast<const T *>(S.cv);
+    uint8_t *wbuf = shb + warp * Cfg::kWarpBytes;              // (K, V) buffer b at 2 b Cfg::kBlockBytes
     Online lr;
-    for (int k = warp; k < nsel; k += kAttendThreads / 32) {
-        const int x = s_list[k];
-        const float sc = dot64<T>(s_qn, ck + ((size_t)x * kS + lane) * kD) * A.scale;
-        lr.block<T>(sc, cv + (size_t)x * kS * kD, kD, lane);
+    {
+        const int nit = nsel > warp ? (nsel - warp + NW - 1) / NW : 0;   // cells warp, warp + NW, ...
+        auto issue = [&](int k) {
+            const int x = s_list[warp + k * NW];
+            uint8_t *b = wbuf + 2 * (k & 1) * Cfg::kBlockBytes;
+            stage_block<T>(b, [&](int row) { return ck + ((size_t)x * kS + row) * kD; }, lane);
+            stage_block<T>(b + Cfg::kBlockBytes, [&](int row) { return cv + ((size_t)x * kS + row) * kD; }, lane);
+            cp_commit();
+        };
+        if (nit > 0) issue(0);
+        for (int k = 0; k < nit; k++) {
+            if (k + 1 < nit) {
+                issue(k + 1);
+                cp_wait<1>();
+            } else {
+                cp_wait<0>();
+            }
+            __syncwarp();
+            const uint8_t *b = wbuf + 2 * (k & 1) * Cfg::kBlockBytes;
+            const float sc = dot64_smem<T>(s_qn, b + lane * Cfg::kRowStride) * A.scale;
+            lr.add<T>(sc, b + Cfg::kBlockBytes, lane);
+            __syncwarp();                                        // before the buffer is refilled
+        }
     }
-    fold_warps(lr, &s_m, &s_l, s_acc, s_u, t, warp, lane);
+    fold_warps<NW>(lr, &s_m, &s_l, s_acc, s_u, t, warp, lane);
     if (t < kD) {                                 // RMSNorm (no gain), then alpha_h
         const float ss = warp_sum(s_u[t] * s_u[t]);
         if (lane == 0) s_ss[warp] = ss;
@@ -432,30 +520,41 @@ __global__ void __launch_bounds__(kAttendThreads) cache_attend_kernel(uint8_t *c
     const long long jlo = i - A.w < 0 ? 0 : i - A.w;
     const int L = (int)(i - jlo) + 1;
     Online sr;
-    for (int b = warp; b * kS < L; b += kAttendThreads / 32) {
-        const long long j = jlo + (long long)b * kS + lane;
-        const bool valid = j <= i;
-        const long long jj = valid ? j : i;      // any ring row in range for the idle lanes
-        const float sc = valid ? dot64<T>(s_qr, rr + (size_t)(jj % A.R) * kD) * A.scale : -INFINITY;
-        // the 32 value rows of this block are not contiguous in the ring: gather per token
-        const float mc = warp_max(sc);
-        const float mn = fmaxf(sr.m, mc);
-        const float corr = sr.m == -INFINITY ? 0.f : expf(sr.m - mn);
-        const float p = valid ? expf(sc - mn) : 0.f;
-        sr.l = sr.l * corr + warp_sum(p);
-        sr.a0 *= corr;
-        sr.a1 *= corr;
-        for (int e = 0; e < kS; e++) {
-            const float pe = __shfl_sync(kFull, p, e);
-            const long long je = jlo + (long long)b * kS + e;
-            if (je > i) break;
-            const T *vr = rv + (size_t)(je % A.R) * kD + 2 * lane;
-            sr.a0 = fmaf(pe, to_f<T>(vr[0]), sr.a0);
-            sr.a1 = fmaf(pe, to_f<T>(vr[1]), sr.a1);
+    {
+        const int nblk = (L + kS - 1) / kS;
+        const int nit = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;   // blocks warp, warp + NW, ...
+        const int ri = (int)(i % A.R);                        // ring row of the query's own token
+        auto issue = [&](int k) {
+            // ring row of token `row` of block k (no 64-bit modulo per row: one per block)
+            const long long j0 = jlo + (long long)(warp + k * NW) * kS;
+            const int r0 = (int)(j0 % A.R), last = (int)(i - j0);   // rows past `last` are past i
+            auto row_of = [&](int row) {
+                if (row > last) return (size_t)ri * kD;           // past i: any row in range
+                const int rr0 = r0 + row;
+                return (size_t)(rr0 >= A.R ? rr0 - A.R : rr0) * kD;
+            };
+            uint8_t *b = wbuf + 2 * (k & 1) * Cfg::kBlockBytes;
+            stage_block<T>(b, [&](int row) { return rr + row_of(row); }, lane);
+            stage_block<T>(b + Cfg::kBlockBytes, [&](int row) { return rv + row_of(row); }, lane);
+            cp_commit();
+        };
+        if (nit > 0) issue(0);
+        for (int k = 0; k < nit; k++) {
+            if (k + 1 < nit) {
+                issue(k + 1);
+                cp_wait<1>();
+            } else {
+                cp_wait<0>();
+            }
+            __syncwarp();
+            const uint8_t *b = wbuf + 2 * (k & 1) * Cfg::kBlockBytes;
+            const long long j = jlo + (long long)(warp + k * NW) * kS + lane;
+            const float sc = j <= i ? dot64_smem<T>(s_qr, b + lane * Cfg::kRowStride) * A.scale : -INFINITY;
+            sr.add<T>(sc, b + Cfg::kBlockBytes, lane);
+            __syncwarp();
         }
-        sr.m = mn;
     }
-    fold_warps(sr, &s_m, &s_l, s_acc, s_o, t, warp, lane);
+    fold_warps<NW>(sr, &s_m, &s_l, s_acc, s_o, t, warp, lane);
 
     // 5. O = o^sr + alpha_h RMSNorm(u)  (eq. (2))
     if (t < kD) O[((size_t)bh * n_q + r) * kD + t] = from_f<T>(s_o[t] + f * s_u[t]);
@@ -500,7 +599,7 @@ CacheArgs cache_args(const fs_params *p, int max_block, const CacheGeom &g) {
     std::memset(&A, 0, sizeof(A));
     A.R = g.R; A.M = g.M; A.maxnew = g.maxnew; A.max_block = max_block;
     A.w = p->w; A.K = p->K; A.W = p->W; A.P = p->P; A.H = p->H;
-    A.rope_base = (double)p->rope_base;
+    for (int m = 0; m < kD / 2; m++) A.theta[m] = std::pow((double)p->rope_base, -2.0 * m / (double)p->d);
     A.scale = (float)(1.0 / std::sqrt((double)p->d));
     A.rms_eps = p->rms_eps;
     A.o_t = g.o_t; A.o_rk = g.o_rk; A.o_rr = g.o_rr; A.o_rv = g.o_rv; A.o_cell = g.o_cell;
@@ -563,11 +662,11 @@ namespace {
 template <typename T>
 cudaError_t attend_launch(const CacheArgs &A, uint8_t *c, const void *Q, int n_q, int32_t *idx, void *O,
                           int BH, cudaStream_t st) {
-    const size_t smem = (size_t)(3 * A.M + kMaxK) * 4;
+    const size_t smem = (size_t)AttendCfg<T>::kWarps * AttendCfg<T>::kWarpBytes + (size_t)A.M * 16 + (size_t)kMaxK * 4;
     const dim3 grid(n_q, BH);
     auto kern = A.has_prior ? cache_attend_kernel<T, true> : cache_attend_kernel<T, false>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<grid, kAttendThreads, smem, st>>>(c, static_cast<const T *>(Q), n_q, idx, static_cast<T *>(O), A);
+    kern<<<grid, AttendCfg<T>::kThreads, smem, st>>>(c, static_cast<const T *>(Q), n_q, idx, static_cast<T *>(O), A);
     return cudaGetLastError();
 }
 }  // namespace
