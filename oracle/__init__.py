@@ -36,7 +36,7 @@ class OrcParams(ctypes.Structure):
 MUTATIONS = {
     "rope_key_sign": 1, "drop_prior": 2, "window_short": 3, "cand_loose": 4,
     "amax_mean": 5, "no_eps": 6, "alpha_on_sr": 7, "rope_in_readout": 8,
-    "scale_d": 9, "tie_high_index": 10,
+    "scale_d": 9, "tie_high_index": 10, "rerank_mean": 11, "rerank_rope": 12,
 }
 
 
@@ -59,6 +59,8 @@ def lib():
                                   f64p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         L.orc_select_row.argtypes = [P, f32p, f64p, f64p, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_int, i32p, i32p, f64p]
+        L.orc_rerank_row.argtypes = [P, f32p, f32p, f64p, f64p, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_int, ctypes.c_int, i32p, i32p, f64p]
         L.orc_readout_rows.argtypes = [P, f32p, f32p, f32p, ctypes.c_longlong, i64p, i32p,
                                        ctypes.c_void_p, f64p]
         L.orc_readout_rows.restype = None
@@ -159,6 +161,20 @@ class Problem:
                                   np.ascontiguousarray(amax, np.float64),
                                   b, h, r, idx, acells, ascores)
         return idx[:self.p.K].copy(), acells[:nA].copy(), ascores[:nA].copy()
+
+    def rerank_row(self, kbar, amax, b, h, r, shortlist=0):
+        """eq. (12) token-level rerank for one row: the `shortlist` best cells of A_i by
+        eq. (7) (0: all of A_i) rescored by the log-sum-exp of their tokens' logits plus
+        the prior; returns (idx[K], shortlist cells ascending, their eq. (12) scores)."""
+        C = self.C
+        idx = np.zeros(max(self.p.K, 1), np.int32)
+        cells = np.zeros(max(C, 1), np.int32)
+        scores = np.zeros(max(C, 1), np.float64)
+        ns = lib().orc_rerank_row(ctypes.byref(self.p), self.Q, self.K,
+                                  np.ascontiguousarray(kbar, np.float64),
+                                  np.ascontiguousarray(amax, np.float64),
+                                  b, h, r, int(shortlist), idx, cells, scores)
+        return idx[:self.p.K].copy(), cells[:ns].copy(), scores[:ns].copy()
 
     def readout_rows(self, rows, idx):
         """eq. (9) for the given flat rows on caller-given cells idx [n,K]: (u, o^lr)."""

@@ -13,6 +13,8 @@
  *                          eq. (7)   cell score r_ic with the erf position prior
  *                          eq. (8)   FS-L pruning A_i = Recent_W(C_i) u TopP(a_c)
  *                          eq. (9)   NoPE token readout over the selected cells, RMSNorm
+ *   §3.4                   eq. (12)  token-level rerank: a cell scored by the log-sum-exp
+ *                                    of its tokens' NoPE logits plus the prior term
  * "Introduction and Theoretical Foundation": RoPE (Su et al.) stays inside the
  * local window; long-range routing and readout use unrotated vectors.
  *
@@ -24,6 +26,9 @@
  *   - ties in TopP and top-K: larger value first, then the lower cell index
  *   - |A_i| < K: all of A_i is selected; S_i empty gives o^lr = 0
  *   - W < 0 and P < 0 together mean "no pruning" (base FS: A_i = C_i)
+ *   - eq. (12) reranks a shortlist: the `shortlist` best cells of A_i by eq. (7)
+ *     (shortlist <= 0: all of A_i) are rescored by eq. (12) and the K best kept; its
+ *     g_h is eq. (7)'s erf((i - p_c) / (2 sigma_h)) (eq. (11) uses the same name)
  *
  * Every quantity is computed in double from the float32 inputs (bf16 inputs are
  * passed as their exact float32 values).  No tiling, fusion or reordering beyond
@@ -63,6 +68,8 @@ enum {
     MUT_ROPE_IN_READOUT = 8, /* long-range readout uses rotated vectors */
     MUT_SCALE_D = 9,         /* logits scaled by 1/d instead of 1/sqrt(d) */
     MUT_TIE_HIGH_INDEX = 10, /* ties broken toward the higher cell index */
+    MUT_RERANK_MEAN = 11,    /* eq. (12) with the mean logit instead of the log-sum-exp */
+    MUT_RERANK_ROPE = 12,    /* eq. (12) with rotated query and keys */
 };
 
 int orc_num_cells(const orc_params *p) { return p->s > 0 ? p->Nk / p->s : 0; }
@@ -402,6 +409,80 @@ int orc_forward(const orc_params *p, const float *Q, const float *K, const float
     }
     free(order); free(start);
     return 0;
+}
+
+/* ---- eq. (12): token-level rerank for one query row ----
+ * The shortlist (the `shortlist` best cells of A_i by eq. (7); all of A_i if
+ * shortlist <= 0) is rescored by
+ *     rt_ic = log sum_{j in I_c} exp(q_i . k_j / sqrt(d)) + lambda_h a_c erf((i - p_c)/(2 sigma_h))
+ * over the raw (unrotated) keys of the cell's tokens I_c, and the K best form S_i (ties:
+ * lower cell).  idx_out[K] ascending, -1 padded; cells/scores (capacity >= |A_i|) receive
+ * the shortlist (ascending) and its rt.  Returns the shortlist size. */
+int orc_rerank_row(const orc_params *p, const float *Q, const float *K, const double *kbar,
+                   const double *amax, int b, int h, int r, int shortlist, int *idx_out,
+                   int *cells, double *scores)
+{
+    const int C = orc_num_cells(p), d = p->d, s = p->s;
+    size_t bh = (size_t)b * p->H + h;
+    long long i = (long long)(p->Nk - p->Nq) + r;
+    const float *qrow = Q + (bh * p->Nq + r) * d;
+    const float *Kbh = K + bh * (size_t)p->Nk * d;
+    /* shortlist by eq. (7): select_row with K = shortlist (or |C_i| for all of A_i) */
+    orc_params ps = *p;
+    int n = orc_candidate_count(p, i);
+    ps.K = shortlist > 0 ? shortlist : (n > 0 ? n : 1);
+    int *sl = (int *)malloc(sizeof(int) * (size_t)ps.K);
+    select_row(&ps, qrow, i, h, kbar + bh * C * d, amax + bh * C, sl, NULL, NULL);
+    int ns = 0;
+    while (ns < ps.K && sl[ns] >= 0) ns++;
+    vi_pair *x = (vi_pair *)malloc(sizeof(vi_pair) * (size_t)(ns > 0 ? ns : 1));
+    vi_pair *tmp = (vi_pair *)malloc(sizeof(vi_pair) * (size_t)(ns > 0 ? ns : 1));
+    double lam = p->lambda ? p->lambda[h] : 0.0;
+    double sig = p->sigma ? p->sigma[h] : 1.0;
+    double pos_i = (double)(p->pos0 + i);
+    double *lg = (double *)malloc(sizeof(double) * (size_t)s);
+    double qv[512], kv[512];
+    for (int t = 0; t < ns; t++) {
+        int c = sl[t];
+        double mx = -INFINITY, acc = 0.0;
+        for (int j = 0; j < s; j++) {            /* the cell's token logits */
+            long long jj = (long long)c * s + j;
+            const float *k = Kbh + (size_t)jj * d;
+            double dot = 0.0;
+            if (p->mutation == MUT_RERANK_ROPE) {
+                rope_rotate(p, qrow, p->pos0 + i, qv);
+                rope_rotate(p, k, p->pos0 + jj, kv);
+                for (int m = 0; m < d; m++) dot += qv[m] * kv[m];
+            } else {
+                for (int m = 0; m < d; m++) dot += (double)qrow[m] * k[m];
+            }
+            lg[j] = dot * logit_scale(p);
+            if (lg[j] > mx) mx = lg[j];
+            acc += lg[j];
+        }
+        double rt;
+        if (p->mutation == MUT_RERANK_MEAN) {
+            rt = acc / s;
+        } else {                                  /* log-sum-exp, shifted by the max */
+            double se = 0.0;
+            for (int j = 0; j < s; j++) se += exp(lg[j] - mx);
+            rt = mx + log(se);
+        }
+        if (lam != 0.0) {
+            double p_c = (double)p->pos0 + (c + 0.5) * s;
+            rt += lam * amax[bh * C + c] * erf((pos_i - p_c) / (2.0 * sig));
+        }
+        x[t].v = rt; x[t].idx = c;
+        if (cells) cells[t] = c;
+        if (scores) scores[t] = rt;
+    }
+    sort_desc(x, ns, tmp, p->mutation == MUT_TIE_HIGH_INDEX);
+    int keep = ns < p->K ? ns : p->K;
+    for (int t = 0; t < keep; t++) idx_out[t] = x[t].idx;
+    qsort(idx_out, (size_t)keep, sizeof(int), cmp_int);
+    for (int t = keep; t < p->K; t++) idx_out[t] = -1;
+    free(sl); free(x); free(tmp); free(lg);
+    return ns;
 }
 
 /* ---- single-step entry points for the tests ---- */

@@ -295,6 +295,81 @@ def test_golden_select_ties_eq7():
         assert idx.tolist() == cells, Kc
 
 
+# ---------------------------------------------------------------- eq. (12) rerank
+def _constant_cells(inp):
+    """The same problem with every cell's keys replaced by one vector (its mean)."""
+    K = inp.K.copy()
+    s = inp.wl.s
+    C = K.shape[2] // s
+    for c in range(C):
+        K[:, :, c * s:(c + 1) * s] = K[:, :, c * s:(c + 1) * s].mean(axis=2, keepdims=True)
+    return type(inp)(wl=inp.wl, Q=inp.Q, K=np.ascontiguousarray(K), V=inp.V, alpha=inp.alpha,
+                     lam=None, sigma=None)
+
+
+def _rerank_pin_failures(mutation=0):
+    """Pins of the eq. (12) rerank; returns the names of those that fail."""
+    fails = []
+    # (a) constant cells: log-sum-exp over s equal logits is that logit + log s, so the
+    #     rerank keeps exactly eq. (7)'s cells and its scores sit log s above eq. (7)'s
+    inp = _constant_cells(tiny(d=16, Nq=200, Nk=200, seed=43))
+    prob = make_problem(inp, mutation=mutation, lam=None, sigma=None)
+    kb, am = prob.summaries()
+    wl = inp.wl
+    for r in range(0, wl.Nq, 7):
+        i7, cells7, sc7 = prob.select_row(kb, am, 0, 1, r)
+        i12, cells12, sc12 = prob.rerank_row(kb, am, 0, 1, r)
+        if i7.tolist() != i12.tolist():
+            fails.append("constant_cells_selection")
+            break
+        want = {c: v + math.log(wl.s) for c, v in zip(cells7.tolist(), sc7.tolist())}
+        if any(abs(want[c] - v) > 1e-9 for c, v in zip(cells12.tolist(), sc12.tolist())):
+            fails.append("constant_cells_offset")
+            break
+    # (b) bounds: max_j logit <= log-sum-exp <= max_j logit + log s, logits from numpy
+    inp = tiny(d=16, Nq=200, Nk=200, seed=44)
+    prob = make_problem(inp, mutation=mutation, lam=None, sigma=None)
+    kb, am = prob.summaries()
+    wl = inp.wl
+    for r in range(wl.s + wl.w, wl.Nq, 11):
+        _, cells, sc = prob.rerank_row(kb, am, 0, 0, r)
+        q = inp.Q[0, 0, r].astype(np.float64)
+        for c, v in zip(cells.tolist(), sc.tolist()):
+            lg = inp.K[0, 0, c * wl.s:(c + 1) * wl.s].astype(np.float64) @ q / math.sqrt(wl.d)
+            if not (lg.max() - 1e-9 <= v <= lg.max() + math.log(wl.s) + 1e-9):
+                fails.append("lse_bounds")
+                break
+        if "lse_bounds" in fails:
+            break
+    # (c) a shortlist of exactly K keeps eq. (7)'s set (the rerank only reorders it)
+    for r in range(wl.s + wl.w, wl.Nq, 13):
+        if prob.select_row(kb, am, 0, 0, r)[0].tolist() != prob.rerank_row(kb, am, 0, 0, r, wl.K)[0].tolist():
+            fails.append("shortlist_K")
+            break
+    # (d) rescue: a cell whose mean key is orthogonal to q but which holds one token along
+    #     q (and its negative, so the mean cancels) is missed by eq. (7) and kept by eq. (12)
+    inp = tiny(d=16, Nq=160, Nk=160, K=2, W=-1, P=-1, seed=45)
+    K = inp.K.copy()
+    q = inp.Q[0, 0, 159].astype(np.float64)
+    u = q / np.linalg.norm(q)
+    c0, s_ = 3, inp.wl.s
+    K[0, 0, c0 * s_:(c0 + 1) * s_] = 0.0
+    K[0, 0, c0 * s_] = 6.0 * u
+    K[0, 0, c0 * s_ + 1] = -6.0 * u
+    inp = type(inp)(wl=inp.wl, Q=inp.Q, K=np.ascontiguousarray(K, np.float32), V=inp.V,
+                    alpha=inp.alpha, lam=None, sigma=None)
+    prob = make_problem(inp, mutation=mutation, lam=None, sigma=None, W=-1, P=-1)
+    kb, am = prob.summaries()
+    if c0 in prob.select_row(kb, am, 0, 0, 159)[0].tolist() or \
+            c0 not in prob.rerank_row(kb, am, 0, 0, 159)[0].tolist():
+        fails.append("rescue")
+    return fails
+
+
+def test_rerank_pins():
+    assert _rerank_pin_failures() == []
+
+
 # ---------------------------------------------------------------- sensitivity
 def _pins_fail(mutation):
     """Run a compact set of the pins above against a mutated oracle; True if any fails."""
@@ -316,6 +391,7 @@ def _pins_fail(mutation):
             failures.append("golden_prune")
     except Exception:
         failures.append("golden_prune")
+    failures += _rerank_pin_failures(mutation)
     return failures
 
 
