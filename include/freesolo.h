@@ -92,6 +92,20 @@ fs_status fs_select_topk(const fs_params *p, const void *Q, const float *kbar,
                          const float *amax, int32_t *idx, void *ws, size_t ws_bytes,
                          void *stream);
 
+/* Token-level rerank of the selection ("FreeSolo" summary §3.4, eq. (12)): each cell of a
+ * shortlist of A_i is rescored by
+ *     rt_ic = log sum_{j in I_c} exp(q_i.k_j/sqrt(d)) + lambda_h a_c erf((i - p_c)/(2 sigma_h))
+ * over its tokens' raw (unrotated) keys, and the K best form S_i, written to idx
+ * [B,H,Nq,K] (ascending, -1 padded; ties go to the lower cell).  The shortlist is the
+ * `shortlist` best cells of A_i by eq. (7), or all of A_i when shortlist = 0 (the summary
+ * gives no size; with shortlist = K the set equals fs_select_topk's).  K is the keys array
+ * [B,H,Nk,d] of type p->dtype; kbar/amax as for fs_select_topk.  The readout on these cells
+ * is fs_forward with idx.  Requires |A_i| <= 128 (W + P <= 128, or without pruning
+ * floor(Nk/s) <= 128), else FS_ERR_UNSUPPORTED; shortlist < 0 is FS_ERR_INVALID_ARG. */
+fs_status fs_select_topk_rerank(const fs_params *p, const void *Q, const void *K, const float *kbar,
+                                const float *amax, int shortlist, int32_t *idx, void *ws,
+                                size_t ws_bytes, void *stream);
+
 /* The whole forward pass, eq. (2): O = o^sr + alpha_h o^lr.
  * kbar/amax may be NULL (then computed here into the workspace) or caller-given summaries
  * (e.g. an archive summarised once for decoding).  idx may be NULL (then selected here)

@@ -194,6 +194,28 @@ extern "C" fs_status fs_select_topk(const fs_params *p, const void *Q, const flo
     return cuda_status(launch_selection(p, D, Q, kbar, amax, exitn, idx, at<int>(ws, L.flag), st));
 }
 
+extern "C" fs_status fs_select_topk_rerank(const fs_params *p, const void *Q, const void *K, const float *kbar,
+                                           const float *amax, int shortlist, int32_t *idx, void *ws,
+                                           size_t ws_bytes, void *stream) {
+    fs_status s = validate(p);
+    if (s != FS_OK) return s;
+    if (shortlist < 0) return FS_ERR_INVALID_ARG;
+    if (!rerank_supported(p)) return FS_ERR_UNSUPPORTED;
+    if (p->Nq == 0 || p->K == 0) return FS_OK;
+    if (!Q || !K || !idx) return FS_ERR_INVALID_ARG;
+    const WsLayout L = layout(p);
+    if (!ws || ws_bytes < L.total) return FS_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    const Dev D = make_dev(p);
+    if (D.C == 0 || !has_long_range(p)) {
+        return cuda_status(cudaMemsetAsync(idx, 0xff, (size_t)p->B * p->H * p->Nq * p->K * 4, st));
+    }
+    if (!kbar || !amax) return FS_ERR_INVALID_ARG;
+    int *exitn = at<int>(ws, L.exitn);
+    if (D.prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
+    return cuda_status(launch_rerank(D, p->dtype, Q, K, kbar, amax, exitn, shortlist, idx, st));
+}
+
 extern "C" fs_status fs_forward(const fs_params *p, const void *Q, const void *K, const void *V,
                                 const float *kbar, const float *amax, const int32_t *idx, void *O,
                                 void *ws, size_t ws_bytes, void *stream) {

@@ -102,7 +102,7 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 // ---- kernel ids for the diagnostics (fs_kernel_times) ----
 enum KernelId : int {
     kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
-    kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kNumKernels
+    kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kRerank, kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
@@ -123,6 +123,10 @@ bool params_have_long_range(const fs_params *p);
 cudaError_t launch_summaries(const Dev &P, fs_dtype dt, const void *K, float *kbar,
                              float *amax, cudaStream_t st);
 cudaError_t launch_exit_times(const Dev &P, const float *amax, int *exitn, cudaStream_t st);
+// eq. (12) token-level rerank of the selection (CUDA cores, |A_i| <= 128)
+bool rerank_supported(const fs_params *p);
+cudaError_t launch_rerank(const Dev &P, fs_dtype dt, const void *Q, const void *K, const float *kbar,
+                          const float *amax, const int *exitn, int shortlist, int32_t *idx, cudaStream_t st);
 cudaError_t launch_select(const Dev &P, fs_dtype dt, const void *Q, const float *kbar,
                           const float *amax, const int *exitn, int32_t *idx, cudaStream_t st);
 cudaError_t launch_readout(const Dev &P, fs_dtype dt, const void *Q, const void *K,
