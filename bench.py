@@ -389,6 +389,42 @@ def time_stream(fs, torch, inp, max_block=128, warmup=20):
                     "state size is independent of length" % (n_arch, max_block, len(steps) - warmup, wl.B, wl.H)}
 
 
+def time_rerank(fs, torch, inp, steps=5, warmup=3):
+    """The eq. (12) rerank variant of the forward pass on a workload: fs_forward_rerank
+    (summaries, rerank of all of A_i, then the fused readout + window on the reranked
+    cells).  Returns query-tokens/s and the rerank kernel's share (CUDA events)."""
+    wl = inp.wl
+    p = make_params(fs, inp)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    Q, K, V = (torch.from_numpy(x).cuda().to(dt) for x in (inp.Q, inp.K, inp.V))
+    O = torch.empty_like(Q)
+    ws = fs.alloc_workspace(p)
+    idx = torch.empty((wl.B, wl.H, wl.Nq, wl.K), dtype=torch.int32, device="cuda")
+
+    def step():
+        fs.forward_rerank(p, Q, K, V, O, ws, idx=idx)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    fs.timing_enable(True)
+    fs.kernel_times()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    kt = fs.kernel_times()
+    fs.timing_enable(False)
+    fs.sync_status(ws)
+    ms = a.elapsed_time(b) / steps
+    rr = kt.get("rerank", (0, 0.0))[1] / steps
+    return {"value": wl.queries / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "rerank_ms": rr,
+            "note": "fs_forward_rerank: eq. (12) token-level rerank of all of A_i (CUDA cores), then "
+                    "the fused tensor-core readout + window on the reranked cells; per-kernel "
+                    "timing on (events around each launch)"}
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup()
@@ -519,6 +555,8 @@ def run_ours(args):
                     extras["stream256k"] = time_stream(fs, torch, inp2)
                 del inp2
                 torch.cuda.empty_cache()
+            extras[wl.name + "_rerank"] = time_rerank(fs, torch, inp)
+            torch.cuda.empty_cache()
             line["other_workloads"] = extras
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -106,6 +106,15 @@ fs_status fs_select_topk_rerank(const fs_params *p, const void *Q, const void *K
                                 const float *amax, int shortlist, int32_t *idx, void *ws,
                                 size_t ws_bytes, void *stream);
 
+/* The forward pass with the eq. (12) rerank as its selection: fs_select_topk_rerank's
+ * cells (shortlist as there), then the readout on them and the window, O = o^sr + alpha_h
+ * o^lr.  kbar/amax may be NULL (computed here); idx, if not NULL, receives the selected
+ * cells [B,H,Nq,K].  bf16 runs the fused tensor-core readout + window on the reranked
+ * cells; f32 runs the CUDA-core readout.  Requirements as for fs_select_topk_rerank. */
+fs_status fs_forward_rerank(const fs_params *p, const void *Q, const void *K, const void *V,
+                            const float *kbar, const float *amax, int shortlist, int32_t *idx,
+                            void *O, void *ws, size_t ws_bytes, void *stream);
+
 /* The whole forward pass, eq. (2): O = o^sr + alpha_h o^lr.
  * kbar/amax may be NULL (then computed here into the workspace) or caller-given summaries
  * (e.g. an archive summarised once for decoding).  idx may be NULL (then selected here)

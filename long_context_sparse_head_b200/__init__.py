@@ -26,7 +26,7 @@ EXPORTS = ("fs_workspace_size", "fs_cell_summaries", "fs_select_topk", "fs_forwa
            "fs_host_scratch_size", "fs_forward_host", "fs_sync_status", "fs_status_string",
            "fs_launch_count", "fs_timing_enable", "fs_kernel_times", "fs_kernel_name",
            "fs_select_topk_noalloc", "fs_cache_bytes", "fs_cache_reset", "fs_cache_append",
-           "fs_cache_attend", "fs_cache_status", "fs_select_topk_rerank")
+           "fs_cache_attend", "fs_cache_status", "fs_select_topk_rerank", "fs_forward_rerank")
 
 
 class FsError(RuntimeError):
@@ -67,6 +67,7 @@ def load():
         L.fs_select_topk.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
         L.fs_select_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp]
         L.fs_select_topk_rerank.argtypes = [P, vp, vp, vp, vp, ctypes.c_int, vp, vp, sz, vp]
+        L.fs_forward_rerank.argtypes = [P, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp, sz, vp]
         L.fs_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.fs_host_scratch_size.argtypes = [P, ctypes.POINTER(sz)]
         L.fs_forward_host.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
@@ -181,6 +182,13 @@ def select_topk_rerank(params, Q, K, kbar, amax, idx, ws, shortlist=0, stream=No
                                         int(shortlist), _ptr(idx), _ptr(ws),
                                         ws.numel() * ws.element_size(), _stream(stream)),
            "fs_select_topk_rerank")
+
+
+def forward_rerank(params, Q, K, V, O, ws, kbar=None, amax=None, idx=None, shortlist=0, stream=None):
+    """The forward pass with the eq. (12) rerank as its selection (idx: optional output)."""
+    _check(load().fs_forward_rerank(params.ref(), _ptr(Q), _ptr(K), _ptr(V), _ptr(kbar), _ptr(amax),
+                                    int(shortlist), _ptr(idx), _ptr(O), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream)), "fs_forward_rerank")
 
 
 def select_topk_noalloc(params, Q, kbar, amax, idx, stream=None):

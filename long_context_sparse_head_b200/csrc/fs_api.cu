@@ -216,6 +216,49 @@ extern "C" fs_status fs_select_topk_rerank(const fs_params *p, const void *Q, co
     return cuda_status(launch_rerank(D, p->dtype, Q, K, kbar, amax, exitn, shortlist, idx, st));
 }
 
+extern "C" fs_status fs_forward_rerank(const fs_params *p, const void *Q, const void *K, const void *V,
+                                       const float *kbar, const float *amax, int shortlist, int32_t *idx,
+                                       void *O, void *ws, size_t ws_bytes, void *stream) {
+    fs_status s = validate(p);
+    if (s != FS_OK) return s;
+    if (shortlist < 0) return FS_ERR_INVALID_ARG;
+    if (!rerank_supported(p)) return FS_ERR_UNSUPPORTED;
+    if (p->Nq == 0) return FS_OK;
+    if (!Q || !K || !V || !O) return FS_ERR_INVALID_ARG;
+    if ((kbar == nullptr) != (amax == nullptr)) return FS_ERR_INVALID_ARG;
+    const WsLayout L = layout(p);
+    if (!ws || ws_bytes < L.total) return FS_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (!has_long_range(p)) {                      // window only; no cells to select
+        if (idx && p->K > 0 &&
+            cudaMemsetAsync(idx, 0xff, (size_t)p->B * p->H * p->Nq * p->K * 4, st) != cudaSuccess)
+            return FS_ERR_CUDA;
+        return run_forward(p, Q, K, V, nullptr, nullptr, nullptr, O, ws, st);
+    }
+    const Dev D = make_dev(p);
+    if (!kbar) {
+        float *kb = at<float>(ws, L.kbar), *am = at<float>(ws, L.amax);
+        if (launch_summaries(D, p->dtype, K, kb, am, st) != cudaSuccess) return FS_ERR_CUDA;
+        kbar = kb;
+        amax = am;
+    }
+    int *exitn = at<int>(ws, L.exitn);
+    if (D.prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
+    int32_t *sel = idx ? idx : at<int32_t>(ws, L.idx);
+    if (launch_rerank(D, p->dtype, Q, K, kbar, amax, exitn, shortlist, sel, st) != cudaSuccess) return FS_ERR_CUDA;
+    if (attn_tc_supported(p)) {                    // bf16: the fused tensor-core readout + window
+        uint32_t *tiles = at<uint32_t>(ws, L.tiles);
+        if (launch_idx_tiles(D, sel, tiles, at<int>(ws, L.flag), st) != cudaSuccess) return FS_ERR_CUDA;
+        float2 *lo = at<float2>(ws, L.rope_abs), *hi = lo + kRopeLo * 32;
+        void *krot = at<void>(ws, L.krot);
+        if (launch_rope_abs_table(p->Nk, p->rope_base, lo, hi, st) != cudaSuccess ||
+            launch_rope_keys(D, K, krot, lo, hi, st) != cudaSuccess)
+            return FS_ERR_CUDA;
+        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), st));
+    }
+    return run_forward(p, Q, K, V, kbar, amax, sel, O, ws, st);
+}
+
 extern "C" fs_status fs_forward(const fs_params *p, const void *Q, const void *K, const void *V,
                                 const float *kbar, const float *amax, const int32_t *idx, void *O,
                                 void *ws, size_t ws_bytes, void *stream) {

@@ -102,7 +102,7 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 // ---- kernel ids for the diagnostics (fs_kernel_times) ----
 enum KernelId : int {
     kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
-    kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kRerank, kNumKernels
+    kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kRerank, kIdxTiles, kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
@@ -127,6 +127,8 @@ cudaError_t launch_exit_times(const Dev &P, const float *amax, int *exitn, cudaS
 bool rerank_supported(const fs_params *p);
 cudaError_t launch_rerank(const Dev &P, fs_dtype dt, const void *Q, const void *K, const float *kbar,
                           const float *amax, const int *exitn, int shortlist, int32_t *idx, cudaStream_t st);
+// per-tile selection records (the fused kernel's input) from a selection idx
+cudaError_t launch_idx_tiles(const Dev &P, const int32_t *idx, uint32_t *tiles, int *dev_flag, cudaStream_t st);
 cudaError_t launch_select(const Dev &P, fs_dtype dt, const void *Q, const float *kbar,
                           const float *amax, const int *exitn, int32_t *idx, cudaStream_t st);
 cudaError_t launch_readout(const Dev &P, fs_dtype dt, const void *Q, const void *K,

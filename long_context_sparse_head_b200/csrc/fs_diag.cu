@@ -32,7 +32,7 @@ cudaEvent_t take_event() {
 const char *const kNames[kNumKernels] = {"cell_summaries", "exit_times", "select_topk",
                                          "readout", "window_combine", "rope_table",
                                          "window_tc", "attn_tc", "select_tc", "rope_keys",
-                                         "cache_append", "cache_attend", "rerank"};
+                                         "cache_append", "cache_attend", "rerank", "idx_tiles"};
 }  // namespace
 
 LaunchScope::LaunchScope(int id_, cudaStream_t st_) : id(id_), st(st_), slot(-1) {

@@ -9,9 +9,9 @@
 // TopP exit table, then
 //   - eq. (7) scores of every (row, admitted cell), one thread per pair;
 //   - eq. (12): each warp takes admitted cells in turn, stages the cell's 32 keys in
-//     shared memory, and lane r (the group's row r, query in registers) runs the 32 token
-//     logits through an online log-sum-exp: no reductions across lanes, and each key is
-//     read once per group instead of once per row;
+//     shared memory, and lane r (the group's row r, query in registers) computes the 32
+//     token logits, their max and sum of exponentials: no reductions across lanes, and
+//     each key is read once per group instead of once per row;
 //   - per row: the shortlist by eq. (7), then the top-K by eq. (12), by rank counting.
 // CUDA cores; |A_i| <= 128 cells.
 #include "fs_common.cuh"
@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(kThreads) rerank_kernel(const RerankArgs A, co
             r += A.lambda[h] * am[c] * erff(((float)(g0 + row - c * kS) - 0.5f * kS) * A.inv2sigma[h]);
         sm.r7[row][a] = r;
     }
-    // ---- eq. (12): warp per cell, lane = row, online log-sum-exp over the cell's tokens
+    // ---- eq. (12): warp per cell, lane = row, log-sum-exp over the cell's tokens
     float q[kD];
 #pragma unroll
     for (int e = 0; e < kD; e++) q[e] = sm.q[lane][e];
@@ -105,19 +105,38 @@ __global__ void __launch_bounds__(kThreads) rerank_kernel(const RerankArgs A, co
     for (int a = warp; a < nA; a += kWarps) {
         const int c = sm.acell[a];
         const T *src = Kbh + (size_t)c * kS * kD;
-        for (int e = lane; e < kS * kD; e += 32) sm.kt[warp][e / kD][e % kD] = to_f<T>(src[e]);
+        // the cell's 32 x 64 keys, 16-byte loads (coalesced), widened to float
+        for (int e = lane * Vec<T>::N; e < kS * kD; e += 32 * Vec<T>::N) {
+            float x[Vec<T>::N];
+            Vec<T>::load(src + e, x);
+#pragma unroll
+            for (int u = 0; u < Vec<T>::N; u++) sm.kt[warp][(e + u) / kD][(e + u) % kD] = x[u];
+        }
         __syncwarp();
-        float m = -INFINITY, se = 0.f;
+        // the 32 token logits (independent), then one max and one sum of exponentials
+        float lg[kS];
+#pragma unroll
         for (int j = 0; j < kS; j++) {
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            const float4 *kj = reinterpret_cast<const float4 *>(sm.kt[warp][j]);   // broadcast
 #pragma unroll
-            for (int e = 0; e < kD; e++) acc[e & 3] = fmaf(q[e], sm.kt[warp][j][e], acc[e & 3]);
-            const float x = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * A.scale;
-            const float mn = fmaxf(m, x);
-            se = se * expf(m - mn) + expf(x - mn);
-            m = mn;
+            for (int e4 = 0; e4 < kD / 4; e4++) {
+                const float4 k4 = kj[e4];
+                acc[0] = fmaf(q[4 * e4], k4.x, acc[0]);
+                acc[1] = fmaf(q[4 * e4 + 1], k4.y, acc[1]);
+                acc[2] = fmaf(q[4 * e4 + 2], k4.z, acc[2]);
+                acc[3] = fmaf(q[4 * e4 + 3], k4.w, acc[3]);
+            }
+            lg[j] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * A.scale;
         }
-        float r = m + logf(se);
+        float m = lg[0];
+#pragma unroll
+        for (int j = 1; j < kS; j++) m = fmaxf(m, lg[j]);
+        float se[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < kS; j++) se[j & 3] += exp2f((lg[j] - m) * 1.4426950408889634f);
+        const float sum = (se[0] + se[1]) + (se[2] + se[3]);
+        float r = m + logf(sum);
         if (A.lambda[h] != 0.f)
             r += A.lambda[h] * am[c] * erff(((float)(g0 + lane - c * kS) - 0.5f * kS) * A.inv2sigma[h]);
         sm.r12[lane][a] = r;
@@ -172,6 +191,78 @@ __global__ void __launch_bounds__(kThreads) rerank_kernel(const RerankArgs A, co
 }
 
 }  // namespace
+
+// Per-tile selection records for the fused kernel from a selection idx [B,H,Nq,K]: one
+// CTA per 128-row tile; the union of the rows' cells goes into a bitmap over the cells,
+// is compacted in ascending order, and each row marks the union positions of its cells.
+// A union above 128 cells (impossible for cells of A_i when W + P + 10 <= 128) raises the
+// check flag and is cut.
+__global__ void __launch_bounds__(128) idx_tiles_kernel(const int32_t *__restrict__ idx, int Nq, int K, int C,
+                                                        uint32_t *__restrict__ tiles, int *dev_flag) {
+    extern __shared__ uint32_t bm[];             // bitmap over cells [ceil(C / 32)]
+    __shared__ int ulist[128], wsum[4], s_tot;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int bh = blockIdx.y, r0 = blockIdx.x * 128, row = r0 + t;
+    const int nw = (C + 31) / 32;
+    for (int e = t; e < nw; e += 128) bm[e] = 0u;
+    if (t == 0) s_tot = 0;
+    __syncthreads();
+    const int32_t *mine = idx + ((size_t)bh * Nq + row) * K;
+    if (row < Nq)
+        for (int k = 0; k < K; k++) {
+            const int c = mine[k];
+            if (c >= 0 && c < C) atomicOr(&bm[c >> 5], 1u << (c & 31));
+        }
+    __syncthreads();
+    // ascending compaction: thread t owns words [t * wpt, (t + 1) * wpt)
+    const int wpt = (nw + 127) / 128;
+    int cnt = 0;
+    for (int e = t * wpt; e < min(nw, (t + 1) * wpt); e++) cnt += __popc(bm[e]);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int pos = incl - cnt;
+    for (int k = 0; k < warp; k++) pos += wsum[k];
+    if (t == 127) s_tot = pos + cnt;
+    for (int e = t * wpt; e < min(nw, (t + 1) * wpt); e++)
+        for (uint32_t w = bm[e]; w; w &= w - 1) {
+            if (pos < 128) ulist[pos] = 32 * e + __ffs(w) - 1;
+            pos++;
+        }
+    __syncthreads();
+    const int total = s_tot, nU = min(total, 128);
+    if (total > 128 && t == 0 && dev_flag) atomicExch(dev_flag, kFlagCheck);
+    uint32_t mw[4] = {0u, 0u, 0u, 0u};
+    if (row < Nq)
+        for (int k = 0; k < K; k++) {
+            const int c = mine[k];
+            if (c < 0) continue;
+            int lo = 0, hi = nU;                     // first union position >= c
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (ulist[mid] < c) lo = mid + 1; else hi = mid;
+            }
+            if (lo < nU && ulist[lo] == c) mw[lo >> 5] |= 1u << (lo & 31);
+        }
+    uint32_t *rec = tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords;
+    *reinterpret_cast<uint4 *>(rec + kTileMaskOff + 4 * t) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+    rec[kTileUlistOff + t] = t < nU ? (uint32_t)ulist[t] : 0xffffffffu;
+    if (t == 0) rec[kTileCountOff] = (uint32_t)nU;
+}
+
+cudaError_t launch_idx_tiles(const Dev &P, const int32_t *idx, uint32_t *tiles, int *dev_flag, cudaStream_t st) {
+    if (P.Nq == 0) return cudaSuccess;
+    const dim3 grid((P.Nq + 127) / 128, P.B * P.H);
+    const size_t smem = (size_t)((P.C + 31) / 32) * 4;
+    LaunchScope scope(kIdxTiles, st);
+    idx_tiles_kernel<<<grid, 128, smem, st>>>(idx, P.Nq, P.K, P.C, tiles, dev_flag);
+    return cudaGetLastError();
+}
 
 bool rerank_supported(const fs_params *p) {
     const int C = p->Nk / p->s;

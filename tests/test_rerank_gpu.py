@@ -102,3 +102,55 @@ def test_rerank_rescues_hidden_tokens():
     idx = run_rerank(inp)
     for h, r, c0 in planted:
         assert c0 in idx[0, h, r], (h, r, c0, idx[0, h, r])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", [dict(), dict(Nq=300, Nk=1700), dict(lam=0.6, sigma=300.0, shortlist=10)])
+def test_forward_rerank(dtype, case):
+    """fs_forward_rerank: the same cells as fs_select_topk_rerank, and the output of the
+    readout (fused tensor-core kernel in bf16) on them within tolerance of the oracle's."""
+    kw = dict(B=1, H=2, Nq=1536, Nk=1536, K=6, W=4, P=9, dtype=dtype, seed=403)
+    kw.update(case)
+    shortlist = kw.pop("shortlist", 0)
+    lam = kw.pop("lam", None)
+    sigma = kw.pop("sigma", 1024.0)
+    inp = generate(small("fwd_rerank", lam=lam, sigma=sigma, **kw))
+    wl = inp.wl
+    g = GpuRun(inp)
+    prob = oracle_for(inp)
+    g.summaries()
+    fs.select_topk_rerank(g.p, g.Q, g.K, g.kbar, g.amax, g.idx, g.ws, shortlist)
+    ref_idx = g.numpy(g.idx).copy()
+    idx2 = torch.full_like(g.idx, -7)
+    g.O.fill_(float("nan"))
+    fs.forward_rerank(g.p, g.Q, g.K, g.V, g.O, g.ws, idx=idx2, shortlist=shortlist)
+    fs.sync_status(g.ws)
+    idx2 = g.numpy(idx2)
+    assert np.array_equal(idx2, ref_idx)
+    rows = [(b, h, r) for b in range(wl.B) for h in range(wl.H) for r in range(wl.Nq)]
+    O = g.numpy(g.O).reshape(wl.B, wl.H, wl.Nq, wl.d)
+    got = np.stack([O[b, h, r] for b, h, r in rows])
+    err = np.abs(got - expected_output(inp, prob, rows, idx2)).max()
+    assert err <= TOL[wl.dtype], err
+
+
+def test_forward_rerank_full_size_sampled():
+    """The 64k prefill workload through fs_forward_rerank, judged on sampled rows."""
+    from workloads import CONFIGS
+    from tests._parity import sample_rows
+    inp = generate(CONFIGS["prefill64k"])
+    wl = inp.wl
+    g = GpuRun(inp)
+    prob = oracle_for(inp)
+    idx = torch.empty((wl.B, wl.H, wl.Nq, wl.K), dtype=torch.int32, device="cuda")
+    fs.forward_rerank(g.p, g.Q, g.K, g.V, g.O, g.ws, idx=idx)
+    fs.sync_status(g.ws)
+    idx = g.numpy(idx)
+    rows = sample_rows(wl, 48, seed=7)
+    kbar_o, amax_o = prob.summaries()
+    exact, tie = check_rerank(prob, kbar_o, amax_o, idx, rows, 0)
+    assert tie <= max(2, len(rows) // 20), (exact, tie)
+    O = g.numpy(g.O).reshape(wl.B, wl.H, wl.Nq, wl.d)
+    got = np.stack([O[b, h, r] for b, h, r in rows])
+    err = np.abs(got - expected_output(inp, prob, rows, idx)).max()
+    assert err <= TOL[wl.dtype], err
