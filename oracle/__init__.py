@@ -37,6 +37,7 @@ MUTATIONS = {
     "rope_key_sign": 1, "drop_prior": 2, "window_short": 3, "cand_loose": 4,
     "amax_mean": 5, "no_eps": 6, "alpha_on_sr": 7, "rope_in_readout": 8,
     "scale_d": 9, "tie_high_index": 10, "rerank_mean": 11, "rerank_rope": 12,
+    "bwd_no_rms": 13,
 }
 
 
@@ -61,6 +62,7 @@ def lib():
                                      ctypes.c_int, i32p, i32p, f64p]
         L.orc_rerank_row.argtypes = [P, f32p, f32p, f64p, f64p, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_int, ctypes.c_int, i32p, i32p, f64p]
+        L.orc_backward.argtypes = [P, f32p, f32p, f32p, i32p, f64p, f64p, f64p, f64p, f64p]
         L.orc_readout_rows.argtypes = [P, f32p, f32p, f32p, ctypes.c_longlong, i64p, i32p,
                                        ctypes.c_void_p, f64p]
         L.orc_readout_rows.restype = None
@@ -175,6 +177,18 @@ class Problem:
                                   np.ascontiguousarray(amax, np.float64),
                                   b, h, r, int(shortlist), idx, cells, scores)
         return idx[:self.p.K].copy(), cells[:ns].copy(), scores[:ns].copy()
+
+    def backward(self, idx, dO):
+        """Gradients of eq. (2) with the selection idx [B,H,Nq,K] held fixed, for the
+        upstream gradient dO [B,H,Nq,d]: (dQ, dK, dV, dalpha) in float64."""
+        B, H, Nq, Nk, d = self.p.B, self.p.H, self.p.Nq, self.p.Nk, self.d
+        dQ = np.zeros((B, H, Nq, d)); dK = np.zeros((B, H, Nk, d)); dV = np.zeros((B, H, Nk, d))
+        dal = np.zeros(H)
+        lib().orc_backward(ctypes.byref(self.p), self.Q, self.K, self.V,
+                           np.ascontiguousarray(idx, np.int32).reshape(-1),
+                           np.ascontiguousarray(dO, np.float64).reshape(-1),
+                           dQ.reshape(-1), dK.reshape(-1), dV.reshape(-1), dal)
+        return dQ, dK, dV, dal
 
     def readout_rows(self, rows, idx):
         """eq. (9) for the given flat rows on caller-given cells idx [n,K]: (u, o^lr)."""

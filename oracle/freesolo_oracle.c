@@ -26,6 +26,8 @@
  *   - ties in TopP and top-K: larger value first, then the lower cell index
  *   - |A_i| < K: all of A_i is selected; S_i empty gives o^lr = 0
  *   - W < 0 and P < 0 together mean "no pruning" (base FS: A_i = C_i)
+ *   - backward pass: the selection (a top-K, piecewise constant in Q and K) is held
+ *     fixed, and the summaries, which only feed the selection, get no gradient
  *   - eq. (12) reranks a shortlist: the `shortlist` best cells of A_i by eq. (7)
  *     (shortlist <= 0: all of A_i) are rescored by eq. (12) and the K best kept; its
  *     g_h is eq. (7)'s erf((i - p_c) / (2 sigma_h)) (eq. (11) uses the same name)
@@ -70,6 +72,7 @@ enum {
     MUT_TIE_HIGH_INDEX = 10, /* ties broken toward the higher cell index */
     MUT_RERANK_MEAN = 11,    /* eq. (12) with the mean logit instead of the log-sum-exp */
     MUT_RERANK_ROPE = 12,    /* eq. (12) with rotated query and keys */
+    MUT_BWD_NO_RMS = 13,     /* backward: RMSNorm treated as a constant scale */
 };
 
 int orc_num_cells(const orc_params *p) { return p->s > 0 ? p->Nk / p->s : 0; }
@@ -483,6 +486,151 @@ int orc_rerank_row(const orc_params *p, const float *Q, const float *K, const do
     for (int t = keep; t < p->K; t++) idx_out[t] = -1;
     free(sl); free(x); free(tmp); free(lg);
     return ns;
+}
+
+/* x rotated by R(pos)^T = R(-pos) (double vectors): the adjoint of the RoPE rotation */
+static void rope_rotate_back(const orc_params *p, const double *x, long long pos, double *out)
+{
+    const int d = p->d;
+    for (int m = 0; m < d / 2; m++) {
+        double theta = pow(p->rope_base, -2.0 * m / (double)d);
+        double ang = (double)pos * theta;
+        double cs = cos(ang), sn = sin(ang);
+        out[2 * m] = x[2 * m] * cs + x[2 * m + 1] * sn;
+        out[2 * m + 1] = -x[2 * m] * sn + x[2 * m + 1] * cs;
+    }
+}
+
+/* ---- backward of eq. (2) with the selection held fixed ----
+ * O_i = o_i^sr + alpha_h RMSNorm(u_i):
+ *   window (eqs. (3)-(4)):  o^sr = sum_j p_j v_j, p = softmax(l), l_j = (R_i q).(R_j k_j)/sqrt(d)
+ *   readout (eq. (9)):      u = sum_t pi_t v_t, pi = softmax(lambda), lambda_t = q.k_t/sqrt(d)
+ * For an upstream gradient dO, each softmax branch o = sum_j p_j v_j with output gradient
+ * g gives dv_j += p_j g, dl_j = p_j (g.v_j - g.o), and dl flows to q and k through the dot
+ * products (for the window, through the rotations and back by R^T).  RMSNorm y = u r,
+ * r = (mean(u^2) + eps)^(-1/2): du = r (dy - y (dy.y)/d).  dalpha_h = sum_i dO_i.y_i.
+ * idx [B,H,Nq,K] are the cells the forward pass selected.  Outputs are overwritten:
+ * dQ [B,H,Nq,d], dK, dV [B,H,Nk,d], dalpha [H].  Returns 0. */
+int orc_backward(const orc_params *p, const float *Q, const float *K, const float *V, const int *idx,
+                 const double *dO, double *dQ, double *dK, double *dV, double *dalpha)
+{
+    const int d = p->d, s = p->s, Kc = p->K, BH = p->B * p->H;
+    const double sc = logit_scale(p);
+    memset(dQ, 0, sizeof(double) * (size_t)BH * p->Nq * d);
+    memset(dK, 0, sizeof(double) * (size_t)BH * p->Nk * d);
+    memset(dV, 0, sizeof(double) * (size_t)BH * p->Nk * d);
+    memset(dalpha, 0, sizeof(double) * (size_t)p->H);
+    double *krot = (double *)malloc(sizeof(double) * (size_t)p->Nk * d);
+    double *lg = (double *)malloc(sizeof(double) * (size_t)(p->Nk > 0 ? p->Nk : 1));
+    double qrot[512], dqrot[512], dk[512], tmp[512], o[512], u[512], y[512], du[512];
+    for (int bh = 0; bh < BH; bh++) {
+        const int h = bh % p->H;
+        const double a = p->alpha ? p->alpha[h] : 0.0;
+        const float *Kbh = K + (size_t)bh * p->Nk * d, *Vbh = V + (size_t)bh * p->Nk * d;
+        double *dKbh = dK + (size_t)bh * p->Nk * d, *dVbh = dV + (size_t)bh * p->Nk * d;
+        for (int j = 0; j < p->Nk; j++) rope_rotate(p, Kbh + (size_t)j * d, p->pos0 + j, krot + (size_t)j * d);
+        for (int r = 0; r < p->Nq; r++) {
+            const long long i = (long long)(p->Nk - p->Nq) + r;
+            const float *q = Q + ((size_t)bh * p->Nq + r) * d;
+            const double *g = dO + ((size_t)bh * p->Nq + r) * d;
+            double *dq = dQ + ((size_t)bh * p->Nq + r) * d;
+            /* window branch */
+            rope_rotate(p, q, p->pos0 + i, qrot);
+            long long j0 = i - p->w < 0 ? 0 : i - p->w;
+            double mx = -INFINITY, den = 0.0;
+            for (long long j = j0; j <= i; j++) {
+                double dot = 0.0;
+                for (int m = 0; m < d; m++) dot += qrot[m] * krot[(size_t)j * d + m];
+                lg[j - j0] = dot * sc;
+                if (lg[j - j0] > mx) mx = lg[j - j0];
+            }
+            for (int m = 0; m < d; m++) o[m] = 0.0;
+            for (long long j = j0; j <= i; j++) {
+                lg[j - j0] = exp(lg[j - j0] - mx);
+                den += lg[j - j0];
+            }
+            for (long long j = j0; j <= i; j++) {
+                lg[j - j0] /= den;
+                for (int m = 0; m < d; m++) o[m] += lg[j - j0] * Vbh[(size_t)j * d + m];
+            }
+            double D = 0.0;
+            for (int m = 0; m < d; m++) D += g[m] * o[m];
+            for (int m = 0; m < d; m++) dqrot[m] = 0.0;
+            for (long long j = j0; j <= i; j++) {
+                const double pj = lg[j - j0];
+                double dp = 0.0;
+                for (int m = 0; m < d; m++) dp += g[m] * Vbh[(size_t)j * d + m];
+                const double ds = pj * (dp - D) * sc;
+                for (int m = 0; m < d; m++) {
+                    dVbh[(size_t)j * d + m] += pj * g[m];
+                    dqrot[m] += ds * krot[(size_t)j * d + m];
+                    dk[m] = ds * qrot[m];
+                }
+                rope_rotate_back(p, dk, p->pos0 + j, tmp);
+                for (int m = 0; m < d; m++) dKbh[(size_t)j * d + m] += tmp[m];
+            }
+            rope_rotate_back(p, dqrot, p->pos0 + i, tmp);
+            for (int m = 0; m < d; m++) dq[m] += tmp[m];
+            /* readout branch */
+            const int *sel = idx + ((size_t)bh * p->Nq + r) * Kc;
+            int ncell = 0;
+            for (int e = 0; e < Kc; e++) ncell += sel[e] >= 0;
+            if (ncell == 0) continue;
+            mx = -INFINITY;
+            int t = 0;
+            for (int e = 0; e < Kc; e++) {
+                if (sel[e] < 0) continue;
+                for (int j = sel[e] * s; j < (sel[e] + 1) * s; j++, t++) {
+                    double dot = 0.0;
+                    for (int m = 0; m < d; m++) dot += (double)q[m] * Kbh[(size_t)j * d + m];
+                    lg[t] = dot * sc;
+                    if (lg[t] > mx) mx = lg[t];
+                }
+            }
+            const int ntok = t;
+            den = 0.0;
+            for (t = 0; t < ntok; t++) { lg[t] = exp(lg[t] - mx); den += lg[t]; }
+            for (int m = 0; m < d; m++) u[m] = 0.0;
+            t = 0;
+            for (int e = 0; e < Kc; e++) {
+                if (sel[e] < 0) continue;
+                for (int j = sel[e] * s; j < (sel[e] + 1) * s; j++, t++) {
+                    lg[t] /= den;
+                    for (int m = 0; m < d; m++) u[m] += lg[t] * Vbh[(size_t)j * d + m];
+                }
+            }
+            double ms = 0.0;
+            for (int m = 0; m < d; m++) ms += u[m] * u[m];
+            const double rin = 1.0 / sqrt(ms / d + p->rms_eps);
+            double dyy = 0.0, gy = 0.0;
+            for (int m = 0; m < d; m++) {
+                y[m] = u[m] * rin;
+                dyy += a * g[m] * y[m];
+                gy += g[m] * y[m];
+            }
+            dalpha[h] += gy;
+            for (int m = 0; m < d; m++)
+                du[m] = p->mutation == MUT_BWD_NO_RMS ? rin * a * g[m] : rin * (a * g[m] - y[m] * dyy / d);
+            D = 0.0;
+            for (int m = 0; m < d; m++) D += du[m] * u[m];
+            t = 0;
+            for (int e = 0; e < Kc; e++) {
+                if (sel[e] < 0) continue;
+                for (int j = sel[e] * s; j < (sel[e] + 1) * s; j++, t++) {
+                    double dp = 0.0;
+                    for (int m = 0; m < d; m++) dp += du[m] * Vbh[(size_t)j * d + m];
+                    const double ds = lg[t] * (dp - D) * sc;
+                    for (int m = 0; m < d; m++) {
+                        dVbh[(size_t)j * d + m] += lg[t] * du[m];
+                        dq[m] += ds * Kbh[(size_t)j * d + m];
+                        dKbh[(size_t)j * d + m] += ds * q[m];
+                    }
+                }
+            }
+        }
+    }
+    free(krot); free(lg);
+    return 0;
 }
 
 /* ---- single-step entry points for the tests ---- */

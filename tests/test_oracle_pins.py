@@ -370,6 +370,56 @@ def test_rerank_pins():
     assert _rerank_pin_failures() == []
 
 
+# ---------------------------------------------------------------- backward
+def _fd_failures(mutation=0, n_entries=12):
+    """Gradients of L = sum(dO * O) from the oracle's backward against central finite
+    differences of its forward (selection held fixed: perturbations that change it are
+    skipped).  Returns the names of the inputs whose check fails."""
+    inp = tiny(d=8, Nq=96, Nk=96, w=16, s=8, K=3, W=2, P=3, lam=0.5, sigma=16.0, seed=47)
+    wl = inp.wl
+
+    def problem(Q, K, V, alpha):
+        return oracle.Problem(Q, K, V, w=wl.w, s=wl.s, K_cells=wl.K, W=wl.W, P=wl.P, alpha=alpha,
+                              lam=inp.lam, sigma=inp.sigma, rope_base=wl.rope_base,
+                              rms_eps=wl.rms_eps, mutation=mutation)
+    O, idx = problem(inp.Q, inp.K, inp.V, inp.alpha).forward(want_idx=True)
+    dO = np.random.default_rng(48).standard_normal(O.shape)
+    grads = problem(inp.Q, inp.K, inp.V, inp.alpha).backward(idx, dO)
+    rng = np.random.default_rng(49)
+    fails = []
+    for name, arr_i, g in (("Q", 0, grads[0]), ("K", 1, grads[1]), ("V", 2, grads[2])):
+        base = [inp.Q, inp.K, inp.V]
+        for _ in range(n_entries):
+            e = tuple(int(rng.integers(0, n)) for n in base[arr_i].shape)
+            vals = []
+            for sgn in (1, -1):
+                arrs = [a.copy() for a in base]
+                arrs[arr_i][e] = np.float32(arrs[arr_i][e] + sgn * 2.0 ** -10)
+                O2, idx2 = problem(*arrs, inp.alpha).forward(want_idx=True)
+                vals.append((float((dO * O2).sum()), float(arrs[arr_i][e]), np.array_equal(idx2, idx)))
+            if not (vals[0][2] and vals[1][2]):
+                continue
+            fd = (vals[0][0] - vals[1][0]) / (vals[0][1] - vals[1][1])
+            if abs(fd - g[e]) > 1e-4 * max(1.0, abs(g[e])):
+                fails.append(name)
+                break
+    for h in range(wl.H):
+        vals = []
+        for sgn in (1, -1):
+            al = np.array(inp.alpha, np.float64)
+            al[h] += sgn * 1e-4
+            O2, _ = problem(inp.Q, inp.K, inp.V, al).forward(want_idx=True)
+            vals.append(float((dO * O2).sum()))
+        if abs((vals[0] - vals[1]) / 2e-4 - grads[3][h]) > 1e-4 * max(1.0, abs(grads[3][h])):
+            fails.append("alpha")
+            break
+    return fails
+
+
+def test_backward_matches_finite_differences():
+    assert _fd_failures(n_entries=20) == []
+
+
 # ---------------------------------------------------------------- sensitivity
 def _pins_fail(mutation):
     """Run a compact set of the pins above against a mutated oracle; True if any fails."""
@@ -392,6 +442,7 @@ def _pins_fail(mutation):
     except Exception:
         failures.append("golden_prune")
     failures += _rerank_pin_failures(mutation)
+    failures += _fd_failures(mutation, n_entries=6)
     return failures
 
 
