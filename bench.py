@@ -425,6 +425,53 @@ def time_rerank(fs, torch, inp, steps=5, warmup=3):
                     "timing on (events around each launch)"}
 
 
+def time_backward(fs, torch, inp, steps=3, warmup=3):
+    """The backward pass of eq. (2) on a workload (fs_backward on the cells fs_select_topk
+    chose; the selection is outside the timed region).  Returns query-tokens/s and the
+    per-kernel split (CUDA events around each launch)."""
+    wl = inp.wl
+    p = make_params(fs, inp)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    Q, K, V = (torch.from_numpy(x).cuda().to(dt) for x in (inp.Q, inp.K, inp.V))
+    ws = fs.alloc_workspace(p)
+    C = wl.Nk // wl.s
+    kbar = torch.empty((wl.B, wl.H, C, wl.d), dtype=torch.float32, device="cuda")
+    amax = torch.empty((wl.B, wl.H, C), dtype=torch.float32, device="cuda")
+    idx = torch.empty((wl.B, wl.H, wl.Nq, wl.K), dtype=torch.int32, device="cuda")
+    fs.cell_summaries(p, K, kbar, amax)
+    fs.select_topk(p, Q, kbar, amax, idx, ws)
+    fs.sync_status(ws)
+    del ws
+    dO = torch.randn(Q.shape, generator=torch.Generator(device="cuda").manual_seed(5), device="cuda").to(dt)
+    dQ = torch.empty(Q.shape, dtype=torch.float32, device="cuda")
+    dK = torch.empty(K.shape, dtype=torch.float32, device="cuda")
+    dV = torch.empty_like(dK)
+    dal = torch.empty(wl.H, dtype=torch.float32, device="cuda")
+    bws = fs.alloc_backward_workspace(p)
+
+    def step():
+        fs.backward(p, Q, K, V, idx, dO, dQ, dK, dV, dal, bws)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    fs.timing_enable(True)
+    fs.kernel_times()
+    step()
+    torch.cuda.synchronize()
+    kt = {k: round(v[1], 3) for k, v in fs.kernel_times().items() if k.startswith("bwd")}
+    fs.timing_enable(False)
+    return {"value": wl.queries / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "kernel_ms": kt,
+            "note": "fs_backward (dQ, dK, dV, dalpha in float32; CUDA cores) on fs_select_topk's "
+                    "cells; selection outside the timed region"}
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup()
@@ -556,6 +603,8 @@ def run_ours(args):
                 del inp2
                 torch.cuda.empty_cache()
             extras[wl.name + "_rerank"] = time_rerank(fs, torch, inp)
+            torch.cuda.empty_cache()
+            extras[wl.name + "_backward"] = time_backward(fs, torch, inp)
             torch.cuda.empty_cache()
             line["other_workloads"] = extras
     if rank == 0:

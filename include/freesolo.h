@@ -167,6 +167,27 @@ const char *fs_status_string(fs_status s);
 fs_status fs_select_topk_noalloc(const fs_params *p, const void *Q, const float *kbar,
                                  const float *amax, int32_t *idx, void *stream);
 
+/* ---- backward pass of eq. (2) ----
+ * Gradients of O = o^sr + alpha_h RMSNorm(u) (eqs. (2)-(4), (9)) with respect to Q, K, V
+ * and alpha, for an upstream gradient dO, with the selection held fixed: the cells idx
+ * [B,H,Nq,K] the forward pass read (from fs_select_topk, or fs_forward_rerank's idx).  The
+ * top-K is piecewise constant in Q and K, and the summaries only feed it, so neither
+ * carries a gradient (reading; the summary gives no backward pass).
+ *   window:  dv_j += p_j dO, dl_j = p_j (dO.v_j - dO.o^sr), through the RoPE rotations
+ *   readout: du = r (dy - y (dy.y)/d) with y = u r, r = (mean(u^2)+eps)^(-1/2),
+ *            dy = alpha_h dO; then the same softmax rule on NoPE logits
+ *   dalpha_h = sum_i dO_i . y_i
+ * Q, K, V, dO are device arrays of type p->dtype ([B,H,Nq,d] / [B,H,Nk,d]); dQ [B,H,Nq,d],
+ * dK, dV [B,H,Nk,d] and dalpha [H] (or NULL) are device float32 outputs, overwritten.
+ * idx entries outside [0, Nk/s) (the -1 padding) are skipped; a row with no cell has y = 0.
+ * bws/bws_bytes: device scratch of fs_backward_workspace_size bytes (rotated keys and
+ * queries, per-row softmax terms, the readout's du, the cell-to-rows lists).  Enqueued on
+ * `stream`; FS_ERR_INVALID_ARG / FS_ERR_UNSUPPORTED as for fs_forward.  CUDA cores. */
+fs_status fs_backward_workspace_size(const fs_params *p, size_t *bytes);
+fs_status fs_backward(const fs_params *p, const void *Q, const void *K, const void *V, const int32_t *idx,
+                      const void *dO, float *dQ, float *dK, float *dV, float *dalpha, void *bws,
+                      size_t bws_bytes, void *stream);
+
 /* ---- FS-L streaming cache ("FreeSolo" summary, "Practical Implications" 3: bounded
  * memory, O((P+W)s + w + B + s)d token state per head, independent of sequence length) ----
  * Tokens arrive in blocks of at most max_block (the B of that bound); after each block,

@@ -26,7 +26,8 @@ EXPORTS = ("fs_workspace_size", "fs_cell_summaries", "fs_select_topk", "fs_forwa
            "fs_host_scratch_size", "fs_forward_host", "fs_sync_status", "fs_status_string",
            "fs_launch_count", "fs_timing_enable", "fs_kernel_times", "fs_kernel_name",
            "fs_select_topk_noalloc", "fs_cache_bytes", "fs_cache_reset", "fs_cache_append",
-           "fs_cache_attend", "fs_cache_status", "fs_select_topk_rerank", "fs_forward_rerank")
+           "fs_cache_attend", "fs_cache_status", "fs_select_topk_rerank", "fs_forward_rerank",
+           "fs_backward_workspace_size", "fs_backward")
 
 
 class FsError(RuntimeError):
@@ -208,6 +209,25 @@ def forward_host(params, hQ, hK, hV, hO, dscratch, stream=None):
     _check(load().fs_forward_host(params.ref(), _ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hO),
                                   _ptr(dscratch), dscratch.numel() * dscratch.element_size(),
                                   _stream(stream)), "fs_forward_host")
+
+
+def backward_workspace_size(params):
+    n = ctypes.c_size_t()
+    _check(load().fs_backward_workspace_size(params.ref(), ctypes.byref(n)), "fs_backward_workspace_size")
+    return n.value
+
+
+def alloc_backward_workspace(params, device="cuda"):
+    import torch
+    return torch.empty(backward_workspace_size(params), dtype=torch.uint8, device=device)
+
+
+def backward(params, Q, K, V, idx, dO, dQ, dK, dV, dalpha, bws, stream=None):
+    """Gradients of eq. (2) for the upstream gradient dO with the cells idx held fixed:
+    dQ, dK, dV (float32, [B,H,N,d]) and dalpha (float32 [H], or None)."""
+    _check(load().fs_backward(params.ref(), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(dO),
+                              _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dalpha), _ptr(bws),
+                              bws.numel() * bws.element_size(), _stream(stream)), "fs_backward")
 
 
 def sync_status(ws, stream=None):

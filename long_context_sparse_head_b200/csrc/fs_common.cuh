@@ -102,7 +102,8 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 // ---- kernel ids for the diagnostics (fs_kernel_times) ----
 enum KernelId : int {
     kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
-    kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kRerank, kIdxTiles, kNumKernels
+    kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kRerank, kIdxTiles, kBwdRotate, kBwdRows,
+    kBwdWindowKv, kBwdCells, kBwdReadoutKv, kBwdDalpha, kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.

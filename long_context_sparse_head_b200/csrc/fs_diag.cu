@@ -32,7 +32,9 @@ cudaEvent_t take_event() {
 const char *const kNames[kNumKernels] = {"cell_summaries", "exit_times", "select_topk",
                                          "readout", "window_combine", "rope_table",
                                          "window_tc", "attn_tc", "select_tc", "rope_keys",
-                                         "cache_append", "cache_attend", "rerank", "idx_tiles"};
+                                         "cache_append", "cache_attend", "rerank", "idx_tiles",
+                                         "bwd_rotate", "bwd_rows", "bwd_window_kv", "bwd_cells",
+                                         "bwd_readout_kv", "bwd_dalpha"};
 }  // namespace
 
 LaunchScope::LaunchScope(int id_, cudaStream_t st_) : id(id_), st(st_), slot(-1) {

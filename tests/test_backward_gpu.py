@@ -1,0 +1,90 @@
+"""GPU parity of the backward pass of eq. (2) (fs_backward) against the float64 oracle's
+Problem.backward, on the oracle's own selection (the cells are an input held fixed).
+
+Both sides see the same bf16-representable inputs; the GPU accumulates in float32.  The
+bar is the dtype's output tolerance (2e-2 bf16, 1e-4 f32) relative to the gradient's scale
+max(1, max|ref|), for dQ, dK, dV and dalpha separately."""
+import numpy as np
+import pytest
+import torch
+
+import long_context_sparse_head_b200 as fs
+from workloads import generate, small, upstream_grad
+from tests._parity import TOL, oracle_for, params_for, tdtype
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_backward(inp, idx, dO, with_dalpha=True):
+    wl = inp.wl
+    p = params_for(inp)
+    dt = tdtype(wl)
+    Q, K, V, G = (torch.from_numpy(np.ascontiguousarray(x)).cuda().to(dt) for x in (inp.Q, inp.K, inp.V, dO))
+    I = torch.from_numpy(np.ascontiguousarray(idx, np.int32)).cuda()
+    dQ = torch.full((wl.B, wl.H, wl.Nq, wl.d), float("nan"), device="cuda")
+    dK = torch.full((wl.B, wl.H, wl.Nk, wl.d), float("nan"), device="cuda")
+    dV = torch.full_like(dK, float("nan"))
+    dal = torch.full((wl.H,), float("nan"), device="cuda") if with_dalpha else None
+    bws = fs.alloc_backward_workspace(p)
+    fs.backward(p, Q, K, V, I, G, dQ, dK, dV, dal, bws)
+    torch.cuda.synchronize()
+    out = [t.cpu().numpy().astype(np.float64) for t in (dQ, dK, dV)]
+    return out + [dal.cpu().numpy().astype(np.float64) if with_dalpha else None]
+
+
+def compare(got, ref, dtype):
+    for name, g, r in zip(("dQ", "dK", "dV", "dalpha"), got, ref):
+        if g is None:
+            continue
+        assert np.isfinite(g).all(), name
+        scale = max(1.0, float(np.abs(r).max()) if r.size else 1.0)
+        err = float(np.abs(g - r).max()) if r.size else 0.0
+        assert err <= TOL[dtype] * scale, (name, err, scale)
+
+
+def run_case(inp, seed=77):
+    prob = oracle_for(inp)
+    _, idx = prob.forward(want_idx=True)
+    dO = upstream_grad(inp.wl, seed)
+    ref = prob.backward(idx, dO)
+    got = gpu_backward(inp, idx, dO)
+    compare(got, ref, inp.wl.dtype)
+    return idx
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", [
+    dict(),                                        # FS-L, early rows with -1 padding
+    dict(lam=0.6, sigma=300.0),                    # erf prior on (a different selection)
+    dict(Nq=300, Nk=1700),                         # appended queries, ragged last cell
+    dict(W=-1, P=-1, K=5, Nq=1200, Nk=1200),       # base FS
+    dict(w=64, K=4, W=2, P=5, Nq=777, Nk=1001),    # short window, ragged everything
+    dict(B=2, H=3, K=3, Nq=640, Nk=640),           # several (b, h)
+])
+def test_backward_small(dtype, case):
+    kw = dict(B=1, H=2, Nq=1536, Nk=1536, K=6, W=4, P=9, dtype=dtype, seed=501)
+    kw.update(case)
+    lam = kw.pop("lam", None)
+    sigma = kw.pop("sigma", 1024.0)
+    run_case(generate(small("bwd", lam=lam, sigma=sigma, **kw)))
+
+
+def test_backward_no_cells_and_no_dalpha():
+    """Rows with no candidate cell (prefix shorter than w + s) have y = 0: only the window
+    carries gradient; dalpha = NULL is accepted."""
+    inp = generate(small("bwd_short", Nq=500, Nk=500, K=4, W=2, P=3, dtype="f32", seed=502))
+    prob = oracle_for(inp)
+    _, idx = prob.forward(want_idx=True)
+    assert (idx < 0).all()
+    dO = upstream_grad(inp.wl, 5)
+    ref = prob.backward(idx, dO)
+    got = gpu_backward(inp, idx, dO, with_dalpha=False)
+    compare(got[:3], ref[:3], "f32")
+    assert np.abs(ref[3]).max() == 0.0
+
+
+def test_backward_empty_queries():
+    """Nq = 0: nothing to differentiate; dK = dV = 0 for every key."""
+    inp = generate(small("bwd_empty", Nq=0, Nk=256, dtype="f32", seed=503))
+    got = gpu_backward(inp, np.zeros((1, 2, 0, inp.wl.K), np.int32), np.zeros((1, 2, 0, 64), np.float32))
+    assert np.abs(got[1]).max() == 0.0 and np.abs(got[2]).max() == 0.0 and np.abs(got[3]).max() == 0.0

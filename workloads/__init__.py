@@ -86,7 +86,7 @@ def _normal_fill(ss_children, shape, scale):
     """N(0,1)*scale float32 array; one independent stream per leading (b, h) slice,
     filled by a thread pool (deterministic whatever the scheduling)."""
     out = np.empty(shape, np.float32)
-    flat = out.reshape(-1, *shape[2:])
+    flat = out.reshape(shape[0] * shape[1], *shape[2:])
 
     def fill(t):
         g = np.random.Generator(np.random.PCG64(ss_children[t]))
@@ -176,6 +176,13 @@ def generate(wl: Workload) -> Inputs:
         lam = np.full(H, wl.lam, np.float64)
         sig = np.full(H, wl.sigma, np.float64)
     return Inputs(wl, Q, K, V, alpha, lam, sig, needles)
+
+
+def upstream_grad(wl: Workload, seed: int) -> np.ndarray:
+    """A seeded N(0,1) upstream gradient dO [B,H,Nq,d] for the backward pass (bf16 values
+    for bf16 workloads), float32."""
+    g = np.random.default_rng(seed).standard_normal((wl.B, wl.H, wl.Nq, wl.d)).astype(np.float32)
+    return round_bf16(g) if wl.dtype == "bf16" else g
 
 
 def small(name="small", **kw) -> Workload:
