@@ -4,7 +4,7 @@ TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's C
 baseline may import this package; the CUDA library and its Python binding never do.
 
 It follows the "FreeSolo" technical summary (picx.dev/p/IEuVxx), §3.1 eq. (2),
-§3.2 eqs. (3)-(4) and §3.3 eqs. (5), (7)-(9); the readings taken where the page is
+§3.2 eqs. (3)-(4), §3.3 eqs. (5), (7)-(9) and §3.4 eqs. (10)-(12); the readings taken where the page is
 silent are stated at the top of the C source.  Inputs are float32 arrays holding
 the exact input values (bf16 inputs widened); all arithmetic is float64.
 """
@@ -37,7 +37,7 @@ MUTATIONS = {
     "rope_key_sign": 1, "drop_prior": 2, "window_short": 3, "cand_loose": 4,
     "amax_mean": 5, "no_eps": 6, "alpha_on_sr": 7, "rope_in_readout": 8,
     "scale_d": 9, "tie_high_index": 10, "rerank_mean": 11, "rerank_rope": 12,
-    "bwd_no_rms": 13,
+    "bwd_no_rms": 13, "tree_no_rho": 14, "tree_pmax": 15, "tree_sort_desc": 16,
 }
 
 
@@ -66,6 +66,11 @@ def lib():
         L.orc_readout_rows.argtypes = [P, f32p, f32p, f32p, ctypes.c_longlong, i64p, i32p,
                                        ctypes.c_void_p, f64p]
         L.orc_readout_rows.restype = None
+        L.orc_tree_select_rows.argtypes = [P, f32p, f64p, f64p, ctypes.c_void_p, ctypes.c_int,
+                                           ctypes.c_double, ctypes.c_longlong, ctypes.c_void_p,
+                                           i32p, f64p]
+        L.orc_tree_node.argtypes = [P, f32p, f64p, f64p, ctypes.c_void_p] + [ctypes.c_int] * 7 + [
+            ctypes.c_double, i32p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]
         L.orc_rope.argtypes = [P, f32p, ctypes.c_longlong, f64p]
         L.orc_rope.restype = None
         _lib = L
@@ -189,6 +194,41 @@ class Problem:
                            np.ascontiguousarray(dO, np.float64).reshape(-1),
                            dQ.reshape(-1), dK.reshape(-1), dV.reshape(-1), dal)
         return dQ, dK, dV, dal
+
+    def tree_select(self, kbar, amax, beam, c_explore=1.0, tau=None, rows=None):
+        """FS-B selection (eqs. (10)-(11), readings in the C source) for flat rows (or all):
+        (idx [n,K] ascending -1 padded, margin [n]: smallest relative gap at a beam cut)."""
+        n = self.B * self.H * self.Nq if rows is None else len(rows)
+        rows_arr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+        tau_arr = None if tau is None else np.ascontiguousarray(tau, dtype=np.float64)
+        idx = np.zeros((max(n, 1), max(self.p.K, 1)), np.int32)
+        margin = np.ones(max(n, 1), np.float64)
+        vp = lambda a: None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+        rc = lib().orc_tree_select_rows(ctypes.byref(self.p), self.Q,
+                                        np.ascontiguousarray(kbar, np.float64).reshape(-1),
+                                        np.ascontiguousarray(amax, np.float64).reshape(-1),
+                                        vp(tau_arr), int(beam), float(c_explore), n, vp(rows_arr),
+                                        idx.reshape(-1), margin)
+        if rc != 0:
+            raise ValueError("oracle rejected the FS-B problem")
+        return idx[:n, :self.p.K], margin[:n]
+
+    def tree_node(self, kbar, amax, b, h, forest, k, blk, v, r, c_explore=1.0, tau=None):
+        """One FS-B tree node: (leaf cells in code order, U_v of eq. (11) for row r,
+        forest sequence length), or (None, None, n) if the node does not exist."""
+        leaves = np.zeros(1 << max(k, 0), np.int32)
+        U = ctypes.c_double()
+        nseq = ctypes.c_int()
+        tau_arr = None if tau is None else np.ascontiguousarray(tau, dtype=np.float64)
+        cnt = lib().orc_tree_node(ctypes.byref(self.p), self.Q,
+                                  np.ascontiguousarray(kbar, np.float64).reshape(-1),
+                                  np.ascontiguousarray(amax, np.float64).reshape(-1),
+                                  None if tau_arr is None else tau_arr.ctypes.data_as(ctypes.c_void_p),
+                                  b, h, forest, k, blk, v, r, float(c_explore), leaves,
+                                  ctypes.byref(U), ctypes.byref(nseq))
+        if cnt < 0:
+            return None, None, nseq.value
+        return leaves[:cnt].copy(), U.value, nseq.value
 
     def readout_rows(self, rows, idx):
         """eq. (9) for the given flat rows on caller-given cells idx [n,K]: (u, o^lr)."""

@@ -13,7 +13,9 @@
  *                          eq. (7)   cell score r_ic with the erf position prior
  *                          eq. (8)   FS-L pruning A_i = Recent_W(C_i) u TopP(a_c)
  *                          eq. (9)   NoPE token readout over the selected cells, RMSNorm
- *   §3.4                   eq. (12)  token-level rerank: a cell scored by the log-sum-exp
+ *   §3.4                   eqs. (10)-(11) FS-B: beam search over two causal forests of
+ *                                    balanced trees (all candidates; cells with a_c >= tau_h)
+ *                          eq. (12)  token-level rerank: a cell scored by the log-sum-exp
  *                                    of its tokens' NoPE logits plus the prior term
  * "Introduction and Theoretical Foundation": RoPE (Su et al.) stays inside the
  * local window; long-range routing and readout use unrotated vectors.
@@ -31,6 +33,8 @@
  *   - eq. (12) reranks a shortlist: the `shortlist` best cells of A_i by eq. (7)
  *     (shortlist <= 0: all of A_i) are rescored by eq. (12) and the K best kept; its
  *     g_h is eq. (7)'s erf((i - p_c) / (2 sigma_h)) (eq. (11) uses the same name)
+ *   - FS-B (eqs. (10)-(11)): the forests, leaf order, node statistics and beam rules
+ *     are stated above orc_tree_select_rows
  *
  * Every quantity is computed in double from the float32 inputs (bf16 inputs are
  * passed as their exact float32 values).  No tiling, fusion or reordering beyond
@@ -73,6 +77,9 @@ enum {
     MUT_RERANK_MEAN = 11,    /* eq. (12) with the mean logit instead of the log-sum-exp */
     MUT_RERANK_ROPE = 12,    /* eq. (12) with rotated query and keys */
     MUT_BWD_NO_RMS = 13,     /* backward: RMSNorm treated as a constant scale */
+    MUT_TREE_NO_RHO = 14,    /* eq. (11) without the c ||q|| rho_v term */
+    MUT_TREE_PMAX = 15,      /* eq. (11) prior at the latest cell of v instead of p_v^min */
+    MUT_TREE_SORT_DESC = 16, /* tree leaves in descending code order */
 };
 
 int orc_num_cells(const orc_params *p) { return p->s > 0 ? p->Nk / p->s : 0; }
@@ -677,4 +684,322 @@ void orc_readout_rows(const orc_params *p, const float *Q, const float *K, const
 void orc_rope(const orc_params *p, const float *x, long long pos, double *out)
 {
     rope_rotate(p, x, pos, out);
+}
+
+/* ==== FS-B: balanced-tree search over two causal forests (§3.4 eqs. (10)-(11)) ====
+ * The summary prints the admitted sets (10) and the node score (11) only; the rest is
+ * read as follows (the "growing archive" with radix-sort-built balanced trees, §3.4, §5):
+ *  - a forest is built over a sequence of cells: forest 0 over all cells in time order
+ *    (A^0_i = C_i), forest tau over the cells with a_c >= tau_h in time order (A^tau_i);
+ *  - for every k and every aligned block of 2^k consecutive sequence entries there is one
+ *    balanced binary tree over the block's cells; a prefix of n entries is covered by the
+ *    trees of the set bits of n (those a binary counter holds after n insertions), so a
+ *    query only reaches cells of its prefix (causal);
+ *  - a tree's leaves are its cells radix-sorted by a 16-bit code, the signs of the first
+ *    16 coordinates of kbar_c (coordinate 0 most significant), ties by time; node v of the
+ *    complete binary tree over that order holds a run of consecutive leaves;
+ *  - mu_v = mean of kbar_c, rho_v = max ||kbar_c - mu_v||, A_v = max a_c, p_v^min =
+ *    min p_c over the leaves of v; c of eq. (11) is a parameter; g_h is eq. (7)'s;
+ *  - beam search of width beta on each forest: the beam starts as the prefix's roots (the
+ *    beta best); then every internal node of the beam is replaced by its two children and
+ *    the beta best kept (by U_v, ties to the lower p_v^min), until only leaves remain;
+ *  - S_i = the K best cells by eq. (7) among the leaves both beams end on (a leaf's U_v
+ *    is its eq. (7) score), ascending, -1 padded.
+ * With c >= 1 and lambda_h >= 0, U_v bounds the eq. (7) score of every leaf below v
+ * (Cauchy-Schwarz for the dot product; erf increasing for the prior). */
+
+typedef struct {
+    int n, L;          /* sequence length; levels k = 0 .. L-1 (2^k <= n) */
+    int *seq;          /* [n] cell of each sequence entry */
+    int **ord;         /* ord[k][(blk << k) + j]: leaf j (code order) of block blk */
+    double **mu;       /* mu[k][((blk << (k+1)) + v) * d], heap index v in [1, 2^(k+1)) */
+    double **rho, **A;
+    int **pmin;
+} orc_forest;
+
+static unsigned cell_code(const orc_params *p, const double *kb)
+{
+    int nb = p->d < 16 ? p->d : 16;
+    unsigned code = 0;
+    for (int b = 0; b < nb; b++) code = (code << 1) | (kb[b] > 0.0 ? 1u : 0u);
+    return code;
+}
+
+/* stable LSD radix sort of cells by their code, two 8-bit digits */
+static void radix_sort_cells(int *cells, int n, const unsigned *code, int *tmp)
+{
+    for (int shift = 0; shift < 16; shift += 8) {
+        int cnt[257];
+        memset(cnt, 0, sizeof(cnt));
+        for (int t = 0; t < n; t++) cnt[((code[cells[t]] >> shift) & 255u) + 1]++;
+        for (int b = 0; b < 256; b++) cnt[b + 1] += cnt[b];
+        for (int t = 0; t < n; t++) tmp[cnt[(code[cells[t]] >> shift) & 255u]++] = cells[t];
+        memcpy(cells, tmp, sizeof(int) * (size_t)n);
+    }
+}
+
+static void forest_build(const orc_params *p, const double *kbar_bh, const double *amax_bh,
+                         const double *tau_h, orc_forest *F)
+{
+    const int C = orc_num_cells(p), d = p->d;
+    memset(F, 0, sizeof(*F));
+    F->seq = (int *)malloc(sizeof(int) * (size_t)(C > 0 ? C : 1));
+    for (int c = 0; c < C; c++)
+        if (!tau_h || amax_bh[c] >= *tau_h) F->seq[F->n++] = c;
+    while (F->L < 31 && (1 << F->L) <= F->n) F->L++;
+    unsigned *code = (unsigned *)malloc(sizeof(unsigned) * (size_t)(C > 0 ? C : 1));
+    for (int c = 0; c < C; c++) code[c] = cell_code(p, kbar_bh + (size_t)c * d);
+    int *tmp = (int *)malloc(sizeof(int) * (size_t)(F->n > 0 ? F->n : 1));
+    F->ord = (int **)calloc((size_t)(F->L + 1), sizeof(int *));
+    F->mu = (double **)calloc((size_t)(F->L + 1), sizeof(double *));
+    F->rho = (double **)calloc((size_t)(F->L + 1), sizeof(double *));
+    F->A = (double **)calloc((size_t)(F->L + 1), sizeof(double *));
+    F->pmin = (int **)calloc((size_t)(F->L + 1), sizeof(int *));
+    for (int k = 0; k < F->L; k++) {
+        const int nblk = F->n >> k, nleaf = 1 << k, nnode = 2 << k;
+        F->ord[k] = (int *)malloc(sizeof(int) * (size_t)nblk * nleaf);
+        F->mu[k] = (double *)calloc((size_t)nblk * nnode * d, sizeof(double));
+        F->rho[k] = (double *)calloc((size_t)nblk * nnode, sizeof(double));
+        F->A[k] = (double *)calloc((size_t)nblk * nnode, sizeof(double));
+        F->pmin[k] = (int *)calloc((size_t)nblk * nnode, sizeof(int));
+        for (int blk = 0; blk < nblk; blk++) {
+            int *o = F->ord[k] + (size_t)blk * nleaf;
+            memcpy(o, F->seq + (size_t)blk * nleaf, sizeof(int) * (size_t)nleaf);
+            radix_sort_cells(o, nleaf, code, tmp);
+            if (p->mutation == MUT_TREE_SORT_DESC)
+                for (int a = 0, b = nleaf - 1; a < b; a++, b--) { int x = o[a]; o[a] = o[b]; o[b] = x; }
+            for (int v = 1; v < nnode; v++) {
+                int t = 0;
+                while ((2 << t) <= v) t++;                  /* depth of v */
+                const int first = (v - (1 << t)) << (k - t), cnt = 1 << (k - t);
+                const size_t nv = (size_t)blk * nnode + v;
+                double *mu = F->mu[k] + nv * d;
+                double Av = -INFINITY;
+                int pm = o[first];
+                for (int j = first; j < first + cnt; j++) {
+                    const double *kb = kbar_bh + (size_t)o[j] * d;
+                    for (int m = 0; m < d; m++) mu[m] += kb[m];
+                    if (amax_bh[o[j]] > Av) Av = amax_bh[o[j]];
+                    if (p->mutation == MUT_TREE_PMAX ? o[j] > pm : o[j] < pm) pm = o[j];
+                }
+                for (int m = 0; m < d; m++) mu[m] /= cnt;
+                double rho = 0.0;
+                for (int j = first; j < first + cnt; j++) {
+                    const double *kb = kbar_bh + (size_t)o[j] * d;
+                    double sq = 0.0;
+                    for (int m = 0; m < d; m++) sq += (kb[m] - mu[m]) * (kb[m] - mu[m]);
+                    if (sqrt(sq) > rho) rho = sqrt(sq);
+                }
+                F->rho[k][nv] = rho;
+                F->A[k][nv] = Av;
+                F->pmin[k][nv] = pm;
+            }
+        }
+    }
+    free(code);
+    free(tmp);
+}
+
+static void forest_free(orc_forest *F)
+{
+    for (int k = 0; k < F->L; k++) {
+        free(F->ord[k]); free(F->mu[k]); free(F->rho[k]); free(F->A[k]); free(F->pmin[k]);
+    }
+    free(F->ord); free(F->mu); free(F->rho); free(F->A); free(F->pmin); free(F->seq);
+    memset(F, 0, sizeof(*F));
+}
+
+/* eq. (11) for node (k, blk, v) and the query q at position i of head h */
+static double node_U(const orc_params *p, const orc_forest *F, int k, int blk, int v,
+                     const float *qrow, long long i, int h, double c_explore)
+{
+    const int d = p->d;
+    const size_t nv = (size_t)blk * (2 << k) + v;
+    const double *mu = F->mu[k] + nv * d;
+    double dot = 0.0, qq = 0.0;
+    for (int m = 0; m < d; m++) {
+        dot += (double)qrow[m] * mu[m];
+        qq += (double)qrow[m] * qrow[m];
+    }
+    const double rho_term = p->mutation == MUT_TREE_NO_RHO ? 0.0 : c_explore * sqrt(qq) * F->rho[k][nv];
+    double U = (dot + rho_term) * logit_scale(p);
+    const double lam = p->lambda ? p->lambda[h] : 0.0;
+    if (lam != 0.0) {
+        const double pv = (double)p->pos0 + (F->pmin[k][nv] + 0.5) * p->s;
+        U += lam * F->A[k][nv] * erf(((double)(p->pos0 + i) - pv) / (2.0 * p->sigma[h]));
+    }
+    return U;
+}
+
+/* eq. (7) for one cell */
+static double eq7_score(const orc_params *p, const float *qrow, long long i, int h,
+                        const double *kbar_bh, const double *amax_bh, int c)
+{
+    const double *kb = kbar_bh + (size_t)c * p->d;
+    double dot = 0.0;
+    for (int m = 0; m < p->d; m++) dot += (double)qrow[m] * kb[m];
+    double r = dot * logit_scale(p);
+    const double lam = p->lambda ? p->lambda[h] : 0.0;
+    if (lam != 0.0) {
+        const double pc = (double)p->pos0 + (c + 0.5) * p->s;
+        r += lam * amax_bh[c] * erf(((double)(p->pos0 + i) - pc) / (2.0 * p->sigma[h]));
+    }
+    return r;
+}
+
+typedef struct { double U; int k, blk, v, pmin; } beam_node;
+
+static int beam_before(const beam_node *a, const beam_node *b)
+{
+    if (a->U != b->U) return a->U > b->U;
+    return a->pmin < b->pmin;
+}
+
+/* keep the beta best of x[0..n) (sorted, best first); returns the new count and lowers
+ * *margin to the cut's relative gap when something is cut */
+static int beam_cut(beam_node *x, int n, int beta, double *margin)
+{
+    for (int a = 1; a < n; a++) {                      /* insertion sort, best first */
+        beam_node t = x[a];
+        int b = a - 1;
+        while (b >= 0 && beam_before(&t, &x[b])) { x[b + 1] = x[b]; b--; }
+        x[b + 1] = t;
+    }
+    if (n <= beta) return n;
+    const double gap = (x[beta - 1].U - x[beta].U) / fmax(1.0, fabs(x[beta - 1].U));
+    if (gap < *margin) *margin = gap;
+    return beta;
+}
+
+/* beam search on one forest for the prefix of m sequence entries: the leaf cells it ends on */
+static int forest_search(const orc_params *p, const orc_forest *F, int m, const float *qrow,
+                         long long i, int h, int beta, double c_explore, int *cells, double *margin)
+{
+    beam_node *cur = (beam_node *)malloc(sizeof(beam_node) * (size_t)(2 * beta + 64));
+    int n = 0;
+    for (int k = F->L - 1; k >= 0; k--) {              /* roots: the set bits of m */
+        if (!((m >> k) & 1)) continue;
+        beam_node r;
+        r.k = k; r.blk = (m >> k) - 1; r.v = 1;
+        r.U = node_U(p, F, k, r.blk, 1, qrow, i, h, c_explore);
+        r.pmin = F->pmin[k][(size_t)r.blk * (2 << k) + 1];
+        cur[n++] = r;
+    }
+    n = beam_cut(cur, n, beta, margin);
+    for (;;) {
+        beam_node *next = (beam_node *)malloc(sizeof(beam_node) * (size_t)(2 * beta + 64));
+        int nn = 0, expanded = 0;
+        for (int t = 0; t < n; t++) {
+            const beam_node e = cur[t];
+            if (e.v >= (1 << e.k)) { next[nn++] = e; continue; }      /* a leaf */
+            expanded = 1;
+            for (int ch = 0; ch < 2; ch++) {
+                beam_node c = e;
+                c.v = 2 * e.v + ch;
+                c.U = node_U(p, F, e.k, e.blk, c.v, qrow, i, h, c_explore);
+                c.pmin = F->pmin[e.k][(size_t)e.blk * (2 << e.k) + c.v];
+                next[nn++] = c;
+            }
+        }
+        free(cur);
+        cur = next;
+        n = nn;
+        if (!expanded) break;
+        n = beam_cut(cur, n, beta, margin);
+    }
+    for (int t = 0; t < n; t++) {
+        const beam_node e = cur[t];
+        cells[t] = F->ord[e.k][((size_t)e.blk << e.k) + (e.v - (1 << e.k))];
+    }
+    free(cur);
+    return n;
+}
+
+/* FS-B selection for a list of rows (flat (b*H + h)*Nq + r; NULL = all rows in order).
+ * tau: [H] thresholds of forest tau, or NULL for forest 0 alone.  idx_out [nrows, K];
+ * margin_out (or NULL): per row, the smallest relative gap at any beam cut (1 if none).
+ * Returns 0, or -1 for bad arguments. */
+int orc_tree_select_rows(const orc_params *p, const float *Q, const double *kbar, const double *amax,
+                         const double *tau, int beta, double c_explore, long long nrows,
+                         const long long *rows, int *idx_out, double *margin_out)
+{
+    const int C = orc_num_cells(p), BH = p->B * p->H, Kc = p->K;
+    if (beta < 1 || (p->lambda && !p->sigma)) return -1;
+    if (!rows) nrows = (long long)BH * p->Nq;
+    for (int bh = 0; bh < BH; bh++) {
+        int any = 0;
+        for (long long t = 0; t < nrows && !any; t++) any = (rows ? rows[t] : t) / p->Nq == bh;
+        if (!any) continue;
+        const int h = bh % p->H;
+        const double *kb = kbar + (size_t)bh * C * p->d, *am = amax + (size_t)bh * C;
+        orc_forest F0, Ft;
+        forest_build(p, kb, am, NULL, &F0);
+        if (tau) forest_build(p, kb, am, tau + h, &Ft);
+        #pragma omp parallel for schedule(dynamic, 16)
+        for (long long t = 0; t < nrows; t++) {
+            const long long f = rows ? rows[t] : t;
+            if (f / p->Nq != bh) continue;
+            const int r = (int)(f % p->Nq);
+            const long long i = (long long)(p->Nk - p->Nq) + r;
+            const float *q = Q + (size_t)f * p->d;
+            const int n = orc_candidate_count(p, i);
+            double margin = 1.0;
+            int *cells = (int *)malloc(sizeof(int) * (size_t)(4 * beta + 128));
+            int nc = forest_search(p, &F0, n, q, i, h, beta, c_explore, cells, &margin);
+            if (tau) {
+                int m = 0;
+                while (m < Ft.n && Ft.seq[m] < n) m++;          /* admitted cells of C_i */
+                nc += forest_search(p, &Ft, m, q, i, h, beta, c_explore, cells + nc, &margin);
+            }
+            vi_pair *x = (vi_pair *)malloc(sizeof(vi_pair) * (size_t)(nc > 0 ? nc : 1));
+            vi_pair *tmp = (vi_pair *)malloc(sizeof(vi_pair) * (size_t)(nc > 0 ? nc : 1));
+            int nx = 0;
+            for (int a = 0; a < nc; a++) {                      /* the union (a cell once) */
+                int dup = 0;
+                for (int b = 0; b < a && !dup; b++) dup = cells[b] == cells[a];
+                if (dup) continue;
+                x[nx].v = eq7_score(p, q, i, h, kb, am, cells[a]);
+                x[nx].idx = cells[a];
+                nx++;
+            }
+            sort_desc(x, nx, tmp, 0);
+            int *out = idx_out + (size_t)t * Kc;
+            const int keep = nx < Kc ? nx : Kc;
+            for (int a = 0; a < keep; a++) out[a] = x[a].idx;
+            qsort(out, (size_t)keep, sizeof(int), cmp_int);
+            for (int a = keep; a < Kc; a++) out[a] = -1;
+            if (margin_out) margin_out[t] = margin;
+            free(cells); free(x); free(tmp);
+        }
+        forest_free(&F0);
+        if (tau) forest_free(&Ft);
+    }
+    return 0;
+}
+
+/* One node of one (b,h) forest (0: all cells; 1: cells with a_c >= tau[h]): its leaves in
+ * code order into `leaves` (capacity >= 2^k) and eq. (11) for query row r into *U.
+ * *nseq receives the forest's sequence length.  Returns the leaf count, or -1 if the node
+ * does not exist. */
+int orc_tree_node(const orc_params *p, const float *Q, const double *kbar, const double *amax,
+                  const double *tau, int b, int h, int forest, int k, int blk, int v, int r,
+                  double c_explore, int *leaves, double *U, int *nseq)
+{
+    const int C = orc_num_cells(p);
+    const size_t bh = (size_t)b * p->H + h;
+    orc_forest F;
+    forest_build(p, kbar + bh * C * p->d, amax + bh * C, forest ? tau + h : NULL, &F);
+    *nseq = F.n;
+    int cnt = -1;
+    if (k >= 0 && k < F.L && blk >= 0 && blk < (F.n >> k) && v >= 1 && v < (2 << k)) {
+        int t = 0;
+        while ((2 << t) <= v) t++;
+        const int first = (v - (1 << t)) << (k - t);
+        cnt = 1 << (k - t);
+        for (int j = 0; j < cnt; j++) leaves[j] = F.ord[k][((size_t)blk << k) + first + j];
+        const long long i = (long long)(p->Nk - p->Nq) + r;
+        *U = node_U(p, &F, k, blk, v, Q + (bh * p->Nq + r) * p->d, i, h, c_explore);
+    }
+    forest_free(&F);
+    return cnt;
 }

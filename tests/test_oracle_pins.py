@@ -420,6 +420,117 @@ def test_backward_matches_finite_differences():
     assert _fd_failures(n_entries=20) == []
 
 
+# ---------------------------------------------------------------- FS-B (eqs. (10)-(11))
+def _codes(kbar_bh):
+    """16-bit code of each cell: the signs of its mean key's first 16 coordinates,
+    coordinate 0 the most significant bit."""
+    nb = min(16, kbar_bh.shape[1])
+    bits = (kbar_bh[:, :nb] > 0).astype(np.int64)
+    return (bits * (1 << np.arange(nb - 1, -1, -1))).sum(axis=1)
+
+
+def _eq7(q, kbar_bh, amax_bh, i, c, s, lam, sigma):
+    r = float(q.astype(np.float64) @ kbar_bh[c]) / math.sqrt(q.shape[0])
+    if lam:
+        r += lam * amax_bh[c] * math.erf((i - (c + 0.5) * s) / (2.0 * sigma))
+    return r
+
+
+def _tree_pin_failures(mutation=0):
+    """Pins of the FS-B oracle; returns the names of those that fail."""
+    fails = set()
+    inp = tiny(d=16, Nq=160, Nk=400, w=32, s=8, K=4, W=-1, P=-1, lam=0.7, sigma=40.0, seed=61)
+    wl = inp.wl
+    prob = make_problem(inp, mutation=mutation)
+    kb, am = prob.summaries()
+    tau = np.array([np.median(am[0, 0]), np.quantile(am[0, 1], 0.7)])
+    # (a) an exhaustive beam keeps every leaf: S_i is eq. (7)'s top-K over C_i (brute force)
+    _, sel, _, _, _ = brute_forward(inp.Q, inp.K, inp.V, w=wl.w, s=wl.s, K_cells=wl.K, W=-1, P=-1,
+                                    alpha=inp.alpha, lam=inp.lam, sigma=inp.sigma,
+                                    rope_base=wl.rope_base, rms_eps=wl.rms_eps)
+    want = sel_to_idx(sel, wl.K).reshape(-1, wl.K)
+    for t in (None, tau):
+        idx, _ = prob.tree_select(kb, am, beam=64, tau=t)
+        if not np.array_equal(idx, want):
+            fails.add("exhaustive")
+    lam, sig = inp.lam[0], inp.sigma[0]
+    for h in range(wl.H):
+        kbh, amh = kb[0, h], am[0, h]
+        code = _codes(kbh)
+        for forest in (0, 1):
+            seq = np.arange(kbh.shape[0]) if forest == 0 else np.nonzero(amh >= tau[h])[0]
+            n = len(seq)
+            _, _, nseq = prob.tree_node(kb, am, 0, h, forest, 0, 0, 1, 0, tau=tau)
+            if nseq != n:
+                fails.add("sequence")
+            k = 0
+            while (1 << k) <= n:
+                for blk in range(n >> k):
+                    cells = seq[blk << k:(blk + 1) << k]
+                    order = cells[np.lexsort((np.arange(len(cells)), code[cells]))]
+                    leaves, _, _ = prob.tree_node(kb, am, 0, h, forest, k, blk, 1, 0, tau=tau)
+                    if leaves is None or leaves.tolist() != order.tolist():   # (b) radix order
+                        fails.add("leaf_order")
+                k += 1
+            # (c) node statistics and eq. (11): closed forms per node, for a few rows
+            for r in (wl.Nq - 1, wl.Nq // 2):
+                i = wl.Nk - wl.Nq + r
+                ncand = prob.candidate_count(i)
+                q = inp.Q[0, h, r].astype(np.float64)
+                for k in range(0, 5):
+                    for blk in range(n >> k):
+                        for v in range(1, 2 << k):
+                            leaves, U1, _ = prob.tree_node(kb, am, 0, h, forest, k, blk, v, r, 1.0, tau)
+                            _, U0, _ = prob.tree_node(kb, am, 0, h, forest, k, blk, v, r, 0.0, tau)
+                            mu = kbh[leaves].mean(axis=0)
+                            rho = np.sqrt(((kbh[leaves] - mu) ** 2).sum(axis=1)).max()
+                            prior = lam * amh[leaves].max() * math.erf(
+                                (i - (leaves.min() + 0.5) * wl.s) / (2.0 * sig))
+                            if abs(U0 - (q @ mu / math.sqrt(wl.d) + prior)) > 1e-12:
+                                fails.add("mu_prior")
+                            if abs((U1 - U0) - np.linalg.norm(q) * rho / math.sqrt(wl.d)) > 1e-12:
+                                fails.add("rho")
+                            best = max(_eq7(q, kbh, amh, i, c, wl.s, lam, sig) for c in leaves)
+                            # (d) U_v bounds its leaves (nodes of the row's prefix: there
+                            #     the erf argument is positive)
+                            if leaves.max() < ncand and U1 < best - 1e-12:
+                                fails.add("bound")
+                            if len(leaves) == 1 and abs(U1 - best) > 1e-12:
+                                fails.add("leaf_is_eq7")
+    # (e) a beam of width 1 descends greedily: one cell per forest, and on the path from
+    #     its root every node beats its sibling
+    idx, _ = prob.tree_select(kb, am, beam=1)
+    for h in range(wl.H):
+        for r in (wl.Nq - 1, 60, 100):
+            row = (0 * wl.H + h) * wl.Nq + r
+            got = [c for c in idx[row] if c >= 0]
+            n = prob.candidate_count(wl.Nk - wl.Nq + r)
+            if n == 0:
+                continue
+            if len(got) != 1:
+                fails.add("greedy")
+                continue
+            c = got[0]
+            k = max(kk for kk in range(12) if (n >> kk) & 1 and ((n >> kk) - 1) << kk <= c)
+            blk = (n >> k) - 1
+            roots = [(kk, (n >> kk) - 1) for kk in range(12) if (n >> kk) & 1]
+            Uroot = {rt: prob.tree_node(kb, am, 0, h, 0, rt[0], rt[1], 1, r)[1] for rt in roots}
+            if max(Uroot.values()) != Uroot[(k, blk)]:
+                fails.add("greedy")
+            v = 1
+            while v < (1 << k):
+                kids = [prob.tree_node(kb, am, 0, h, 0, k, blk, 2 * v + e, r) for e in (0, 1)]
+                e = 0 if c in kids[0][0] else 1
+                if kids[e][1] < kids[1 - e][1]:
+                    fails.add("greedy")
+                v = 2 * v + e
+    return sorted(fails)
+
+
+def test_tree_pins():
+    assert _tree_pin_failures() == []
+
+
 # ---------------------------------------------------------------- sensitivity
 def _pins_fail(mutation):
     """Run a compact set of the pins above against a mutated oracle; True if any fails."""
@@ -443,6 +554,7 @@ def _pins_fail(mutation):
         failures.append("golden_prune")
     failures += _rerank_pin_failures(mutation)
     failures += _fd_failures(mutation, n_entries=6)
+    failures += _tree_pin_failures(mutation)
     return failures
 
 
