@@ -425,6 +425,49 @@ def time_rerank(fs, torch, inp, steps=5, warmup=3):
                     "timing on (events around each launch)"}
 
 
+def time_tree(fs, torch, inp, beam=32, steps=5, warmup=3):
+    """The FS-B variant of the forward pass (eqs. (10)-(11)): fs_forward_tree (summaries,
+    both forests built, beam search, then the per-row readout and the window), with
+    tau_h at each head's 75th percentile of a_c.  Returns query-tokens/s and the split."""
+    wl = inp.wl
+    p = make_params(fs, inp)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    Q, K, V = (torch.from_numpy(x).cuda().to(dt) for x in (inp.Q, inp.K, inp.V))
+    O = torch.empty_like(Q)
+    ws = fs.alloc_workspace(p)
+    C = wl.Nk // wl.s
+    kbar = torch.empty((wl.B, wl.H, C, wl.d), dtype=torch.float32, device="cuda")
+    amax = torch.empty((wl.B, wl.H, C), dtype=torch.float32, device="cuda")
+    fs.cell_summaries(p, K, kbar, amax)
+    tau = torch.quantile(amax.transpose(0, 1).reshape(wl.H, -1), 0.75, dim=1).cpu().tolist()
+    forest = fs.alloc_forest(p)
+    idx = torch.empty((wl.B, wl.H, wl.Nq, wl.K), dtype=torch.int32, device="cuda")
+
+    def step():
+        fs.forward_tree(p, Q, K, V, O, ws, forest, beam, 1.0, tau, idx=idx)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    fs.timing_enable(True)
+    fs.kernel_times()
+    step()
+    torch.cuda.synchronize()
+    kt = {k: round(v[1], 3) for k, v in fs.kernel_times().items() if v[0]}
+    fs.timing_enable(False)
+    fs.sync_status(ws)
+    return {"value": wl.queries / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "kernel_ms": kt,
+            "note": "fs_forward_tree: FS-B beam search (width %d, c = 1) over both forests "
+                    "(tau_h = 75th percentile of a_c), forests rebuilt every step, then the "
+                    "per-row readout and the tensor-core window + combine" % beam}
+
+
 def time_backward(fs, torch, inp, steps=3, warmup=3):
     """The backward pass of eq. (2) on a workload (fs_backward on the cells fs_select_topk
     chose; the selection is outside the timed region).  Returns query-tokens/s and the
@@ -605,6 +648,8 @@ def run_ours(args):
             extras[wl.name + "_rerank"] = time_rerank(fs, torch, inp)
             torch.cuda.empty_cache()
             extras[wl.name + "_backward"] = time_backward(fs, torch, inp)
+            torch.cuda.empty_cache()
+            extras[wl.name + "_tree"] = time_tree(fs, torch, inp)
             torch.cuda.empty_cache()
             line["other_workloads"] = extras
     if rank == 0:

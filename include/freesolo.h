@@ -231,6 +231,48 @@ fs_status fs_cache_attend(const fs_params *p, int max_block, void *cache, size_t
  * FS_ERR_CUDA if the stream reports an error, else FS_OK. */
 fs_status fs_cache_status(void *cache, void *stream);
 
+/* ---- FS-B: balanced-tree search ("FreeSolo" summary §3.4, eqs. (10)-(11)) ----
+ * Two causal forests per (batch, head): forest 0 over every cell in time order (admitted
+ * set A^0_i = C_i), forest tau over the cells with a_c >= tau_h in time order (A^tau_i),
+ * eq. (10).  Over a forest's sequence there is one balanced binary tree per aligned block
+ * of 2^k entries, every k; the query at position i searches the trees covering its
+ * candidate prefix (the set bits of its length).  A tree's leaves are its cells sorted by a
+ * 16-bit code, the signs of kbar_c's first 16 coordinates (coordinate 0 most significant),
+ * ties by time; node v stores mu_v = mean kbar_c, rho_v = max ||kbar_c - mu_v||, A_v =
+ * max a_c and p_v^min = min p_c over its leaves and is ranked by eq. (11):
+ *   U_v = (q_i.mu_v + c ||q_i|| rho_v) / sqrt(d) + lambda_h A_v erf((i - p_v^min) / (2 sigma_h)).
+ * Beam search of width `beam` on each forest (from the prefix's roots; every internal node
+ * of the beam replaced by its two children, the `beam` best kept by U_v, ties to the lower
+ * p_v^min, until only leaves remain); S_i = the K best cells by eq. (7) among the leaves
+ * both beams end on.  W and P are not used (FS-B does not prune).  With c >= 1 and
+ * lambda_h >= 0, U_v bounds eq. (7) over the leaves below v; a beam that holds every leaf
+ * gives base FS's selection. */
+#define FS_TREE_MAX_BEAM 64
+
+/* Bytes of the forest buffer for p (B, H, Nk, s): O(B H (Nk/s) log2(Nk/s) d) floats. */
+fs_status fs_forest_bytes(const fs_params *p, size_t *bytes);
+
+/* Builds both forests from the cell summaries (fs_cell_summaries' kbar [B,H,C,d], amax
+ * [B,H,C], device f32) into the caller's device buffer `forest`.  tau: HOST [H]
+ * thresholds of eq. (10), or NULL for forest 0 alone. */
+fs_status fs_forest_build(const fs_params *p, const float *kbar, const float *amax, const float *tau,
+                          void *forest, size_t forest_bytes, void *stream);
+
+/* FS-B selection: idx [B,H,Nq,K] (ascending, -1 padded) for the device queries Q, from a
+ * forest built with the same p.  1 <= beam <= FS_TREE_MAX_BEAM; c_explore is eq. (11)'s
+ * c.  ws (fs_workspace_size bytes) carries the device error flag: a forest not built for
+ * these sizes is reported by fs_sync_status as FS_ERR_KERNEL_CHECK. */
+fs_status fs_select_topk_tree(const fs_params *p, const void *Q, const void *forest, size_t forest_bytes,
+                              int beam, float c_explore, int32_t *idx, void *ws, size_t ws_bytes,
+                              void *stream);
+
+/* The forward pass with the FS-B selection: summaries, forest build, search, then the
+ * per-row readout (eq. (9)) on the selected cells and the window + combine (eqs. (2)-(4)).
+ * idx, if not NULL, receives the selection. */
+fs_status fs_forward_tree(const fs_params *p, const void *Q, const void *K, const void *V, const float *tau,
+                          int beam, float c_explore, int32_t *idx, void *O, void *ws, size_t ws_bytes,
+                          void *forest, size_t forest_bytes, void *stream);
+
 /* ---- diagnostics (no counterpart in the method: measurement support) ----
  * fs_launch_count: kernels this library has launched since load (all calls, streams).
  * fs_timing_enable(1): from now on every kernel launch is bracketed by two CUDA events

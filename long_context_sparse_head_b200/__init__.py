@@ -27,7 +27,8 @@ EXPORTS = ("fs_workspace_size", "fs_cell_summaries", "fs_select_topk", "fs_forwa
            "fs_launch_count", "fs_timing_enable", "fs_kernel_times", "fs_kernel_name",
            "fs_select_topk_noalloc", "fs_cache_bytes", "fs_cache_reset", "fs_cache_append",
            "fs_cache_attend", "fs_cache_status", "fs_select_topk_rerank", "fs_forward_rerank",
-           "fs_backward_workspace_size", "fs_backward")
+           "fs_backward_workspace_size", "fs_backward", "fs_forest_bytes", "fs_forest_build",
+           "fs_select_topk_tree", "fs_forward_tree")
 
 
 class FsError(RuntimeError):
@@ -87,6 +88,14 @@ def load():
         L.fs_cache_status.argtypes = [vp, vp]
         L.fs_kernel_name.argtypes = [ctypes.c_int]
         L.fs_kernel_name.restype = ctypes.c_char_p
+        L.fs_backward_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
+        L.fs_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        fp = ctypes.POINTER(ctypes.c_float)
+        L.fs_forest_bytes.argtypes = [P, ctypes.POINTER(sz)]
+        L.fs_forest_build.argtypes = [P, vp, vp, fp, vp, sz, vp]
+        L.fs_select_topk_tree.argtypes = [P, vp, vp, sz, ctypes.c_int, ctypes.c_float, vp, vp, sz, vp]
+        L.fs_forward_tree.argtypes = [P, vp, vp, vp, fp, ctypes.c_int, ctypes.c_float, vp, vp, vp, sz, vp,
+                                      sz, vp]
         for name in EXPORTS:
             if name not in ("fs_status_string", "fs_launch_count", "fs_kernel_name"):
                 getattr(L, name).restype = ctypes.c_int
@@ -209,6 +218,47 @@ def forward_host(params, hQ, hK, hV, hO, dscratch, stream=None):
     _check(load().fs_forward_host(params.ref(), _ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hO),
                                   _ptr(dscratch), dscratch.numel() * dscratch.element_size(),
                                   _stream(stream)), "fs_forward_host")
+
+
+# ---- FS-B: balanced-tree search (eqs. (10)-(11)) --------------------------------------
+def forest_bytes(params):
+    n = ctypes.c_size_t()
+    _check(load().fs_forest_bytes(params.ref(), ctypes.byref(n)), "fs_forest_bytes")
+    return n.value
+
+
+def alloc_forest(params, device="cuda"):
+    import torch
+    return torch.empty(forest_bytes(params), dtype=torch.uint8, device=device)
+
+
+def _tau(params, tau):
+    if tau is None:
+        return None
+    arr = (ctypes.c_float * params.H)(*[float(x) for x in tau])
+    return ctypes.cast(arr, ctypes.POINTER(ctypes.c_float)), arr
+
+
+def forest_build(params, kbar, amax, forest, tau=None, stream=None):
+    """Both FS-B forests from the cell summaries; tau: per-head thresholds (None: forest 0 only)."""
+    t = _tau(params, tau)
+    _check(load().fs_forest_build(params.ref(), _ptr(kbar), _ptr(amax), t[0] if t else None, _ptr(forest),
+                                  forest.numel() * forest.element_size(), _stream(stream)), "fs_forest_build")
+
+
+def select_topk_tree(params, Q, forest, idx, ws, beam, c_explore=1.0, stream=None):
+    _check(load().fs_select_topk_tree(params.ref(), _ptr(Q), _ptr(forest), forest.numel() * forest.element_size(),
+                                      int(beam), ctypes.c_float(c_explore), _ptr(idx), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)), "fs_select_topk_tree")
+
+
+def forward_tree(params, Q, K, V, O, ws, forest, beam, c_explore=1.0, tau=None, idx=None, stream=None):
+    """The forward pass with the FS-B selection (idx: optional output of the selection)."""
+    t = _tau(params, tau)
+    _check(load().fs_forward_tree(params.ref(), _ptr(Q), _ptr(K), _ptr(V), t[0] if t else None, int(beam),
+                                  ctypes.c_float(c_explore), _ptr(idx), _ptr(O), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _ptr(forest),
+                                  forest.numel() * forest.element_size(), _stream(stream)), "fs_forward_tree")
 
 
 def backward_workspace_size(params):

@@ -259,6 +259,76 @@ extern "C" fs_status fs_forward_rerank(const fs_params *p, const void *Q, const 
     return run_forward(p, Q, K, V, kbar, amax, sel, O, ws, st);
 }
 
+extern "C" fs_status fs_forest_bytes(const fs_params *p, size_t *bytes) {
+    fs_status s = validate(p);
+    if (s != FS_OK) return s;
+    if (!bytes) return FS_ERR_INVALID_ARG;
+    *bytes = forest_bytes(p);
+    return FS_OK;
+}
+
+extern "C" fs_status fs_forest_build(const fs_params *p, const float *kbar, const float *amax, const float *tau,
+                                     void *forest, size_t forest_bytes_, void *stream) {
+    fs_status s = validate(p);
+    if (s != FS_OK) return s;
+    if (!forest || forest_bytes_ < forest_bytes(p)) return FS_ERR_WORKSPACE;
+    if (p->Nk / p->s > 0 && (!kbar || !amax)) return FS_ERR_INVALID_ARG;
+    if (tau)
+        for (int h = 0; h < p->H; h++)
+            if (std::isnan(tau[h])) return FS_ERR_INVALID_ARG;
+    return cuda_status(launch_tree_build(p, kbar, amax, tau, forest, (cudaStream_t)stream));
+}
+
+extern "C" fs_status fs_select_topk_tree(const fs_params *p, const void *Q, const void *forest,
+                                         size_t forest_bytes_, int beam, float c_explore, int32_t *idx,
+                                         void *ws, size_t ws_bytes, void *stream) {
+    fs_status s = validate(p);
+    if (s != FS_OK) return s;
+    if (beam < 1 || beam > FS_TREE_MAX_BEAM || !(c_explore >= 0.f) || std::isinf(c_explore)) return FS_ERR_INVALID_ARG;
+    if (p->Nq == 0 || p->K == 0) return FS_OK;
+    if (!Q || !idx) return FS_ERR_INVALID_ARG;
+    if (!forest || forest_bytes_ < forest_bytes(p)) return FS_ERR_WORKSPACE;
+    if (!ws || ws_bytes < layout(p).total) return FS_ERR_WORKSPACE;
+    const Dev D = make_dev(p);
+    return cuda_status(launch_tree_search(p, D, Q, forest, beam, c_explore, idx, at<int>(ws, layout(p).flag),
+                                          (cudaStream_t)stream));
+}
+
+extern "C" fs_status fs_forward_tree(const fs_params *p, const void *Q, const void *K, const void *V,
+                                     const float *tau, int beam, float c_explore, int32_t *idx, void *O,
+                                     void *ws, size_t ws_bytes, void *forest, size_t forest_bytes_,
+                                     void *stream) {
+    fs_status s = validate(p);
+    if (s != FS_OK) return s;
+    if (beam < 1 || beam > FS_TREE_MAX_BEAM || !(c_explore >= 0.f) || std::isinf(c_explore)) return FS_ERR_INVALID_ARG;
+    if (p->Nq == 0) return FS_OK;
+    if (!Q || !K || !V || !O) return FS_ERR_INVALID_ARG;
+    const WsLayout L = layout(p);
+    if (!ws || ws_bytes < L.total) return FS_ERR_WORKSPACE;
+    if (!forest || forest_bytes_ < forest_bytes(p)) return FS_ERR_WORKSPACE;
+    if (tau)
+        for (int h = 0; h < p->H; h++)
+            if (std::isnan(tau[h])) return FS_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (!has_long_range(p)) {                      // window only; no cells to select
+        if (idx && p->K > 0 &&
+            cudaMemsetAsync(idx, 0xff, (size_t)p->B * p->H * p->Nq * p->K * 4, st) != cudaSuccess)
+            return FS_ERR_CUDA;
+        return run_forward(p, Q, K, V, nullptr, nullptr, nullptr, O, ws, st);
+    }
+    const Dev D = make_dev(p);
+    float *kb = at<float>(ws, L.kbar), *am = at<float>(ws, L.amax);
+    if (launch_summaries(D, p->dtype, K, kb, am, st) != cudaSuccess) return FS_ERR_CUDA;
+    if (launch_tree_build(p, kb, am, tau, forest, st) != cudaSuccess) return FS_ERR_CUDA;
+    int32_t *sel = idx ? idx : at<int32_t>(ws, L.idx);
+    if (launch_tree_search(p, D, Q, forest, beam, c_explore, sel, at<int>(ws, L.flag), st) != cudaSuccess)
+        return FS_ERR_CUDA;
+    // FS-B rows of one query tile pick cells across the whole prefix (their union is not
+    // bounded like FS-L's), so the readout gathers per row: the readout kernel on the
+    // selection, then the tensor-core window + combine
+    return run_forward(p, Q, K, V, kb, am, sel, O, ws, st);
+}
+
 extern "C" fs_status fs_forward(const fs_params *p, const void *Q, const void *K, const void *V,
                                 const float *kbar, const float *amax, const int32_t *idx, void *O,
                                 void *ws, size_t ws_bytes, void *stream) {

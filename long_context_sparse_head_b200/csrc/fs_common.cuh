@@ -103,7 +103,8 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 enum KernelId : int {
     kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
     kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kRerank, kIdxTiles, kBwdRotate, kBwdRows,
-    kBwdWindowKv, kBwdCells, kBwdReadoutKv, kBwdDalpha, kNumKernels
+    kBwdWindowKv, kBwdCells, kBwdReadoutKv, kBwdDalpha, kTreePrep, kTreeMerge, kTreeNodes, kTreeSearch,
+    kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
@@ -156,6 +157,12 @@ cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, con
 cudaError_t launch_selection(const fs_params *p, const Dev &D, const void *Q, const float *kbar,
                              const float *amax, const int *exitn, int32_t *idx, int *dev_flag,
                              cudaStream_t st);
+// FS-B (eqs. (10)-(11)): forest buffer size, build (tau: host [H] or NULL), search
+size_t forest_bytes(const fs_params *p);
+cudaError_t launch_tree_build(const fs_params *p, const float *kbar, const float *amax, const float *tau,
+                              void *forest, cudaStream_t st);
+cudaError_t launch_tree_search(const fs_params *p, const Dev &D, const void *Q, const void *forest, int beam,
+                               float c_explore, int32_t *idx, int *dev_flag, cudaStream_t st);
 // fused tensor-core readout + window + combine (bf16, internally selected cells)
 bool attn_tc_supported(const fs_params *p);
 cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V, const void *Krot,

@@ -1,0 +1,499 @@
+// FS-B selection ("FreeSolo" summary §3.4, eqs. (10)-(11)): beam search over two causal
+// forests of balanced trees.
+//   forest 0 holds every cell in time order (admitted set A^0_i = C_i, eq. (10));
+//   forest 1 the cells with a_c >= tau_h in time order (A^tau_i, eq. (10)).
+// Over a forest's sequence there is one balanced binary tree per aligned block of 2^k
+// entries, every k; a query whose prefix holds m entries searches the trees of the set
+// bits of m (those a binary counter holds after m insertions: the growing archive).
+// A tree's leaves are its block's cells sorted by a 16-bit code (the signs of the first
+// 16 coordinates of kbar_c, coordinate 0 the most significant bit; ties by time): level
+// k's order is the stable merge of level k-1's two halves, i.e. the radix order.  Node v
+// of the complete binary tree over that order stores
+//   mu_v = mean kbar_c, rho_v = max ||kbar_c - mu_v||, A_v = max a_c, p_v^min = min p_c
+// over its leaves, and eq. (11) scores it for query i:
+//   U_v = (q_i.mu_v + c ||q_i|| rho_v) / sqrt(d) + lambda_h A_v erf((i - p_v^min) / (2 sigma_h)).
+// Beam search of width beta per forest: start from the prefix's roots (keep the beta best),
+// then replace every internal node of the beam by its two children and keep the beta best
+// (U descending, ties to the lower p_v^min), until the beam holds only leaves.  S_i = the K
+// best cells by eq. (7) among both beams' leaves (a leaf's U_v is its eq. (7) score),
+// ascending, -1 padded.
+//
+// Kernels: prep (codes, admitted prefix counts, sequences; one CTA per head), merge (one
+// launch per level; each entry's place by binary search in the other half), nodes (one
+// warp per node: mean, radius, max norm, first cell), search (one warp per query row).
+#include <cmath>
+
+#include "fs_common.cuh"
+
+namespace fs {
+
+namespace {
+
+constexpr int kTreeMagic = 0x46534254;
+constexpr int kMaxBeam = FS_TREE_MAX_BEAM;
+constexpr int kCodeBits = 16;
+constexpr int kSearchWarps = 4;
+constexpr int kCandCap = 2 * kMaxBeam + 32;   // children of a full beam, or the roots
+
+struct ForestGeom {
+    int BH, C, L;
+    size_t hdr, nseq, seq, admp, code, ord, mu, meta, total;
+};
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+ForestGeom forest_geom(const fs_params *p) {
+    ForestGeom g;
+    g.BH = p->B * p->H;
+    g.C = p->Nk / p->s;
+    g.L = 0;
+    while (g.L < 31 && (1LL << g.L) <= g.C) g.L++;
+    const size_t BH = g.BH, C = g.C, L = g.L > 0 ? g.L : 1;
+    size_t off = 0;
+    auto seg = [&](size_t bytes) {
+        const size_t o = off;
+        off += al256(bytes);
+        return o;
+    };
+    g.hdr = seg(16 * 4);
+    g.nseq = seg(BH * 2 * 4);
+    g.seq = seg(BH * 2 * C * 4);
+    g.admp = seg(BH * (C + 1) * 4);
+    g.code = seg(BH * C * 4);
+    g.ord = seg(BH * 2 * L * C * 4);
+    g.mu = seg(BH * 2 * L * 2 * C * kD * 4);
+    g.meta = seg(BH * 2 * L * 2 * C * 16);
+    g.total = off;
+    return g;
+}
+
+// Device view of a forest buffer.
+struct Forest {
+    int *hdr, *nseq, *seq, *admp;
+    uint32_t *code;
+    int *ord;
+    float *mu;
+    float4 *meta;       // (rho, A, pmin as int bits, 0)
+    int C, L;
+    __device__ __forceinline__ size_t lvl(int bh, int f, int k) const {
+        return ((size_t)(bh * 2 + f) * L + k);
+    }
+};
+
+Forest forest_view(void *buf, const ForestGeom &g) {
+    uint8_t *b = static_cast<uint8_t *>(buf);
+    Forest F;
+    F.hdr = reinterpret_cast<int *>(b + g.hdr);
+    F.nseq = reinterpret_cast<int *>(b + g.nseq);
+    F.seq = reinterpret_cast<int *>(b + g.seq);
+    F.admp = reinterpret_cast<int *>(b + g.admp);
+    F.code = reinterpret_cast<uint32_t *>(b + g.code);
+    F.ord = reinterpret_cast<int *>(b + g.ord);
+    F.mu = reinterpret_cast<float *>(b + g.mu);
+    F.meta = reinterpret_cast<float4 *>(b + g.meta);
+    F.C = g.C;
+    F.L = g.L;
+    return F;
+}
+
+// codes, sequences and admitted prefix counts of one (b, h); 1024 threads
+struct TauArgs {
+    float tau[FS_MAX_HEADS];
+};
+
+__global__ void __launch_bounds__(1024) tree_prep_kernel(Forest F, const float *__restrict__ kbar,
+                                                         const float *__restrict__ amax, int H, int has_tau,
+                                                         const TauArgs T) {
+    __shared__ int wsum[32];
+    __shared__ int carry;
+    const int bh = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int C = F.C;
+    const float tau = has_tau ? T.tau[bh % H] : 0.f;
+    if (bh == 0 && t == 0) {
+        F.hdr[0] = kTreeMagic;
+        F.hdr[1] = has_tau;
+        F.hdr[2] = C;
+        F.hdr[3] = F.L;
+        F.hdr[4] = gridDim.x;
+    }
+    if (t == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < C; base += 1024) {
+        const int c = base + t;
+        int adm = 0;
+        if (c < C) {
+            const float *kb = kbar + ((size_t)bh * C + c) * kD;
+            uint32_t code = 0;
+#pragma unroll
+            for (int b = 0; b < kCodeBits; b++) code = (code << 1) | (kb[b] > 0.f ? 1u : 0u);
+            F.code[(size_t)bh * C + c] = code;
+            F.seq[((size_t)bh * 2 + 0) * C + c] = c;
+            adm = has_tau && amax[(size_t)bh * C + c] >= tau;
+        }
+        int incl = adm;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        int before = carry;
+        for (int k = 0; k < warp; k++) before += wsum[k];
+        const int excl = before + incl - adm;
+        if (c < C) {
+            F.admp[(size_t)bh * (C + 1) + c] = excl;
+            if (adm) F.seq[((size_t)bh * 2 + 1) * C + excl] = c;
+        }
+        __syncthreads();
+        if (t == 1023) carry = excl + adm;
+        __syncthreads();
+    }
+    if (t == 0) {
+        F.admp[(size_t)bh * (C + 1) + C] = carry;
+        F.nseq[bh * 2 + 0] = C;
+        F.nseq[bh * 2 + 1] = carry;
+    }
+}
+
+__device__ __forceinline__ unsigned long long sort_key(const Forest &F, int bh, int cell) {
+    return ((unsigned long long)F.code[(size_t)bh * F.C + cell] << 32) | (unsigned)cell;
+}
+
+// level k's leaf order: level 0 copies the sequence; level k >= 1 merges the two sorted
+// halves of each block (an entry's place = its index in its half + the number of keys
+// below it in the other half)
+__global__ void tree_merge_kernel(Forest F, int BH, int k) {
+    const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int C = F.C;
+    if (e >= (long long)BH * 2 * C) return;
+    const int pos = (int)(e % C);
+    const int bhf = (int)(e / C), bh = bhf >> 1, f = bhf & 1;
+    const int n = F.nseq[bhf];
+    if (pos >= ((n >> k) << k)) return;
+    int *out = F.ord + F.lvl(bh, f, k) * C;
+    if (k == 0) {
+        out[pos] = F.seq[(size_t)bhf * C + pos];
+        return;
+    }
+    const int *in = F.ord + F.lvl(bh, f, k - 1) * C;
+    const int hlen = 1 << (k - 1);
+    const int blk = pos >> k, half = (pos >> (k - 1)) & 1, a = pos & (hlen - 1);
+    const int cell = in[pos];
+    const unsigned long long key = sort_key(F, bh, cell);
+    const int *other = in + ((size_t)(2 * blk + (half ^ 1)) << (k - 1));
+    int lo = 0, hi = hlen;                      // keys of the other half below `key`
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (sort_key(F, bh, other[mid]) < key) lo = mid + 1;
+        else hi = mid;
+    }
+    out[(blk << k) + a + lo] = cell;
+}
+
+// one warp per node of level k: mean key, radius, max norm, first cell
+__global__ void __launch_bounds__(256) tree_nodes_kernel(Forest F, const float *__restrict__ kbar,
+                                                         const float *__restrict__ amax, int BH, int k) {
+    const int lane = threadIdx.x & 31;
+    const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int C = F.C;
+    const long long per = 2LL * C;               // node slots per (bh, f) at this level
+    if (wid >= (long long)BH * 2 * per) return;
+    const int bhf = (int)(wid / per), bh = bhf >> 1, f = bhf & 1;
+    const int node = (int)(wid % per);
+    const int blk = node >> (k + 1), v = node & ((2 << k) - 1);
+    const int n = F.nseq[bhf];
+    if (v == 0 || blk >= (n >> k)) return;
+    const int t = 31 - __clz(v);                 // depth of v
+    const int cnt = 1 << (k - t);
+    const int *leaves = F.ord + F.lvl(bh, f, k) * C + ((size_t)blk << k) + ((size_t)(v - (1 << t)) << (k - t));
+    const float *kb = kbar + (size_t)bh * C * kD;
+    float s0 = 0.f, s1 = 0.f, A = -INFINITY;
+    int pmin = 0x7fffffff;
+    for (int j = 0; j < cnt; j++) {
+        const int c = leaves[j];
+        const float2 x = *reinterpret_cast<const float2 *>(kb + (size_t)c * kD + 2 * lane);
+        s0 += x.x;
+        s1 += x.y;
+        A = fmaxf(A, amax[(size_t)bh * C + c]);
+        pmin = min(pmin, c);
+    }
+    const float inv = 1.f / (float)cnt;
+    const float m0 = s0 * inv, m1 = s1 * inv;
+    float r2 = 0.f;
+    for (int j = 0; j < cnt; j++) {
+        const float2 x = *reinterpret_cast<const float2 *>(kb + (size_t)leaves[j] * kD + 2 * lane);
+        const float d0 = x.x - m0, d1 = x.y - m1;
+        r2 = fmaxf(r2, warp_sum(d0 * d0 + d1 * d1));
+    }
+    const size_t ni = F.lvl(bh, f, k) * 2 * C + node;
+    *reinterpret_cast<float2 *>(F.mu + ni * kD + 2 * lane) = make_float2(m0, m1);
+    if (lane == 0) F.meta[ni] = make_float4(cnt == 1 ? 0.f : sqrtf(r2), A, __int_as_float(pmin), 0.f);
+}
+
+struct SearchArgs {
+    int Nq, H, w, K, q0, beam;
+    float scale, c_explore;
+    float lambda[FS_MAX_HEADS], inv2sigma[FS_MAX_HEADS];
+};
+
+struct SearchSmem {
+    float q[kD];
+    float U[kCandCap];
+    int ref[kCandCap];      // level << 26 | node slot
+    int pmin[kCandCap];
+    float bU[kMaxBeam];
+    int bref[kMaxBeam], bpmin[kMaxBeam];
+    float rU[2 * kMaxBeam];  // leaves both beams end on
+    int rcell[2 * kMaxBeam];
+};
+
+__device__ __forceinline__ bool beats(float Ua, int pa, float Ub, int pb) {
+    return Ua > Ub || (Ua == Ub && pa < pb);
+}
+
+// eq. (11) for one node (lane-local: the whole dot product in this lane)
+template <bool PRIOR>
+__device__ __forceinline__ float node_U(const Forest &F, size_t lvl_base, int node, const float *q, float qn,
+                                        const SearchArgs &A, int h, int i, int *pmin_out) {
+    const size_t ni = lvl_base + node;
+    const float4 *mu = reinterpret_cast<const float4 *>(F.mu + ni * kD);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < kD / 4; e++) {
+        const float4 x = __ldg(mu + e);
+        acc[0] = fmaf(q[4 * e], x.x, acc[0]);
+        acc[1] = fmaf(q[4 * e + 1], x.y, acc[1]);
+        acc[2] = fmaf(q[4 * e + 2], x.z, acc[2]);
+        acc[3] = fmaf(q[4 * e + 3], x.w, acc[3]);
+    }
+    const float4 mt = __ldg(F.meta + ni);
+    const int pmin = __float_as_int(mt.z);
+    *pmin_out = pmin;
+    float U = ((acc[0] + acc[1]) + (acc[2] + acc[3]) + A.c_explore * qn * mt.x) * A.scale;
+    if (PRIOR) U += A.lambda[h] * mt.y * erff(((float)i - ((float)pmin + 0.5f) * kS) * A.inv2sigma[h]);
+    return U;
+}
+
+// beam search on one forest for a prefix of m entries; appends the final leaves to the
+// result list (returns the new count)
+template <bool PRIOR>
+__device__ int search_forest(const Forest &F, SearchSmem &S, int bh, int f, int m, float qn, const SearchArgs &A,
+                             int h, int i, int nres, int lane, int ncells, int *dev_flag) {
+    if (m <= 0) return nres;
+    const int C = F.C;
+    // roots: the set bits of m
+    int ncand = 0;
+    {
+        const int k = lane;
+        const bool root = k < F.L && ((m >> k) & 1);
+        const unsigned bal = __ballot_sync(kFull, root);
+        if (root) {
+            const int slot = __popc(bal >> (k + 1));      // high bits first
+            const int node = (((m >> k) - 1) << (k + 1)) + 1;
+            int pm;
+            S.U[slot] = node_U<PRIOR>(F, F.lvl(bh, f, k) * 2 * C, node, S.q, qn, A, h, i, &pm);
+            S.ref[slot] = (k << 26) | node;
+            S.pmin[slot] = pm;
+        }
+        ncand = __popc(bal);
+    }
+    __syncwarp();
+    for (int guard = 0; guard < 64; guard++) {
+        // keep the beam best candidates: rank = number of candidates that beat this one
+        int nb = min(ncand, A.beam);
+        for (int j = lane; j < ncand; j += 32) {
+            const float Uj = S.U[j];
+            const int pj = S.pmin[j];
+            int rank = 0;
+            for (int x = 0; x < ncand; x++) rank += beats(S.U[x], S.pmin[x], Uj, pj);
+            if (rank < A.beam) {
+                S.bU[rank] = Uj;
+                S.bref[rank] = S.ref[j];
+                S.bpmin[rank] = pj;
+            }
+        }
+        __syncwarp();
+        // expand every internal node
+        int cnt0 = 0, cnt1 = 0;
+        bool int0 = false, int1 = false;
+        if (lane < nb) {
+            const int k = S.bref[lane] >> 26, v = (S.bref[lane] & ((1 << 26) - 1)) & ((2 << k) - 1);
+            int0 = v < (1 << k);
+            cnt0 = int0 ? 2 : 1;
+        }
+        if (lane + 32 < nb) {
+            const int k = S.bref[lane + 32] >> 26, v = (S.bref[lane + 32] & ((1 << 26) - 1)) & ((2 << k) - 1);
+            int1 = v < (1 << k);
+            cnt1 = int1 ? 2 : 1;
+        }
+        if (!__any_sync(kFull, int0 || int1)) {
+            for (int j = lane; j < nb; j += 32) {          // all leaves: the result
+                const int k = S.bref[j] >> 26, node = S.bref[j] & ((1 << 26) - 1);
+                const int blk = node >> (k + 1), v = node & ((2 << k) - 1);
+                int cell = F.ord[F.lvl(bh, f, k) * C + ((size_t)blk << k) + (v - (1 << k))];
+                if ((unsigned)cell >= (unsigned)ncells) {  // a forest not built from these summaries
+                    atomicOr(dev_flag, kFlagCheck);
+                    cell = -1;
+                }
+                S.rcell[nres + j] = cell;
+                S.rU[nres + j] = S.bU[j];
+            }
+            __syncwarp();
+            return nres + nb;
+        }
+        int inc0 = cnt0, inc1 = cnt1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y0 = __shfl_up_sync(kFull, inc0, o), y1 = __shfl_up_sync(kFull, inc1, o);
+            if (lane >= o) { inc0 += y0; inc1 += y1; }
+        }
+        const int tot0 = __shfl_sync(kFull, inc0, 31), tot1 = __shfl_sync(kFull, inc1, 31);
+        const int pos0 = inc0 - cnt0, pos1 = tot0 + inc1 - cnt1;
+        for (int half = 0; half < 2; half++) {
+            const int j = lane + 32 * half;
+            if (j >= nb) continue;
+            const int ref = S.bref[j];
+            const int k = ref >> 26, node = ref & ((1 << 26) - 1);
+            const int v = node & ((2 << k) - 1);
+            const int o = half ? pos1 : pos0;
+            if (v >= (1 << k)) {                            // a leaf stays
+                S.U[o] = S.bU[j];
+                S.ref[o] = ref;
+                S.pmin[o] = S.bpmin[j];
+            } else {
+                const size_t base = F.lvl(bh, f, k) * 2 * C;
+                const int c0 = node + v, c1 = node + v + 1;  // heap children 2v, 2v + 1
+                int p0, p1;
+                S.U[o] = node_U<PRIOR>(F, base, c0, S.q, qn, A, h, i, &p0);
+                S.ref[o] = (k << 26) | c0;
+                S.pmin[o] = p0;
+                S.U[o + 1] = node_U<PRIOR>(F, base, c1, S.q, qn, A, h, i, &p1);
+                S.ref[o + 1] = (k << 26) | c1;
+                S.pmin[o + 1] = p1;
+            }
+        }
+        ncand = tot0 + tot1;
+        __syncwarp();
+    }
+    return nres;                                           // unreachable: depth < 64
+}
+
+template <typename T, bool PRIOR>
+__global__ void __launch_bounds__(kSearchWarps * 32) tree_search_kernel(Forest F, const T *__restrict__ Q,
+                                                                        SearchArgs A, int32_t *__restrict__ idx,
+                                                                        int *dev_flag) {
+    __shared__ SearchSmem smem[kSearchWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    SearchSmem &S = smem[warp];
+    const int bh = blockIdx.y, h = bh % A.H;
+    const int r = blockIdx.x * kSearchWarps + warp;
+    if (r >= A.Nq) return;
+    const size_t row = (size_t)bh * A.Nq + r;
+    int32_t *out = idx + row * A.K;
+    if (F.hdr[0] != kTreeMagic || F.hdr[2] != F.C || F.hdr[3] != F.L || F.hdr[4] != (int)gridDim.y) {
+        for (int j = lane; j < A.K; j += 32) out[j] = -1;
+        if (lane == 0) atomicOr(dev_flag, kFlagCheck);
+        return;
+    }
+    const int i = A.q0 + r;
+    const float q0 = to_f<T>(Q[row * kD + 2 * lane]), q1 = to_f<T>(Q[row * kD + 2 * lane + 1]);
+    S.q[2 * lane] = q0;
+    S.q[2 * lane + 1] = q1;
+    const float qn = sqrtf(warp_sum(q0 * q0 + q1 * q1));
+    __syncwarp();
+    const int n = cand_count(i, A.w, F.C);
+    int nres = search_forest<PRIOR>(F, S, bh, 0, n, qn, A, h, i, 0, lane, n, dev_flag);
+    const int n0 = nres;
+    if (F.hdr[1] && n > 0) {
+        const int m = F.admp[(size_t)bh * (F.C + 1) + n];
+        nres = search_forest<PRIOR>(F, S, bh, 1, m, qn, A, h, i, nres, lane, n, dev_flag);
+    }
+    // a cell both beams reached counts once (forest 0's copy)
+    for (int j = n0 + lane; j < nres; j += 32) {
+        bool dup = false;
+        for (int x = 0; x < n0; x++) dup |= S.rcell[x] == S.rcell[j];
+        if (dup) S.rcell[j] = -1;
+    }
+    __syncwarp();
+    // the K best by eq. (7) (U desc, cell asc), written in ascending cell order; the
+    // candidate arrays are free now: S.ref holds each result's rank
+    int nsel = 0;
+    for (int j = 0; j < nres; j++) nsel += S.rcell[j] >= 0;
+    nsel = min(nsel, A.K);
+    for (int j = lane; j < nres; j += 32) {
+        const int cj = S.rcell[j];
+        int rank = 0x7fffffff;
+        if (cj >= 0) {
+            const float Uj = S.rU[j];
+            rank = 0;
+            for (int x = 0; x < nres; x++) rank += S.rcell[x] >= 0 && beats(S.rU[x], S.rcell[x], Uj, cj);
+        }
+        S.ref[j] = rank;
+    }
+    __syncwarp();
+    for (int j = lane; j < nres; j += 32) {
+        const int cj = S.rcell[j];
+        if (S.ref[j] >= A.K) continue;
+        int pos = 0;
+        for (int x = 0; x < nres; x++) pos += S.ref[x] < A.K && S.rcell[x] < cj;
+        out[pos] = cj;
+    }
+    for (int j = nsel + lane; j < A.K; j += 32) out[j] = -1;
+}
+
+}  // namespace
+
+size_t forest_bytes(const fs_params *p) { return forest_geom(p).total; }
+
+cudaError_t launch_tree_build(const fs_params *p, const float *kbar, const float *amax, const float *tau,
+                              void *forest, cudaStream_t st) {
+    const ForestGeom g = forest_geom(p);
+    const Forest F = forest_view(forest, g);
+    TauArgs T;
+    for (int h = 0; h < FS_MAX_HEADS; h++) T.tau[h] = tau && h < p->H ? tau[h] : 0.f;
+    {
+        LaunchScope sc(kTreePrep, st);
+        tree_prep_kernel<<<g.BH, 1024, 0, st>>>(F, kbar, amax, p->H, tau != nullptr, T);
+        if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
+    }
+    const long long nent = (long long)g.BH * 2 * g.C;
+    for (int k = 0; k < g.L; k++) {
+        LaunchScope sc(kTreeMerge, st);
+        tree_merge_kernel<<<(unsigned)((nent + 255) / 256), 256, 0, st>>>(F, g.BH, k);
+        if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
+    }
+    const long long nwarps = (long long)g.BH * 2 * 2 * g.C;
+    for (int k = 0; k < g.L; k++) {
+        LaunchScope sc(kTreeNodes, st);
+        tree_nodes_kernel<<<(unsigned)((nwarps + 7) / 8), 256, 0, st>>>(F, kbar, amax, g.BH, k);
+        if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_tree_search(const fs_params *p, const Dev &D, const void *Q, const void *forest, int beam,
+                               float c_explore, int32_t *idx, int *dev_flag, cudaStream_t st) {
+    const ForestGeom g = forest_geom(p);
+    const Forest F = forest_view(const_cast<void *>(forest), g);
+    SearchArgs A;
+    A.Nq = p->Nq; A.H = p->H; A.w = p->w; A.K = p->K; A.q0 = p->Nk - p->Nq; A.beam = beam;
+    A.scale = D.scale;
+    A.c_explore = c_explore;
+    for (int h = 0; h < FS_MAX_HEADS; h++) {
+        A.lambda[h] = D.lambda[h];
+        A.inv2sigma[h] = D.inv2sigma[h];
+    }
+    const dim3 grid((p->Nq + kSearchWarps - 1) / kSearchWarps, g.BH);
+    LaunchScope sc(kTreeSearch, st);
+    if (p->dtype == FS_BF16) {
+        auto kern = D.has_prior ? tree_search_kernel<__nv_bfloat16, true> : tree_search_kernel<__nv_bfloat16, false>;
+        kern<<<grid, kSearchWarps * 32, 0, st>>>(F, static_cast<const __nv_bfloat16 *>(Q), A, idx, dev_flag);
+    } else {
+        auto kern = D.has_prior ? tree_search_kernel<float, true> : tree_search_kernel<float, false>;
+        kern<<<grid, kSearchWarps * 32, 0, st>>>(F, static_cast<const float *>(Q), A, idx, dev_flag);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace fs

@@ -31,6 +31,48 @@ def test_library_exports_every_declared_function():
     assert set(fs.EXPORTS) <= set(declared)
 
 
+def test_binding_declares_every_signature():
+    """Every declared function is in the binding with its argument types set (an
+    undeclared size_t would be passed as a 32-bit int)."""
+    L = fs.load()
+    assert set(header_functions()) <= set(fs.EXPORTS)
+    for name in fs.EXPORTS:
+        assert getattr(L, name).argtypes is not None, name
+
+
+def test_tree_arguments_rejected_on_host():
+    p = params(W=-1, P=-1)
+    n = fs.forest_bytes(p)
+    assert n > 0
+    big = fs.Params(B=1, H=2, Nq=256, Nk=4096, alpha=[0.5, 1.0], W=-1, P=-1)
+    assert fs.forest_bytes(big) > n
+    for beam in (0, 65):
+        with pytest.raises(fs.FsError) as e:
+            fs.select_topk_tree(p, _FakeTensor(1), _FakeTensor(n), _FakeTensor(1), _FakeTensor(1 << 20), beam,
+                                stream=0)
+        assert e.value.code == 1
+    with pytest.raises(fs.FsError) as e:          # forest buffer too small
+        fs.select_topk_tree(p, _FakeTensor(1), _FakeTensor(n - 1), _FakeTensor(1), _FakeTensor(1 << 20), 8,
+                            stream=0)
+    assert e.value.code == 3
+
+
+class _FakeTensor:
+    """Stands in for a device tensor in calls that must fail before any launch."""
+
+    def __init__(self, nbytes):
+        self.nbytes = nbytes
+
+    def data_ptr(self):
+        return 0x1000
+
+    def numel(self):
+        return self.nbytes
+
+    def element_size(self):
+        return 1
+
+
 def test_status_strings():
     for code in range(7):
         assert fs.status_string(code)
