@@ -128,9 +128,11 @@ fs_status fs_forward(const fs_params *p, const void *Q, const void *K, const voi
 fs_status fs_host_scratch_size(const fs_params *p, size_t *bytes);
 
 /* fs_forward on HOST buffers hQ, hK, hV -> hO (pinned memory makes the copies async).
- * Copies in, computes and copies out on `stream` using the caller's device scratch
- * (fs_host_scratch_size bytes).  Returns after enqueueing; synchronize `stream` (or call
- * fs_sync_status) before reading hO. */
+ * Copies in, computes and copies out using the caller's device scratch
+ * (fs_host_scratch_size bytes), pipelined over chunks of heads: a chunk's inputs copy in
+ * on an internal stream while the previous chunk computes on `stream` and the one before
+ * copies out on another internal stream; `stream` waits for the last copy out.  Returns
+ * after enqueueing; synchronize `stream` (or call fs_sync_status) before reading hO. */
 fs_status fs_forward_host(const fs_params *p, const void *hQ, const void *hK, const void *hV,
                           void *hO, void *dscratch, size_t scratch_bytes, void *stream);
 

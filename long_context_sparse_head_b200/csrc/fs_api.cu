@@ -2,6 +2,7 @@
 // workspace layout and the launch sequence
 //   summaries (eq. (5)) -> TopP exit table (eq. (8)) -> selection (eq. (7))
 //   -> readout (eq. (9)) -> window + combine (eqs. (2)-(4)).
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 
@@ -365,6 +366,26 @@ extern "C" fs_status fs_host_scratch_size(const fs_params *p, size_t *bytes) {
     return FS_OK;
 }
 
+namespace {
+// Streams and events of one pipelined host call; released when the call has been enqueued
+// (the runtime defers the release until the enqueued work completes).
+struct HostPipe {
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t ev[2 * 64 + 2] = {};
+    int nev = 0;
+    ~HostPipe() {
+        for (int i = 0; i < nev; i++) cudaEventDestroy(ev[i]);
+        if (in) cudaStreamDestroy(in);
+        if (out) cudaStreamDestroy(out);
+    }
+    cudaEvent_t event() {
+        if (nev >= (int)(sizeof(ev) / sizeof(ev[0]))) return nullptr;
+        if (cudaEventCreateWithFlags(&ev[nev], cudaEventDisableTiming) != cudaSuccess) return nullptr;
+        return ev[nev++];
+    }
+};
+}  // namespace
+
 extern "C" fs_status fs_forward_host(const fs_params *p, const void *hQ, const void *hK,
                                      const void *hV, void *hO, void *dscratch,
                                      size_t scratch_bytes, void *stream) {
@@ -375,18 +396,55 @@ extern "C" fs_status fs_forward_host(const fs_params *p, const void *hQ, const v
     const HostScratch h = host_scratch(p);
     if (!dscratch || scratch_bytes < h.total) return FS_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
-    const size_t e = esize(p->dtype), BH = (size_t)p->B * p->H;
-    void *dQ = at<void>(dscratch, h.q), *dK = at<void>(dscratch, h.k);
-    void *dV = at<void>(dscratch, h.v), *dO = at<void>(dscratch, h.o);
+    const size_t e = esize(p->dtype);
+    uint8_t *dQ = at<uint8_t>(dscratch, h.q), *dK = at<uint8_t>(dscratch, h.k);
+    uint8_t *dV = at<uint8_t>(dscratch, h.v), *dO = at<uint8_t>(dscratch, h.o);
     void *ws = at<void>(dscratch, h.ws);
-    // one plain async copy per buffer
-    if (cudaMemcpyAsync(dQ, hQ, BH * p->Nq * kD * e, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(dK, hK, BH * p->Nk * kD * e, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(dV, hV, BH * p->Nk * kD * e, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    // Heads are independent, so the call runs as a pipeline over about 8 chunks (heads of
+    // one batch entry, or whole batch entries): chunk c's inputs copy in (stream `in`) while
+    // chunk c-1 computes (the caller's stream) and chunk c-2's output copies out (stream
+    // `out`).  Each direction is one plain async copy per buffer and chunk.
+    constexpr int kChunks = 8;
+    const int per_b = p->B >= kChunks ? 1 : kChunks / p->B;             // chunks per batch entry
+    const int hc = (p->H + per_b - 1) / per_b;                          // heads per chunk
+    const int bc = p->B >= kChunks ? (p->B + kChunks - 1) / kChunks : 1; // batch entries per chunk
+    HostPipe pp;
+    if (cudaStreamCreateWithFlags(&pp.in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&pp.out, cudaStreamNonBlocking) != cudaSuccess)
         return FS_ERR_CUDA;
-    s = run_forward(p, dQ, dK, dV, nullptr, nullptr, nullptr, dO, ws, st);
-    if (s != FS_OK) return s;
-    return cuda_status(cudaMemcpyAsync(hO, dO, BH * p->Nq * kD * e, cudaMemcpyDeviceToHost, st));
+    cudaEvent_t start = pp.event();
+    if (!start || cudaEventRecord(start, st) != cudaSuccess || cudaStreamWaitEvent(pp.in, start, 0) != cudaSuccess)
+        return FS_ERR_CUDA;                          // earlier work on `stream` may still use the scratch
+    for (int b = 0; b < p->B; b += bc) {
+        for (int h0 = 0; h0 < p->H; h0 += hc) {
+            const int nb = std::min(bc, p->B - b), nh = std::min(hc, p->H - h0);
+            fs_params sub = *p;
+            sub.B = nb;
+            sub.H = nh;
+            sub.alpha = p->alpha + h0;
+            sub.lambda = p->lambda ? p->lambda + h0 : nullptr;
+            sub.sigma = p->sigma ? p->sigma + h0 : nullptr;
+            const size_t hb = (size_t)b * p->H + h0;            // first (b, h) of the chunk
+            const size_t qoff = hb * p->Nq * kD * e, koff = hb * p->Nk * kD * e;
+            const size_t qbytes = (size_t)nb * nh * p->Nq * kD * e, kbytes = (size_t)nb * nh * p->Nk * kD * e;
+            cudaEvent_t in_done = pp.event(), fwd_done = pp.event();
+            if (!in_done || !fwd_done) return FS_ERR_CUDA;
+            if (cudaMemcpyAsync(dQ + qoff, static_cast<const uint8_t *>(hQ) + qoff, qbytes, cudaMemcpyHostToDevice, pp.in) != cudaSuccess ||
+                cudaMemcpyAsync(dK + koff, static_cast<const uint8_t *>(hK) + koff, kbytes, cudaMemcpyHostToDevice, pp.in) != cudaSuccess ||
+                cudaMemcpyAsync(dV + koff, static_cast<const uint8_t *>(hV) + koff, kbytes, cudaMemcpyHostToDevice, pp.in) != cudaSuccess ||
+                cudaEventRecord(in_done, pp.in) != cudaSuccess || cudaStreamWaitEvent(st, in_done, 0) != cudaSuccess)
+                return FS_ERR_CUDA;
+            s = run_forward(&sub, dQ + qoff, dK + koff, dV + koff, nullptr, nullptr, nullptr, dO + qoff, ws, st);
+            if (s != FS_OK) return s;
+            if (cudaEventRecord(fwd_done, st) != cudaSuccess || cudaStreamWaitEvent(pp.out, fwd_done, 0) != cudaSuccess ||
+                cudaMemcpyAsync(static_cast<uint8_t *>(hO) + qoff, dO + qoff, qbytes, cudaMemcpyDeviceToHost, pp.out) != cudaSuccess)
+                return FS_ERR_CUDA;
+        }
+    }
+    cudaEvent_t all_out = pp.event();                 // the caller's stream joins the copies out
+    if (!all_out || cudaEventRecord(all_out, pp.out) != cudaSuccess || cudaStreamWaitEvent(st, all_out, 0) != cudaSuccess)
+        return FS_ERR_CUDA;
+    return FS_OK;
 }
 
 extern "C" fs_status fs_sync_status(void *ws, void *stream) {
