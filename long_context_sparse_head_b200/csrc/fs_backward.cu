@@ -11,8 +11,10 @@
 //
 // Kernels (CUDA cores, float32 throughout):
 //   rotate_keys  k'_j = R_j k_j (absolute positions, double-precision angle tables)
-//   rows         one warp per query row: both branches' softmax statistics, o^sr, u, y, du,
-//                the per-row terms the key kernels need (log-sum-exps, g.o), dQ, dalpha terms
+//   win_rows     one warp per 32 query rows (lane = row), the band's keys staged in shared
+//                memory: the window's log-sum-exp and g.o^sr, its part of dQ, rotated queries
+//   lr_rows      one warp per query row, each selected cell staged in shared memory: the
+//                readout's log-sum-exp, u, RMSNorm, du, g.u-term, its part of dQ, dalpha terms
 //   window_kv    one warp per 32 keys (lane = key): dK, dV over the queries whose window
 //                holds them; writes every key (zeros where none)
 //   cells        cell -> rows lists by counting sort of idx (count, scan, fill)
@@ -81,174 +83,344 @@ __global__ void bwd_rotate_keys_kernel(const T *__restrict__ K, float *__restric
     krot[2 * e + 1] = k0 * cs.y + k1 * cs.x;
 }
 
-// lane j's dot product of the shared 64-vector v with the 64 floats (or T) at row
-template <typename R> __device__ __forceinline__ float dot_row(const float *v, const R *row) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int e = 0; e < kD; e++) acc[e & 3] = fmaf(v[e], to_f<R>(row[e]), acc[e & 3]);
-    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
-}
-template <> __device__ __forceinline__ float dot_row<float>(const float *v, const float *row) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const float4 *r4 = reinterpret_cast<const float4 *>(row);
-#pragma unroll
-    for (int e = 0; e < kD / 4; e++) {
-        const float4 x = __ldg(r4 + e);
-        acc[0] = fmaf(v[4 * e], x.x, acc[0]);
-        acc[1] = fmaf(v[4 * e + 1], x.y, acc[1]);
-        acc[2] = fmaf(v[4 * e + 2], x.z, acc[2]);
-        acc[3] = fmaf(v[4 * e + 3], x.w, acc[3]);
-    }
-    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
-}
-
-constexpr int kRowWarps = 8;
+// ---- window rows: one warp per 32 consecutive query rows (lane = row); the keys of the
+// warp's band [i0 - w, i0 + 31] pass through shared memory in 32-key tiles, read by every
+// lane at once (broadcast).  Pass 1: log-sum-exp and D = dO.o^sr (online, as
+// sum_j p_j (dO.v_j)); pass 2: dq' = sum_j dl_j k'_j.  Writes dQ (window part), the rotated
+// queries and (lse_sr, D_sr).
+constexpr int kWinWarps = 2;                  // 32 KB of static shared memory
 
 template <typename T>
-__global__ void __launch_bounds__(kRowWarps * 32) bwd_rows_kernel(
+__device__ __forceinline__ void load_row64(const T *src, float *dst);
+template <>
+__device__ __forceinline__ void load_row64<float>(const float *src, float *dst) {
+#pragma unroll
+    for (int e = 0; e < kD / 4; e++) {
+        const float4 x = __ldg(reinterpret_cast<const float4 *>(src) + e);
+        dst[4 * e] = x.x; dst[4 * e + 1] = x.y; dst[4 * e + 2] = x.z; dst[4 * e + 3] = x.w;
+    }
+}
+template <>
+__device__ __forceinline__ void load_row64<__nv_bfloat16>(const __nv_bfloat16 *src, float *dst) {
+#pragma unroll
+    for (int e = 0; e < kD / 8; e++) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(src) + e);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            dst[8 * e + 2 * k] = __uint_as_float(w[k] << 16);
+            dst[8 * e + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+        }
+    }
+}
+
+// 32 rows x 64 of f32 from rows [j0, j0 + 32) of src (rows past `n` read as zeros) into a
+// dense [32][64] tile; coalesced 16-byte loads
+template <typename T>
+__device__ __forceinline__ void stage_tile(const T *src, int j0, int n, float (*tile)[kD], int lane);
+template <>
+__device__ __forceinline__ void stage_tile<float>(const float *src, int j0, int n, float (*tile)[kD], int lane) {
+#pragma unroll 4
+    for (int q = lane; q < 32 * kD / 4; q += 32) {
+        const int row = q >> 4, c4 = q & 15;
+        const float4 x = j0 + row < n ? __ldg(reinterpret_cast<const float4 *>(src + (size_t)(j0 + row) * kD) + c4)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(&tile[row][4 * c4]) = x;
+    }
+}
+template <>
+__device__ __forceinline__ void stage_tile<__nv_bfloat16>(const __nv_bfloat16 *src, int j0, int n, float (*tile)[kD],
+                                                          int lane) {
+#pragma unroll 4
+    for (int q = lane; q < 32 * kD / 8; q += 32) {
+        const int row = q >> 3, c8 = q & 7;
+        const uint4 x = j0 + row < n ? __ldg(reinterpret_cast<const uint4 *>(src + (size_t)(j0 + row) * kD) + c8)
+                                     : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        float4 lo, hi;
+        lo.x = __uint_as_float(w[0] << 16); lo.y = __uint_as_float(w[0] & 0xffff0000u);
+        lo.z = __uint_as_float(w[1] << 16); lo.w = __uint_as_float(w[1] & 0xffff0000u);
+        hi.x = __uint_as_float(w[2] << 16); hi.y = __uint_as_float(w[2] & 0xffff0000u);
+        hi.z = __uint_as_float(w[3] << 16); hi.w = __uint_as_float(w[3] & 0xffff0000u);
+        *reinterpret_cast<float4 *>(&tile[row][8 * c8]) = lo;
+        *reinterpret_cast<float4 *>(&tile[row][8 * c8 + 4]) = hi;
+    }
+}
+
+// a.b over 64 with a in registers and b a shared row read by every lane (broadcast)
+__device__ __forceinline__ float dot_bcast(const float *a, const float *b) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < kD / 4; e++) {
+        const float4 x = *reinterpret_cast<const float4 *>(b + 4 * e);
+        acc[0] = fmaf(a[4 * e], x.x, acc[0]);
+        acc[1] = fmaf(a[4 * e + 1], x.y, acc[1]);
+        acc[2] = fmaf(a[4 * e + 2], x.z, acc[2]);
+        acc[3] = fmaf(a[4 * e + 3], x.w, acc[3]);
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kWinWarps * 32) bwd_win_rows_kernel(
+    const BwdArgs A, const T *__restrict__ Q, const T *__restrict__ V, const T *__restrict__ dO,
+    const float *__restrict__ krot, const float2 *__restrict__ lo, const float2 *__restrict__ hi,
+    float *__restrict__ dQ, float *__restrict__ qrot, float *__restrict__ rowst) {
+    __shared__ __align__(16) float s_k[kWinWarps][32][kD];
+    __shared__ __align__(16) float s_v[kWinWarps][32][kD];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y;
+    const int r0 = (blockIdx.x * kWinWarps + warp) * 32;
+    if (r0 >= A.Nq) return;                                   // warp-uniform
+    const int r = r0 + lane;
+    const bool valid = r < A.Nq;
+    const int i = A.q0 + (valid ? r : A.Nq - 1);
+    const size_t row = (size_t)bh * A.Nq + (valid ? r : A.Nq - 1);
+    const size_t kb = (size_t)bh * A.Nk;
+    float qr[kD], g[kD];
+    load_row64<T>(Q + row * kD, qr);
+#pragma unroll
+    for (int m = 0; m < kD / 2; m++) {                        // q' = R_i q
+        const float2 cs = rope_cs_tab(i, m, lo, hi);
+        const float a = qr[2 * m], b = qr[2 * m + 1];
+        qr[2 * m] = a * cs.x - b * cs.y;
+        qr[2 * m + 1] = a * cs.y + b * cs.x;
+    }
+    if (valid) {
+        float4 *d4 = reinterpret_cast<float4 *>(qrot + row * kD);
+#pragma unroll
+        for (int e = 0; e < kD / 4; e++) d4[e] = make_float4(qr[4 * e], qr[4 * e + 1], qr[4 * e + 2], qr[4 * e + 3]);
+    }
+    load_row64<T>(dO + row * kD, g);
+    const int i0 = A.q0 + r0;
+    const int jlo = max(0, i0 - A.w), jhi = min(A.q0 + A.Nq - 1, i0 + 31);
+    float m = -INFINITY, l = 0.f, D = 0.f;
+    for (int t0 = jlo; t0 <= jhi; t0 += 32) {                 // pass 1: statistics
+        __syncwarp();
+        stage_tile<float>(krot + kb * kD, t0, jhi + 1, s_k[warp], lane);
+        stage_tile<T>(V + kb * kD, t0, jhi + 1, s_v[warp], lane);
+        __syncwarp();
+        const int nt = min(32, jhi + 1 - t0);
+        for (int jj = 0; jj < nt; jj++) {
+            const int j = t0 + jj;
+            const float x = dot_bcast(qr, s_k[warp][jj]) * A.scale;
+            const float dp = dot_bcast(g, s_v[warp][jj]);
+            if (valid && j <= i && j >= i - A.w) {
+                const float mn = fmaxf(m, x);
+                const float corr = __expf(m - mn);           // 0 while m is -inf
+                const float pj = __expf(x - mn);
+                l = l * corr + pj;
+                D = D * corr + pj * dp;
+                m = mn;
+            }
+        }
+    }
+    const float lse = m + __logf(l), Dsr = D / l;
+    float dq[kD];
+#pragma unroll
+    for (int e = 0; e < kD; e++) dq[e] = 0.f;
+    for (int t0 = jlo; t0 <= jhi; t0 += 32) {                 // pass 2: dq' = sum_j dl_j k'_j
+        __syncwarp();
+        stage_tile<float>(krot + kb * kD, t0, jhi + 1, s_k[warp], lane);
+        stage_tile<T>(V + kb * kD, t0, jhi + 1, s_v[warp], lane);
+        __syncwarp();
+        const int nt = min(32, jhi + 1 - t0);
+        for (int jj = 0; jj < nt; jj++) {
+            const int j = t0 + jj;
+            const float x = dot_bcast(qr, s_k[warp][jj]) * A.scale;
+            const float dp = dot_bcast(g, s_v[warp][jj]);
+            const bool in = valid && j <= i && j >= i - A.w;
+            const float dl = in ? __expf(x - lse) * (dp - Dsr) * A.scale : 0.f;
+            const float *kr = s_k[warp][jj];
+#pragma unroll
+            for (int e = 0; e < kD / 4; e++) {
+                const float4 k4 = *reinterpret_cast<const float4 *>(kr + 4 * e);
+                dq[4 * e] = fmaf(dl, k4.x, dq[4 * e]);
+                dq[4 * e + 1] = fmaf(dl, k4.y, dq[4 * e + 1]);
+                dq[4 * e + 2] = fmaf(dl, k4.z, dq[4 * e + 2]);
+                dq[4 * e + 3] = fmaf(dl, k4.w, dq[4 * e + 3]);
+            }
+        }
+    }
+    if (!valid) return;
+#pragma unroll
+    for (int mm = 0; mm < kD / 2; mm++) {                     // dq = R_i^T dq'
+        const float2 cs = rope_cs_tab(i, mm, lo, hi);
+        const float a = dq[2 * mm], b = dq[2 * mm + 1];
+        dq[2 * mm] = a * cs.x + b * cs.y;
+        dq[2 * mm + 1] = -a * cs.y + b * cs.x;
+    }
+    float4 *d4 = reinterpret_cast<float4 *>(dQ + row * kD);
+#pragma unroll
+    for (int e = 0; e < kD / 4; e++) d4[e] = make_float4(dq[4 * e], dq[4 * e + 1], dq[4 * e + 2], dq[4 * e + 3]);
+    rowst[row * 4] = lse;
+    rowst[row * 4 + 1] = Dsr;
+}
+
+// ---- readout rows: one warp per query row, lane m holding dimensions (2m, 2m + 1).  A
+// cell's logits are formed as per-lane partial products over the lane's two dimensions,
+// then a transposed butterfly sum hands lane t the total for token t (31 shuffles for 32
+// tokens).  Pass 1: log-sum-exp and u; RMSNorm and du; pass 2: dq += sum_t dl_t k_t.  Adds
+// the readout part to dQ; writes du, (lse_lr, D_lr) and the dalpha terms.
+constexpr int kLrWarps = 4;
+
+template <typename T> __device__ __forceinline__ float2 ld_pair(const T *p);
+template <> __device__ __forceinline__ float2 ld_pair<float>(const float *p) {
+    return __ldg(reinterpret_cast<const float2 *>(p));
+}
+template <> __device__ __forceinline__ float2 ld_pair<__nv_bfloat16>(const __nv_bfloat16 *p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+}
+
+// lane t receives the sum over the warp of v[t]
+__device__ __forceinline__ float transpose_sum32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const bool up = lane & o;
+#pragma unroll
+        for (int k = 0; k < o; k++) {
+            const float send = up ? v[k] : v[k + o];
+            const float keep = up ? v[k + o] : v[k];
+            v[k] = keep + __shfl_xor_sync(kFull, send, o);
+        }
+    }
+    return v[0];
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kLrWarps * 32) bwd_lr_rows_kernel(
     const BwdArgs A, const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V,
-    const int32_t *__restrict__ idx, const T *__restrict__ dO, const float *__restrict__ krot,
-    const float2 *__restrict__ lo, const float2 *__restrict__ hi, float *__restrict__ dQ, float *__restrict__ qrot,
-    float *__restrict__ rowst, float *__restrict__ du_out, float *__restrict__ dal) {
-    __shared__ float s_q[kRowWarps][kD], s_qr[kRowWarps][kD], s_g[kRowWarps][kD], s_du[kRowWarps][kD];
+    const int32_t *__restrict__ idx, const T *__restrict__ dO, float *__restrict__ dQ, float *__restrict__ rowst,
+    float *__restrict__ du_out, float *__restrict__ dal) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.y, h = bh % A.H;
-    const int r = blockIdx.x * kRowWarps + warp;
-    if (r >= A.Nq) return;                                   // warp-uniform
+    const int r = blockIdx.x * kLrWarps + warp;
+    if (r >= A.Nq) return;                                    // warp-uniform
     const size_t row = (size_t)bh * A.Nq + r;
-    const int i = A.q0 + r;
     const size_t kb = (size_t)bh * A.Nk;
-    // lane m holds the pair (2m, 2m+1) of q, R_i q and dO
-    const float q0 = to_f<T>(Q[row * kD + 2 * lane]), q1 = to_f<T>(Q[row * kD + 2 * lane + 1]);
-    const float2 cs = rope_cs_tab(i, lane, lo, hi);
-    const float qr0 = q0 * cs.x - q1 * cs.y, qr1 = q0 * cs.y + q1 * cs.x;
-    const float g0 = to_f<T>(dO[row * kD + 2 * lane]), g1 = to_f<T>(dO[row * kD + 2 * lane + 1]);
-    s_q[warp][2 * lane] = q0; s_q[warp][2 * lane + 1] = q1;
-    s_qr[warp][2 * lane] = qr0; s_qr[warp][2 * lane + 1] = qr1;
-    s_g[warp][2 * lane] = g0; s_g[warp][2 * lane + 1] = g1;
-    qrot[row * kD + 2 * lane] = qr0;
-    qrot[row * kD + 2 * lane + 1] = qr1;
-    __syncwarp();
-
-    // ---- window: statistics and o^sr (lane = key for the logits, lane = pair for p V)
-    const int jlo = max(0, i - A.w), L = i - jlo + 1;
-    float m = -INFINITY, l = 0.f, o0 = 0.f, o1 = 0.f;
-    for (int b = 0; b * 32 < L; b++) {
-        const int j = jlo + 32 * b + lane;
-        const bool ok = j <= i;
-        const float x = ok ? dot_row<float>(s_qr[warp], krot + (kb + j) * kD) * A.scale : -INFINITY;
-        const float mn = fmaxf(m, warp_max(x));
-        const float corr = m == -INFINITY ? 0.f : __expf(m - mn);
-        const float pj = ok ? __expf(x - mn) : 0.f;
-        l = l * corr + warp_sum(pj);
-        o0 *= corr;
-        o1 *= corr;
-        const int nb = min(32, L - 32 * b);
-        for (int e = 0; e < nb; e++) {
-            const float pe = __shfl_sync(kFull, pj, e);
-            const T *vr = V + (kb + jlo + 32 * b + e) * kD + 2 * lane;
-            o0 = fmaf(pe, to_f<T>(vr[0]), o0);
-            o1 = fmaf(pe, to_f<T>(vr[1]), o1);
-        }
-        m = mn;
-    }
-    o0 /= l;
-    o1 /= l;
-    const float lse_sr = m + __logf(l);
-    const float D_sr = warp_sum(g0 * o0 + g1 * o1);
-    // dq' = sum_j dl_j k'_j
-    float dq0 = 0.f, dq1 = 0.f;
-    for (int b = 0; b * 32 < L; b++) {
-        const int j = jlo + 32 * b + lane;
-        const bool ok = j <= i;
-        float dl = 0.f;
-        if (ok) {
-            const float x = dot_row<float>(s_qr[warp], krot + (kb + j) * kD) * A.scale;
-            const float pj = __expf(x - lse_sr);
-            const float dp = dot_row<T>(s_g[warp], V + (kb + j) * kD);
-            dl = pj * (dp - D_sr) * A.scale;
-        }
-        const int nb = min(32, L - 32 * b);
-        for (int e = 0; e < nb; e++) {
-            const float de = __shfl_sync(kFull, dl, e);
-            const float *kr = krot + (kb + jlo + 32 * b + e) * kD + 2 * lane;
-            dq0 = fmaf(de, kr[0], dq0);
-            dq1 = fmaf(de, kr[1], dq1);
-        }
-    }
-    // rotate back: R_i^T
-    float dqa = dq0 * cs.x + dq1 * cs.y, dqb = -dq0 * cs.y + dq1 * cs.x;
-
-    // ---- readout over the selected cells' tokens (NoPE)
     const int32_t *sel = idx + row * A.K;
     int ncell = 0;
     for (int e = 0; e < A.K; e++) ncell += (unsigned)sel[e] < (unsigned)A.C;
-    float lse_lr = -INFINITY, D_lr = 0.f, gy = 0.f;
-    float du0 = 0.f, du1 = 0.f;
+    float lse_lr = -INFINITY, D_lr = 0.f, gy = 0.f, du0 = 0.f, du1 = 0.f;
     if (ncell > 0) {
-        m = -INFINITY; l = 0.f;
-        float u0 = 0.f, u1 = 0.f;
-        for (int e = 0; e < A.K; e++) {
+        const float2 q = ld_pair<T>(Q + row * kD + 2 * lane), g = ld_pair<T>(dO + row * kD + 2 * lane);
+        float m = -INFINITY, l = 0.f, u0 = 0.f, u1 = 0.f;
+        for (int e = 0; e < A.K; e++) {                       // pass 1: lse and u
             const int c = sel[e];
             if ((unsigned)c >= (unsigned)A.C) continue;
-            const size_t t0 = kb + (size_t)c * kS;
-            const float x = dot_row<T>(s_q[warp], K + (t0 + lane) * kD) * A.scale;
+            const T *kc = K + (kb + (size_t)c * kS) * kD + 2 * lane;
+            const T *vc = V + (kb + (size_t)c * kS) * kD + 2 * lane;
+            float v[32];
+#pragma unroll
+            for (int t = 0; t < 32; t++) {
+                const float2 k2 = ld_pair<T>(kc + t * kD);
+                v[t] = fmaf(q.x, k2.x, q.y * k2.y);
+            }
+            const float x = transpose_sum32(v, lane) * A.scale;   // lane t: token t's logit
             const float mn = fmaxf(m, warp_max(x));
-            const float corr = m == -INFINITY ? 0.f : __expf(m - mn);
-            const float pj = __expf(x - mn);
-            l = l * corr + warp_sum(pj);
+            const float corr = __expf(m - mn);
+            const float pt = __expf(x - mn);
+            l = l * corr + warp_sum(pt);
             u0 *= corr;
             u1 *= corr;
-            for (int t = 0; t < kS; t++) {
-                const float pe = __shfl_sync(kFull, pj, t);
-                const T *vr = V + (t0 + t) * kD + 2 * lane;
-                u0 = fmaf(pe, to_f<T>(vr[0]), u0);
-                u1 = fmaf(pe, to_f<T>(vr[1]), u1);
+#pragma unroll
+            for (int t = 0; t < 32; t++) {
+                const float pe = __shfl_sync(kFull, pt, t);
+                const float2 v2 = ld_pair<T>(vc + t * kD);
+                u0 = fmaf(pe, v2.x, u0);
+                u1 = fmaf(pe, v2.y, u1);
             }
             m = mn;
         }
         u0 /= l;
         u1 /= l;
         lse_lr = m + __logf(l);
-        const float ss = warp_sum(u0 * u0 + u1 * u1);
-        const float rin = rsqrtf(ss * (1.f / kD) + A.rms_eps);
+        const float rin = rsqrtf(warp_sum(u0 * u0 + u1 * u1) * (1.f / kD) + A.rms_eps);
         const float y0 = u0 * rin, y1 = u1 * rin;
-        gy = warp_sum(g0 * y0 + g1 * y1);
+        gy = warp_sum(g.x * y0 + g.y * y1);
         const float a = A.alpha[h];
-        const float dyy = a * gy;                                // dy.y with dy = alpha dO
-        du0 = rin * (a * g0 - y0 * dyy * (1.f / kD));
-        du1 = rin * (a * g1 - y1 * dyy * (1.f / kD));
+        const float dyy = a * gy;                             // dy.y with dy = alpha dO
+        du0 = rin * (a * g.x - y0 * dyy * (1.f / kD));
+        du1 = rin * (a * g.y - y1 * dyy * (1.f / kD));
         D_lr = warp_sum(du0 * u0 + du1 * u1);
-        s_du[warp][2 * lane] = du0;
-        s_du[warp][2 * lane + 1] = du1;
-        __syncwarp();
-        for (int e = 0; e < A.K; e++) {
+        float dq0 = 0.f, dq1 = 0.f;
+        for (int e = 0; e < A.K; e++) {                       // pass 2: dq += sum_t dl_t k_t
             const int c = sel[e];
             if ((unsigned)c >= (unsigned)A.C) continue;
-            const size_t t0 = kb + (size_t)c * kS;
-            const float x = dot_row<T>(s_q[warp], K + (t0 + lane) * kD) * A.scale;
-            const float pj = __expf(x - lse_lr);
-            const float dp = dot_row<T>(s_du[warp], V + (t0 + lane) * kD);
-            const float dl = pj * (dp - D_lr) * A.scale;
-            for (int t = 0; t < kS; t++) {
+            const T *kc = K + (kb + (size_t)c * kS) * kD + 2 * lane;
+            const T *vc = V + (kb + (size_t)c * kS) * kD + 2 * lane;
+            float2 k2[32];
+            float v[32], w[32];
+#pragma unroll
+            for (int t = 0; t < 32; t++) {
+                k2[t] = ld_pair<T>(kc + t * kD);
+                const float2 v2 = ld_pair<T>(vc + t * kD);
+                v[t] = fmaf(q.x, k2[t].x, q.y * k2[t].y);
+                w[t] = fmaf(du0, v2.x, du1 * v2.y);
+            }
+            const float x = transpose_sum32(v, lane) * A.scale;
+            const float dp = transpose_sum32(w, lane);
+            const float dl = __expf(x - lse_lr) * (dp - D_lr) * A.scale;
+#pragma unroll
+            for (int t = 0; t < 32; t++) {
                 const float de = __shfl_sync(kFull, dl, t);
-                const T *kr = K + (t0 + t) * kD + 2 * lane;
-                dqa = fmaf(de, to_f<T>(kr[0]), dqa);
-                dqb = fmaf(de, to_f<T>(kr[1]), dqb);
+                dq0 = fmaf(de, k2[t].x, dq0);
+                dq1 = fmaf(de, k2[t].y, dq1);
             }
         }
+        dQ[row * kD + 2 * lane] += dq0;
+        dQ[row * kD + 2 * lane + 1] += dq1;
     }
-    dQ[row * kD + 2 * lane] = dqa;
-    dQ[row * kD + 2 * lane + 1] = dqb;
     du_out[row * kD + 2 * lane] = du0;
     du_out[row * kD + 2 * lane + 1] = du1;
     if (lane == 0) {
-        reinterpret_cast<float4 *>(rowst)[row] = make_float4(lse_sr, D_sr, lse_lr, D_lr);
+        rowst[row * 4 + 2] = lse_lr;
+        rowst[row * 4 + 3] = D_lr;
         dal[row] = gy;
     }
 }
 
-constexpr int kKvWarps = 2, kPad = kD + 1;   // 2 warps: 33 KB of static shared memory
+constexpr int kKvWarps = 2, kPad = kD + 1;   // 2 warps: 41 KB of static shared memory
+constexpr int kRowBatch = 8;                  // query rows staged per round
+
+// x = q.k, dp = g.v with q, g shared rows read by every lane (16-byte broadcasts) and k, v
+// this lane's padded rows; four independent partial sums each
+__device__ __forceinline__ void dot2_lane(const float *q, const float *g, const float *k, const float *v,
+                                          float &x, float &dp) {
+    float xa[4] = {0.f, 0.f, 0.f, 0.f}, pa[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < kD; e += 4) {
+        const float4 q4 = *reinterpret_cast<const float4 *>(q + e);
+        const float4 g4 = *reinterpret_cast<const float4 *>(g + e);
+        xa[0] = fmaf(q4.x, k[e], xa[0]);
+        xa[1] = fmaf(q4.y, k[e + 1], xa[1]);
+        xa[2] = fmaf(q4.z, k[e + 2], xa[2]);
+        xa[3] = fmaf(q4.w, k[e + 3], xa[3]);
+        pa[0] = fmaf(g4.x, v[e], pa[0]);
+        pa[1] = fmaf(g4.y, v[e + 1], pa[1]);
+        pa[2] = fmaf(g4.z, v[e + 2], pa[2]);
+        pa[3] = fmaf(g4.w, v[e + 3], pa[3]);
+    }
+    x = (xa[0] + xa[1]) + (xa[2] + xa[3]);
+    dp = (pa[0] + pa[1]) + (pa[2] + pa[3]);
+}
+
+// dv += a g, dk += b q (g, q shared rows, 16-byte broadcasts)
+__device__ __forceinline__ void axpy2(float a, const float *g, float b, const float *q, float *dv, float *dk) {
+#pragma unroll
+    for (int e = 0; e < kD; e += 4) {
+        const float4 g4 = *reinterpret_cast<const float4 *>(g + e);
+        const float4 q4 = *reinterpret_cast<const float4 *>(q + e);
+        dv[e] = fmaf(a, g4.x, dv[e]);
+        dv[e + 1] = fmaf(a, g4.y, dv[e + 1]);
+        dv[e + 2] = fmaf(a, g4.z, dv[e + 2]);
+        dv[e + 3] = fmaf(a, g4.w, dv[e + 3]);
+        dk[e] = fmaf(b, q4.x, dk[e]);
+        dk[e + 1] = fmaf(b, q4.y, dk[e + 1]);
+        dk[e + 2] = fmaf(b, q4.z, dk[e + 2]);
+        dk[e + 3] = fmaf(b, q4.w, dk[e + 3]);
+    }
+}
 
 // Window dK, dV: warp = 32 consecutive keys (lane = key j), over the queries i whose window
 // [i - w, i] holds some key of the block; dK_j = R_j^T sum_i dl_ij q'_i.  Every key is written.
@@ -258,7 +430,8 @@ __global__ void __launch_bounds__(kKvWarps * 32) bwd_window_kv_kernel(
     const float *__restrict__ qrot, const float *__restrict__ rowst, const float2 *__restrict__ lo,
     const float2 *__restrict__ hi, float *__restrict__ dK, float *__restrict__ dV) {
     __shared__ float s_k[kKvWarps][32][kPad], s_v[kKvWarps][32][kPad];
-    __shared__ float s_qi[kKvWarps][kD], s_gi[kKvWarps][kD];
+    __shared__ __align__(16) float s_qi[kKvWarps][kRowBatch][kD], s_gi[kKvWarps][kRowBatch][kD];
+    __shared__ float4 s_st[kKvWarps][kRowBatch];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.y;
     const int j0 = (blockIdx.x * kKvWarps + warp) * 32;
@@ -273,30 +446,31 @@ __global__ void __launch_bounds__(kKvWarps * 32) bwd_window_kv_kernel(
     float dk[kD], dv[kD];
 #pragma unroll
     for (int e = 0; e < kD; e++) { dk[e] = 0.f; dv[e] = 0.f; }
-    // queries at positions i in [j0, j0 + 31 + w] that exist
+    // queries at positions i in [j0, j0 + 31 + w] that exist, kRowBatch at a time
     const int ilo = max(j0, A.q0), ihi = min(j0 + 31 + A.w, A.q0 + A.Nq - 1);
-    for (int i = ilo; i <= ihi; i++) {
-        const size_t row = (size_t)bh * A.Nq + (i - A.q0);
+    for (int ib = ilo; ib <= ihi; ib += kRowBatch) {
+        const int nb = min(kRowBatch, ihi + 1 - ib);
         __syncwarp();
-        s_qi[warp][2 * lane] = qrot[row * kD + 2 * lane];
-        s_qi[warp][2 * lane + 1] = qrot[row * kD + 2 * lane + 1];
-        s_gi[warp][2 * lane] = to_f<T>(dO[row * kD + 2 * lane]);
-        s_gi[warp][2 * lane + 1] = to_f<T>(dO[row * kD + 2 * lane + 1]);
-        __syncwarp();
-        const float4 st = __ldg(reinterpret_cast<const float4 *>(rowst) + row);   // lse_sr, D_sr, ...
-        if (!kv_ok || j > i || j < i - A.w) continue;
-        float x = 0.f, dp = 0.f;
-#pragma unroll
-        for (int e = 0; e < kD; e++) {
-            x = fmaf(s_qi[warp][e], s_k[warp][lane][e], x);
-            dp = fmaf(s_gi[warp][e], s_v[warp][lane][e], dp);
+        for (int rr = 0; rr < nb; rr++) {
+            const size_t row = (size_t)bh * A.Nq + (ib + rr - A.q0);
+            const float2 q2 = *reinterpret_cast<const float2 *>(qrot + row * kD + 2 * lane);
+            s_qi[warp][rr][2 * lane] = q2.x;
+            s_qi[warp][rr][2 * lane + 1] = q2.y;
+            s_gi[warp][rr][2 * lane] = to_f<T>(dO[row * kD + 2 * lane]);
+            s_gi[warp][rr][2 * lane + 1] = to_f<T>(dO[row * kD + 2 * lane + 1]);
+            if (lane == 0) s_st[warp][rr] = __ldg(reinterpret_cast<const float4 *>(rowst) + row);
         }
-        const float pj = __expf(x * A.scale - st.x);
-        const float dl = pj * (dp - st.y) * A.scale;
-#pragma unroll
-        for (int e = 0; e < kD; e++) {
-            dv[e] = fmaf(pj, s_gi[warp][e], dv[e]);
-            dk[e] = fmaf(dl, s_qi[warp][e], dk[e]);
+        __syncwarp();
+        for (int rr = 0; rr < nb; rr++) {
+            const int i = ib + rr;
+            if (!kv_ok || j > i || j < i - A.w) continue;
+            const float *qi = s_qi[warp][rr], *gi = s_gi[warp][rr];
+            const float4 st = s_st[warp][rr];                // lse_sr, D_sr, ...
+            float x, dp;
+            dot2_lane(qi, gi, s_k[warp][lane], s_v[warp][lane], x, dp);
+            const float pj = __expf(x * A.scale - st.x);
+            const float dl = pj * (dp - st.y) * A.scale;
+            axpy2(pj, gi, dl, qi, dv, dk);
         }
     }
     if (!kv_ok) return;
@@ -369,7 +543,8 @@ __global__ void __launch_bounds__(kKvWarps * 32) bwd_readout_kv_kernel(
     const float *__restrict__ du, const float *__restrict__ rowst, const int *__restrict__ off,
     const int *__restrict__ list, float *__restrict__ dK, float *__restrict__ dV) {
     __shared__ float s_k[kKvWarps][32][kPad], s_v[kKvWarps][32][kPad];
-    __shared__ float s_qi[kKvWarps][kD], s_gi[kKvWarps][kD];
+    __shared__ __align__(16) float s_qi[kKvWarps][kRowBatch][kD], s_gi[kKvWarps][kRowBatch][kD];
+    __shared__ int s_row[kKvWarps][kRowBatch];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.y;
     const int c = blockIdx.x * kKvWarps + warp;
@@ -384,27 +559,27 @@ __global__ void __launch_bounds__(kKvWarps * 32) bwd_readout_kv_kernel(
     float dk[kD], dv[kD];
 #pragma unroll
     for (int e = 0; e < kD; e++) { dk[e] = 0.f; dv[e] = 0.f; }
-    for (int q = b0; q < b1; q++) {
-        const size_t row = (size_t)bh * A.Nq + list[q];
+    for (int qb = b0; qb < b1; qb += kRowBatch) {            // kRowBatch rows at a time
+        const int nb = min(kRowBatch, b1 - qb);
         __syncwarp();
-        s_qi[warp][2 * lane] = to_f<T>(Q[row * kD + 2 * lane]);
-        s_qi[warp][2 * lane + 1] = to_f<T>(Q[row * kD + 2 * lane + 1]);
-        s_gi[warp][2 * lane] = du[row * kD + 2 * lane];
-        s_gi[warp][2 * lane + 1] = du[row * kD + 2 * lane + 1];
-        __syncwarp();
-        const float4 st = __ldg(reinterpret_cast<const float4 *>(rowst) + row);   // ..., lse_lr, D_lr
-        float x = 0.f, dp = 0.f;
-#pragma unroll
-        for (int e = 0; e < kD; e++) {
-            x = fmaf(s_qi[warp][e], s_k[warp][lane][e], x);
-            dp = fmaf(s_gi[warp][e], s_v[warp][lane][e], dp);
+        for (int rr = 0; rr < nb; rr++) {
+            const size_t row = (size_t)bh * A.Nq + list[qb + rr];
+            const float2 d2 = *reinterpret_cast<const float2 *>(du + row * kD + 2 * lane);
+            s_qi[warp][rr][2 * lane] = to_f<T>(Q[row * kD + 2 * lane]);
+            s_qi[warp][rr][2 * lane + 1] = to_f<T>(Q[row * kD + 2 * lane + 1]);
+            s_gi[warp][rr][2 * lane] = d2.x;
+            s_gi[warp][rr][2 * lane + 1] = d2.y;
+            if (lane == 0) s_row[warp][rr] = (int)(row - (size_t)bh * A.Nq);
         }
-        const float pj = __expf(x * A.scale - st.z);
-        const float dl = pj * (dp - st.w) * A.scale;
-#pragma unroll
-        for (int e = 0; e < kD; e++) {
-            dv[e] = fmaf(pj, s_gi[warp][e], dv[e]);
-            dk[e] = fmaf(dl, s_qi[warp][e], dk[e]);
+        __syncwarp();
+        for (int rr = 0; rr < nb; rr++) {
+            const float *qi = s_qi[warp][rr], *gi = s_gi[warp][rr];
+            const float2 st = __ldg(reinterpret_cast<const float2 *>(rowst + ((size_t)bh * A.Nq + s_row[warp][rr]) * 4 + 2));
+            float x, dp;
+            dot2_lane(qi, gi, s_k[warp][lane], s_v[warp][lane], x, dp);
+            const float pj = __expf(x * A.scale - st.x);     // st = (lse_lr, D_lr)
+            const float dl = pj * (dp - st.y) * A.scale;
+            axpy2(pj, gi, dl, qi, dv, dk);
         }
     }
     float4 *dk4 = reinterpret_cast<float4 *>(dK + t * kD), *dv4 = reinterpret_cast<float4 *>(dV + t * kD);
@@ -463,8 +638,14 @@ fs_status run_backward(const fs_params *p, const T *Q, const T *K, const T *V, c
     }
     if (p->Nq > 0) {
         LaunchScope sc(kBwdRows, st);
-        bwd_rows_kernel<T><<<dim3((p->Nq + kRowWarps - 1) / kRowWarps, BH), kRowWarps * 32, 0, st>>>(
-            A, Q, K, V, idx, dO, krot, lo, hi, dQ, qrot, rowst, du, dal);
+        const int nwin = (p->Nq + 32 * kWinWarps - 1) / (32 * kWinWarps);
+        bwd_win_rows_kernel<T><<<dim3(nwin, BH), kWinWarps * 32, 0, st>>>(A, Q, V, dO, krot, lo, hi, dQ, qrot, rowst);
+        if (!ok()) return FS_ERR_CUDA;
+    }
+    if (p->Nq > 0) {
+        LaunchScope sc(kBwdLrRows, st);
+        bwd_lr_rows_kernel<T><<<dim3((p->Nq + kLrWarps - 1) / kLrWarps, BH), kLrWarps * 32, 0, st>>>(
+            A, Q, K, V, idx, dO, dQ, rowst, du, dal);
         if (!ok()) return FS_ERR_CUDA;
     }
     if (p->Nk > 0) {

@@ -104,7 +104,7 @@ enum KernelId : int {
     kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
     kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kRerank, kIdxTiles, kBwdRotate, kBwdRows,
     kBwdWindowKv, kBwdCells, kBwdReadoutKv, kBwdDalpha, kTreePrep, kTreeMerge, kTreeNodes, kTreeSearch,
-    kNumKernels
+    kBwdLrRows, kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.

@@ -33,9 +33,9 @@ const char *const kNames[kNumKernels] = {"cell_summaries", "exit_times", "select
                                          "readout", "window_combine", "rope_table",
                                          "window_tc", "attn_tc", "select_tc", "rope_keys",
                                          "cache_append", "cache_attend", "rerank", "idx_tiles",
-                                         "bwd_rotate", "bwd_rows", "bwd_window_kv", "bwd_cells",
+                                         "bwd_rotate", "bwd_win_rows", "bwd_window_kv", "bwd_cells",
                                          "bwd_readout_kv", "bwd_dalpha", "tree_prep", "tree_merge",
-                                         "tree_nodes", "tree_search"};
+                                         "tree_nodes", "tree_search", "bwd_lr_rows"};
 }  // namespace
 
 LaunchScope::LaunchScope(int id_, cudaStream_t st_) : id(id_), st(st_), slot(-1) {
