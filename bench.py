@@ -418,11 +418,12 @@ def time_rerank(fs, torch, inp, steps=5, warmup=3):
     fs.timing_enable(False)
     fs.sync_status(ws)
     ms = a.elapsed_time(b) / steps
-    rr = kt.get("rerank", (0, 0.0))[1] / steps
-    return {"value": wl.queries / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "rerank_ms": rr,
-            "note": "fs_forward_rerank: eq. (12) token-level rerank of all of A_i (CUDA cores), then "
-                    "the fused tensor-core readout + window on the reranked cells; per-kernel "
-                    "timing on (events around each launch)"}
+    split = {k: round(v[1] / steps, 4) for k, v in kt.items() if v[0]}
+    return {"value": wl.queries / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "kernel_ms": split,
+            "note": "fs_forward_rerank: eq. (12) token-level rerank of all of A_i on the tensor cores "
+                    "(rerank_tc, writing the fused kernel's tile records), then the fused tensor-core "
+                    "readout + window on the reranked cells; per-kernel timing on (events around "
+                    "each launch)"}
 
 
 def time_tree(fs, torch, inp, beam=32, steps=5, warmup=3):

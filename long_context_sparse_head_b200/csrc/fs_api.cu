@@ -214,6 +214,8 @@ extern "C" fs_status fs_select_topk_rerank(const fs_params *p, const void *Q, co
     if (!kbar || !amax) return FS_ERR_INVALID_ARG;
     int *exitn = at<int>(ws, L.exitn);
     if (D.prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
+    if (rerank_tc_supported(p, shortlist))        // bf16, all of A_i: the tensor-core kernel
+        return cuda_status(launch_rerank_tc(D, Q, K, amax, exitn, idx, nullptr, at<int>(ws, L.flag), st));
     return cuda_status(launch_rerank(D, p->dtype, Q, K, kbar, amax, exitn, shortlist, idx, st));
 }
 
@@ -246,6 +248,18 @@ extern "C" fs_status fs_forward_rerank(const fs_params *p, const void *Q, const 
     int *exitn = at<int>(ws, L.exitn);
     if (D.prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
     int32_t *sel = idx ? idx : at<int32_t>(ws, L.idx);
+    if (attn_tc_supported(p) && rerank_tc_supported(p, shortlist)) {
+        // bf16, all of A_i: the tensor-core rerank writes the fused kernel's tile records
+        uint32_t *tiles = at<uint32_t>(ws, L.tiles);
+        if (launch_rerank_tc(D, Q, K, amax, exitn, idx, tiles, at<int>(ws, L.flag), st) != cudaSuccess)
+            return FS_ERR_CUDA;
+        float2 *lo = at<float2>(ws, L.rope_abs), *hi = lo + kRopeLo * 32;
+        void *krot = at<void>(ws, L.krot);
+        if (launch_rope_abs_table(p->Nk, p->rope_base, lo, hi, st) != cudaSuccess ||
+            launch_rope_keys(D, K, krot, lo, hi, st) != cudaSuccess)
+            return FS_ERR_CUDA;
+        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), st));
+    }
     if (launch_rerank(D, p->dtype, Q, K, kbar, amax, exitn, shortlist, sel, st) != cudaSuccess) return FS_ERR_CUDA;
     if (attn_tc_supported(p)) {                    // bf16: the fused tensor-core readout + window
         uint32_t *tiles = at<uint32_t>(ws, L.tiles);

@@ -104,7 +104,7 @@ enum KernelId : int {
     kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
     kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kRerank, kIdxTiles, kBwdRotate, kBwdRows,
     kBwdWindowKv, kBwdCells, kBwdReadoutKv, kBwdDalpha, kTreePrep, kTreeMerge, kTreeNodes, kTreeSearch,
-    kBwdLrRows, kNumKernels
+    kBwdLrRows, kRerankTc, kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
@@ -129,6 +129,10 @@ cudaError_t launch_exit_times(const Dev &P, const float *amax, int *exitn, cudaS
 bool rerank_supported(const fs_params *p);
 cudaError_t launch_rerank(const Dev &P, fs_dtype dt, const void *Q, const void *K, const float *kbar,
                           const float *amax, const int *exitn, int shortlist, int32_t *idx, cudaStream_t st);
+// eq. (12) rerank on the tensor cores (bf16, all of A_i): idx and/or per-tile records
+bool rerank_tc_supported(const fs_params *p, int shortlist);
+cudaError_t launch_rerank_tc(const Dev &P, const void *Q, const void *K, const float *amax, const int *exitn,
+                             int32_t *idx, uint32_t *tiles, int *dev_flag, cudaStream_t st);
 // per-tile selection records (the fused kernel's input) from a selection idx
 cudaError_t launch_idx_tiles(const Dev &P, const int32_t *idx, uint32_t *tiles, int *dev_flag, cudaStream_t st);
 cudaError_t launch_select(const Dev &P, fs_dtype dt, const void *Q, const float *kbar,
