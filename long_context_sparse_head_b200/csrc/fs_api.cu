@@ -87,9 +87,11 @@ bool has_long_range(const fs_params *p) {
     return cand_count(p->Nk - 1, p->w, p->Nk / p->s) > 0;
 }
 
+// per_row_readout: the caller's idx differs across the rows of a group (FS-B), so the
+// readout runs one warp per row instead of staging each group's union of cells.
 fs_status run_forward(const fs_params *p, const void *Q, const void *K, const void *V,
                       const float *kbar, const float *amax, const int32_t *idx, void *O,
-                      void *ws, cudaStream_t st) {
+                      void *ws, cudaStream_t st, bool per_row_readout = false) {
     const Dev D = make_dev(p);
     const WsLayout L = layout(p);
     const float *olr = nullptr;
@@ -130,7 +132,9 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
             sel = wsidx;
         }
         float *o = at<float>(ws, L.olr);
-        if (launch_readout(D, p->dtype, Q, K, V, sel, o, st) != cudaSuccess) return FS_ERR_CUDA;
+        const cudaError_t e = per_row_readout ? launch_readout_rows(D, p->dtype, Q, K, V, sel, o, st)
+                                              : launch_readout(D, p->dtype, Q, K, V, sel, o, st);
+        if (e != cudaSuccess) return FS_ERR_CUDA;
         olr = o;
     }
     if (p->dtype == FS_BF16) {
@@ -341,7 +345,7 @@ extern "C" fs_status fs_forward_tree(const fs_params *p, const void *Q, const vo
     // FS-B rows of one query tile pick cells across the whole prefix (their union is not
     // bounded like FS-L's), so the readout gathers per row: the readout kernel on the
     // selection, then the tensor-core window + combine
-    return run_forward(p, Q, K, V, kb, am, sel, O, ws, st);
+    return run_forward(p, Q, K, V, kb, am, sel, O, ws, st, true);
 }
 
 extern "C" fs_status fs_forward(const fs_params *p, const void *Q, const void *K, const void *V,

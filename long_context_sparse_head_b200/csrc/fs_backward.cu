@@ -264,29 +264,6 @@ __global__ void __launch_bounds__(kWinWarps * 32) bwd_win_rows_kernel(
 // the readout part to dQ; writes du, (lse_lr, D_lr) and the dalpha terms.
 constexpr int kLrWarps = 4;
 
-template <typename T> __device__ __forceinline__ float2 ld_pair(const T *p);
-template <> __device__ __forceinline__ float2 ld_pair<float>(const float *p) {
-    return __ldg(reinterpret_cast<const float2 *>(p));
-}
-template <> __device__ __forceinline__ float2 ld_pair<__nv_bfloat16>(const __nv_bfloat16 *p) {
-    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
-}
-
-// lane t receives the sum over the warp of v[t]
-__device__ __forceinline__ float transpose_sum32(float (&v)[32], int lane) {
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        const bool up = lane & o;
-#pragma unroll
-        for (int k = 0; k < o; k++) {
-            const float send = up ? v[k] : v[k + o];
-            const float keep = up ? v[k + o] : v[k];
-            v[k] = keep + __shfl_xor_sync(kFull, send, o);
-        }
-    }
-    return v[0];
-}
-
 template <typename T>
 __global__ void __launch_bounds__(kLrWarps * 32) bwd_lr_rows_kernel(
     const BwdArgs A, const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V,

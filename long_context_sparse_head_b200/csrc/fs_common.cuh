@@ -93,6 +93,31 @@ template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
     return __bfloat162float(x);
 }
+
+// Two consecutive elements p[0], p[1] as floats (8- or 4-byte load).
+template <typename T> __device__ __forceinline__ float2 ld_pair(const T *p);
+template <> __device__ __forceinline__ float2 ld_pair<float>(const float *p) {
+    return __ldg(reinterpret_cast<const float2 *>(p));
+}
+template <> __device__ __forceinline__ float2 ld_pair<__nv_bfloat16>(const __nv_bfloat16 *p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+}
+
+// Transposed butterfly sum: lane t receives the sum over the warp of v[t] (31 shuffles for
+// 32 values per lane; each step keeps the half whose index bit matches the lane's bit).
+__device__ __forceinline__ float transpose_sum32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const bool up = lane & o;
+#pragma unroll
+        for (int k = 0; k < o; k++) {
+            const float send = up ? v[k] : v[k + o];
+            const float keep = up ? v[k + o] : v[k];
+            v[k] = keep + __shfl_xor_sync(kFull, send, o);
+        }
+    }
+    return v[0];
+}
 template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
@@ -104,7 +129,7 @@ enum KernelId : int {
     kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
     kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kRerank, kIdxTiles, kBwdRotate, kBwdRows,
     kBwdWindowKv, kBwdCells, kBwdReadoutKv, kBwdDalpha, kTreePrep, kTreeMerge, kTreeNodes, kTreeSearch,
-    kBwdLrRows, kRerankTc, kNumKernels
+    kBwdLrRows, kRerankTc, kReadoutRows, kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
@@ -139,6 +164,9 @@ cudaError_t launch_select(const Dev &P, fs_dtype dt, const void *Q, const float 
                           const float *amax, const int *exitn, int32_t *idx, cudaStream_t st);
 cudaError_t launch_readout(const Dev &P, fs_dtype dt, const void *Q, const void *K,
                            const void *V, const int32_t *idx, float *olr, cudaStream_t st);
+// the same, one warp per row (for selections that differ across a group's rows)
+cudaError_t launch_readout_rows(const Dev &P, fs_dtype dt, const void *Q, const void *K,
+                                const void *V, const int32_t *idx, float *olr, cudaStream_t st);
 cudaError_t launch_window(const Dev &P, fs_dtype dt, const void *Q, const void *K,
                           const void *V, const float *olr, void *O, cudaStream_t st);
 // tensor-core window (bf16): angle tables, then the kernel

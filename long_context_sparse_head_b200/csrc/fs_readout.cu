@@ -145,4 +145,78 @@ cudaError_t launch_readout(const Dev &P, fs_dtype dt, const void *Q, const void 
     return cudaGetLastError();
 }
 
+// Per-row variant, for selections that differ across the rows of a group (the FS-B
+// search picks cells anywhere in the prefix, so a group's union is large and each staged
+// cell serves few rows).  One warp per query row, lane m holding dimensions (2m, 2m+1): a
+// cell's 32 logits come from per-lane partial products and a transposed butterfly sum
+// (lane t: token t), then an online softmax over the row's cells; no shared memory.
+namespace {
+constexpr int kRowsPerBlock = 4;
+
+template <typename T>
+__global__ void __launch_bounds__(kRowsPerBlock * 32) readout_rows_kernel(Dev P, const T *__restrict__ Q,
+                                                                         const T *__restrict__ K,
+                                                                         const T *__restrict__ V,
+                                                                         const int32_t *__restrict__ idx,
+                                                                         float *__restrict__ olr) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y, h = bh % P.H;
+    const int r = blockIdx.x * kRowsPerBlock + warp;
+    if (r >= P.Nq) return;                                   // warp-uniform
+    const size_t row = (size_t)bh * P.Nq + r;
+    const size_t kb = (size_t)bh * P.Nk;
+    const float2 q = ld_pair<T>(Q + row * kD + 2 * lane);
+    float m = -INFINITY, l = 0.f, u0 = 0.f, u1 = 0.f;
+    for (int e = 0; e < P.K; e++) {
+        const int c = idx[row * P.K + e];
+        if ((unsigned)c >= (unsigned)P.C) continue;           // -1 padding, out-of-range cells
+        const T *kc = K + (kb + (size_t)c * kS) * kD + 2 * lane;
+        const T *vc = V + (kb + (size_t)c * kS) * kD + 2 * lane;
+        float v[32];
+#pragma unroll
+        for (int t = 0; t < 32; t++) {
+            const float2 k2 = ld_pair<T>(kc + t * kD);
+            v[t] = fmaf(q.x, k2.x, q.y * k2.y);
+        }
+        const float x = transpose_sum32(v, lane) * P.scale;  // lane t: token t's logit
+        const float mn = fmaxf(m, warp_max(x));
+        const float corr = __expf(m - mn);                    // 0 while m is -inf
+        const float p = __expf(x - mn);
+        l = l * corr + warp_sum(p);
+        u0 *= corr;
+        u1 *= corr;
+#pragma unroll
+        for (int t = 0; t < 32; t++) {
+            const float pt = __shfl_sync(kFull, p, t);
+            const float2 v2 = ld_pair<T>(vc + t * kD);
+            u0 = fmaf(pt, v2.x, u0);
+            u1 = fmaf(pt, v2.y, u1);
+        }
+        m = mn;
+    }
+    float o0 = 0.f, o1 = 0.f;
+    if (l > 0.f) {
+        const float y0 = u0 / l, y1 = u1 / l;
+        const float inv = rsqrtf(warp_sum(y0 * y0 + y1 * y1) * (1.f / kD) + P.rms_eps);
+        o0 = P.alpha[h] * y0 * inv;
+        o1 = P.alpha[h] * y1 * inv;
+    }
+    *reinterpret_cast<float2 *>(&olr[row * kD + 2 * lane]) = make_float2(o0, o1);
+}
+}  // namespace
+
+cudaError_t launch_readout_rows(const Dev &P, fs_dtype dt, const void *Q, const void *K,
+                                const void *V, const int32_t *idx, float *olr, cudaStream_t st) {
+    if (P.Nq == 0) return cudaSuccess;
+    const dim3 grid((P.Nq + kRowsPerBlock - 1) / kRowsPerBlock, P.B * P.H);
+    LaunchScope scope(kReadoutRows, st);
+    if (dt == FS_BF16)
+        readout_rows_kernel<__nv_bfloat16><<<grid, kRowsPerBlock * 32, 0, st>>>(
+            P, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, idx, olr);
+    else
+        readout_rows_kernel<float><<<grid, kRowsPerBlock * 32, 0, st>>>(P, (const float *)Q, (const float *)K,
+                                                                        (const float *)V, idx, olr);
+    return cudaGetLastError();
+}
+
 }  // namespace fs
