@@ -87,6 +87,32 @@ bool has_long_range(const fs_params *p) {
     return cand_count(p->Nk - 1, p->w, p->Nk / p->s) > 0;
 }
 
+// A second stream forked from `st` for launches independent of the chain on `st`, joined
+// back before the first launch that needs them.  The stream and events are released on
+// destruction (the runtime defers that until the enqueued work completes).  If it cannot
+// be opened, the launches go to `st` in order.
+struct Fork {
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    cudaStream_t open(cudaStream_t st) {
+        if (cudaStreamCreateWithFlags(&side, cudaStreamNonBlocking) != cudaSuccess) side = nullptr;
+        if (side && cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&join, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventRecord(fork, st) == cudaSuccess && cudaStreamWaitEvent(side, fork, 0) == cudaSuccess)
+            return side;
+        return st;
+    }
+    bool close(cudaStream_t st, cudaStream_t used) {
+        if (used == st) return true;
+        return cudaEventRecord(join, side) == cudaSuccess && cudaStreamWaitEvent(st, join, 0) == cudaSuccess;
+    }
+    ~Fork() {
+        if (fork) cudaEventDestroy(fork);
+        if (join) cudaEventDestroy(join);
+        if (side) cudaStreamDestroy(side);
+    }
+};
+
 // per_row_readout: the caller's idx differs across the rows of a group (FS-B), so the
 // readout runs one warp per row instead of staging each group's union of cells.
 fs_status run_forward(const fs_params *p, const void *Q, const void *K, const void *V,
@@ -97,6 +123,15 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
     const float *olr = nullptr;
     const bool fused = has_long_range(p) && !idx && attn_tc_supported(p) && select_tc_supported(p);
     if (fused) {   // bf16: selection, then one tensor-core kernel for readout + window + combine
+        // the RoPE tables and the rotated keys depend on K only: they run beside the
+        // summaries -> exit times -> selection chain
+        Fork fk;
+        const cudaStream_t rs = fk.open(st);
+        float2 *lo = at<float2>(ws, L.rope_abs), *hi = lo + kRopeLo * 32;
+        void *krot = at<void>(ws, L.krot);
+        if (launch_rope_abs_table(p->Nk, p->rope_base, lo, hi, rs) != cudaSuccess ||
+            launch_rope_keys(D, K, krot, lo, hi, rs) != cudaSuccess)
+            return FS_ERR_CUDA;
         if (!kbar) {
             float *kb = at<float>(ws, L.kbar), *am = at<float>(ws, L.amax);
             if (launch_summaries(D, p->dtype, K, kb, am, st) != cudaSuccess) return FS_ERR_CUDA;
@@ -108,11 +143,7 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
         uint32_t *tiles = at<uint32_t>(ws, L.tiles);
         if (launch_select_tc(D, Q, kbar, amax, exitn, nullptr, tiles, at<int>(ws, L.flag), st) != cudaSuccess)
             return FS_ERR_CUDA;
-        float2 *lo = at<float2>(ws, L.rope_abs), *hi = lo + kRopeLo * 32;
-        void *krot = at<void>(ws, L.krot);
-        if (launch_rope_abs_table(p->Nk, p->rope_base, lo, hi, st) != cudaSuccess ||
-            launch_rope_keys(D, K, krot, lo, hi, st) != cudaSuccess)
-            return FS_ERR_CUDA;
+        if (!fk.close(st, rs)) return FS_ERR_CUDA;
         return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), st));
     }
     if (has_long_range(p)) {
