@@ -88,28 +88,39 @@ bool has_long_range(const fs_params *p) {
 }
 
 // A second stream forked from `st` for launches independent of the chain on `st`, joined
-// back before the first launch that needs them.  The stream and events are released on
-// destruction (the runtime defers that until the enqueued work completes).  If it cannot
-// be opened, the launches go to `st` in order.
-struct Fork {
+// back before the first launch that needs them.  The side stream and its two events are
+// created once per host thread and device and kept (creating them per call costs more
+// host time than a short step runs on the GPU); being per thread, two threads that call
+// the library concurrently never share them.  If they cannot be created, the launches go
+// to `st` in order.
+struct ForkRes {
     cudaStream_t side = nullptr;
     cudaEvent_t fork = nullptr, join = nullptr;
+    bool ok = false, tried = false;
+};
+constexpr int kForkDevices = 64;
+thread_local ForkRes tl_fork[kForkDevices];
+
+struct Fork {
+    ForkRes *r = nullptr;
     cudaStream_t open(cudaStream_t st) {
-        if (cudaStreamCreateWithFlags(&side, cudaStreamNonBlocking) != cudaSuccess) side = nullptr;
-        if (side && cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) == cudaSuccess &&
-            cudaEventCreateWithFlags(&join, cudaEventDisableTiming) == cudaSuccess &&
-            cudaEventRecord(fork, st) == cudaSuccess && cudaStreamWaitEvent(side, fork, 0) == cudaSuccess)
-            return side;
-        return st;
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kForkDevices) return st;
+        ForkRes &x = tl_fork[dev];
+        if (!x.tried) {
+            x.tried = true;
+            x.ok = cudaStreamCreateWithFlags(&x.side, cudaStreamNonBlocking) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) == cudaSuccess;
+        }
+        if (!x.ok || cudaEventRecord(x.fork, st) != cudaSuccess || cudaStreamWaitEvent(x.side, x.fork, 0) != cudaSuccess)
+            return st;
+        r = &x;
+        return x.side;
     }
     bool close(cudaStream_t st, cudaStream_t used) {
-        if (used == st) return true;
-        return cudaEventRecord(join, side) == cudaSuccess && cudaStreamWaitEvent(st, join, 0) == cudaSuccess;
-    }
-    ~Fork() {
-        if (fork) cudaEventDestroy(fork);
-        if (join) cudaEventDestroy(join);
-        if (side) cudaStreamDestroy(side);
+        if (used == st || !r) return true;
+        return cudaEventRecord(r->join, r->side) == cudaSuccess && cudaStreamWaitEvent(st, r->join, 0) == cudaSuccess;
     }
 };
 
