@@ -71,6 +71,7 @@ WsLayout layout(const fs_params *p) {
     L.rope_abs = off; off += align256((size_t)(kRopeLo + rope_hi_rows(p->Nk)) * 32 * 8);
     const int kr0 = p->Nk - p->Nq - p->w > 0 ? p->Nk - p->Nq - p->w : 0;   // first rotated key
     L.krot = off;  off += align256(BH * (size_t)(p->Nk - kr0) * kD * 2);
+    L.part = off;  off += align256(attn_part_bytes(p));      // split CTAs' partial states (decoding)
     L.total = off;
     return L;
 }
@@ -155,7 +156,8 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
         if (launch_select_tc(D, Q, kbar, amax, exitn, nullptr, tiles, at<int>(ws, L.flag), st) != cudaSuccess)
             return FS_ERR_CUDA;
         if (!fk.close(st, rs)) return FS_ERR_CUDA;
-        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), st));
+        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), at<float>(ws, L.part),
+                                          attn_splits(p), st));
     }
     if (has_long_range(p)) {
         const int32_t *sel = idx;
@@ -304,7 +306,8 @@ extern "C" fs_status fs_forward_rerank(const fs_params *p, const void *Q, const 
         if (launch_rope_abs_table(p->Nk, p->rope_base, lo, hi, st) != cudaSuccess ||
             launch_rope_keys(D, K, krot, lo, hi, st) != cudaSuccess)
             return FS_ERR_CUDA;
-        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), st));
+        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), at<float>(ws, L.part),
+                                          attn_splits(p), st));
     }
     if (launch_rerank(D, p->dtype, Q, K, kbar, amax, exitn, shortlist, sel, st) != cudaSuccess) return FS_ERR_CUDA;
     if (attn_tc_supported(p)) {                    // bf16: the fused tensor-core readout + window
@@ -315,7 +318,8 @@ extern "C" fs_status fs_forward_rerank(const fs_params *p, const void *Q, const 
         if (launch_rope_abs_table(p->Nk, p->rope_base, lo, hi, st) != cudaSuccess ||
             launch_rope_keys(D, K, krot, lo, hi, st) != cudaSuccess)
             return FS_ERR_CUDA;
-        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), st));
+        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), at<float>(ws, L.part),
+                                          attn_splits(p), st));
     }
     return run_forward(p, Q, K, V, kbar, amax, sel, O, ws, st);
 }

@@ -24,6 +24,8 @@
 // Warpgroup 1 (lowered to 56): warp 4 TMA, warp 5 MMA, warps 6-7 auxiliary (stage U,
 // rotate Q by its absolute positions).  The window's keys come pre-rotated (absolute
 // positions, double-precision angles) from a workspace copy.
+#include <algorithm>
+
 #include "tc_rope.cuh"
 
 namespace fs {
@@ -60,8 +62,14 @@ struct AttnArgs {
     int kr0;                // first key of the rotated copy
     float scale_log2e;      // log2(e) / sqrt(d)
     float rms_eps;
+    int nsplit;             // CTAs per tile (gridDim.z); > 1: partial states to `part`
+    float *part;
     float alpha[FS_MAX_HEADS];
 };
+
+// A split CTA's partial state per row: m, l (log2 units) of the readout and the window,
+// then the readout's and the window's unnormalised O (64 floats each).
+constexpr int kPartStride = 4 + 2 * kD;
 
 __device__ __forceinline__ void aux_sync() {
     asm volatile("bar.sync %0, %1;" ::"n"(kAuxBarrier), "n"(NAUX) : "memory");
@@ -138,6 +146,7 @@ __device__ __forceinline__ float softmax_chunk(uint32_t tS, int kind, uint32_t s
 }
 }  // namespace
 
+template <bool SPLIT>
 __global__ void __launch_bounds__(NTHREADS, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk32,
                const __grid_constant__ CUtensorMap tv32, const __grid_constant__ CUtensorMap tkr64,
@@ -156,6 +165,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     const int last = pb + nrows - 1;
     const int k_first = jbase < 0 ? (-jbase) / BN : 0;
     const int nW = (last - jbase) / BN - k_first + 1;    // window chunks
+    // with nsplit > 1 this CTA takes the contiguous range [cb, ce) of the tile's chunk list
+    // (readout chunks 0 .. nR-1, then window chunks nR .. nR+nW-1)
+    const int S = SPLIT ? A.nsplit : 1, sidx = SPLIT ? (int)blockIdx.z : 0;
+    auto chunk_range = [&](int nR, int &cb, int &ce) {
+        const int T = nR + nW;
+        cb = (int)((long long)T * sidx / S);
+        ce = (int)((long long)T * (sidx + 1) / S);
+    };
     const tc::Abort ab{dev_flag, &sm.abort};
 
     if (threadIdx.x == 0) {
@@ -198,20 +215,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 tc::tma_load_3d(sm.qn, &tq, &sm.q_full, 0, r0, bh);
                 int it = 0;
                 if (tc::mbar_wait(&sm.u_ready, 0, ab)) {
-                    const int nU = sm.nU, nR = (nU + CPC - 1) / CPC, total = nR + nW;
+                    const int nU = sm.nU, nR = (nU + CPC - 1) / CPC;
+                    int cb, ce;
+                    chunk_range(nR, cb, ce);
+                    const int total = ce - cb;
                     for (; it < total; it++) {
-                        const int s = it % NSTAGE;
+                        const int s = it % NSTAGE, g = cb + it;
                         if (!tc::mbar_wait(&sm.kv_empty[s], ((it / NSTAGE) & 1) ^ 1, ab)) break;
-                        if (it < nR) {          // two gathered cells; unused slots read zeros
+                        if (g < nR) {           // two gathered cells; unused slots read zeros
                             tc::mbar_expect_tx(&sm.kv_full[s], 2 * CPC * CELL_BYTES);
                             for (int j = 0; j < CPC; j++) {
-                                const int u = CPC * it + j;
+                                const int u = CPC * g + j;
                                 const int y = u < nU ? sm.ulist[u] * kS : A.Nk;   // past the end: zeros
                                 tc::tma_load_3d(sm.k[s] + j * kS * kD, &tk32, &sm.kv_full[s], 0, y, bh);
                                 tc::tma_load_3d(sm.v[s] + j * kS * kD, &tv32, &sm.kv_full[s], 0, y, bh);
                             }
                         } else {                // BN consecutive keys of the band (K pre-rotated)
-                            const int jc = jbase + BN * (k_first + it - nR);
+                            const int jc = jbase + BN * (k_first + g - nR);
                             tc::mbar_expect_tx(&sm.kv_full[s], 2 * CHUNK_BYTES);
                             tc::tma_load_3d(sm.k[s], &tkr64, &sm.kv_full[s], 0, jc - A.kr0, bh);
                             tc::tma_load_3d(sm.v[s], &tv64, &sm.kv_full[s], 0, jc, bh);
@@ -262,14 +282,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 const uint64_t dv0 = tc::sdesc_sw128(tc::smem_u32(sm.v[0]), 16, 1024);
                 constexpr uint32_t kStageStep = (BN * kD * 2) >> 4;
                 bool ok = tc::mbar_wait(&sm.u_ready, 0, ab) && tc::mbar_wait(&sm.q_full, 0, ab);
-                const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0, total = nR + nW;
+                const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0;
+                int cb = 0, ce = 0;
+                if (ok) chunk_range(nR, cb, ce);
+                const int total = ce - cb;
                 int issued = 0;
                 // S(c) = Q K(c)^T into buffer c mod 2, with the NoPE or the rotated Q
                 auto issue_qk = [&](int c) -> bool {
                     if (!tc::mbar_wait(&sm.kv_full[c % NSTAGE], (c / NSTAGE) & 1, ab)) return false;
-                    if (c == nR && !tc::mbar_wait(&sm.q_ready, 0, ab)) return false;
+                    const int g = cb + c;
+                    if (g >= nR && (g == nR || c == 0) && !tc::mbar_wait(&sm.q_ready, 0, ab)) return false;
                     tc::tc_fence_after();
-                    const uint64_t da = c < nR ? dqn : dqr;
+                    const uint64_t da = g < nR ? dqn : dqr;
                     const uint64_t db = dk0 + (uint64_t)((c % NSTAGE) * kStageStep);
 #pragma unroll
                     for (int kk = 0; kk < kD / 16; kk++)      // K steps of 16 columns = 32 bytes
@@ -286,8 +310,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     // O += P(c) V(c), into the readout's or the window's O
                     if (!tc::mbar_wait(&sm.p_full[c & 1], (c >> 1) & 1, ab)) { ok = false; break; }
                     tc::tc_fence_after();
-                    const uint32_t ocol = c < nR ? OLR_COL : OSR_COL;
-                    const bool first = c == 0 || c == nR;
+                    const uint32_t ocol = cb + c < nR ? OLR_COL : OSR_COL;
+                    const bool first = c == 0 || cb + c == nR;
                     const uint64_t db = dv0 + (uint64_t)((c % NSTAGE) * kStageStep);
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; kk++)      // K steps of 16 keys = 2048 bytes
@@ -316,12 +340,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         const uint4 m4 = __ldg(reinterpret_cast<const uint4 *>(
             tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords + kTileMaskOff + 4 * row));
         bool ok = tc::mbar_wait(&sm.u_ready, 0, ab);
-        const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0, total = nR + nW;
+        const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0;
+        int cb = 0, ce = 0;
+        if (ok) chunk_range(nR, cb, ce);
+        const int total = ce - cb;
         float m_lr = -INFINITY, l_lr = 0.f, m_sr = -INFINITY, l_sr = 0.f;
         for (int it = 0; ok && it < total; it++) {
+            const int g = cb + it;
             if (!tc::mbar_wait(&sm.s_full[it & 1], (it >> 1) & 1, ab)) { ok = false; break; }
             tc::tc_fence_after();
-            if (it == nR && nR > 0) {   // readout done: O_lr <- alpha_h RMSNorm(O_lr / l)
+            if (!SPLIT && g == nR && nR > 0) {   // readout done: O_lr <- alpha_h RMSNorm(O_lr / l)
                 // the last readout P V may still run (S of this chunk was issued before it)
                 if (!tc::mbar_wait(&sm.o_ready, (it - 1) & 1, ab)) { ok = false; break; }
                 tc::tc_fence_after();
@@ -350,22 +378,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             uint32_t sel = 0u, ocol;
             bool first;
             float m, l;
-            if (it < nR) {
-                const int p0 = CPC * it;
+            if (g < nR) {
+                const int p0 = CPC * g;
                 const int wsel = p0 >> 5;           // word of the row's union mask, in registers
                 const uint32_t mw = wsel == 0 ? m4.x : wsel == 1 ? m4.y : wsel == 2 ? m4.z : m4.w;
                 sel = (mw >> (p0 & 31)) & ((1u << CPC) - 1u);
                 kind = CELLS; ocol = OLR_COL; first = it == 0; m = m_lr; l = l_lr;
             } else {
-                const int jc = jbase + BN * (k_first + it - nR);
+                const int jc = jbase + BN * (k_first + g - nR);
                 const int clo = max(-jc, i - A.w - jc), chi = min(i - jc, BN - 1);
                 lo = clo;
                 width = rvalid ? max(0, chi - clo + 1) : 0;
                 kind = __all_sync(kFull, clo <= 0 && chi >= BN - 1 && rvalid) ? FULL : BAND;
-                ocol = OSR_COL; first = it == nR; m = m_sr; l = l_sr;
+                ocol = OSR_COL; first = g == nR || it == 0; m = m_sr; l = l_sr;
             }
             const float corr = softmax_chunk(trow + BN * (it & 1), kind, sel, lo, width, A.scale_log2e, m, l);
-            if (it < nR) { m_lr = m; l_lr = l; } else { m_sr = m; l_sr = l; }
+            if (g < nR) { m_lr = m; l_lr = l; } else { m_sr = m; l_sr = l; }
             // O rescale, after the exponentials (S no longer occupies registers); the P V of
             // the previous chunk, which accumulates into the same O, must have finished
             if (!first && __any_sync(kFull, corr != 1.f)) {
@@ -386,7 +414,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.p_full[it & 1]);
         }
-        if (ok && tc::mbar_wait(&sm.o_done, 0, ab)) {
+        if (SPLIT && ok && tc::mbar_wait(&sm.o_done, 0, ab)) {
+            // partial state of this CTA's chunks; a branch it had no chunk of stays empty
+            tc::tc_fence_after();
+            const bool had_lr = cb < nR && ce > cb, had_sr = ce > nR && ce > cb;
+            float *dst = A.part + ((((size_t)bh * gridDim.x + blockIdx.x) * S + sidx) * BM + row) * kPartStride;
+            *reinterpret_cast<float4 *>(dst) = make_float4(had_lr ? m_lr : -INFINITY, had_lr ? l_lr : 0.f,
+                                                           had_sr ? m_sr : -INFINITY, had_sr ? l_sr : 0.f);
+#pragma unroll
+            for (int br = 0; br < 2; br++) {
+                const bool had = br == 0 ? had_lr : had_sr;
+                uint32_t a[64];
+                tc::tmem_ld32(trow + (br == 0 ? OLR_COL : OSR_COL), *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+                tc::tmem_ld32(trow + (br == 0 ? OLR_COL : OSR_COL) + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+                tc::tmem_wait_ld();
+                float4 *d4 = reinterpret_cast<float4 *>(dst + 4 + br * kD);
+#pragma unroll
+                for (int q = 0; q < kD / 4; q++)
+                    d4[q] = had ? make_float4(__uint_as_float(a[4 * q]), __uint_as_float(a[4 * q + 1]),
+                                              __uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3]))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        } else if (!SPLIT && ok && tc::mbar_wait(&sm.o_done, 0, ab)) {
             tc::tc_fence_after();
             const float inv = l_sr > 0.f ? 1.f / l_sr : 0.f;
             uint32_t a[64], b[64];
@@ -426,6 +475,68 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     }
 }
 
+namespace {
+// Combination of split CTAs' partial states (decoding shapes): per row, the readout's
+// partials merge into u (rescaled to the largest max), RMSNorm gives alpha_h o^lr; the
+// window's merge into o^sr; O = o^sr + alpha_h o^lr (eq. (2)).  One warp per row, lane m
+// holding dimensions (2m, 2m+1).
+constexpr int kCombWarps = 4;
+__global__ void __launch_bounds__(kCombWarps * 32) attn_combine_kernel(const AttnArgs A, int ntiles,
+                                                                       __nv_bfloat16 *__restrict__ O) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y, h = bh % A.H;
+    const int r = blockIdx.x * kCombWarps + warp;
+    if (r >= A.Nq) return;
+    const int tile = r / BM, row = r % BM, S = A.nsplit;      // S <= 8
+    const float *base = A.part + (((size_t)bh * ntiles + tile) * S * BM + row) * kPartStride;
+    // lanes 0..S-1 hold the splits' (m, l) pairs; every lane then loads its two
+    // dimensions of each split's O at once
+    float4 st = make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+    if (lane < S) st = *reinterpret_cast<const float4 *>(base + (size_t)lane * BM * kPartStride);
+    const float M_lr = warp_max(st.x), M_sr = warp_max(st.z);
+    const float w_lr = st.y > 0.f ? exp2f(st.x - M_lr) : 0.f, w_sr = st.w > 0.f ? exp2f(st.z - M_sr) : 0.f;
+    const float L_lr = warp_sum(st.y * w_lr), L_sr = warp_sum(st.w * w_sr);
+    float u0 = 0.f, u1 = 0.f, o0 = 0.f, o1 = 0.f;
+#pragma unroll
+    for (int s = 0; s < 8; s++) {
+        if (s >= S) break;
+        const float wl = __shfl_sync(kFull, w_lr, s), ws = __shfl_sync(kFull, w_sr, s);
+        const float *p = base + (size_t)s * BM * kPartStride;
+        const float2 x = *reinterpret_cast<const float2 *>(p + 4 + 2 * lane);
+        const float2 z = *reinterpret_cast<const float2 *>(p + 4 + kD + 2 * lane);
+        u0 = fmaf(x.x, wl, u0);
+        u1 = fmaf(x.y, wl, u1);
+        o0 = fmaf(z.x, ws, o0);
+        o1 = fmaf(z.y, ws, o1);
+    }
+    float y0 = 0.f, y1 = 0.f;
+    if (L_lr > 0.f) {
+        u0 /= L_lr;
+        u1 /= L_lr;
+        const float f = A.alpha[h] * rsqrtf(warp_sum(u0 * u0 + u1 * u1) * (1.f / kD) + A.rms_eps);
+        y0 = u0 * f;
+        y1 = u1 * f;
+    }
+    const float inv = L_sr > 0.f ? 1.f / L_sr : 0.f;
+    *reinterpret_cast<uint32_t *>(O + ((size_t)bh * A.Nq + r) * kD + 2 * lane) =
+        tc::pack_bf16x2(o0 * inv + y0, o1 * inv + y1);
+}
+}  // namespace
+
+// CTAs per 128-row tile: 1 when the tiles fill the GPU; otherwise the tile's chunk list is
+// split over up to 8 CTAs (about two CTAs per SM in all) and combined afterwards.
+int attn_splits(const fs_params *p) {
+    const long long tiles = (long long)p->B * p->H * ((p->Nq + BM - 1) / BM);
+    if (tiles <= 0 || tiles >= 148) return 1;
+    return (int)std::min<long long>(8, std::max<long long>(1, (2 * 148) / tiles));
+}
+
+size_t attn_part_bytes(const fs_params *p) {
+    const int S = attn_splits(p);
+    if (S <= 1) return 0;
+    return (size_t)p->B * p->H * ((p->Nq + BM - 1) / BM) * S * BM * kPartStride * 4;
+}
+
 bool attn_tc_supported(const fs_params *p) {
     const int C = p->Nk / p->s;
     if (p->dtype != FS_BF16 || C > 32768) return false;
@@ -435,7 +546,7 @@ bool attn_tc_supported(const fs_params *p) {
 
 cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V, const void *Krot,
                            const uint32_t *tiles, void *O, const float2 *rope_lo, const float2 *rope_hi,
-                           int *dev_flag, cudaStream_t st) {
+                           int *dev_flag, float *part, int nsplit, cudaStream_t st) {
     if (P.Nq == 0) return cudaSuccess;
     const int BH = P.B * P.H;
     const int kr0 = rope_first_key(P);
@@ -452,12 +563,24 @@ cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const voi
     A.scale_log2e = P.scale * 1.4426950408889634f;
     A.rms_eps = P.rms_eps;
     for (int hh = 0; hh < FS_MAX_HEADS; hh++) A.alpha[hh] = P.alpha[hh];
+    A.nsplit = part && nsplit > 1 ? nsplit : 1;
+    A.part = part;
     const size_t smem = sizeof(AttnSmem) + 1024;
-    const dim3 grid((P.Nq + BM - 1) / BM, BH);
-    LaunchScope scope(kAttnTc, st);
-    cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_tc_kernel<<<grid, NTHREADS, smem, st>>>(tq, tk32, tv32, tkr64, tv64, A, tiles, rope_lo, rope_hi,
-                                                 (__nv_bfloat16 *)O, dev_flag);
+    const int ntiles = (P.Nq + BM - 1) / BM;
+    const dim3 grid(ntiles, BH, A.nsplit);
+    {
+        LaunchScope scope(kAttnTc, st);
+        auto kern = A.nsplit > 1 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kern<<<grid, NTHREADS, smem, st>>>(tq, tk32, tv32, tkr64, tv64, A, tiles, rope_lo, rope_hi,
+                                           (__nv_bfloat16 *)O, dev_flag);
+        if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
+    }
+    if (A.nsplit > 1) {
+        LaunchScope scope(kAttnCombine, st);
+        attn_combine_kernel<<<dim3((P.Nq + kCombWarps - 1) / kCombWarps, BH), kCombWarps * 32, 0, st>>>(
+            A, ntiles, (__nv_bfloat16 *)O);
+    }
     return cudaGetLastError();
 }
 

@@ -35,7 +35,7 @@ struct Dev {
 
 // Workspace layout (byte offsets from ws; each segment 256-byte aligned).
 struct WsLayout {
-    size_t flag, exitn, kbar, amax, idx, olr, rope, tiles, rope_abs, krot, total;
+    size_t flag, exitn, kbar, amax, idx, olr, rope, tiles, rope_abs, krot, part, total;
 };
 
 // Per-tile selection record passed from the tensor-core selection kernel to the fused
@@ -129,7 +129,7 @@ enum KernelId : int {
     kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
     kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kRerank, kIdxTiles, kBwdRotate, kBwdRows,
     kBwdWindowKv, kBwdCells, kBwdReadoutKv, kBwdDalpha, kTreePrep, kTreeMerge, kTreeNodes, kTreeSearch,
-    kBwdLrRows, kRerankTc, kReadoutRows, kNumKernels
+    kBwdLrRows, kRerankTc, kReadoutRows, kAttnCombine, kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
@@ -197,8 +197,12 @@ cudaError_t launch_tree_search(const fs_params *p, const Dev &D, const void *Q, 
                                float c_explore, int32_t *idx, int *dev_flag, cudaStream_t st);
 // fused tensor-core readout + window + combine (bf16, internally selected cells)
 bool attn_tc_supported(const fs_params *p);
+// decoding shapes (fewer tiles than SMs): the tile's chunks split over nsplit CTAs whose
+// partial states (part, attn_part_bytes) are combined by a second kernel
+int attn_splits(const fs_params *p);
+size_t attn_part_bytes(const fs_params *p);
 cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V, const void *Krot,
                            const uint32_t *tiles, void *O, const float2 *rope_lo, const float2 *rope_hi,
-                           int *dev_flag, cudaStream_t st);
+                           int *dev_flag, float *part, int nsplit, cudaStream_t st);
 
 }  // namespace fs

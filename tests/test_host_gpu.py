@@ -1,7 +1,9 @@
 """fs_forward_host: the forward pass on host buffers, pipelined over chunks of heads on
-internal streams.  Its output must equal fs_forward's on device copies of the same inputs
-bit for bit (every head is computed by the same kernels either way), and the oracle's on
-sampled rows."""
+internal streams.  In fp32 (no fused kernel) its output must equal fs_forward's on device
+copies of the same inputs bit for bit.  In bf16 a chunk is a smaller call, so the fused
+kernel may split its tiles over a different number of CTAs: each split rounds its P to
+bf16 against its own running maximum, so the two agree within the bf16 output tolerance,
+not bit for bit.  Both must match the oracle on sampled rows."""
 import numpy as np
 import pytest
 import torch
@@ -39,7 +41,10 @@ def test_forward_host_matches_device(dtype, case):
         fs.forward_host(g.p, hQ, hK, hV, hO, scratch, stream)
     stream.synchronize()
     got = hO.float().numpy()
-    assert np.array_equal(got, ref)
+    if wl.dtype == "f32":
+        assert np.array_equal(got, ref)
+    else:
+        assert np.abs(got - ref).max() <= TOL["bf16"], np.abs(got - ref).max()
     prob = oracle_for(inp)
     rows = sample_rows(wl, 24, seed=3)
     idx = g.numpy(g.select())
