@@ -21,9 +21,12 @@
 // TopP if it beats the weakest member (the weakest leaves at that prefix), and it takes a
 // slot if some reachable prefix can admit it.  Keys, values and mean keys are copied into
 // the slots last, in parallel.
-// fs_cache_attend: one CTA per (query, b, h): admission and scores over the slots, top-K,
-// NoPE readout over the selected cells' tokens, RMSNorm, RoPE window over the ring,
-// combination.  CUDA cores: a decode step has a handful of queries per head.
+// fs_cache_attend: kAttendParts CTAs per (query, b, h) (a decode step has a handful of
+// queries per head, so the work of one is spread over several CTAs): part 0 runs the RoPE
+// window over the ring; parts 1..kReadParts each run admission, scores and top-K over the
+// slots, then the NoPE readout of every kReadParts-th selected cell.  Each writes a partial
+// online-softmax state; the last part to finish combines them (RMSNorm of the readout,
+// eq. (2)).  CUDA cores.
 #include <cmath>
 #include <cstring>
 
@@ -44,6 +47,10 @@ template <typename T> struct AttendCfg {
     static constexpr int kBlockBytes = kS * kRowStride;         // one 32-row block
     static constexpr int kWarpBytes = 4 * kBlockBytes;          // (K, V) x 2 buffers
 };
+// Attend runs as kAttendParts CTAs per (query, b, h): part 0 the window, parts 1..kReadParts
+// the readout of every kReadParts-th selected cell; each writes a partial online-softmax
+// state (m, l, then 64 unnormalised outputs) and the last to finish combines them.
+constexpr int kReadParts = 4, kAttendParts = kReadParts + 1, kPartFloats = 4 + kD;
 constexpr int kFlagOff = 0;                     // int error flag at the start of the cache
 constexpr size_t kHeadBytes = 256;
 
@@ -53,7 +60,7 @@ size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 struct CacheGeom {
     int R, M, maxnew;
     size_t elem;
-    size_t o_t, o_rk, o_rr, o_rv, o_cell, o_exit, o_a, o_kbar, o_ck, o_cv, bh_bytes;
+    size_t o_t, o_rk, o_rr, o_rv, o_cell, o_exit, o_a, o_kbar, o_ck, o_cv, o_part, o_cnt, bh_bytes;
 };
 
 CacheGeom cache_geom(const fs_params *p, int max_block) {
@@ -78,6 +85,8 @@ CacheGeom cache_geom(const fs_params *p, int max_block) {
     g.o_kbar = seg((size_t)g.M * kD * 4);                   // mean key (float32)
     g.o_ck = seg((size_t)g.M * kS * kD * g.elem);           // the cell's keys
     g.o_cv = seg((size_t)g.M * kS * kD * g.elem);           // the cell's values
+    g.o_part = seg((size_t)max_block * kAttendParts * kPartFloats * 4);   // attend partial states
+    g.o_cnt = seg((size_t)max_block * 4);                   // attend: parts done per query
     g.bh_bytes = off;
     return g;
 }
@@ -89,7 +98,7 @@ struct CacheArgs {
     double theta[kD / 2];   // RoPE frequencies base^(-2m/d), double precision
     float scale;       // 1 / sqrt(d)
     float rms_eps;
-    size_t o_t, o_rk, o_rr, o_rv, o_cell, o_exit, o_a, o_kbar, o_ck, o_cv, bh_bytes;
+    size_t o_t, o_rk, o_rr, o_rv, o_cell, o_exit, o_a, o_kbar, o_ck, o_cv, o_part, o_cnt, bh_bytes;
     float alpha[FS_MAX_HEADS];
     float lambda[FS_MAX_HEADS];
     float inv2sigma[FS_MAX_HEADS];
@@ -126,6 +135,8 @@ struct Slots {   // pointers into one (b, h) block
     int *cell, *exit;
     float *a, *kbar;
     uint8_t *ck, *cv;
+    float *part;
+    int *cnt;
 };
 __device__ __forceinline__ Slots slots_of(uint8_t *cache, const CacheArgs &A, int bh) {
     uint8_t *b = cache + kHeadBytes + (size_t)bh * A.bh_bytes;
@@ -137,6 +148,8 @@ __device__ __forceinline__ Slots slots_of(uint8_t *cache, const CacheArgs &A, in
     S.a = reinterpret_cast<float *>(b + A.o_a);
     S.kbar = reinterpret_cast<float *>(b + A.o_kbar);
     S.ck = b + A.o_ck; S.cv = b + A.o_cv;
+    S.part = reinterpret_cast<float *>(b + A.o_part);
+    S.cnt = reinterpret_cast<int *>(b + A.o_cnt);
     return S;
 }
 
@@ -391,6 +404,38 @@ __device__ __forceinline__ void fold_warps(const Online &o, float (*s_m)[NW], fl
     __syncthreads();
 }
 
+// Folds the NW warps' online states into one raw state: max m, sum l, and out[64] the
+// outputs scaled to m (not divided by l); written to dst[0], dst[1], dst[4..68).
+template <int NW>
+__device__ __forceinline__ void fold_raw(const Online &o, float (*s_m)[NW], float (*s_l)[NW], float (*s_acc)[kD],
+                                         float *dst, int t, int warp, int lane) {
+    if (lane == 0) {
+        (*s_m)[warp] = o.m;
+        (*s_l)[warp] = o.l;
+    }
+    s_acc[warp][2 * lane] = o.a0;
+    s_acc[warp][2 * lane + 1] = o.a1;
+    __syncthreads();
+    if (t < kD) {
+        float mx = -INFINITY;
+        for (int w2 = 0; w2 < NW; w2++) mx = fmaxf(mx, (*s_m)[w2]);
+        float num = 0.f, den = 0.f;
+        if (mx != -INFINITY)
+            for (int w2 = 0; w2 < NW; w2++) {
+                if ((*s_m)[w2] == -INFINITY) continue;
+                const float f = expf((*s_m)[w2] - mx);
+                num = fmaf(s_acc[w2][t], f, num);
+                den = fmaf((*s_l)[w2], f, den);
+            }
+        dst[4 + t] = num;
+        if (t == 0) {
+            dst[0] = mx;
+            dst[1] = den;
+        }
+    }
+    __syncthreads();
+}
+
 template <typename T, bool PRIOR>
 __global__ void __launch_bounds__(AttendCfg<T>::kThreads) cache_attend_kernel(uint8_t *cache, const T *__restrict__ Qn,
                                                                       int n_q, int32_t *__restrict__ idx,
@@ -403,8 +448,9 @@ __global__ void __launch_bounds__(AttendCfg<T>::kThreads) cache_attend_kernel(ui
     extern __shared__ __align__(16) uint8_t shb[];
     unsigned long long *s_key = reinterpret_cast<unsigned long long *>(shb + NW * Cfg::kWarpBytes);
     int *s_cell = reinterpret_cast<int *>(s_key + A.M), *s_sel = s_cell + A.M, *s_list = s_sel + A.M;
-    __shared__ float s_qn[kD], s_qr[kD], s_u[kD], s_o[kD];
+    __shared__ float s_qn[kD], s_qr[kD];
     __shared__ float s_m[NW], s_l[NW], s_acc[NW][kD], s_ss[2];
+    __shared__ int s_last;
     const int r = blockIdx.x, bh = blockIdx.y, h = bh % A.H;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const Slots S = slots_of(cache, A, bh);
@@ -427,137 +473,170 @@ __global__ void __launch_bounds__(AttendCfg<T>::kThreads) cache_attend_kernel(ui
     }
     __syncthreads();
 
-    // 1. admission (eq. (8)) and scores (eq. (7)) over the slots, one thread per slot (the
-    //    mean-key loads of all slots are in flight together)
-    for (int x = t; x < A.M; x += NT) {
-        const int c = S.cell[x];
-        const bool adm = c >= 0 && c < n && (c >= n - A.W || n < S.exit[x]);
-        float sc = 0.f;
-        if (adm) {
-            const float4 *kb = reinterpret_cast<const float4 *>(S.kbar + (size_t)x * kD);
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int e = 0; e < kD / 4; e++) {
-                const float4 v = __ldg(kb + e);
-                acc[e & 3] = fmaf(s_qn[4 * e], v.x, fmaf(s_qn[4 * e + 1], v.y,
-                             fmaf(s_qn[4 * e + 2], v.z, fmaf(s_qn[4 * e + 3], v.w, acc[e & 3]))));
-            }
-            sc = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * A.scale;
-            if (PRIOR) {
-                const float dpos = (float)(i - (long long)c * kS) - 0.5f * kS;   // i - p_c
-                sc += A.lambda[h] * S.a[x] * erff(dpos * A.inv2sigma[h]);
-            }
-        }
-        const uint32_t ob = __float_as_uint(sc);
-        const uint32_t ok = (ob & 0x80000000u) ? ~ob : (ob | 0x80000000u);
-        s_key[x] = adm ? ((unsigned long long)ok << 32) | (0xffffffffu - (uint32_t)c) : 0ull;
-        s_cell[x] = c;
-    }
-    __syncthreads();
-    // 2. top-K: a slot is selected if fewer than K admitted slots have a larger key (higher
-    //    score, or equal score and lower cell): a branch-free count over the keys
-    for (int x = t; x < A.M; x += NT) {
-        const unsigned long long kx = s_key[x];
-        int rank = 0;
-#pragma unroll 4
-        for (int y = 0; y < A.M; y++) rank += s_key[y] > kx;
-        s_sel[x] = kx != 0ull && rank < A.K;
-    }
-    __syncthreads();
-    for (int x = t; x < A.M; x += NT) {   // selected slots in ascending cell order
-        if (!s_sel[x]) continue;
-        const int cx = s_cell[x];
-        int pos = 0;
-#pragma unroll 4
-        for (int y = 0; y < A.M; y++) pos += s_sel[y] & (s_cell[y] < cx);
-        s_list[pos] = x;
-    }
-    __syncthreads();
-    int nsel = 0;
-    for (int y = 0; y < A.M; y++) nsel += s_sel[y];
-    if (idx && t < A.K) idx[((size_t)bh * n_q + r) * A.K + t] = t < nsel ? s_cell[s_list[t]] : -1;
-
-    // 3. readout (eq. (9)): NoPE softmax over every token of the selected cells; warp w
-    //    takes cells w, w+4, ...; lane = token for the scores, lane = dim pair for P V
-    const T *ck = reinterpret_cast<const T *>(S.ck), *cv = reinterpret_cast<const T *>(S.cv);
+    const int part = blockIdx.z;      // 0: the window; 1..kReadParts: a share of the readout
+    float *mypart = S.part + ((size_t)r * kAttendParts + part) * kPartFloats;
     uint8_t *wbuf = shb + warp * Cfg::kWarpBytes;              // (K, V) buffer b at 2 b Cfg::kBlockBytes
-    Online lr;
-    {
-        const int nit = nsel > warp ? (nsel - warp + NW - 1) / NW : 0;   // cells warp, warp + NW, ...
-        auto issue = [&](int k) {
-            const int x = s_list[warp + k * NW];
-            uint8_t *b = wbuf + 2 * (k & 1) * Cfg::kBlockBytes;
-            stage_block<T>(b, [&](int row) { return ck + ((size_t)x * kS + row) * kD; }, lane);
-            stage_block<T>(b + Cfg::kBlockBytes, [&](int row) { return cv + ((size_t)x * kS + row) * kD; }, lane);
-            cp_commit();
-        };
-        if (nit > 0) issue(0);
-        for (int k = 0; k < nit; k++) {
-            if (k + 1 < nit) {
-                issue(k + 1);
-                cp_wait<1>();
-            } else {
-                cp_wait<0>();
+    if (part == 0) {
+        // 4. window (eqs. (3)-(4)): keys max(0, i-w) .. i from the ring, rotated by their
+        //    absolute positions; 32-token blocks split over the warps
+        const T *rr = reinterpret_cast<const T *>(S.rr), *rv = reinterpret_cast<const T *>(S.rv);
+        const long long jlo = i - A.w < 0 ? 0 : i - A.w;
+        const int L = (int)(i - jlo) + 1;
+        Online sr;
+        {
+            const int nblk = (L + kS - 1) / kS;
+            const int nit = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;   // blocks warp, warp + NW, ...
+            const int ri = (int)(i % A.R);                        // ring row of the query's own token
+            auto issue = [&](int k) {
+                // ring row of token `row` of block k (no 64-bit modulo per row: one per block)
+                const long long j0 = jlo + (long long)(warp + k * NW) * kS;
+                const int r0 = (int)(j0 % A.R), last = (int)(i - j0);   // rows past `last` are past i
+                auto row_of = [&](int row) {
+                    if (row > last) return (size_t)ri * kD;           // past i: any row in range
+                    const int rr0 = r0 + row;
+                    return (size_t)(rr0 >= A.R ? rr0 - A.R : rr0) * kD;
+                };
+                uint8_t *b = wbuf + 2 * (k & 1) * Cfg::kBlockBytes;
+                stage_block<T>(b, [&](int row) { return rr + row_of(row); }, lane);
+                stage_block<T>(b + Cfg::kBlockBytes, [&](int row) { return rv + row_of(row); }, lane);
+                cp_commit();
+            };
+            if (nit > 0) issue(0);
+            for (int k = 0; k < nit; k++) {
+                if (k + 1 < nit) {
+                    issue(k + 1);
+                    cp_wait<1>();
+                } else {
+                    cp_wait<0>();
+                }
+                __syncwarp();
+                const uint8_t *b = wbuf + 2 * (k & 1) * Cfg::kBlockBytes;
+                const long long j = jlo + (long long)(warp + k * NW) * kS + lane;
+                const float sc = j <= i ? dot64_smem<T>(s_qr, b + lane * Cfg::kRowStride) * A.scale : -INFINITY;
+                sr.add<T>(sc, b + Cfg::kBlockBytes, lane);
+                __syncwarp();
             }
-            __syncwarp();
-            const uint8_t *b = wbuf + 2 * (k & 1) * Cfg::kBlockBytes;
-            const float sc = dot64_smem<T>(s_qn, b + lane * Cfg::kRowStride) * A.scale;
-            lr.add<T>(sc, b + Cfg::kBlockBytes, lane);
-            __syncwarp();                                        // before the buffer is refilled
         }
+        fold_raw<NW>(sr, &s_m, &s_l, s_acc, mypart, t, warp, lane);
+    } else {
+        // 1. admission (eq. (8)) and scores (eq. (7)) over the slots, one thread per slot (the
+        //    mean-key loads of all slots are in flight together)
+        for (int x = t; x < A.M; x += NT) {
+            const int c = S.cell[x];
+            const bool adm = c >= 0 && c < n && (c >= n - A.W || n < S.exit[x]);
+            float sc = 0.f;
+            if (adm) {
+                const float4 *kb = reinterpret_cast<const float4 *>(S.kbar + (size_t)x * kD);
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+                for (int e = 0; e < kD / 4; e++) {
+                    const float4 v = __ldg(kb + e);
+                    acc[e & 3] = fmaf(s_qn[4 * e], v.x, fmaf(s_qn[4 * e + 1], v.y,
+                                 fmaf(s_qn[4 * e + 2], v.z, fmaf(s_qn[4 * e + 3], v.w, acc[e & 3]))));
+                }
+                sc = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * A.scale;
+                if (PRIOR) {
+                    const float dpos = (float)(i - (long long)c * kS) - 0.5f * kS;   // i - p_c
+                    sc += A.lambda[h] * S.a[x] * erff(dpos * A.inv2sigma[h]);
+                }
+            }
+            const uint32_t ob = __float_as_uint(sc);
+            const uint32_t ok = (ob & 0x80000000u) ? ~ob : (ob | 0x80000000u);
+            s_key[x] = adm ? ((unsigned long long)ok << 32) | (0xffffffffu - (uint32_t)c) : 0ull;
+            s_cell[x] = c;
+        }
+        __syncthreads();
+        // 2. top-K: a slot is selected if fewer than K admitted slots have a larger key (higher
+        //    score, or equal score and lower cell): a branch-free count over the keys
+        for (int x = t; x < A.M; x += NT) {
+            const unsigned long long kx = s_key[x];
+            int rank = 0;
+    #pragma unroll 4
+            for (int y = 0; y < A.M; y++) rank += s_key[y] > kx;
+            s_sel[x] = kx != 0ull && rank < A.K;
+        }
+        __syncthreads();
+        for (int x = t; x < A.M; x += NT) {   // selected slots in ascending cell order
+            if (!s_sel[x]) continue;
+            const int cx = s_cell[x];
+            int pos = 0;
+    #pragma unroll 4
+            for (int y = 0; y < A.M; y++) pos += s_sel[y] & (s_cell[y] < cx);
+            s_list[pos] = x;
+        }
+        __syncthreads();
+        int nsel = 0;
+        for (int y = 0; y < A.M; y++) nsel += s_sel[y];
+        if (part == 1 && idx && t < A.K) idx[((size_t)bh * n_q + r) * A.K + t] = t < nsel ? s_cell[s_list[t]] : -1;
+
+        // 3. readout (eq. (9)): NoPE softmax over this part's share of the selected cells
+        //    (list positions part-1, part-1+kReadParts, ...), warp w taking every NW-th of
+        //    them; lane = token for the scores, lane = dim pair for P V
+        const T *ck = reinterpret_cast<const T *>(S.ck), *cv = reinterpret_cast<const T *>(S.cv);
+        Online lr;
+        {
+            const int p0 = part - 1;
+            const int nloc = nsel > p0 ? (nsel - p0 + kReadParts - 1) / kReadParts : 0;   // this part's cells
+            const int nit = nloc > warp ? (nloc - warp + NW - 1) / NW : 0;
+            auto issue = [&](int k) {
+                const int x = s_list[p0 + kReadParts * (warp + k * NW)];
+                uint8_t *b = wbuf + 2 * (k & 1) * Cfg::kBlockBytes;
+                stage_block<T>(b, [&](int row) { return ck + ((size_t)x * kS + row) * kD; }, lane);
+                stage_block<T>(b + Cfg::kBlockBytes, [&](int row) { return cv + ((size_t)x * kS + row) * kD; }, lane);
+                cp_commit();
+            };
+            if (nit > 0) issue(0);
+            for (int k = 0; k < nit; k++) {
+                if (k + 1 < nit) {
+                    issue(k + 1);
+                    cp_wait<1>();
+                } else {
+                    cp_wait<0>();
+                }
+                __syncwarp();
+                const uint8_t *b = wbuf + 2 * (k & 1) * Cfg::kBlockBytes;
+                const float sc = dot64_smem<T>(s_qn, b + lane * Cfg::kRowStride) * A.scale;
+                lr.add<T>(sc, b + Cfg::kBlockBytes, lane);
+                __syncwarp();                                        // before the buffer is refilled
+            }
+        }
+        fold_raw<NW>(lr, &s_m, &s_l, s_acc, mypart, t, warp, lane);
     }
-    fold_warps<NW>(lr, &s_m, &s_l, s_acc, s_u, t, warp, lane);
-    if (t < kD) {                                 // RMSNorm (no gain), then alpha_h
-        const float ss = warp_sum(s_u[t] * s_u[t]);
+
+    // 5. the last part to finish combines: u from the readout parts (rescaled to their
+    //    largest max), RMSNorm, O = o^sr + alpha_h RMSNorm(u)  (eq. (2))
+    __threadfence();
+    __syncthreads();
+    if (t == 0) s_last = atomicAdd(S.cnt + r, 1) == kAttendParts - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const float *P0 = S.part + (size_t)r * kAttendParts * kPartFloats;
+    float u = 0.f, o = 0.f, den = 0.f;
+    if (t < kD) {
+        float mx = -INFINITY;
+        for (int pp = 1; pp <= kReadParts; pp++) mx = fmaxf(mx, __ldcg(P0 + pp * kPartFloats));
+        float num = 0.f;
+        if (mx != -INFINITY)
+            for (int pp = 1; pp <= kReadParts; pp++) {
+                const float mp = __ldcg(P0 + pp * kPartFloats);
+                if (mp == -INFINITY) continue;
+                const float fct = expf(mp - mx);
+                num = fmaf(__ldcg(P0 + pp * kPartFloats + 4 + t), fct, num);
+                den = fmaf(__ldcg(P0 + pp * kPartFloats + 1), fct, den);
+            }
+        u = den > 0.f ? num / den : 0.f;
+        const float l0 = __ldcg(P0 + 1);
+        o = l0 > 0.f ? __ldcg(P0 + 4 + t) / l0 : 0.f;
+        const float ss = warp_sum(u * u);
         if (lane == 0) s_ss[warp] = ss;
     }
     __syncthreads();
-    const float f = nsel > 0 ? A.alpha[h] / sqrtf((s_ss[0] + s_ss[1]) * (1.f / kD) + A.rms_eps) : 0.f;
-
-    // 4. window (eqs. (3)-(4)): keys max(0, i-w) .. i from the ring, rotated by their
-    //    absolute positions; 32-token blocks split over the warps
-    const T *rr = reinterpret_cast<const T *>(S.rr), *rv = reinterpret_cast<const T *>(S.rv);
-    const long long jlo = i - A.w < 0 ? 0 : i - A.w;
-    const int L = (int)(i - jlo) + 1;
-    Online sr;
-    {
-        const int nblk = (L + kS - 1) / kS;
-        const int nit = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;   // blocks warp, warp + NW, ...
-        const int ri = (int)(i % A.R);                        // ring row of the query's own token
-        auto issue = [&](int k) {
-            // ring row of token `row` of block k (no 64-bit modulo per row: one per block)
-            const long long j0 = jlo + (long long)(warp + k * NW) * kS;
-            const int r0 = (int)(j0 % A.R), last = (int)(i - j0);   // rows past `last` are past i
-            auto row_of = [&](int row) {
-                if (row > last) return (size_t)ri * kD;           // past i: any row in range
-                const int rr0 = r0 + row;
-                return (size_t)(rr0 >= A.R ? rr0 - A.R : rr0) * kD;
-            };
-            uint8_t *b = wbuf + 2 * (k & 1) * Cfg::kBlockBytes;
-            stage_block<T>(b, [&](int row) { return rr + row_of(row); }, lane);
-            stage_block<T>(b + Cfg::kBlockBytes, [&](int row) { return rv + row_of(row); }, lane);
-            cp_commit();
-        };
-        if (nit > 0) issue(0);
-        for (int k = 0; k < nit; k++) {
-            if (k + 1 < nit) {
-                issue(k + 1);
-                cp_wait<1>();
-            } else {
-                cp_wait<0>();
-            }
-            __syncwarp();
-            const uint8_t *b = wbuf + 2 * (k & 1) * Cfg::kBlockBytes;
-            const long long j = jlo + (long long)(warp + k * NW) * kS + lane;
-            const float sc = j <= i ? dot64_smem<T>(s_qr, b + lane * Cfg::kRowStride) * A.scale : -INFINITY;
-            sr.add<T>(sc, b + Cfg::kBlockBytes, lane);
-            __syncwarp();
-        }
+    if (t < kD) {
+        const float f = den > 0.f ? A.alpha[h] / sqrtf((s_ss[0] + s_ss[1]) * (1.f / kD) + A.rms_eps) : 0.f;
+        O[((size_t)bh * n_q + r) * kD + t] = from_f<T>(o + f * u);
     }
-    fold_warps<NW>(sr, &s_m, &s_l, s_acc, s_o, t, warp, lane);
-
-    // 5. O = o^sr + alpha_h RMSNorm(u)  (eq. (2))
-    if (t < kD) O[((size_t)bh * n_q + r) * kD + t] = from_f<T>(s_o[t] + f * s_u[t]);
+    if (t == 0) S.cnt[r] = 0;                     // ready for the next call
 }
 
 __global__ void cache_reset_kernel(uint8_t *cache, const CacheArgs A) {
@@ -568,6 +647,7 @@ __global__ void cache_reset_kernel(uint8_t *cache, const CacheArgs A) {
         S.cell[x] = -1;
         S.exit[x] = 0;
     }
+    for (int x = threadIdx.x; x < A.max_block; x += blockDim.x) S.cnt[x] = 0;
 }
 
 }  // namespace
@@ -604,6 +684,7 @@ CacheArgs cache_args(const fs_params *p, int max_block, const CacheGeom &g) {
     A.rms_eps = p->rms_eps;
     A.o_t = g.o_t; A.o_rk = g.o_rk; A.o_rr = g.o_rr; A.o_rv = g.o_rv; A.o_cell = g.o_cell;
     A.o_exit = g.o_exit; A.o_a = g.o_a; A.o_kbar = g.o_kbar; A.o_ck = g.o_ck; A.o_cv = g.o_cv;
+    A.o_part = g.o_part; A.o_cnt = g.o_cnt;
     A.bh_bytes = g.bh_bytes;
     for (int h = 0; h < p->H; h++) {
         A.alpha[h] = p->alpha[h];
@@ -663,7 +744,7 @@ template <typename T>
 cudaError_t attend_launch(const CacheArgs &A, uint8_t *c, const void *Q, int n_q, int32_t *idx, void *O,
                           int BH, cudaStream_t st) {
     const size_t smem = (size_t)AttendCfg<T>::kWarps * AttendCfg<T>::kWarpBytes + (size_t)A.M * 16 + (size_t)kMaxK * 4;
-    const dim3 grid(n_q, BH);
+    const dim3 grid(n_q, BH, kAttendParts);
     auto kern = A.has_prior ? cache_attend_kernel<T, true> : cache_attend_kernel<T, false>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     kern<<<grid, AttendCfg<T>::kThreads, smem, st>>>(c, static_cast<const T *>(Q), n_q, idx, static_cast<T *>(O), A);
