@@ -252,6 +252,72 @@ __device__ __forceinline__ bool beats(float Ua, int pa, float Ub, int pb) {
     return Ua > Ub || (Ua == Ub && pa < pb);
 }
 
+// Bitonic sort of the warp's 32E entries (entry i = e*32 + lane: score U, tie key pm, ref),
+// better first (beats()).  Partners closer than 32 are exchanged by shuffles, the others
+// within the lane's registers.
+template <int E>
+__device__ __forceinline__ void warp_sort(float (&U)[E], int (&pm)[E], int (&rf)[E], int lane) {
+    constexpr int P = 32 * E;
+#pragma unroll
+    for (int k = 2; k <= P; k <<= 1) {
+#pragma unroll
+        for (int d = k >> 1; d > 0; d >>= 1) {
+            if (d >= 32) {
+#pragma unroll
+                for (int e = 0; e < E; e++) {
+                    const int f = e ^ (d >> 5);
+                    if (f <= e) continue;              // each pair once, from its lower entry
+                    const bool desc = ((e * 32 + lane) & k) == 0;   // better to the lower index
+                    if (beats(U[f], pm[f], U[e], pm[e]) == desc) {
+                        const float tu = U[e]; U[e] = U[f]; U[f] = tu;
+                        const int tp = pm[e]; pm[e] = pm[f]; pm[f] = tp;
+                        const int tr = rf[e]; rf[e] = rf[f]; rf[f] = tr;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < E; e++) {
+                    const float Ub = __shfl_xor_sync(kFull, U[e], d);
+                    const int pb = __shfl_xor_sync(kFull, pm[e], d);
+                    const int rb = __shfl_xor_sync(kFull, rf[e], d);
+                    const bool lower = (lane & d) == 0, desc = ((e * 32 + lane) & k) == 0;
+                    const bool better = beats(Ub, pb, U[e], pm[e]);
+                    if ((lower == desc) ? better : !better) {
+                        U[e] = Ub;
+                        pm[e] = pb;
+                        rf[e] = rb;
+                    }
+                }
+            }
+        }
+    }
+}
+
+// The beam: the nb = min(n, beta) best of the n candidates in S.U/S.pmin/S.ref, sorted,
+// into S.bU/S.bpmin/S.bref (entries past n are padding that never wins)
+template <int E, typename Smem>
+__device__ __forceinline__ void beam_cut(Smem &S, int n, int nb, int lane) {
+    float U[E];
+    int pm[E], rf[E];
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        const int i = e * 32 + lane;
+        U[e] = i < n ? S.U[i] : -INFINITY;
+        pm[e] = i < n ? S.pmin[i] : 0x7fffffff;
+        rf[e] = i < n ? S.ref[i] : 0;
+    }
+    warp_sort<E>(U, pm, rf, lane);
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        const int i = e * 32 + lane;
+        if (i < nb) {
+            S.bU[i] = U[e];
+            S.bpmin[i] = pm[e];
+            S.bref[i] = rf[e];
+        }
+    }
+}
+
 // eq. (11) for one node (lane-local: the whole dot product in this lane)
 template <bool PRIOR>
 __device__ __forceinline__ float node_U(const Forest &F, size_t lvl_base, int node, const float *q, float qn,
@@ -300,19 +366,11 @@ __device__ int search_forest(const Forest &F, SearchSmem &S, int bh, int f, int 
     }
     __syncwarp();
     for (int guard = 0; guard < 64; guard++) {
-        // keep the beam best candidates: rank = number of candidates that beat this one
-        int nb = min(ncand, A.beam);
-        for (int j = lane; j < ncand; j += 32) {
-            const float Uj = S.U[j];
-            const int pj = S.pmin[j];
-            int rank = 0;
-            for (int x = 0; x < ncand; x++) rank += beats(S.U[x], S.pmin[x], Uj, pj);
-            if (rank < A.beam) {
-                S.bU[rank] = Uj;
-                S.bref[rank] = S.ref[j];
-                S.bpmin[rank] = pj;
-            }
-        }
+        // keep the beam best candidates (a warp-wide bitonic sort of the candidates)
+        const int nb = min(ncand, A.beam);
+        if (ncand <= 32) beam_cut<1>(S, ncand, nb, lane);
+        else if (ncand <= 64) beam_cut<2>(S, ncand, nb, lane);
+        else beam_cut<4>(S, ncand, nb, lane);
         __syncwarp();
         // expand every internal node
         int cnt0 = 0, cnt1 = 0;
