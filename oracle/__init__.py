@@ -71,6 +71,9 @@ def lib():
                                            i32p, f64p]
         L.orc_tree_node.argtypes = [P, f32p, f64p, f64p, ctypes.c_void_p] + [ctypes.c_int] * 7 + [
             ctypes.c_double, i32p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)]
+        L.orc_backward_sampled.argtypes = [P, f32p, f32p, f32p, i32p, f64p, ctypes.c_longlong, i64p, f64p,
+                                           ctypes.c_longlong, i64p, f64p, f64p]
+        L.orc_select_all.argtypes = [P, f32p, f64p, f64p, i32p]
         L.orc_rope.argtypes = [P, f32p, ctypes.c_longlong, f64p]
         L.orc_rope.restype = None
         _lib = L
@@ -229,6 +232,29 @@ class Problem:
         if cnt < 0:
             return None, None, nseq.value
         return leaves[:cnt].copy(), U.value, nseq.value
+
+    def backward_sampled(self, idx, dO, rows, keys):
+        """Gradients of eq. (2) on samples: dQ [len(rows), d] of flat rows (b*H + h)*Nq + r
+        and dK, dV [len(keys), d] of flat keys (b*H + h)*Nk + j, for every row's cells idx
+        [B,H,Nq,K] and upstream gradient dO [B,H,Nq,d] (float64)."""
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        keys = np.ascontiguousarray(keys, dtype=np.int64)
+        dQ = np.zeros((max(len(rows), 1), self.d)); dK = np.zeros((max(len(keys), 1), self.d))
+        dV = np.zeros_like(dK)
+        lib().orc_backward_sampled(ctypes.byref(self.p), self.Q, self.K, self.V,
+                                   np.ascontiguousarray(idx, np.int32).reshape(-1),
+                                   np.ascontiguousarray(dO, np.float64).reshape(-1),
+                                   len(rows), rows if len(rows) else np.zeros(1, np.int64), dQ.reshape(-1),
+                                   len(keys), keys if len(keys) else np.zeros(1, np.int64), dK.reshape(-1),
+                                   dV.reshape(-1))
+        return dQ[:len(rows)], dK[:len(keys)], dV[:len(keys)]
+
+    def select_all(self, kbar, amax):
+        """eq. (7) selection of every row: idx [B,H,Nq,K] (ascending, -1 padded)."""
+        idx = np.zeros((self.B, self.H, self.Nq, max(self.p.K, 1)), np.int32)
+        lib().orc_select_all(ctypes.byref(self.p), self.Q, np.ascontiguousarray(kbar, np.float64).reshape(-1),
+                             np.ascontiguousarray(amax, np.float64).reshape(-1), idx.reshape(-1))
+        return idx[..., :self.p.K]
 
     def readout_rows(self, rows, idx):
         """eq. (9) for the given flat rows on caller-given cells idx [n,K]: (u, o^lr)."""

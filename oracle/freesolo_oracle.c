@@ -640,6 +640,168 @@ int orc_backward(const orc_params *p, const float *Q, const float *K, const floa
     return 0;
 }
 
+/* ---- backward on samples (full-size checks) ----
+ * One row's contribution to the gradients of eq. (2), the same arithmetic as orc_backward:
+ * adds the row's dq (if dq) and its contribution to key `key` (dk, dv; key < 0: none).
+ * krot holds the head's keys rotated by their positions. */
+static void row_grad(const orc_params *p, const float *Kbh, const float *Vbh, const double *krot,
+                     const float *q, long long i, const int *sel, const double *g, double a,
+                     double *dq, int key, double *dk, double *dv)
+{
+    const int d = p->d, s = p->s, Kc = p->K;
+    const double sc = logit_scale(p);
+    double qrot[512], dqrot[512], tmp[512], o[512], u[512], y[512], du[512], kk[512];
+    memset(dqrot, 0, sizeof(dqrot));
+    /* window branch */
+    rope_rotate(p, q, p->pos0 + i, qrot);
+    const long long j0 = i - p->w < 0 ? 0 : i - p->w;
+    const int n = (int)(i - j0 + 1);
+    double *lg = (double *)malloc(sizeof(double) * (size_t)(n > Kc * s ? n : Kc * s + 1));
+    double mx = -INFINITY, den = 0.0;
+    for (long long j = j0; j <= i; j++) {
+        double dot = 0.0;
+        for (int m = 0; m < d; m++) dot += qrot[m] * krot[(size_t)j * d + m];
+        lg[j - j0] = dot * sc;
+        if (lg[j - j0] > mx) mx = lg[j - j0];
+    }
+    for (int m = 0; m < d; m++) o[m] = 0.0;
+    for (long long j = j0; j <= i; j++) { lg[j - j0] = exp(lg[j - j0] - mx); den += lg[j - j0]; }
+    for (long long j = j0; j <= i; j++) {
+        lg[j - j0] /= den;
+        for (int m = 0; m < d; m++) o[m] += lg[j - j0] * Vbh[(size_t)j * d + m];
+    }
+    double D = 0.0;
+    for (int m = 0; m < d; m++) { D += g[m] * o[m]; dqrot[m] = 0.0; }
+    for (long long j = j0; j <= i; j++) {
+        double dp = 0.0;
+        for (int m = 0; m < d; m++) dp += g[m] * Vbh[(size_t)j * d + m];
+        const double ds = lg[j - j0] * (dp - D) * sc;
+        if (dq) for (int m = 0; m < d; m++) dqrot[m] += ds * krot[(size_t)j * d + m];
+        if (j == key) {
+            for (int m = 0; m < d; m++) { dv[m] += lg[j - j0] * g[m]; kk[m] = ds * qrot[m]; }
+            rope_rotate_back(p, kk, p->pos0 + j, tmp);
+            for (int m = 0; m < d; m++) dk[m] += tmp[m];
+        }
+    }
+    if (dq) {
+        rope_rotate_back(p, dqrot, p->pos0 + i, tmp);
+        for (int m = 0; m < d; m++) dq[m] += tmp[m];
+    }
+    /* readout branch */
+    int ncell = 0;
+    for (int e = 0; e < Kc; e++) ncell += sel[e] >= 0;
+    if (ncell == 0) { free(lg); return; }
+    mx = -INFINITY;
+    int t = 0;
+    for (int e = 0; e < Kc; e++) {
+        if (sel[e] < 0) continue;
+        for (int j = sel[e] * s; j < (sel[e] + 1) * s; j++, t++) {
+            double dot = 0.0;
+            for (int m = 0; m < d; m++) dot += (double)q[m] * Kbh[(size_t)j * d + m];
+            lg[t] = dot * sc;
+            if (lg[t] > mx) mx = lg[t];
+        }
+    }
+    const int ntok = t;
+    den = 0.0;
+    for (t = 0; t < ntok; t++) { lg[t] = exp(lg[t] - mx); den += lg[t]; }
+    for (int m = 0; m < d; m++) u[m] = 0.0;
+    t = 0;
+    for (int e = 0; e < Kc; e++) {
+        if (sel[e] < 0) continue;
+        for (int j = sel[e] * s; j < (sel[e] + 1) * s; j++, t++) {
+            lg[t] /= den;
+            for (int m = 0; m < d; m++) u[m] += lg[t] * Vbh[(size_t)j * d + m];
+        }
+    }
+    double ms = 0.0;
+    for (int m = 0; m < d; m++) ms += u[m] * u[m];
+    const double rin = 1.0 / sqrt(ms / d + p->rms_eps);
+    double dyy = 0.0;
+    for (int m = 0; m < d; m++) { y[m] = u[m] * rin; dyy += a * g[m] * y[m]; }
+    for (int m = 0; m < d; m++) du[m] = rin * (a * g[m] - y[m] * dyy / d);
+    D = 0.0;
+    for (int m = 0; m < d; m++) D += du[m] * u[m];
+    t = 0;
+    for (int e = 0; e < Kc; e++) {
+        if (sel[e] < 0) continue;
+        for (int j = sel[e] * s; j < (sel[e] + 1) * s; j++, t++) {
+            double dp = 0.0;
+            for (int m = 0; m < d; m++) dp += du[m] * Vbh[(size_t)j * d + m];
+            const double ds = lg[t] * (dp - D) * sc;
+            if (dq) for (int m = 0; m < d; m++) dq[m] += ds * Kbh[(size_t)j * d + m];
+            if (j == key) for (int m = 0; m < d; m++) { dv[m] += lg[t] * du[m]; dk[m] += ds * q[m]; }
+        }
+    }
+    free(lg);
+}
+
+/* Gradients of eq. (2) on samples of a (possibly full-size) problem: dQ of the given rows
+ * (flat (b*H + h)*Nq + r) and dK, dV of the given keys (flat (b*H + h)*Nk + j), with every
+ * row's cells idx [B,H,Nq,K] and upstream gradient dO [B,H,Nq,d] given.  A key gathers
+ * every row whose window holds it and every row whose cells hold it. */
+int orc_backward_sampled(const orc_params *p, const float *Q, const float *K, const float *V, const int *idx,
+                         const double *dO, long long nrows, const long long *rows, double *dQ,
+                         long long nkeys, const long long *keys, double *dK, double *dV)
+{
+    const int d = p->d, s = p->s, Kc = p->K, BH = p->B * p->H;
+    const long long q0 = (long long)(p->Nk - p->Nq);
+    memset(dQ, 0, sizeof(double) * (size_t)(nrows > 0 ? nrows : 0) * d);
+    memset(dK, 0, sizeof(double) * (size_t)(nkeys > 0 ? nkeys : 0) * d);
+    memset(dV, 0, sizeof(double) * (size_t)(nkeys > 0 ? nkeys : 0) * d);
+    for (int bh = 0; bh < BH; bh++) {
+        int used = 0;
+        for (long long t = 0; t < nrows && !used; t++) used = rows[t] / p->Nq == bh;
+        for (long long t = 0; t < nkeys && !used; t++) used = keys[t] / p->Nk == bh;
+        if (!used) continue;
+        const int h = bh % p->H;
+        const double a = p->alpha ? p->alpha[h] : 0.0;
+        const float *Kbh = K + (size_t)bh * p->Nk * d, *Vbh = V + (size_t)bh * p->Nk * d;
+        double *krot = (double *)malloc(sizeof(double) * (size_t)p->Nk * d);
+        #pragma omp parallel for schedule(static)
+        for (int j = 0; j < p->Nk; j++) rope_rotate(p, Kbh + (size_t)j * d, p->pos0 + j, krot + (size_t)j * d);
+        #pragma omp parallel for schedule(dynamic, 1)
+        for (long long t = 0; t < nrows; t++) {
+            if (rows[t] / p->Nq != bh) continue;
+            const int r = (int)(rows[t] % p->Nq);
+            row_grad(p, Kbh, Vbh, krot, Q + ((size_t)bh * p->Nq + r) * d, q0 + r,
+                     idx + ((size_t)bh * p->Nq + r) * Kc, dO + ((size_t)bh * p->Nq + r) * d, a,
+                     dQ + (size_t)t * d, -1, NULL, NULL);
+        }
+        #pragma omp parallel for schedule(dynamic, 1)
+        for (long long t = 0; t < nkeys; t++) {
+            if (keys[t] / p->Nk != bh) continue;
+            const int j = (int)(keys[t] % p->Nk);
+            const int cj = j / s;
+            for (int r = 0; r < p->Nq; r++) {
+                const long long i = q0 + r;
+                const int *sel = idx + ((size_t)bh * p->Nq + r) * Kc;
+                int in = j <= i && j >= i - p->w;
+                for (int e = 0; e < Kc && !in; e++) in = sel[e] == cj && cj < orc_num_cells(p);
+                if (!in) continue;
+                row_grad(p, Kbh, Vbh, krot, Q + ((size_t)bh * p->Nq + r) * d, i, sel,
+                         dO + ((size_t)bh * p->Nq + r) * d, a, NULL, j, dK + (size_t)t * d, dV + (size_t)t * d);
+            }
+        }
+        free(krot);
+    }
+    return 0;
+}
+
+/* eq. (7) selection (steps 3-6) for every row, no outputs: idx [B,H,Nq,K]. */
+int orc_select_all(const orc_params *p, const float *Q, const double *kbar, const double *amax, int *idx)
+{
+    const int C = orc_num_cells(p), BH = p->B * p->H;
+    #pragma omp parallel for schedule(dynamic, 64)
+    for (long long f = 0; f < (long long)BH * p->Nq; f++) {
+        const int bh = (int)(f / p->Nq), r = (int)(f % p->Nq);
+        const long long i = (long long)(p->Nk - p->Nq) + r;
+        select_row(p, Q + (size_t)f * p->d, i, bh % p->H, kbar + (size_t)bh * C * p->d, amax + (size_t)bh * C,
+                   idx + (size_t)f * p->K, NULL, NULL);
+    }
+    return 0;
+}
+
 /* ---- single-step entry points for the tests ---- */
 
 /* Selection for one row (b,h,r) given its head's summaries.  Writes idx_out[K];

@@ -88,3 +88,35 @@ def test_backward_empty_queries():
     inp = generate(small("bwd_empty", Nq=0, Nk=256, dtype="f32", seed=503))
     got = gpu_backward(inp, np.zeros((1, 2, 0, inp.wl.K), np.int32), np.zeros((1, 2, 0, 64), np.float32))
     assert np.abs(got[1]).max() == 0.0 and np.abs(got[2]).max() == 0.0 and np.abs(got[3]).max() == 0.0
+
+
+def test_backward_full_size_sampled():
+    """The 16k prefill workload (B=2, H=16, 16384 tokens) at full size, on the oracle's own
+    selection of every row: dQ of sampled rows and dK, dV of sampled keys (each gathering
+    every row whose window or cells hold it) against the float64 oracle."""
+    from workloads import CONFIGS
+    inp = generate(CONFIGS["prefill16k"])
+    wl = inp.wl
+    prob = oracle_for(inp)
+    kb, am = prob.summaries()
+    idx = prob.select_all(kb, am)
+    dO = upstream_grad(wl, 91)
+    got = gpu_backward(inp, idx, dO)
+    rng = np.random.default_rng(92)
+    rows = rng.integers(0, wl.B * wl.H * wl.Nq, 48)
+    # keys: some inside needle cells and frequently selected cells, the rest uniform
+    flat = idx.reshape(wl.B * wl.H, -1)
+    keys = []
+    for _ in range(12):
+        bh = int(rng.integers(0, wl.B * wl.H))
+        cells = flat[bh][flat[bh] >= 0]
+        c = int(rng.choice(cells)) if len(cells) else int(rng.integers(0, wl.Nk // wl.s))
+        keys.append(bh * wl.Nk + c * wl.s + int(rng.integers(0, wl.s)))
+    keys += rng.integers(0, wl.B * wl.H * wl.Nk, 8).tolist()
+    keys = np.array(keys, np.int64)
+    sq, sk, sv = prob.backward_sampled(idx, dO, rows, keys)
+    d = wl.d
+    gq, gk, gv = got[0].reshape(-1, d)[rows], got[1].reshape(-1, d)[keys], got[2].reshape(-1, d)[keys]
+    for name, g, r in (("dQ", gq, sq), ("dK", gk, sk), ("dV", gv, sv)):
+        scale = max(1.0, float(np.abs(r).max()))
+        assert np.abs(g - r).max() <= TOL[wl.dtype] * scale, (name, float(np.abs(g - r).max()), scale)

@@ -105,3 +105,35 @@ def test_cache_attend_past_the_stream_is_reported():
         fs.cache_status(cache)
     assert e.value.code == 6
     fs.cache_status(cache)          # the flag was cleared
+
+
+def test_cache_full_size_decode_sampled():
+    """The 256k-token decode workload through the streaming cache: the archive appended in
+    blocks of 128, then the 128 new tokens appended and their queries attended in one call;
+    selection (near-tie rule) and output judged against the float64 oracle on sampled rows
+    (the same rows the batch decode test uses)."""
+    from workloads import CONFIGS
+    from tests._parity import sample_rows
+    inp = generate(CONFIGS["decode256k"])
+    wl = inp.wl
+    p = params_for(inp)
+    mb = 128
+    cache = fs.alloc_cache(p, mb)
+    dt = tdtype(wl)
+    K, V = (torch.from_numpy(x).cuda().to(dt) for x in (inp.K, inp.V))
+    for a in range(0, wl.Nk, mb):
+        fs.cache_append(p, mb, cache, K[:, :, a:a + mb].contiguous(), V[:, :, a:a + mb].contiguous())
+    Qd = torch.from_numpy(inp.Q).cuda().to(dt)
+    O = torch.full_like(Qd, float("nan"))
+    idx = torch.empty((wl.B, wl.H, wl.Nq, wl.K), dtype=torch.int32, device="cuda")
+    fs.cache_attend(p, mb, cache, Qd, O, idx)
+    fs.cache_status(cache)
+    prob = oracle_for(inp)
+    rows = sample_rows(wl, 200, seed=1)
+    idx_n = idx.cpu().numpy()
+    exact, tie = check_selection(inp, prob.summaries(), idx_n, rows)
+    assert tie <= max(2, len(rows) // 50), (exact, tie)
+    got = O.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    err = np.abs(np.stack([got[b, h, r] for b, h, r in rows]) - expected_output(inp, prob, rows, idx_n)).max()
+    assert err <= TOL[wl.dtype], err

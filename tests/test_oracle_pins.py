@@ -420,6 +420,26 @@ def test_backward_matches_finite_differences():
     assert _fd_failures(n_entries=20) == []
 
 
+def test_backward_sampled_matches_full_backward():
+    """The sampled backward (rows' dQ, keys' dK and dV, for full-size checks) equals the
+    whole backward pass, itself pinned by finite differences, on every row and key; and
+    the all-rows selection equals the forward pass's."""
+    inp = tiny(d=16, Nq=150, Nk=260, w=32, s=8, K=3, W=2, P=3, lam=0.5, sigma=30.0, seed=71)
+    prob = make_problem(inp)
+    _, idx = prob.forward(want_idx=True)
+    kb, am = prob.summaries()
+    assert np.array_equal(prob.select_all(kb, am), idx)
+    dO = np.random.default_rng(72).standard_normal((inp.wl.B, inp.wl.H, inp.wl.Nq, inp.wl.d))
+    dQ, dK, dV, _ = prob.backward(idx, dO)
+    rows = np.arange(inp.wl.B * inp.wl.H * inp.wl.Nq)
+    keys = np.arange(inp.wl.B * inp.wl.H * inp.wl.Nk)
+    sq, sk, sv = prob.backward_sampled(idx, dO, rows, keys)
+    d = inp.wl.d
+    assert np.abs(sq - dQ.reshape(-1, d)).max() <= 1e-12
+    assert np.abs(sk - dK.reshape(-1, d)).max() <= 1e-12
+    assert np.abs(sv - dV.reshape(-1, d)).max() <= 1e-12
+
+
 # ---------------------------------------------------------------- FS-B (eqs. (10)-(11))
 def _codes(kbar_bh):
     """16-bit code of each cell: the signs of its mean key's first 16 coordinates,
