@@ -190,8 +190,8 @@ fs_status fs_backward(const fs_params *p, const void *Q, const void *K, const vo
                       const void *dO, float *dQ, float *dK, float *dV, float *dalpha, void *bws,
                       size_t bws_bytes, void *stream);
 
-/* ---- FS-L streaming cache ("FreeSolo" summary, "Practical Implications" 3: bounded
- * memory, O((P+W)s + w + B + s)d token state per head, independent of sequence length) ----
+/* ---- FS-L streaming cache ("FreeSolo" summary, "Practical Implications" 3: the per-head
+ * memory of a stream is bounded by O((P+W)s + w + B + s)·d, whatever its length) ----
  * Tokens arrive in blocks of at most max_block (the B of that bound); after each block,
  * attention can be computed for any of its most recent positions from the cache alone.
  * The cache keeps, per (batch, head):

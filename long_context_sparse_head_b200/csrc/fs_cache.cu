@@ -1,6 +1,6 @@
 // FS-L streaming cache: the forward pass over a token stream with bounded state per head,
-// "FreeSolo" summary, "Practical Implications" 3 (O((P+W)s + w + B + s)d token state per
-// head) and §3.3 eq. (8).  Same arithmetic as the batch forward pass (§3.1 eq. (2), §3.2
+// "FreeSolo" summary, "Practical Implications" 3 (per-head memory bounded by
+// O((P+W)s + w + B + s)·d) and §3.3 eq. (8).  Same arithmetic as the batch forward pass (§3.1 eq. (2), §3.2
 // eqs. (3)-(4), §3.3 eqs. (5), (7), (9)); what differs is where the keys and values live.
 //
 // State of one (batch, head):

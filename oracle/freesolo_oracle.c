@@ -17,8 +17,8 @@
  *                                    balanced trees (all candidates; cells with a_c >= tau_h)
  *                          eq. (12)  token-level rerank: a cell scored by the log-sum-exp
  *                                    of its tokens' NoPE logits plus the prior term
- * "Introduction and Theoretical Foundation": RoPE (Su et al.) stays inside the
- * local window; long-range routing and readout use unrotated vectors.
+ * "Introduction and Theoretical Foundation": RoPE (Su et al.) is applied only inside the
+ * local window; the long-range branch selects and reads cells without rotation.
  *
  * Readings where the page is silent or garbled (each is also listed in the design notes):
  *   - L_i = { j : max(0, i-w) <= j <= i }            ("look-back radius w", §3.2)
