@@ -42,7 +42,7 @@ def oracle_for(inp, **over):
     return oracle.Problem(inp.Q, inp.K, inp.V, **kw)
 
 
-class GpuRun:
+class DeviceRun:
     """Device copies of the inputs and the C-ABI calls on them."""
 
     def __init__(self, inp, **over):

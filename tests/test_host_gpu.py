@@ -10,7 +10,7 @@ import torch
 
 import long_context_sparse_head_b200 as fs
 from workloads import generate, small
-from tests._parity import TOL, GpuRun, check_selection, expected_output, oracle_for, sample_rows, tdtype
+from tests._parity import TOL, DeviceRun, check_selection, expected_output, oracle_for, sample_rows, tdtype
 
 pytestmark = pytest.mark.gpu
 
@@ -30,7 +30,7 @@ def test_forward_host_matches_device(dtype, case):
     sigma = kw.pop("sigma", 1024.0)
     inp = generate(small("host", lam=lam, sigma=sigma, **kw))
     wl = inp.wl
-    g = GpuRun(inp)
+    g = DeviceRun(inp)
     ref = g.numpy(g.forward()).copy()
     dt = tdtype(wl)
     hQ, hK, hV = (torch.from_numpy(x).to(dt).pin_memory() for x in (inp.Q, inp.K, inp.V))

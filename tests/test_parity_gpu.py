@@ -8,7 +8,7 @@ import pytest
 import torch
 
 from workloads import CONFIGS, generate, small
-from tests._parity import (TOL, GpuRun, check_selection, expected_output, oracle_for,
+from tests._parity import (TOL, DeviceRun, check_selection, expected_output, oracle_for,
                            sample_rows)
 
 pytestmark = pytest.mark.gpu
@@ -21,7 +21,7 @@ def all_rows(wl):
 def run_case(inp, rows=None, check_needles=True, **over):
     """Summaries, selection and output parity for one problem."""
     wl = inp.wl
-    g = GpuRun(inp, **over)
+    g = DeviceRun(inp, **over)
     prob = oracle_for(inp, **over)
     kbar_o, amax_o = prob.summaries()
     kbar_g, amax_g = (g.numpy(t) for t in g.summaries())
@@ -89,7 +89,7 @@ def test_caller_idx_runs_readout_on_given_cells():
     those cells, and with the internally selected path when given the GPU's own cells."""
     inp = generate(small("given", Nq=1024, Nk=1024, K=5, W=3, P=6, dtype="bf16", seed=7))
     wl = inp.wl
-    g = GpuRun(inp)
+    g = DeviceRun(inp)
     idx_sel = g.select().clone()
     O_sel = g.forward().clone()
     O_given = g.forward(idx=idx_sel)
@@ -117,7 +117,7 @@ def test_caller_idx_runs_readout_on_given_cells():
 
 def test_caller_summaries_match_internal():
     inp = generate(small("sums", Nq=512, Nk=2048, K=4, W=3, P=5, dtype="bf16", seed=8))
-    g = GpuRun(inp)
+    g = DeviceRun(inp)
     kbar, amax = g.summaries()
     O1 = g.forward().clone()
     O2 = g.forward(kbar=kbar, amax=amax)
@@ -126,7 +126,7 @@ def test_caller_summaries_match_internal():
 
 def test_repeated_calls_are_deterministic():
     inp = generate(small("det", Nq=2048, Nk=2048, K=8, dtype="bf16", seed=9))
-    g = GpuRun(inp)
+    g = DeviceRun(inp)
     a = g.forward().clone()
     b = g.forward().clone()
     assert torch.equal(a, b)

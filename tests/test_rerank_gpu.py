@@ -11,7 +11,7 @@ import torch
 
 import long_context_sparse_head_b200 as fs
 from workloads import Inputs, generate, small
-from tests._parity import TIE, TOL, GpuRun, expected_output, oracle_for
+from tests._parity import TIE, TOL, DeviceRun, expected_output, oracle_for
 
 pytestmark = pytest.mark.gpu
 
@@ -47,7 +47,7 @@ def check_rerank(prob, kbar, amax, gidx, rows, shortlist):
 
 def run_rerank(inp, shortlist=0, rows=None, **over):
     wl = inp.wl
-    g = GpuRun(inp, **over)
+    g = DeviceRun(inp, **over)
     prob = oracle_for(inp, **over)
     kbar_o, amax_o = prob.summaries()
     g.summaries()
@@ -116,7 +116,7 @@ def test_forward_rerank(dtype, case):
     sigma = kw.pop("sigma", 1024.0)
     inp = generate(small("fwd_rerank", lam=lam, sigma=sigma, **kw))
     wl = inp.wl
-    g = GpuRun(inp)
+    g = DeviceRun(inp)
     prob = oracle_for(inp)
     g.summaries()
     fs.select_topk_rerank(g.p, g.Q, g.K, g.kbar, g.amax, g.idx, g.ws, shortlist)
@@ -140,7 +140,7 @@ def test_forward_rerank_full_size_sampled():
     from tests._parity import sample_rows
     inp = generate(CONFIGS["prefill64k"])
     wl = inp.wl
-    g = GpuRun(inp)
+    g = DeviceRun(inp)
     prob = oracle_for(inp)
     idx = torch.empty((wl.B, wl.H, wl.Nq, wl.K), dtype=torch.int32, device="cuda")
     fs.forward_rerank(g.p, g.Q, g.K, g.V, g.O, g.ws, idx=idx)

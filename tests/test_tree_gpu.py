@@ -14,7 +14,7 @@ import torch
 
 import long_context_sparse_head_b200 as fs
 from workloads import generate, small
-from tests._parity import TIE, TOL, GpuRun, expected_output, oracle_for, sample_rows
+from tests._parity import TIE, TOL, DeviceRun, expected_output, oracle_for, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -64,7 +64,7 @@ def check_tree(inp, prob, base, gidx, rows_bhr, beam, c_explore, tau):
 
 def run_tree(inp, beam, c_explore=1.0, tau_q=None, rows=None, forward=True):
     wl = inp.wl
-    g = GpuRun(inp)
+    g = DeviceRun(inp)
     prob = oracle_for(inp)
     base = oracle_for(inp, W=-1, P=-1)
     kb_o, am_o = prob.summaries()
@@ -120,7 +120,7 @@ def test_tree_exhaustive_beam_is_base_selection(tau_q):
     FS's eq. (7) top-K over C_i (checked against the oracle's base selection directly)."""
     inp = generate(small("tree_all", Nq=1536, Nk=1536, K=7, W=-1, P=-1, dtype="f32", seed=602))
     wl = inp.wl
-    g = GpuRun(inp)
+    g = DeviceRun(inp)
     base = oracle_for(inp)
     kb_o, am_o = base.summaries()
     tau = None if tau_q is None else pick_tau(am_o, tau_q)
@@ -138,7 +138,7 @@ def test_tree_exhaustive_beam_is_base_selection(tau_q):
 def test_tree_forest_for_other_sizes_is_reported():
     """A forest built for a shorter sequence is caught by the search kernel's check."""
     inp = generate(small("tree_chk", Nq=512, Nk=2048, K=4, W=-1, P=-1, dtype="f32", seed=603))
-    g = GpuRun(inp)
+    g = DeviceRun(inp)
     g.summaries()
     forest = fs.alloc_forest(g.p)
     short = fs.Params(B=1, H=2, Nq=512, Nk=1024, K=4, W=-1, P=-1, alpha=inp.alpha, dtype="f32")

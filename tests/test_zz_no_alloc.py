@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import long_context_sparse_head_b200 as fs
-from tests._parity import GpuRun
+from tests._parity import DeviceRun
 from workloads import CONFIGS, generate, small
 
 
@@ -27,7 +27,7 @@ def _problems():
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_selection_twice():
     for inp in _problems():          # two calls in a row: large problem, then small one
-        g = GpuRun(inp)
+        g = DeviceRun(inp)
         want = g.select().clone()    # fs_select_topk with a workspace
         got = torch.full_like(want, -7)
         fs.select_topk_noalloc(g.p, g.Q, g.kbar, g.amax, got)
@@ -39,7 +39,7 @@ def test_noalloc_matches_workspace_selection_twice():
 @pytest.mark.gpu
 def test_noalloc_full_size_prefill_matches():
     inp = generate(CONFIGS["prefill16k"])
-    g = GpuRun(inp)
+    g = DeviceRun(inp)
     want = g.select().clone()
     got = torch.full_like(want, -7)
     fs.select_topk_noalloc(g.p, g.Q, g.kbar, g.amax, got)
