@@ -20,7 +20,8 @@
 //
 // Kernels: prep (codes, admitted prefix counts, sequences; one CTA per head), merge (one
 // launch per level; each entry's place by binary search in the other half), nodes (one
-// warp per node: mean, radius, max norm, first cell), search (one warp per query row).
+// warp per node: mean, radius, max norm, first cell), search (one warp per query row; a
+// right child's q.mu is 2 q.mu_parent - q.mu_left, so an expansion reads one mean).
 #include <cmath>
 
 #include "fs_common.cuh"
@@ -242,8 +243,10 @@ struct SearchSmem {
     float U[kCandCap];
     int ref[kCandCap];      // level << 26 | node slot
     int pmin[kCandCap];
+    float dot[kCandCap];    // q . mu_v
     float bU[kMaxBeam];
     int bref[kMaxBeam], bpmin[kMaxBeam];
+    float bdot[kMaxBeam];
     float rU[2 * kMaxBeam];  // leaves both beams end on
     int rcell[2 * kMaxBeam];
 };
@@ -304,7 +307,7 @@ __device__ __forceinline__ void beam_cut(Smem &S, int n, int nb, int lane) {
         const int i = e * 32 + lane;
         U[e] = i < n ? S.U[i] : -INFINITY;
         pm[e] = i < n ? S.pmin[i] : 0x7fffffff;
-        rf[e] = i < n ? S.ref[i] : 0;
+        rf[e] = i < n ? i : 0;                        // the candidate's index
     }
     warp_sort<E>(U, pm, rf, lane);
 #pragma unroll
@@ -313,15 +316,28 @@ __device__ __forceinline__ void beam_cut(Smem &S, int n, int nb, int lane) {
         if (i < nb) {
             S.bU[i] = U[e];
             S.bpmin[i] = pm[e];
-            S.bref[i] = rf[e];
+            S.bref[i] = S.ref[rf[e]];
+            S.bdot[i] = S.dot[rf[e]];
         }
     }
 }
 
 // eq. (11) for one node (lane-local: the whole dot product in this lane)
+// eq. (11) for a node whose q . mu_v is known (meta loads only)
+template <bool PRIOR>
+__device__ __forceinline__ float node_U_dot(const Forest &F, size_t lvl_base, int node, float dot, float qn,
+                                            const SearchArgs &A, int h, int i, int *pmin_out) {
+    const float4 mt = __ldg(F.meta + lvl_base + node);
+    const int pmin = __float_as_int(mt.z);
+    *pmin_out = pmin;
+    float U = (dot + A.c_explore * qn * mt.x) * A.scale;
+    if (PRIOR) U += A.lambda[h] * mt.y * erff(((float)i - ((float)pmin + 0.5f) * kS) * A.inv2sigma[h]);
+    return U;
+}
+
 template <bool PRIOR>
 __device__ __forceinline__ float node_U(const Forest &F, size_t lvl_base, int node, const float *q, float qn,
-                                        const SearchArgs &A, int h, int i, int *pmin_out) {
+                                        const SearchArgs &A, int h, int i, int *pmin_out, float *dot_out) {
     const size_t ni = lvl_base + node;
     const float4 *mu = reinterpret_cast<const float4 *>(F.mu + ni * kD);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -333,12 +349,9 @@ __device__ __forceinline__ float node_U(const Forest &F, size_t lvl_base, int no
         acc[2] = fmaf(q[4 * e + 2], x.z, acc[2]);
         acc[3] = fmaf(q[4 * e + 3], x.w, acc[3]);
     }
-    const float4 mt = __ldg(F.meta + ni);
-    const int pmin = __float_as_int(mt.z);
-    *pmin_out = pmin;
-    float U = ((acc[0] + acc[1]) + (acc[2] + acc[3]) + A.c_explore * qn * mt.x) * A.scale;
-    if (PRIOR) U += A.lambda[h] * mt.y * erff(((float)i - ((float)pmin + 0.5f) * kS) * A.inv2sigma[h]);
-    return U;
+    const float dot = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    *dot_out = dot;
+    return node_U_dot<PRIOR>(F, lvl_base, node, dot, qn, A, h, i, pmin_out);
 }
 
 // beam search on one forest for a prefix of m entries; appends the final leaves to the
@@ -358,7 +371,9 @@ __device__ int search_forest(const Forest &F, SearchSmem &S, int bh, int f, int 
             const int slot = __popc(bal >> (k + 1));      // high bits first
             const int node = (((m >> k) - 1) << (k + 1)) + 1;
             int pm;
-            S.U[slot] = node_U<PRIOR>(F, F.lvl(bh, f, k) * 2 * C, node, S.q, qn, A, h, i, &pm);
+            float dt;
+            S.U[slot] = node_U<PRIOR>(F, F.lvl(bh, f, k) * 2 * C, node, S.q, qn, A, h, i, &pm, &dt);
+            S.dot[slot] = dt;
             S.ref[slot] = (k << 26) | node;
             S.pmin[slot] = pm;
         }
@@ -419,14 +434,21 @@ __device__ int search_forest(const Forest &F, SearchSmem &S, int bh, int f, int 
                 S.U[o] = S.bU[j];
                 S.ref[o] = ref;
                 S.pmin[o] = S.bpmin[j];
+                S.dot[o] = S.bdot[j];
             } else {
                 const size_t base = F.lvl(bh, f, k) * 2 * C;
                 const int c0 = node + v, c1 = node + v + 1;  // heap children 2v, 2v + 1
                 int p0, p1;
-                S.U[o] = node_U<PRIOR>(F, base, c0, S.q, qn, A, h, i, &p0);
+                // left child from its mean; the right child's mean is 2 mu_v - mu_left (both
+                // halves hold 2^(depth) leaves), so its dot needs no load of its mean
+                float d0;
+                S.U[o] = node_U<PRIOR>(F, base, c0, S.q, qn, A, h, i, &p0, &d0);
+                S.dot[o] = d0;
                 S.ref[o] = (k << 26) | c0;
                 S.pmin[o] = p0;
-                S.U[o + 1] = node_U<PRIOR>(F, base, c1, S.q, qn, A, h, i, &p1);
+                const float d1 = 2.f * S.bdot[j] - d0;
+                S.U[o + 1] = node_U_dot<PRIOR>(F, base, c1, d1, qn, A, h, i, &p1);
+                S.dot[o + 1] = d1;
                 S.ref[o + 1] = (k << 26) | c1;
                 S.pmin[o + 1] = p1;
             }
