@@ -11,13 +11,13 @@
 // U (|U| <= 128, ascending), two cells (64 keys) per chunk, each cell fetched by its own
 // 32-row TMA box; a row masks the cells it did not select (masked-dense on the tensor
 // cores).  Then the window runs over 64-key chunks.  Both softmaxes accumulate in tensor
-// memory: two S buffers in columns [0,64) and [64,128) (chunk c uses buffer c mod 2, and
-// its P overwrites the first 32 columns of that buffer), the readout's O in [128,192), the
-// window's O in [192,256).  With two S buffers the MMA warp computes S of chunk c+1 while
-// the softmax threads work on chunk c, and a softmax warp that finishes early can start
-// the next chunk while slower warps finish this one.  When the first window chunk arrives
-// the readout is finished: the softmax threads turn its O into alpha_h * RMSNorm(u) in
-// place, and the epilogue adds it to the window's output.  No intermediate leaves the SM.
+// memory: three S buffers in columns [0,64), [64,128) and [128,192) (chunk c uses buffer
+// c mod 3, and its P overwrites the first 32 columns of that buffer) and one O in
+// [192,256).  The MMA warp keeps Q K^T two chunks ahead of P V, so a softmax warp that
+// finishes early finds the next S ready while slower warps finish this chunk.  When the
+// first window chunk arrives the readout is finished: the softmax threads read its O,
+// keep alpha_h * RMSNorm(u) in registers (fp32), and the window's first P V overwrites O;
+// the epilogue adds the two.  No intermediate leaves the SM.
 //
 // Warpgroup 0 (warps 0-3): softmax, thread = query row = TMEM lane; it holds a chunk's
 // S row in registers (one TMEM wait per chunk), raised to 200 registers by setmaxnreg.
@@ -37,7 +37,8 @@ constexpr int CPC = BN / kS;                     // cells per readout chunk (2)
 constexpr int NSOFT = 4, W_TMA = 4, W_MMA = 5, W_AUX0 = 6, NWARPS = 8, NAUX = 64;
 constexpr int NTHREADS = NWARPS * 32;
 constexpr int REGS_SOFTMAX = 200, REGS_PRODUCER = 56;   // 128 * (200 + 56) = 256 * 128
-constexpr uint32_t TMEM_COLS = 256, OLR_COL = 128, OSR_COL = 192;   // S buffers at 0 and BN
+constexpr int NSBUF = 3;                        // S buffers (BN columns each) in tensor memory
+constexpr uint32_t TMEM_COLS = 256, O_COL = NSBUF * BN;   // S at 0, BN, 2 BN; O at 192
 constexpr int TILE_BYTES = BM * kD * 2;         // 128 x 64 bf16: 16 KiB
 constexpr int CHUNK_BYTES = BN * kD * 2;        // 64 x 64 bf16: 8 KiB
 constexpr int CELL_BYTES = kS * kD * 2;         // 32 x 64 bf16: 4 KiB
@@ -50,8 +51,9 @@ struct AttnSmem {
     __nv_bfloat16 v[NSTAGE][BN * kD];
     int ulist[UMAX];                            // union cells, ascending
     int nU;
-    uint64_t q_full, q_ready, u_ready, o_ready, o_done, drain;
-    uint64_t s_full[2], p_full[2];              // per S buffer
+    uint64_t q_full, q_ready, u_ready, o_done, drain;
+    uint64_t o_ready[2];                        // P V of chunk c completes phase c / 2 of [c % 2]
+    uint64_t s_full[NSBUF], p_full[NSBUF];      // per S buffer
     uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
     uint32_t tmem_base;
     int abort;
@@ -180,9 +182,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         tc::mbar_init(&sm.q_full, 1);
         tc::mbar_init(&sm.q_ready, NAUX);
         tc::mbar_init(&sm.u_ready, NAUX);
-        tc::mbar_init(&sm.o_ready, 1);
+        tc::mbar_init(&sm.o_ready[0], 1);
+        tc::mbar_init(&sm.o_ready[1], 1);
         tc::mbar_init(&sm.o_done, 1);
-        for (int b = 0; b < 2; b++) {
+        for (int b = 0; b < NSBUF; b++) {
             tc::mbar_init(&sm.s_full[b], 1);
             tc::mbar_init(&sm.p_full[b], NSOFT);       // one arrival per softmax warp
         }
@@ -287,7 +290,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 if (ok) chunk_range(nR, cb, ce);
                 const int total = ce - cb;
                 int issued = 0;
-                // S(c) = Q K(c)^T into buffer c mod 2, with the NoPE or the rotated Q
+                // S(c) = Q K(c)^T into buffer c mod 3, with the NoPE or the rotated Q
                 auto issue_qk = [&](int c) -> bool {
                     if (!tc::mbar_wait(&sm.kv_full[c % NSTAGE], (c / NSTAGE) & 1, ab)) return false;
                     const int g = cb + c;
@@ -297,28 +300,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     const uint64_t db = dk0 + (uint64_t)((c % NSTAGE) * kStageStep);
 #pragma unroll
                     for (int kk = 0; kk < kD / 16; kk++)      // K steps of 16 columns = 32 bytes
-                        tc::mma_ss(tmem + BN * (c & 1), da + 2 * kk, db + 2 * kk, id_qk, kk > 0 ? 1u : 0u);
-                    tc::mma_commit(&sm.s_full[c & 1]);
+                        tc::mma_ss(tmem + BN * (c % NSBUF), da + 2 * kk, db + 2 * kk, id_qk, kk > 0 ? 1u : 0u);
+                    tc::mma_commit(&sm.s_full[c % NSBUF]);
                     issued++;
                     return true;
                 };
                 if (ok && total > 0) ok = issue_qk(0);
+                if (ok && total > 1) ok = issue_qk(1);
                 for (int c = 0; ok && c < total; c++) {
-                    // S(c+1) goes into the other buffer while the softmax works on chunk c; the
-                    // buffer's previous P (chunk c-1) was consumed by a P V issued before this
-                    if (c + 1 < total && !issue_qk(c + 1)) { ok = false; break; }
-                    // O += P(c) V(c), into the readout's or the window's O
-                    if (!tc::mbar_wait(&sm.p_full[c & 1], (c >> 1) & 1, ab)) { ok = false; break; }
+                    // S(c+2) goes into the buffer of chunk c-1, whose P was consumed by a P V
+                    // issued before this, while the softmax works on chunks c and c+1
+                    if (c + 2 < total && !issue_qk(c + 2)) { ok = false; break; }
+                    // O += P(c) V(c); the first chunk of each branch overwrites O
+                    if (!tc::mbar_wait(&sm.p_full[c % NSBUF], (c / NSBUF) & 1, ab)) { ok = false; break; }
                     tc::tc_fence_after();
-                    const uint32_t ocol = cb + c < nR ? OLR_COL : OSR_COL;
                     const bool first = c == 0 || cb + c == nR;
                     const uint64_t db = dv0 + (uint64_t)((c % NSTAGE) * kStageStep);
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; kk++)      // K steps of 16 keys = 2048 bytes
-                        tc::mma_ts(tmem + ocol, tmem + BN * (c & 1) + 8 * kk, db + 128 * kk, id_pv,
+                        tc::mma_ts(tmem + O_COL, tmem + BN * (c % NSBUF) + 8 * kk, db + 128 * kk, id_pv,
                                    (!first || kk > 0) ? 1u : 0u);
                     tc::mma_commit(&sm.kv_empty[c % NSTAGE]);
-                    tc::mma_commit(&sm.o_ready);
+                    tc::mma_commit(&sm.o_ready[c & 1]);
                     issued++;
                 }
                 if (ok) tc::mma_commit(&sm.o_done);
@@ -345,37 +348,46 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         if (ok) chunk_range(nR, cb, ce);
         const int total = ce - cb;
         float m_lr = -INFINITY, l_lr = 0.f, m_sr = -INFINITY, l_sr = 0.f;
+        float y[kD];                            // alpha_h RMSNorm(u), once the readout is done
+#pragma unroll
+        for (int e = 0; e < kD; e++) y[e] = 0.f;
+        float *part_row = SPLIT ? A.part + ((((size_t)bh * gridDim.x + blockIdx.x) * S + sidx) * BM + row) * kPartStride
+                                : nullptr;
         for (int it = 0; ok && it < total; it++) {
             const int g = cb + it;
-            if (!tc::mbar_wait(&sm.s_full[it & 1], (it >> 1) & 1, ab)) { ok = false; break; }
+            if (!tc::mbar_wait(&sm.s_full[it % NSBUF], (it / NSBUF) & 1, ab)) { ok = false; break; }
             tc::tc_fence_after();
-            if (!SPLIT && g == nR && nR > 0) {   // readout done: O_lr <- alpha_h RMSNorm(O_lr / l)
-                // the last readout P V may still run (S of this chunk was issued before it)
-                if (!tc::mbar_wait(&sm.o_ready, (it - 1) & 1, ab)) { ok = false; break; }
+            if (g == nR && it > 0) {
+                // readout done (its last P V may still run): take its O out of tensor memory
+                // before the window's first P V overwrites it
+                if (!tc::mbar_wait(&sm.o_ready[(it - 1) & 1], ((it - 1) >> 1) & 1, ab)) { ok = false; break; }
                 tc::tc_fence_after();
-                uint32_t a[32], b[32];
-                tc::tmem_ld32(trow + OLR_COL, a);
-                tc::tmem_ld32(trow + OLR_COL + 32, b);
+                uint32_t a[kD];
+                tc::tmem_ld32(trow + O_COL, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+                tc::tmem_ld32(trow + O_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
                 tc::tmem_wait_ld();
-                const float inv_l = l_lr > 0.f ? 1.f / l_lr : 0.f;
-                float ss = 0.f;
+                if (SPLIT) {                    // the readout's partial state, unnormalised
+                    float4 *d4 = reinterpret_cast<float4 *>(part_row + 4);
 #pragma unroll
-                for (int e = 0; e < 32; e++) {
-                    const float x = __uint_as_float(a[e]) * inv_l, y = __uint_as_float(b[e]) * inv_l;
-                    ss = fmaf(x, x, fmaf(y, y, ss));
-                }
-                const float f = l_lr > 0.f ? A.alpha[h] * inv_l / sqrtf(ss * (1.f / kD) + A.rms_eps) : 0.f;
+                    for (int q = 0; q < kD / 4; q++)
+                        d4[q] = make_float4(__uint_as_float(a[4 * q]), __uint_as_float(a[4 * q + 1]),
+                                            __uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3]));
+                } else {                        // O_lr <- alpha_h RMSNorm(O_lr / l)
+                    const float inv_l = l_lr > 0.f ? 1.f / l_lr : 0.f;
+                    float ss = 0.f;
 #pragma unroll
-                for (int e = 0; e < 32; e++) {
-                    a[e] = __float_as_uint(__uint_as_float(a[e]) * f);
-                    b[e] = __float_as_uint(__uint_as_float(b[e]) * f);
+                    for (int e = 0; e < kD; e++) {
+                        const float x = __uint_as_float(a[e]) * inv_l;
+                        ss = fmaf(x, x, ss);
+                    }
+                    const float f = l_lr > 0.f ? A.alpha[h] * inv_l / sqrtf(ss * (1.f / kD) + A.rms_eps) : 0.f;
+#pragma unroll
+                    for (int e = 0; e < kD; e++) y[e] = __uint_as_float(a[e]) * f;
                 }
-                tc::tmem_st32(trow + OLR_COL, a);
-                tc::tmem_st32(trow + OLR_COL + 32, b);
             }
             // one call site for every kind of chunk keeps the unrolled body in the code once
             int kind, lo = 0, width = BN;
-            uint32_t sel = 0u, ocol;
+            uint32_t sel = 0u;
             bool first;
             float m, l;
             if (g < nR) {
@@ -383,70 +395,62 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 const int wsel = p0 >> 5;           // word of the row's union mask, in registers
                 const uint32_t mw = wsel == 0 ? m4.x : wsel == 1 ? m4.y : wsel == 2 ? m4.z : m4.w;
                 sel = (mw >> (p0 & 31)) & ((1u << CPC) - 1u);
-                kind = CELLS; ocol = OLR_COL; first = it == 0; m = m_lr; l = l_lr;
+                kind = CELLS; first = it == 0; m = m_lr; l = l_lr;
             } else {
                 const int jc = jbase + BN * (k_first + g - nR);
                 const int clo = max(-jc, i - A.w - jc), chi = min(i - jc, BN - 1);
                 lo = clo;
                 width = rvalid ? max(0, chi - clo + 1) : 0;
                 kind = __all_sync(kFull, clo <= 0 && chi >= BN - 1 && rvalid) ? FULL : BAND;
-                ocol = OSR_COL; first = g == nR || it == 0; m = m_sr; l = l_sr;
+                first = g == nR || it == 0; m = m_sr; l = l_sr;
             }
-            const float corr = softmax_chunk(trow + BN * (it & 1), kind, sel, lo, width, A.scale_log2e, m, l);
+            const float corr = softmax_chunk(trow + BN * (it % NSBUF), kind, sel, lo, width, A.scale_log2e, m, l);
             if (g < nR) { m_lr = m; l_lr = l; } else { m_sr = m; l_sr = l; }
             // O rescale, after the exponentials (S no longer occupies registers); the P V of
             // the previous chunk, which accumulates into the same O, must have finished
             if (!first && __any_sync(kFull, corr != 1.f)) {
-                if (!tc::mbar_wait(&sm.o_ready, (it - 1) & 1, ab)) { ok = false; break; }
+                if (!tc::mbar_wait(&sm.o_ready[(it - 1) & 1], ((it - 1) >> 1) & 1, ab)) { ok = false; break; }
                 tc::tc_fence_after();
 #pragma unroll
                 for (int b = 0; b < kD / 32; b++) {
                     uint32_t r[32];
-                    tc::tmem_ld32(trow + ocol + 32 * b, r);
+                    tc::tmem_ld32(trow + O_COL + 32 * b, r);
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; e++) r[e] = __float_as_uint(__uint_as_float(r[e]) * corr);
-                    tc::tmem_st32(trow + ocol + 32 * b, r);
+                    tc::tmem_st32(trow + O_COL + 32 * b, r);
                 }
             }
             tc::tmem_wait_st();
             tc::tc_fence_before();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&sm.p_full[it & 1]);
+            if (lane == 0) tc::mbar_arrive(&sm.p_full[it % NSBUF]);
         }
-        if (SPLIT && ok && tc::mbar_wait(&sm.o_done, 0, ab)) {
-            // partial state of this CTA's chunks; a branch it had no chunk of stays empty
+        if (ok && tc::mbar_wait(&sm.o_done, 0, ab)) {
             tc::tc_fence_after();
-            const bool had_lr = cb < nR && ce > cb, had_sr = ce > nR && ce > cb;
-            float *dst = A.part + ((((size_t)bh * gridDim.x + blockIdx.x) * S + sidx) * BM + row) * kPartStride;
-            *reinterpret_cast<float4 *>(dst) = make_float4(had_lr ? m_lr : -INFINITY, had_lr ? l_lr : 0.f,
-                                                           had_sr ? m_sr : -INFINITY, had_sr ? l_sr : 0.f);
-#pragma unroll
-            for (int br = 0; br < 2; br++) {
-                const bool had = br == 0 ? had_lr : had_sr;
-                uint32_t a[64];
-                tc::tmem_ld32(trow + (br == 0 ? OLR_COL : OSR_COL), *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-                tc::tmem_ld32(trow + (br == 0 ? OLR_COL : OSR_COL) + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
-                tc::tmem_wait_ld();
-                float4 *d4 = reinterpret_cast<float4 *>(dst + 4 + br * kD);
-#pragma unroll
-                for (int q = 0; q < kD / 4; q++)
-                    d4[q] = had ? make_float4(__uint_as_float(a[4 * q]), __uint_as_float(a[4 * q + 1]),
-                                              __uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3]))
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        } else if (!SPLIT && ok && tc::mbar_wait(&sm.o_done, 0, ab)) {
-            tc::tc_fence_after();
-            const float inv = l_sr > 0.f ? 1.f / l_sr : 0.f;
-            uint32_t a[64], b[64];
-            tc::tmem_ld32(trow + OSR_COL, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-            tc::tmem_ld32(trow + OSR_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
-            if (nR > 0) {
-                tc::tmem_ld32(trow + OLR_COL, *reinterpret_cast<uint32_t(*)[32]>(&b[0]));
-                tc::tmem_ld32(trow + OLR_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&b[32]));
-            }
+            uint32_t a[kD];
+            tc::tmem_ld32(trow + O_COL, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+            tc::tmem_ld32(trow + O_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
             tc::tmem_wait_ld();
-            if (rvalid) {
+            if (SPLIT) {
+                // partial state of this CTA's chunks; a branch it had no chunk of stays empty.
+                // O holds the window's sum if the CTA had window chunks, else the readout's.
+                const bool had_lr = cb < nR && ce > cb, had_sr = ce > nR && ce > cb;
+                *reinterpret_cast<float4 *>(part_row) = make_float4(had_lr ? m_lr : -INFINITY, had_lr ? l_lr : 0.f,
+                                                                    had_sr ? m_sr : -INFINITY, had_sr ? l_sr : 0.f);
+                float4 *d_lr = reinterpret_cast<float4 *>(part_row + 4);
+                float4 *d_sr = reinterpret_cast<float4 *>(part_row + 4 + kD);
+#pragma unroll
+                for (int q = 0; q < kD / 4; q++) {
+                    const float4 v = make_float4(__uint_as_float(a[4 * q]), __uint_as_float(a[4 * q + 1]),
+                                                 __uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3]));
+                    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+                    d_sr[q] = had_sr ? v : z;
+                    if (!had_lr) d_lr[q] = z;
+                    else if (!had_sr) d_lr[q] = v;      // else written when the window began
+                }
+            } else if (rvalid) {
+                const float inv = l_sr > 0.f ? 1.f / l_sr : 0.f;
                 uint4 *dst = reinterpret_cast<uint4 *>(O + ((size_t)bh * A.Nq + r0 + row) * kD);
 #pragma unroll
                 for (int q = 0; q < 8; q++) {
@@ -454,12 +458,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
                         const int j = 8 * q + 2 * e;
-                        float o0 = __uint_as_float(a[j]) * inv, o1 = __uint_as_float(a[j + 1]) * inv;
-                        if (nR > 0) {
-                            o0 += __uint_as_float(b[j]);
-                            o1 += __uint_as_float(b[j + 1]);
-                        }
-                        w4[e] = tc::pack_bf16x2(o0, o1);
+                        w4[e] = tc::pack_bf16x2(fmaf(__uint_as_float(a[j]), inv, y[j]),
+                                                fmaf(__uint_as_float(a[j + 1]), inv, y[j + 1]));
                     }
                     dst[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }

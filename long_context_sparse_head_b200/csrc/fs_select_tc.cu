@@ -13,9 +13,12 @@
 // 128-byte-swizzled layout of a K-major MMA operand.  One thread issues
 // S = Q (hi + mid + lo)^T (M = 128, N = |U| rounded up to 16) into tensor memory.  Each
 // thread then takes its row's scores, keeps the admitted ones and finds the K-th largest
-// by bisection on order-preserving integer keys whose low 7 bits carry (127 - position):
-// keys are unique, and among scores that agree to 2^-17 relative the lower cell index
-// wins, inside the 1e-4 near-tie tolerance of the selection check.
+// by bisection on integer keys: the score's 24-bit fixed-point place within the row's
+// admitted range, above 7 bits of (127 - position).  Keys are unique, and among scores
+// within 2^-24 of the row's range of each other the lower cell index wins, inside the
+// near-tie tolerance of the selection check.  The search stops once exactly K keys
+// remain; keys spread over one range per row separate in far fewer halvings than
+// order-preserving bit patterns of the raw fp32 scores.
 // Outputs: idx (selected cells per row, ascending, -1 padded) and/or, for the fused
 // kernel, one compact record per tile: each row's selected union positions as a 128-bit
 // mask, the union's cells and its size.
@@ -54,11 +57,6 @@ struct SelArgs {
 
 __device__ __forceinline__ void sel_sync() {
     asm volatile("bar.sync %0, %1;" ::"n"(kSelBarrier), "n"(128) : "memory");
-}
-
-__device__ __forceinline__ uint32_t order_key(float f) {
-    const uint32_t b = __float_as_uint(f);
-    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
 __device__ __forceinline__ void split3(float x, __nv_bfloat16 &hi, __nv_bfloat16 &mid, __nv_bfloat16 &lo) {
@@ -257,9 +255,10 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
             for (int b = 0; b < UM / 16; b++)
                 if (16 * b < N) tc::tmem_ld16(trow + 16 * b, &key[16 * b]);
             tc::tmem_wait_ld();
-            uint32_t kmn[8], kmx[8];
+            // scores r_ic, and their range over the admitted cells
+            float fmn[4], fmx[4];
 #pragma unroll
-            for (int k = 0; k < 8; k++) { kmn[k] = 0xffffffffu; kmx[k] = 0u; }
+            for (int k = 0; k < 4; k++) { fmn[k] = INFINITY; fmx[k] = -INFINITY; }
 #pragma unroll
             for (int u = 0; u < UM; u++) {
                 if (16 * (u / 16) < N) {
@@ -268,20 +267,31 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                         const float pc = (float)(sm.ulist[u] * kS) + 0.5f * kS;
                         sc += lam * sm.acell[u] * erff(((float)i - pc) * i2s);
                     }
-                    const uint32_t k = ((aw[u >> 5] >> (u & 31)) & 1u) ? (order_key(sc) & ~0x7fu) | (uint32_t)(127 - u) : 0u;
-                    key[u] = k;
-                    kmn[u & 7] = min(kmn[u & 7], k ? k : 0xffffffffu);
-                    kmx[u & 7] = max(kmx[u & 7], k);
+                    const bool adm = (aw[u >> 5] >> (u & 31)) & 1u;
+                    key[u] = __float_as_uint(sc);
+                    fmn[u & 3] = adm ? fminf(fmn[u & 3], sc) : fmn[u & 3];
+                    fmx[u & 3] = adm ? fmaxf(fmx[u & 3], sc) : fmx[u & 3];
+                }
+            }
+            const float mn = fminf(fminf(fmn[0], fmn[1]), fminf(fmn[2], fmn[3]));
+            const float span = fmaxf(fmaxf(fmx[0], fmx[1]), fmaxf(fmx[2], fmx[3])) - mn;
+            const float q24 = span > 0.f ? 16777215.f / span : 0.f;
+            // integer keys: 1 + the score's 24-bit fixed-point place in the row's range, then
+            // 7 bits of (127 - position); 0 for a cell that is not admitted
+#pragma unroll
+            for (int u = 0; u < UM; u++) {
+                if (16 * (u / 16) < N) {
+                    const bool adm = (aw[u >> 5] >> (u & 31)) & 1u;
+                    const uint32_t fx = min(__float2uint_rz((__uint_as_float(key[u]) - mn) * q24), 0xffffffu);
+                    key[u] = adm ? ((fx + 1u) << 7) | (uint32_t)(127 - u) : 0u;
                 } else {
                     key[u] = 0u;
                 }
             }
-            const uint32_t kmin = min(min(min(kmn[0], kmn[1]), min(kmn[2], kmn[3])), min(min(kmn[4], kmn[5]), min(kmn[6], kmn[7])));
-            const uint32_t kmax = max(max(max(kmx[0], kmx[1]), max(kmx[2], kmx[3])), max(max(kmx[4], kmx[5]), max(kmx[6], kmx[7])));
             // K-th largest key by bisection: count(key >= lo) >= K > count(key >= hi)
             uint32_t tau = 1u;
             if (na > A.K) {
-                uint32_t lo = kmin, hi = kmax + 1u;
+                uint32_t lo = 1u << 7, hi = (0x1000000u + 1u) << 7;
                 while (hi - lo > 1u) {
                     const uint32_t mid = lo + ((hi - lo) >> 1);
                     int cp[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent partial counts
