@@ -72,6 +72,7 @@ WsLayout layout(const fs_params *p) {
     const int kr0 = p->Nk - p->Nq - p->w > 0 ? p->Nk - p->Nq - p->w : 0;   // first rotated key
     L.krot = off;  off += align256(BH * (size_t)(p->Nk - kr0) * kD * 2);
     L.part = off;  off += align256(attn_part_bytes(p));      // split CTAs' partial states (decoding)
+    L.tlist = off; off += align256(BH * (size_t)exit_list_words(p->P) * 4);   // TopP member lists (decoding)
     L.total = off;
     return L;
 }
@@ -151,9 +152,10 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
             amax = am;
         }
         int *exitn = at<int>(ws, L.exitn);
-        if (D.prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
+        int *tlist = D.prune && exit_list_mode(D) ? at<int>(ws, L.tlist) : nullptr;
+        if (D.prune && launch_exit_times(D, amax, exitn, st, tlist) != cudaSuccess) return FS_ERR_CUDA;
         uint32_t *tiles = at<uint32_t>(ws, L.tiles);
-        if (launch_select_tc(D, Q, kbar, amax, exitn, nullptr, tiles, at<int>(ws, L.flag), st) != cudaSuccess)
+        if (launch_select_tc(D, Q, kbar, amax, exitn, nullptr, tiles, at<int>(ws, L.flag), st, tlist) != cudaSuccess)
             return FS_ERR_CUDA;
         if (!fk.close(st, rs)) return FS_ERR_CUDA;
         return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), at<float>(ws, L.part),

@@ -35,7 +35,7 @@ struct Dev {
 
 // Workspace layout (byte offsets from ws; each segment 256-byte aligned).
 struct WsLayout {
-    size_t flag, exitn, kbar, amax, idx, olr, rope, tiles, rope_abs, krot, part, total;
+    size_t flag, exitn, kbar, amax, idx, olr, rope, tiles, rope_abs, krot, part, tlist, total;
 };
 
 // Per-tile selection record passed from the tensor-core selection kernel to the fused
@@ -149,7 +149,13 @@ bool params_have_long_range(const fs_params *p);
 // ---- launchers (one per kernel file) ----
 cudaError_t launch_summaries(const Dev &P, fs_dtype dt, const void *K, float *kbar,
                              float *amax, cudaStream_t st);
-cudaError_t launch_exit_times(const Dev &P, const float *amax, int *exitn, cudaStream_t st);
+// exit times; for a call whose queries span few prefixes (decoding) the table is only right
+// at the asked prefixes, and with tlist the kernel also lists, per (b, h), the cells that are
+// TopP members at one of them: tlist[0] = their count, then the cells (unordered)
+bool exit_list_mode(const Dev &P);
+int exit_list_words(int P);                      // per (b, h)
+cudaError_t launch_exit_times(const Dev &P, const float *amax, int *exitn, cudaStream_t st,
+                              int *tlist = nullptr);
 // eq. (12) token-level rerank of the selection (CUDA cores, |A_i| <= 128)
 bool rerank_supported(const fs_params *p);
 cudaError_t launch_rerank(const Dev &P, fs_dtype dt, const void *Q, const void *K, const float *kbar,
@@ -182,9 +188,11 @@ cudaError_t launch_rope_keys(const Dev &P, const void *K, void *Krot, const floa
                              cudaStream_t st);
 // tensor-core selection (bf16): scores against the bf16x3 split of the mean keys
 bool select_tc_supported(const fs_params *p);
+// (tlist: the exit-times kernel's member lists, when it wrote them: the union is then built
+// from them and the recent cells instead of a scan of the whole exit table)
 cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, const float *amax,
                              const int *exitn, int32_t *idx, uint32_t *tiles, int *dev_flag,
-                             cudaStream_t st);
+                             cudaStream_t st, const int *tlist = nullptr);
 // selection with whichever kernel applies (tensor cores for bf16 when supported)
 cudaError_t launch_selection(const fs_params *p, const Dev &D, const void *Q, const float *kbar,
                              const float *amax, const int *exitn, int32_t *idx, int *dev_flag,

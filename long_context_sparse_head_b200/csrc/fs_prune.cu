@@ -82,7 +82,8 @@ __device__ __forceinline__ uint32_t order_key(float a) {
 
 __global__ void __launch_bounds__(kRangeThreads) topp_range_kernel(const float *__restrict__ amax,
                                                                    int *__restrict__ exitn, int C, int P,
-                                                                   int n_lo, int n_hi) {
+                                                                   int n_lo, int n_hi, int *__restrict__ tlist,
+                                                                   int tl_words) {
     extern __shared__ uint32_t list[];           // TopP members: keys [P], then cells [P]
     __shared__ int hist[256];
     __shared__ int wsum[kRangeThreads / 32];
@@ -93,6 +94,7 @@ __global__ void __launch_bounds__(kRangeThreads) topp_range_kernel(const float *
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const float *a = amax + (size_t)blockIdx.x * C;
     int *ex = exitn + (size_t)blockIdx.x * C;
+    int *tl = tlist ? tlist + (size_t)blockIdx.x * tl_words : nullptr;   // [0] count, then cells
     for (int c = t; c < C; c += kRangeThreads) ex[c] = c + 1;
     const int n0 = min(n_lo, C), m0 = min(P, n0);  // |TopP(n0)| = m0
     if (t == 0) s_count = 0;
@@ -173,6 +175,7 @@ __global__ void __launch_bounds__(kRangeThreads) topp_range_kernel(const float *
                 lkey[slot] = k;
                 lidx[slot] = c;
                 ex[c] = kNever;
+                if (tl) tl[1 + slot] = c;
             }
             eq_before += tot;
             __syncthreads();
@@ -180,7 +183,7 @@ __global__ void __launch_bounds__(kRangeThreads) topp_range_kernel(const float *
     }
     __syncthreads();
     if (warp == 0) {   // prefixes n0 + 1 .. n_hi, one joining cell each
-        int cnt = s_count;
+        int cnt = s_count, nl = s_count;        // members now; cells listed
         for (int n = n0 + 1; n <= n_hi && n <= C; n++) {
             const int c = n - 1;
             const uint32_t kc = order_key(__ldg(a + c));
@@ -189,7 +192,9 @@ __global__ void __launch_bounds__(kRangeThreads) topp_range_kernel(const float *
                     lkey[cnt] = kc;
                     lidx[cnt] = c;
                     ex[c] = kNever;
+                    if (tl) tl[1 + nl] = c;
                 }
+                nl++;
                 cnt++;
                 __syncwarp();
                 continue;
@@ -212,21 +217,32 @@ __global__ void __launch_bounds__(kRangeThreads) topp_range_kernel(const float *
                 lkey[ws] = kc;
                 lidx[ws] = c;
                 ex[c] = kNever;
+                if (tl) tl[1 + nl] = c;
             }
+            nl += kc > wk;
             __syncwarp();
         }
+        if (tl && lane == 0) tl[0] = nl;
     }
 }
 
-cudaError_t launch_exit_times(const Dev &P, const float *amax, int *exitn, cudaStream_t st) {
+bool exit_list_mode(const Dev &P) {
+    if (!(P.P > 0 && P.Nq > 0 && P.B * P.H * P.C > 0)) return false;
+    const int n_lo = cand_count(P.q0, P.w, P.C), n_hi = cand_count(P.q0 + P.Nq - 1, P.w, P.C);
+    return n_hi - n_lo <= kRangeMaxSteps;
+}
+
+int exit_list_words(int P) { return 1 + (P > 0 ? P : 0) + kRangeMaxSteps; }
+
+cudaError_t launch_exit_times(const Dev &P, const float *amax, int *exitn, cudaStream_t st, int *tlist) {
     const long long ncell = (long long)P.B * P.H * P.C;
     if (ncell == 0) return cudaSuccess;
     if (P.P > 0 && P.Nq > 0) {
         const int n_lo = cand_count(P.q0, P.w, P.C), n_hi = cand_count(P.q0 + P.Nq - 1, P.w, P.C);
         if (n_hi - n_lo <= kRangeMaxSteps) {
             LaunchScope scope(kExitTimes, st);
-            topp_range_kernel<<<(unsigned)(P.B * P.H), kRangeThreads, (size_t)P.P * 8, st>>>(amax, exitn, P.C, P.P,
-                                                                                               n_lo, n_hi);
+            topp_range_kernel<<<(unsigned)(P.B * P.H), kRangeThreads, (size_t)P.P * 8, st>>>(
+                amax, exitn, P.C, P.P, n_lo, n_hi, tlist, exit_list_words(P.P));
             return cudaGetLastError();
         }
     }

@@ -7,7 +7,9 @@
 // One CTA per 128 query rows of a (batch, head).  The rows of a tile have at most five
 // distinct candidate prefixes n (a prefix grows by one cell every s = 32 positions), so
 // U = union of their admitted sets is at most W + P + 10 cells (<= 128 here).  Warps 0-3
-// build U from the TopP exit table (ordered compaction), then stage the fp32 mean keys of
+// build U from the TopP exit table (ordered compaction; when decoding, from the exit-times
+// kernel's list of the cells that are TopP members at an asked prefix plus the recent
+// cells, so the whole table is not scanned), then stage the fp32 mean keys of
 // U as three bf16 parts hi + mid + lo (the split carries the fp32 mantissa, so the bf16
 // tensor-core products sum to the fp32 dot product up to accumulation rounding), in the
 // 128-byte-swizzled layout of a K-major MMA operand.  One thread issues
@@ -41,7 +43,7 @@ template <int UM> struct SelSmem {       // UM: capacity of the union (a multipl
     uint8_t amask[UM];                     // bit g: admitted for prefix n_min + g
     uint32_t admit[5][(UM + 31) / 32];     // per prefix n_min + g: admitted union positions
     int warp_cnt[4];
-    int nU;
+    int nU, ncand;
     uint64_t q_full, kb_ready, s_full, drain;
     uint32_t tmem_base;
     int abort;
@@ -49,6 +51,7 @@ template <int UM> struct SelSmem {       // UM: capacity of the union (a multipl
 
 struct SelArgs {
     int Nq, Nk, q0, w, C, K, W, P, H;
+    int tl_words;           // words per (b, h) of the member lists (with tlist)
     int prune, has_prior;
     float scale;
     float lambda[FS_MAX_HEADS];
@@ -73,7 +76,8 @@ template <bool PRIOR, int UM>
 __global__ void __launch_bounds__(NTHREADS, UM <= 80 ? 3 : 2)
 select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const float *__restrict__ kbar,
                  const float *__restrict__ amax, const int *__restrict__ exitn,
-                 int32_t *__restrict__ idx, uint32_t *__restrict__ tiles, int *dev_flag) {
+                 int32_t *__restrict__ idx, uint32_t *__restrict__ tiles, int *dev_flag,
+                 const int *__restrict__ tlist) {
     extern __shared__ uint8_t smraw[];
     const uint32_t sbase = tc::smem_u32(smraw);
     SelSmem<UM> &sm = *reinterpret_cast<SelSmem<UM> *>(smraw + (((sbase + 1023u) & ~1023u) - sbase));
@@ -136,60 +140,125 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
         const float *am = amax + (size_t)bh * A.C;
         const int ng = n_max - n_min;   // <= 4
         int total = 0;
-        // 1024 cells per round, eight consecutive ones per thread: the exit times are
-        // fetched with two 16-byte loads before any of them is used, then one block-wide
-        // exclusive scan orders the members
-        for (int c0 = 0; c0 < n_max; c0 += 1024) {
-            const int cb = c0 + 8 * t;
-            int e8[8];
-            if (A.prune && cb + 8 <= n_max && (reinterpret_cast<uintptr_t>(ex + cb) & 15) == 0) {
-                const int4 x0 = __ldg(reinterpret_cast<const int4 *>(ex + cb));
-                const int4 x1 = __ldg(reinterpret_cast<const int4 *>(ex + cb) + 1);
-                e8[0] = x0.x; e8[1] = x0.y; e8[2] = x0.z; e8[3] = x0.w;
-                e8[4] = x1.x; e8[5] = x1.y; e8[6] = x1.z; e8[7] = x1.w;
-            } else {
+        // admission bits of cell c (exit time e) for the prefixes n_min + g
+        auto admit_bits = [&](int c, int e) {
+            uint32_t m = 0;
 #pragma unroll
-                for (int j = 0; j < 8; j++) e8[j] = (A.prune && cb + j < n_max) ? ex[cb + j] : 0;
+            for (int g = 0; g <= 4; g++) {
+                const int n = n_min + g;
+                if (g <= ng && c < n && (!A.prune || c >= n - A.W || n < e)) m |= 1u << g;
             }
-            uint32_t amk[8];
-            int cnt = 0;
-#pragma unroll
-            for (int j = 0; j < 8; j++) {
-                const int c = cb + j;
-                amk[j] = 0;
-#pragma unroll
-                for (int g = 0; g <= 4; g++) {
-                    const int n = n_min + g;
-                    if (g <= ng && c < n && (!A.prune || c >= n - A.W || n < e8[j])) amk[j] |= 1u << g;
-                }
-                cnt += amk[j] != 0;
-            }
-            int incl = cnt;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(kFull, incl, o);
-                if (lane >= o) incl += y;
-            }
-            if (lane == 31) sm.warp_cnt[warp] = incl;
+            return m;
+        };
+        if (tlist) {
+            // decoding: the candidates are the cells listed as TopP members at an asked prefix
+            // and the recent cells [n_min - W, n_max); listed cells older than that range are
+            // ordered by counting, and the recent ones follow in index order
+            const int *tl = tlist + (size_t)bh * A.tl_words;
+            const int nl = min(__ldg(tl), A.tl_words - 1);
+            const int rlo = max(0, n_min - A.W);
+            int *cand = reinterpret_cast<int *>(sm.kb[0]);             // scratch until staging
+            uint8_t *cmask = reinterpret_cast<uint8_t *>(sm.kb[1]);
+            if (t == 0) sm.ncand = 0;
             sel_sync();
-            int pos = total + incl - cnt, tot = 0;
-            for (int k = 0; k < 4; k++) {
-                if (k < warp) pos += sm.warp_cnt[k];
-                tot += sm.warp_cnt[k];
-            }
-#pragma unroll
-            for (int j = 0; j < 8; j++) {
-                if (amk[j]) {
-                    if (pos < UM) {
-                        sm.ulist[pos] = cb + j;
-                        sm.amask[pos] = (uint8_t)amk[j];
-                        sm.acell[pos] = A.has_prior ? am[cb + j] : 0.f;
+            for (int j = t; j < nl; j += 128) {
+                const int c = __ldg(tl + 1 + j);
+                if (c >= 0 && c < rlo) {
+                    const uint32_t m = admit_bits(c, ex[c]);
+                    if (m) {
+                        const int slot = atomicAdd(&sm.ncand, 1);
+                        cand[slot] = c;
+                        cmask[slot] = (uint8_t)m;
                     }
-                    pos++;
                 }
             }
-            total += tot;
             sel_sync();
+            const int nc = sm.ncand;
+            for (int j = t; j < nc; j += 128) {
+                const int c = cand[j];
+                int rank = 0;
+                for (int x = 0; x < nc; x++) rank += cand[x] < c;
+                if (rank < UM) {
+                    sm.ulist[rank] = c;
+                    sm.amask[rank] = cmask[j];
+                    sm.acell[rank] = A.has_prior ? am[c] : 0.f;
+                }
+            }
+            if (warp == 0) {
+                int pos = nc;
+                for (int c0 = rlo; c0 < n_max; c0 += 32) {
+                    const int c = c0 + lane;
+                    const uint32_t m = c < n_max ? admit_bits(c, __ldg(ex + c)) : 0u;
+                    const unsigned bal = __ballot_sync(kFull, m != 0u);
+                    const int p = pos + __popc(bal & ((1u << lane) - 1u));
+                    if (m && p < UM) {
+                        sm.ulist[p] = c;
+                        sm.amask[p] = (uint8_t)m;
+                        sm.acell[p] = A.has_prior ? am[c] : 0.f;
+                    }
+                    pos += __popc(bal);
+                }
+                if (lane == 0) sm.warp_cnt[0] = pos;
+            }
+            sel_sync();
+            total = sm.warp_cnt[0];
+            sel_sync();
+        } else {
+            // 1024 cells per round, eight consecutive ones per thread: the exit times are
+            // fetched with two 16-byte loads before any of them is used, then one block-wide
+            // exclusive scan orders the members
+            for (int c0 = 0; c0 < n_max; c0 += 1024) {
+                const int cb = c0 + 8 * t;
+                int e8[8];
+                if (A.prune && cb + 8 <= n_max && (reinterpret_cast<uintptr_t>(ex + cb) & 15) == 0) {
+                    const int4 x0 = __ldg(reinterpret_cast<const int4 *>(ex + cb));
+                    const int4 x1 = __ldg(reinterpret_cast<const int4 *>(ex + cb) + 1);
+                    e8[0] = x0.x; e8[1] = x0.y; e8[2] = x0.z; e8[3] = x0.w;
+                    e8[4] = x1.x; e8[5] = x1.y; e8[6] = x1.z; e8[7] = x1.w;
+                } else {
+    #pragma unroll
+                    for (int j = 0; j < 8; j++) e8[j] = (A.prune && cb + j < n_max) ? ex[cb + j] : 0;
+                }
+                uint32_t amk[8];
+                int cnt = 0;
+    #pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    const int c = cb + j;
+                    amk[j] = 0;
+    #pragma unroll
+                    for (int g = 0; g <= 4; g++) {
+                        const int n = n_min + g;
+                        if (g <= ng && c < n && (!A.prune || c >= n - A.W || n < e8[j])) amk[j] |= 1u << g;
+                    }
+                    cnt += amk[j] != 0;
+                }
+                int incl = cnt;
+    #pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(kFull, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                if (lane == 31) sm.warp_cnt[warp] = incl;
+                sel_sync();
+                int pos = total + incl - cnt, tot = 0;
+                for (int k = 0; k < 4; k++) {
+                    if (k < warp) pos += sm.warp_cnt[k];
+                    tot += sm.warp_cnt[k];
+                }
+    #pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    if (amk[j]) {
+                        if (pos < UM) {
+                            sm.ulist[pos] = cb + j;
+                            sm.amask[pos] = (uint8_t)amk[j];
+                            sm.acell[pos] = A.has_prior ? am[cb + j] : 0.f;
+                        }
+                        pos++;
+                    }
+                }
+                total += tot;
+                sel_sync();
+            }
         }
         if (t == 0) {
             sm.nU = min(total, UM);
@@ -353,19 +422,19 @@ namespace {
 int union_bound(const Dev &P) { return P.prune ? P.W + P.P + 10 : P.C; }
 template <int UM> cudaError_t launch_um(const CUtensorMap &tq, const SelArgs &A, bool prior, dim3 grid,
                                          const float *kbar, const float *amax, const int *exitn, int32_t *idx,
-                                         uint32_t *tiles, int *dev_flag, cudaStream_t st) {
+                                         uint32_t *tiles, int *dev_flag, const int *tlist, cudaStream_t st) {
     const size_t smem = sizeof(SelSmem<UM>) + 1024;
     // the erf prior is a separate instantiation: without it the unrolled score loop stays small
     auto kern = prior ? select_tc_kernel<true, UM> : select_tc_kernel<false, UM>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<grid, NTHREADS, smem, st>>>(tq, A, kbar, amax, exitn, idx, tiles, dev_flag);
+    kern<<<grid, NTHREADS, smem, st>>>(tq, A, kbar, amax, exitn, idx, tiles, dev_flag, tlist);
     return cudaGetLastError();
 }
 }  // namespace
 
 cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, const float *amax,
                              const int *exitn, int32_t *idx, uint32_t *tiles, int *dev_flag,
-                             cudaStream_t st) {
+                             cudaStream_t st, const int *tlist) {
     if (P.Nq == 0) return cudaSuccess;
     const int BH = P.B * P.H;
     CUtensorMap tq;
@@ -374,6 +443,8 @@ cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, con
     A.Nq = P.Nq; A.Nk = P.Nk; A.q0 = P.q0; A.w = P.w; A.C = P.C; A.K = P.K;
     A.W = P.W; A.P = P.P; A.H = P.H; A.prune = P.prune; A.has_prior = P.has_prior;
     A.scale = P.scale;
+    A.tl_words = exit_list_words(P.P);
+    if (!P.prune) tlist = nullptr;
     for (int h = 0; h < FS_MAX_HEADS; h++) {
         A.lambda[h] = P.lambda[h];
         A.inv2sigma[h] = P.inv2sigma[h];
@@ -381,8 +452,8 @@ cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, con
     const dim3 grid((P.Nq + BM - 1) / BM, BH);
     LaunchScope scope(kSelectTc, st);
     if (union_bound(P) <= 80)
-        return launch_um<80>(tq, A, P.has_prior, grid, kbar, amax, exitn, idx, tiles, dev_flag, st);
-    return launch_um<UMAX>(tq, A, P.has_prior, grid, kbar, amax, exitn, idx, tiles, dev_flag, st);
+        return launch_um<80>(tq, A, P.has_prior, grid, kbar, amax, exitn, idx, tiles, dev_flag, tlist, st);
+    return launch_um<UMAX>(tq, A, P.has_prior, grid, kbar, amax, exitn, idx, tiles, dev_flag, tlist, st);
 }
 
 }  // namespace fs
