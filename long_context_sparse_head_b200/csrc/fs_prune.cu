@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(256) exit_times_kernel(const float *__restrict
 namespace {
 constexpr int kRangeThreads = 512;
 constexpr int kRangeMaxSteps = 128;              // largest n_hi - n_lo this kernel takes
+constexpr int kEqCap = 512;                      // cells equal to the threshold ranked directly
 
 // order-preserving integer key of a float (larger float, larger key)
 __device__ __forceinline__ uint32_t order_key(float a) {
@@ -88,7 +89,8 @@ __global__ void __launch_bounds__(kRangeThreads) topp_range_kernel(const float *
     __shared__ int hist[256];
     __shared__ int wsum[kRangeThreads / 32];
     __shared__ uint32_t s_prefix;
-    __shared__ int s_remaining, s_count;
+    __shared__ int s_remaining, s_count, s_neq;
+    __shared__ int eq_list[kEqCap];              // cells whose key equals tau
     uint32_t *lkey = list;
     int *lidx = reinterpret_cast<int *>(list + P);
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -150,35 +152,54 @@ __global__ void __launch_bounds__(kRangeThreads) topp_range_kernel(const float *
                 __syncthreads();
             }
         }
-        // members of TopP(n0), in rounds of kRangeThreads cells in index order (the rank of
-        // a tau-valued cell among its equals decides ties)
-        int eq_before = 0;
-        for (int base = 0; base < n0; base += kRangeThreads) {
-            const int c = base + t;
-            uint32_t k = 0;
-            bool gt = false, eq = false;
-            if (c < n0) {
-                k = order_key(__ldg(a + c));
-                gt = all || k > tau;
-                eq = !all && k == tau;
+        // members of TopP(n0): every cell whose key beats tau, and the `remaining` lowest-
+        // indexed cells whose key equals tau.  One pass lists the equal ones (usually a
+        // handful), which are then ranked by index; with very many equal keys they are
+        // taken in rounds of kRangeThreads cells in index order instead.
+        auto add_member = [&](int c, uint32_t k) {
+            const int slot = atomicAdd(&s_count, 1);
+            lkey[slot] = k;
+            lidx[slot] = c;
+            ex[c] = kNever;
+            if (tl) tl[1 + slot] = c;
+        };
+        if (t == 0) s_neq = 0;
+        __syncthreads();
+        for (int c = t; c < n0; c += kRangeThreads) {
+            const uint32_t k = order_key(__ldg(a + c));
+            if (all || k > tau) {
+                add_member(c, k);
+            } else if (k == tau) {
+                const int e = atomicAdd(&s_neq, 1);
+                if (e < kEqCap) eq_list[e] = c;
             }
-            const unsigned bal = __ballot_sync(kFull, eq);
-            if (lane == 0) wsum[warp] = __popc(bal);
-            __syncthreads();
-            int before = eq_before + __popc(bal & ((1u << lane) - 1u)), tot = 0;
-            for (int w2 = 0; w2 < kRangeThreads / 32; w2++) {
-                if (w2 < warp) before += wsum[w2];
-                tot += wsum[w2];
+        }
+        __syncthreads();
+        const int neq = s_neq;
+        if (neq <= kEqCap) {
+            for (int j = t; j < neq; j += kRangeThreads) {
+                const int c = eq_list[j];
+                int rank = 0;
+                for (int x = 0; x < neq; x++) rank += eq_list[x] < c;
+                if (rank < remaining) add_member(c, tau);
             }
-            if (gt || (eq && before < remaining)) {
-                const int slot = atomicAdd(&s_count, 1);
-                lkey[slot] = k;
-                lidx[slot] = c;
-                ex[c] = kNever;
-                if (tl) tl[1 + slot] = c;
+        } else {
+            int eq_before = 0;
+            for (int base = 0; base < n0; base += kRangeThreads) {
+                const int c = base + t;
+                const bool eq = c < n0 && order_key(__ldg(a + c)) == tau;
+                const unsigned bal = __ballot_sync(kFull, eq);
+                if (lane == 0) wsum[warp] = __popc(bal);
+                __syncthreads();
+                int before = eq_before + __popc(bal & ((1u << lane) - 1u)), tot = 0;
+                for (int w2 = 0; w2 < kRangeThreads / 32; w2++) {
+                    if (w2 < warp) before += wsum[w2];
+                    tot += wsum[w2];
+                }
+                if (eq && before < remaining) add_member(c, tau);
+                eq_before += tot;
+                __syncthreads();
             }
-            eq_before += tot;
-            __syncthreads();
         }
     }
     __syncthreads();

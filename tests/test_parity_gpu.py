@@ -84,6 +84,24 @@ def test_small_cases(dtype, case):
     run_case(generate(wl))
 
 
+@pytest.mark.parametrize("distinct", [3, 1])
+def test_decoding_prune_ties(distinct):
+    """A decoding-shaped call (few prefixes) whose cells are copies of `distinct` cells, so
+    hundreds of cells share the P-th largest a_c and the lower-index rule decides TopP.
+    With 3 distinct cells the equal ones are ranked directly; with 1, there are more equal
+    cells than that ranking takes and they go in index order instead.  Equal cells also
+    tie on every score, so the top-K rule (lower cell first) is exercised too."""
+    import dataclasses
+    inp = generate(small("ties", B=1, H=2, Nq=64, Nk=20480, K=6, W=4, P=9, dtype="bf16", seed=44,
+                         needles=0))
+    s, C = inp.wl.s, inp.wl.Nk // inp.wl.s
+    K = inp.K.copy()
+    for c in range(distinct, C):
+        src = c % distinct
+        K[:, :, c * s:(c + 1) * s] = K[:, :, src * s:(src + 1) * s]
+    run_case(dataclasses.replace(inp, K=K), check_needles=False)
+
+
 def test_caller_idx_runs_readout_on_given_cells():
     """fs_forward with caller cells skips selection: compare with the oracle readout on
     those cells, and with the internally selected path when given the GPU's own cells."""
