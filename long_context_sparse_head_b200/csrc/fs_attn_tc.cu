@@ -204,6 +204,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    griddep_wait();                             // the selection's tile records are complete
 
     if (warp >= NSOFT) {
         tc::regs_dec<REGS_PRODUCER>();
@@ -483,6 +484,7 @@ namespace {
 constexpr int kCombWarps = 4;
 __global__ void __launch_bounds__(kCombWarps * 32) attn_combine_kernel(const AttnArgs A, int ntiles,
                                                                        __nv_bfloat16 *__restrict__ O) {
+    griddep_wait();                             // the split CTAs' partial states are complete
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.y, h = bh % A.H;
     const int r = blockIdx.x * kCombWarps + warp;
@@ -572,14 +574,15 @@ cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const voi
         LaunchScope scope(kAttnTc, st);
         auto kern = A.nsplit > 1 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kern<<<grid, NTHREADS, smem, st>>>(tq, tk32, tv32, tkr64, tv64, A, tiles, rope_lo, rope_hi,
-                                           (__nv_bfloat16 *)O, dev_flag);
-        if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
+        if (launch_pdl(kern, grid, dim3(NTHREADS), smem, st, tq, tk32, tv32, tkr64, tv64, A, tiles, rope_lo, rope_hi,
+                       (__nv_bfloat16 *)O, dev_flag) != cudaSuccess)
+            return cudaErrorLaunchFailure;
     }
     if (A.nsplit > 1) {
         LaunchScope scope(kAttnCombine, st);
-        attn_combine_kernel<<<dim3((P.Nq + kCombWarps - 1) / kCombWarps, BH), kCombWarps * 32, 0, st>>>(
-            A, ntiles, (__nv_bfloat16 *)O);
+        if (launch_pdl(attn_combine_kernel, dim3((P.Nq + kCombWarps - 1) / kCombWarps, BH), dim3(kCombWarps * 32), 0, st,
+                       A, ntiles, (__nv_bfloat16 *)O) != cudaSuccess)
+            return cudaErrorLaunchFailure;
     }
     return cudaGetLastError();
 }

@@ -1,6 +1,8 @@
 // Shared definitions of the FreeSolo CUDA library (sm_100a).
 #pragma once
 
+#include <utility>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -133,6 +135,29 @@ enum KernelId : int {
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
+// Programmatic dependent launch: a kernel launched this way may be scheduled as soon as
+// every CTA of the previous kernel on the stream has exited, so its launch and prologue
+// overlap that kernel's completion.  It must execute griddep_wait() (which returns once
+// the previous kernel has completed and its writes are visible) before it reads anything
+// an earlier kernel wrote or writes anything an earlier kernel reads.  griddep_wait() is a
+// no-op in a kernel launched without the attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 struct LaunchScope {
     LaunchScope(int id, cudaStream_t st);
     ~LaunchScope();

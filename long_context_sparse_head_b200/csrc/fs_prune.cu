@@ -22,6 +22,7 @@ constexpr int kScanBlocks = 8;                   // 32-cell blocks loaded per ro
 __global__ void __launch_bounds__(256) exit_times_kernel(const float *__restrict__ amax,
                                                          int *__restrict__ exitn,
                                                          long long ncell, int C, int P) {
+    griddep_wait();
     const long long cell = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (cell >= ncell) return;
     const int lane = threadIdx.x & 31;
@@ -97,6 +98,7 @@ __global__ void __launch_bounds__(kRangeThreads) topp_range_kernel(const float *
     const float *a = amax + (size_t)blockIdx.x * C;
     int *ex = exitn + (size_t)blockIdx.x * C;
     int *tl = tlist ? tlist + (size_t)blockIdx.x * tl_words : nullptr;   // [0] count, then cells
+    griddep_wait();
     for (int c = t; c < C; c += kRangeThreads) ex[c] = c + 1;
     const int n0 = min(n_lo, C), m0 = min(P, n0);  // |TopP(n0)| = m0
     if (t == 0) s_count = 0;
@@ -262,16 +264,14 @@ cudaError_t launch_exit_times(const Dev &P, const float *amax, int *exitn, cudaS
         const int n_lo = cand_count(P.q0, P.w, P.C), n_hi = cand_count(P.q0 + P.Nq - 1, P.w, P.C);
         if (n_hi - n_lo <= kRangeMaxSteps) {
             LaunchScope scope(kExitTimes, st);
-            topp_range_kernel<<<(unsigned)(P.B * P.H), kRangeThreads, (size_t)P.P * 8, st>>>(
-                amax, exitn, P.C, P.P, n_lo, n_hi, tlist, exit_list_words(P.P));
-            return cudaGetLastError();
+            return launch_pdl(topp_range_kernel, dim3((unsigned)(P.B * P.H)), dim3(kRangeThreads), (size_t)P.P * 8,
+                              st, amax, exitn, P.C, P.P, n_lo, n_hi, tlist, exit_list_words(P.P));
         }
     }
     const int warps = 8;
     const long long blocks = (ncell + warps - 1) / warps;
     LaunchScope scope(kExitTimes, st);
-    exit_times_kernel<<<(unsigned)blocks, warps * 32, 0, st>>>(amax, exitn, ncell, P.C, P.P);
-    return cudaGetLastError();
+    return launch_pdl(exit_times_kernel, dim3((unsigned)blocks), dim3(warps * 32), 0, st, amax, exitn, ncell, P.C, P.P);
 }
 
 }  // namespace fs

@@ -106,6 +106,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    griddep_wait();                             // the summaries and exit times are complete
 
     if (warp == W_MMA) {
         if (lane == 0) {
@@ -427,8 +428,7 @@ template <int UM> cudaError_t launch_um(const CUtensorMap &tq, const SelArgs &A,
     // the erf prior is a separate instantiation: without it the unrolled score loop stays small
     auto kern = prior ? select_tc_kernel<true, UM> : select_tc_kernel<false, UM>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<grid, NTHREADS, smem, st>>>(tq, A, kbar, amax, exitn, idx, tiles, dev_flag, tlist);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(NTHREADS), smem, st, tq, A, kbar, amax, exitn, idx, tiles, dev_flag, tlist);
 }
 }  // namespace
 
