@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(256) exit_times_kernel(const float *__restrict
 // that evicts them (never, if none in range); every other cell gets c + 1, which makes
 // c < n < exit(c) false for every n >= n_lo.  One CTA per (b, h).
 namespace {
-constexpr int kRangeThreads = 512;
+constexpr int kRangeThreads = 1024;
 constexpr int kRangeMaxSteps = 128;              // largest n_hi - n_lo this kernel takes
 constexpr int kEqCap = 512;                      // cells equal to the threshold ranked directly
 
