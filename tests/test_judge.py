@@ -1,6 +1,7 @@
 """The GPU parity judge itself, checked on the CPU: it accepts the oracle's own
-selections and rejects plausible wrong ones (a worse cell swapped in, a non-candidate,
-unsorted output, a missing pad)."""
+selections and rejects plausible wrong ones (a worse cell swapped in, the best unselected
+cell swapped for the K-th where their gap exceeds the near-tie tolerance, a
+non-candidate, unsorted output, a missing pad)."""
 import numpy as np
 import pytest
 
@@ -56,3 +57,28 @@ def test_rejects_non_candidate_and_bad_layout(case):
     bad[b, h, r] = bad[b, h, r][::-1]                     # descending
     with pytest.raises(AssertionError):
         check_selection(inp, sums, bad, [(b, h, r)])
+
+
+def test_rejects_boundary_swap_outside_tolerance(case):
+    # the K-th selected cell traded for the best unselected one: a near-tie only if their
+    # scores lie within 1e-4 of the row's score scale; rows with a wider gap must fail
+    inp, prob, sums, full, rows = case
+    tested = 0
+    for b, h, r in rows:
+        _, acells, scores = prob.select_row(sums[0], sums[1], b, h, r)
+        sc = dict(zip(acells.tolist(), scores.tolist()))
+        chosen = [int(c) for c in full[b, h, r] if c >= 0]
+        rest = [c for c in sc if c not in chosen]
+        if not rest:
+            continue
+        kth = min(chosen, key=lambda c: sc[c])
+        best_out = max(rest, key=lambda c: sc[c])
+        if sc[kth] - sc[best_out] <= 1e-4 * max(np.abs(scores).max(), abs(sc[kth])):
+            continue
+        bad = full.copy()
+        row = sorted([c for c in chosen if c != kth] + [best_out])
+        bad[b, h, r, :len(row)] = row
+        with pytest.raises(AssertionError):
+            check_selection(inp, sums, bad, [(b, h, r)])
+        tested += 1
+    assert tested >= 10, tested

@@ -1,15 +1,14 @@
 """GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
 
-Small cases are compared on every row; the full-size workloads run exactly as the
-benchmark launches them and are compared on sampled rows (plus every needle row).
+Small cases and the full-size workloads (run exactly as the benchmark launches them)
+are compared on every row.
 """
 import numpy as np
 import pytest
 import torch
 
 from workloads import CONFIGS, generate, small
-from tests._parity import (TOL, DeviceRun, check_selection, expected_output, oracle_for,
-                           sample_rows)
+from tests._parity import TOL, DeviceRun, check_selection, expected_output, oracle_for
 
 pytestmark = pytest.mark.gpu
 
@@ -152,29 +151,53 @@ def test_repeated_calls_are_deterministic():
 
 # ---------------------------------------------------------------- full-size workloads
 @pytest.mark.parametrize("name", ["prefill4k", "prefill16k", "prefill64k", "decode256k"])
-def test_full_size_sampled(name):
+def test_full_size_every_row(name):
+    """The four full-size workloads, run as the benchmark launches them, against the
+    oracle on every query row of every head: selected cells (near-tie rule, at most 1% of
+    rows differing), and the fused output (oracle window branch plus the oracle readout on
+    the GPU's own cells) within the bf16 tolerance."""
     wl = CONFIGS[name]
     inp = generate(wl)
-    needle_rows = [(b, h, r) for b, h, c, rs in inp.needle_cells for r in rs[:4]]
-    rows = sample_rows(wl, 400, seed=1, extra=needle_rows)
-    g, idx, O, err = run_case(inp, rows=rows, check_needles=False)
-    # every needle row whose needle cell survives FS-L pruning selects it (eq. (8) can
-    # drop a low-norm needle before the query arrives; the oracle agrees on sampled rows)
+    g = DeviceRun(inp)
     prob = oracle_for(inp)
-    _, amax = prob.summaries()
+    kbar_o, amax_o = prob.summaries()
+    kbar_g, amax_g = (g.numpy(t) for t in g.summaries())
+    np.testing.assert_allclose(kbar_g, kbar_o, rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(amax_g, amax_o, rtol=1e-5, atol=1e-6)
+    idx = g.numpy(g.select())
+    O = g.numpy(g.forward()).reshape(-1, wl.d)
+    assert np.isfinite(O).all()
+    # the oracle on every row: its own selection and the window branch o^sr
+    _, idx_o, _, osr = prob.forward(want_idx=True, want_parts=True)
+    same = (idx == idx_o).all(axis=-1)
+    differ = [tuple(int(x) for x in t) for t in np.argwhere(~same)]
+    n_rows = same.size
+    assert len(differ) <= max(2, n_rows // 100), (len(differ), n_rows)
+    if differ:
+        exact, tie = check_selection(inp, (kbar_o, amax_o), idx, differ)
+        assert exact == 0 and tie == len(differ)
+    # output: oracle window branch + alpha_h * oracle readout on the GPU's cells
+    flat = np.arange(n_rows, dtype=np.int64)
+    _, olr = prob.readout_rows(flat, idx.reshape(n_rows, wl.K))
+    alpha = np.repeat(np.tile(np.asarray(inp.alpha, np.float64), wl.B), wl.Nq)[:, None]
+    want = osr.reshape(n_rows, wl.d) + alpha * olr
+    err = float(np.abs(O - want).max())
+    assert err <= TOL[wl.dtype], err
+    # planted needles: every needle row whose needle cell survives FS-L pruning selects it
+    # (eq. (8) can drop a low-norm needle before the query arrives)
     kept = seen = 0
     for b, h, c, rs in inp.needle_cells:
         for r in rs:
             n = prob.candidate_count(wl.Nk - wl.Nq + r)
             seen += 1
-            if c in prob.admitted(amax[b, h], n):
+            if c in prob.admitted(amax_o[b, h], n):
                 kept += 1
                 assert c in idx[b, h, r], ("needle missed", b, h, c, r)
-    assert kept >= seen // 2, (kept, seen)
-    # properties at every row: finite, ascending selections inside the candidate prefix
-    assert np.isfinite(O).all()
+    # structure at every row: ascending selections, -1 only as trailing padding
     sel = idx.reshape(-1, wl.K).astype(np.int64)
     valid = sel >= 0
     both = valid[:, 1:] & valid[:, :-1]
     assert (np.diff(sel, axis=1)[both] > 0).all()
-    assert not (valid[:, 1:] & ~valid[:, :-1]).any()        # -1 only as trailing padding
+    assert not (valid[:, 1:] & ~valid[:, :-1]).any()
+    print("%s: %d rows, %d differ within the near-tie rule, max-abs %.2e, needle rows "
+          "whose needle survives pruning %d of %d" % (name, n_rows, len(differ), err, kept, seen))
