@@ -10,7 +10,10 @@
 // One CTA per 128 query rows of a (batch, head); two CTAs per SM.  The readout runs over
 // U (|U| <= 128, ascending), two cells (64 keys) per chunk, each cell fetched by its own
 // 32-row TMA box; a row masks the cells it did not select (masked-dense on the tensor
-// cores).  Then the window runs over 64-key chunks.  Both softmaxes accumulate in tensor
+// cores).  The readout's exponent reference is the row's bound from the record (an upper
+// bound of its logits within 96 of their maximum, so every P is at most 1 and none
+// underflows): no running maximum, no rescaling.  Then the window runs over 64-key chunks
+// with a running maximum and lazy rescaling.  Both softmaxes accumulate in tensor
 // memory: three S buffers in columns [0,64), [64,128) and [128,192) (chunk c uses buffer
 // c mod 3, and its P overwrites the first 32 columns of that buffer) and one O in
 // [192,256).  The MMA warp keeps Q K^T two chunks ahead of P V, so a softmax warp that
@@ -145,6 +148,41 @@ __device__ __forceinline__ float softmax_chunk(uint32_t tS, int kind, uint32_t s
     tc::f2_unpack(tc::f2_add(tc::f2_add(ls[0], ls[1]), tc::f2_add(ls[2], ls[3])), u, v);
     l += u + v;
     return corr;
+}
+
+// One readout chunk (two cells) against a fixed reference mref (log2 units, an upper
+// bound of the row's logits, so every exponent is <= 0 and nothing is ever rescaled).
+// Block b of 32 columns counts only if bit b of sel is set; otherwise its exponent bias is
+// -inf and its P is 0.  P is written back as bf16 pairs over the buffer's first BN/2
+// columns; l gathers the row sum.
+__device__ __forceinline__ void softmax_chunk_fixed(uint32_t tS, uint32_t sel, float mref, float c_log2, float &l) {
+    uint32_t s[BN];
+    tc::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+    tc::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+    tc::tmem_wait_ld();
+    const uint64_t c2 = tc::f2_pack(c_log2, c_log2);
+    uint64_t ls[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) ls[k] = tc::f2_pack(0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < BN / 32; q++) {
+        const float nb = ((sel >> q) & 1u) ? -mref : -INFINITY;
+        const uint64_t nb2 = tc::f2_pack(nb, nb);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; e++) {
+            const int j = 32 * q + 2 * e;
+            float x0, x1;
+            tc::f2_unpack(tc::f2_fma(tc::f2_pack(__uint_as_float(s[j]), __uint_as_float(s[j + 1])), c2, nb2), x0, x1);
+            const float p0 = tc::ex2(x0), p1 = tc::ex2(x1);
+            ls[e & 3] = tc::f2_add(ls[e & 3], tc::f2_pack(p0, p1));
+            pk[e] = tc::pack_bf16x2(p0, p1);
+        }
+        tc::tmem_st16(tS + 16 * q, pk);
+    }
+    float u, v;
+    tc::f2_unpack(tc::f2_add(tc::f2_add(ls[0], ls[1]), tc::f2_add(ls[2], ls[3])), u, v);
+    l += u + v;
 }
 }  // namespace
 
@@ -341,27 +379,76 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         const int i = pb + row;
         const bool rvalid = row < nrows;
         const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-        const uint4 m4 = __ldg(reinterpret_cast<const uint4 *>(
-            tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords + kTileMaskOff + 4 * row));
+        const uint32_t *rec = tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords;
+        const uint4 m4 = __ldg(reinterpret_cast<const uint4 *>(rec + kTileMaskOff + 4 * row));
+        const float mref = __uint_as_float(__ldg(rec + kTileMrefOff + row));
+        // the readout runs against each row's fixed reference unless one of the warp's rows
+        // has none; it then tracks a running maximum with lazy rescaling, as the window does
+        const bool fixed = __all_sync(kFull, !isnan(mref));
         bool ok = tc::mbar_wait(&sm.u_ready, 0, ab);
         const int nR = ok ? (sm.nU + CPC - 1) / CPC : 0;
         int cb = 0, ce = 0;
         if (ok) chunk_range(nR, cb, ce);
         const int total = ce - cb;
-        float m_lr = -INFINITY, l_lr = 0.f, m_sr = -INFINITY, l_sr = 0.f;
+        const int nread = max(0, min(ce, nR) - cb);     // this CTA's readout chunks come first
+        float m_lr = fixed ? mref : -INFINITY, l_lr = 0.f, m_sr = -INFINITY, l_sr = 0.f;
+        float *part_row = SPLIT ? A.part + ((((size_t)bh * gridDim.x + blockIdx.x) * S + sidx) * BM + row) * kPartStride
+                                : nullptr;
+        // O rescale, after the exponentials (S no longer occupies registers); the P V of the
+        // previous chunk, which accumulates into the same O, must have finished.  Called only
+        // after chunk it's S wait: that S was issued after the P V of chunk it - 3, which
+        // shares o_ready[(it - 1) & 1], so the parity wait cannot match an older phase.
+        auto rescale_o = [&](int it, float corr) -> bool {
+            if (!tc::mbar_wait(&sm.o_ready[(it - 1) & 1], ((it - 1) >> 1) & 1, ab)) return false;
+            tc::tc_fence_after();
+#pragma unroll
+            for (int b = 0; b < kD / 32; b++) {
+                uint32_t r[32];
+                tc::tmem_ld32(trow + O_COL + 32 * b, r);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; e++) r[e] = __float_as_uint(__uint_as_float(r[e]) * corr);
+                tc::tmem_st32(trow + O_COL + 32 * b, r);
+            }
+            return true;
+        };
+        auto release = [&](int it) {            // P of chunk it is in tensor memory
+            tc::tmem_wait_st();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sm.p_full[it % NSBUF]);
+        };
+        int it = 0;
+        // ---- readout chunks (eq. (9)): two union cells each, the unselected ones masked
+        for (; ok && it < nread; it++) {
+            if (!tc::mbar_wait(&sm.s_full[it % NSBUF], (it / NSBUF) & 1, ab)) { ok = false; break; }
+            tc::tc_fence_after();
+            const int p0 = CPC * (cb + it);
+            const int wsel = p0 >> 5;           // word of the row's union mask, in registers
+            const uint32_t mw = wsel == 0 ? m4.x : wsel == 1 ? m4.y : wsel == 2 ? m4.z : m4.w;
+            const uint32_t sel = (mw >> (p0 & 31)) & ((1u << CPC) - 1u);
+            if (fixed) {
+                softmax_chunk_fixed(trow + BN * (it % NSBUF), sel, mref, A.scale_log2e, l_lr);
+            } else {
+                const float corr = softmax_chunk(trow + BN * (it % NSBUF), CELLS, sel, 0, BN, A.scale_log2e, m_lr, l_lr);
+                if (it > 0 && __any_sync(kFull, corr != 1.f) && !rescale_o(it, corr)) { ok = false; break; }
+            }
+            release(it);
+        }
         float y[kD];                            // alpha_h RMSNorm(u), once the readout is done
 #pragma unroll
         for (int e = 0; e < kD; e++) y[e] = 0.f;
-        float *part_row = SPLIT ? A.part + ((((size_t)bh * gridDim.x + blockIdx.x) * S + sidx) * BM + row) * kPartStride
-                                : nullptr;
-        for (int it = 0; ok && it < total; it++) {
+        // ---- window chunks (eqs. (3)-(4)): 64 consecutive keys of the band each
+        for (; ok && it < total; it++) {
             const int g = cb + it;
             if (!tc::mbar_wait(&sm.s_full[it % NSBUF], (it / NSBUF) & 1, ab)) { ok = false; break; }
             tc::tc_fence_after();
-            if (g == nR && it > 0) {
+            if (it == nread && nread > 0) {
                 // readout done (its last P V may still run): take its O out of tensor memory
-                // before the window's first P V overwrites it
-                if (!tc::mbar_wait(&sm.o_ready[(it - 1) & 1], ((it - 1) >> 1) & 1, ab)) { ok = false; break; }
+                // before the window's first P V overwrites it.  This chunk's S was issued
+                // after the P V of chunk nread - 3, which shares the barrier of chunk nread - 1,
+                // so the parity wait below cannot match an older phase.
+                if (!tc::mbar_wait(&sm.o_ready[(nread - 1) & 1], ((nread - 1) >> 1) & 1, ab)) { ok = false; break; }
                 tc::tc_fence_after();
                 uint32_t a[kD];
                 tc::tmem_ld32(trow + O_COL, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
@@ -386,46 +473,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     for (int e = 0; e < kD; e++) y[e] = __uint_as_float(a[e]) * f;
                 }
             }
-            // one call site for every kind of chunk keeps the unrolled body in the code once
-            int kind, lo = 0, width = BN;
-            uint32_t sel = 0u;
-            bool first;
-            float m, l;
-            if (g < nR) {
-                const int p0 = CPC * g;
-                const int wsel = p0 >> 5;           // word of the row's union mask, in registers
-                const uint32_t mw = wsel == 0 ? m4.x : wsel == 1 ? m4.y : wsel == 2 ? m4.z : m4.w;
-                sel = (mw >> (p0 & 31)) & ((1u << CPC) - 1u);
-                kind = CELLS; first = it == 0; m = m_lr; l = l_lr;
-            } else {
-                const int jc = jbase + BN * (k_first + g - nR);
-                const int clo = max(-jc, i - A.w - jc), chi = min(i - jc, BN - 1);
-                lo = clo;
-                width = rvalid ? max(0, chi - clo + 1) : 0;
-                kind = __all_sync(kFull, clo <= 0 && chi >= BN - 1 && rvalid) ? FULL : BAND;
-                first = g == nR || it == 0; m = m_sr; l = l_sr;
-            }
-            const float corr = softmax_chunk(trow + BN * (it % NSBUF), kind, sel, lo, width, A.scale_log2e, m, l);
-            if (g < nR) { m_lr = m; l_lr = l; } else { m_sr = m; l_sr = l; }
-            // O rescale, after the exponentials (S no longer occupies registers); the P V of
-            // the previous chunk, which accumulates into the same O, must have finished
-            if (!first && __any_sync(kFull, corr != 1.f)) {
-                if (!tc::mbar_wait(&sm.o_ready[(it - 1) & 1], ((it - 1) >> 1) & 1, ab)) { ok = false; break; }
-                tc::tc_fence_after();
-#pragma unroll
-                for (int b = 0; b < kD / 32; b++) {
-                    uint32_t r[32];
-                    tc::tmem_ld32(trow + O_COL + 32 * b, r);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; e++) r[e] = __float_as_uint(__uint_as_float(r[e]) * corr);
-                    tc::tmem_st32(trow + O_COL + 32 * b, r);
-                }
-            }
-            tc::tmem_wait_st();
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&sm.p_full[it % NSBUF]);
+            const int jc = jbase + BN * (k_first + g - nR);
+            const int clo = max(-jc, i - A.w - jc), chi = min(i - jc, BN - 1);
+            const int width = rvalid ? max(0, chi - clo + 1) : 0;
+            const int kind = __all_sync(kFull, clo <= 0 && chi >= BN - 1 && rvalid) ? FULL : BAND;
+            const float corr = softmax_chunk(trow + BN * (it % NSBUF), kind, 0u, clo, width, A.scale_log2e, m_sr, l_sr);
+            if (it > nread && __any_sync(kFull, corr != 1.f) && !rescale_o(it, corr)) { ok = false; break; }
+            release(it);
         }
         if (ok && tc::mbar_wait(&sm.o_done, 0, ab)) {
             tc::tc_fence_after();

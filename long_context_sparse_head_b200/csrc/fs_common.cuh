@@ -43,8 +43,15 @@ struct WsLayout {
 // Per-tile selection record passed from the tensor-core selection kernel to the fused
 // attention kernel (128 query rows, union of at most 128 cells), in 32-bit words:
 // [0, 512) row masks [128][4] (bit u of a row: union position u selected), [512, 640)
-// union cells ascending (0xffffffff past |U|), [640] |U|.  2576 bytes, 16-byte multiple.
-constexpr int kTileMaskOff = 0, kTileUlistOff = 512, kTileCountOff = 640, kTileRecWords = 644;
+// union cells ascending (0xffffffff past |U|), [640] |U|, [644, 772) per row a float
+// softmax reference for the readout in log2 units (an upper bound of every logit of the
+// row's selected tokens that lies within 96 of their largest one), or NaN where none was
+// found (the readout then tracks a running maximum).  3088 bytes, 16-byte multiple.
+constexpr int kTileMaskOff = 0, kTileUlistOff = 512, kTileCountOff = 640, kTileMrefOff = 644,
+              kTileRecWords = 772;
+// Largest gap (log2 units) between a row's readout reference and its largest selected
+// logit: p = 2^(x - ref) then stays a normal float for the row's heaviest tokens.
+constexpr float kMrefMaxGap = 96.f;
 
 // Device error flag codes (first int of the workspace).
 enum : int { kFlagOk = 0, kFlagTimeout = 1, kFlagCheck = 2 };
@@ -222,6 +229,8 @@ cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, con
 cudaError_t launch_selection(const fs_params *p, const Dev &D, const void *Q, const float *kbar,
                              const float *amax, const int *exitn, int32_t *idx, int *dev_flag,
                              cudaStream_t st);
+// status word of fs_select_topk_noalloc on the current device, read and cleared
+fs_status noalloc_take_status();
 // FS-B (eqs. (10)-(11)): forest buffer size, build (tau: host [H] or NULL), search
 size_t forest_bytes(const fs_params *p);
 cudaError_t launch_tree_build(const fs_params *p, const float *kbar, const float *amax, const float *tau,

@@ -252,6 +252,7 @@ __global__ void __launch_bounds__(128) idx_tiles_kernel(const int32_t *__restric
     uint32_t *rec = tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords;
     *reinterpret_cast<uint4 *>(rec + kTileMaskOff + 4 * t) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
     rec[kTileUlistOff + t] = t < nU ? (uint32_t)ulist[t] : 0xffffffffu;
+    rec[kTileMrefOff + t] = 0x7fc00000u;          // no reference: running maximum
     if (t == 0) rec[kTileCountOff] = (uint32_t)nU;
 }
 

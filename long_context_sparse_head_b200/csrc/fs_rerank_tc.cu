@@ -340,6 +340,7 @@ rerank_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
                 uint32_t *rec = tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords;
                 *reinterpret_cast<uint4 *>(rec + kTileMaskOff + 4 * row) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
                 rec[kTileUlistOff + t] = t < nU ? (uint32_t)sm.ulist[t] : 0xffffffffu;
+                rec[kTileMrefOff + row] = 0x7fc00000u;    // no reference: running maximum
                 if (t == 0) rec[kTileCountOff] = (uint32_t)nU;
             }
             if (idx && row < nrows) {

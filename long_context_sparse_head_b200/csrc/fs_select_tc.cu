@@ -34,15 +34,17 @@ constexpr int W_MMA = 4, NWARPS = 5, NTHREADS = NWARPS * 32;   // warp 4: Q load
 constexpr uint32_t TMEM_COLS = 128;
 constexpr int TILE_BYTES = BM * kD * 2;
 constexpr int kSelBarrier = 1;   // named barrier of the 128 selection threads
+constexpr int kSmall = 16;       // bracket size at which the K-th search finishes by ranks
 
 template <int UM> struct SelSmem {       // UM: capacity of the union (a multiple of 16)
     __nv_bfloat16 q[BM * kD];              // Q tile (NoPE)
     __nv_bfloat16 kb[3][UM * kD];          // kbar of U as hi, mid, lo bf16 parts
     int ulist[UM];
-    float acell[UM];                       // a_c of the union cells (prior)
+    float acell[UM];                       // a_c of the union cells (prior, readout reference)
     uint8_t amask[UM];                     // bit g: admitted for prefix n_min + g
     uint32_t admit[5][(UM + 31) / 32];     // per prefix n_min + g: admitted union positions
     int warp_cnt[4];
+    float amax_w[4];                       // per warp: largest a_c of its union positions
     int nU, ncand;
     uint64_t q_full, kb_ready, s_full, drain;
     uint32_t tmem_base;
@@ -182,7 +184,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                 if (rank < UM) {
                     sm.ulist[rank] = c;
                     sm.amask[rank] = cmask[j];
-                    sm.acell[rank] = A.has_prior ? am[c] : 0.f;
+                    sm.acell[rank] = am[c];
                 }
             }
             if (warp == 0) {
@@ -195,7 +197,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                     if (m && p < UM) {
                         sm.ulist[p] = c;
                         sm.amask[p] = (uint8_t)m;
-                        sm.acell[p] = A.has_prior ? am[c] : 0.f;
+                        sm.acell[p] = am[c];
                     }
                     pos += __popc(bal);
                 }
@@ -252,7 +254,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                         if (pos < UM) {
                             sm.ulist[pos] = cb + j;
                             sm.amask[pos] = (uint8_t)amk[j];
-                            sm.acell[pos] = A.has_prior ? am[cb + j] : 0.f;
+                            sm.acell[pos] = am[cb + j];
                         }
                         pos++;
                     }
@@ -268,7 +270,9 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
         sel_sync();
         const int nU = min(total, UM);
         constexpr int NW = (UM + 31) / 32;      // admission words
-        {   // admission masks per prefix, one 32-position word per warp
+        {   // admission masks per prefix, one 32-position word per warp; the largest a_c of U
+            const float au = warp_max(t < nU ? sm.acell[t] : 0.f);
+            if (lane == 0) sm.amax_w[warp] = au;
             const uint32_t am = t < nU ? sm.amask[t] : 0u;
 #pragma unroll
             for (int gg = 0; gg < 5; gg++) {
@@ -308,6 +312,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
         const int n_r = cand_count(i, A.w, A.C);
         const int g = n_r - n_min;
         if (!tc::mbar_wait(&sm.s_full, 0, ab)) goto done;
+        if (tiles && !tc::mbar_wait(&sm.q_full, 0, ab)) goto done;   // Q rows read for |q|
         {
             tc::tc_fence_after();
             const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
@@ -344,7 +349,8 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                 }
             }
             const float mn = fminf(fminf(fmn[0], fmn[1]), fminf(fmn[2], fmn[3]));
-            const float span = fmaxf(fmaxf(fmx[0], fmx[1]), fmaxf(fmx[2], fmx[3])) - mn;
+            const float smax = fmaxf(fmaxf(fmx[0], fmx[1]), fmaxf(fmx[2], fmx[3]));
+            const float span = smax - mn;
             const float q24 = span > 0.f ? 16777215.f / span : 0.f;
             // integer keys: 1 + the score's 24-bit fixed-point place in the row's range, then
             // 7 bits of (127 - position); 0 for a cell that is not admitted
@@ -358,11 +364,16 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                     key[u] = 0u;
                 }
             }
-            // K-th largest key by bisection: count(key >= lo) >= K > count(key >= hi)
+            // K-th largest key: bisection while more than kSmall keys lie in the bracket
+            // [lo, hi), with clo = count(key >= lo) >= K > chi = count(key >= hi) (keys are
+            // unique, so the bracket holds exactly clo - chi of them); then those keys are
+            // compacted into shared memory and the (K - chi)-th largest among them is found
+            // by counting ranks, with no data-dependent loop
             uint32_t tau = 1u;
             if (na > A.K) {
                 uint32_t lo = 1u << 7, hi = (0x1000000u + 1u) << 7;
-                while (hi - lo > 1u) {
+                int clo = na, chi = 0;
+                while (clo - chi > kSmall && clo != A.K) {
                     const uint32_t mid = lo + ((hi - lo) >> 1);
                     int cp[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent partial counts
 #pragma unroll
@@ -374,21 +385,90 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                     const int cnt = ((cp[0] + cp[1]) + (cp[2] + cp[3])) + ((cp[4] + cp[5]) + (cp[6] + cp[7]));
                     if (cnt >= A.K) {
                         lo = mid;
-                        if (cnt == A.K) break;
+                        clo = cnt;
                     } else {
                         hi = mid;
+                        chi = cnt;
                     }
                 }
                 tau = lo;
-            }
-            if (tiles) {   // compact record for the fused kernel: row masks | union | |U|
-                uint32_t *rec = tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords;
-                uint32_t mw[UMAX / 32] = {0u, 0u, 0u, 0u};
+                if (clo != A.K) {
+                    // the mean-key operand is no longer read once S is in tensor memory; its
+                    // first kSmall x BM words hold the brackets, key j of row r at j * BM + r
+                    uint32_t *buf = reinterpret_cast<uint32_t *>(sm.kb[0]);
+                    int m = 0;
 #pragma unroll
-                for (int u = 0; u < UM; u++)
-                    if (key[u] >= tau && key[u] != 0u) mw[u >> 5] |= 1u << (u & 31);
+                    for (int u = 0; u < UM; u++) {
+                        if (16 * (u / 16) < N && key[u] >= lo && key[u] < hi) {
+                            buf[m * BM + row] = key[u];
+                            m++;
+                        }
+                    }
+                    uint32_t bk[kSmall];
+#pragma unroll
+                    for (int j = 0; j < kSmall; j++) bk[j] = j < m ? buf[j * BM + row] : 0u;
+                    const int need = A.K - chi;            // 1 <= need < m
+#pragma unroll
+                    for (int j = 0; j < kSmall; j++) {
+                        int r = 0;
+#pragma unroll
+                        for (int k = 0; k < kSmall; k++) r += bk[k] > bk[j];
+                        if (j < m && r == need - 1) tau = bk[j];
+                    }
+                }
+            }
+            uint32_t mw[UMAX / 32] = {0u, 0u, 0u, 0u};   // selected union positions
+#pragma unroll
+            for (int u = 0; u < UM; u++)
+                if (16 * (u / 16) < N && key[u] >= tau && key[u] != 0u) mw[u >> 5] |= 1u << (u & 31);
+            if (tiles) {   // compact record for the fused kernel: row masks | union | |U| | reference
+                // Readout reference (log2 units): every NoPE logit q.k_j / sqrt(d) of a selected
+                // token is at most |q| max_{c in U} a_c / sqrt(d) (Cauchy-Schwarz), and the
+                // largest is at least any selected cell's mean-key logit q.kbar_c / sqrt(d) (a
+                // maximum is at least the mean).  The row's best admitted cell is always
+                // selected; without the prior its eq. (7) score is that mean-key logit, with
+                // the prior the selected cells' raw products are read again from tensor
+                // memory.  Where the two bounds lie within kMrefMaxGap, the upper one serves
+                // as the softmax's fixed reference (no running maximum).
+                const float c = A.scale * 1.4426950408889634f;
+                float lower = smax * 1.4426950408889634f;
+                if (PRIOR) {
+                    // warp-collective loads (.sync.aligned): every lane issues them
+                    uint32_t raw[UM];
+#pragma unroll
+                    for (int b = 0; b < UM / 16; b++)
+                        if (16 * b < N) tc::tmem_ld16(trow + 16 * b, &raw[16 * b]);
+                    tc::tmem_wait_ld();
+                    float dmax = -INFINITY;
+#pragma unroll
+                    for (int u = 0; u < UM; u++)
+                        if (16 * (u / 16) < N && ((mw[u >> 5] >> (u & 31)) & 1u))
+                            dmax = fmaxf(dmax, __uint_as_float(raw[u]));
+                    lower = dmax * c;
+                }
+                float mref = 0.f;
+                if (na > 0) {
+                    // |q| of this row from the tile in shared memory (128-byte swizzle)
+                    const uint8_t *qrow = reinterpret_cast<const uint8_t *>(sm.q) + row * 128;
+                    float qq = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(qrow + ((j ^ (row & 7)) << 4));
+                        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            const float lo = __uint_as_float(w4[e] << 16), hi = __uint_as_float(w4[e] & 0xffff0000u);
+                            qq = fmaf(lo, lo, fmaf(hi, hi, qq));
+                        }
+                    }
+                    const float amx = fmaxf(fmaxf(sm.amax_w[0], sm.amax_w[1]), fmaxf(sm.amax_w[2], sm.amax_w[3]));
+                    const float ub = sqrtf(qq) * amx * c;
+                    mref = (ub - lower <= kMrefMaxGap) ? ub : __uint_as_float(0x7fc00000u);
+                }
+                uint32_t *rec = tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords;
                 *reinterpret_cast<uint4 *>(rec + kTileMaskOff + 4 * row) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
                 rec[kTileUlistOff + t] = t < nU ? (uint32_t)sm.ulist[t] : 0xffffffffu;
+                rec[kTileMrefOff + row] = __float_as_uint(mref);
                 if (t == 0) rec[kTileCountOff] = (uint32_t)nU;
             }
             if (idx && row < nrows) {
@@ -396,7 +476,7 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                 int o = 0;
 #pragma unroll
                 for (int u = 0; u < UM; u++)
-                    if (16 * (u / 16) < N && key[u] >= tau && key[u] != 0u && o < A.K) out[o++] = sm.ulist[u];
+                    if (((mw[u >> 5] >> (u & 31)) & 1u) && o < A.K) out[o++] = sm.ulist[u];
                 for (; o < A.K; o++) out[o] = -1;
             }
         }
