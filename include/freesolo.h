@@ -140,7 +140,9 @@ fs_status fs_forward_host(const fs_params *p, const void *hQ, const void *hK, co
  * Returns FS_ERR_TIMEOUT if a kernel gave up a bounded wait since the last check,
  * FS_ERR_KERNEL_CHECK if a kernel found its inputs inconsistent (e.g. more distinct
  * selected cells in a 128-row tile than the bound derived from W and P),
- * FS_ERR_CUDA if the stream reports an error, else FS_OK. */
+ * FS_ERR_CUDA if the stream reports an error, else FS_OK.
+ * ws == NULL: the flag read and cleared is the status word of fs_select_topk_noalloc on
+ * the current device (FS_OK without touching the GPU if that call never ran there). */
 fs_status fs_sync_status(void *ws, void *stream);
 
 /* Static description of a status code. */
@@ -152,19 +154,27 @@ const char *fs_status_string(fs_status s);
  * a fixed device-memory budget planned in advance, plugins whose host framework owns all
  * device allocations, and latency-critical loops where cudaMalloc/cudaFree would stall on
  * a device-wide synchronization.  Its one scratch buffer, the TopP exit table, is a
- * fixed array of FS_NOALLOC_MAX_CELLS ints (4 MiB) compiled into the library; every GPU
- * that loads the library holds it until the process exits.  The call allocates nothing:
- * no cudaMalloc, no cudaFree, no allocating library routine.
+ * fixed array of FS_NOALLOC_MAX_CELLS ints (4 MiB) compiled into the library, beside a
+ * one-int status word; every GPU that loads the library holds them until the process
+ * exits.  The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ * routine.
  *   - With pruning on (W, P >= 0), B * H * floor(Nk / s) must not exceed
  *     FS_NOALLOC_MAX_CELLS, else FS_ERR_UNSUPPORTED is returned before anything runs.
- *   - The first call on a device does a one-time set-up with that device current (it
- *     looks up the array's device address); make that first call before any stream
- *     capture begins.
+ *   - Set-up: with the device current, the call looks up the array's device address (a
+ *     host-side query).  It does so on every call made outside stream capture, so a device
+ *     reset (cudaDeviceReset, which reloads the library's module) leaves nothing stale;
+ *     inside a capture it reuses the address an earlier call on that device found.  So make
+ *     the first call on a device, and the first call after a device reset, before any
+ *     stream capture begins.
  *   - All calls on a device share the one array, which keeps the last call's contents
  *     (nothing in it has to start at zero: each call writes every entry it reads).  Calls
  *     that overlap on the GPU (different streams, or threads, without ordering between
  *     them) race on it; order them, e.g. by issuing them on one stream.
- * Arguments, layouts and the other errors are those of fs_select_topk. */
+ *   - Device-side failures (a bounded wait that ran out, a failed consistency check:
+ *     idx may then be partly unwritten) are recorded in the status word, which stays set
+ *     until fs_sync_status(NULL, stream) reads and clears it (FS_ERR_TIMEOUT or
+ *     FS_ERR_KERNEL_CHECK).
+ * Arguments, layouts and the argument errors are those of fs_select_topk. */
 #define FS_NOALLOC_MAX_CELLS (1 << 20)
 fs_status fs_select_topk_noalloc(const fs_params *p, const void *Q, const float *kbar,
                                  const float *amax, int32_t *idx, void *stream);

@@ -516,7 +516,7 @@ extern "C" fs_status fs_forward_host(const fs_params *p, const void *hQ, const v
 extern "C" fs_status fs_sync_status(void *ws, void *stream) {
     cudaStream_t st = (cudaStream_t)stream;
     if (cudaStreamSynchronize(st) != cudaSuccess) return FS_ERR_CUDA;
-    if (!ws) return FS_OK;
+    if (!ws) return noalloc_take_status();      // fs_select_topk_noalloc's status word
     int flag = 0;
     if (cudaMemcpy(&flag, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FS_ERR_CUDA;
     if (flag != kFlagOk) {
