@@ -73,6 +73,8 @@ WsLayout layout(const fs_params *p) {
     L.krot = off;  off += align256(BH * (size_t)(p->Nk - kr0) * kD * 2);
     L.part = off;  off += align256(attn_part_bytes(p));      // split CTAs' partial states (decoding)
     L.tlist = off; off += align256(BH * (size_t)exit_list_words(p->P) * 4);   // TopP member lists (decoding)
+    const Dev D = make_dev(p);
+    L.tplist = off; off += align256(BH * (size_t)((p->Nq + 127) / 128) * tile_list_words(D) * 4);   // tiles' TopP
     L.total = off;
     return L;
 }
@@ -154,8 +156,11 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
         int *exitn = at<int>(ws, L.exitn);
         int *tlist = D.prune && exit_list_mode(D) ? at<int>(ws, L.tlist) : nullptr;
         if (D.prune && launch_exit_times(D, amax, exitn, st, tlist) != cudaSuccess) return FS_ERR_CUDA;
+        int *tplist = tile_list_words(D) > 0 ? at<int>(ws, L.tplist) : nullptr;
+        if (tplist && launch_tile_lists(D, exitn, tplist, st) != cudaSuccess) return FS_ERR_CUDA;
         uint32_t *tiles = at<uint32_t>(ws, L.tiles);
-        if (launch_select_tc(D, Q, kbar, amax, exitn, nullptr, tiles, at<int>(ws, L.flag), st, tlist) != cudaSuccess)
+        if (launch_select_tc(D, Q, kbar, amax, exitn, nullptr, tiles, at<int>(ws, L.flag), st, tlist, tplist) !=
+            cudaSuccess)
             return FS_ERR_CUDA;
         if (!fk.close(st, rs)) return FS_ERR_CUDA;
         return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), at<float>(ws, L.part),
@@ -197,8 +202,9 @@ fs_status validate_params(const fs_params *p) { return validate(p); }
 
 cudaError_t launch_selection(const fs_params *p, const Dev &D, const void *Q, const float *kbar,
                              const float *amax, const int *exitn, int32_t *idx, int *dev_flag,
-                             cudaStream_t st) {
-    if (select_tc_supported(p)) return launch_select_tc(D, Q, kbar, amax, exitn, idx, nullptr, dev_flag, st);
+                             cudaStream_t st, const int *tplist) {
+    if (select_tc_supported(p))
+        return launch_select_tc(D, Q, kbar, amax, exitn, idx, nullptr, dev_flag, st, nullptr, tplist);
     return launch_select(D, p->dtype, Q, kbar, amax, exitn, idx, st);
 }
 Dev make_dev_params(const fs_params *p) { return make_dev(p); }
@@ -242,7 +248,9 @@ extern "C" fs_status fs_select_topk(const fs_params *p, const void *Q, const flo
     if (!kbar || !amax) return FS_ERR_INVALID_ARG;
     int *exitn = at<int>(ws, L.exitn);
     if (D.prune && launch_exit_times(D, amax, exitn, st) != cudaSuccess) return FS_ERR_CUDA;
-    return cuda_status(launch_selection(p, D, Q, kbar, amax, exitn, idx, at<int>(ws, L.flag), st));
+    int *tplist = select_tc_supported(p) && tile_list_words(D) > 0 ? at<int>(ws, L.tplist) : nullptr;
+    if (tplist && launch_tile_lists(D, exitn, tplist, st) != cudaSuccess) return FS_ERR_CUDA;
+    return cuda_status(launch_selection(p, D, Q, kbar, amax, exitn, idx, at<int>(ws, L.flag), st, tplist));
 }
 
 extern "C" fs_status fs_select_topk_rerank(const fs_params *p, const void *Q, const void *K, const float *kbar,

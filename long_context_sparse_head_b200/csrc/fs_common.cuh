@@ -37,7 +37,7 @@ struct Dev {
 
 // Workspace layout (byte offsets from ws; each segment 256-byte aligned).
 struct WsLayout {
-    size_t flag, exitn, kbar, amax, idx, olr, rope, tiles, rope_abs, krot, part, tlist, total;
+    size_t flag, exitn, kbar, amax, idx, olr, rope, tiles, rope_abs, krot, part, tlist, tplist, total;
 };
 
 // Per-tile selection record passed from the tensor-core selection kernel to the fused
@@ -138,7 +138,7 @@ enum KernelId : int {
     kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
     kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kRerank, kIdxTiles, kBwdRotate, kBwdRows,
     kBwdWindowKv, kBwdCells, kBwdReadoutKv, kBwdDalpha, kTreePrep, kTreeMerge, kTreeNodes, kTreeSearch,
-    kBwdLrRows, kRerankTc, kReadoutRows, kAttnCombine, kNumKernels
+    kBwdLrRows, kRerankTc, kReadoutRows, kAttnCombine, kTileLists, kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
@@ -188,6 +188,11 @@ bool exit_list_mode(const Dev &P);
 int exit_list_words(int P);                      // per (b, h)
 cudaError_t launch_exit_times(const Dev &P, const float *amax, int *exitn, cudaStream_t st,
                               int *tlist = nullptr);
+// TopP(n_min) of every 128-query tile, from the exit table: per (b, h, tile) tile_list_words
+// ints, the count then the member cells ascending.  Used when the call is not decoding-
+// shaped, pruning is on with W >= 1 and the tensor-core selection applies (0 words else).
+int tile_list_words(const Dev &P);
+cudaError_t launch_tile_lists(const Dev &P, const int *exitn, int *lists, cudaStream_t st);
 // eq. (12) token-level rerank of the selection (CUDA cores, |A_i| <= 128)
 bool rerank_supported(const fs_params *p);
 cudaError_t launch_rerank(const Dev &P, fs_dtype dt, const void *Q, const void *K, const float *kbar,
@@ -224,11 +229,11 @@ bool select_tc_supported(const fs_params *p);
 // from them and the recent cells instead of a scan of the whole exit table)
 cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, const float *amax,
                              const int *exitn, int32_t *idx, uint32_t *tiles, int *dev_flag,
-                             cudaStream_t st, const int *tlist = nullptr);
+                             cudaStream_t st, const int *tlist = nullptr, const int *tplist = nullptr);
 // selection with whichever kernel applies (tensor cores for bf16 when supported)
 cudaError_t launch_selection(const fs_params *p, const Dev &D, const void *Q, const float *kbar,
                              const float *amax, const int *exitn, int32_t *idx, int *dev_flag,
-                             cudaStream_t st);
+                             cudaStream_t st, const int *tplist = nullptr);
 // status word of fs_select_topk_noalloc on the current device, read and cleared
 fs_status noalloc_take_status();
 // FS-B (eqs. (10)-(11)): forest buffer size, build (tau: host [H] or NULL), search

@@ -35,7 +35,8 @@ const char *const kNames[kNumKernels] = {"cell_summaries", "exit_times", "select
                                          "cache_append", "cache_attend", "rerank", "idx_tiles",
                                          "bwd_rotate", "bwd_win_rows", "bwd_window_kv", "bwd_cells",
                                          "bwd_readout_kv", "bwd_dalpha", "tree_prep", "tree_merge",
-                                         "tree_nodes", "tree_search", "bwd_lr_rows", "rerank_tc", "readout_rows", "attn_combine"};
+                                         "tree_nodes", "tree_search", "bwd_lr_rows", "rerank_tc", "readout_rows", "attn_combine",
+                                         "tile_lists"};
 }  // namespace
 
 LaunchScope::LaunchScope(int id_, cudaStream_t st_) : id(id_), st(st_), slot(-1) {

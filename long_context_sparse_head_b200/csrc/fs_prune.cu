@@ -249,6 +249,62 @@ __global__ void __launch_bounds__(kRangeThreads) topp_range_kernel(const float *
     }
 }
 
+// TopP(n_min) of each 128-query tile (n_min = the candidate count of its first row): the
+// cells c < n_min with exit(c) > n_min, ascending, count first.  With W >= 1 the union of a
+// tile's admitted sets is exactly these members below n_min - W followed by the recent
+// range [n_min - W, n_max), so the selection builds it without scanning the prefix.  One
+// warp per (b, h, tile); eight coalesced exit-time loads per lane in flight.
+namespace {
+constexpr int kListWarps = 4;
+}
+__global__ void __launch_bounds__(kListWarps * 32) tile_lists_kernel(const int *__restrict__ exitn, int C, int q0,
+                                                                      int w, int ntiles, long long ntot, int P,
+                                                                      int *__restrict__ lists, int words) {
+    griddep_wait();
+    const long long id = (long long)blockIdx.x * kListWarps + (threadIdx.x >> 5);
+    if (id >= ntot) return;
+    const int lane = threadIdx.x & 31;
+    const long long bh = id / ntiles;
+    const int t = (int)(id - bh * ntiles);
+    const int n = cand_count(q0 + 128 * t, w, C);
+    const int *ex = exitn + bh * C;
+    int *out = lists + id * words;
+    int cnt = 0;
+    for (int base = 0; base < n; base += 32 * kScanBlocks) {
+        int e[kScanBlocks];
+#pragma unroll
+        for (int k = 0; k < kScanBlocks; k++) {
+            const int c = base + 32 * k + lane;
+            e[k] = c < n ? __ldg(ex + c) : 0;
+        }
+#pragma unroll
+        for (int k = 0; k < kScanBlocks; k++) {
+            const int c = base + 32 * k + lane;
+            const bool in = c < n && e[k] > n;
+            const unsigned m = __ballot_sync(kFull, in);
+            const int pos = cnt + __popc(m & ((1u << lane) - 1u));
+            if (in && pos < P) out[1 + pos] = c;
+            cnt += __popc(m);
+        }
+    }
+    if (lane == 0) out[0] = min(cnt, P);
+}
+
+int tile_list_words(const Dev &P) {
+    if (!P.prune || P.W < 1 || P.Nq <= 0 || exit_list_mode(P) || P.W + P.P + 10 > 128) return 0;
+    return 1 + (P.P > 0 ? P.P : 0);
+}
+
+cudaError_t launch_tile_lists(const Dev &P, const int *exitn, int *lists, cudaStream_t st) {
+    const int words = tile_list_words(P);
+    const int ntiles = (P.Nq + 127) / 128;
+    const long long ntot = (long long)P.B * P.H * ntiles;
+    if (words == 0 || ntot == 0) return cudaSuccess;
+    LaunchScope scope(kTileLists, st);
+    return launch_pdl(tile_lists_kernel, dim3((unsigned)((ntot + kListWarps - 1) / kListWarps)), dim3(kListWarps * 32),
+                      0, st, exitn, P.C, P.q0, P.w, ntiles, ntot, P.P, lists, words);
+}
+
 bool exit_list_mode(const Dev &P) {
     if (!(P.P > 0 && P.Nq > 0 && P.B * P.H * P.C > 0)) return false;
     const int n_lo = cand_count(P.q0, P.w, P.C), n_hi = cand_count(P.q0 + P.Nq - 1, P.w, P.C);

@@ -7,9 +7,10 @@
 // One CTA per 128 query rows of a (batch, head).  The rows of a tile have at most five
 // distinct candidate prefixes n (a prefix grows by one cell every s = 32 positions), so
 // U = union of their admitted sets is at most W + P + 10 cells (<= 128 here).  Warps 0-3
-// build U from the TopP exit table (ordered compaction; when decoding, from the exit-times
-// kernel's list of the cells that are TopP members at an asked prefix plus the recent
-// cells, so the whole table is not scanned), then stage the fp32 mean keys of
+// build U: with W >= 1, from the tile's TopP(n_min) list (tile-list kernel) below the
+// recent range followed by that range; when decoding, from the exit-times kernel's list of
+// the cells that are TopP members at an asked prefix plus the recent cells; otherwise by
+// an ordered compaction of the TopP exit table.  Then they stage the fp32 mean keys of
 // U as three bf16 parts hi + mid + lo (the split carries the fp32 mantissa, so the bf16
 // tensor-core products sum to the fp32 dot product up to accumulation rounding), in the
 // 128-byte-swizzled layout of a K-major MMA operand.  One thread issues
@@ -34,7 +35,6 @@ constexpr int W_MMA = 4, NWARPS = 5, NTHREADS = NWARPS * 32;   // warp 4: Q load
 constexpr uint32_t TMEM_COLS = 128;
 constexpr int TILE_BYTES = BM * kD * 2;
 constexpr int kSelBarrier = 1;   // named barrier of the 128 selection threads
-constexpr int kSmall = 16;       // bracket size at which the K-th search finishes by ranks
 
 template <int UM> struct SelSmem {       // UM: capacity of the union (a multiple of 16)
     __nv_bfloat16 q[BM * kD];              // Q tile (NoPE)
@@ -54,6 +54,7 @@ template <int UM> struct SelSmem {       // UM: capacity of the union (a multipl
 struct SelArgs {
     int Nq, Nk, q0, w, C, K, W, P, H;
     int tl_words;           // words per (b, h) of the member lists (with tlist)
+    int tp_words;           // words per (b, h, tile) of the tiles' TopP lists (with tplist)
     int prune, has_prior;
     float scale;
     float lambda[FS_MAX_HEADS];
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(NTHREADS, UM <= 80 ? 3 : 2)
 select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const float *__restrict__ kbar,
                  const float *__restrict__ amax, const int *__restrict__ exitn,
                  int32_t *__restrict__ idx, uint32_t *__restrict__ tiles, int *dev_flag,
-                 const int *__restrict__ tlist) {
+                 const int *__restrict__ tlist, const int *__restrict__ tplist) {
     extern __shared__ uint8_t smraw[];
     const uint32_t sbase = tc::smem_u32(smraw);
     SelSmem<UM> &sm = *reinterpret_cast<SelSmem<UM> *>(smraw + (((sbase + 1023u) & ~1023u) - sbase));
@@ -205,6 +206,30 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
             }
             sel_sync();
             total = sm.warp_cnt[0];
+            sel_sync();
+        } else if (tplist) {
+            // prefill with W >= 1: U is TopP(n_min) below the recent range, then the recent
+            // range [n_min - W, n_max) itself (every cell there is recent for some prefix of
+            // the tile); TopP(n_min) comes ascending from the tile-list kernel
+            const int *lst = tplist + ((size_t)bh * gridDim.x + blockIdx.x) * A.tp_words;
+            const int nl = min(__ldg(lst), A.tp_words - 1);
+            const int rlo = max(0, n_min - A.W);
+            if (t == 0) sm.ncand = 0;
+            sel_sync();
+            if (t < nl) {                       // members below rlo form a prefix of the list
+                const bool below = __ldg(lst + 1 + t) < rlo;
+                const bool next_below = t + 1 < nl && __ldg(lst + 2 + t) < rlo;
+                if (below && !next_below) sm.ncand = t + 1;
+            }
+            sel_sync();
+            const int nold = sm.ncand;
+            total = nold + max(0, n_max - rlo);
+            for (int u = t; u < min(total, UM); u += 128) {
+                const int c = u < nold ? __ldg(lst + 1 + u) : rlo + (u - nold);
+                sm.ulist[u] = c;
+                sm.amask[u] = (uint8_t)admit_bits(c, __ldg(ex + c));
+                sm.acell[u] = am[c];
+            }
             sel_sync();
         } else {
             // 1024 cells per round, eight consecutive ones per thread: the exit times are
@@ -364,16 +389,11 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                     key[u] = 0u;
                 }
             }
-            // K-th largest key: bisection while more than kSmall keys lie in the bracket
-            // [lo, hi), with clo = count(key >= lo) >= K > chi = count(key >= hi) (keys are
-            // unique, so the bracket holds exactly clo - chi of them); then those keys are
-            // compacted into shared memory and the (K - chi)-th largest among them is found
-            // by counting ranks, with no data-dependent loop
+            // K-th largest key by bisection: count(key >= lo) >= K > count(key >= hi)
             uint32_t tau = 1u;
             if (na > A.K) {
                 uint32_t lo = 1u << 7, hi = (0x1000000u + 1u) << 7;
-                int clo = na, chi = 0;
-                while (clo - chi > kSmall && clo != A.K) {
+                while (hi - lo > 1u) {
                     const uint32_t mid = lo + ((hi - lo) >> 1);
                     int cp[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent partial counts
 #pragma unroll
@@ -385,37 +405,12 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                     const int cnt = ((cp[0] + cp[1]) + (cp[2] + cp[3])) + ((cp[4] + cp[5]) + (cp[6] + cp[7]));
                     if (cnt >= A.K) {
                         lo = mid;
-                        clo = cnt;
+                        if (cnt == A.K) break;
                     } else {
                         hi = mid;
-                        chi = cnt;
                     }
                 }
                 tau = lo;
-                if (clo != A.K) {
-                    // the mean-key operand is no longer read once S is in tensor memory; its
-                    // first kSmall x BM words hold the brackets, key j of row r at j * BM + r
-                    uint32_t *buf = reinterpret_cast<uint32_t *>(sm.kb[0]);
-                    int m = 0;
-#pragma unroll
-                    for (int u = 0; u < UM; u++) {
-                        if (16 * (u / 16) < N && key[u] >= lo && key[u] < hi) {
-                            buf[m * BM + row] = key[u];
-                            m++;
-                        }
-                    }
-                    uint32_t bk[kSmall];
-#pragma unroll
-                    for (int j = 0; j < kSmall; j++) bk[j] = j < m ? buf[j * BM + row] : 0u;
-                    const int need = A.K - chi;            // 1 <= need < m
-#pragma unroll
-                    for (int j = 0; j < kSmall; j++) {
-                        int r = 0;
-#pragma unroll
-                        for (int k = 0; k < kSmall; k++) r += bk[k] > bk[j];
-                        if (j < m && r == need - 1) tau = bk[j];
-                    }
-                }
             }
             uint32_t mw[UMAX / 32] = {0u, 0u, 0u, 0u};   // selected union positions
 #pragma unroll
@@ -503,18 +498,20 @@ namespace {
 int union_bound(const Dev &P) { return P.prune ? P.W + P.P + 10 : P.C; }
 template <int UM> cudaError_t launch_um(const CUtensorMap &tq, const SelArgs &A, bool prior, dim3 grid,
                                          const float *kbar, const float *amax, const int *exitn, int32_t *idx,
-                                         uint32_t *tiles, int *dev_flag, const int *tlist, cudaStream_t st) {
+                                         uint32_t *tiles, int *dev_flag, const int *tlist, const int *tplist,
+                                         cudaStream_t st) {
     const size_t smem = sizeof(SelSmem<UM>) + 1024;
     // the erf prior is a separate instantiation: without it the unrolled score loop stays small
     auto kern = prior ? select_tc_kernel<true, UM> : select_tc_kernel<false, UM>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    return launch_pdl(kern, grid, dim3(NTHREADS), smem, st, tq, A, kbar, amax, exitn, idx, tiles, dev_flag, tlist);
+    return launch_pdl(kern, grid, dim3(NTHREADS), smem, st, tq, A, kbar, amax, exitn, idx, tiles, dev_flag, tlist,
+                      tplist);
 }
 }  // namespace
 
 cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, const float *amax,
                              const int *exitn, int32_t *idx, uint32_t *tiles, int *dev_flag,
-                             cudaStream_t st, const int *tlist) {
+                             cudaStream_t st, const int *tlist, const int *tplist) {
     if (P.Nq == 0) return cudaSuccess;
     const int BH = P.B * P.H;
     CUtensorMap tq;
@@ -524,7 +521,9 @@ cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, con
     A.W = P.W; A.P = P.P; A.H = P.H; A.prune = P.prune; A.has_prior = P.has_prior;
     A.scale = P.scale;
     A.tl_words = exit_list_words(P.P);
+    A.tp_words = tile_list_words(P);
     if (!P.prune) tlist = nullptr;
+    if (tlist || A.tp_words == 0) tplist = nullptr;
     for (int h = 0; h < FS_MAX_HEADS; h++) {
         A.lambda[h] = P.lambda[h];
         A.inv2sigma[h] = P.inv2sigma[h];
@@ -532,8 +531,8 @@ cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, con
     const dim3 grid((P.Nq + BM - 1) / BM, BH);
     LaunchScope scope(kSelectTc, st);
     if (union_bound(P) <= 80)
-        return launch_um<80>(tq, A, P.has_prior, grid, kbar, amax, exitn, idx, tiles, dev_flag, tlist, st);
-    return launch_um<UMAX>(tq, A, P.has_prior, grid, kbar, amax, exitn, idx, tiles, dev_flag, tlist, st);
+        return launch_um<80>(tq, A, P.has_prior, grid, kbar, amax, exitn, idx, tiles, dev_flag, tlist, tplist, st);
+    return launch_um<UMAX>(tq, A, P.has_prior, grid, kbar, amax, exitn, idx, tiles, dev_flag, tlist, tplist, st);
 }
 
 }  // namespace fs
