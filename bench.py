@@ -50,6 +50,12 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--quick", action="store_true", help="skip e2e, CPU baseline, extras")
+    ap.add_argument("--variant", choices=["forward", "rerank", "backward", "tree", "tree_decode"],
+                    default="forward",
+                    help="time only this variant of the pass on --workload (one JSON line, no "
+                         "roofline or baselines): the eq. (12) rerank, the backward pass, or "
+                         "FS-B; 'forward' is the benchmark itself")
+    ap.add_argument("--beam", type=int, default=32, help="FS-B beam width for --variant tree")
     return ap.parse_args()
 
 
@@ -490,6 +496,55 @@ def time_tree(fs, torch, inp, beam=32, steps=5, warmup=3):
                     "per-row readout and the tensor-core window + combine" % beam}
 
 
+def time_tree_decode(fs, torch, inp, beam=32, steps=20, warmup=3):
+    """FS-B decoding on a growing archive: the forest of the archive (all but the last Nq
+    tokens) is built once; each step appends the last Nq tokens' cells to it (only the
+    trees those cells complete are rebuilt), searches both forests for the Nq queries and
+    runs the readout + window on the selected cells.  Archive summaries precomputed."""
+    wl = inp.wl
+    p = make_params(fs, inp)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    Q, K, V = (torch.from_numpy(x).cuda().to(dt) for x in (inp.Q, inp.K, inp.V))
+    O = torch.empty_like(Q)
+    ws = fs.alloc_workspace(p)
+    C = wl.Nk // wl.s
+    arch = (wl.Nk - wl.Nq) // wl.s                     # cells before the appended queries
+    kbar = torch.empty((wl.B, wl.H, C, wl.d), dtype=torch.float32, device="cuda")
+    amax = torch.empty((wl.B, wl.H, C), dtype=torch.float32, device="cuda")
+    fs.cell_summaries(p, K, kbar, amax)
+    tau = torch.quantile(amax.transpose(0, 1).reshape(wl.H, -1), 0.75, dim=1).cpu().tolist()
+    forest = fs.alloc_forest(p)
+    fs.forest_build(p, kbar, amax, forest, tau)        # then rewritten from `arch` every step
+    idx = torch.empty((wl.B, wl.H, wl.Nq, wl.K), dtype=torch.int32, device="cuda")
+
+    def step():
+        fs.forest_append(p, arch, kbar, amax, forest, tau)
+        fs.select_topk_tree(p, Q, forest, idx, ws, beam, 1.0)
+        fs.forward(p, Q, K, V, O, ws, kbar=kbar, amax=amax, idx=idx)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    fs.timing_enable(True)
+    fs.kernel_times()
+    step()
+    torch.cuda.synchronize()
+    kt = {k: round(v[1], 4) for k, v in fs.kernel_times().items() if v[0]}
+    fs.timing_enable(False)
+    fs.sync_status(ws)
+    return {"value": wl.queries / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "kernel_ms": kt,
+            "note": "FS-B on a growing archive: forest of the %d-cell archive built once; per step "
+                    "fs_forest_append of the %d new cells (only the trees they complete), the "
+                    "beam search (width %d, c = 1, both forests) and the readout + window on the "
+                    "selection; archive summaries precomputed" % (arch, C - arch, beam)}
+
+
 def time_backward(fs, torch, inp, steps=3, warmup=3):
     """The backward pass of eq. (2) on a workload (fs_backward on the cells fs_select_topk
     chose; the selection is outside the timed region).  Returns query-tokens/s and the
@@ -698,6 +753,7 @@ def run_ours(args):
                                 "note": "archive summaries precomputed" if arch else ""}
                 if name == "decode256k":   # the same tokens through the FS-L streaming cache
                     extras["stream256k"] = time_stream(fs, torch, inp2)
+                    extras["decode256k_tree_append"] = time_tree_decode(fs, torch, inp2)
                 del inp2
                 torch.cuda.empty_cache()
             extras[wl.name + "_rerank"] = time_rerank(fs, torch, inp)
@@ -714,10 +770,41 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_variant(args):
+    """One variant of the pass on one workload, on this process's GPU (rank 0 prints)."""
+    import torch
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    import long_context_sparse_head_b200 as fs
+    from workloads import CONFIGS, generate
+    fs.load()
+    wl = CONFIGS[args.workload].with_(seed=replica_seed(CONFIGS[args.workload].seed, rank))
+    inp = generate(wl)
+    warm = max(args.warmup, 1)
+    if args.variant == "rerank":
+        res = time_rerank(fs, torch, inp, steps=args.steps, warmup=warm)
+    elif args.variant == "backward":
+        res = time_backward(fs, torch, inp, steps=args.steps, warmup=warm)
+    elif args.variant == "tree_decode":
+        res = time_tree_decode(fs, torch, inp, beam=args.beam, steps=args.steps, warmup=warm)
+    else:
+        res = time_tree(fs, torch, inp, beam=args.beam, steps=args.steps, warmup=warm)
+    ms, value = aggregate(res["ms_per_step"], wl.queries, world)
+    res.update({"variant": args.variant, "workload": wl.name, "n_gpus": world, "steps": args.steps,
+                "warmup": warm, "ms_per_step": ms, "value": value})
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.variant != "forward":
+        run_variant(args)
     else:
         run_ours(args)
 

@@ -261,17 +261,33 @@ fs_status fs_cache_status(void *cache, void *stream);
  * gives base FS's selection. */
 #define FS_TREE_MAX_BEAM 64
 
-/* Bytes of the forest buffer for p (B, H, Nk, s): O(B H (Nk/s) log2(Nk/s) d) floats. */
+/* Bytes of the forest buffer for p (B, H, Nk, s): O(B H (Nk/s) log2(Nk/s) d) floats.
+ * A forest buffer is laid out for its capacity: the largest cell count whose forest fits
+ * in its bytes (so a buffer sized for a longer archive serves every shorter one).  Pass
+ * the same forest_bytes to every call on one buffer. */
 fs_status fs_forest_bytes(const fs_params *p, size_t *bytes);
 
-/* Builds both forests from the cell summaries (fs_cell_summaries' kbar [B,H,C,d], amax
- * [B,H,C], device f32) into the caller's device buffer `forest`.  tau: HOST [H]
- * thresholds of eq. (10), or NULL for forest 0 alone. */
+/* Builds both forests for the C = Nk/s cells of p from the cell summaries
+ * (fs_cell_summaries' kbar [B,H,C,d], amax [B,H,C], device f32) into the caller's device
+ * buffer `forest`.  tau: HOST [H] thresholds of eq. (10), or NULL for forest 0 alone. */
 fs_status fs_forest_build(const fs_params *p, const float *kbar, const float *amax, const float *tau,
                           void *forest, size_t forest_bytes, void *stream);
 
+/* The archive grew ("FreeSolo" summary §3.4: balanced trees over an archive that keeps
+ * growing): brings a forest built for at least prev_cells cells to the C = Nk/s cells of p
+ * by rebuilding only the trees whose blocks end after cell prev_cells, as a binary counter
+ * carries (amortised O(log C) trees per appended cell; a block of 2^k completes once every
+ * 2^k cells).  kbar, amax: summaries of all C cells; those of the first prev_cells cells,
+ * B, H, the capacity and tau (same values, or NULL as before) must be those of the earlier
+ * build.  prev_cells below the cells built rebuilds from there (the later cells were
+ * rewritten).  A forest that does not match (other sizes, fewer than prev_cells cells
+ * built) is marked in its header, and the next search reports FS_ERR_KERNEL_CHECK through
+ * fs_sync_status.  0 <= prev_cells <= C; prev_cells = 0 is fs_forest_build. */
+fs_status fs_forest_append(const fs_params *p, int prev_cells, const float *kbar, const float *amax,
+                           const float *tau, void *forest, size_t forest_bytes, void *stream);
+
 /* FS-B selection: idx [B,H,Nq,K] (ascending, -1 padded) for the device queries Q, from a
- * forest built with the same p.  1 <= beam <= FS_TREE_MAX_BEAM; c_explore is eq. (11)'s
+ * forest built (or appended to) for the same B, H and C = Nk/s.  1 <= beam <= FS_TREE_MAX_BEAM; c_explore is eq. (11)'s
  * c.  ws (fs_workspace_size bytes) carries the device error flag: a forest not built for
  * these sizes is reported by fs_sync_status as FS_ERR_KERNEL_CHECK. */
 fs_status fs_select_topk_tree(const fs_params *p, const void *Q, const void *forest, size_t forest_bytes,

@@ -28,7 +28,7 @@ EXPORTS = ("fs_workspace_size", "fs_cell_summaries", "fs_select_topk", "fs_forwa
            "fs_select_topk_noalloc", "fs_cache_bytes", "fs_cache_reset", "fs_cache_append",
            "fs_cache_attend", "fs_cache_status", "fs_select_topk_rerank", "fs_forward_rerank",
            "fs_backward_workspace_size", "fs_backward", "fs_forest_bytes", "fs_forest_build",
-           "fs_select_topk_tree", "fs_forward_tree")
+           "fs_select_topk_tree", "fs_forward_tree", "fs_forest_append")
 
 
 class FsError(RuntimeError):
@@ -93,6 +93,7 @@ def load():
         fp = ctypes.POINTER(ctypes.c_float)
         L.fs_forest_bytes.argtypes = [P, ctypes.POINTER(sz)]
         L.fs_forest_build.argtypes = [P, vp, vp, fp, vp, sz, vp]
+        L.fs_forest_append.argtypes = [P, ctypes.c_int, vp, vp, fp, vp, sz, vp]
         L.fs_select_topk_tree.argtypes = [P, vp, vp, sz, ctypes.c_int, ctypes.c_float, vp, vp, sz, vp]
         L.fs_forward_tree.argtypes = [P, vp, vp, vp, fp, ctypes.c_int, ctypes.c_float, vp, vp, vp, sz, vp,
                                       sz, vp]
@@ -244,6 +245,14 @@ def forest_build(params, kbar, amax, forest, tau=None, stream=None):
     t = _tau(params, tau)
     _check(load().fs_forest_build(params.ref(), _ptr(kbar), _ptr(amax), t[0] if t else None, _ptr(forest),
                                   forest.numel() * forest.element_size(), _stream(stream)), "fs_forest_build")
+
+
+def forest_append(params, prev_cells, kbar, amax, forest, tau=None, stream=None):
+    """Rebuild only the trees whose blocks end after cell prev_cells (growing archive)."""
+    t = _tau(params, tau)
+    _check(load().fs_forest_append(params.ref(), int(prev_cells), _ptr(kbar), _ptr(amax), t[0] if t else None,
+                                   _ptr(forest), forest.numel() * forest.element_size(), _stream(stream)),
+           "fs_forest_append")
 
 
 def select_topk_tree(params, Q, forest, idx, ws, beam, c_explore=1.0, stream=None):

@@ -351,7 +351,21 @@ extern "C" fs_status fs_forest_build(const fs_params *p, const float *kbar, cons
     if (tau)
         for (int h = 0; h < p->H; h++)
             if (std::isnan(tau[h])) return FS_ERR_INVALID_ARG;
-    return cuda_status(launch_tree_build(p, kbar, amax, tau, forest, (cudaStream_t)stream));
+    return cuda_status(launch_tree_build(p, kbar, amax, tau, forest, forest_bytes_, 0, (cudaStream_t)stream));
+}
+
+extern "C" fs_status fs_forest_append(const fs_params *p, int prev_cells, const float *kbar, const float *amax,
+                                      const float *tau, void *forest, size_t forest_bytes_, void *stream) {
+    fs_status s = validate(p);
+    if (s != FS_OK) return s;
+    const int C = p->Nk / p->s;
+    if (prev_cells < 0 || prev_cells > C) return FS_ERR_INVALID_ARG;
+    if (!forest || forest_bytes_ < forest_bytes(p)) return FS_ERR_WORKSPACE;
+    if (C > 0 && (!kbar || !amax)) return FS_ERR_INVALID_ARG;
+    if (tau)
+        for (int h = 0; h < p->H; h++)
+            if (std::isnan(tau[h])) return FS_ERR_INVALID_ARG;
+    return cuda_status(launch_tree_build(p, kbar, amax, tau, forest, forest_bytes_, prev_cells, (cudaStream_t)stream));
 }
 
 extern "C" fs_status fs_select_topk_tree(const fs_params *p, const void *Q, const void *forest,
@@ -365,8 +379,8 @@ extern "C" fs_status fs_select_topk_tree(const fs_params *p, const void *Q, cons
     if (!forest || forest_bytes_ < forest_bytes(p)) return FS_ERR_WORKSPACE;
     if (!ws || ws_bytes < layout(p).total) return FS_ERR_WORKSPACE;
     const Dev D = make_dev(p);
-    return cuda_status(launch_tree_search(p, D, Q, forest, beam, c_explore, idx, at<int>(ws, layout(p).flag),
-                                          (cudaStream_t)stream));
+    return cuda_status(launch_tree_search(p, D, Q, forest, forest_bytes_, beam, c_explore, idx,
+                                          at<int>(ws, layout(p).flag), (cudaStream_t)stream));
 }
 
 extern "C" fs_status fs_forward_tree(const fs_params *p, const void *Q, const void *K, const void *V,
@@ -394,9 +408,10 @@ extern "C" fs_status fs_forward_tree(const fs_params *p, const void *Q, const vo
     const Dev D = make_dev(p);
     float *kb = at<float>(ws, L.kbar), *am = at<float>(ws, L.amax);
     if (launch_summaries(D, p->dtype, K, kb, am, st) != cudaSuccess) return FS_ERR_CUDA;
-    if (launch_tree_build(p, kb, am, tau, forest, st) != cudaSuccess) return FS_ERR_CUDA;
+    if (launch_tree_build(p, kb, am, tau, forest, forest_bytes_, 0, st) != cudaSuccess) return FS_ERR_CUDA;
     int32_t *sel = idx ? idx : at<int32_t>(ws, L.idx);
-    if (launch_tree_search(p, D, Q, forest, beam, c_explore, sel, at<int>(ws, L.flag), st) != cudaSuccess)
+    if (launch_tree_search(p, D, Q, forest, forest_bytes_, beam, c_explore, sel, at<int>(ws, L.flag), st) !=
+        cudaSuccess)
         return FS_ERR_CUDA;
     // FS-B rows of one query tile pick cells across the whole prefix (their union is not
     // bounded like FS-L's), so the readout gathers per row: the readout kernel on the

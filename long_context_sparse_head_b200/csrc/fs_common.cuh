@@ -238,10 +238,13 @@ cudaError_t launch_selection(const fs_params *p, const Dev &D, const void *Q, co
 fs_status noalloc_take_status();
 // FS-B (eqs. (10)-(11)): forest buffer size, build (tau: host [H] or NULL), search
 size_t forest_bytes(const fs_params *p);
+// a forest buffer's layout is that of its capacity, the largest cell count whose forest fits
+// in its bytes (-1: not even p's cells fit); prev: cells already built (0: a full build)
+int forest_capacity(const fs_params *p, size_t bytes);
 cudaError_t launch_tree_build(const fs_params *p, const float *kbar, const float *amax, const float *tau,
-                              void *forest, cudaStream_t st);
-cudaError_t launch_tree_search(const fs_params *p, const Dev &D, const void *Q, const void *forest, int beam,
-                               float c_explore, int32_t *idx, int *dev_flag, cudaStream_t st);
+                              void *forest, size_t bytes, int prev, cudaStream_t st);
+cudaError_t launch_tree_search(const fs_params *p, const Dev &D, const void *Q, const void *forest, size_t bytes,
+                               int beam, float c_explore, int32_t *idx, int *dev_flag, cudaStream_t st);
 // fused tensor-core readout + window + combine (bf16, internally selected cells)
 bool attn_tc_supported(const fs_params *p);
 // decoding shapes (fewer tiles than SMs): the tile's chunks split over nsplit CTAs whose

@@ -19,9 +19,11 @@
 // ascending, -1 padded.
 //
 // Kernels: prep (codes, admitted prefix counts, sequences; one CTA per head), merge (one
-// launch per level; each entry's place by binary search in the other half), nodes (one
-// warp per node: mean, radius, max norm, first cell), search (one warp per query row; a
-// right child's q.mu is 2 q.mu_parent - q.mu_left, so an expansion reads one mean).
+// launch per level; each entry's place by binary search in the other half), node
+// statistics (bottom-up means, max norms and first cells per tree, then radii with one
+// thread per leaf), search (one warp per query row; a right child's q.mu is
+// 2 q.mu_parent - q.mu_left, so an expansion reads one mean).
+#include <algorithm>
 #include <cmath>
 
 #include "fs_common.cuh"
@@ -36,17 +38,22 @@ constexpr int kCodeBits = 16;
 constexpr int kSearchWarps = 4;
 constexpr int kCandCap = 2 * kMaxBeam + 32;   // children of a full beam, or the roots
 
+// A forest buffer is laid out for a capacity of C cells (the largest count whose forest
+// fits in the buffer's bytes); the cells built so far may be fewer.  Header words: magic,
+// has_tau, capacity, levels, B*H, cells built, error (a failed append check).
+enum { kHdrMagic = 0, kHdrTau, kHdrCap, kHdrLevels, kHdrBH, kHdrCells, kHdrError };
+
 struct ForestGeom {
-    int BH, C, L;
-    size_t hdr, nseq, seq, admp, code, ord, mu, meta, total;
+    int BH, C, L;           // C: capacity (layout stride)
+    size_t hdr, nseq, nprev, seq, admp, code, ord, mu, meta, total;
 };
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
-ForestGeom forest_geom(const fs_params *p) {
+ForestGeom forest_geom(int BHn, int Ccap) {
     ForestGeom g;
-    g.BH = p->B * p->H;
-    g.C = p->Nk / p->s;
+    g.BH = BHn;
+    g.C = Ccap;
     g.L = 0;
     while (g.L < 31 && (1LL << g.L) <= g.C) g.L++;
     const size_t BH = g.BH, C = g.C, L = g.L > 0 ? g.L : 1;
@@ -58,6 +65,7 @@ ForestGeom forest_geom(const fs_params *p) {
     };
     g.hdr = seg(16 * 4);
     g.nseq = seg(BH * 2 * 4);
+    g.nprev = seg(BH * 2 * 4);              // sequence lengths before the last build / append
     g.seq = seg(BH * 2 * C * 4);
     g.admp = seg(BH * (C + 1) * 4);
     g.code = seg(BH * C * 4);
@@ -70,7 +78,7 @@ ForestGeom forest_geom(const fs_params *p) {
 
 // Device view of a forest buffer.
 struct Forest {
-    int *hdr, *nseq, *seq, *admp;
+    int *hdr, *nseq, *nprev, *seq, *admp;
     uint32_t *code;
     int *ord;
     float *mu;
@@ -86,6 +94,7 @@ Forest forest_view(void *buf, const ForestGeom &g) {
     Forest F;
     F.hdr = reinterpret_cast<int *>(b + g.hdr);
     F.nseq = reinterpret_cast<int *>(b + g.nseq);
+    F.nprev = reinterpret_cast<int *>(b + g.nprev);
     F.seq = reinterpret_cast<int *>(b + g.seq);
     F.admp = reinterpret_cast<int *>(b + g.admp);
     F.code = reinterpret_cast<uint32_t *>(b + g.code);
@@ -102,34 +111,41 @@ struct TauArgs {
     float tau[FS_MAX_HEADS];
 };
 
+// cells [prev, Cn) of one (b, h): codes, sequences, admitted prefix counts (continuing the
+// scan at admp[prev]).  An append (prev > 0) first checks that the forest was built for
+// these sizes, these thresholds' presence and at least prev cells; a mismatch is recorded
+// in the header and reported by the search.
 __global__ void __launch_bounds__(1024) tree_prep_kernel(Forest F, const float *__restrict__ kbar,
                                                          const float *__restrict__ amax, int H, int has_tau,
-                                                         const TauArgs T) {
+                                                         const TauArgs T, int Cn, int prev) {
     __shared__ int wsum[32];
     __shared__ int carry;
     const int bh = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int C = F.C;
+    const int C = F.C;                             // capacity: the layout's stride
     const float tau = has_tau ? T.tau[bh % H] : 0.f;
-    if (bh == 0 && t == 0) {
-        F.hdr[0] = kTreeMagic;
-        F.hdr[1] = has_tau;
-        F.hdr[2] = C;
-        F.hdr[3] = F.L;
-        F.hdr[4] = gridDim.x;
+    if (t == 0) {
+        carry = 0;
+        if (prev > 0) {
+            const bool ok = F.hdr[kHdrMagic] == kTreeMagic && F.hdr[kHdrTau] == has_tau && F.hdr[kHdrCap] == C &&
+                            F.hdr[kHdrLevels] == F.L && F.hdr[kHdrBH] == (int)gridDim.x && F.hdr[kHdrCells] >= prev;
+            if (!ok) atomicOr(F.hdr + kHdrError, kFlagCheck);
+            carry = ok ? F.admp[(size_t)bh * (C + 1) + prev] : 0;
+        }
+        F.nprev[bh * 2 + 0] = prev;
+        F.nprev[bh * 2 + 1] = carry;
     }
-    if (t == 0) carry = 0;
     __syncthreads();
-    for (int base = 0; base < C; base += 1024) {
+    for (int base = prev; base < Cn; base += 1024) {
         const int c = base + t;
         int adm = 0;
-        if (c < C) {
-            const float *kb = kbar + ((size_t)bh * C + c) * kD;
+        if (c < Cn) {
+            const float *kb = kbar + ((size_t)bh * Cn + c) * kD;      // caller's arrays: [B*H, Cn]
             uint32_t code = 0;
 #pragma unroll
             for (int b = 0; b < kCodeBits; b++) code = (code << 1) | (kb[b] > 0.f ? 1u : 0u);
             F.code[(size_t)bh * C + c] = code;
             F.seq[((size_t)bh * 2 + 0) * C + c] = c;
-            adm = has_tau && amax[(size_t)bh * C + c] >= tau;
+            adm = has_tau && amax[(size_t)bh * Cn + c] >= tau;
         }
         int incl = adm;
 #pragma unroll
@@ -142,7 +158,7 @@ __global__ void __launch_bounds__(1024) tree_prep_kernel(Forest F, const float *
         int before = carry;
         for (int k = 0; k < warp; k++) before += wsum[k];
         const int excl = before + incl - adm;
-        if (c < C) {
+        if (c < Cn) {
             F.admp[(size_t)bh * (C + 1) + c] = excl;
             if (adm) F.seq[((size_t)bh * 2 + 1) * C + excl] = c;
         }
@@ -151,10 +167,21 @@ __global__ void __launch_bounds__(1024) tree_prep_kernel(Forest F, const float *
         __syncthreads();
     }
     if (t == 0) {
-        F.admp[(size_t)bh * (C + 1) + C] = carry;
-        F.nseq[bh * 2 + 0] = C;
+        F.admp[(size_t)bh * (C + 1) + Cn] = carry;
+        F.nseq[bh * 2 + 0] = Cn;
         F.nseq[bh * 2 + 1] = carry;
     }
+}
+
+// Header of a finished build or append (one thread, after every other kernel of it).
+__global__ void tree_header_kernel(Forest F, int BH, int has_tau, int Cn, int full) {
+    F.hdr[kHdrMagic] = kTreeMagic;
+    F.hdr[kHdrTau] = has_tau;
+    F.hdr[kHdrCap] = F.C;
+    F.hdr[kHdrLevels] = F.L;
+    F.hdr[kHdrBH] = BH;
+    F.hdr[kHdrCells] = Cn;
+    if (full) F.hdr[kHdrError] = 0;
 }
 
 __device__ __forceinline__ unsigned long long sort_key(const Forest &F, int bh, int cell) {
@@ -163,13 +190,14 @@ __device__ __forceinline__ unsigned long long sort_key(const Forest &F, int bh, 
 
 // level k's leaf order: level 0 copies the sequence; level k >= 1 merges the two sorted
 // halves of each block (an entry's place = its index in its half + the number of keys
-// below it in the other half)
-__global__ void tree_merge_kernel(Forest F, int BH, int k) {
+// below it in the other half).  Only the blocks completed since the previous build are
+// done: entry positions base + r, base = the first position of a new block, r < span.
+__global__ void tree_merge_kernel(Forest F, int BH, int k, int span) {
     const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const int C = F.C;
-    if (e >= (long long)BH * 2 * C) return;
-    const int pos = (int)(e % C);
-    const int bhf = (int)(e / C), bh = bhf >> 1, f = bhf & 1;
+    if (e >= (long long)BH * 2 * span) return;
+    const int bhf = (int)(e / span), bh = bhf >> 1, f = bhf & 1;
+    const int pos = ((F.nprev[bhf] >> k) << k) + (int)(e % span);
     const int n = F.nseq[bhf];
     if (pos >= ((n >> k) << k)) return;
     int *out = F.ord + F.lvl(bh, f, k) * C;
@@ -192,48 +220,137 @@ __global__ void tree_merge_kernel(Forest F, int BH, int k) {
     out[(blk << k) + a + lo] = cell;
 }
 
-// one warp per node of level k: mean key, radius, max norm, first cell
-__global__ void __launch_bounds__(256) tree_nodes_kernel(Forest F, const float *__restrict__ kbar,
-                                                         const float *__restrict__ amax, int BH, int k) {
+// Node statistics of level k, in two passes.
+// (1) tree_up_kernel: bottom-up over each tree's depths.  A leaf holds its cell's kbar_c,
+//     a_c and index; an internal node's mean is the average of its two children's (they
+//     cover equally many leaves), its max norm and first cell the larger / smaller of
+//     theirs; every radius starts at 0.  Work items are subtrees of at most 128 leaves,
+//     one warp each (grid-stride): depths k down to d0 = max(0, k - 7); for k > 7 a second
+//     launch takes each tree's top depths d0 - 1 .. 0 (at most 63 nodes), again one warp.
+//     A warp takes four nodes of a depth at a time, their loads issued together.
+// (2) tree_radius_kernel: rho_v = max ||kbar_c - mu_v|| over v's leaves.  One thread per
+//     leaf holds its kbar_c and walks the depths above it; a node of fewer than 32 leaves
+//     lies inside one warp and takes a butterfly maximum, a larger one a warp maximum and
+//     an atomic maximum on the radius's bits (non-negative floats order as integers, so
+//     the result does not depend on the order).
+constexpr int kUpThreads = 256, kUpSubK = 7, kUpBatch = 4, kUpMaxBlocks = 148 * 8;
+
+__device__ __forceinline__ size_t node_index(const Forest &F, int bh, int f, int k, int blk, int v) {
+    return F.lvl(bh, f, k) * 2 * (size_t)F.C + ((size_t)blk << (k + 1)) + v;
+}
+
+// top == 0: items are (tree, subtree rooted at depth d0); top == 1: items are trees, and the
+// warp fills depths d0 - 1 .. 0.  The trees are those completed since the previous build:
+// blocks nprev >> k + r, r < per, below nseq >> k.
+__global__ void __launch_bounds__(kUpThreads) tree_up_kernel(Forest F, const float *__restrict__ kbar,
+                                                             const float *__restrict__ amax, int BH, int k, int top,
+                                                             int per, int Cn) {
     const int lane = threadIdx.x & 31;
-    const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int C = F.C;
-    const long long per = 2LL * C;               // node slots per (bh, f) at this level
-    if (wid >= (long long)BH * 2 * per) return;
-    const int bhf = (int)(wid / per), bh = bhf >> 1, f = bhf & 1;
-    const int node = (int)(wid % per);
-    const int blk = node >> (k + 1), v = node & ((2 << k) - 1);
-    const int n = F.nseq[bhf];
-    if (v == 0 || blk >= (n >> k)) return;
-    const int t = 31 - __clz(v);                 // depth of v
-    const int cnt = 1 << (k - t);
-    const int *leaves = F.ord + F.lvl(bh, f, k) * C + ((size_t)blk << k) + ((size_t)(v - (1 << t)) << (k - t));
-    const float *kb = kbar + (size_t)bh * C * kD;
-    float s0 = 0.f, s1 = 0.f, A = -INFINITY;
-    int pmin = 0x7fffffff;
-    for (int j = 0; j < cnt; j++) {
-        const int c = leaves[j];
-        const float2 x = *reinterpret_cast<const float2 *>(kb + (size_t)c * kD + 2 * lane);
-        s0 += x.x;
-        s1 += x.y;
-        A = fmaxf(A, amax[(size_t)bh * C + c]);
-        pmin = min(pmin, c);
+    const int d0 = k > kUpSubK ? k - kUpSubK : 0;
+    const int subs = top ? 1 : 1 << d0;                     // items per tree
+    const long long items = (long long)BH * 2 * per * subs;
+    const long long nwarps = (long long)gridDim.x * (kUpThreads / 32);
+    for (long long it = ((long long)blockIdx.x * kUpThreads + threadIdx.x) >> 5; it < items; it += nwarps) {
+        const long long tree = it / subs;
+        const int sub = (int)(it - tree * subs);
+        const int bhf = (int)(tree / per), bh = bhf >> 1, f = bhf & 1;
+        const int blk = (F.nprev[bhf] >> k) + (int)(tree % per);
+        if (blk >= (F.nseq[bhf] >> k)) continue;             // uniform across the warp
+        const int *ord = F.ord + F.lvl(bh, f, k) * C + ((size_t)blk << k);
+        const float *kb = kbar + (size_t)bh * Cn * kD;         // caller's arrays: [B*H, Cn]
+        const int t_hi = top ? d0 - 1 : k, t_lo = top ? 0 : d0;
+        for (int t = t_hi; t >= t_lo; t--) {
+            // nodes of this item at depth t: [v_first, v_first + n)
+            const int n = top ? 1 << t : 1 << (t - d0);
+            const int v_first = top ? 1 << t : ((1 << d0) + sub) << (t - d0);
+            for (int i0 = 0; i0 < n; i0 += kUpBatch) {
+                float2 m[kUpBatch];
+                float A[kUpBatch];
+                int pmin[kUpBatch];
+#pragma unroll
+                for (int u = 0; u < kUpBatch; u++) {
+                    const int v = v_first + i0 + u;
+                    if (i0 + u >= n) continue;
+                    if (t == k) {
+                        const int c = ord[v - (1 << k)];
+                        m[u] = *reinterpret_cast<const float2 *>(kb + (size_t)c * kD + 2 * lane);
+                        A[u] = amax[(size_t)bh * Cn + c];
+                        pmin[u] = c;
+                    } else {
+                        const size_t nl = node_index(F, bh, f, k, blk, 2 * v), nr = nl + 1;   // children
+                        const float2 a = *reinterpret_cast<const float2 *>(F.mu + nl * kD + 2 * lane);
+                        const float2 b = *reinterpret_cast<const float2 *>(F.mu + nr * kD + 2 * lane);
+                        m[u] = make_float2(0.5f * (a.x + b.x), 0.5f * (a.y + b.y));
+                        const float4 ml = F.meta[nl], mr = F.meta[nr];
+                        A[u] = fmaxf(ml.y, mr.y);
+                        pmin[u] = min(__float_as_int(ml.z), __float_as_int(mr.z));
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kUpBatch; u++) {
+                    if (i0 + u >= n) continue;
+                    const size_t ni = node_index(F, bh, f, k, blk, v_first + i0 + u);
+                    *reinterpret_cast<float2 *>(F.mu + ni * kD + 2 * lane) = m[u];
+                    if (lane == 0) F.meta[ni] = make_float4(0.f, A[u], __int_as_float(pmin[u]), 0.f);
+                }
+            }
+            __syncwarp();
+        }
     }
-    const float inv = 1.f / (float)cnt;
-    const float m0 = s0 * inv, m1 = s1 * inv;
-    float r2 = 0.f;
-    for (int j = 0; j < cnt; j++) {
-        const float2 x = *reinterpret_cast<const float2 *>(kb + (size_t)leaves[j] * kD + 2 * lane);
-        const float d0 = x.x - m0, d1 = x.y - m1;
-        r2 = fmaxf(r2, warp_sum(d0 * d0 + d1 * d1));
+}
+
+__global__ void __launch_bounds__(256) tree_radius_kernel(Forest F, const float *__restrict__ kbar, int BH, int k,
+                                                          int per, int Cn) {
+    const int lane = threadIdx.x & 31;
+    const int C = F.C;
+    const long long per_bhf = (long long)per << k;          // leaf slots per (bh, f): new trees only
+    const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if ((id & ~31LL) >= (long long)BH * 2 * per_bhf) return;   // whole warps only
+    const bool live = id < (long long)BH * 2 * per_bhf;
+    const int bhf = live ? (int)(id / per_bhf) : 0, bh = bhf >> 1, f = bhf & 1;
+    const long long r = live ? id % per_bhf : 0;
+    const int blk = (F.nprev[bhf] >> k) + (int)(r >> k), j = (int)(r & ((1 << k) - 1));
+    const bool have = live && blk < (F.nseq[bhf] >> k);
+    float x[kD];
+    if (have) {
+        const int c = F.ord[F.lvl(bh, f, k) * C + ((size_t)blk << k) + j];
+        const float4 *src = reinterpret_cast<const float4 *>(kbar + ((size_t)bh * Cn + c) * kD);
+#pragma unroll
+        for (int q = 0; q < kD / 4; q++) {
+            const float4 v = __ldg(src + q);
+            x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+        }
     }
-    const size_t ni = F.lvl(bh, f, k) * 2 * C + node;
-    *reinterpret_cast<float2 *>(F.mu + ni * kD + 2 * lane) = make_float2(m0, m1);
-    if (lane == 0) F.meta[ni] = make_float4(cnt == 1 ? 0.f : sqrtf(r2), A, __int_as_float(pmin), 0.f);
+    for (int t = k - 1; t >= 0; t--) {
+        const int sz = 1 << (k - t);                         // leaves per node at depth t
+        const int v = (1 << t) + (j >> (k - t));
+        const size_t ni = have ? node_index(F, bh, f, k, blk, v) : 0;
+        float d2 = 0.f;
+        if (have) {
+            const float4 *mu = reinterpret_cast<const float4 *>(F.mu + ni * kD);
+#pragma unroll
+            for (int q = 0; q < kD / 4; q++) {
+                const float4 m = mu[q];
+                const float a = x[4 * q] - m.x, b = x[4 * q + 1] - m.y, c = x[4 * q + 2] - m.z, e = x[4 * q + 3] - m.w;
+                d2 = fmaf(a, a, fmaf(b, b, fmaf(c, c, fmaf(e, e, d2))));
+            }
+        }
+        // trees never straddle a warp (sizes are powers of two), and a tree missing from
+        // the sequence is missing for all of its lanes, so `have` is uniform per node
+        const int span = sz < 32 ? sz : 32;
+        for (int o = 1; o < span; o <<= 1) d2 = fmaxf(d2, __shfl_xor_sync(kFull, d2, o));
+        if (have && (lane & (span - 1)) == 0) {
+            const float rho = sqrtf(d2);
+            if (sz <= 32) F.meta[ni].x = rho;                // the node lies inside this warp
+            else atomicMax(reinterpret_cast<int *>(&F.meta[ni].x), __float_as_int(rho));
+        }
+    }
 }
 
 struct SearchArgs {
     int Nq, H, w, K, q0, beam;
+    int cells;              // C = floor(Nk / s) of the call (at most the forest's capacity)
     float scale, c_explore;
     float lambda[FS_MAX_HEADS], inv2sigma[FS_MAX_HEADS];
 };
@@ -471,7 +588,8 @@ __global__ void __launch_bounds__(kSearchWarps * 32) tree_search_kernel(Forest F
     if (r >= A.Nq) return;
     const size_t row = (size_t)bh * A.Nq + r;
     int32_t *out = idx + row * A.K;
-    if (F.hdr[0] != kTreeMagic || F.hdr[2] != F.C || F.hdr[3] != F.L || F.hdr[4] != (int)gridDim.y) {
+    if (F.hdr[kHdrMagic] != kTreeMagic || F.hdr[kHdrCap] != F.C || F.hdr[kHdrLevels] != F.L ||
+        F.hdr[kHdrBH] != (int)gridDim.y || F.hdr[kHdrCells] != A.cells || F.hdr[kHdrError] != 0) {
         for (int j = lane; j < A.K; j += 32) out[j] = -1;
         if (lane == 0) atomicOr(dev_flag, kFlagCheck);
         return;
@@ -482,10 +600,10 @@ __global__ void __launch_bounds__(kSearchWarps * 32) tree_search_kernel(Forest F
     S.q[2 * lane + 1] = q1;
     const float qn = sqrtf(warp_sum(q0 * q0 + q1 * q1));
     __syncwarp();
-    const int n = cand_count(i, A.w, F.C);
+    const int n = cand_count(i, A.w, A.cells);
     int nres = search_forest<PRIOR>(F, S, bh, 0, n, qn, A, h, i, 0, lane, n, dev_flag);
     const int n0 = nres;
-    if (F.hdr[1] && n > 0) {
+    if (F.hdr[kHdrTau] && n > 0) {
         const int m = F.admp[(size_t)bh * (F.C + 1) + n];
         nres = search_forest<PRIOR>(F, S, bh, 1, m, qn, A, h, i, nres, lane, n, dev_flag);
     }
@@ -524,40 +642,84 @@ __global__ void __launch_bounds__(kSearchWarps * 32) tree_search_kernel(Forest F
 
 }  // namespace
 
-size_t forest_bytes(const fs_params *p) { return forest_geom(p).total; }
+size_t forest_bytes(const fs_params *p) { return forest_geom(p->B * p->H, p->Nk / p->s).total; }
+
+// The capacity of a forest buffer of `bytes`: the largest cell count whose layout fits
+// (the layout grows strictly with the count), or -1 if not even p's cells fit.
+int forest_capacity(const fs_params *p, size_t bytes) {
+    const int BH = p->B * p->H, C = p->Nk / p->s;
+    const long long kMax = 1 << 26;
+    auto fits = [&](long long c) { return forest_geom(BH, (int)c).total <= bytes; };
+    if (!fits(C)) return -1;
+    long long lo = C, step = C > 0 ? C : 1;       // lo fits; grow until lo + step does not
+    while (lo < kMax && fits(std::min(lo + step, kMax))) {
+        lo = std::min(lo + step, kMax);
+        step *= 2;
+    }
+    long long hi = std::min(lo + step, kMax);      // lo fits, hi may not
+    while (lo < hi) {
+        const long long mid = lo + (hi - lo + 1) / 2;
+        if (fits(mid)) lo = mid;
+        else hi = mid - 1;
+    }
+    return (int)lo;
+}
 
 cudaError_t launch_tree_build(const fs_params *p, const float *kbar, const float *amax, const float *tau,
-                              void *forest, cudaStream_t st) {
-    const ForestGeom g = forest_geom(p);
+                              void *forest, size_t bytes, int prev, cudaStream_t st) {
+    const int cap = forest_capacity(p, bytes);
+    if (cap < 0) return cudaErrorInvalidValue;
+    const ForestGeom g = forest_geom(p->B * p->H, cap);
     const Forest F = forest_view(forest, g);
+    const int Cn = p->Nk / p->s;
     TauArgs T;
     for (int h = 0; h < FS_MAX_HEADS; h++) T.tau[h] = tau && h < p->H ? tau[h] : 0.f;
     {
         LaunchScope sc(kTreePrep, st);
-        tree_prep_kernel<<<g.BH, 1024, 0, st>>>(F, kbar, amax, p->H, tau != nullptr, T);
+        tree_prep_kernel<<<g.BH, 1024, 0, st>>>(F, kbar, amax, p->H, tau != nullptr, T, Cn, prev);
         if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
     }
-    const long long nent = (long long)g.BH * 2 * g.C;
+    const int fresh = Cn - prev;                 // cells since the previous build
     for (int k = 0; k < g.L; k++) {
         LaunchScope sc(kTreeMerge, st);
-        tree_merge_kernel<<<(unsigned)((nent + 255) / 256), 256, 0, st>>>(F, g.BH, k);
+        const int span = fresh + (1 << k);       // entries of the blocks completed since then
+        const long long nent = (long long)g.BH * 2 * span;
+        tree_merge_kernel<<<(unsigned)((nent + 255) / 256), 256, 0, st>>>(F, g.BH, k, span);
         if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
     }
-    const long long nwarps = (long long)g.BH * 2 * 2 * g.C;
     for (int k = 0; k < g.L; k++) {
         LaunchScope sc(kTreeNodes, st);
-        tree_nodes_kernel<<<(unsigned)((nwarps + 7) / 8), 256, 0, st>>>(F, kbar, amax, g.BH, k);
+        const int per = (fresh >> k) + 1;        // trees per (bh, f) completed since then, at most
+        const int d0 = k > kUpSubK ? k - kUpSubK : 0;
+        const long long items = (long long)g.BH * 2 * per << d0;
+        const long long blocks = std::min<long long>(kUpMaxBlocks, (items + kUpThreads / 32 - 1) / (kUpThreads / 32));
+        tree_up_kernel<<<(unsigned)blocks, kUpThreads, 0, st>>>(F, kbar, amax, g.BH, k, 0, per, Cn);
         if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
+        if (d0 > 0) {                           // the top depths of each tree, after its subtrees
+            const long long trees = (long long)g.BH * 2 * per;
+            const long long tb = std::min<long long>(kUpMaxBlocks, (trees + kUpThreads / 32 - 1) / (kUpThreads / 32));
+            tree_up_kernel<<<(unsigned)tb, kUpThreads, 0, st>>>(F, kbar, amax, g.BH, k, 1, per, Cn);
+            if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
+        }
+        if (k > 0) {
+            const long long leaves = (long long)g.BH * 2 * ((long long)per << k);
+            tree_radius_kernel<<<(unsigned)((leaves + 255) / 256), 256, 0, st>>>(F, kbar, g.BH, k, per, Cn);
+            if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
+        }
     }
-    return cudaSuccess;
+    tree_header_kernel<<<1, 1, 0, st>>>(F, g.BH, tau != nullptr, Cn, prev == 0);
+    return cudaGetLastError();
 }
 
-cudaError_t launch_tree_search(const fs_params *p, const Dev &D, const void *Q, const void *forest, int beam,
-                               float c_explore, int32_t *idx, int *dev_flag, cudaStream_t st) {
-    const ForestGeom g = forest_geom(p);
+cudaError_t launch_tree_search(const fs_params *p, const Dev &D, const void *Q, const void *forest, size_t bytes,
+                               int beam, float c_explore, int32_t *idx, int *dev_flag, cudaStream_t st) {
+    const int cap = forest_capacity(p, bytes);
+    if (cap < 0) return cudaErrorInvalidValue;
+    const ForestGeom g = forest_geom(p->B * p->H, cap);
     const Forest F = forest_view(const_cast<void *>(forest), g);
     SearchArgs A;
     A.Nq = p->Nq; A.H = p->H; A.w = p->w; A.K = p->K; A.q0 = p->Nk - p->Nq; A.beam = beam;
+    A.cells = p->Nk / p->s;
     A.scale = D.scale;
     A.c_explore = c_explore;
     for (int h = 0; h < FS_MAX_HEADS; h++) {

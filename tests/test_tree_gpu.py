@@ -157,3 +157,57 @@ def test_tree_full_size_sampled():
     inp = generate(CONFIGS["prefill64k"])
     rows = sample_rows(inp.wl, 40, seed=11)
     run_tree(inp, 32, 1.0, 0.75, rows=rows)
+
+
+@pytest.mark.parametrize("with_tau", [False, True])
+def test_forest_append_matches_full_build(with_tau):
+    """A growing archive ("FreeSolo" summary §3.4): cells appended in irregular steps --
+    one cell, steps that complete trees of several levels at once, a rewrite of the last
+    cells -- must leave the forest searching bit for bit like one built from scratch for
+    the same cells, in a buffer sized for the final archive.  An append that claims more
+    cells than were built is reported by the next search."""
+    B, H, s, Nq, c_final = 2, 3, 32, 40, 700
+    inp = generate(small("grow", B=B, H=H, Nq=Nq, Nk=c_final * s, K=6, W=4, P=9, dtype="bf16", seed=331))
+    Kd = torch.from_numpy(inp.K).cuda().to(torch.bfloat16)
+    Qd = torch.from_numpy(inp.Q).cuda().to(torch.bfloat16)
+
+    def params(cells):
+        return fs.Params(B=B, H=H, Nq=Nq, Nk=cells * s, K=6, W=4, P=9, alpha=inp.alpha, dtype="bf16")
+
+    pf = params(c_final)
+    grown = fs.alloc_forest(pf)
+    kb_f = torch.empty((B, H, c_final, 64), dtype=torch.float32, device="cuda")
+    am_f = torch.empty((B, H, c_final), dtype=torch.float32, device="cuda")
+    fs.cell_summaries(pf, Kd, kb_f, am_f)
+    tau = (torch.quantile(am_f.transpose(0, 1).reshape(H, -1), 0.6, dim=1).cpu().tolist() if with_tau else None)
+    for cells, start in [(64, 0), (65, 64), (128, 65), (300, 128), (511, 300), (512, 511), (512, 480), (700, 512)]:
+        p = params(cells)
+        Kc = Kd[:, :, :cells * s].contiguous()
+        kb = torch.empty((B, H, cells, 64), dtype=torch.float32, device="cuda")
+        am = torch.empty((B, H, cells), dtype=torch.float32, device="cuda")
+        fs.cell_summaries(p, Kc, kb, am)
+        fs.forest_append(p, start, kb, am, grown, tau)
+        fresh = torch.zeros_like(grown)
+        fs.forest_build(p, kb, am, fresh, tau)
+        ws = fs.alloc_workspace(p)
+        got = torch.full((B, H, Nq, 6), -7, dtype=torch.int32, device="cuda")
+        want = torch.full_like(got, -8)
+        fs.select_topk_tree(p, Qd, grown, got, ws, 8, 1.0)
+        fs.select_topk_tree(p, Qd, fresh, want, ws, 8, 1.0)
+        fs.sync_status(ws)
+        assert torch.equal(got, want), (cells, start)
+    # claiming more cells than the forest holds (built for 300, appended from 400):
+    # marked, and reported by the next search
+    p300 = params(300)
+    kb = torch.empty((B, H, 300, 64), dtype=torch.float32, device="cuda")
+    am = torch.empty((B, H, 300), dtype=torch.float32, device="cuda")
+    fs.cell_summaries(p300, Kd[:, :, :300 * s].contiguous(), kb, am)
+    fs.forest_build(p300, kb, am, grown, tau)
+    p = params(c_final)
+    fs.forest_append(p, 400, kb_f, am_f, grown, tau)
+    ws = fs.alloc_workspace(p)
+    got = torch.empty((B, H, Nq, 6), dtype=torch.int32, device="cuda")
+    fs.select_topk_tree(p, Qd, grown, got, ws, 8, 1.0)
+    with pytest.raises(fs.FsError) as e:
+        fs.sync_status(ws)
+    assert e.value.code == 6
