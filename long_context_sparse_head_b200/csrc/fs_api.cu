@@ -164,7 +164,7 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
             return FS_ERR_CUDA;
         if (!fk.close(st, rs)) return FS_ERR_CUDA;
         return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), at<float>(ws, L.part),
-                                          attn_splits(p), st));
+                                          attn_splits(p), amax, st));
     }
     if (has_long_range(p)) {
         const int32_t *sel = idx;
@@ -317,7 +317,7 @@ extern "C" fs_status fs_forward_rerank(const fs_params *p, const void *Q, const 
             launch_rope_keys(D, K, krot, lo, hi, st) != cudaSuccess)
             return FS_ERR_CUDA;
         return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), at<float>(ws, L.part),
-                                          attn_splits(p), st));
+                                          attn_splits(p), amax, st));
     }
     if (launch_rerank(D, p->dtype, Q, K, kbar, amax, exitn, shortlist, sel, st) != cudaSuccess) return FS_ERR_CUDA;
     if (attn_tc_supported(p)) {                    // bf16: the fused tensor-core readout + window
@@ -329,7 +329,7 @@ extern "C" fs_status fs_forward_rerank(const fs_params *p, const void *Q, const 
             launch_rope_keys(D, K, krot, lo, hi, st) != cudaSuccess)
             return FS_ERR_CUDA;
         return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), at<float>(ws, L.part),
-                                          attn_splits(p), st));
+                                          attn_splits(p), amax, st));
     }
     return run_forward(p, Q, K, V, kbar, amax, sel, O, ws, st);
 }

@@ -13,14 +13,17 @@
 // cores).  The readout's exponent reference is the row's bound from the record (an upper
 // bound of its logits within 96 of their maximum, so every P is at most 1 and none
 // underflows): no running maximum, no rescaling.  Then the window runs over 64-key chunks
-// with a running maximum and lazy rescaling.  Both softmaxes accumulate in tensor
+// with a fixed reference or a running maximum.  Both softmaxes accumulate in tensor
 // memory: three S buffers in columns [0,64), [64,128) and [128,192) (chunk c uses buffer
 // c mod 3, and its P overwrites the first 32 columns of that buffer) and one O in
 // [192,256).  The MMA warp keeps Q K^T two chunks ahead of P V, so a softmax warp that
 // finishes early finds the next S ready while slower warps finish this chunk.  When the
 // first window chunk arrives the readout is finished: the softmax threads read its O,
 // keep alpha_h * RMSNorm(u) in registers (fp32), and the window's first P V overwrites O;
-// the epilogue adds the two.  No intermediate leaves the SM.
+// the epilogue adds the two.  No intermediate leaves the SM.  The window, like the readout,
+// subtracts a fixed per-row reference where one exists (|q_i| times the largest key norm
+// of the band's cells, within 96 of the row's own logit), computed by the auxiliary warps
+// while the readout runs; otherwise it keeps a running maximum with lazy rescaling.
 //
 // Warpgroup 0 (warps 0-3): softmax, thread = query row = TMEM lane; it holds a chunk's
 // S row in registers (one TMEM wait per chunk), raised to 200 registers by setmaxnreg.
@@ -54,7 +57,9 @@ struct AttnSmem {
     __nv_bfloat16 v[NSTAGE][BN * kD];
     int ulist[UMAX];                            // union cells, ascending
     int nU;
-    uint64_t q_full, q_ready, u_ready, o_done, drain;
+    float wref[BM];                             // window reference per row (log2 units) or NaN
+    float amax_band;                            // largest a_c of the cells the band touches
+    uint64_t q_full, q_ready, u_ready, w_ready, o_done, drain;
     uint64_t o_ready[2];                        // P V of chunk c completes phase c / 2 of [c % 2]
     uint64_t s_full[NSBUF], p_full[NSBUF];      // per S buffer
     uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
@@ -184,6 +189,44 @@ __device__ __forceinline__ void softmax_chunk_fixed(uint32_t tS, uint32_t sel, f
     tc::f2_unpack(tc::f2_add(tc::f2_add(ls[0], ls[1]), tc::f2_add(ls[2], ls[3])), u, v);
     l += u + v;
 }
+
+// One window chunk against a fixed reference (log2 units, an upper bound of the row's
+// logits): a BAND chunk masks the columns outside lo <= j < lo + width with -inf, every
+// exponent is then <= 0, and nothing is rescaled.  P goes to the buffer's first BN/2
+// columns; l gathers the row sum.
+__device__ __forceinline__ void softmax_chunk_band_fixed(uint32_t tS, int kind, int lo, int width, float ref,
+                                                         float c_log2, float &l) {
+    uint32_t s[BN];
+    tc::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+    tc::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+    tc::tmem_wait_ld();
+    if (kind == BAND) {
+#pragma unroll
+        for (int j = 0; j < BN; j++)
+            if ((unsigned)(j - lo) >= (unsigned)width) s[j] = 0xff800000u;
+    }
+    const uint64_t c2 = tc::f2_pack(c_log2, c_log2), nb2 = tc::f2_pack(-ref, -ref);
+    uint64_t ls[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) ls[k] = tc::f2_pack(0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < BN / 32; q++) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; e++) {
+            const int j = 32 * q + 2 * e;
+            float x0, x1;
+            tc::f2_unpack(tc::f2_fma(tc::f2_pack(__uint_as_float(s[j]), __uint_as_float(s[j + 1])), c2, nb2), x0, x1);
+            const float p0 = tc::ex2(x0), p1 = tc::ex2(x1);
+            ls[e & 3] = tc::f2_add(ls[e & 3], tc::f2_pack(p0, p1));
+            pk[e] = tc::pack_bf16x2(p0, p1);
+        }
+        tc::tmem_st16(tS + 16 * q, pk);
+    }
+    float u, v;
+    tc::f2_unpack(tc::f2_add(tc::f2_add(ls[0], ls[1]), tc::f2_add(ls[2], ls[3])), u, v);
+    l += u + v;
+}
 }  // namespace
 
 template <bool SPLIT>
@@ -192,7 +235,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                const __grid_constant__ CUtensorMap tv32, const __grid_constant__ CUtensorMap tkr64,
                const __grid_constant__ CUtensorMap tv64, const AttnArgs A,
                const uint32_t *__restrict__ tiles, const float2 *__restrict__ rope_lo,
-               const float2 *__restrict__ rope_hi, __nv_bfloat16 *__restrict__ O, int *dev_flag) {
+               const float2 *__restrict__ rope_hi, __nv_bfloat16 *__restrict__ O, int *dev_flag,
+               const __nv_bfloat16 *__restrict__ Kraw, const float *__restrict__ amax) {
     extern __shared__ uint8_t smraw[];
     const uint32_t sbase = tc::smem_u32(smraw);
     AttnSmem &sm = *reinterpret_cast<AttnSmem *>(smraw + (((sbase + 1023u) & ~1023u) - sbase));
@@ -220,6 +264,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         tc::mbar_init(&sm.q_full, 1);
         tc::mbar_init(&sm.q_ready, NAUX);
         tc::mbar_init(&sm.u_ready, NAUX);
+        tc::mbar_init(&sm.w_ready, NAUX);
         tc::mbar_init(&sm.o_ready[0], 1);
         tc::mbar_init(&sm.o_ready[1], 1);
         tc::mbar_init(&sm.o_done, 1);
@@ -312,7 +357,52 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 }
                 tc::fence_async_shared();
                 tc::mbar_arrive(&sm.q_ready);
+                // ---- window reference per row (log2 units).  Every window logit of row i is
+                // at most |q_i| max_j |k_j| / sqrt(d) (Cauchy-Schwarz; rotations keep norms),
+                // bounded by the largest a_c of the cells the tile's band touches; the
+                // largest is at least the row's own logit q_i.k_i / sqrt(d) (key i is always
+                // in its window, and R(i) cancels).  Within kMrefMaxGap the upper bound is the
+                // reference; a band reaching past the last full cell (no a_c) gets none.
+                const int c_lo = max(0, jbase) / kS, c_hi = (pb + nrows - 1) / kS;
+                const bool band_ok = c_hi < A.C;
+                if (t < 32) {
+                    float am = 0.f;
+                    if (band_ok)
+                        for (int c = c_lo + t; c <= c_hi; c += 32) am = fmaxf(am, __ldg(amax + (size_t)bh * A.C + c));
+                    am = warp_max(am);
+                    if (t == 0) sm.amax_band = am;
+                }
+                aux_sync();
+                const float cl2 = A.scale_log2e;
+                for (int row = t; row < BM; row += NAUX) {
+                    float ref = 0.f;
+                    if (row < nrows) {
+                        ref = __uint_as_float(0x7fc00000u);
+                        if (band_ok) {
+                            const uint8_t *qrow = reinterpret_cast<const uint8_t *>(sm.qn) + row * 128;
+                            const uint4 *krow = reinterpret_cast<const uint4 *>(Kraw + ((size_t)bh * A.Nk + pb + row) * kD);
+                            float qq = 0.f, qk = 0.f;
+#pragma unroll
+                            for (int j = 0; j < 8; j++) {
+                                const uint4 qv = *reinterpret_cast<const uint4 *>(qrow + ((j ^ (row & 7)) << 4));
+                                const uint4 kv = __ldg(krow + j);
+                                const uint32_t q4[4] = {qv.x, qv.y, qv.z, qv.w}, k4[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+                                for (int e = 0; e < 4; e++) {
+                                    const float q0 = __uint_as_float(q4[e] << 16), q1 = __uint_as_float(q4[e] & 0xffff0000u);
+                                    const float k0 = __uint_as_float(k4[e] << 16), k1 = __uint_as_float(k4[e] & 0xffff0000u);
+                                    qq = fmaf(q0, q0, fmaf(q1, q1, qq));
+                                    qk = fmaf(q0, k0, fmaf(q1, k1, qk));
+                                }
+                            }
+                            const float ub = sqrtf(qq) * sm.amax_band * cl2;
+                            if (ub - qk * cl2 <= kMrefMaxGap) ref = ub;
+                        }
+                    }
+                    sm.wref[row] = ref;
+                }
             }
+            tc::mbar_arrive(&sm.w_ready);
         } else if (warp == W_MMA) {
             if (lane == 0) {
                 const uint32_t id_qk = tc::idesc_bf16(BM, BN, false, false);
@@ -438,6 +528,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         float y[kD];                            // alpha_h RMSNorm(u), once the readout is done
 #pragma unroll
         for (int e = 0; e < kD; e++) y[e] = 0.f;
+        // the window runs against each row's fixed reference (from the auxiliary warps)
+        // unless one of the warp's rows has none
+        float wref = 0.f;
+        if (ok && total > nread) {
+            if (tc::mbar_wait(&sm.w_ready, 0, ab)) wref = sm.wref[row];
+            else ok = false;
+        }
+        const bool wfixed = __all_sync(kFull, !isnan(wref));
+        if (wfixed) m_sr = wref;
         // ---- window chunks (eqs. (3)-(4)): 64 consecutive keys of the band each
         for (; ok && it < total; it++) {
             const int g = cb + it;
@@ -477,8 +576,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             const int clo = max(-jc, i - A.w - jc), chi = min(i - jc, BN - 1);
             const int width = rvalid ? max(0, chi - clo + 1) : 0;
             const int kind = __all_sync(kFull, clo <= 0 && chi >= BN - 1 && rvalid) ? FULL : BAND;
-            const float corr = softmax_chunk(trow + BN * (it % NSBUF), kind, 0u, clo, width, A.scale_log2e, m_sr, l_sr);
-            if (it > nread && __any_sync(kFull, corr != 1.f) && !rescale_o(it, corr)) { ok = false; break; }
+            if (wfixed) {
+                softmax_chunk_band_fixed(trow + BN * (it % NSBUF), kind, clo, width, wref, A.scale_log2e, l_sr);
+            } else {
+                const float corr = softmax_chunk(trow + BN * (it % NSBUF), kind, 0u, clo, width, A.scale_log2e, m_sr,
+                                                 l_sr);
+                if (it > nread && __any_sync(kFull, corr != 1.f) && !rescale_o(it, corr)) { ok = false; break; }
+            }
             release(it);
         }
         if (ok && tc::mbar_wait(&sm.o_done, 0, ab)) {
@@ -602,7 +706,7 @@ bool attn_tc_supported(const fs_params *p) {
 
 cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V, const void *Krot,
                            const uint32_t *tiles, void *O, const float2 *rope_lo, const float2 *rope_hi,
-                           int *dev_flag, float *part, int nsplit, cudaStream_t st) {
+                           int *dev_flag, float *part, int nsplit, const float *amax, cudaStream_t st) {
     if (P.Nq == 0) return cudaSuccess;
     const int BH = P.B * P.H;
     const int kr0 = rope_first_key(P);
@@ -629,7 +733,7 @@ cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const voi
         auto kern = A.nsplit > 1 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (launch_pdl(kern, grid, dim3(NTHREADS), smem, st, tq, tk32, tv32, tkr64, tv64, A, tiles, rope_lo, rope_hi,
-                       (__nv_bfloat16 *)O, dev_flag) != cudaSuccess)
+                       (__nv_bfloat16 *)O, dev_flag, (const __nv_bfloat16 *)K, amax) != cudaSuccess)
             return cudaErrorLaunchFailure;
     }
     if (A.nsplit > 1) {

@@ -251,8 +251,9 @@ bool attn_tc_supported(const fs_params *p);
 // partial states (part, attn_part_bytes) are combined by a second kernel
 int attn_splits(const fs_params *p);
 size_t attn_part_bytes(const fs_params *p);
+// amax: the cell summaries' max key norms (the window's fixed reference)
 cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V, const void *Krot,
                            const uint32_t *tiles, void *O, const float2 *rope_lo, const float2 *rope_hi,
-                           int *dev_flag, float *part, int nsplit, cudaStream_t st);
+                           int *dev_flag, float *part, int nsplit, const float *amax, cudaStream_t st);
 
 }  // namespace fs
