@@ -50,11 +50,12 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--quick", action="store_true", help="skip e2e, CPU baseline, extras")
-    ap.add_argument("--variant", choices=["forward", "rerank", "backward", "tree", "tree_decode"],
+    ap.add_argument("--variant", choices=["forward", "rerank", "backward", "tree", "tree_decode", "stream"],
                     default="forward",
                     help="time only this variant of the pass on --workload (one JSON line, no "
                          "roofline or baselines): the eq. (12) rerank, the backward pass, or "
-                         "FS-B; 'forward' is the benchmark itself")
+                         "FS-B, FS-B decoding on a growing archive, or the FS-L streaming cache; "
+                         "'forward' is the benchmark itself")
     ap.add_argument("--beam", type=int, default=32, help="FS-B beam width for --variant tree")
     return ap.parse_args()
 
@@ -787,9 +788,12 @@ def run_variant(args):
         res = time_backward(fs, torch, inp, steps=args.steps, warmup=warm)
     elif args.variant == "tree_decode":
         res = time_tree_decode(fs, torch, inp, beam=args.beam, steps=args.steps, warmup=warm)
+    elif args.variant == "stream":
+        res = time_stream(fs, torch, inp, warmup=max(warm, min(20, wl.Nq - 1)))
     else:
         res = time_tree(fs, torch, inp, beam=args.beam, steps=args.steps, warmup=warm)
-    ms, value = aggregate(res["ms_per_step"], wl.queries, world)
+    # a streaming decode step attends one query token per (batch, head) stream
+    ms, value = aggregate(res["ms_per_step"], 1 if args.variant == "stream" else wl.queries, world)
     res.update({"variant": args.variant, "workload": wl.name, "n_gpus": world, "steps": args.steps,
                 "warmup": warm, "ms_per_step": ms, "value": value})
     if rank == 0:
