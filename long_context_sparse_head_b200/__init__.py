@@ -141,16 +141,15 @@ class Params:
 
 
 def _ptr(t):
-    if t is None:
-        return None
-    return ctypes.c_void_p(t.data_ptr())
+    # a plain int converts to void * through the argtypes (cheaper than a c_void_p object)
+    return None if t is None else t.data_ptr()
 
 
 def _stream(stream):
     if stream is None:
         import torch
         stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(getattr(stream, "cuda_stream", stream))
+    return getattr(stream, "cuda_stream", stream)
 
 
 def _check(code, where):

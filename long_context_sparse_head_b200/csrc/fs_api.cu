@@ -71,7 +71,6 @@ WsLayout layout(const fs_params *p) {
     L.rope_abs = off; off += align256((size_t)(kRopeLo + rope_hi_rows(p->Nk)) * 32 * 8);
     const int kr0 = p->Nk - p->Nq - p->w > 0 ? p->Nk - p->Nq - p->w : 0;   // first rotated key
     L.krot = off;  off += align256(BH * (size_t)(p->Nk - kr0) * kD * 2);
-    L.part = off;  off += align256(attn_part_bytes(p));      // split CTAs' partial states (decoding)
     L.tlist = off; off += align256(BH * (size_t)exit_list_words(p->P) * 4);   // TopP member lists (decoding)
     const Dev D = make_dev(p);
     L.tplist = off; off += align256(BH * (size_t)((p->Nq + 127) / 128) * tile_list_words(D) * 4);   // tiles' TopP
@@ -144,9 +143,7 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
         const cudaStream_t rs = fk.open(st);
         float2 *lo = at<float2>(ws, L.rope_abs), *hi = lo + kRopeLo * 32;
         void *krot = at<void>(ws, L.krot);
-        if (launch_rope_abs_table(p->Nk, p->rope_base, lo, hi, rs) != cudaSuccess ||
-            launch_rope_keys(D, K, krot, lo, hi, rs) != cudaSuccess)
-            return FS_ERR_CUDA;
+        if (launch_rope(D, p->rope_base, K, krot, lo, hi, rs) != cudaSuccess) return FS_ERR_CUDA;
         if (!kbar) {
             float *kb = at<float>(ws, L.kbar), *am = at<float>(ws, L.amax);
             if (launch_summaries(D, p->dtype, K, kb, am, st) != cudaSuccess) return FS_ERR_CUDA;
@@ -163,7 +160,7 @@ fs_status run_forward(const fs_params *p, const void *Q, const void *K, const vo
             cudaSuccess)
             return FS_ERR_CUDA;
         if (!fk.close(st, rs)) return FS_ERR_CUDA;
-        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), at<float>(ws, L.part),
+        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag),
                                           attn_splits(p), amax, st));
     }
     if (has_long_range(p)) {
@@ -313,10 +310,8 @@ extern "C" fs_status fs_forward_rerank(const fs_params *p, const void *Q, const 
             return FS_ERR_CUDA;
         float2 *lo = at<float2>(ws, L.rope_abs), *hi = lo + kRopeLo * 32;
         void *krot = at<void>(ws, L.krot);
-        if (launch_rope_abs_table(p->Nk, p->rope_base, lo, hi, st) != cudaSuccess ||
-            launch_rope_keys(D, K, krot, lo, hi, st) != cudaSuccess)
-            return FS_ERR_CUDA;
-        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), at<float>(ws, L.part),
+        if (launch_rope(D, p->rope_base, K, krot, lo, hi, st) != cudaSuccess) return FS_ERR_CUDA;
+        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag),
                                           attn_splits(p), amax, st));
     }
     if (launch_rerank(D, p->dtype, Q, K, kbar, amax, exitn, shortlist, sel, st) != cudaSuccess) return FS_ERR_CUDA;
@@ -325,10 +320,8 @@ extern "C" fs_status fs_forward_rerank(const fs_params *p, const void *Q, const 
         if (launch_idx_tiles(D, sel, tiles, at<int>(ws, L.flag), st) != cudaSuccess) return FS_ERR_CUDA;
         float2 *lo = at<float2>(ws, L.rope_abs), *hi = lo + kRopeLo * 32;
         void *krot = at<void>(ws, L.krot);
-        if (launch_rope_abs_table(p->Nk, p->rope_base, lo, hi, st) != cudaSuccess ||
-            launch_rope_keys(D, K, krot, lo, hi, st) != cudaSuccess)
-            return FS_ERR_CUDA;
-        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag), at<float>(ws, L.part),
+        if (launch_rope(D, p->rope_base, K, krot, lo, hi, st) != cudaSuccess) return FS_ERR_CUDA;
+        return cuda_status(launch_attn_tc(D, Q, K, V, krot, tiles, O, lo, hi, at<int>(ws, L.flag),
                                           attn_splits(p), amax, st));
     }
     return run_forward(p, Q, K, V, kbar, amax, sel, O, ws, st);

@@ -31,6 +31,7 @@
 // rotate Q by its absolute positions).  The window's keys come pre-rotated (absolute
 // positions, double-precision angles) from a workspace copy.
 #include <algorithm>
+#include <cstddef>
 
 #include "tc_rope.cuh"
 
@@ -58,6 +59,7 @@ struct AttnSmem {
     int ulist[UMAX];                            // union cells, ascending
     int nU;
     float wref[BM];                             // window reference per row (log2 units) or NaN
+    float4 phead[BM];                           // split CTAs: per row (m, l) of both branches
     float amax_band;                            // largest a_c of the cells the band touches
     uint64_t q_full, q_ready, u_ready, w_ready, o_done, drain;
     uint64_t o_ready[2];                        // P V of chunk c completes phase c / 2 of [c % 2]
@@ -72,14 +74,16 @@ struct AttnArgs {
     int kr0;                // first key of the rotated copy
     float scale_log2e;      // log2(e) / sqrt(d)
     float rms_eps;
-    int nsplit;             // CTAs per tile (gridDim.z); > 1: partial states to `part`
-    float *part;
+    int nsplit;             // CTAs per tile (gridDim.z, one cluster); > 1: split and combined
     float alpha[FS_MAX_HEADS];
 };
 
-// A split CTA's partial state per row: m, l (log2 units) of the readout and the window,
-// then the readout's and the window's unnormalised O (64 floats each).
-constexpr int kPartStride = 4 + 2 * kD;
+// A split CTA's partial state per row: m, l (log2 units) of the readout and the window
+// (phead), then the readout's and the window's unnormalised O, 64 floats each, over the
+// K / V stages (free once the last P V has completed): row r's 16-byte chunk q (0-15 the
+// readout's, 16-31 the window's) at slot q ^ (r mod 8) of the row's 512 bytes, so that the
+// rows a warp writes at once fall in different banks.
+constexpr int kPartRowBytes = 2 * kD * 4;
 
 __device__ __forceinline__ void aux_sync() {
     asm volatile("bar.sync %0, %1;" ::"n"(kAuxBarrier), "n"(NAUX) : "memory");
@@ -462,6 +466,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 }
             }
         }
+        if (SPLIT) {                            // the softmax warps' two cluster barriers
+            __syncwarp();
+            tc::cluster_sync();
+            tc::cluster_sync();
+        }
     } else {
         tc::regs_inc<REGS_SOFTMAX>();
         // ---- softmax: thread = query row
@@ -482,8 +491,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         const int total = ce - cb;
         const int nread = max(0, min(ce, nR) - cb);     // this CTA's readout chunks come first
         float m_lr = fixed ? mref : -INFINITY, l_lr = 0.f, m_sr = -INFINITY, l_sr = 0.f;
-        float *part_row = SPLIT ? A.part + ((((size_t)bh * gridDim.x + blockIdx.x) * S + sidx) * BM + row) * kPartStride
-                                : nullptr;
+        float4 *part_row = SPLIT ? reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(sm.k) + row * kPartRowBytes)
+                                 : nullptr;
         // O rescale, after the exponentials (S no longer occupies registers); the P V of the
         // previous chunk, which accumulates into the same O, must have finished.  Called only
         // after chunk it's S wait: that S was issued after the P V of chunk it - 3, which
@@ -553,12 +562,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 tc::tmem_ld32(trow + O_COL, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
                 tc::tmem_ld32(trow + O_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
                 tc::tmem_wait_ld();
-                if (SPLIT) {                    // the readout's partial state, unnormalised
-                    float4 *d4 = reinterpret_cast<float4 *>(part_row + 4);
+                if (SPLIT) {                    // the readout's partial O, unnormalised, until the end
 #pragma unroll
-                    for (int q = 0; q < kD / 4; q++)
-                        d4[q] = make_float4(__uint_as_float(a[4 * q]), __uint_as_float(a[4 * q + 1]),
-                                            __uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3]));
+                    for (int e = 0; e < kD; e++) y[e] = __uint_as_float(a[e]);
                 } else {                        // O_lr <- alpha_h RMSNorm(O_lr / l)
                     const float inv_l = l_lr > 0.f ? 1.f / l_lr : 0.f;
                     float ss = 0.f;
@@ -585,7 +591,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             }
             release(it);
         }
-        if (ok && tc::mbar_wait(&sm.o_done, 0, ab)) {
+        const bool done = ok && tc::mbar_wait(&sm.o_done, 0, ab);
+        if (done) {
             tc::tc_fence_after();
             uint32_t a[kD];
             tc::tmem_ld32(trow + O_COL, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
@@ -593,20 +600,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             tc::tmem_wait_ld();
             if (SPLIT) {
                 // partial state of this CTA's chunks; a branch it had no chunk of stays empty.
-                // O holds the window's sum if the CTA had window chunks, else the readout's.
+                // O holds the window's sum if the CTA had window chunks, else the readout's
+                // (which, with window chunks, was kept in y when the window began).
                 const bool had_lr = cb < nR && ce > cb, had_sr = ce > nR && ce > cb;
-                *reinterpret_cast<float4 *>(part_row) = make_float4(had_lr ? m_lr : -INFINITY, had_lr ? l_lr : 0.f,
-                                                                    had_sr ? m_sr : -INFINITY, had_sr ? l_sr : 0.f);
-                float4 *d_lr = reinterpret_cast<float4 *>(part_row + 4);
-                float4 *d_sr = reinterpret_cast<float4 *>(part_row + 4 + kD);
+                sm.phead[row] = make_float4(had_lr ? m_lr : -INFINITY, had_lr ? l_lr : 0.f, had_sr ? m_sr : -INFINITY,
+                                            had_sr ? l_sr : 0.f);
 #pragma unroll
                 for (int q = 0; q < kD / 4; q++) {
                     const float4 v = make_float4(__uint_as_float(a[4 * q]), __uint_as_float(a[4 * q + 1]),
                                                  __uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3]));
+                    const float4 yv = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
                     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-                    d_sr[q] = had_sr ? v : z;
-                    if (!had_lr) d_lr[q] = z;
-                    else if (!had_sr) d_lr[q] = v;      // else written when the window began
+                    part_row[q ^ (row & 7)] = !had_lr ? z : had_sr ? yv : v;
+                    part_row[16 + (q ^ (row & 7))] = had_sr ? v : z;
                 }
             } else if (rvalid) {
                 const float inv = l_sr > 0.f ? 1.f / l_sr : 0.f;
@@ -624,6 +630,90 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 }
             }
         }
+        if (SPLIT && !done)                     // an aborted CTA contributes nothing (and sets the flag)
+            sm.phead[row] = make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+        if (SPLIT) {
+            // the tile's S CTAs form one cluster: once every partial state is in place, CTA r
+            // combines rows [r R, (r + 1) R) (R = ceil(128 / S)) from all S CTAs' shared memory:
+            // the readout's partials merge into u (rescaled to the largest max) and RMSNorm
+            // gives alpha_h o^lr, the window's merge into o^sr, and O = o^sr + alpha_h o^lr
+            // (eq. (2)).  A softmax warp takes 4 rows at once: lane 8k + s reads split s's
+            // (m, l) of row k; then, two rows at a time, every lane reads dimensions (2 lane,
+            // 2 lane + 1) of the rows' partial O from every split before using any.  The
+            // producer warps take part in both cluster barriers; the second keeps every CTA's
+            // shared memory alive until all reads are done.
+            __syncwarp();
+            tc::cluster_sync();
+            const int R = (BM + S - 1) / S;
+            const int rlo = sidx * R, rhi = min(min(BM, nrows), rlo + R);
+            const uint32_t hbase = tc::smem_u32(sm.phead), vbase = tc::smem_u32(sm.k);
+            const int kk = lane >> 3, sp = lane & 7;
+            for (int rw = rlo + 4 * warp; rw < rhi; rw += 4 * NSOFT) {
+                float4 st = make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+                if (sp < S && rw + kk < rhi)
+                    st = tc::ld_cluster_f4(tc::cluster_map(hbase + (uint32_t)((rw + kk) * 16), (uint32_t)sp));
+                float M_lr = st.x, M_sr = st.z;
+#pragma unroll
+                for (int o = 4; o > 0; o >>= 1) {       // maxima over the 8 lanes of a row
+                    M_lr = fmaxf(M_lr, __shfl_xor_sync(kFull, M_lr, o));
+                    M_sr = fmaxf(M_sr, __shfl_xor_sync(kFull, M_sr, o));
+                }
+                const float w_lr = st.y > 0.f ? exp2f(st.x - M_lr) : 0.f, w_sr = st.w > 0.f ? exp2f(st.z - M_sr) : 0.f;
+                float L_lr = st.y * w_lr, L_sr = st.w * w_sr;
+#pragma unroll
+                for (int o = 4; o > 0; o >>= 1) {
+                    L_lr += __shfl_xor_sync(kFull, L_lr, o);
+                    L_sr += __shfl_xor_sync(kFull, L_sr, o);
+                }
+#pragma unroll
+                for (int kb = 0; kb < 4; kb += 2) {     // two rows' loads in flight at a time
+                    float2 x[2][8], z[2][8];
+#pragma unroll
+                    for (int k = 0; k < 2; k++) {
+                        const int r = rw + kb + k;
+                        const uint32_t ro = vbase + (uint32_t)(r * kPartRowBytes) + (uint32_t)((lane & 1) * 8);
+                        const uint32_t cu = (uint32_t)(((lane >> 1) ^ (r & 7)) * 16);
+#pragma unroll
+                        for (int sx = 0; sx < 8; sx++) {
+                            x[k][sx] = make_float2(0.f, 0.f);
+                            z[k][sx] = make_float2(0.f, 0.f);
+                            if (sx < S && r < rhi) {
+                                x[k][sx] = tc::ld_cluster_f2(tc::cluster_map(ro + cu, (uint32_t)sx));
+                                z[k][sx] = tc::ld_cluster_f2(tc::cluster_map(ro + 256u + cu, (uint32_t)sx));
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int k = 0; k < 2; k++) {
+                        const int r = rw + kb + k, src = 8 * (kb + k);
+                        float u0 = 0.f, u1 = 0.f, o0 = 0.f, o1 = 0.f;
+#pragma unroll
+                        for (int sx = 0; sx < 8; sx++) {
+                            const float wl = __shfl_sync(kFull, w_lr, src + sx), ws = __shfl_sync(kFull, w_sr, src + sx);
+                            u0 = fmaf(x[k][sx].x, wl, u0);
+                            u1 = fmaf(x[k][sx].y, wl, u1);
+                            o0 = fmaf(z[k][sx].x, ws, o0);
+                            o1 = fmaf(z[k][sx].y, ws, o1);
+                        }
+                        const float Ll = __shfl_sync(kFull, L_lr, src), Ls = __shfl_sync(kFull, L_sr, src);
+                        float y0 = 0.f, y1 = 0.f;
+                        if (Ll > 0.f) {
+                            u0 /= Ll;
+                            u1 /= Ll;
+                            const float f = A.alpha[h] * rsqrtf(warp_sum(u0 * u0 + u1 * u1) * (1.f / kD) + A.rms_eps);
+                            y0 = u0 * f;
+                            y1 = u1 * f;
+                        }
+                        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+                        if (r < rhi)
+                            *reinterpret_cast<uint32_t *>(O + ((size_t)bh * A.Nq + r0 + r) * kD + 2 * lane) =
+                                tc::pack_bf16x2(o0 * inv + y0, o1 * inv + y1);
+                    }
+                }
+            }
+            __syncwarp();
+            tc::cluster_sync();
+        }
     }
 
     tc::tc_fence_before();
@@ -634,67 +724,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     }
 }
 
-namespace {
-// Combination of split CTAs' partial states (decoding shapes): per row, the readout's
-// partials merge into u (rescaled to the largest max), RMSNorm gives alpha_h o^lr; the
-// window's merge into o^sr; O = o^sr + alpha_h o^lr (eq. (2)).  One warp per row, lane m
-// holding dimensions (2m, 2m+1).
-constexpr int kCombWarps = 4;
-__global__ void __launch_bounds__(kCombWarps * 32) attn_combine_kernel(const AttnArgs A, int ntiles,
-                                                                       __nv_bfloat16 *__restrict__ O) {
-    griddep_wait();                             // the split CTAs' partial states are complete
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.y, h = bh % A.H;
-    const int r = blockIdx.x * kCombWarps + warp;
-    if (r >= A.Nq) return;
-    const int tile = r / BM, row = r % BM, S = A.nsplit;      // S <= 8
-    const float *base = A.part + (((size_t)bh * ntiles + tile) * S * BM + row) * kPartStride;
-    // lanes 0..S-1 hold the splits' (m, l) pairs; every lane then loads its two
-    // dimensions of each split's O at once
-    float4 st = make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
-    if (lane < S) st = *reinterpret_cast<const float4 *>(base + (size_t)lane * BM * kPartStride);
-    const float M_lr = warp_max(st.x), M_sr = warp_max(st.z);
-    const float w_lr = st.y > 0.f ? exp2f(st.x - M_lr) : 0.f, w_sr = st.w > 0.f ? exp2f(st.z - M_sr) : 0.f;
-    const float L_lr = warp_sum(st.y * w_lr), L_sr = warp_sum(st.w * w_sr);
-    float u0 = 0.f, u1 = 0.f, o0 = 0.f, o1 = 0.f;
-#pragma unroll
-    for (int s = 0; s < 8; s++) {
-        if (s >= S) break;
-        const float wl = __shfl_sync(kFull, w_lr, s), ws = __shfl_sync(kFull, w_sr, s);
-        const float *p = base + (size_t)s * BM * kPartStride;
-        const float2 x = *reinterpret_cast<const float2 *>(p + 4 + 2 * lane);
-        const float2 z = *reinterpret_cast<const float2 *>(p + 4 + kD + 2 * lane);
-        u0 = fmaf(x.x, wl, u0);
-        u1 = fmaf(x.y, wl, u1);
-        o0 = fmaf(z.x, ws, o0);
-        o1 = fmaf(z.y, ws, o1);
-    }
-    float y0 = 0.f, y1 = 0.f;
-    if (L_lr > 0.f) {
-        u0 /= L_lr;
-        u1 /= L_lr;
-        const float f = A.alpha[h] * rsqrtf(warp_sum(u0 * u0 + u1 * u1) * (1.f / kD) + A.rms_eps);
-        y0 = u0 * f;
-        y1 = u1 * f;
-    }
-    const float inv = L_sr > 0.f ? 1.f / L_sr : 0.f;
-    *reinterpret_cast<uint32_t *>(O + ((size_t)bh * A.Nq + r) * kD + 2 * lane) =
-        tc::pack_bf16x2(o0 * inv + y0, o1 * inv + y1);
-}
-}  // namespace
-
 // CTAs per 128-row tile: 1 when the tiles fill the GPU; otherwise the tile's chunk list is
-// split over up to 8 CTAs (about two CTAs per SM in all) and combined afterwards.
+// split over up to 8 CTAs (about two CTAs per SM in all), one thread-block cluster, which
+// combines its partial states itself.
 int attn_splits(const fs_params *p) {
     const long long tiles = (long long)p->B * p->H * ((p->Nq + BM - 1) / BM);
     if (tiles <= 0 || tiles >= 148) return 1;
     return (int)std::min<long long>(8, std::max<long long>(1, (2 * 148) / tiles));
-}
-
-size_t attn_part_bytes(const fs_params *p) {
-    const int S = attn_splits(p);
-    if (S <= 1) return 0;
-    return (size_t)p->B * p->H * ((p->Nq + BM - 1) / BM) * S * BM * kPartStride * 4;
 }
 
 bool attn_tc_supported(const fs_params *p) {
@@ -706,7 +742,7 @@ bool attn_tc_supported(const fs_params *p) {
 
 cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V, const void *Krot,
                            const uint32_t *tiles, void *O, const float2 *rope_lo, const float2 *rope_hi,
-                           int *dev_flag, float *part, int nsplit, const float *amax, cudaStream_t st) {
+                           int *dev_flag, int nsplit, const float *amax, cudaStream_t st) {
     if (P.Nq == 0) return cudaSuccess;
     const int BH = P.B * P.H;
     const int kr0 = rope_first_key(P);
@@ -723,25 +759,33 @@ cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const voi
     A.scale_log2e = P.scale * 1.4426950408889634f;
     A.rms_eps = P.rms_eps;
     for (int hh = 0; hh < FS_MAX_HEADS; hh++) A.alpha[hh] = P.alpha[hh];
-    A.nsplit = part && nsplit > 1 ? nsplit : 1;
-    A.part = part;
+    A.nsplit = std::min(std::max(nsplit, 1), 8);
     const size_t smem = sizeof(AttnSmem) + 1024;
+    static_assert(sizeof(AttnSmem::k) + sizeof(AttnSmem::v) >= (size_t)BM * kPartRowBytes &&
+                      offsetof(AttnSmem, v) == offsetof(AttnSmem, k) + sizeof(AttnSmem::k),
+                  "the split partial states fit over the K / V stages");
     const int ntiles = (P.Nq + BM - 1) / BM;
     const dim3 grid(ntiles, BH, A.nsplit);
-    {
-        LaunchScope scope(kAttnTc, st);
-        auto kern = A.nsplit > 1 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (launch_pdl(kern, grid, dim3(NTHREADS), smem, st, tq, tk32, tv32, tkr64, tv64, A, tiles, rope_lo, rope_hi,
-                       (__nv_bfloat16 *)O, dev_flag, (const __nv_bfloat16 *)K, amax) != cudaSuccess)
-            return cudaErrorLaunchFailure;
-    }
-    if (A.nsplit > 1) {
-        LaunchScope scope(kAttnCombine, st);
-        if (launch_pdl(attn_combine_kernel, dim3((P.Nq + kCombWarps - 1) / kCombWarps, BH), dim3(kCombWarps * 32), 0, st,
-                       A, ntiles, (__nv_bfloat16 *)O) != cudaSuccess)
-            return cudaErrorLaunchFailure;
-    }
+    LaunchScope scope(kAttnTc, st);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;       // a split tile's CTAs: one cluster
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = A.nsplit;
+    cfg.attrs = attr;
+    cfg.numAttrs = A.nsplit > 1 ? 2 : 1;
+    auto kern = A.nsplit > 1 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (cudaLaunchKernelEx(&cfg, kern, tq, tk32, tv32, tkr64, tv64, A, tiles, rope_lo, rope_hi, (__nv_bfloat16 *)O,
+                           dev_flag, (const __nv_bfloat16 *)K, amax) != cudaSuccess)
+        return cudaErrorLaunchFailure;
     return cudaGetLastError();
 }
 

@@ -37,7 +37,7 @@ struct Dev {
 
 // Workspace layout (byte offsets from ws; each segment 256-byte aligned).
 struct WsLayout {
-    size_t flag, exitn, kbar, amax, idx, olr, rope, tiles, rope_abs, krot, part, tlist, tplist, total;
+    size_t flag, exitn, kbar, amax, idx, olr, rope, tiles, rope_abs, krot, tlist, tplist, total;
 };
 
 // Per-tile selection record passed from the tensor-core selection kernel to the fused
@@ -138,7 +138,7 @@ enum KernelId : int {
     kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
     kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kRerank, kIdxTiles, kBwdRotate, kBwdRows,
     kBwdWindowKv, kBwdCells, kBwdReadoutKv, kBwdDalpha, kTreePrep, kTreeMerge, kTreeNodes, kTreeSearch,
-    kBwdLrRows, kRerankTc, kReadoutRows, kAttnCombine, kTileLists, kNumKernels
+    kBwdLrRows, kRerankTc, kReadoutRows, kTileLists, kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
@@ -223,6 +223,9 @@ int rope_hi_rows(int Nk);
 cudaError_t launch_rope_abs_table(int Nk, float rope_base, float2 *lo, float2 *hi, cudaStream_t st);
 cudaError_t launch_rope_keys(const Dev &P, const void *K, void *Krot, const float2 *lo, const float2 *hi,
                              cudaStream_t st);
+// the RoPE tables and the rotated keys of a call: two launches, or one when few keys rotate
+cudaError_t launch_rope(const Dev &P, float rope_base, const void *K, void *Krot, float2 *lo, float2 *hi,
+                        cudaStream_t st);
 // tensor-core selection (bf16): scores against the bf16x3 split of the mean keys
 bool select_tc_supported(const fs_params *p);
 // (tlist: the exit-times kernel's member lists, when it wrote them: the union is then built
@@ -247,13 +250,12 @@ cudaError_t launch_tree_search(const fs_params *p, const Dev &D, const void *Q, 
                                int beam, float c_explore, int32_t *idx, int *dev_flag, cudaStream_t st);
 // fused tensor-core readout + window + combine (bf16, internally selected cells)
 bool attn_tc_supported(const fs_params *p);
-// decoding shapes (fewer tiles than SMs): the tile's chunks split over nsplit CTAs whose
-// partial states (part, attn_part_bytes) are combined by a second kernel
+// decoding shapes (fewer tiles than SMs): the tile's chunks split over nsplit CTAs, one
+// thread-block cluster that combines its partial states in shared memory
 int attn_splits(const fs_params *p);
-size_t attn_part_bytes(const fs_params *p);
 // amax: the cell summaries' max key norms (the window's fixed reference)
 cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V, const void *Krot,
                            const uint32_t *tiles, void *O, const float2 *rope_lo, const float2 *rope_hi,
-                           int *dev_flag, float *part, int nsplit, const float *amax, cudaStream_t st);
+                           int *dev_flag, int nsplit, const float *amax, cudaStream_t st);
 
 }  // namespace fs

@@ -35,7 +35,7 @@ const char *const kNames[kNumKernels] = {"cell_summaries", "exit_times", "select
                                          "cache_append", "cache_attend", "rerank", "idx_tiles",
                                          "bwd_rotate", "bwd_win_rows", "bwd_window_kv", "bwd_cells",
                                          "bwd_readout_kv", "bwd_dalpha", "tree_prep", "tree_merge",
-                                         "tree_nodes", "tree_search", "bwd_lr_rows", "rerank_tc", "readout_rows", "attn_combine",
+                                         "tree_nodes", "tree_search", "bwd_lr_rows", "rerank_tc", "readout_rows",
                                          "tile_lists"};
 }  // namespace
 

@@ -316,8 +316,11 @@ rerank_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
             }
             uint32_t tau = 1u;                        // selected: key >= tau (key 0: not admitted)
             if (na > A.K) {
-                uint32_t lo = kmin, hi = kmax + 1u;   // count(key >= lo) >= K > count(key >= hi)
-                while (hi - lo > 1u) {
+                // bisection keeps count(key >= lo) >= K > count(key >= hi) and stops once the
+                // bracket pins the K-th key to within one key; one pass then gives tau
+                uint32_t lo = kmin, hi = kmax + 1u;
+                int clo = na, chi = 0;
+                while (clo > A.K + 1 && chi < A.K - 1 && hi - lo > 1u) {
                     const uint32_t mid = lo + ((hi - lo) >> 1);
                     int cp[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -325,12 +328,25 @@ rerank_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
                     const int cnt = (cp[0] + cp[1]) + (cp[2] + cp[3]);
                     if (cnt >= A.K) {
                         lo = mid;
-                        if (cnt == A.K) break;
+                        clo = cnt;
                     } else {
                         hi = mid;
+                        chi = cnt;
                     }
                 }
-                tau = lo;
+                if (clo == A.K) {
+                    tau = lo;
+                } else if (clo == A.K + 1) {          // the (K+1)-th key is the smallest >= lo
+                    uint32_t m = 0xffffffffu;
+#pragma unroll
+                    for (int u = 0; u < UM; u++) m = key[u] >= lo ? min(m, key[u]) : m;
+                    tau = m + 1u;
+                } else {                               // count(key >= hi) = K - 1
+                    uint32_t m = 0u;
+#pragma unroll
+                    for (int u = 0; u < UM; u++) m = key[u] < hi ? max(m, key[u]) : m;
+                    tau = m;
+                }
             }
             uint32_t mw[4] = {0u, 0u, 0u, 0u};        // selected union positions of this row
 #pragma unroll

@@ -57,8 +57,17 @@ struct SelArgs {
     int tp_words;           // words per (b, h, tile) of the tiles' TopP lists (with tplist)
     int prune, has_prior;
     float scale;
+};
+// The eq. (7) prior's per-head parameters travel only with the instantiation that uses
+// them: a kernel's argument block is copied at every launch, so the prior-free launch
+// stays small.
+struct SelPrior {
     float lambda[FS_MAX_HEADS];
     float inv2sigma[FS_MAX_HEADS];
+};
+template <bool PRIOR> struct SelArgsT : SelArgs {};
+template <> struct SelArgsT<true> : SelArgs {
+    SelPrior pr;
 };
 
 __device__ __forceinline__ void sel_sync() {
@@ -77,7 +86,7 @@ __device__ __forceinline__ void split3(float x, __nv_bfloat16 &hi, __nv_bfloat16
 // sub-partition, so up to 128 registers) or 128 (two CTAs per SM)
 template <bool PRIOR, int UM>
 __global__ void __launch_bounds__(NTHREADS, UM <= 80 ? 3 : 2)
-select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const float *__restrict__ kbar,
+select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgsT<PRIOR> A, const float *__restrict__ kbar,
                  const float *__restrict__ amax, const int *__restrict__ exitn,
                  int32_t *__restrict__ idx, uint32_t *__restrict__ tiles, int *dev_flag,
                  const int *__restrict__ tlist, const int *__restrict__ tplist) {
@@ -341,8 +350,11 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
         {
             tc::tc_fence_after();
             const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-            const float lam = PRIOR ? A.lambda[h] : 0.f;
-            const float i2s = PRIOR ? A.inv2sigma[h] : 0.f;
+            float lam = 0.f, i2s = 0.f;
+            if constexpr (PRIOR) {
+                lam = A.pr.lambda[h];
+                i2s = A.pr.inv2sigma[h];
+            }
             uint32_t aw[NW];                        // admitted union positions of this row
 #pragma unroll
             for (int b = 0; b < NW; b++) aw[b] = row < nrows ? sm.admit[g][b] : 0u;
@@ -389,11 +401,17 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                     key[u] = 0u;
                 }
             }
-            // K-th largest key by bisection: count(key >= lo) >= K > count(key >= hi)
+            // K-th largest key: bisection on c(x) = count(key >= x) keeps c(lo) >= K > c(hi)
+            // and stops as soon as the bracket pins the K-th key to within one key, i.e.
+            // c(lo) = K or K + 1, or c(hi) = K - 1; one more pass over the keys then gives
+            // tau with c(tau) = K exactly (keys are unique).  Stopping at any of the three gaps
+            // around the K-th key instead of only the one below it cuts the halvings of the
+            // warp's slowest row, which sets the warp's loop count.
             uint32_t tau = 1u;
             if (na > A.K) {
                 uint32_t lo = 1u << 7, hi = (0x1000000u + 1u) << 7;
-                while (hi - lo > 1u) {
+                int clo = na, chi = 0;
+                while (clo > A.K + 1 && chi < A.K - 1 && hi - lo > 1u) {
                     const uint32_t mid = lo + ((hi - lo) >> 1);
                     int cp[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent partial counts
 #pragma unroll
@@ -405,12 +423,41 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgs A, const 
                     const int cnt = ((cp[0] + cp[1]) + (cp[2] + cp[3])) + ((cp[4] + cp[5]) + (cp[6] + cp[7]));
                     if (cnt >= A.K) {
                         lo = mid;
-                        if (cnt == A.K) break;
+                        clo = cnt;
                     } else {
                         hi = mid;
+                        chi = cnt;
                     }
                 }
-                tau = lo;
+                if (clo == A.K) {
+                    tau = lo;
+                } else if (clo == A.K + 1) {            // the (K+1)-th key is the smallest >= lo
+                    uint32_t m0 = 0xffffffffu, m1 = 0xffffffffu;
+#pragma unroll
+                    for (int b = 0; b < UM / 16; b++)
+                        if (16 * b < N) {
+#pragma unroll
+                            for (int e = 0; e < 16; e += 2) {
+                                const uint32_t k0 = key[16 * b + e], k1 = key[16 * b + e + 1];
+                                m0 = k0 >= lo ? min(m0, k0) : m0;
+                                m1 = k1 >= lo ? min(m1, k1) : m1;
+                            }
+                        }
+                    tau = min(m0, m1) + 1u;
+                } else {                                 // c(hi) = K - 1: the K-th key is the largest < hi
+                    uint32_t m0 = 0u, m1 = 0u;
+#pragma unroll
+                    for (int b = 0; b < UM / 16; b++)
+                        if (16 * b < N) {
+#pragma unroll
+                            for (int e = 0; e < 16; e += 2) {
+                                const uint32_t k0 = key[16 * b + e], k1 = key[16 * b + e + 1];
+                                m0 = k0 < hi ? max(m0, k0) : m0;
+                                m1 = k1 < hi ? max(m1, k1) : m1;
+                            }
+                        }
+                    tau = max(m0, m1);
+                }
             }
             uint32_t mw[UMAX / 32] = {0u, 0u, 0u, 0u};   // selected union positions
 #pragma unroll
@@ -496,16 +543,24 @@ bool select_tc_supported(const fs_params *p) {
 namespace {
 // the largest union a tile of this call can have (W + P + 10 with pruning, else C)
 int union_bound(const Dev &P) { return P.prune ? P.W + P.P + 10 : P.C; }
-template <int UM> cudaError_t launch_um(const CUtensorMap &tq, const SelArgs &A, bool prior, dim3 grid,
-                                         const float *kbar, const float *amax, const int *exitn, int32_t *idx,
-                                         uint32_t *tiles, int *dev_flag, const int *tlist, const int *tplist,
-                                         cudaStream_t st) {
+// the erf prior is a separate instantiation: without it the unrolled score loop stays small
+template <bool PRIOR, int UM>
+cudaError_t launch_um(const CUtensorMap &tq, const SelArgsT<PRIOR> &A, dim3 grid, const float *kbar,
+                      const float *amax, const int *exitn, int32_t *idx, uint32_t *tiles, int *dev_flag,
+                      const int *tlist, const int *tplist, cudaStream_t st) {
     const size_t smem = sizeof(SelSmem<UM>) + 1024;
-    // the erf prior is a separate instantiation: without it the unrolled score loop stays small
-    auto kern = prior ? select_tc_kernel<true, UM> : select_tc_kernel<false, UM>;
+    auto kern = select_tc_kernel<PRIOR, UM>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     return launch_pdl(kern, grid, dim3(NTHREADS), smem, st, tq, A, kbar, amax, exitn, idx, tiles, dev_flag, tlist,
                       tplist);
+}
+template <bool PRIOR>
+cudaError_t launch_sel(const Dev &P, const CUtensorMap &tq, const SelArgsT<PRIOR> &A, dim3 grid, const float *kbar,
+                       const float *amax, const int *exitn, int32_t *idx, uint32_t *tiles, int *dev_flag,
+                       const int *tlist, const int *tplist, cudaStream_t st) {
+    if (union_bound(P) <= 80)
+        return launch_um<PRIOR, 80>(tq, A, grid, kbar, amax, exitn, idx, tiles, dev_flag, tlist, tplist, st);
+    return launch_um<PRIOR, UMAX>(tq, A, grid, kbar, amax, exitn, idx, tiles, dev_flag, tlist, tplist, st);
 }
 }  // namespace
 
@@ -516,7 +571,7 @@ cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, con
     const int BH = P.B * P.H;
     CUtensorMap tq;
     if (!encode_tmap_3d_bf16(&tq, Q, kD, P.Nq, BH, kD, BM)) return cudaErrorInvalidValue;
-    SelArgs A;
+    SelArgsT<true> A;
     A.Nq = P.Nq; A.Nk = P.Nk; A.q0 = P.q0; A.w = P.w; A.C = P.C; A.K = P.K;
     A.W = P.W; A.P = P.P; A.H = P.H; A.prune = P.prune; A.has_prior = P.has_prior;
     A.scale = P.scale;
@@ -524,15 +579,18 @@ cudaError_t launch_select_tc(const Dev &P, const void *Q, const float *kbar, con
     A.tp_words = tile_list_words(P);
     if (!P.prune) tlist = nullptr;
     if (tlist || A.tp_words == 0) tplist = nullptr;
-    for (int h = 0; h < FS_MAX_HEADS; h++) {
-        A.lambda[h] = P.lambda[h];
-        A.inv2sigma[h] = P.inv2sigma[h];
-    }
     const dim3 grid((P.Nq + BM - 1) / BM, BH);
     LaunchScope scope(kSelectTc, st);
-    if (union_bound(P) <= 80)
-        return launch_um<80>(tq, A, P.has_prior, grid, kbar, amax, exitn, idx, tiles, dev_flag, tlist, tplist, st);
-    return launch_um<UMAX>(tq, A, P.has_prior, grid, kbar, amax, exitn, idx, tiles, dev_flag, tlist, tplist, st);
+    if (!P.has_prior) {
+        SelArgsT<false> A0;
+        static_cast<SelArgs &>(A0) = A;         // the common part only
+        return launch_sel<false>(P, tq, A0, grid, kbar, amax, exitn, idx, tiles, dev_flag, tlist, tplist, st);
+    }
+    for (int h = 0; h < FS_MAX_HEADS; h++) {
+        A.pr.lambda[h] = P.lambda[h];
+        A.pr.inv2sigma[h] = P.inv2sigma[h];
+    }
+    return launch_sel<true>(P, tq, A, grid, kbar, amax, exitn, idx, tiles, dev_flag, tlist, tplist, st);
 }
 
 }  // namespace fs
