@@ -193,8 +193,16 @@ fs_status fs_select_topk_noalloc(const fs_params *p, const void *Q, const float 
  * dK, dV [B,H,Nk,d] and dalpha [H] (or NULL) are device float32 outputs, overwritten.
  * idx entries outside [0, Nk/s) (the -1 padding) are skipped; a row with no cell has y = 0.
  * bws/bws_bytes: device scratch of fs_backward_workspace_size bytes (rotated keys and
- * queries, per-row softmax terms, the readout's du, the cell-to-rows lists).  Enqueued on
- * `stream`; FS_ERR_INVALID_ARG / FS_ERR_UNSUPPORTED as for fs_forward.  CUDA cores. */
+ * queries, per-row softmax terms, the readout's du, the cell-to-rows lists, tile records).
+ * Its first bytes hold a device error flag that must be zero before the first call (as a
+ * forward workspace's); fs_sync_status(bws, stream) reads and clears it.  Enqueued on
+ * `stream`; FS_ERR_INVALID_ARG / FS_ERR_UNSUPPORTED as for fs_forward.
+ * The window's part runs on CUDA cores.  With bf16 and at most 128 distinct cells per
+ * 128-row tile (W + P + 10 <= 128 with pruning, floor(Nk/s) <= 128 without; true of any
+ * selection from A_i), the readout's part runs on the tensor cores (dK, dV added with
+ * float32 atomics, so their last bits depend on the order); a tile whose rows select more
+ * than 128 cells then sets the flag (FS_ERR_KERNEL_CHECK from fs_sync_status) and its
+ * extra cells are left out.  Otherwise, and for float32, it runs on CUDA cores. */
 fs_status fs_backward_workspace_size(const fs_params *p, size_t *bytes);
 fs_status fs_backward(const fs_params *p, const void *Q, const void *K, const void *V, const int32_t *idx,
                       const void *dO, float *dQ, float *dK, float *dV, float *dalpha, void *bws,

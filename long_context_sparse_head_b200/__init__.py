@@ -276,8 +276,9 @@ def backward_workspace_size(params):
 
 
 def alloc_backward_workspace(params, device="cuda"):
+    """A zero-filled backward workspace (its device error flag must start at zero)."""
     import torch
-    return torch.empty(backward_workspace_size(params), dtype=torch.uint8, device=device)
+    return torch.zeros(backward_workspace_size(params), dtype=torch.uint8, device=device)
 
 
 def backward(params, Q, K, V, idx, dO, dQ, dK, dV, dalpha, bws, stream=None):

@@ -22,6 +22,7 @@
 //                that selected the cell
 //   dalpha       per-head sum of the rows' dO.y
 #include <cmath>
+#include <type_traits>
 
 #include "tc_rope.cuh"
 
@@ -36,7 +37,7 @@ struct BwdArgs {
 
 // Byte layout of the backward scratch (256-byte aligned segments).
 struct BwdLayout {
-    size_t rope, krot, qrot, rowst, du, dal, cnt, off, fill, list, total;
+    size_t flag, rope, krot, qrot, rowst, du, dal, cnt, off, fill, list, tiles, total;
 };
 
 size_t a256b(size_t x) { return (x + 255) & ~size_t(255); }
@@ -50,6 +51,7 @@ BwdLayout bwd_layout(const fs_params *p) {
         off += a256b(bytes);
         return o;
     };
+    L.flag = seg(256);                                                   // device error flag
     L.rope = seg((size_t)(kRopeLo + rope_hi_rows(p->Nk)) * 32 * 8);   // lo, hi angle tables
     L.krot = seg(BH * p->Nk * kD * 4);                                   // rotated keys, float
     L.qrot = seg(R * kD * 4);                                            // rotated queries
@@ -60,6 +62,7 @@ BwdLayout bwd_layout(const fs_params *p) {
     L.off = seg((BH * C + 1) * 4);
     L.fill = seg((BH * C + 1) * 4);
     L.list = seg(R * (size_t)(p->K > 0 ? p->K : 1) * 4);                 // rows of each cell
+    L.tiles = seg(BH * (size_t)((p->Nq + 127) / 128) * kTileRecWords * 4);   // tile records (bf16)
     L.total = off;
     return L;
 }
@@ -619,7 +622,10 @@ fs_status run_backward(const fs_params *p, const T *Q, const T *K, const T *V, c
         bwd_win_rows_kernel<T><<<dim3(nwin, BH), kWinWarps * 32, 0, st>>>(A, Q, V, dO, krot, lo, hi, dQ, qrot, rowst);
         if (!ok()) return FS_ERR_CUDA;
     }
-    if (p->Nq > 0) {
+    // bf16 with tiles of at most 128 distinct cells: the readout's part runs on the tensor
+    // cores after the window's dK, dV are written (it adds to them)
+    const bool tc_readout = std::is_same<T, __nv_bfloat16>::value && bwd_readout_tc_supported(p);
+    if (p->Nq > 0 && !tc_readout) {
         LaunchScope sc(kBwdLrRows, st);
         bwd_lr_rows_kernel<T><<<dim3((p->Nq + kLrWarps - 1) / kLrWarps, BH), kLrWarps * 32, 0, st>>>(
             A, Q, K, V, idx, dO, dQ, rowst, du, dal);
@@ -632,7 +638,13 @@ fs_status run_backward(const fs_params *p, const T *Q, const T *K, const T *V, c
         if (!ok()) return FS_ERR_CUDA;
     }
     const long long nsel = (long long)BH * p->Nq * p->K;
-    if (nsel > 0 && A.C > 0) {
+    if (tc_readout && p->Nq > 0) {
+        uint32_t *tiles = reinterpret_cast<uint32_t *>(ws + L.tiles);
+        int *flag = reinterpret_cast<int *>(ws + L.flag);
+        if (launch_idx_tiles(make_dev_params(p), idx, tiles, flag, st) != cudaSuccess ||
+            launch_bwd_readout_tc(p, Q, K, V, tiles, dO, dQ, dK, dV, dal, flag, st) != cudaSuccess)
+            return FS_ERR_CUDA;
+    } else if (nsel > 0 && A.C > 0) {
         const int ncell = BH * A.C;
         {
             LaunchScope sc(kBwdCells, st);

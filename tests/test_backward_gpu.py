@@ -27,6 +27,7 @@ def gpu_backward(inp, idx, dO, with_dalpha=True):
     dal = torch.full((wl.H,), float("nan"), device="cuda") if with_dalpha else None
     bws = fs.alloc_backward_workspace(p)
     fs.backward(p, Q, K, V, I, G, dQ, dK, dV, dal, bws)
+    fs.sync_status(bws)                            # no bounded wait ran out, no check failed
     torch.cuda.synchronize()
     out = [t.cpu().numpy().astype(np.float64) for t in (dQ, dK, dV)]
     return out + [dal.cpu().numpy().astype(np.float64) if with_dalpha else None]
