@@ -609,6 +609,31 @@ fs_status run_backward(const fs_params *p, const T *Q, const T *K, const T *V, c
     int *cnt = reinterpret_cast<int *>(ws + L.cnt), *off = reinterpret_cast<int *>(ws + L.off);
     int *fill = reinterpret_cast<int *>(ws + L.fill), *list = reinterpret_cast<int *>(ws + L.list);
     auto ok = [] { return cudaGetLastError() == cudaSuccess; };
+    if (std::is_same<T, __nv_bfloat16>::value && bwd_tc_supported(p)) {
+        // bf16 with tiles of at most 128 distinct cells: both branches on the tensor cores.
+        // The RoPE tables and the rotated keys (bf16, into the rotated-key segment); dK, dV
+        // start at zero and take both branches' additions; the window stores dQ, the
+        // readout adds to it and writes each row's dO.y.
+        const Dev D = make_dev_params(p);
+        void *krot16 = ws + L.krot;
+        uint32_t *tiles = reinterpret_cast<uint32_t *>(ws + L.tiles);
+        int *flag = reinterpret_cast<int *>(ws + L.flag);
+        if (p->Nk > 0 && (launch_rope(D, p->rope_base, K, krot16, lo, hi, st) != cudaSuccess ||
+                          cudaMemsetAsync(dK, 0, (size_t)BH * p->Nk * kD * 4, st) != cudaSuccess ||
+                          cudaMemsetAsync(dV, 0, (size_t)BH * p->Nk * kD * 4, st) != cudaSuccess))
+            return FS_ERR_CUDA;
+        if (p->Nq > 0 &&
+            (launch_bwd_tc(p, true, Q, K, V, krot16, nullptr, dO, dQ, dK, dV, dal, lo, hi, flag, st) != cudaSuccess ||
+             launch_idx_tiles(D, idx, tiles, flag, st) != cudaSuccess ||
+             launch_bwd_tc(p, false, Q, K, V, nullptr, tiles, dO, dQ, dK, dV, dal, lo, hi, flag, st) != cudaSuccess))
+            return FS_ERR_CUDA;
+        if (dalpha) {
+            LaunchScope sc(kBwdDalpha, st);
+            bwd_dalpha_kernel<<<p->H, 256, 0, st>>>(dal, p->B, p->H, p->Nq, dalpha);
+            if (!ok()) return FS_ERR_CUDA;
+        }
+        return FS_OK;
+    }
     if (launch_rope_abs_table(p->Nk, p->rope_base, lo, hi, st) != cudaSuccess) return FS_ERR_CUDA;
     if (p->Nk > 0) {
         const long long n_pairs = (long long)BH * p->Nk * (kD / 2);
@@ -622,10 +647,7 @@ fs_status run_backward(const fs_params *p, const T *Q, const T *K, const T *V, c
         bwd_win_rows_kernel<T><<<dim3(nwin, BH), kWinWarps * 32, 0, st>>>(A, Q, V, dO, krot, lo, hi, dQ, qrot, rowst);
         if (!ok()) return FS_ERR_CUDA;
     }
-    // bf16 with tiles of at most 128 distinct cells: the readout's part runs on the tensor
-    // cores after the window's dK, dV are written (it adds to them)
-    const bool tc_readout = std::is_same<T, __nv_bfloat16>::value && bwd_readout_tc_supported(p);
-    if (p->Nq > 0 && !tc_readout) {
+    if (p->Nq > 0) {
         LaunchScope sc(kBwdLrRows, st);
         bwd_lr_rows_kernel<T><<<dim3((p->Nq + kLrWarps - 1) / kLrWarps, BH), kLrWarps * 32, 0, st>>>(
             A, Q, K, V, idx, dO, dQ, rowst, du, dal);
@@ -638,13 +660,7 @@ fs_status run_backward(const fs_params *p, const T *Q, const T *K, const T *V, c
         if (!ok()) return FS_ERR_CUDA;
     }
     const long long nsel = (long long)BH * p->Nq * p->K;
-    if (tc_readout && p->Nq > 0) {
-        uint32_t *tiles = reinterpret_cast<uint32_t *>(ws + L.tiles);
-        int *flag = reinterpret_cast<int *>(ws + L.flag);
-        if (launch_idx_tiles(make_dev_params(p), idx, tiles, flag, st) != cudaSuccess ||
-            launch_bwd_readout_tc(p, Q, K, V, tiles, dO, dQ, dK, dV, dal, flag, st) != cudaSuccess)
-            return FS_ERR_CUDA;
-    } else if (nsel > 0 && A.C > 0) {
+    if (nsel > 0 && A.C > 0) {
         const int ncell = BH * A.C;
         {
             LaunchScope sc(kBwdCells, st);

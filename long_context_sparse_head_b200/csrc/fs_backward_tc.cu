@@ -21,12 +21,19 @@
 // The Q, du, P and dS tiles serve both as K-major operands ([rows][d or keys]) and, read
 // the other way, as MN-major ones (the transposed products), in 128-byte-swizzled rows.
 //
+// The window's part (§3.2 eqs. (3)-(4)) is the same kernel over the band's keys instead of
+// the cells (WIN): 128 consecutive keys per chunk from the rotated copy R(j) k_j, Q rotated
+// in place by R(i), a row's valid keys [i - w, i], g = dO itself in place of du and
+// D = dO.o^sr; dK and dQ are rotated back (R^T) before they are stored.  It runs first and
+// stores dQ; the readout adds to it.
+//
 // Warps: 0-7 rows (warp w: rows 32 (w mod 4) .. + 31, keys 64 (w / 4) .. + 63 of every
-// chunk; raised to 192 registers), 8-11 the dK / dV drain (lane = key of cell w - 8 of the
-// chunk), 12 TMA, 13 MMA, 14 loads U (all lowered to 64 registers), 15 idle.
+// chunk; raised to 192 registers), 8-11 the dK / dV drain (lane = key of key block w - 8 of
+// the chunk), 12 TMA, 13 MMA, 14 loads U (readout) or with 15 rotates Q (window; all
+// lowered to 64 registers).
 #include <cmath>
 
-#include "tc_common.cuh"
+#include "tc_rope.cuh"
 
 namespace fs {
 
@@ -51,7 +58,7 @@ struct BtcSmem {
     int ulist[UMAX];
     float xch[6][2][BM];                                 // exchanges between a row's two warps
     int nU;
-    uint64_t q_full, u_ready, du_ready, u_done, dq_done;
+    uint64_t q_full, q_rot, u_ready, du_ready, u_done, dq_done;
     uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
     uint64_t s_full[2], s_free[2];                       // passes A1 / A2: two S buffers
     uint64_t sd_full, sd_free, pds_full, pds_free, dkv_full, dkv_free;   // pass B
@@ -61,7 +68,7 @@ struct BtcSmem {
 };
 
 struct BtcArgs {
-    int Nq, Nk, C, H;
+    int Nq, Nk, C, H, q0, w, kr0;
     float scale, c2;        // 1 / sqrt(d), log2(e) / sqrt(d)
     float rms_eps;
     float alpha[FS_MAX_HEADS];
@@ -87,11 +94,16 @@ __device__ __forceinline__ void red_add_v4(float *dst, float a, float b, float c
 }
 }  // namespace
 
+// WIN = false: the readout over the tile's cells (tk, tv: 32-row boxes of K, V; tg unused);
+// WIN = true: the window over the band (tk: 128-row boxes of the rotated keys from kr0 on,
+// tv: of V, tg: the dO tile)
+template <bool WIN>
 __global__ void __launch_bounds__(NTHREADS, 1)
-bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk32,
-                      const __grid_constant__ CUtensorMap tv32, const BtcArgs A, const uint32_t *__restrict__ tiles,
-                      const __nv_bfloat16 *__restrict__ dO, float *__restrict__ dQ, float *__restrict__ dK,
-                      float *__restrict__ dV, float *__restrict__ dal, int *dev_flag) {
+bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tg,
+              const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, const BtcArgs A,
+              const uint32_t *__restrict__ tiles, const __nv_bfloat16 *__restrict__ dO, float *__restrict__ dQ,
+              float *__restrict__ dK, float *__restrict__ dV, float *__restrict__ dal,
+              const float2 *__restrict__ rope_lo, const float2 *__restrict__ rope_hi, int *dev_flag) {
     extern __shared__ uint8_t smraw[];
     const uint32_t sbase = tc::smem_u32(smraw);
     BtcSmem &sm = *reinterpret_cast<BtcSmem *>(smraw + (((sbase + 1023u) & ~1023u) - sbase));
@@ -99,12 +111,16 @@ bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
     const int bh = blockIdx.y, h = bh % A.H;
     const int r0 = blockIdx.x * BM;
     const int nrows = min(BM, A.Nq - r0);
-    const uint32_t *rec = tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords;
+    const uint32_t *rec = WIN ? nullptr : tiles + ((size_t)bh * gridDim.x + blockIdx.x) * kTileRecWords;
+    const int pb = A.q0 + r0, jbase = pb - A.w, last = pb + nrows - 1;   // window: the tile's band
     const tc::Abort ab{dev_flag, &sm.abort};
+    // chunks of the tile: four union cells each (readout), 128 band keys each (window)
+    auto chunks = [&]() { return WIN ? (last - jbase) / BN + 1 : (sm.nU + CPC - 1) / CPC; };
 
     if (threadIdx.x == 0) {
         sm.abort = 0;
         tc::mbar_init(&sm.q_full, 1);
+        tc::mbar_init(&sm.q_rot, 2);
         tc::mbar_init(&sm.u_ready, 1);
         tc::mbar_init(&sm.du_ready, NROWW);
         tc::mbar_init(&sm.u_done, 1);
@@ -137,32 +153,61 @@ bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
 
     if (warp >= NROWW) {
         tc::regs_dec<REGS_OTHER>();
-        if (warp == W_AUX) {
-            for (int u = lane; u < UMAX; u += 32) sm.ulist[u] = (int)__ldg(rec + kTileUlistOff + u);
-            if (lane == 0) sm.nU = min((int)__ldg(rec + kTileCountOff), UMAX);
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&sm.u_ready);
+        if (warp >= W_AUX) {
+            if (!WIN) {
+                if (warp == W_AUX) {
+                    for (int u = lane; u < UMAX; u += 32) sm.ulist[u] = (int)__ldg(rec + kTileUlistOff + u);
+                    if (lane == 0) sm.nU = min((int)__ldg(rec + kTileCountOff), UMAX);
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&sm.u_ready);
+                }
+            } else {
+                if (warp == W_AUX && lane == 0) tc::mbar_arrive(&sm.u_ready);
+                // rotate Q in place by its absolute positions (16-byte chunks, 128-byte swizzle)
+                if (tc::mbar_wait(&sm.q_full, 0, ab)) {
+                    const int t = threadIdx.x - W_AUX * 32;
+                    uint8_t *qb = reinterpret_cast<uint8_t *>(sm.q);
+#pragma unroll 2
+                    for (int j = 0; j < BM * 8 / 64; j++) {
+                        const int item = t + 64 * j, row = item >> 3, c = item & 7;
+                        uint4 *ptr = reinterpret_cast<uint4 *>(qb + row * 128 + ((c ^ (row & 7)) << 4));
+                        float cs[4], sn[4];
+                        rope_angles(pb + row, c, rope_lo, rope_hi, cs, sn);
+                        *ptr = rope_rotate8(*ptr, cs, sn);
+                    }
+                    tc::fence_async_shared();
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&sm.q_rot);
+            }
         } else if (warp == W_TMA) {
             if (lane == 0) {
                 tc::prefetch_tmap(&tq);
-                tc::prefetch_tmap(&tk32);
-                tc::prefetch_tmap(&tv32);
-                tc::mbar_expect_tx(&sm.q_full, TILE_BYTES);
+                tc::prefetch_tmap(&tk);
+                tc::prefetch_tmap(&tv);
+                tc::mbar_expect_tx(&sm.q_full, (WIN ? 2 : 1) * TILE_BYTES);
                 tc::tma_load_3d(sm.q, &tq, &sm.q_full, 0, r0, bh);
+                if (WIN) tc::tma_load_3d(sm.du, &tg, &sm.q_full, 0, r0, bh);   // g = dO
                 int g = 0, total = 0;
                 if (tc::mbar_wait(&sm.u_ready, 0, ab)) {
-                    const int nU = sm.nU, nC = (nU + CPC - 1) / CPC;
+                    const int nU = WIN ? 0 : sm.nU, nC = chunks();
                     total = 3 * nC;                       // passes A1 (K only), A2, B
                     for (; g < total; g++) {
                         const int s = g % NSTAGE, c = g % nC;
                         const bool withv = g >= nC;
                         if (!tc::mbar_wait(&sm.kv_empty[s], ((g / NSTAGE) & 1) ^ 1, ab)) break;
-                        tc::mbar_expect_tx(&sm.kv_full[s], (withv ? 2 : 1) * CPC * CELL_BYTES);
-                        for (int j = 0; j < CPC; j++) {
-                            const int u = CPC * c + j;
-                            const int y = u < nU ? sm.ulist[u] * kS : A.Nk;   // past the end: zeros
-                            tc::tma_load_3d(sm.k[s] + j * kS * kD, &tk32, &sm.kv_full[s], 0, y, bh);
-                            if (withv) tc::tma_load_3d(sm.v[s] + j * kS * kD, &tv32, &sm.kv_full[s], 0, y, bh);
+                        tc::mbar_expect_tx(&sm.kv_full[s], (withv ? 2 : 1) * BN * kD * 2);
+                        if (WIN) {                        // 128 band keys; before key 0: zeros
+                            const int jc = jbase + BN * c;
+                            tc::tma_load_3d(sm.k[s], &tk, &sm.kv_full[s], 0, jc - A.kr0, bh);
+                            if (withv) tc::tma_load_3d(sm.v[s], &tv, &sm.kv_full[s], 0, jc, bh);
+                        } else {
+                            for (int j = 0; j < CPC; j++) {
+                                const int u = CPC * c + j;
+                                const int y = u < nU ? sm.ulist[u] * kS : A.Nk;   // past the end: zeros
+                                tc::tma_load_3d(sm.k[s] + j * kS * kD, &tk, &sm.kv_full[s], 0, y, bh);
+                                if (withv) tc::tma_load_3d(sm.v[s] + j * kS * kD, &tv, &sm.kv_full[s], 0, y, bh);
+                            }
                         }
                     }
                 }
@@ -184,8 +229,9 @@ bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
                 const uint32_t ak0 = tc::smem_u32(sm.k[0]), av0 = tc::smem_u32(sm.v[0]);
                 const uint32_t ap = tc::smem_u32(sm.p[0]), ads = tc::smem_u32(sm.ds[0]);
                 constexpr uint32_t kStage = BN * kD * 2, kHalf = BM * kD * 2;
-                bool ok = tc::mbar_wait(&sm.u_ready, 0, ab) && tc::mbar_wait(&sm.q_full, 0, ab);
-                const int nC = ok ? (sm.nU + CPC - 1) / CPC : 0;
+                bool ok = tc::mbar_wait(&sm.u_ready, 0, ab) && tc::mbar_wait(&sm.q_full, 0, ab) &&
+                          (!WIN || tc::mbar_wait(&sm.q_rot, 0, ab));
+                const int nC = ok ? chunks() : 0;
                 int g = 0;                                // K / V load sequence
                 int issued = 0;
                 // [rows x keys] (+)= X [rows x 64] Y^T, X = Q or du (K-major), Y = the stage's K or V
@@ -270,25 +316,51 @@ bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
             // dK, dV of the chunk's cell (warp - W_EPI): lane = token of the cell
             const int e = warp - W_EPI;
             bool ok = tc::mbar_wait(&sm.u_ready, 0, ab);
-            const int nU = ok ? sm.nU : 0, nC = (nU + CPC - 1) / CPC;
+            const int nU = ok && !WIN ? sm.nU : 0, nC = ok ? chunks() : 0;
             const uint32_t trow = tmem + ((uint32_t)(e * 32) << 16);
             for (int c = 0; ok && c < nC; c++) {
                 if (!tc::mbar_wait(&sm.dkv_full, c & 1, ab)) { ok = false; break; }
                 tc::tc_fence_after();
-                const int u = CPC * c + e;
-                if (u < nU) {
-                    const size_t key = (size_t)bh * A.Nk + (size_t)sm.ulist[u] * kS + lane;
+                int j = 0;                                   // this lane's key
+                bool has = false;
+                if (WIN) {
+                    j = jbase + BN * c + 32 * e + lane;
+                    has = j >= max(0, jbase) && j <= last;
+                } else {
+                    const int u = CPC * c + e;
+                    has = u < nU;
+                    if (has) j = sm.ulist[u] * kS + lane;
+                }
+                if (__any_sync(kFull, has)) {
+                    const int jj = has ? j : 0;              // lanes without a key read position 0
+                    const size_t key = (size_t)bh * A.Nk + (size_t)jj;
                     float *dv = dV + key * kD, *dk = dK + key * kD;
 #pragma unroll 1
                     for (int b = 0; b < 2 * kD / 16; b++) {      // dV columns, then dK's, 16 at a time
                         uint32_t x[16];
                         tc::tmem_ld16(trow + DV_COL + 16 * b, x);   // DK_COL = DV_COL + 64
                         tc::tmem_wait_ld();
-                        float *dst = (b < kD / 16 ? dv : dk - kD) + 16 * b;
+                        float y[16];
 #pragma unroll
-                        for (int q = 0; q < 4; q++)
-                            red_add_v4(dst + 4 * q, __uint_as_float(x[4 * q]), __uint_as_float(x[4 * q + 1]),
-                                       __uint_as_float(x[4 * q + 2]), __uint_as_float(x[4 * q + 3]));
+                        for (int q = 0; q < 16; q++) y[q] = __uint_as_float(x[q]);
+                        if (WIN && b >= kD / 16) {           // dK_j = R(j)^T dK'_j, pairs 8 (b - 4) ..
+#pragma unroll
+                            for (int hc = 0; hc < 2; hc++) {
+                                float cs[4], sn[4];
+                                rope_angles(jj, 2 * (b - kD / 16) + hc, rope_lo, rope_hi, cs, sn);
+#pragma unroll
+                                for (int t = 0; t < 4; t++) {
+                                    const float a0 = y[8 * hc + 2 * t], a1 = y[8 * hc + 2 * t + 1];
+                                    y[8 * hc + 2 * t] = a0 * cs[t] + a1 * sn[t];
+                                    y[8 * hc + 2 * t + 1] = -a0 * sn[t] + a1 * cs[t];
+                                }
+                            }
+                        }
+                        float *dst = (b < kD / 16 ? dv : dk - kD) + 16 * b;
+                        if (has)
+#pragma unroll
+                            for (int q = 0; q < 4; q++)
+                                red_add_v4(dst + 4 * q, y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
                     }
                 }
                 tc::tc_fence_before();
@@ -301,19 +373,30 @@ bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
         const int quarter = warp & 3, half = warp >> 2;
         const int row = quarter * 32 + lane;
         const bool rvalid = row < nrows;
+        const int i = pb + row;
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
-        const uint4 m4 = __ldg(reinterpret_cast<const uint4 *>(rec + kTileMaskOff + 4 * row));
+        const uint4 m4 = WIN ? make_uint4(0u, 0u, 0u, 0u)
+                             : __ldg(reinterpret_cast<const uint4 *>(rec + kTileMaskOff + 4 * row));
         bool ok = tc::mbar_wait(&sm.u_ready, 0, ab);
-        const int nU = ok ? sm.nU : 0, nC = (nU + CPC - 1) / CPC;
-        // bits of this row's selected cells among the chunk's cells 2 half, 2 half + 1
-        auto sel2 = [&](int c) -> uint32_t {
+        const int nC = ok ? chunks() : 0;
+        // valid columns of this row among its half's 64 keys of chunk c: the selected cells
+        // 4c + 2 half, + 1 (readout), or the keys of [i - w, i] at or after key 0 (window)
+        auto colmask = [&](int c) -> uint64_t {
+            if (!rvalid) return 0ull;
+            if (WIN) {
+                const int base = jbase + BN * c + 64 * half;
+                const int lo = max(max(i - A.w - base, -base), 0), hi = min(i - base, 63);
+                if (lo > hi) return 0ull;
+                return (hi == 63 ? ~0ull : (2ull << hi) - 1ull) & ~((1ull << lo) - 1ull);
+            }
             const int p0 = CPC * c + 2 * half;
             const int ws = p0 >> 5;
             const uint32_t mw = ws == 0 ? m4.x : ws == 1 ? m4.y : ws == 2 ? m4.z : m4.w;
-            return rvalid ? (mw >> (p0 & 31)) & 3u : 0u;
+            const uint32_t sel = (mw >> (p0 & 31)) & 3u;
+            return ((sel & 1u) ? 0xffffffffull : 0ull) | ((sel & 2u) ? 0xffffffff00000000ull : 0ull);
         };
         const float c2 = A.c2;
-        // ---- A1: the row's largest selected logit (log2 units)
+        // ---- A1: the row's largest valid logit (log2 units)
         float m = -INFINITY;
         for (int c = 0; ok && c < nC; c++) {
             const int b = c & 1;
@@ -326,22 +409,22 @@ bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.s_free[b]);
-            const uint32_t sel = sel2(c);
+            const uint64_t vm = colmask(c);
             float mx = -INFINITY;
 #pragma unroll
             for (int j = 0; j < 64; j++)
-                if ((sel >> (j >> 5)) & 1u) mx = fmaxf(mx, __uint_as_float(x[j]));
+                if ((vm >> j) & 1ull) mx = fmaxf(mx, __uint_as_float(x[j]));
             m = fmaxf(m, mx * c2);
         }
         m = pair_sum(sm, 0, half, row, quarter, m, true);
         const float mb = m == -INFINITY ? 0.f : m;
-        // ---- A2: P = exp2(S c - m) (selected cells) into tensor memory for U += P V
+        // ---- A2: P = exp2(S c - m) (valid columns) into tensor memory for U += P V
         float l = 0.f;
         for (int c = 0; ok && c < nC; c++) {
             const int sc = nC + c, b = sc & 1;
             if (!tc::mbar_wait(&sm.s_full[b], (sc >> 1) & 1, ab)) { ok = false; break; }
             tc::tc_fence_after();
-            const uint32_t sel = sel2(c);
+            const uint64_t vm = colmask(c);
             const uint32_t tS = trow + S_COL + 128 * b + 64 * half;
             uint32_t x[64];
             tc::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
@@ -350,9 +433,8 @@ bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
             uint32_t pk[32];
 #pragma unroll
             for (int j = 0; j < 64; j += 2) {
-                const bool on = (sel >> (j >> 5)) & 1u;
-                const float p0 = on ? tc::ex2(fmaf(__uint_as_float(x[j]), c2, -mb)) : 0.f;
-                const float p1 = on ? tc::ex2(fmaf(__uint_as_float(x[j + 1]), c2, -mb)) : 0.f;
+                const float p0 = ((vm >> j) & 1ull) ? tc::ex2(fmaf(__uint_as_float(x[j]), c2, -mb)) : 0.f;
+                const float p1 = ((vm >> (j + 1)) & 1ull) ? tc::ex2(fmaf(__uint_as_float(x[j + 1]), c2, -mb)) : 0.f;
                 l += p0 + p1;
                 pk[j >> 1] = tc::pack_bf16x2(p0, p1);
             }
@@ -363,8 +445,9 @@ bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
             if (lane == 0) tc::mbar_arrive(&sm.s_free[b]);
         }
         l = pair_sum(sm, 1, half, row, quarter, l, false);
-        // ---- row statistics: u, RMSNorm, du (dimensions 32 half .. + 31 here), D, dO.y
-        float dsum = 0.f, gy = 0.f;
+        // ---- row statistics (dimensions 32 half .. + 31 here): the branch's normalised output
+        // o (u for the readout, o^sr for the window), then for the readout RMSNorm, du and
+        // dO.y; D = du.u (readout) or dO.o^sr (window)
         float uu[32];
 #pragma unroll
         for (int e = 0; e < 32; e++) uu[e] = 0.f;
@@ -379,11 +462,6 @@ bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
         } else {
             ok = false;
         }
-        float ss = 0.f;
-#pragma unroll
-        for (int e = 0; e < 32; e++) ss = fmaf(uu[e], uu[e], ss);
-        ss = pair_sum(sm, 2, half, row, quarter, ss, false);
-        const float rin = rsqrtf(ss * (1.f / kD) + A.rms_eps);
         float g[32];
         {
             const uint4 *src = reinterpret_cast<const uint4 *>(dO + ((size_t)bh * A.Nq + r0 + (rvalid ? row : 0)) * kD + 32 * half);
@@ -399,26 +477,40 @@ bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
             }
         }
         const bool has = l > 0.f;
+        float D = 0.f;
+        if (WIN) {
+            float dsum = 0.f;
 #pragma unroll
-        for (int e = 0; e < 32; e++) gy = fmaf(g[e], uu[e] * rin, gy);
-        gy = pair_sum(sm, 3, half, row, quarter, has ? gy : 0.f, false);
-        const float a = A.alpha[h], dyy = a * gy;
-        float dus[32];
+            for (int e = 0; e < 32; e++) dsum = fmaf(g[e], uu[e], dsum);
+            D = pair_sum(sm, 4, half, row, quarter, dsum, false);
+        } else {
+            float ss = 0.f;
 #pragma unroll
-        for (int e = 0; e < 32; e++) {
-            dus[e] = has ? rin * (a * g[e] - uu[e] * rin * dyy * (1.f / kD)) : 0.f;
-            dsum = fmaf(dus[e], uu[e], dsum);
+            for (int e = 0; e < 32; e++) ss = fmaf(uu[e], uu[e], ss);
+            ss = pair_sum(sm, 2, half, row, quarter, ss, false);
+            const float rin = rsqrtf(ss * (1.f / kD) + A.rms_eps);
+            float gy = 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; e++) gy = fmaf(g[e], uu[e] * rin, gy);
+            gy = pair_sum(sm, 3, half, row, quarter, has ? gy : 0.f, false);
+            const float a = A.alpha[h], dyy = a * gy;
+            float dus[32], dsum = 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; e++) {
+                dus[e] = has ? rin * (a * g[e] - uu[e] * rin * dyy * (1.f / kD)) : 0.f;
+                dsum = fmaf(dus[e], uu[e], dsum);
+            }
+            D = pair_sum(sm, 4, half, row, quarter, dsum, false);
+#pragma unroll
+            for (int q = 0; q < 4; q++) {      // 16-byte chunks 4 half .. 4 half + 3 of the row
+                uint32_t w4[4];
+#pragma unroll
+                for (int t = 0; t < 4; t++) w4[t] = tc::pack_bf16x2(dus[8 * q + 2 * t], dus[8 * q + 2 * t + 1]);
+                *sw_chunk(sm.du, row, 4 * half + q) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            if (half == 0 && rvalid) dal[(size_t)bh * A.Nq + r0 + row] = gy;
+            tc::fence_async_shared();
         }
-        const float D = pair_sum(sm, 4, half, row, quarter, dsum, false);
-#pragma unroll
-        for (int q = 0; q < 4; q++) {          // 16-byte chunks 4 half .. 4 half + 3 of the row
-            uint32_t w4[4];
-#pragma unroll
-            for (int t = 0; t < 4; t++) w4[t] = tc::pack_bf16x2(dus[8 * q + 2 * t], dus[8 * q + 2 * t + 1]);
-            *sw_chunk(sm.du, row, 4 * half + q) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-        }
-        if (half == 0 && rvalid) dal[(size_t)bh * A.Nq + r0 + row] = gy;
-        tc::fence_async_shared();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&sm.du_ready);
         const float lse2 = has ? mb + log2f(l) : INFINITY;        // P = exp2(S c - lse2); none: 0
@@ -426,19 +518,19 @@ bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
         for (int c = 0; ok && c < nC; c++) {
             if (!tc::mbar_wait(&sm.sd_full, c & 1, ab)) { ok = false; break; }
             tc::tc_fence_after();
-            const uint32_t sel = sel2(c);
+            const uint64_t vm = colmask(c);
             uint32_t pk[32], dk[32];
 #pragma unroll
-            for (int hb = 0; hb < 2; hb++) {            // 32 keys (one cell) at a time
+            for (int hb = 0; hb < 2; hb++) {            // 32 keys at a time
                 uint32_t x[32], y[32];
                 tc::tmem_ld32(trow + S_COL + 64 * half + 32 * hb, x);
                 tc::tmem_ld32(trow + DP_COL + 64 * half + 32 * hb, y);
                 tc::tmem_wait_ld();
-                const bool on = (sel >> hb) & 1u;
+                const uint32_t vw = (uint32_t)(vm >> (32 * hb));
 #pragma unroll
                 for (int j = 0; j < 32; j += 2) {
-                    const float p0 = on ? tc::ex2(fmaf(__uint_as_float(x[j]), c2, -lse2)) : 0.f;
-                    const float p1 = on ? tc::ex2(fmaf(__uint_as_float(x[j + 1]), c2, -lse2)) : 0.f;
+                    const float p0 = ((vw >> j) & 1u) ? tc::ex2(fmaf(__uint_as_float(x[j]), c2, -lse2)) : 0.f;
+                    const float p1 = ((vw >> (j + 1)) & 1u) ? tc::ex2(fmaf(__uint_as_float(x[j + 1]), c2, -lse2)) : 0.f;
                     const float d0 = p0 * (__uint_as_float(y[j]) - D) * A.scale;
                     const float d1 = p1 * (__uint_as_float(y[j + 1]) - D) * A.scale;
                     pk[16 * hb + (j >> 1)] = tc::pack_bf16x2(p0, p1);
@@ -458,24 +550,48 @@ bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.pds_full);
         }
-        // ---- dQ of the readout, added to the window's
+        // ---- dQ: the window's, rotated back by R(i)^T, is stored; the readout's is added
         if (ok && nC > 0 && tc::mbar_wait(&sm.dq_done, 0, ab)) {
             tc::tc_fence_after();
             uint32_t qr[32];
             tc::tmem_ld32(trow + U_COL + 32 * half, qr);
             tc::tmem_wait_ld();
             if (rvalid) {
-                float *dst = dQ + ((size_t)bh * A.Nq + r0 + row) * kD + 32 * half;
+                float dq[32];
 #pragma unroll
-                for (int q = 0; q < 8; q++) {
-                    float4 v = *reinterpret_cast<float4 *>(dst + 4 * q);
-                    v.x += __uint_as_float(qr[4 * q]);
-                    v.y += __uint_as_float(qr[4 * q + 1]);
-                    v.z += __uint_as_float(qr[4 * q + 2]);
-                    v.w += __uint_as_float(qr[4 * q + 3]);
-                    *reinterpret_cast<float4 *>(dst + 4 * q) = v;
+                for (int e = 0; e < 32; e++) dq[e] = __uint_as_float(qr[e]);
+                float *dst = dQ + ((size_t)bh * A.Nq + r0 + row) * kD + 32 * half;
+                if (WIN) {
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; c4++) {   // pairs 16 half + 4 c4 .. + 3
+                        float cs[4], sn[4];
+                        rope_angles(i, 4 * half + c4, rope_lo, rope_hi, cs, sn);
+#pragma unroll
+                        for (int t = 0; t < 4; t++) {
+                            const float a0 = dq[8 * c4 + 2 * t], a1 = dq[8 * c4 + 2 * t + 1];
+                            dq[8 * c4 + 2 * t] = a0 * cs[t] + a1 * sn[t];
+                            dq[8 * c4 + 2 * t + 1] = -a0 * sn[t] + a1 * cs[t];
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < 8; q++)
+                        *reinterpret_cast<float4 *>(dst + 4 * q) = make_float4(dq[4 * q], dq[4 * q + 1], dq[4 * q + 2], dq[4 * q + 3]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; q++) {
+                        float4 v = *reinterpret_cast<float4 *>(dst + 4 * q);
+                        v.x += dq[4 * q];
+                        v.y += dq[4 * q + 1];
+                        v.z += dq[4 * q + 2];
+                        v.w += dq[4 * q + 3];
+                        *reinterpret_cast<float4 *>(dst + 4 * q) = v;
+                    }
                 }
             }
+        } else if (WIN && rvalid) {               // no chunk ran (an aborted CTA): dQ defined anyway
+            float *dst = dQ + ((size_t)bh * A.Nq + r0 + row) * kD + 32 * half;
+#pragma unroll
+            for (int q = 0; q < 8; q++) *reinterpret_cast<float4 *>(dst + 4 * q) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
 
@@ -487,34 +603,44 @@ bwd_readout_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
     }
 }
 
-bool bwd_readout_tc_supported(const fs_params *p) {
+bool bwd_tc_supported(const fs_params *p) {
     if (p->dtype != FS_BF16) return false;
     const int C = p->Nk / p->s;
     const int bound = p->W >= 0 ? p->W + p->P + 10 : C;   // largest union of a tile's cells
     return bound <= UMAX && p->Nk < (1 << 30);
 }
 
-cudaError_t launch_bwd_readout_tc(const fs_params *p, const void *Q, const void *K, const void *V,
-                                  const uint32_t *tiles, const void *dO, float *dQ, float *dK, float *dV, float *dal,
-                                  int *dev_flag, cudaStream_t st) {
+cudaError_t launch_bwd_tc(const fs_params *p, bool win, const void *Q, const void *K, const void *V,
+                          const void *Krot, const uint32_t *tiles, const void *dO, float *dQ, float *dK, float *dV,
+                          float *dal, const float2 *rope_lo, const float2 *rope_hi, int *dev_flag, cudaStream_t st) {
     if (p->Nq == 0) return cudaSuccess;
     const int BH = p->B * p->H;
-    CUtensorMap tq, tk32, tv32;
-    if (!encode_tmap_3d_bf16(&tq, Q, kD, p->Nq, BH, kD, BM) || !encode_tmap_3d_bf16(&tk32, K, kD, p->Nk, BH, kD, kS) ||
-        !encode_tmap_3d_bf16(&tv32, V, kD, p->Nk, BH, kD, kS))
-        return cudaErrorInvalidValue;
+    const int q0 = p->Nk - p->Nq, kr0 = q0 - p->w > 0 ? q0 - p->w : 0;
+    CUtensorMap tq, tg, tk, tv;
+    bool enc = encode_tmap_3d_bf16(&tq, Q, kD, p->Nq, BH, kD, BM);
+    if (win)
+        enc = enc && encode_tmap_3d_bf16(&tg, dO, kD, p->Nq, BH, kD, BM) &&
+              encode_tmap_3d_bf16(&tk, Krot, kD, p->Nk - kr0, BH, kD, BN) &&
+              encode_tmap_3d_bf16(&tv, V, kD, p->Nk, BH, kD, BN);
+    else
+        enc = enc && encode_tmap_3d_bf16(&tk, K, kD, p->Nk, BH, kD, kS) &&
+              encode_tmap_3d_bf16(&tv, V, kD, p->Nk, BH, kD, kS);
+    if (!enc) return cudaErrorInvalidValue;
+    if (!win) tg = tq;                                     // unused
     BtcArgs A;
     A.Nq = p->Nq; A.Nk = p->Nk; A.C = p->Nk / p->s; A.H = p->H;
+    A.q0 = q0; A.w = p->w; A.kr0 = kr0;
     A.scale = (float)(1.0 / std::sqrt((double)p->d));
     A.c2 = A.scale * 1.4426950408889634f;
     A.rms_eps = p->rms_eps;
     for (int hh = 0; hh < FS_MAX_HEADS; hh++) A.alpha[hh] = hh < p->H ? p->alpha[hh] : 0.f;
     const size_t smem = sizeof(BtcSmem) + 1024;
     const dim3 grid((p->Nq + BM - 1) / BM, BH);
-    LaunchScope scope(kBwdReadoutTc, st);
-    cudaFuncSetAttribute(bwd_readout_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    bwd_readout_tc_kernel<<<grid, NTHREADS, smem, st>>>(tq, tk32, tv32, A, tiles, (const __nv_bfloat16 *)dO, dQ, dK,
-                                                        dV, dal, dev_flag);
+    LaunchScope scope(win ? kBwdWindowTc : kBwdReadoutTc, st);
+    auto kern = win ? bwd_tc_kernel<true> : bwd_tc_kernel<false>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    kern<<<grid, NTHREADS, smem, st>>>(tq, tg, tk, tv, A, tiles, (const __nv_bfloat16 *)dO, dQ, dK, dV, dal, rope_lo,
+                                       rope_hi, dev_flag);
     return cudaGetLastError();
 }
 

@@ -138,7 +138,7 @@ enum KernelId : int {
     kSummaries = 0, kExitTimes, kSelect, kReadout, kWindow, kRopeTable, kWindowTc, kAttnTc,
     kSelectTc, kRopeKeys, kCacheAppend, kCacheAttend, kRerank, kIdxTiles, kBwdRotate, kBwdRows,
     kBwdWindowKv, kBwdCells, kBwdReadoutKv, kBwdDalpha, kTreePrep, kTreeMerge, kTreeNodes, kTreeSearch,
-    kBwdLrRows, kRerankTc, kReadoutRows, kTileLists, kBwdReadoutTc, kNumKernels
+    kBwdLrRows, kRerankTc, kReadoutRows, kTileLists, kBwdReadoutTc, kBwdWindowTc, kNumKernels
 };
 
 // Brackets one kernel launch: counts it and, when timing is on, records events around it.
@@ -252,11 +252,13 @@ cudaError_t launch_tree_search(const fs_params *p, const Dev &D, const void *Q, 
 bool attn_tc_supported(const fs_params *p);
 // decoding shapes (fewer tiles than SMs): the tile's chunks split over nsplit CTAs, one
 // thread-block cluster that combines its partial states in shared memory
-// backward of the readout on the tensor cores (bf16; unions of at most 128 cells per tile)
-bool bwd_readout_tc_supported(const fs_params *p);
-cudaError_t launch_bwd_readout_tc(const fs_params *p, const void *Q, const void *K, const void *V,
-                                  const uint32_t *tiles, const void *dO, float *dQ, float *dK, float *dV, float *dal,
-                                  int *dev_flag, cudaStream_t st);
+// backward on the tensor cores (bf16; unions of at most 128 cells per tile): the window's
+// part (win: stores dQ; Krot = the rotated keys from rope_first_key on, bf16) or the
+// readout's (tiles from idx; adds to dQ; writes dO.y per row to dal); both add to dK, dV
+bool bwd_tc_supported(const fs_params *p);
+cudaError_t launch_bwd_tc(const fs_params *p, bool win, const void *Q, const void *K, const void *V,
+                          const void *Krot, const uint32_t *tiles, const void *dO, float *dQ, float *dK, float *dV,
+                          float *dal, const float2 *rope_lo, const float2 *rope_hi, int *dev_flag, cudaStream_t st);
 int attn_splits(const fs_params *p);
 // amax: the cell summaries' max key norms (the window's fixed reference)
 cudaError_t launch_attn_tc(const Dev &P, const void *Q, const void *K, const void *V, const void *Krot,

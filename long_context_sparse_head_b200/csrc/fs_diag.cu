@@ -36,7 +36,7 @@ const char *const kNames[kNumKernels] = {"cell_summaries", "exit_times", "select
                                          "bwd_rotate", "bwd_win_rows", "bwd_window_kv", "bwd_cells",
                                          "bwd_readout_kv", "bwd_dalpha", "tree_prep", "tree_merge",
                                          "tree_nodes", "tree_search", "bwd_lr_rows", "rerank_tc", "readout_rows",
-                                         "tile_lists", "bwd_readout_tc"};
+                                         "tile_lists", "bwd_readout_tc", "bwd_window_tc"};
 }  // namespace
 
 LaunchScope::LaunchScope(int id_, cudaStream_t st_) : id(id_), st(st_), slot(-1) {
