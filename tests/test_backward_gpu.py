@@ -121,3 +121,30 @@ def test_backward_full_size_sampled():
     for name, g, r in (("dQ", gq, sq), ("dK", gk, sk), ("dV", gv, sv)):
         scale = max(1.0, float(np.abs(r).max()))
         assert np.abs(g - r).max() <= TOL[wl.dtype] * scale, (name, float(np.abs(g - r).max()), scale)
+
+
+def test_backward_union_overflow_sets_flag():
+    """bf16 with pruning takes the tensor-core path, which holds at most 128 distinct cells
+    per 128-row tile (true of any selection from A_i).  Cells drawn at random from the whole
+    prefix exceed that: the call still completes, and the workspace flag reports the
+    failed check (FS_ERR_KERNEL_CHECK) through fs_sync_status."""
+    inp = generate(small("bwd_over", Nq=256, Nk=8192, K=6, W=4, P=9, dtype="bf16", seed=504))
+    wl = inp.wl
+    C = wl.Nk // wl.s
+    rng = np.random.default_rng(505)
+    idx = np.stack([np.sort(rng.choice(C, wl.K, replace=False)) for _ in range(wl.B * wl.H * wl.Nq)])
+    idx = idx.reshape(wl.B, wl.H, wl.Nq, wl.K).astype(np.int32)
+    p = params_for(inp)
+    dt = tdtype(wl)
+    dO = upstream_grad(wl, 6)
+    Q, K, V, G = (torch.from_numpy(np.ascontiguousarray(x)).cuda().to(dt) for x in (inp.Q, inp.K, inp.V, dO))
+    I = torch.from_numpy(idx).cuda()
+    dQ = torch.empty((wl.B, wl.H, wl.Nq, wl.d), device="cuda")
+    dK = torch.empty((wl.B, wl.H, wl.Nk, wl.d), device="cuda")
+    dV = torch.empty_like(dK)
+    bws = fs.alloc_backward_workspace(p)
+    fs.backward(p, Q, K, V, I, G, dQ, dK, dV, None, bws)
+    with pytest.raises(fs.FsError) as err:
+        fs.sync_status(bws)
+    assert err.value.code == 6
+    fs.sync_status(bws)                            # the flag was cleared by the first read

@@ -73,6 +73,8 @@ def test_tiny2k_all_cells_no_pruning_fp32():
     dict(Nq=3072, Nk=3072, W=-1, P=-1, K=8),          # base FS, unions of up to 96 cells
     dict(Nq=2048, Nk=3072, W=30, P=50, K=12),         # wide budgets: unions above 80 cells
     dict(Nq=40, Nk=1000, w=64, K=4, W=2, P=3),        # few chunks per tile: some split CTAs idle
+    dict(H=5, Nq=1280, Nk=1280),                      # 50 tiles: clusters of 5 split CTAs
+    dict(H=3, Nq=3200, Nk=3200),                      # 75 tiles: clusters of 3
 ])
 def test_small_cases(dtype, case):
     kw = dict(B=1, H=2, Nq=1536, Nk=1536, K=6, W=4, P=9, dtype=dtype, seed=101)
