@@ -39,7 +39,7 @@ namespace fs {
 
 namespace {
 constexpr int BM = 128, BN = 128, CPC = BN / kS;        // rows per tile, keys (4 cells) per chunk
-constexpr int UMAX = 128, NSTAGE = 2;
+constexpr int UMAX = 128, NSTAGE = 3;
 constexpr int NROWW = 8, W_EPI = 8, W_TMA = 12, W_MMA = 13, W_AUX = 14, NWARPS = 16;
 constexpr int NTHREADS = NWARPS * 32;
 constexpr int REGS_ROW = 192, REGS_OTHER = 64;           // 256 * 192 + 256 * 64 = 512 * 128
