@@ -315,11 +315,18 @@ fs_status fs_forward_tree(const fs_params *p, const void *Q, const void *K, cons
  *   recorded on its own stream.  fs_kernel_times waits for the recorded events, writes per
  *   kernel id (0 <= id < max_ids) the launches and summed device milliseconds since the
  *   previous read, clears them, and returns the number of kernel ids.
- * fs_kernel_name: the name of a kernel id, or NULL past the last one. */
+ * fs_kernel_name: the name of a kernel id, or NULL past the last one.
+ * fs_selftest_timeout: enqueues one small kernel that waits on a shared-memory barrier
+ *   nothing arrives at, with the bounded wait every tensor-core kernel of this library
+ *   uses (about 2 s); the wait runs out and the kernel records the timeout in the device
+ *   error flag at the start of ws (a workspace of any of the calls above) and returns.
+ *   fs_sync_status(ws, stream) then returns FS_ERR_TIMEOUT and clears the flag; the
+ *   context stays usable.  It checks the failure-reporting path without a fault. */
 long long fs_launch_count(void);
 fs_status fs_timing_enable(int on);
 int fs_kernel_times(int max_ids, long long *launches, double *ms);
 const char *fs_kernel_name(int id);
+fs_status fs_selftest_timeout(void *ws, void *stream);
 
 #ifdef __cplusplus
 }

@@ -28,7 +28,7 @@ EXPORTS = ("fs_workspace_size", "fs_cell_summaries", "fs_select_topk", "fs_forwa
            "fs_select_topk_noalloc", "fs_cache_bytes", "fs_cache_reset", "fs_cache_append",
            "fs_cache_attend", "fs_cache_status", "fs_select_topk_rerank", "fs_forward_rerank",
            "fs_backward_workspace_size", "fs_backward", "fs_forest_bytes", "fs_forest_build",
-           "fs_select_topk_tree", "fs_forward_tree", "fs_forest_append")
+           "fs_select_topk_tree", "fs_forward_tree", "fs_forest_append", "fs_selftest_timeout")
 
 
 class FsError(RuntimeError):
@@ -97,6 +97,7 @@ def load():
         L.fs_select_topk_tree.argtypes = [P, vp, vp, sz, ctypes.c_int, ctypes.c_float, vp, vp, sz, vp]
         L.fs_forward_tree.argtypes = [P, vp, vp, vp, fp, ctypes.c_int, ctypes.c_float, vp, vp, vp, sz, vp,
                                       sz, vp]
+        L.fs_selftest_timeout.argtypes = [vp, vp]
         for name in EXPORTS:
             if name not in ("fs_status_string", "fs_launch_count", "fs_kernel_name"):
                 getattr(L, name).restype = ctypes.c_int
@@ -287,6 +288,12 @@ def backward(params, Q, K, V, idx, dO, dQ, dK, dV, dalpha, bws, stream=None):
     _check(load().fs_backward(params.ref(), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(dO),
                               _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dalpha), _ptr(bws),
                               bws.numel() * bws.element_size(), _stream(stream)), "fs_backward")
+
+
+def selftest_timeout(ws, stream=None):
+    """Enqueue a kernel whose bounded wait runs out (about 2 s): the next sync_status(ws)
+    raises FsError with FS_ERR_TIMEOUT."""
+    _check(load().fs_selftest_timeout(_ptr(ws), _stream(stream)), "fs_selftest_timeout")
 
 
 def sync_status(ws, stream=None):

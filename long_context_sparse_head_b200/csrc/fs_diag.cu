@@ -3,7 +3,7 @@
 #include <mutex>
 #include <vector>
 
-#include "fs_common.cuh"
+#include "tc_common.cuh"
 
 namespace fs {
 namespace {
@@ -59,6 +59,30 @@ LaunchScope::~LaunchScope() {
 }  // namespace fs
 
 using namespace fs;
+
+namespace fs {
+namespace {
+// waits (bounded) on a barrier nothing arrives at: the wait runs out and records the timeout
+__global__ void selftest_wait_kernel(int *dev_flag) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_word;
+    if (threadIdx.x == 0) {
+        abort_word = 0;
+        tc::mbar_init(&bar, 1);
+        tc::fence_barrier_init();
+    }
+    __syncthreads();
+    const tc::Abort ab{dev_flag, &abort_word};
+    if (threadIdx.x == 0) (void)tc::mbar_wait(&bar, 0, ab);
+}
+}  // namespace
+}  // namespace fs
+
+extern "C" fs_status fs_selftest_timeout(void *ws, void *stream) {
+    if (!ws) return FS_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(static_cast<int *>(ws));
+    return cudaGetLastError() == cudaSuccess ? FS_OK : FS_ERR_CUDA;
+}
 
 extern "C" long long fs_launch_count(void) { return g_launches.load(); }
 
