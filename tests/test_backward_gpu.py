@@ -70,23 +70,25 @@ def test_backward_small(dtype, case):
     run_case(generate(small("bwd", lam=lam, sigma=sigma, **kw)))
 
 
-def test_backward_no_cells_and_no_dalpha():
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_no_cells_and_no_dalpha(dtype):
     """Rows with no candidate cell (prefix shorter than w + s) have y = 0: only the window
-    carries gradient; dalpha = NULL is accepted."""
-    inp = generate(small("bwd_short", Nq=500, Nk=500, K=4, W=2, P=3, dtype="f32", seed=502))
+    carries gradient; dalpha = NULL is accepted (bf16: tiles with an empty union)."""
+    inp = generate(small("bwd_short", Nq=500, Nk=500, K=4, W=2, P=3, dtype=dtype, seed=502))
     prob = oracle_for(inp)
     _, idx = prob.forward(want_idx=True)
     assert (idx < 0).all()
     dO = upstream_grad(inp.wl, 5)
     ref = prob.backward(idx, dO)
     got = gpu_backward(inp, idx, dO, with_dalpha=False)
-    compare(got[:3], ref[:3], "f32")
+    compare(got[:3], ref[:3], dtype)
     assert np.abs(ref[3]).max() == 0.0
 
 
-def test_backward_empty_queries():
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_empty_queries(dtype):
     """Nq = 0: nothing to differentiate; dK = dV = 0 for every key."""
-    inp = generate(small("bwd_empty", Nq=0, Nk=256, dtype="f32", seed=503))
+    inp = generate(small("bwd_empty", Nq=0, Nk=256, dtype=dtype, seed=503))
     got = gpu_backward(inp, np.zeros((1, 2, 0, inp.wl.K), np.int32), np.zeros((1, 2, 0, 64), np.float32))
     assert np.abs(got[1]).max() == 0.0 and np.abs(got[2]).max() == 0.0 and np.abs(got[3]).max() == 0.0
 
