@@ -482,11 +482,13 @@ extern "C" fs_status fs_forward_host(const fs_params *p, const void *hQ, const v
     uint8_t *dQ = at<uint8_t>(dscratch, h.q), *dK = at<uint8_t>(dscratch, h.k);
     uint8_t *dV = at<uint8_t>(dscratch, h.v), *dO = at<uint8_t>(dscratch, h.o);
     void *ws = at<void>(dscratch, h.ws);
-    // Heads are independent, so the call runs as a pipeline over about 8 chunks (heads of
+    // Heads are independent, so the call runs as a pipeline over about 16 chunks (heads of
     // one batch entry, or whole batch entries): chunk c's inputs copy in (stream `in`) while
     // chunk c-1 computes (the caller's stream) and chunk c-2's output copies out (stream
-    // `out`).  Each direction is one plain async copy per buffer and chunk.
-    constexpr int kChunks = 8;
+    // `out`).  Each direction is one plain async copy per buffer and chunk.  The copy in is
+    // the bound; what the pipeline cannot hide is the last chunk's compute and copy out,
+    // so more chunks shorten the tail.
+    constexpr int kChunks = 16;
     const int per_b = p->B >= kChunks ? 1 : kChunks / p->B;             // chunks per batch entry
     const int hc = (p->H + per_b - 1) / per_b;                          // heads per chunk
     const int bc = p->B >= kChunks ? (p->B + kChunks - 1) / kChunks : 1; // batch entries per chunk
