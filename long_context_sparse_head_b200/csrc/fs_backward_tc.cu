@@ -1,5 +1,6 @@
-// Readout part of the backward pass on the 5th-generation tensor cores (bf16), "FreeSolo"
-// summary §3.3 eq. (9) with the selection held fixed.  For the rows of one 128-row tile of
+// Backward pass on the 5th-generation tensor cores (bf16), readout and window, "FreeSolo"
+// summary §3.3 eq. (9) and §3.2 eqs. (3)-(4) with the selection held fixed.  The readout:
+// for the rows of one 128-row tile of
 // a (batch, head) and the union U of their selected cells (the tile record of the fused
 // forward kernel, here built from idx):
 //   u_i = sum_t pi_it v_t,  pi_i = softmax_t(s_it),  s_it = q_i.k_t / sqrt(d)  (t in cells(S_i))
@@ -46,7 +47,6 @@ constexpr int REGS_ROW = 192, REGS_OTHER = 64;           // 256 * 192 + 256 * 64
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t S_COL = 0, DP_COL = 128, U_COL = 256, DV_COL = 320, DK_COL = DV_COL + 64;
 constexpr int TILE_BYTES = BM * kD * 2;                  // 128 rows x 64 bf16: 16 KiB
-constexpr int CELL_BYTES = kS * kD * 2;                  // 32 x 64 bf16: 4 KiB
 
 struct BtcSmem {
     __nv_bfloat16 q[BM * kD];                            // Q tile (NoPE), 128-byte swizzled rows
