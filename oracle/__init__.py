@@ -3,7 +3,7 @@
 TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's CPU
 baseline may import this package; the CUDA library and its Python binding never do.
 
-It follows the "FreeSolo" technical summary (picx.dev/p/IEuVxx), §3.1 eq. (2),
+It follows the "FreeSolo" technical summary, §3.1 eq. (2),
 §3.2 eqs. (3)-(4), §3.3 eqs. (5), (7)-(9) and §3.4 eqs. (10)-(12); the readings taken where the page is
 silent are stated at the top of the C source.  Inputs are float32 arrays holding
 the exact input values (bf16 inputs widened); all arithmetic is float64.

@@ -5,7 +5,7 @@
  * leg of the benchmark may load this code.  The CUDA library never links, calls or
  * includes it, and this file includes nothing from the CUDA library.
  *
- * Source: "FreeSolo" technical summary (picx.dev/p/IEuVxx), section "Methodology":
+ * Source: "FreeSolo" technical summary, section "Methodology":
  *   §3.1 Range Separation  eq. (2)   o_i = o_i^sr + alpha_h o_i^lr
  *   §3.2 Local Branch      eq. (3)   RoPE logits inside the look-back radius w
  *                          eq. (4)   softmax readout over the local set L_i
