@@ -31,8 +31,10 @@
  * Ownership and errors: the caller owns every buffer; the library allocates nothing and
  * enqueues its kernels on `stream` (a cudaStream_t; NULL is the legacy default stream).
  * Pointers named d* / Q, K, V, O, kbar, amax, idx, ws are device pointers; the per-head
- * arrays alpha / lambda / sigma are HOST pointers read during the call.  Argument errors
- * are returned before anything is enqueued.  No exception crosses the ABI.
+ * arrays alpha / lambda / sigma are HOST pointers read during the call.  Device arrays
+ * start on a 16-byte boundary (as cudaMalloc and torch allocations do): the kernels read
+ * and write them in 16-byte vectors and describe them to the tensor-memory-access unit.
+ * Argument errors are returned before anything is enqueued.  No exception crosses the ABI.
  *
  * Supported: d = 64, s = 32, w a multiple of s, 0 <= K <= 64, W + P <= 2048,
  * 1 <= H <= 256; dtype bf16 or f32.  Anything else returns FS_ERR_UNSUPPORTED.
