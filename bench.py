@@ -206,6 +206,45 @@ def algorithmic_work(wl, n_sel_cells):
     }
 
 
+def fused_executed_exps(wl, amax):
+    """Exponentials the fused kernel evaluates per launch.  It runs the readout masked-dense
+    over each 128-row tile's union of admitted cells (eq. (8): the recent range and the
+    TopP sets of the tile's prefixes; two cells per 64-key chunk) and the window over the
+    tile's band in 64-key chunks, every chunk for all 128 rows."""
+    C, q0, s, w, W, P = wl.Nk // wl.s, wl.Nk - wl.Nq, wl.s, wl.w, wl.W, wl.P
+
+    def cand(i):                                     # cells wholly before the window of i
+        lim = i - w
+        return 0 if lim < s else min(lim // s, C)
+    total = 0
+    ntiles = (wl.Nq + 127) // 128
+    for b in range(wl.B):
+        for h in range(wl.H):
+            a = amax[b, h]
+            rank = np.empty(C, np.int64)
+            rank[np.lexsort((np.arange(C), -a))] = np.arange(C)   # larger a first, then lower index
+            for t in range(ntiles):
+                r0 = 128 * t
+                nrows = min(128, wl.Nq - r0)
+                pb = q0 + r0
+                nmin, nmax = cand(pb), cand(pb + nrows - 1)
+                if W < 0:
+                    nU = nmax
+                elif nmax > 0:
+                    cells = set(range(max(0, nmin - W), nmax))
+                    for n in range(max(nmin, 1), nmax + 1):
+                        cells.update(np.argsort(rank[:n], kind="stable")[:P].tolist())
+                    nU = len(cells)
+                else:
+                    nU = 0
+                nR = (nU + 1) // 2
+                jbase, last = pb - w, pb + nrows - 1
+                k_first = (-jbase) // 64 if jbase < 0 else 0
+                nW = (last - jbase) // 64 - k_first + 1
+                total += 128 * 64 * (nR + nW)
+    return total
+
+
 def source_hash(kernel):
     files = {"readout": "fs_readout.cu", "window_combine": "fs_window.cu",
              "cell_summaries": "fs_summaries.cu", "exit_times": "fs_prune.cu",
@@ -672,6 +711,7 @@ def run_ours(args):
     fs.select_topk(p, Q, kbar, amax, idx, ws)
     n_sel = int((idx >= 0).sum().item())
     work = algorithmic_work(wl, n_sel)
+    executed_exps = fused_executed_exps(wl, amax.cpu().numpy()) if wl.dtype == "bf16" else None
     dom = max((k for k in ktimes if ktimes[k][0] > 0), key=lambda k: ktimes[k][1])
     cnt, tot_ms = ktimes[dom]
     avg_s = tot_ms / cnt * 1e-3
@@ -720,6 +760,13 @@ def run_ours(args):
                             "all_flops_us": 1e6 * t_all, "exps_us": 1e6 * t_mufu},
             "algorithmic_exps": work["_exps"], "exp_rate_per_s": exp_rate,
             "tensor_peak_tflops": tensor_peak, "selected_cells": n_sel}
+    if executed_exps is not None and "attn_tc" in ktimes and ktimes["attn_tc"][0] > 0:
+        t_attn = ktimes["attn_tc"][1] / ktimes["attn_tc"][0] * 1e-3
+        # the fused kernel's exponentials as it runs them (masked-dense readout, whole
+        # 64-key band chunks) against the exponential unit's peak over its launch time
+        path["fused_kernel_exps"] = {"executed": executed_exps,
+                                     "executed_over_algorithmic": executed_exps / work["_exps"],
+                                     "exp_unit_frac": executed_exps / (t_attn * exp_rate)}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
