@@ -31,10 +31,13 @@ namespace fs {
 
 namespace {
 constexpr int BM = 128, UMAX = 128;              // largest union; UM = 80 or UMAX per launch
-constexpr int W_MMA = 4, NWARPS = 5, NTHREADS = NWARPS * 32;   // warp 4: Q load, then the MMA
+// warps 0-3: union, staging, scores and keys (thread = row = TMEM lane); warps 0-7: the
+// K-th search, two threads per row; warp 8: Q load, then the MMA
+constexpr int NROWW = 4, NSRCHW = 8, W_MMA = 8, NWARPS = 9, NTHREADS = NWARPS * 32;
 constexpr uint32_t TMEM_COLS = 128;
 constexpr int TILE_BYTES = BM * kD * 2;
-constexpr int kSelBarrier = 1;   // named barrier of the 128 selection threads
+constexpr int kSelBarrier = 1;   // named barrier of the 128 row threads
+constexpr int kSrchBarrier = 2;  // named barrier of the 256 search threads
 
 template <int UM> struct SelSmem {       // UM: capacity of the union (a multiple of 16)
     __nv_bfloat16 q[BM * kD];              // Q tile (NoPE)
@@ -47,6 +50,7 @@ template <int UM> struct SelSmem {       // UM: capacity of the union (a multipl
     float amax_w[4];                       // per warp: largest a_c of its union positions
     int nU, ncand;
     uint64_t q_full, kb_ready, s_full, drain;
+    uint4 hmask[BM][2];                    // per row and half: its selected union positions
     uint32_t tmem_base;
     int abort;
 };
@@ -71,7 +75,98 @@ template <> struct SelArgsT<true> : SelArgs {
 };
 
 __device__ __forceinline__ void sel_sync() {
-    asm volatile("bar.sync %0, %1;" ::"n"(kSelBarrier), "n"(128) : "memory");
+    asm volatile("bar.sync %0, %1;" ::"n"(kSelBarrier), "n"(NROWW * 32) : "memory");
+}
+__device__ __forceinline__ void srch_sync() {
+    asm volatile("bar.sync %0, %1;" ::"n"(kSrchBarrier), "n"(NSRCHW * 32) : "memory");
+}
+
+// The rows' integer keys in shared memory, over the Q tile and the mean-key parts once the
+// score MMA has read them: row r's 16-byte chunk c (keys 4c .. 4c + 3).  With UM = 80 a row
+// takes 21 chunks (one of padding), so eight consecutive rows start in eight different
+// bank groups; with UM = 128 (32 chunks, no room to pad) chunk c is stored at c ^ (r mod 8).
+template <int UM> __device__ __forceinline__ int key_chunk(int r, int c) {
+    if constexpr (UM == 128) return r * 32 + (c ^ (r & 7));
+    else return r * (UM / 4 + 1) + c;
+}
+template <int UM> constexpr size_t key_bytes() { return (size_t)BM * (UM == 128 ? 32 : UM / 4 + 1) * 16; }
+template <int UM> constexpr bool keys_fit() {
+    return offsetof(SelSmem<UM>, kb) == sizeof(SelSmem<UM>::q) &&
+           key_bytes<UM>() <= sizeof(SelSmem<UM>::q) + sizeof(SelSmem<UM>::kb);
+}
+static_assert(keys_fit<80>() && keys_fit<UMAX>(), "the keys fit over Q and the mean-key parts");
+
+// K-th largest key of one row, by two threads (lanes l and l + 16 of a warp, each holding
+// half of the row's keys): the bisection on c(x) = count(key >= x) with the stopping rule of
+// the one-thread search, every count the sum of the two halves' (one shuffle).  The loop
+// runs while any row of the warp is still searching; a finished row's threads take part in
+// the shuffles without updating.  Writes the half's selected union positions.
+template <int UM>
+__device__ __forceinline__ void search_half(const uint4 *keys, uint4 (*hmask)[2], int K, int warp, int lane) {
+    constexpr int HK = UM / 2, HC = HK / 4;     // keys and 16-byte chunks per half
+    const int srow = 16 * warp + (lane & 15), half = lane >> 4;
+    uint32_t key[HK];
+#pragma unroll
+    for (int j = 0; j < HC; j++) {
+        const uint4 v = keys[key_chunk<UM>(srow, half * HC + j)];
+        key[4 * j] = v.x; key[4 * j + 1] = v.y; key[4 * j + 2] = v.z; key[4 * j + 3] = v.w;
+    }
+    int nh = 0;
+#pragma unroll
+    for (int u = 0; u < HK; u++) nh += key[u] != 0u;
+    const int na = nh + __shfl_xor_sync(kFull, nh, 16);
+    uint32_t lo = 1u << 7, hi = (0x1000000u + 1u) << 7;
+    int clo = na, chi = 0;
+    const bool active = na > K;
+    auto going = [&]() { return active && clo > K + 1 && chi < K - 1 && hi - lo > 1u; };
+    while (__any_sync(kFull, going())) {
+        const bool go = going();
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        int cp[4] = {0, 0, 0, 0};               // independent partial counts
+#pragma unroll
+        for (int u = 0; u < HK; u++) cp[u & 3] += key[u] >= mid;
+        int cnt = (cp[0] + cp[1]) + (cp[2] + cp[3]);
+        cnt += __shfl_xor_sync(kFull, cnt, 16);
+        if (go) {
+            if (cnt >= K) { lo = mid; clo = cnt; }
+            else { hi = mid; chi = cnt; }
+        }
+    }
+    // the bracket pins the K-th key: c(lo) = K, or the (K+1)-th key is the smallest >= lo, or
+    // (c(hi) = K - 1) the K-th key is the largest < hi; both extremes over the row's halves
+    uint32_t m0 = 0xffffffffu, m1 = 0u;
+#pragma unroll
+    for (int u = 0; u < HK; u++) {
+        m0 = key[u] >= lo ? min(m0, key[u]) : m0;
+        m1 = key[u] < hi ? max(m1, key[u]) : m1;
+    }
+    m0 = min(m0, __shfl_xor_sync(kFull, m0, 16));
+    m1 = max(m1, __shfl_xor_sync(kFull, m1, 16));
+    const uint32_t tau = !active ? 1u : clo == K ? lo : clo == K + 1 ? m0 + 1u : m1;
+    uint32_t w[HK / 32 + 1];
+#pragma unroll
+    for (int b = 0; b <= HK / 32; b++) w[b] = 0u;
+#pragma unroll
+    for (int u = 0; u < HK; u++)
+        if (key[u] >= tau && key[u] != 0u) w[u >> 5] |= 1u << (u & 31);
+    // the half's bits at union positions half * HK + u, as a 128-bit mask
+    uint32_t o[4] = {0u, 0u, 0u, 0u};
+    if (half == 0) {
+#pragma unroll
+        for (int b = 0; b <= HK / 32; b++) o[b] = w[b];
+    } else {
+        constexpr int s0 = HK >> 5, sh = HK & 31;   // HK = 32 s0 + sh
+#pragma unroll
+        for (int b = 0; b <= HK / 32; b++) {
+            if constexpr (sh == 0) {
+                if (s0 + b < 4) o[s0 + b] |= w[b];
+            } else {
+                if (s0 + b < 4) o[s0 + b] |= w[b] << sh;
+                if (s0 + b + 1 < 4) o[s0 + b + 1] |= w[b] >> (32 - sh);
+            }
+        }
+    }
+    hmask[srow][half] = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 __device__ __forceinline__ void split3(float x, __nv_bfloat16 &hi, __nv_bfloat16 &mid, __nv_bfloat16 &lo) {
@@ -146,6 +241,12 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgsT<PRIOR> A
                 }
             }
         }
+    } else if (warp >= NROWW) {
+        // ---- helper warps: the K-th search of rows 16 (warp) .. 16 (warp) + 15, once the row
+        // threads have written every row's keys
+        srch_sync();
+        search_half<UM>(reinterpret_cast<const uint4 *>(sm.q), sm.hmask, A.K, warp, lane);
+        srch_sync();
     } else {
         const int t = threadIdx.x;     // 0..127: union builder, then the row this thread owns
         // ---- U: ordered union of the admitted sets of the tile's prefixes n_min..n_max
@@ -340,129 +441,115 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgsT<PRIOR> A
         tc::fence_async_shared();
         tc::mbar_arrive(&sm.kb_ready);
 
-        // ---- this thread's row: scores -> admitted keys -> K best
+        // ---- this thread's row: scores -> admitted keys (to shared memory) -> K best (eight
+        // warps, two threads per row) -> the row's record
         const int row = t;
         const int i = pb + row;
         const int n_r = cand_count(i, A.w, A.C);
         const int g = n_r - n_min;
-        if (!tc::mbar_wait(&sm.s_full, 0, ab)) goto done;
-        if (tiles && !tc::mbar_wait(&sm.q_full, 0, ab)) goto done;   // Q rows read for |q|
-        {
-            tc::tc_fence_after();
-            const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-            float lam = 0.f, i2s = 0.f;
-            if constexpr (PRIOR) {
-                lam = A.pr.lambda[h];
-                i2s = A.pr.inv2sigma[h];
+        const bool ok = tc::mbar_wait(&sm.s_full, 0, ab) && (!tiles || tc::mbar_wait(&sm.q_full, 0, ab));
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+        float lam = 0.f, i2s = 0.f;
+        if constexpr (PRIOR) {
+            lam = A.pr.lambda[h];
+            i2s = A.pr.inv2sigma[h];
+        }
+        uint32_t aw[NW];                            // admitted union positions of this row
+#pragma unroll
+        for (int b = 0; b < NW; b++) aw[b] = row < nrows ? sm.admit[g][b] : 0u;
+        int na = 0;
+#pragma unroll
+        for (int b = 0; b < NW; b++) na += __popc(aw[b]);
+        float qq = 0.f;                             // |q|^2 of this row, before the keys cover Q
+        if (ok && tiles) {
+            const uint8_t *qrow = reinterpret_cast<const uint8_t *>(sm.q) + row * 128;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(qrow + ((j ^ (row & 7)) << 4));
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const float lo = __uint_as_float(w4[e] << 16), hi = __uint_as_float(w4[e] & 0xffff0000u);
+                    qq = fmaf(lo, lo, fmaf(hi, hi, qq));
+                }
             }
-            uint32_t aw[NW];                        // admitted union positions of this row
-#pragma unroll
-            for (int b = 0; b < NW; b++) aw[b] = row < nrows ? sm.admit[g][b] : 0u;
-            int na = 0;
-#pragma unroll
-            for (int b = 0; b < NW; b++) na += __popc(aw[b]);
-            // raw scores of the N used columns, loaded in 16-column blocks before one wait
-            uint32_t key[UM];
-#pragma unroll
-            for (int b = 0; b < UM / 16; b++)
-                if (16 * b < N) tc::tmem_ld16(trow + 16 * b, &key[16 * b]);
-            tc::tmem_wait_ld();
-            // scores r_ic, and their range over the admitted cells
+        }
+        // score r_ic of union position u from its raw product (the same arithmetic in both passes)
+        auto score = [&](uint32_t raw, int u) {
+            float sc = __uint_as_float(raw) * A.scale;
+            if (PRIOR) {
+                const float pc = (float)(sm.ulist[u] * kS) + 0.5f * kS;
+                sc += lam * sm.acell[u] * erff(((float)i - pc) * i2s);
+            }
+            return sc;
+        };
+        float smax = -INFINITY;
+        if (ok) {
+            tc::tc_fence_after();
+            // pass 1: the range of the admitted scores, 16 columns at a time
             float fmn[4], fmx[4];
 #pragma unroll
             for (int k = 0; k < 4; k++) { fmn[k] = INFINITY; fmx[k] = -INFINITY; }
 #pragma unroll
-            for (int u = 0; u < UM; u++) {
-                if (16 * (u / 16) < N) {
-                    float sc = __uint_as_float(key[u]) * A.scale;
-                    if (PRIOR) {
-                        const float pc = (float)(sm.ulist[u] * kS) + 0.5f * kS;
-                        sc += lam * sm.acell[u] * erff(((float)i - pc) * i2s);
+            for (int b = 0; b < UM / 16; b++) {
+                if (16 * b < N) {
+                    uint32_t r[16];
+                    tc::tmem_ld16(trow + 16 * b, r);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; e++) {
+                        const int u = 16 * b + e;
+                        const float sc = score(r[e], u);
+                        const bool adm = (aw[u >> 5] >> (u & 31)) & 1u;
+                        fmn[e & 3] = adm ? fminf(fmn[e & 3], sc) : fmn[e & 3];
+                        fmx[e & 3] = adm ? fmaxf(fmx[e & 3], sc) : fmx[e & 3];
                     }
-                    const bool adm = (aw[u >> 5] >> (u & 31)) & 1u;
-                    key[u] = __float_as_uint(sc);
-                    fmn[u & 3] = adm ? fminf(fmn[u & 3], sc) : fmn[u & 3];
-                    fmx[u & 3] = adm ? fmaxf(fmx[u & 3], sc) : fmx[u & 3];
                 }
             }
             const float mn = fminf(fminf(fmn[0], fmn[1]), fminf(fmn[2], fmn[3]));
-            const float smax = fmaxf(fmaxf(fmx[0], fmx[1]), fmaxf(fmx[2], fmx[3]));
+            smax = fmaxf(fmaxf(fmx[0], fmx[1]), fmaxf(fmx[2], fmx[3]));
             const float span = smax - mn;
             const float q24 = span > 0.f ? 16777215.f / span : 0.f;
-            // integer keys: 1 + the score's 24-bit fixed-point place in the row's range, then
-            // 7 bits of (127 - position); 0 for a cell that is not admitted
+            // every row thread has read Q (and the MMA has read Q and the mean keys)
+            sel_sync();
+            // pass 2: integer keys, 1 + the score's 24-bit fixed-point place in the row's range,
+            // then 7 bits of (127 - position); 0 for a cell that is not admitted (and for the
+            // columns past N)
+            uint4 *kdst = reinterpret_cast<uint4 *>(sm.q);
 #pragma unroll
-            for (int u = 0; u < UM; u++) {
-                if (16 * (u / 16) < N) {
-                    const bool adm = (aw[u >> 5] >> (u & 31)) & 1u;
-                    const uint32_t fx = min(__float2uint_rz((__uint_as_float(key[u]) - mn) * q24), 0xffffffu);
-                    key[u] = adm ? ((fx + 1u) << 7) | (uint32_t)(127 - u) : 0u;
-                } else {
-                    key[u] = 0u;
+            for (int b = 0; b < UM / 16; b++) {
+                uint32_t r[16];
+                if (16 * b < N) {
+                    tc::tmem_ld16(trow + 16 * b, r);
+                    tc::tmem_wait_ld();
                 }
-            }
-            // K-th largest key: bisection on c(x) = count(key >= x) keeps c(lo) >= K > c(hi)
-            // and stops as soon as the bracket pins the K-th key to within one key, i.e.
-            // c(lo) = K or K + 1, or c(hi) = K - 1; one more pass over the keys then gives
-            // tau with c(tau) = K exactly (keys are unique).  Stopping at any of the three gaps
-            // around the K-th key instead of only the one below it cuts the halvings of the
-            // warp's slowest row, which sets the warp's loop count.
-            uint32_t tau = 1u;
-            if (na > A.K) {
-                uint32_t lo = 1u << 7, hi = (0x1000000u + 1u) << 7;
-                int clo = na, chi = 0;
-                while (clo > A.K + 1 && chi < A.K - 1 && hi - lo > 1u) {
-                    const uint32_t mid = lo + ((hi - lo) >> 1);
-                    int cp[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent partial counts
 #pragma unroll
-                    for (int b = 0; b < UM / 16; b++)
-                        if (16 * b < N) {
-#pragma unroll
-                            for (int e = 0; e < 16; e++) cp[e & 7] += key[16 * b + e] >= mid;
-                        }
-                    const int cnt = ((cp[0] + cp[1]) + (cp[2] + cp[3])) + ((cp[4] + cp[5]) + (cp[6] + cp[7]));
-                    if (cnt >= A.K) {
-                        lo = mid;
-                        clo = cnt;
-                    } else {
-                        hi = mid;
-                        chi = cnt;
+                for (int e = 0; e < 16; e++) {
+                    const int u = 16 * b + e;
+                    uint32_t key = 0u;
+                    if (16 * b < N) {
+                        const bool adm = (aw[u >> 5] >> (u & 31)) & 1u;
+                        const uint32_t fx = min(__float2uint_rz((score(r[e], u) - mn) * q24), 0xffffffu);
+                        key = adm ? ((fx + 1u) << 7) | (uint32_t)(127 - u) : 0u;
                     }
+                    r[e] = key;
                 }
-                if (clo == A.K) {
-                    tau = lo;
-                } else if (clo == A.K + 1) {            // the (K+1)-th key is the smallest >= lo
-                    uint32_t m0 = 0xffffffffu, m1 = 0xffffffffu;
 #pragma unroll
-                    for (int b = 0; b < UM / 16; b++)
-                        if (16 * b < N) {
-#pragma unroll
-                            for (int e = 0; e < 16; e += 2) {
-                                const uint32_t k0 = key[16 * b + e], k1 = key[16 * b + e + 1];
-                                m0 = k0 >= lo ? min(m0, k0) : m0;
-                                m1 = k1 >= lo ? min(m1, k1) : m1;
-                            }
-                        }
-                    tau = min(m0, m1) + 1u;
-                } else {                                 // c(hi) = K - 1: the K-th key is the largest < hi
-                    uint32_t m0 = 0u, m1 = 0u;
-#pragma unroll
-                    for (int b = 0; b < UM / 16; b++)
-                        if (16 * b < N) {
-#pragma unroll
-                            for (int e = 0; e < 16; e += 2) {
-                                const uint32_t k0 = key[16 * b + e], k1 = key[16 * b + e + 1];
-                                m0 = k0 < hi ? max(m0, k0) : m0;
-                                m1 = k1 < hi ? max(m1, k1) : m1;
-                            }
-                        }
-                    tau = max(m0, m1);
-                }
+                for (int c = 0; c < 4; c++)
+                    kdst[key_chunk<UM>(row, 4 * b + c)] = make_uint4(r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
             }
-            uint32_t mw[UMAX / 32] = {0u, 0u, 0u, 0u};   // selected union positions
-#pragma unroll
-            for (int u = 0; u < UM; u++)
-                if (16 * (u / 16) < N && key[u] >= tau && key[u] != 0u) mw[u >> 5] |= 1u << (u & 31);
+        } else {
+            sel_sync();
+        }
+        srch_sync();
+        search_half<UM>(reinterpret_cast<const uint4 *>(sm.q), sm.hmask, A.K, warp, lane);
+        srch_sync();
+        if (ok) {
+            uint32_t mw[UMAX / 32];                 // selected union positions
+            {
+                const uint4 h0 = sm.hmask[row][0], h1 = sm.hmask[row][1];
+                mw[0] = h0.x | h1.x; mw[1] = h0.y | h1.y; mw[2] = h0.z | h1.z; mw[3] = h0.w | h1.w;
+            }
             if (tiles) {   // compact record for the fused kernel: row masks | union | |U| | reference
                 // Readout reference (log2 units): every NoPE logit q.k_j / sqrt(d) of a selected
                 // token is at most |q| max_{c in U} a_c / sqrt(d) (Cauchy-Schwarz), and the
@@ -476,33 +563,25 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgsT<PRIOR> A
                 float lower = smax * 1.4426950408889634f;
                 if (PRIOR) {
                     // warp-collective loads (.sync.aligned): every lane issues them
-                    uint32_t raw[UM];
-#pragma unroll
-                    for (int b = 0; b < UM / 16; b++)
-                        if (16 * b < N) tc::tmem_ld16(trow + 16 * b, &raw[16 * b]);
-                    tc::tmem_wait_ld();
                     float dmax = -INFINITY;
 #pragma unroll
-                    for (int u = 0; u < UM; u++)
-                        if (16 * (u / 16) < N && ((mw[u >> 5] >> (u & 31)) & 1u))
-                            dmax = fmaxf(dmax, __uint_as_float(raw[u]));
+                    for (int b = 0; b < UM / 16; b++) {
+                        if (16 * b < N) {
+                            uint32_t raw[16];
+                            tc::tmem_ld16(trow + 16 * b, raw);
+                            tc::tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 16; e++) {
+                                const int u = 16 * b + e;
+                                if ((mw[u >> 5] >> (u & 31)) & 1u) dmax = fmaxf(dmax, __uint_as_float(raw[e]));
+                            }
+                        }
+                    }
                     lower = dmax * c;
                 }
                 float mref = 0.f;
                 if (na > 0) {
-                    // |q| of this row from the tile in shared memory (128-byte swizzle)
-                    const uint8_t *qrow = reinterpret_cast<const uint8_t *>(sm.q) + row * 128;
-                    float qq = 0.f;
-#pragma unroll
-                    for (int j = 0; j < 8; j++) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(qrow + ((j ^ (row & 7)) << 4));
-                        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                        for (int e = 0; e < 4; e++) {
-                            const float lo = __uint_as_float(w4[e] << 16), hi = __uint_as_float(w4[e] & 0xffff0000u);
-                            qq = fmaf(lo, lo, fmaf(hi, hi, qq));
-                        }
-                    }
+                    // |q| of this row (read from the tile before the keys covered it)
                     const float amx = fmaxf(fmaxf(sm.amax_w[0], sm.amax_w[1]), fmaxf(sm.amax_w[2], sm.amax_w[3]));
                     const float ub = sqrtf(qq) * amx * c;
                     mref = (ub - lower <= kMrefMaxGap) ? ub : __uint_as_float(0x7fc00000u);
@@ -522,7 +601,6 @@ select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgsT<PRIOR> A
                 for (; o < A.K; o++) out[o] = -1;
             }
         }
-    done:;
     }
 
     tc::tc_fence_before();
