@@ -15,13 +15,14 @@
 // tensor-core products sum to the fp32 dot product up to accumulation rounding), in the
 // 128-byte-swizzled layout of a K-major MMA operand.  One thread issues
 // S = Q (hi + mid + lo)^T (M = 128, N = |U| rounded up to 16) into tensor memory.  Each
-// thread then takes its row's scores, keeps the admitted ones and finds the K-th largest
-// by bisection on integer keys: the score's 24-bit fixed-point place within the row's
-// admitted range, above 7 bits of (127 - position).  Keys are unique, and among scores
-// within 2^-24 of the row's range of each other the lower cell index wins, inside the
-// near-tie tolerance of the selection check.  The search stops once exactly K keys
-// remain; keys spread over one range per row separate in far fewer halvings than
-// order-preserving bit patterns of the raw fp32 scores.
+// row thread then reads its row's scores (twice, 16 columns at a time: the admitted range,
+// then the keys) and writes integer keys to shared memory, over Q and the mean-key parts:
+// the score's 24-bit fixed-point place within the row's admitted range, above 7 bits of
+// (127 - position).  Keys are unique, and among scores within 2^-24 of the row's range of
+// each other the lower cell index wins, inside the near-tie tolerance of the selection
+// check.  Eight warps then find each row's K-th largest key by bisection, two threads per
+// row with half of its keys each; keys spread over one range per row separate in far
+// fewer halvings than order-preserving bit patterns of the raw fp32 scores.
 // Outputs: idx (selected cells per row, ascending, -1 padded) and/or, for the fused
 // kernel, one compact record per tile: each row's selected union positions as a 128-bit
 // mask, the union's cells and its size.
@@ -177,8 +178,8 @@ __device__ __forceinline__ void split3(float x, __nv_bfloat16 &hi, __nv_bfloat16
 }
 }  // namespace
 
-// UM = 80 (|U| <= 80: three CTAs of five warps per SM, at most four warps per SM
-// sub-partition, so up to 128 registers) or 128 (two CTAs per SM)
+// UM = 80 (|U| <= 80: three CTAs of nine warps per SM, 72 registers a thread) or 128 (two
+// CTAs per SM)
 template <bool PRIOR, int UM>
 __global__ void __launch_bounds__(NTHREADS, UM <= 80 ? 3 : 2)
 select_tc_kernel(const __grid_constant__ CUtensorMap tq, const SelArgsT<PRIOR> A, const float *__restrict__ kbar,
